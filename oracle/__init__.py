@@ -1,0 +1,17 @@
+"""fp64 CPU oracle of the cone-beam DRR ray-march -- TEST INFRASTRUCTURE.
+
+Only tests/, the smoke check in __graft_entry__ and the cpu_baseline leg of
+bench.py may import this package.  The product path (cone_beam_ct_b200)
+never imports it and shares no code with it.
+"""
+from .oracle import (  # noqa: F401
+    adjoint,
+    bf16_to_float,
+    build,
+    load,
+    ray,
+    render,
+    render_rays,
+    round_bf16,
+    trilinear,
+)

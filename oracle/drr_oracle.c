@@ -1,0 +1,347 @@
+/*
+ * drr_oracle.c -- fp64 CPU oracle of the cone-beam DRR ray-march.
+ *
+ * TEST INFRASTRUCTURE, NOT PRODUCT CODE.  Only tests/, the smoke check in
+ * __graft_entry__ and the cpu_baseline leg of bench.py may load this
+ * library.  It shares no code, header, table or helper with the CUDA path.
+ *
+ * What it computes, step by step, in the order of the method:
+ *
+ *  1. Camera ray (nanodrr page, introduction: Hartley-Zisserman pinhole
+ *     x ~ K [R | t] X).  Pixel (row r, column c) has its centre at
+ *     (u, v) = (c, r).  Solve K q = (u, v, 1) by back substitution (K is
+ *     upper triangular), direction d = R^T q normalised to unit length in
+ *     world mm, camera centre C = -R^T t.
+ *  2. World -> IJK (flashdrr.rendering API docs, VolumeRaycaster.forward:
+ *     the volume lives in IJK voxel space and an affine maps world to IJK;
+ *     here the axis-aligned case x_world = origin + spacing * ijk, origin
+ *     being the centre of voxel 0): C_ijk = (C - origin) / spacing,
+ *     d_ijk = d / spacing, so a ray parameter t stays in world mm.
+ *  3. Clip to the volume (flashdrr.rendering API docs,
+ *     compute_clipping_distances: near/far from the volume bounds in IJK
+ *     space), done per ray with the slab method on the box spanned by the
+ *     voxel centres, [0, n-1] per axis.  A zero direction component is a
+ *     miss if C lies outside that slab and no constraint otherwise.
+ *     t0 = max(t_near, 0), t1 = t_far; t1 <= t0 is a miss (integral 0).
+ *  4. N samples along each camera ray (VolumeRaycaster.__init__, parameter
+ *     ray_samples), read as the midpoint rule: dt = (t1 - t0) / N,
+ *     t_i = t0 + (i + 1/2) dt; each sample is a zero-padded trilinear
+ *     interpolation of the volume (the grid_sample path of VolumeRaycaster)
+ *     at C_ijk + t_i d_ijk; the samples are summed in order, in fp64.
+ *  5. I = density_factor * dt * sum (VolumeRaycaster.__init__, parameter
+ *     density_factor).  Output RAW: I; BEER_LAMBERT: 1 - exp(-I)
+ *     (parameter use_beer_lambert), evaluated as -expm1(-I).
+ *  6. Adjoint (TorchTomo page, "Discrete Adjoint and Learned Primal-Dual":
+ *     the transpose satisfies <A x, y> = <x, A^T y>): the same loop, each
+ *     sample scattering g * w_corner into the gradient volume, with
+ *     g = grad_out * density_factor * dt, times exp(-I) in Beer-Lambert
+ *     mode (the derivative of 1 - exp(-I)); I is the oracle's own forward.
+ *  7. bf16 storage: round-to-nearest-even of the fp32 bit pattern to the
+ *     upper 16 bits (the IEEE rounding rule, written out).
+ *
+ * Rays are independent, so the forward may run rays on several threads;
+ * every ray is still summed sequentially, so the result does not depend on
+ * the thread count.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORACLE_RAW 0
+#define ORACLE_BEER_LAMBERT 1
+
+typedef struct {
+    int64_t n[3];         /* nx, ny, nz; i is the fastest index */
+    double spacing[3];    /* mm per voxel along i, j, k */
+    double origin[3];     /* world mm of the centre of voxel (0, 0, 0) */
+} grid_t;
+
+static int make_grid(const int dims[3], const double spacing[3],
+                     const double origin[3], grid_t *g) {
+    for (int a = 0; a < 3; ++a) {
+        if (dims[a] < 1 || !(spacing[a] > 0.0)) return -1;
+        g->n[a] = dims[a];
+        g->spacing[a] = spacing[a];
+        g->origin[a] = origin[a];
+    }
+    return 0;
+}
+
+/* Step 1: ray of pixel centre (u, v) in world coordinates. */
+static void camera_ray(const double K[9], const double Rt[12], double u, double v,
+                       double C[3], double d[3]) {
+    /* back substitution of K q = (u, v, 1), K = [k0 k1 k2; 0 k4 k5; 0 0 k8] */
+    double q[3];
+    q[2] = 1.0 / K[8];
+    q[1] = (v - K[5] * q[2]) / K[4];
+    q[0] = (u - K[1] * q[1] - K[2] * q[2]) / K[0];
+    double norm2 = 0.0;
+    for (int a = 0; a < 3; ++a) {
+        /* (R^T q)_a = sum_r R[r][a] q[r]; (R^T t)_a likewise */
+        double da = 0.0, ca = 0.0;
+        for (int r = 0; r < 3; ++r) {
+            da += Rt[4 * r + a] * q[r];
+            ca += Rt[4 * r + a] * Rt[4 * r + 3];
+        }
+        d[a] = da;
+        C[a] = -ca;
+        norm2 += da * da;
+    }
+    double inv = 1.0 / sqrt(norm2);
+    for (int a = 0; a < 3; ++a) d[a] *= inv;
+}
+
+/* Steps 2-3: ray in IJK and its clipped parameter range; returns 1 on hit. */
+static int ray_in_volume(const grid_t *g, const double K[9], const double Rt[12],
+                         double u, double v, double Cijk[3], double dijk[3],
+                         double *t0, double *t1) {
+    double C[3], d[3];
+    camera_ray(K, Rt, u, v, C, d);
+    double t_near = -INFINITY, t_far = INFINITY;
+    for (int a = 0; a < 3; ++a) {
+        Cijk[a] = (C[a] - g->origin[a]) / g->spacing[a];
+        dijk[a] = d[a] / g->spacing[a];
+        double lo = 0.0, hi = (double)(g->n[a] - 1);
+        if (dijk[a] == 0.0) {
+            if (Cijk[a] < lo || Cijk[a] > hi) return 0;
+            continue;
+        }
+        double tA = (lo - Cijk[a]) / dijk[a];
+        double tB = (hi - Cijk[a]) / dijk[a];
+        double tmin = tA < tB ? tA : tB;
+        double tmax = tA < tB ? tB : tA;
+        if (tmin > t_near) t_near = tmin;
+        if (tmax < t_far) t_far = tmax;
+    }
+    *t0 = t_near > 0.0 ? t_near : 0.0;
+    *t1 = t_far;
+    return (*t1 > *t0) ? 1 : 0;
+}
+
+static double voxel(const float *vol, const grid_t *g, int64_t i, int64_t j, int64_t k) {
+    if (i < 0 || j < 0 || k < 0 || i >= g->n[0] || j >= g->n[1] || k >= g->n[2]) return 0.0;
+    return (double)vol[(k * g->n[1] + j) * g->n[0] + i];
+}
+
+/* Zero-padded trilinear interpolation at IJK point p. */
+static double trilinear(const float *vol, const grid_t *g, const double p[3]) {
+    double fl[3], f[3];
+    int64_t i0[3];
+    for (int a = 0; a < 3; ++a) {
+        fl[a] = floor(p[a]);
+        f[a] = p[a] - fl[a];
+        i0[a] = (int64_t)fl[a];
+    }
+    double s = 0.0;
+    for (int dk = 0; dk < 2; ++dk)
+        for (int dj = 0; dj < 2; ++dj)
+            for (int di = 0; di < 2; ++di) {
+                double w = (di ? f[0] : 1.0 - f[0]) * (dj ? f[1] : 1.0 - f[1]) *
+                           (dk ? f[2] : 1.0 - f[2]);
+                s += w * voxel(vol, g, i0[0] + di, i0[1] + dj, i0[2] + dk);
+            }
+    return s;
+}
+
+/* Steps 4-5 for one ray: returns the integral I (0 on a miss). */
+static double ray_integral(const float *vol, const grid_t *g, const double K[9],
+                           const double Rt[12], double u, double v, int n_samples,
+                           double density_factor, double *dt_out) {
+    double C[3], d[3], t0, t1;
+    *dt_out = 0.0;
+    if (!ray_in_volume(g, K, Rt, u, v, C, d, &t0, &t1)) return 0.0;
+    double dt = (t1 - t0) / (double)n_samples;
+    double sum = 0.0;
+    for (int i = 0; i < n_samples; ++i) {
+        double t = t0 + ((double)i + 0.5) * dt;
+        double p[3] = {C[0] + t * d[0], C[1] + t * d[1], C[2] + t * d[2]};
+        sum += trilinear(vol, g, p);
+    }
+    *dt_out = dt;
+    return density_factor * dt * sum;
+}
+
+static double apply_mode(double I, int mode) {
+    return mode == ORACLE_BEER_LAMBERT ? -expm1(-I) : I;
+}
+
+/* ------------------------------------------------------------------------ */
+/* forward over a list of rays, threaded over contiguous chunks of rays      */
+
+typedef struct {
+    const float *vol;
+    const grid_t *g;
+    const double *K, *Rt;
+    int H, W, n_samples, mode;
+    double density_factor;
+    const int64_t *ray_ids;   /* NULL: rays [begin, end) in order */
+    int64_t begin, end;
+    double *out;
+} fwd_job_t;
+
+static void *fwd_worker(void *arg) {
+    fwd_job_t *job = (fwd_job_t *)arg;
+    const int64_t hw = (int64_t)job->H * job->W;
+    for (int64_t n = job->begin; n < job->end; ++n) {
+        int64_t id = job->ray_ids ? job->ray_ids[n] : n;
+        int64_t b = id / hw, rc = id % hw;
+        double u = (double)(rc % job->W), v = (double)(rc / job->W);
+        double dt;
+        double I = ray_integral(job->vol, job->g, job->K, job->Rt + 12 * b, u, v,
+                                job->n_samples, job->density_factor, &dt);
+        job->out[n] = apply_mode(I, job->mode);
+    }
+    return NULL;
+}
+
+static int run_forward(const float *vol, const grid_t *g, const double *K, const double *Rt,
+                       int H, int W, int n_samples, double df, int mode,
+                       const int64_t *ray_ids, int64_t n_rays, double *out, int nthreads) {
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > 256) nthreads = 256;
+    if ((int64_t)nthreads > n_rays) nthreads = n_rays > 0 ? (int)n_rays : 1;
+    pthread_t tid[256];
+    int running[256];
+    fwd_job_t jobs[256];
+    int64_t chunk = (n_rays + nthreads - 1) / nthreads;
+    for (int t = 0; t < nthreads; ++t) {
+        int64_t begin = t * chunk, end = (t + 1) * chunk;
+        if (begin > n_rays) begin = n_rays;
+        if (end > n_rays) end = n_rays;
+        fwd_job_t j = {vol, g, K, Rt, H, W, n_samples, mode, df, ray_ids, begin, end, out};
+        jobs[t] = j;
+        running[t] = 0;
+        if (begin >= end) continue;
+        if (nthreads > 1 && pthread_create(&tid[t], NULL, fwd_worker, &jobs[t]) == 0)
+            running[t] = 1;
+        else
+            fwd_worker(&jobs[t]);   /* one thread, or thread creation failed */
+    }
+    for (int t = 0; t < nthreads; ++t)
+        if (running[t]) pthread_join(tid[t], NULL);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* exported API                                                              */
+
+/* Full image: out[b][r][c], B*H*W doubles. Returns 0, or -1 on bad sizes. */
+int oracle_render(const float *vol, const int dims[3], const double spacing[3],
+                  const double origin[3], const double K[9], const double *Rt, int B,
+                  int H, int W, int n_samples, double density_factor, int mode,
+                  double *out, int nthreads) {
+    grid_t g;
+    if (make_grid(dims, spacing, origin, &g) || B < 0 || H < 0 || W < 0 || n_samples < 1)
+        return -1;
+    return run_forward(vol, &g, K, Rt, H, W, n_samples, density_factor, mode, NULL,
+                       (int64_t)B * H * W, out, nthreads);
+}
+
+/* Selected rays, id = (b*H + r)*W + c; out[n] for ray_ids[n]. */
+int oracle_render_rays(const float *vol, const int dims[3], const double spacing[3],
+                       const double origin[3], const double K[9], const double *Rt, int B,
+                       int H, int W, int n_samples, double density_factor, int mode,
+                       const int64_t *ray_ids, int64_t n_rays, double *out, int nthreads) {
+    grid_t g;
+    if (make_grid(dims, spacing, origin, &g) || H < 1 || W < 1 || n_samples < 1) return -1;
+    for (int64_t n = 0; n < n_rays; ++n)
+        if (ray_ids[n] < 0 || ray_ids[n] >= (int64_t)B * H * W) return -1;
+    return run_forward(vol, &g, K, Rt, H, W, n_samples, density_factor, mode, ray_ids,
+                       n_rays, out, nthreads);
+}
+
+/* Ray geometry of one pixel: C_ijk, d_ijk (per mm), t0, t1. Returns hit flag. */
+int oracle_ray(const int dims[3], const double spacing[3], const double origin[3],
+               const double K[9], const double Rt[12], double u, double v,
+               double Cijk[3], double dijk[3], double t01[2]) {
+    grid_t g;
+    if (make_grid(dims, spacing, origin, &g)) return -1;
+    return ray_in_volume(&g, K, Rt, u, v, Cijk, dijk, &t01[0], &t01[1]);
+}
+
+/* Zero-padded trilinear interpolation at n points p[n][3] (IJK). */
+int oracle_trilinear(const float *vol, const int dims[3], const double *p, int64_t n,
+                     double *out) {
+    grid_t g;
+    const double one[3] = {1.0, 1.0, 1.0}, zero[3] = {0.0, 0.0, 0.0};
+    if (make_grid(dims, one, zero, &g)) return -1;
+    for (int64_t m = 0; m < n; ++m) out[m] = trilinear(vol, &g, p + 3 * m);
+    return 0;
+}
+
+/* Adjoint: grad_vol[k][j][i] += sum over rays and samples of g * w_corner.
+ * vol is read only in Beer-Lambert mode (for exp(-I)); it may be NULL in RAW.
+ * Single-threaded: a plain, fixed-order accumulation. */
+int oracle_adjoint(const float *vol, const int dims[3], const double spacing[3],
+                   const double origin[3], const double K[9], const double *Rt, int B,
+                   int H, int W, int n_samples, double density_factor, int mode,
+                   const double *grad_out, double *grad_vol) {
+    grid_t g;
+    if (make_grid(dims, spacing, origin, &g) || B < 0 || H < 0 || W < 0 || n_samples < 1)
+        return -1;
+    if (mode == ORACLE_BEER_LAMBERT && vol == NULL) return -1;
+    for (int b = 0; b < B; ++b)
+        for (int r = 0; r < H; ++r)
+            for (int c = 0; c < W; ++c) {
+                double go = grad_out[((int64_t)b * H + r) * W + c];
+                double C[3], d[3], t0, t1;
+                if (!ray_in_volume(&g, K, Rt + 12 * b, c, r, C, d, &t0, &t1)) continue;
+                double dt = (t1 - t0) / (double)n_samples;
+                double scale = go * density_factor * dt;
+                if (mode == ORACLE_BEER_LAMBERT) {
+                    double dt2;
+                    double I = ray_integral(vol, &g, K, Rt + 12 * b, c, r, n_samples,
+                                            density_factor, &dt2);
+                    scale *= exp(-I);
+                }
+                for (int i = 0; i < n_samples; ++i) {
+                    double t = t0 + ((double)i + 0.5) * dt;
+                    double p[3] = {C[0] + t * d[0], C[1] + t * d[1], C[2] + t * d[2]};
+                    double fl[3], f[3];
+                    int64_t i0[3];
+                    for (int a = 0; a < 3; ++a) {
+                        fl[a] = floor(p[a]);
+                        f[a] = p[a] - fl[a];
+                        i0[a] = (int64_t)fl[a];
+                    }
+                    for (int dk = 0; dk < 2; ++dk)
+                        for (int dj = 0; dj < 2; ++dj)
+                            for (int di = 0; di < 2; ++di) {
+                                int64_t ii = i0[0] + di, jj = i0[1] + dj, kk = i0[2] + dk;
+                                if (ii < 0 || jj < 0 || kk < 0 || ii >= g.n[0] ||
+                                    jj >= g.n[1] || kk >= g.n[2])
+                                    continue;
+                                double w = (di ? f[0] : 1.0 - f[0]) * (dj ? f[1] : 1.0 - f[1]) *
+                                           (dk ? f[2] : 1.0 - f[2]);
+                                grad_vol[(kk * g.n[1] + jj) * g.n[0] + ii] += scale * w;
+                            }
+                }
+            }
+    return 0;
+}
+
+/* bf16 storage: round-to-nearest-even of each fp32 value to its upper 16
+ * bits; NaN stays a (quiet) NaN. */
+void oracle_round_bf16(const float *in, uint16_t *out, int64_t n) {
+    for (int64_t m = 0; m < n; ++m) {
+        uint32_t bits;
+        memcpy(&bits, &in[m], 4);
+        if ((bits & 0x7f800000u) == 0x7f800000u && (bits & 0x007fffffu)) {
+            out[m] = (uint16_t)((bits >> 16) | 0x0040u);
+            continue;
+        }
+        uint32_t lsb = (bits >> 16) & 1u;
+        bits += 0x7fffu + lsb;
+        out[m] = (uint16_t)(bits >> 16);
+    }
+}
+
+/* Widen bf16 bit patterns back to fp32 values. */
+void oracle_bf16_to_float(const uint16_t *in, float *out, int64_t n) {
+    for (int64_t m = 0; m < n; ++m) {
+        uint32_t bits = (uint32_t)in[m] << 16;
+        memcpy(&out[m], &bits, 4);
+    }
+}

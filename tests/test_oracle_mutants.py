@@ -1,0 +1,72 @@
+"""The oracle's pins must fail on plausible slips (CPU only).
+
+Each case plants one mistake in a temporary copy of the oracle's C source,
+builds it, and runs the pin suite against that copy in a subprocess
+(DRR_ORACLE_LIB points the oracle binding at the mutant).  A mutant that
+passes every pin would mean the pins leave that part of the oracle unchecked.
+"""
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SRC = os.path.join(ROOT, "oracle", "drr_oracle.c")
+
+MUTANTS = {
+    "trilinear weights f <-> 1-f": (
+        "(di ? f[0] : 1.0 - f[0]) * (dj ? f[1] : 1.0 - f[1]) *\n"
+        "                           (dk ? f[2] : 1.0 - f[2]);\n                s += w",
+        "(di ? 1.0 - f[0] : f[0]) * (dj ? f[1] : 1.0 - f[1]) *\n"
+        "                           (dk ? f[2] : 1.0 - f[2]);\n                s += w"),
+    "left-endpoint instead of midpoint samples": (
+        "double t = t0 + ((double)i + 0.5) * dt;\n        double p[3]",
+        "double t = t0 + ((double)i) * dt;\n        double p[3]"),
+    "camera centre sign": ("C[a] = -ca;", "C[a] = ca;"),
+    "direction not normalised": ("for (int a = 0; a < 3; ++a) d[a] *= inv;", "(void)inv;"),
+    "R instead of R^T": ("da += Rt[4 * r + a] * q[r];", "da += Rt[4 * a + r] * q[r];"),
+    "box [0, n] instead of [0, n-1]": (
+        "double lo = 0.0, hi = (double)(g->n[a] - 1);", "double lo = 0.0, hi = (double)(g->n[a]);"),
+    "Beer-Lambert as exp(-I)": (
+        "return mode == ORACLE_BEER_LAMBERT ? -expm1(-I) : I;",
+        "return mode == ORACLE_BEER_LAMBERT ? exp(-I) : I;"),
+    "adjoint without dt": (
+        "double scale = go * density_factor * dt;", "double scale = go * density_factor;"),
+    "adjoint i/j transposed": (
+        "grad_vol[(kk * g.n[1] + jj) * g.n[0] + ii] += scale * w;",
+        "grad_vol[(kk * g.n[1] + ii) * g.n[0] + jj] += scale * w;"),
+    "no clamp of t0 at the camera": ("*t0 = t_near > 0.0 ? t_near : 0.0;", "*t0 = t_near;"),
+    "half-pixel shift": (
+        "double u = (double)(rc % job->W), v = (double)(rc / job->W);",
+        "double u = (double)(rc % job->W) + 0.5, v = (double)(rc / job->W) + 0.5;"),
+    "Beer-Lambert adjoint without exp(-I)": ("scale *= exp(-I);", "scale *= 1.0;"),
+    "skew sign": ("q[0] = (u - K[1] * q[1] - K[2] * q[2]) / K[0];",
+                  "q[0] = (u + K[1] * q[1] - K[2] * q[2]) / K[0];"),
+    "slab plane counted as outside": (
+        "if (Cijk[a] < lo || Cijk[a] > hi) return 0;", "if (Cijk[a] < lo || Cijk[a] >= hi) return 0;"),
+    "clamp instead of zero padding": (
+        "if (i < 0 || j < 0 || k < 0 || i >= g->n[0] || j >= g->n[1] || k >= g->n[2]) return 0.0;",
+        "if (i < 0) i = 0; if (j < 0) j = 0; if (k < 0) k = 0; if (i >= g->n[0]) i = g->n[0] - 1;"
+        " if (j >= g->n[1]) j = g->n[1] - 1; if (k >= g->n[2]) k = g->n[2] - 1;"),
+    "spacing ignored in the direction": ("dijk[a] = d[a] / g->spacing[a];", "dijk[a] = d[a];"),
+    "bf16 truncation instead of rounding": ("bits += 0x7fffu + lsb;", "(void)lsb;"),
+}
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_mutant(name, tmp_path):
+    before, after = MUTANTS[name]
+    src = open(SRC).read()
+    assert src.count(before) == 1, "mutation site not found: " + name
+    c_file = tmp_path / "mutant.c"
+    lib = tmp_path / "mutant.so"
+    c_file.write_text(src.replace(before, after))
+    subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-o", str(lib),
+                           str(c_file), "-lm", "-lpthread"])
+    env = dict(os.environ, DRR_ORACLE_LIB=str(lib))
+    r = subprocess.run([sys.executable, "-m", "pytest", os.path.join(ROOT, "tests",
+                        "test_oracle_pins.py"), "-q", "-x", "-p", "no:cacheprovider"],
+                       env=env, cwd=ROOT, capture_output=True, text=True, timeout=600)
+    assert r.returncode != 0, f"mutant '{name}' passed every pin:\n{r.stdout[-2000:]}"
