@@ -1,0 +1,476 @@
+#!/usr/bin/env python
+"""Throughput of the cone-beam DRR hot path on B200 (one JSON line on stdout).
+
+A step is one pass of the whole path over one batch of synthetic input:
+prepare the volume (fp32 -> padded layout, bf16 for the bf16 workload),
+forward ray-march of every view, zero the gradient volume, adjoint scatter
+of an N(0,1) upstream gradient.  Inputs are resident in HBM when timing
+starts.  L2 is flushed (a 256 MiB write) before every step, outside the
+step's timing.  Each step is timed with CUDA events on the launching stream;
+for N > 1 (torchrun, one process per GPU) every rank runs the same workload
+on its own GPU (weak scaling, no collective in the data path) and the time
+is the max over ranks.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 2]
+    python bench.py --impl reference ...   # the fp64 CPU oracle, same metric
+
+`e2e` repeats the step through the public API with pinned HOST buffers:
+host->device copies of the volume, poses and upstream gradient, and
+device->host reads of the image and the gradient volume, inside the timing.
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "Gsamples/s (ray×samples) and DRR FPS at 1 B200; % of L2/HBM gather roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+L2_BYTES = 126 * 1000 * 1000
+FLUSH_BYTES = 256 << 20
+
+
+def parse_args():
+    p = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--config", type=int, default=2, choices=[1, 2, 3, 4],
+                   help="workload (default 2: 256^3 fp32, 64 views 200x200, 256 samples)")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+# ---------------------------------------------------------------------------
+# workload description
+
+def workload(cfg):
+    from cone_beam_ct_b200 import workloads as wl
+    w = wl.make_config(cfg)
+    if w.grad_out is None:
+        w.grad_out = np.random.default_rng(2000 + cfg).standard_normal(
+            (w.B, w.H, w.W)).astype(np.float32)
+    return w
+
+
+def config_block(w, cfg, layout_name):
+    from cone_beam_ct_b200 import workloads as wl
+    nx, ny, nz = w.dims
+    vol_dtype = "bf16" if w.dtype == wl.DTYPE_BF16 else "fp32"
+    mode = "Beer-Lambert" if w.mode == wl.MODE_BEER_LAMBERT else "raw"
+    return {
+        "workload": f"{nx}^3 {vol_dtype} volume, {w.B} views x {w.H}x{w.W}, "
+                    f"{w.n_samples} samples/ray: prepare + forward ({mode}) + adjoint",
+        "config_index": cfg,
+        "volume": f"{nx}x{ny}x{nz} {vol_dtype}, {layout_name} layout, "
+                  f"{float(w.spacing[0])} mm voxels",
+        "views": w.B, "detector": [w.H, w.W], "samples_per_ray": w.n_samples,
+        "samples_per_step": w.samples,
+        "l2": "flushed before every step (256 MiB write, outside the step timing)",
+        "inputs": "seeded synthetic phantom and poses (cone_beam_ct_b200.workloads)",
+    }
+
+
+# ---------------------------------------------------------------------------
+# clocks
+
+def physical_gpu(ordinal):
+    """nvidia-smi id of torch device ``ordinal`` (honours CUDA_VISIBLE_DEVICES)."""
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "").strip()
+    if vis:
+        ids = [v.strip() for v in vis.split(",") if v.strip()]
+        if ordinal < len(ids):
+            return ids[ordinal]
+    return str(ordinal)
+
+
+class ClockSampler:
+    """nvidia-smi sampled every 200 ms during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in getattr(self, "lines", []):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# roofline helpers
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def l2_read_peak_gbs(torch, nbytes):
+    """L2 read bandwidth over a buffer of ``nbytes`` (the prepared volume's
+    size), best of 5 launches of libdrr_probe.so, in GB/s."""
+    import ctypes
+    lib = ctypes.CDLL(os.path.join(ROOT, "cone_beam_ct_b200", "libdrr_probe.so"))
+    lib.drr_probe_l2_read.argtypes = [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int,
+                                      ctypes.c_void_p, ctypes.c_void_p]
+    lib.drr_probe_l2_read.restype = ctypes.c_int
+    n16 = max(1, nbytes // 16)
+    buf = torch.ones(n16 * 4, dtype=torch.float32, device="cuda")
+    sink = torch.zeros(1, dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream()
+    reps = 20
+    best = 0.0
+    for _ in range(6):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        rc = lib.drr_probe_l2_read(buf.data_ptr(), n16, reps, sink.data_ptr(), stream.cuda_stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if rc != 0:
+            return None
+        best = max(best, n16 * 16 * reps / (e0.elapsed_time(e1) * 1e-3) / 1e9)
+    return best
+
+
+def traffic_for(kernel, workload_name):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current source of the kernel (else None)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        table = json.load(f)
+    entry = table.get(kernel, {}).get(workload_name)
+    if not entry:
+        return None
+    src = os.path.join(ROOT, entry["source"])
+    if not os.path.exists(src):
+        return None
+    digest = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    return entry["dram_bytes_per_launch"] if digest == entry["source_sha256_16"] else None
+
+
+# ---------------------------------------------------------------------------
+# the reference arm: the fp64 CPU oracle, timed on the host cores
+
+def run_reference(args):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    import oracle
+    oracle.build()
+    w = workload(args.config)
+    cores = len(os.sched_getaffinity(0))
+    per_view = w.H * w.W * w.n_samples
+
+    def step(b):
+        Rt = w.Rt[b:b + 1]
+        out = oracle.render(w.vol, w.dims, w.spacing, w.origin, w.K, Rt, w.H, w.W, w.n_samples,
+                            w.density_factor, w.mode, nthreads=cores)
+        oracle.adjoint(w.dims, w.spacing, w.origin, w.K, Rt, w.H, w.W, w.n_samples,
+                       w.density_factor, w.mode, w.grad_out[b:b + 1], vol=w.vol, nthreads=1)
+        return out
+
+    for s in range(args.warmup):
+        step(s % w.B)
+    t0 = time.perf_counter()
+    for s in range(args.steps):
+        step((args.warmup + s) % w.B)
+    dt = time.perf_counter() - t0
+    value = args.steps * per_view / dt / 1e9
+    sample = (f"one view per step ({w.H}x{w.W} rays x {w.n_samples} samples): fp64 forward "
+              f"threaded over rays on {cores} cores + fp64 adjoint on one thread")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "Gsamples/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_block(w, args.config, "linear"),
+        "cpu_baseline": {"value": value, "unit": "Gsamples/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "Gsamples/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# our arm
+
+def cpu_baseline(w):
+    """The oracle, as it stands, on a bounded sample of the same workload."""
+    import oracle
+    oracle.build()
+    cores = len(os.sched_getaffinity(0))
+    views = min(w.B, 16)
+    Rt = w.Rt[:views]
+    t0 = time.perf_counter()
+    oracle.render(w.vol, w.dims, w.spacing, w.origin, w.K, Rt, w.H, w.W, w.n_samples,
+                  w.density_factor, w.mode, nthreads=cores)
+    oracle.adjoint(w.dims, w.spacing, w.origin, w.K, Rt, w.H, w.W, w.n_samples,
+                   w.density_factor, w.mode, w.grad_out[:views], vol=w.vol,
+                   nthreads=min(cores, views))
+    dt = time.perf_counter() - t0
+    samples = views * w.H * w.W * w.n_samples
+    return {"value": samples / dt / 1e9, "unit": "Gsamples/s", "cores": cores, "kind": "oracle",
+            "sample": f"first {views} of {w.B} views, forward + adjoint (fp64), {dt:.1f} s"}
+
+
+def run_ours(args):
+    import torch
+    from cone_beam_ct_b200 import drr
+    from cone_beam_ct_b200 import workloads as wl
+
+    world, rank, local = dist_env()
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    drr.lib()
+
+    w = workload(args.config)
+    layout = drr.DRR_LAYOUT_PADDED
+    dtype = drr.DRR_BF16 if w.dtype == wl.DTYPE_BF16 else drr.DRR_F32
+    elem = 2 if dtype == drr.DRR_BF16 else 4
+    nx, ny, nz = w.dims
+    vol32 = torch.from_numpy(w.vol).to(dev)
+    Rt = torch.from_numpy(np.ascontiguousarray(w.Rt.reshape(-1, 12))).to(dev)
+    grad_out = torch.from_numpy(w.grad_out).to(dev)
+    pbytes = drr.drr_prepared_bytes(w.dims, dtype, layout)
+    prep = torch.empty(pbytes, dtype=torch.uint8, device=dev)
+    out = torch.empty((w.B, w.H, w.W), dtype=torch.float32, device=dev)
+    grad = torch.empty((nz, ny, nx), dtype=torch.float32, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    fwd_needed = w.mode == wl.MODE_BEER_LAMBERT
+
+    def step(events=None):
+        if events:
+            events[0].record(stream)
+        drr.drr_prepare_volume(vol32, w.dims, dtype, layout, prep, pbytes, stream=stream)
+        if events:
+            events[1].record(stream)
+        drr.drr_render(prep, dtype, layout, w.dims, w.spacing, w.origin, w.K, Rt, w.B, w.H, w.W,
+                       w.n_samples, w.density_factor, w.mode, out, stream=stream)
+        if events:
+            events[2].record(stream)
+        grad.zero_()
+        if events:
+            events[3].record(stream)
+        drr.drr_render_adjoint(w.dims, w.spacing, w.origin, w.K, Rt, w.B, w.H, w.W, w.n_samples,
+                               w.density_factor, w.mode, grad_out, out if fwd_needed else None,
+                               grad, stream=stream)
+        if events:
+            events[4].record(stream)
+
+    warmup_run = max(args.warmup, 3)          # never time a cold first step
+    for _ in range(warmup_run):
+        flush.fill_(1)
+        step()
+    torch.cuda.synchronize()
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    bracket = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(physical_gpu(dev.index)) as clk:
+        bracket[0].record(stream)
+        for s in range(args.steps):
+            flush.fill_(s & 0xFF)
+            step(ev[s])
+        bracket[1].record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+
+    per = np.array([[ev[s][i].elapsed_time(ev[s][i + 1]) for i in range(4)]
+                    for s in range(args.steps)])          # ms: prepare, forward, zero, adjoint
+    step_ms = per.sum(axis=1)
+    total_ms = float(step_ms.sum())
+    kern_ms = per.mean(axis=0)
+    if world > 1:
+        t = torch.tensor([total_ms] + list(kern_ms), dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(t[0])
+        kern_ms = t[1:].cpu().numpy()
+    ms_per_step = total_ms / args.steps
+    samples = w.samples
+    value = world * samples * args.steps / (total_ms * 1e-3) / 1e9
+    fps = world * w.B * args.steps / (total_ms * 1e-3)
+
+    # e2e through the public API with pinned host buffers
+    e2e = None
+    if not args.no_e2e:
+        h_vol = torch.from_numpy(w.vol).pin_memory()
+        h_Rt = torch.from_numpy(np.ascontiguousarray(w.Rt.reshape(-1, 12))).pin_memory()
+        h_go = torch.from_numpy(w.grad_out).pin_memory()
+        h_out = torch.empty((w.B, w.H, w.W), dtype=torch.float32).pin_memory()
+        h_grad = torch.empty((nz, ny, nx), dtype=torch.float32).pin_memory()
+
+        def e2e_step():
+            vol32.copy_(h_vol, non_blocking=True)
+            Rt.copy_(h_Rt, non_blocking=True)
+            grad_out.copy_(h_go, non_blocking=True)
+            step()
+            h_out.copy_(out, non_blocking=True)
+            h_grad.copy_(grad, non_blocking=True)
+            torch.cuda.current_stream().synchronize()
+
+        for _ in range(2):
+            e2e_step()
+        if world > 1:
+            torch.distributed.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            flush.fill_(0)
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = e0.elapsed_time(e1)
+        if world > 1:
+            t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+            e2e_ms = float(t[0])
+        h2d = h_vol.numel() * 4 + h_Rt.numel() * 4 + h_go.numel() * 4
+        d2h = h_out.numel() * 4 + h_grad.numel() * 4
+        e2e = {"value": world * samples * args.steps / (e2e_ms * 1e-3) / 1e9,
+               "unit": "Gsamples/s", "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "ms_per_step": e2e_ms / args.steps,
+               "note": "includes the 256 MiB L2 flush write before each step"}
+
+    # roofline of the dominant kernel
+    peaks, peak_src = measured_peaks()
+    fwd_ms, adj_ms = float(kern_ms[1]), float(kern_ms[3])
+    fwd_bytes = 8 * elem * samples            # 8 voxel reads per sample
+    adj_bytes = 8 * 4 * samples               # 8 fp32 atomic adds per sample
+    vol_fits_l2 = pbytes < L2_BYTES
+    l2_peak = l2_read_peak_gbs(torch, pbytes) if vol_fits_l2 else None
+    hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+
+    def roof(name, ms, nbytes, kernel_key, wname):
+        achieved = nbytes / (ms * 1e-3) / 1e9
+        if vol_fits_l2 and l2_peak:
+            bound, peak, src = "l2", l2_peak, "L2 read probe in this run (libdrr_probe.so)"
+        else:
+            bound, peak, src = "hbm", hbm_peak, f"MEASURED_PEAKS.json hbm_gbs ({peak_src})"
+        return {"kernel": name, "bound": bound, "achieved": achieved, "peak": peak,
+                "unit": "GB/s", "frac": achieved / peak, "peak_source": src,
+                "frac_of_hbm": achieved / hbm_peak,
+                "algorithmic_bytes_per_launch": int(nbytes), "ms_per_launch": ms,
+                "traffic": traffic_for(kernel_key, wname)}
+
+    wname = config_block(w, args.config, "")["workload"]
+    fwd_roof = roof("forward_kernel", fwd_ms, fwd_bytes, "forward_kernel", wname)
+    adj_roof = roof("adjoint_kernel", adj_ms, adj_bytes, "adjoint_kernel", wname)
+    dominant = adj_roof if adj_ms >= fwd_ms else fwd_roof
+
+    base = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        base = cpu_baseline(w)
+
+    clocks = clk.summary()
+    line = {
+        "metric": METRIC, "value": value, "unit": "Gsamples/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "warmup_run": warmup_run,
+        "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32", "data": "synthetic",
+        "config": config_block(w, args.config, "padded"),
+        "fps": fps,
+        "kernels_ms": {"prepare": float(kern_ms[0]), "forward": fwd_ms,
+                       "zero_grad (torch)": float(kern_ms[2]), "adjoint": adj_ms},
+        "forward": {"gsamples_s": samples / (fwd_ms * 1e-3) / 1e9,
+                    "fps": w.B / (fwd_ms * 1e-3), "roofline": fwd_roof},
+        "adjoint": {"gsamples_s": samples / (adj_ms * 1e-3) / 1e9, "roofline": adj_roof},
+        "roofline": dominant,
+        "cpu_baseline": base,
+        "e2e": e2e,
+        "gpu_launches": 3 * args.steps,
+        "clocks": clocks,
+        "bracket_ms": bracket[0].elapsed_time(bracket[1]),
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse_args()
+    if args.steps < 1 or args.warmup < 0:
+        raise SystemExit("--steps must be >= 1 and --warmup >= 0")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

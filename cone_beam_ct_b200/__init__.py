@@ -1,1 +1,21 @@
-"""B200-native cone-beam DRR ray-marcher (forward projection and its adjoint)."""
+"""B200-native cone-beam DRR ray-marcher (forward projection and its adjoint).
+
+The compute path is libdrr.so (hand-written sm_100a CUDA behind the C ABI of
+include/drr.h); ``cone_beam_ct_b200.drr`` binds it with the same names.
+``cone_beam_ct_b200.workloads`` makes seeded synthetic inputs.
+"""
+from .drr import (  # noqa: F401
+    DRR_BF16,
+    DRR_F32,
+    DRR_LAYOUT_LINEAR,
+    DRR_LAYOUT_PADDED,
+    DRR_MODE_BEER_LAMBERT,
+    DRR_MODE_RAW,
+    DrrError,
+    drr_abi_version,
+    drr_get_last_error,
+    drr_prepare_volume,
+    drr_prepared_bytes,
+    drr_render,
+    drr_render_adjoint,
+)

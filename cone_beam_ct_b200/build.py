@@ -1,0 +1,59 @@
+"""Build libdrr.so (the CUDA path) in-tree with nvcc for sm_100a.
+
+    python -m cone_beam_ct_b200.build [--force]
+
+No fast-math: expm1f / division / sqrt keep their IEEE behaviour.
+"""
+import os
+import subprocess
+import sys
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+CSRC = os.path.join(HERE, "csrc")
+INCLUDE = os.path.join(os.path.dirname(HERE), "include")
+LIB = os.path.join(HERE, "libdrr.so")
+PROBE_LIB = os.path.join(HERE, "libdrr_probe.so")
+SOURCES = ["drr_api.cu", "drr_forward.cu", "drr_adjoint.cu", "drr_prepare.cu"]
+HEADERS = ["drr_internal.cuh"]
+PROBE_SOURCES = ["drr_probe.cu"]
+ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
+FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-fvisibility=hidden",
+         "-shared", "-cudart", "shared"]
+
+
+def _nvcc():
+    home = os.environ.get("CUDA_HOME", "/usr/local/cuda")
+    cand = os.path.join(home, "bin", "nvcc")
+    return cand if os.path.exists(cand) else "nvcc"
+
+
+def _stale(lib, sources, headers):
+    if not os.path.exists(lib):
+        return True
+    t = os.path.getmtime(lib)
+    deps = [os.path.join(CSRC, f) for f in sources + headers]
+    deps += [os.path.join(INCLUDE, h) for h in ("drr.h", "drr_probe.h")]
+    return any(os.path.getmtime(d) > t for d in deps)
+
+
+def _nvcc_shared(lib, sources, verbose_ptxas):
+    cmd = [_nvcc()] + ARCH + FLAGS + ["-I", INCLUDE, "-o", lib + ".tmp"]
+    if verbose_ptxas:
+        cmd += ["-Xptxas", "-v"]
+    cmd += [os.path.join(CSRC, f) for f in sources]
+    subprocess.check_call(cmd)
+    os.replace(lib + ".tmp", lib)
+
+
+def build(force: bool = False, verbose_ptxas: bool = False) -> str:
+    """Build libdrr.so (the ray-march) and libdrr_probe.so (the bench's L2
+    bandwidth probe); returns the path of libdrr.so."""
+    if force or _stale(LIB, SOURCES, HEADERS):
+        _nvcc_shared(LIB, SOURCES, verbose_ptxas)
+    if force or _stale(PROBE_LIB, PROBE_SOURCES, []):
+        _nvcc_shared(PROBE_LIB, PROBE_SOURCES, verbose_ptxas)
+    return LIB
+
+
+if __name__ == "__main__":
+    print(build(force="--force" in sys.argv, verbose_ptxas="-v" in sys.argv))

@@ -1,0 +1,221 @@
+// drr_api.cu -- the extern "C" entry points of libdrr.so (include/drr.h).
+//
+// Host side only: validate every argument before touching the device,
+// precompute K^-1 in double, fill the kernel parameter block and launch on
+// the caller's stream.  No allocation, no synchronisation, no state kept
+// between calls (the last-error string is per thread).
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+
+#include "../../include/drr.h"
+#include "drr_internal.cuh"
+
+namespace {
+
+thread_local char g_last_error[512] = "";
+
+drr_status fail(drr_status st, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+    va_end(ap);
+    return st;
+}
+
+drr_status ok() {
+    g_last_error[0] = '\0';
+    return DRR_OK;
+}
+
+drr_status cuda_status(cudaError_t e, const char* what) {
+    if (e == cudaSuccess) return ok();
+    return fail(DRR_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+constexpr int kMaxSamples = 1 << 20;
+constexpr int kMaxViews = 65535;
+constexpr int kMaxRows = 65535 * drr::kTileH;
+constexpr int64_t kMaxElements = (int64_t(1) << 31) - 1;
+constexpr int kMaxDim = (1 << 22) - 4;   // keeps padded coordinates inside the exact floor range
+
+int64_t stored_elements(const int dims[3], int layout) {
+    const int pad = layout == DRR_LAYOUT_PADDED ? 2 : 0;
+    return (int64_t)(dims[0] + pad) * (dims[1] + pad) * (dims[2] + pad);
+}
+
+drr_status check_volume(const int dims[3], const float spacing[3], const float origin[3]) {
+    if (!dims || !spacing || !origin) return fail(DRR_ERR_INVALID_ARG, "dims, spacing and origin must be non-NULL");
+    for (int a = 0; a < 3; ++a) {
+        if (dims[a] < 2 || dims[a] > kMaxDim)
+            return fail(DRR_ERR_INVALID_ARG, "dims[%d] = %d must be in [2, %d]", a, dims[a], kMaxDim);
+        if (!(spacing[a] > 0.0f) || !std::isfinite(spacing[a]))
+            return fail(DRR_ERR_INVALID_ARG, "spacing[%d] must be finite and > 0", a);
+        if (!std::isfinite(origin[a])) return fail(DRR_ERR_INVALID_ARG, "origin[%d] must be finite", a);
+    }
+    return DRR_OK;
+}
+
+drr_status check_rays(const float K[9], const float* Rt, int B, int H, int W, int n_samples,
+                      float density_factor, int mode) {
+    if (!K) return fail(DRR_ERR_INVALID_ARG, "K must be a non-NULL host array of 9 floats");
+    for (int m = 0; m < 9; ++m)
+        if (!std::isfinite(K[m])) return fail(DRR_ERR_INVALID_ARG, "K[%d] is not finite", m);
+    if (K[3] != 0.0f || K[6] != 0.0f || K[7] != 0.0f)
+        return fail(DRR_ERR_INVALID_ARG, "K must be upper triangular (K[3] = K[6] = K[7] = 0)");
+    if (K[0] == 0.0f || K[4] == 0.0f || K[8] == 0.0f)
+        return fail(DRR_ERR_INVALID_ARG, "K must be invertible (K[0], K[4], K[8] non-zero)");
+    if (B < 0 || H < 0 || W < 0) return fail(DRR_ERR_INVALID_ARG, "B, H, W must be >= 0");
+    if (B > kMaxViews) return fail(DRR_ERR_UNSUPPORTED, "B = %d exceeds %d views per call", B, kMaxViews);
+    if (H > kMaxRows) return fail(DRR_ERR_UNSUPPORTED, "H = %d exceeds %d rows", H, kMaxRows);
+    if ((int64_t)B * H * W >= (int64_t(1) << 40)) return fail(DRR_ERR_UNSUPPORTED, "B*H*W too large");
+    if (n_samples < 1 || n_samples > kMaxSamples)
+        return fail(DRR_ERR_INVALID_ARG, "n_samples = %d must be in [1, %d]", n_samples, kMaxSamples);
+    if (!std::isfinite(density_factor)) return fail(DRR_ERR_INVALID_ARG, "density_factor must be finite");
+    if (mode != DRR_MODE_RAW && mode != DRR_MODE_BEER_LAMBERT)
+        return fail(DRR_ERR_INVALID_ARG, "unknown mode %d", mode);
+    if ((int64_t)B * H * W > 0 && (!Rt || !aligned(Rt, 4)))
+        return fail(DRR_ERR_INVALID_ARG, "Rt must be a non-NULL, 4-byte aligned device pointer");
+    return DRR_OK;
+}
+
+void fill_geom(drr::Geom& g, const int dims[3], const float spacing[3], const float origin[3],
+               const float K[9], int B, int H, int W, int n_samples, float density_factor,
+               int layout) {
+    std::memset(&g, 0, sizeof(g));
+    g.nx = dims[0];
+    g.ny = dims[1];
+    g.nz = dims[2];
+    const int pad = layout == DRR_LAYOUT_PADDED ? 2 : 0;
+    g.row = dims[0] + pad;
+    g.slice = (dims[0] + pad) * (dims[1] + pad);
+    for (int a = 0; a < 3; ++a) {
+        g.hi[a] = (float)(dims[a] - 1);
+        g.hi_clamp[a] = std::nextafter(g.hi[a], 0.0f);
+        g.inv_sp[a] = (float)(1.0 / (double)spacing[a]);
+        g.origin[a] = origin[a];
+    }
+    // inverse of the upper-triangular K in double
+    const double k0 = K[0], k1 = K[1], k2 = K[2], k4 = K[4], k5 = K[5], k8 = K[8];
+    g.kinv[0] = (float)(1.0 / k0);
+    g.kinv[1] = (float)(-k1 / (k0 * k4));
+    g.kinv[2] = (float)((k1 * k5 - k2 * k4) / (k0 * k4 * k8));
+    g.kinv[3] = (float)(1.0 / k4);
+    g.kinv[4] = (float)(-k5 / (k4 * k8));
+    g.kinv[5] = (float)(1.0 / k8);
+    g.B = B;
+    g.H = H;
+    g.W = W;
+    g.N = n_samples;
+    g.density_factor = density_factor;
+}
+
+bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+    const uintptr_t pa = reinterpret_cast<uintptr_t>(a), pb = reinterpret_cast<uintptr_t>(b);
+    return pa < pb + nb && pb < pa + na;
+}
+
+}  // namespace
+
+extern "C" {
+
+DRR_API int drr_abi_version(void) { return 1; }
+
+DRR_API const char* drr_get_last_error(void) { return g_last_error; }
+
+DRR_API size_t drr_prepared_bytes(const int dims[3], drr_dtype dtype, drr_layout layout) {
+    if (!dims) return 0;
+    for (int a = 0; a < 3; ++a)
+        if (dims[a] < 2 || dims[a] > kMaxDim) return 0;
+    if (dtype != DRR_F32 && dtype != DRR_BF16) return 0;
+    if (layout != DRR_LAYOUT_LINEAR && layout != DRR_LAYOUT_PADDED) return 0;
+    const int64_t n = stored_elements(dims, layout);
+    if (n > kMaxElements) return 0;
+    return (size_t)n * (dtype == DRR_F32 ? 4 : 2);
+}
+
+DRR_API drr_status drr_prepare_volume(const float* src, const int dims[3], drr_dtype dtype,
+                                      drr_layout layout, void* dst, size_t dst_bytes,
+                                      void* stream) {
+    if (!dims) return fail(DRR_ERR_INVALID_ARG, "dims must be non-NULL");
+    for (int a = 0; a < 3; ++a)
+        if (dims[a] < 2 || dims[a] > kMaxDim)
+            return fail(DRR_ERR_INVALID_ARG, "dims[%d] = %d must be in [2, %d]", a, dims[a], kMaxDim);
+    if (dtype != DRR_F32 && dtype != DRR_BF16) return fail(DRR_ERR_INVALID_ARG, "unknown dtype %d", dtype);
+    if (layout != DRR_LAYOUT_LINEAR && layout != DRR_LAYOUT_PADDED)
+        return fail(DRR_ERR_INVALID_ARG, "unknown layout %d", layout);
+    const size_t need = drr_prepared_bytes(dims, dtype, layout);
+    if (need == 0) return fail(DRR_ERR_UNSUPPORTED, "volume too large (max 2^31 - 1 stored elements)");
+    if (!src || !dst) return fail(DRR_ERR_INVALID_ARG, "src and dst must be non-NULL");
+    if (!aligned(src, 4) || !aligned(dst, 4)) return fail(DRR_ERR_INVALID_ARG, "src and dst must be 4-byte aligned");
+    if (dst_bytes < need)
+        return fail(DRR_ERR_INVALID_ARG, "dst holds %zu bytes, %zu needed", dst_bytes, need);
+    const size_t src_bytes = (size_t)dims[0] * dims[1] * dims[2] * 4;
+    if (overlaps(src, src_bytes, dst, need)) return fail(DRR_ERR_INVALID_ARG, "src and dst overlap");
+    return cuda_status(drr::launch_prepare(src, dims[0], dims[1], dims[2], dtype, layout, dst,
+                                           static_cast<cudaStream_t>(stream)),
+                       "drr_prepare_volume launch");
+}
+
+DRR_API drr_status drr_render(const void* vol, drr_dtype dtype, drr_layout layout,
+                              const int dims[3], const float spacing[3], const float origin[3],
+                              const float K[9], const float* Rt, int B, int H, int W,
+                              int n_samples, float density_factor, drr_mode mode, float* out,
+                              void* stream) {
+    drr_status st = check_volume(dims, spacing, origin);
+    if (st != DRR_OK) return st;
+    st = check_rays(K, Rt, B, H, W, n_samples, density_factor, mode);
+    if (st != DRR_OK) return st;
+    if (dtype != DRR_F32 && dtype != DRR_BF16) return fail(DRR_ERR_INVALID_ARG, "unknown dtype %d", dtype);
+    if (layout != DRR_LAYOUT_LINEAR && layout != DRR_LAYOUT_PADDED)
+        return fail(DRR_ERR_INVALID_ARG, "unknown layout %d", layout);
+    if (stored_elements(dims, layout) > kMaxElements)
+        return fail(DRR_ERR_UNSUPPORTED, "volume too large (max 2^31 - 1 stored elements)");
+    if ((int64_t)B * H * W == 0) return ok();   // empty batch or image: nothing to do
+    if (!vol || !aligned(vol, dtype == DRR_F32 ? 4 : 2))
+        return fail(DRR_ERR_INVALID_ARG, "vol must be a non-NULL, element-aligned device pointer");
+    if (!out || !aligned(out, 4)) return fail(DRR_ERR_INVALID_ARG, "out must be a non-NULL, 4-byte aligned device pointer");
+    drr::Geom g;
+    fill_geom(g, dims, spacing, origin, K, B, H, W, n_samples, density_factor, layout);
+    return cuda_status(drr::launch_forward(vol, dtype, layout, g, Rt, mode, out,
+                                           static_cast<cudaStream_t>(stream)),
+                       "drr_render launch");
+}
+
+DRR_API drr_status drr_render_adjoint(const int dims[3], const float spacing[3],
+                                      const float origin[3], const float K[9], const float* Rt,
+                                      int B, int H, int W, int n_samples, float density_factor,
+                                      drr_mode mode, const float* grad_out, const float* fwd_out,
+                                      float* grad_vol, void* stream) {
+    drr_status st = check_volume(dims, spacing, origin);
+    if (st != DRR_OK) return st;
+    st = check_rays(K, Rt, B, H, W, n_samples, density_factor, mode);
+    if (st != DRR_OK) return st;
+    if (stored_elements(dims, DRR_LAYOUT_LINEAR) > kMaxElements)
+        return fail(DRR_ERR_UNSUPPORTED, "volume too large (max 2^31 - 1 elements)");
+    const int64_t npix = (int64_t)B * H * W;
+    if (npix == 0) return ok();
+    if (!grad_out || !aligned(grad_out, 4))
+        return fail(DRR_ERR_INVALID_ARG, "grad_out must be a non-NULL, 4-byte aligned device pointer");
+    if (mode == DRR_MODE_BEER_LAMBERT && (!fwd_out || !aligned(fwd_out, 4)))
+        return fail(DRR_ERR_INVALID_ARG, "fwd_out is required in Beer-Lambert mode");
+    if (!grad_vol || !aligned(grad_vol, 4))
+        return fail(DRR_ERR_INVALID_ARG, "grad_vol must be a non-NULL, 4-byte aligned device pointer");
+    const size_t vbytes = (size_t)dims[0] * dims[1] * dims[2] * 4, ibytes = (size_t)npix * 4;
+    if (overlaps(grad_vol, vbytes, grad_out, ibytes) ||
+        (mode == DRR_MODE_BEER_LAMBERT && overlaps(grad_vol, vbytes, fwd_out, ibytes)))
+        return fail(DRR_ERR_INVALID_ARG, "grad_vol overlaps an image buffer");
+    drr::Geom g;
+    fill_geom(g, dims, spacing, origin, K, B, H, W, n_samples, density_factor, DRR_LAYOUT_LINEAR);
+    return cuda_status(drr::launch_adjoint(g, Rt, mode, grad_out, fwd_out, grad_vol,
+                                           static_cast<cudaStream_t>(stream)),
+                       "drr_render_adjoint launch");
+}
+
+}  // extern "C"

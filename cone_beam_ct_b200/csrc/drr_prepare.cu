@@ -1,0 +1,83 @@
+// drr_prepare.cu -- volume re-layout / conversion kernels (sm_100a).
+//
+// fp32 -> bf16 storage rounds to nearest even (the bf16 rendering mode of
+// nanodrr's page, "Benchmarks": mixed precision; here storage only, the
+// arithmetic stays fp32).  The padded layout surrounds the volume with a
+// one-voxel zero border, which is exactly the zero padding of the trilinear
+// interpolation.  Plain grid-stride loops: a one-off HBM-bound copy.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "drr_internal.cuh"
+
+namespace drr {
+namespace {
+
+template <typename T>
+__device__ __forceinline__ T store_value(float x);
+
+template <>
+__device__ __forceinline__ float store_value<float>(float x) {
+    return x;
+}
+
+template <>
+__device__ __forceinline__ uint16_t store_value<uint16_t>(float x) {
+    return __bfloat16_as_ushort(__float2bfloat16_rn(x));
+}
+
+template <typename T>
+__global__ void to_linear(const float* __restrict__ src, T* __restrict__ dst, int64_t n) {
+    for (int64_t m = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; m < n;
+         m += (int64_t)gridDim.x * blockDim.x)
+        dst[m] = store_value<T>(__ldg(src + m));
+}
+
+template <typename T>
+__global__ void to_padded(const float* __restrict__ src, T* __restrict__ dst, int nx, int ny,
+                          int nz) {
+    const int px = nx + 2, py = ny + 2;
+    const int64_t n = (int64_t)px * py * (nz + 2);
+    for (int64_t m = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; m < n;
+         m += (int64_t)gridDim.x * blockDim.x) {
+        const int i = (int)(m % px);
+        const int j = (int)((m / px) % py);
+        const int k = (int)(m / ((int64_t)px * py));
+        float v = 0.0f;
+        if (i >= 1 && i <= nx && j >= 1 && j <= ny && k >= 1 && k <= nz)
+            v = __ldg(src + (((int64_t)(k - 1) * ny + (j - 1)) * nx + (i - 1)));
+        dst[m] = store_value<T>(v);
+    }
+}
+
+int grid_for(int64_t n) {
+    int64_t blocks = (n + 255) / 256;
+    const int64_t cap = 148 * 16;   // enough CTAs to fill every SM; the loops stride
+    return (int)(blocks < cap ? (blocks > 0 ? blocks : 1) : cap);
+}
+
+}  // namespace
+
+cudaError_t launch_prepare(const float* src, int nx, int ny, int nz, int dtype, int layout,
+                           void* dst, cudaStream_t stream) {
+    if (layout == 0) {
+        const int64_t n = (int64_t)nx * ny * nz;
+        if (dtype == 0)
+            to_linear<float><<<grid_for(n), 256, 0, stream>>>(src, static_cast<float*>(dst), n);
+        else
+            to_linear<uint16_t><<<grid_for(n), 256, 0, stream>>>(src, static_cast<uint16_t*>(dst),
+                                                                 n);
+    } else {
+        const int64_t n = (int64_t)(nx + 2) * (ny + 2) * (nz + 2);
+        if (dtype == 0)
+            to_padded<float><<<grid_for(n), 256, 0, stream>>>(src, static_cast<float*>(dst), nx,
+                                                              ny, nz);
+        else
+            to_padded<uint16_t><<<grid_for(n), 256, 0, stream>>>(
+                src, static_cast<uint16_t*>(dst), nx, ny, nz);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace drr

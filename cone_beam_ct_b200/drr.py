@@ -1,0 +1,152 @@
+"""Python binding of libdrr.so: the C ABI of include/drr.h, same names.
+
+Argument marshalling only -- every step of the ray-march runs in the CUDA
+kernels of libdrr.so.  Device arguments are CUDA tensors (or raw device
+addresses as int); host arguments (dims, spacing, origin, K) are sequences
+or numpy arrays.  ``stream`` defaults to torch's current CUDA stream.  A
+non-OK status raises DrrError with the library's own message.  If the
+library has not been built, every call raises: there is no fallback.
+"""
+import ctypes
+import os
+
+import numpy as np
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libdrr.so")
+
+DRR_OK, DRR_ERR_INVALID_ARG, DRR_ERR_UNSUPPORTED, DRR_ERR_CUDA = 0, 1, 2, 3
+DRR_MODE_RAW, DRR_MODE_BEER_LAMBERT = 0, 1
+DRR_F32, DRR_BF16 = 0, 1
+DRR_LAYOUT_LINEAR, DRR_LAYOUT_PADDED = 0, 1
+
+# names exported by libdrr.so (include/drr.h)
+EXPORTED = ("drr_render", "drr_render_adjoint", "drr_prepared_bytes", "drr_prepare_volume",
+            "drr_get_last_error", "drr_abi_version")
+
+
+class DrrError(RuntimeError):
+    def __init__(self, status, message):
+        super().__init__(f"libdrr status {status}: {message}")
+        self.status = status
+
+
+_lib = None
+_c = ctypes
+_vp = ctypes.c_void_p
+_i3 = ctypes.c_int * 3
+_f3 = ctypes.c_float * 3
+_f9 = ctypes.c_float * 9
+
+
+def lib():
+    """The loaded libdrr.so (built in-tree by cone_beam_ct_b200.build)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"libdrr.so is not built ({LIB_PATH}); run "
+                           "`python -m cone_beam_ct_b200.build` -- there is no CPU fallback")
+    L = ctypes.CDLL(LIB_PATH)
+    L.drr_render.argtypes = [_vp, _c.c_int, _c.c_int, _i3, _f3, _f3, _f9, _vp, _c.c_int,
+                             _c.c_int, _c.c_int, _c.c_int, _c.c_float, _c.c_int, _vp, _vp]
+    L.drr_render.restype = _c.c_int
+    L.drr_render_adjoint.argtypes = [_i3, _f3, _f3, _f9, _vp, _c.c_int, _c.c_int, _c.c_int,
+                                     _c.c_int, _c.c_float, _c.c_int, _vp, _vp, _vp, _vp]
+    L.drr_render_adjoint.restype = _c.c_int
+    L.drr_prepared_bytes.argtypes = [_i3, _c.c_int, _c.c_int]
+    L.drr_prepared_bytes.restype = _c.c_size_t
+    L.drr_prepare_volume.argtypes = [_vp, _i3, _c.c_int, _c.c_int, _vp, _c.c_size_t, _vp]
+    L.drr_prepare_volume.restype = _c.c_int
+    L.drr_get_last_error.argtypes = []
+    L.drr_get_last_error.restype = _c.c_char_p
+    L.drr_abi_version.argtypes = []
+    L.drr_abi_version.restype = _c.c_int
+    _lib = L
+    return L
+
+
+def _dev(x, name, allow_none=False):
+    """Device address of a CUDA tensor (or an int address)."""
+    if x is None:
+        if allow_none:
+            return None
+        raise TypeError(f"{name} must be a CUDA tensor or a device address")
+    if isinstance(x, int):
+        return x
+    if not getattr(x, "is_cuda", False):
+        raise TypeError(f"{name} must live on a CUDA device")
+    if not x.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return x.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _i3v(v):
+    a = np.asarray(v, dtype=np.int64).reshape(-1)
+    if a.size != 3:
+        raise ValueError("expected 3 values")
+    return _i3(*(int(x) for x in a))
+
+
+def _f3v(v):
+    a = np.asarray(v, dtype=np.float32).reshape(-1)
+    if a.size != 3:
+        raise ValueError("expected 3 values")
+    return _f3(*(float(x) for x in a))
+
+
+def _f9v(v):
+    a = np.asarray(v, dtype=np.float32).reshape(-1)
+    if a.size != 9:
+        raise ValueError("K must have 9 values")
+    return _f9(*(float(x) for x in a))
+
+
+def _check(status):
+    if status != DRR_OK:
+        raise DrrError(status, drr_get_last_error())
+
+
+def drr_get_last_error():
+    return lib().drr_get_last_error().decode()
+
+
+def drr_abi_version():
+    return lib().drr_abi_version()
+
+
+def drr_prepared_bytes(dims, dtype, layout):
+    return int(lib().drr_prepared_bytes(_i3v(dims), int(dtype), int(layout)))
+
+
+def drr_prepare_volume(src, dims, dtype, layout, dst, dst_bytes=None, stream=None):
+    if dst_bytes is None:
+        dst_bytes = dst.numel() * dst.element_size()
+    _check(lib().drr_prepare_volume(_dev(src, "src"), _i3v(dims), int(dtype), int(layout),
+                                    _dev(dst, "dst"), int(dst_bytes), _stream(stream)))
+
+
+def drr_render(vol, dtype, layout, dims, spacing, origin, K, Rt, B, H, W, n_samples,
+               density_factor, mode, out, stream=None):
+    _check(lib().drr_render(_dev(vol, "vol", True), int(dtype), int(layout), _i3v(dims),
+                            _f3v(spacing), _f3v(origin), _f9v(K), _dev(Rt, "Rt", True), int(B),
+                            int(H), int(W), int(n_samples), float(density_factor), int(mode),
+                            _dev(out, "out", True), _stream(stream)))
+
+
+def drr_render_adjoint(dims, spacing, origin, K, Rt, B, H, W, n_samples, density_factor, mode,
+                       grad_out, fwd_out, grad_vol, stream=None):
+    _check(lib().drr_render_adjoint(_i3v(dims), _f3v(spacing), _f3v(origin), _f9v(K),
+                                    _dev(Rt, "Rt", True), int(B), int(H), int(W), int(n_samples),
+                                    float(density_factor), int(mode),
+                                    _dev(grad_out, "grad_out", True),
+                                    _dev(fwd_out, "fwd_out", True),
+                                    _dev(grad_vol, "grad_vol", True), _stream(stream)))

@@ -132,44 +132,55 @@ class Ellipsoid:
     value: float            # additive value (HU or mu)
 
 
-def _slab_coordinates(dims, spacing, origin, k_lo, k_hi):
-    nx, ny, _ = dims
-    x = origin[0] + spacing[0] * np.arange(nx, dtype=np.float64)
-    y = origin[1] + spacing[1] * np.arange(ny, dtype=np.float64)
-    z = origin[2] + spacing[2] * np.arange(k_lo, k_hi, dtype=np.float64)
-    Z, Y, X = np.meshgrid(z, y, x, indexing="ij")
-    return X, Y, Z
+def _index_range(centre, half, origin, spacing, n):
+    lo = int(np.floor((centre - half - origin) / spacing)) - 1
+    hi = int(np.ceil((centre + half - origin) / spacing)) + 2
+    return max(lo, 0), min(hi, n)
+
+
+def _inside_box(e: Ellipsoid, spacing, origin, rng) -> np.ndarray:
+    """Voxel centres of the index box ``rng`` that lie inside ``e``.  The
+    ellipsoid-frame coordinates are sums of per-axis terms, so the quadratic
+    form is assembled from 1-D coordinate vectors by broadcasting."""
+    axes = [origin[a] + spacing[a] * np.arange(rng[a][0], rng[a][1], dtype=np.float64)
+            - e.centre[a] for a in range(3)]
+    X = axes[0][None, None, :]
+    Y = axes[1][None, :, None]
+    Z = axes[2][:, None, None]
+    q = np.zeros((len(axes[2]), len(axes[1]), len(axes[0])))
+    for m in range(3):      # coordinate along the ellipsoid's m-th axis
+        loc = X * e.rotation[0, m] + Y * e.rotation[1, m] + Z * e.rotation[2, m]
+        q += (loc / e.semi_axes[m]) ** 2
+    return q <= 1.0
+
+
+def _add_ellipsoid(out: np.ndarray, dims, spacing, origin, e: Ellipsoid,
+                   mask: Optional[Ellipsoid] = None) -> None:
+    """out[k][j][i] += e.value where the voxel centre lies inside e (and
+    inside ``mask``), evaluated on the ellipsoid's bounding box only."""
+    half = np.sqrt(((e.rotation * e.semi_axes[None, :]) ** 2).sum(axis=1))
+    rng = [_index_range(e.centre[a], half[a], origin[a], spacing[a], dims[a]) for a in range(3)]
+    if any(lo >= hi for lo, hi in rng):
+        return
+    inside = _inside_box(e, spacing, origin, rng)
+    if mask is not None:
+        inside &= _inside_box(mask, spacing, origin, rng)
+    out[rng[2][0]:rng[2][1], rng[1][0]:rng[1][1], rng[0][0]:rng[0][1]] += inside * e.value
 
 
 def voxelize(dims: Sequence[int], spacing: Sequence[float], origin: Sequence[float],
              ellipsoids: Sequence[Ellipsoid], background: float = 0.0,
-             mask: Optional[Ellipsoid] = None, slab: int = 32) -> np.ndarray:
+             mask: Optional[Ellipsoid] = None) -> np.ndarray:
     """Sum of ellipsoid indicator functions (voxel centre inside) times value,
     on a ``vol[k][j][i]`` float64 grid.  ``mask`` (optional) zeroes the
     ellipsoid contributions outside another ellipsoid."""
-    nx, ny, nz = dims
-    out = np.empty((nz, ny, nx), dtype=np.float64)
-    for k_lo in range(0, nz, slab):
-        k_hi = min(nz, k_lo + slab)
-        X, Y, Z = _slab_coordinates(dims, spacing, origin, k_lo, k_hi)
-        P = np.stack([X, Y, Z], axis=-1)
-        acc = np.full(X.shape, background, dtype=np.float64)
-        msk = None
-        if mask is not None:
-            msk = _inside(P, mask)
-        for e in ellipsoids:
-            inside = _inside(P, e)
-            if msk is not None:
-                inside &= msk
-            acc += inside * e.value
-        out[k_lo:k_hi] = acc
+    nx, ny, nz = (int(n) for n in dims)
+    sp = np.asarray(spacing, dtype=np.float64)
+    org = np.asarray(origin, dtype=np.float64)
+    out = np.full((nz, ny, nx), background, dtype=np.float64)
+    for e in ellipsoids:
+        _add_ellipsoid(out, (nx, ny, nz), sp, org, e, mask)
     return out
-
-
-def _inside(P: np.ndarray, e: Ellipsoid) -> np.ndarray:
-    local = (P - e.centre) @ e.rotation          # coordinates along ellipsoid axes
-    q = (local / e.semi_axes) ** 2
-    return q.sum(axis=-1) <= 1.0
 
 
 def hu_to_mu(hu: np.ndarray) -> np.ndarray:

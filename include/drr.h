@@ -1,0 +1,166 @@
+/*
+ * drr.h -- C ABI of the B200 cone-beam DRR ray-marcher (libdrr.so).
+ *
+ * What the library computes (all entry points follow the same geometry):
+ *
+ *   A digitally reconstructed radiograph of a 3-D attenuation volume seen by
+ *   a pinhole camera.  For every detector pixel of every view, a ray leaves
+ *   the source through the pixel centre (Hartley-Zisserman camera
+ *   x ~ K [R | t] X: nanodrr page, introduction), is clipped to the volume
+ *   box with the slab method (flashdrr.rendering API docs,
+ *   VolumeRaycaster.compute_clipping_distances: near/far from the volume
+ *   bounds), is sampled n_samples times uniformly with zero-padded trilinear
+ *   interpolation in IJK voxel space (VolumeRaycaster.forward: the volume
+ *   lives in IJK space, an affine maps world to IJK; VolumeRaycaster.__init__:
+ *   ray_samples), and yields I = density_factor * sum(mu * dt)
+ *   (VolumeRaycaster.__init__: density_factor), written raw or as the
+ *   Beer-Lambert image 1 - exp(-I) (VolumeRaycaster.__init__:
+ *   use_beer_lambert).  The adjoint scatters an image-space gradient back
+ *   along the same rays (TorchTomo page, "Discrete Adjoint and Learned
+ *   Primal-Dual": <A x, y> = <x, A^T y>; FlashDRR page, "Train vs. Eval
+ *   Dynamics": backward gradient kernels of the fused renderer).
+ *
+ * Conventions shared by every entry point
+ *
+ *   volume    vol[k][j][i], i fastest; dims = {nx, ny, nz}, each >= 2.
+ *             World position of voxel (i, j, k) = origin + spacing * (i, j, k):
+ *             origin (mm) is the CENTRE of voxel 0, spacing (mm) > 0.
+ *   box       rays are clipped to the box spanned by the voxel centres,
+ *             [0, n-1] per axis in IJK.  Samples: midpoint rule,
+ *             dt = (t1 - t0) / n_samples, t_i = t0 + (i + 1/2) dt, with
+ *             t0 = max(t_near, 0), t1 = t_far in world mm along the unit
+ *             ray; t1 <= t0 is a miss and gives I = 0.
+ *   camera    K: HOST array, 9 floats row-major, upper triangular
+ *             [fx s cx; 0 fy cy; 0 0 k22], fx, fy, k22 non-zero.
+ *             Rt: DEVICE array, B x 12 floats, row-major [R | t] per view,
+ *             world -> camera, R a rotation.  Pixel (row r, col c) has its
+ *             centre at (u, v) = (c, r); camera +z looks into the scene.
+ *   images    out / grad_out / fwd_out: DEVICE, float32 [B][H][W].
+ *   stream    a cudaStream_t passed as void* (NULL = legacy default stream).
+ *
+ * Ownership and semantics: the caller owns every buffer.  The library keeps
+ * no state between calls and allocates no device memory.  Host arrays
+ * (dims, spacing, origin, K) are read during the call only.  Every call is
+ * asynchronous on `stream`; results are valid once the stream has reached
+ * the work.  All device pointers must be 4-byte aligned and must stay valid
+ * until the work completes.
+ *
+ * Errors: arguments are checked on the host before anything is launched;
+ * DRR_ERR_INVALID_ARG / DRR_ERR_UNSUPPORTED return without touching the
+ * device.  A failed launch returns DRR_ERR_CUDA.  Faults of earlier
+ * asynchronous work surface at the caller's next synchronisation, as in
+ * CUDA.  drr_get_last_error() describes the last failure of this thread.
+ * No C++ exception crosses the ABI.  The kernels contain no waits, so a
+ * launch always terminates; a ray whose geometry is not finite (NaN/inf in
+ * Rt) is treated as a miss.
+ */
+#ifndef DRR_H
+#define DRR_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define DRR_API __attribute__((visibility("default")))
+#else
+#define DRR_API
+#endif
+
+typedef enum {
+    DRR_OK = 0,
+    DRR_ERR_INVALID_ARG = 1,   /* bad pointer, size, enum value or geometry */
+    DRR_ERR_UNSUPPORTED = 2,   /* valid but not implemented (e.g. too large) */
+    DRR_ERR_CUDA = 3           /* a CUDA launch or query failed */
+} drr_status;
+
+typedef enum {
+    DRR_MODE_RAW = 0,          /* out = I */
+    DRR_MODE_BEER_LAMBERT = 1  /* out = 1 - exp(-I), evaluated as -expm1(-I) */
+} drr_mode;
+
+typedef enum {
+    DRR_F32 = 0,               /* float32 voxels */
+    DRR_BF16 = 1               /* bfloat16 voxels (round-to-nearest-even), fp32 arithmetic */
+} drr_dtype;
+
+typedef enum {
+    /* vol[k][j][i] exactly as the caller holds it (float32 or bfloat16). */
+    DRR_LAYOUT_LINEAR = 0,
+    /* vol[k+1][j+1][i+1] inside a one-voxel zero border: dims (nx+2, ny+2,
+       nz+2).  Written by drr_prepare_volume.  The border is the zero padding
+       of the interpolation, so the sample loop needs no clamping. */
+    DRR_LAYOUT_PADDED = 1
+} drr_layout;
+
+/* Forward projection.
+ *   vol         DEVICE, volume in `layout` and `dtype` (LINEAR: nx*ny*nz
+ *               elements; other layouts: as written by drr_prepare_volume).
+ *   dims        HOST int[3] {nx, ny, nz}, each in [2, 2^22 - 4].
+ *   spacing     HOST float[3] voxel size (mm), > 0.
+ *   origin      HOST float[3] centre of voxel 0 (mm).
+ *   K           HOST float[9] intrinsics (see conventions).
+ *   Rt          DEVICE float[B*12] extrinsics.
+ *   B, H, W     views and detector rows / columns, >= 0 (any of them 0:
+ *               nothing to do, DRR_OK); B <= 65535.
+ *   n_samples   samples per ray, 1 <= n_samples <= 1048576.
+ *   density_factor  finite scale of the integral.
+ *   mode        DRR_MODE_RAW or DRR_MODE_BEER_LAMBERT.
+ *   out         DEVICE float[B*H*W], overwritten.
+ * Limits: the volume (with its border, for PADDED) must hold fewer than
+ * 2^31 elements; B*H*W < 2^40.
+ */
+DRR_API drr_status drr_render(const void *vol, drr_dtype dtype, drr_layout layout,
+                              const int dims[3], const float spacing[3], const float origin[3],
+                              const float K[9], const float *Rt, int B, int H, int W,
+                              int n_samples, float density_factor, drr_mode mode, float *out,
+                              void *stream);
+
+/* Adjoint (transpose) of drr_render with respect to the volume, i.e. the
+ * volume gradient of sum(grad_out * out).
+ *   grad_out    DEVICE float[B*H*W], upstream gradient dL/d(out).
+ *   fwd_out     DEVICE float[B*H*W], the Beer-Lambert image this gradient
+ *               belongs to (required in DRR_MODE_BEER_LAMBERT, where each
+ *               ray's gradient is scaled by exp(-I) = 1 - out; ignored and
+ *               may be NULL in DRR_MODE_RAW).
+ *   grad_vol    DEVICE float32 [nz][ny][nx] (linear layout), ACCUMULATED
+ *               into with atomic adds (zero it first for a plain gradient).
+ *               The order of the atomic adds is not deterministic, so results
+ *               may differ between runs in the last bits.
+ * Other arguments as drr_render.  grad_vol must not overlap the images.
+ */
+DRR_API drr_status drr_render_adjoint(const int dims[3], const float spacing[3],
+                                      const float origin[3], const float K[9], const float *Rt,
+                                      int B, int H, int W, int n_samples, float density_factor,
+                                      drr_mode mode, const float *grad_out, const float *fwd_out,
+                                      float *grad_vol, void *stream);
+
+/* Bytes that drr_prepare_volume writes for this volume, dtype and layout
+ * (0 if the arguments are invalid or the volume is too large). */
+DRR_API size_t drr_prepared_bytes(const int dims[3], drr_dtype dtype, drr_layout layout);
+
+/* Re-lay-out (and optionally convert) a volume for drr_render.
+ *   src         DEVICE float32 [nz][ny][nx].
+ *   dst         DEVICE, at least drr_prepared_bytes(dims, dtype, layout)
+ *               bytes (dst_bytes says how many are available); must not
+ *               overlap src.  Every byte of the prepared volume is written.
+ * bf16 conversion rounds to nearest even.  Done once per volume (or once per
+ * update of the volume), not per render. */
+DRR_API drr_status drr_prepare_volume(const float *src, const int dims[3], drr_dtype dtype,
+                                      drr_layout layout, void *dst, size_t dst_bytes,
+                                      void *stream);
+
+/* Human-readable description of the last failure on this thread ("" if
+ * none).  The string stays valid until the next call on this thread. */
+DRR_API const char *drr_get_last_error(void);
+
+/* ABI version of this header: 1. */
+DRR_API int drr_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DRR_H */

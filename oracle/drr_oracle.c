@@ -271,54 +271,115 @@ int oracle_trilinear(const float *vol, const int dims[3], const double *p, int64
     return 0;
 }
 
-/* Adjoint: grad_vol[k][j][i] += sum over rays and samples of g * w_corner.
- * vol is read only in Beer-Lambert mode (for exp(-I)); it may be NULL in RAW.
- * Single-threaded: a plain, fixed-order accumulation. */
+/* Adjoint of one view: grad[k][j][i] += sum over its rays and samples of
+ * g * w_corner, accumulated in order. */
+static void adjoint_view(const float *vol, const grid_t *g, const double K[9],
+                         const double Rt[12], int H, int W, int n_samples,
+                         double density_factor, int mode, const double *grad_out,
+                         double *grad) {
+    for (int r = 0; r < H; ++r)
+        for (int c = 0; c < W; ++c) {
+            double go = grad_out[(int64_t)r * W + c];
+            double C[3], d[3], t0, t1;
+            if (go == 0.0) continue;   /* contributes exactly nothing */
+            if (!ray_in_volume(g, K, Rt, c, r, C, d, &t0, &t1)) continue;
+            double dt = (t1 - t0) / (double)n_samples;
+            double scale = go * density_factor * dt;
+            if (mode == ORACLE_BEER_LAMBERT) {
+                double dt2;
+                double I = ray_integral(vol, g, K, Rt, c, r, n_samples, density_factor, &dt2);
+                scale *= exp(-I);
+            }
+            for (int i = 0; i < n_samples; ++i) {
+                double t = t0 + ((double)i + 0.5) * dt;
+                double p[3] = {C[0] + t * d[0], C[1] + t * d[1], C[2] + t * d[2]};
+                double fl[3], f[3];
+                int64_t i0[3];
+                for (int a = 0; a < 3; ++a) {
+                    fl[a] = floor(p[a]);
+                    f[a] = p[a] - fl[a];
+                    i0[a] = (int64_t)fl[a];
+                }
+                for (int dk = 0; dk < 2; ++dk)
+                    for (int dj = 0; dj < 2; ++dj)
+                        for (int di = 0; di < 2; ++di) {
+                            int64_t ii = i0[0] + di, jj = i0[1] + dj, kk = i0[2] + dk;
+                            if (ii < 0 || jj < 0 || kk < 0 || ii >= g->n[0] || jj >= g->n[1] ||
+                                kk >= g->n[2])
+                                continue;
+                            double w = (di ? f[0] : 1.0 - f[0]) * (dj ? f[1] : 1.0 - f[1]) *
+                                       (dk ? f[2] : 1.0 - f[2]);
+                            grad[(kk * g->n[1] + jj) * g->n[0] + ii] += scale * w;
+                        }
+            }
+        }
+}
+
+typedef struct {
+    const float *vol;
+    const grid_t *g;
+    const double *K, *Rt;
+    int B, H, W, n_samples, mode, stride, first;
+    double density_factor;
+    const double *grad_out;
+    double *grad;
+} adj_job_t;
+
+static void *adj_worker(void *arg) {
+    adj_job_t *j = (adj_job_t *)arg;
+    for (int b = j->first; b < j->B; b += j->stride)
+        adjoint_view(j->vol, j->g, j->K, j->Rt + 12 * b, j->H, j->W, j->n_samples,
+                     j->density_factor, j->mode, j->grad_out + (int64_t)b * j->H * j->W, j->grad);
+    return NULL;
+}
+
+/* Adjoint: grad_vol[k][j][i] += A^T grad_out (times exp(-I) per ray in
+ * Beer-Lambert mode, I from the oracle's own forward).  vol is read only in
+ * Beer-Lambert mode and may be NULL in RAW.  With nthreads > 1, thread t
+ * takes views t, t + nthreads, ... into a private fp64 buffer, and the
+ * buffers are added to grad_vol in thread order, so the result depends only
+ * on (inputs, nthreads). */
 int oracle_adjoint(const float *vol, const int dims[3], const double spacing[3],
                    const double origin[3], const double K[9], const double *Rt, int B,
                    int H, int W, int n_samples, double density_factor, int mode,
-                   const double *grad_out, double *grad_vol) {
+                   const double *grad_out, double *grad_vol, int nthreads) {
     grid_t g;
     if (make_grid(dims, spacing, origin, &g) || B < 0 || H < 0 || W < 0 || n_samples < 1)
         return -1;
     if (mode == ORACLE_BEER_LAMBERT && vol == NULL) return -1;
-    for (int b = 0; b < B; ++b)
-        for (int r = 0; r < H; ++r)
-            for (int c = 0; c < W; ++c) {
-                double go = grad_out[((int64_t)b * H + r) * W + c];
-                double C[3], d[3], t0, t1;
-                if (!ray_in_volume(&g, K, Rt + 12 * b, c, r, C, d, &t0, &t1)) continue;
-                double dt = (t1 - t0) / (double)n_samples;
-                double scale = go * density_factor * dt;
-                if (mode == ORACLE_BEER_LAMBERT) {
-                    double dt2;
-                    double I = ray_integral(vol, &g, K, Rt + 12 * b, c, r, n_samples,
-                                            density_factor, &dt2);
-                    scale *= exp(-I);
-                }
-                for (int i = 0; i < n_samples; ++i) {
-                    double t = t0 + ((double)i + 0.5) * dt;
-                    double p[3] = {C[0] + t * d[0], C[1] + t * d[1], C[2] + t * d[2]};
-                    double fl[3], f[3];
-                    int64_t i0[3];
-                    for (int a = 0; a < 3; ++a) {
-                        fl[a] = floor(p[a]);
-                        f[a] = p[a] - fl[a];
-                        i0[a] = (int64_t)fl[a];
-                    }
-                    for (int dk = 0; dk < 2; ++dk)
-                        for (int dj = 0; dj < 2; ++dj)
-                            for (int di = 0; di < 2; ++di) {
-                                int64_t ii = i0[0] + di, jj = i0[1] + dj, kk = i0[2] + dk;
-                                if (ii < 0 || jj < 0 || kk < 0 || ii >= g.n[0] ||
-                                    jj >= g.n[1] || kk >= g.n[2])
-                                    continue;
-                                double w = (di ? f[0] : 1.0 - f[0]) * (dj ? f[1] : 1.0 - f[1]) *
-                                           (dk ? f[2] : 1.0 - f[2]);
-                                grad_vol[(kk * g.n[1] + jj) * g.n[0] + ii] += scale * w;
-                            }
-                }
-            }
+    if (nthreads > B) nthreads = B;
+    if (nthreads > 64) nthreads = 64;
+    if (nthreads < 1) nthreads = 1;
+    const int64_t nvox = g.n[0] * g.n[1] * g.n[2];
+    double *bufs[64];
+    int got = 0;
+    for (; got < nthreads && nthreads > 1; ++got) {
+        bufs[got] = (double *)calloc((size_t)nvox, sizeof(double));
+        if (!bufs[got]) break;
+    }
+    if (got < nthreads || nthreads == 1) {     /* one thread, straight into grad_vol */
+        for (int t = 0; t < got; ++t) free(bufs[t]);
+        adj_job_t j = {vol, &g, K, Rt, B, H, W, n_samples, mode, 1, 0, density_factor,
+                       grad_out, grad_vol};
+        adj_worker(&j);
+        return 0;
+    }
+    pthread_t tid[64];
+    int running[64];
+    adj_job_t jobs[64];
+    for (int t = 0; t < nthreads; ++t) {
+        adj_job_t j = {vol, &g, K, Rt, B, H, W, n_samples, mode, nthreads, t, density_factor,
+                       grad_out, bufs[t]};
+        jobs[t] = j;
+        running[t] = pthread_create(&tid[t], NULL, adj_worker, &jobs[t]) == 0;
+        if (!running[t]) adj_worker(&jobs[t]);
+    }
+    for (int t = 0; t < nthreads; ++t)
+        if (running[t]) pthread_join(tid[t], NULL);
+    for (int t = 0; t < nthreads; ++t) {
+        for (int64_t m = 0; m < nvox; ++m) grad_vol[m] += bufs[t][m];
+        free(bufs[t]);
+    }
     return 0;
 }
 

@@ -40,7 +40,7 @@ def load():
     lib.oracle_trilinear.restype = _c.c_int
     lib.oracle_adjoint.argtypes = [_c.c_void_p, _i32p, _f64p, _f64p, _f64p, _f64p, _c.c_int,
                                    _c.c_int, _c.c_int, _c.c_int, _c.c_double, _c.c_int, _f64p,
-                                   _f64p]
+                                   _f64p, _c.c_int]
     lib.oracle_adjoint.restype = _c.c_int
     lib.oracle_round_bf16.argtypes = [_f32p, _u16p, _c.c_int64]
     lib.oracle_round_bf16.restype = None
@@ -114,7 +114,7 @@ def trilinear(vol, dims, points):
 
 
 def adjoint(dims, spacing, origin, K, Rt, H, W, n_samples, density_factor, mode, grad_out,
-            vol=None):
+            vol=None, nthreads=1):
     """grad_vol[k][j][i] (float64) = A^T grad_out (times exp(-I) in Beer-Lambert)."""
     dims, spacing, origin, K, Rt = _geom(dims, spacing, origin, K, Rt)
     B = Rt.shape[0]
@@ -127,7 +127,7 @@ def adjoint(dims, spacing, origin, K, Rt, H, W, n_samples, density_factor, mode,
         keep = _vol(vol, dims)
         vptr = keep.ctypes.data
     rc = load().oracle_adjoint(vptr, dims, spacing, origin, K, Rt.reshape(-1), B, H, W,
-                               n_samples, density_factor, mode, go, grad)
+                               n_samples, density_factor, mode, go, grad, int(nthreads))
     assert rc == 0, "oracle_adjoint rejected its arguments"
     nx, ny, nz = (int(x) for x in dims)
     return grad.reshape(nz, ny, nx)

@@ -1,0 +1,87 @@
+"""Helpers of the GPU parity tests: run the CUDA path through the C ABI
+(cone_beam_ct_b200.drr) on a Workload, and compare against the oracle with
+the tolerances the tests state."""
+import numpy as np
+
+from cone_beam_ct_b200 import drr
+
+LINEAR, PADDED = drr.DRR_LAYOUT_LINEAR, drr.DRR_LAYOUT_PADDED
+F32, BF16 = drr.DRR_F32, drr.DRR_BF16
+
+
+def device_inputs(w, vol=None):
+    import torch
+    v = torch.from_numpy(np.ascontiguousarray(w.vol if vol is None else vol)).cuda()
+    Rt = torch.from_numpy(np.ascontiguousarray(w.Rt.reshape(-1, 12))).cuda()
+    return v, Rt
+
+
+def prepared(vol32, dims, dtype, layout):
+    """The volume in the layout/dtype drr_render reads (prepared on the GPU)."""
+    import torch
+    if dtype == F32 and layout == LINEAR:
+        return vol32
+    nbytes = drr.drr_prepared_bytes(dims, dtype, layout)
+    buf = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    drr.drr_prepare_volume(vol32, dims, dtype, layout, buf)
+    return buf
+
+
+def gpu_forward(w, layout=PADDED, dtype=None, mode=None, vol=None, Rt=None):
+    import torch
+    dtype = w.dtype if dtype is None else dtype
+    mode = w.mode if mode is None else mode
+    v32, Rt_d = device_inputs(w, vol)
+    if Rt is not None:
+        Rt_d = torch.from_numpy(np.ascontiguousarray(Rt.reshape(-1, 12), dtype=np.float32)).cuda()
+    B = Rt_d.shape[0]
+    src = prepared(v32, w.dims, dtype, layout)
+    out = torch.full((B, w.H, w.W), float("nan"), dtype=torch.float32, device="cuda")
+    drr.drr_render(src, dtype, layout, w.dims, w.spacing, w.origin, w.K, Rt_d, B, w.H, w.W,
+                   w.n_samples, w.density_factor, mode, out)
+    torch.cuda.synchronize()
+    return out.cpu().numpy()
+
+
+def gpu_adjoint(w, grad_out, mode=None, fwd_out=None):
+    import torch
+    mode = w.mode if mode is None else mode
+    _, Rt_d = device_inputs(w, vol=np.zeros((1,), np.float32))
+    go = torch.from_numpy(np.ascontiguousarray(grad_out, dtype=np.float32)).cuda()
+    fo = None
+    if fwd_out is not None:
+        fo = torch.from_numpy(np.ascontiguousarray(fwd_out, dtype=np.float32)).cuda()
+    nx, ny, nz = w.dims
+    grad = torch.zeros((nz, ny, nx), dtype=torch.float32, device="cuda")
+    drr.drr_render_adjoint(w.dims, w.spacing, w.origin, w.K, Rt_d, w.B, w.H, w.W, w.n_samples,
+                           w.density_factor, mode, go, fo, grad)
+    torch.cuda.synchronize()
+    return grad.cpu().numpy()
+
+
+def bf16_values(vol):
+    """The volume as bf16-rounded fp32 values (oracle-side rounding)."""
+    import oracle
+    return oracle.bf16_to_float(oracle.round_bf16(vol))
+
+
+def parity_errors(got, ref, floor=1e-2):
+    """(normwise max error / max|ref|, worst per-element relative error over
+    elements with |ref| >= floor * max|ref|)."""
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert got.shape == ref.shape
+    assert np.all(np.isfinite(got)), "non-finite values in the GPU result"
+    scale = float(np.max(np.abs(ref)))
+    if scale == 0.0:
+        return float(np.max(np.abs(got))), 0.0
+    diff = np.abs(got - ref)
+    big = np.abs(ref) >= floor * scale
+    rel = float(np.max(diff[big] / np.abs(ref[big]))) if np.any(big) else 0.0
+    return float(np.max(diff)) / scale, rel
+
+
+def assert_parity(got, ref, tol, floor=1e-2, what=""):
+    norm, rel = parity_errors(got, ref, floor)
+    assert norm <= tol and rel <= tol, f"{what}: normwise {norm:.3g}, per-element {rel:.3g} > {tol}"
+    return norm, rel

@@ -1,0 +1,189 @@
+"""The C ABI on the host (CPU only): libdrr.so loads, exports every entry
+point include/drr.h declares, and rejects bad arguments before launching.
+
+Every call here fails host-side validation (or is an empty batch), so no
+kernel is ever launched and the fake device addresses are never touched.
+"""
+import os
+import re
+import subprocess
+
+import numpy as np
+import pytest
+
+from cone_beam_ct_b200 import drr
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "drr.h")
+PROBE_HEADER = os.path.join(ROOT, "include", "drr_probe.h")
+PROBE_LIB = os.path.join(ROOT, "cone_beam_ct_b200", "libdrr_probe.so")
+FAKE = 0x7F0000000000          # a plausible device address; never dereferenced here
+K_OK = [500.0, 0.0, 99.5, 0.0, 500.0, 99.5, 0.0, 0.0, 1.0]
+DIMS, SP, ORG = (16, 16, 16), (1.0, 1.0, 1.0), (0.0, 0.0, 0.0)
+
+
+def declared_names(header=HEADER, macro="DRR_API"):
+    text = open(header).read()
+    return sorted(set(re.findall(macro + r"\s+[\w\s\*]+?\b(drr_\w+)\s*\(", text)))
+
+
+def exported_names(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", lib], capture_output=True,
+                         text=True, check=True).stdout
+    return set(re.findall(r"\bT\s+(drr_\w+)", out))
+
+
+def test_header_declares_the_entry_points():
+    assert declared_names() == sorted(drr.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol():
+    drr.lib()
+    exported = exported_names(drr.LIB_PATH)
+    # every declared entry point, and nothing but the ABI, leaves the library
+    assert exported == set(declared_names())
+    assert drr.drr_abi_version() == 1
+
+
+def test_probe_library_exports_its_declared_symbol():
+    import ctypes
+    ctypes.CDLL(PROBE_LIB)
+    names = declared_names(PROBE_HEADER, "DRR_PROBE_API")
+    assert names == ["drr_probe_l2_read"]
+    assert exported_names(PROBE_LIB) == set(names)
+
+
+def test_every_header_is_covered():
+    headers = sorted(f for f in os.listdir(os.path.join(ROOT, "include")) if f.endswith(".h"))
+    assert headers == ["drr.h", "drr_probe.h"]
+
+
+def _render(**kw):
+    args = dict(vol=FAKE, dtype=drr.DRR_F32, layout=drr.DRR_LAYOUT_LINEAR, dims=DIMS, spacing=SP,
+                origin=ORG, K=K_OK, Rt=FAKE, B=2, H=8, W=8, n_samples=16, density_factor=1.0,
+                mode=drr.DRR_MODE_RAW, out=FAKE + (1 << 24), stream=0)
+    args.update(kw)
+    return drr.drr_render(**args)
+
+
+def _adjoint(**kw):
+    args = dict(dims=DIMS, spacing=SP, origin=ORG, K=K_OK, Rt=FAKE, B=2, H=8, W=8,
+                n_samples=16, density_factor=1.0, mode=drr.DRR_MODE_RAW,
+                grad_out=FAKE + (1 << 20), fwd_out=FAKE + (1 << 21), grad_vol=FAKE + (1 << 24),
+                stream=0)
+    args.update(kw)
+    return drr.drr_render_adjoint(**args)
+
+
+RENDER_BAD = [
+    (dict(dims=(1, 16, 16)), drr.DRR_ERR_INVALID_ARG, "dims"),
+    (dict(dims=(16, 16, 1 << 23)), drr.DRR_ERR_INVALID_ARG, "dims"),
+    (dict(dims=(2048, 2048, 1024)), drr.DRR_ERR_UNSUPPORTED, "too large"),
+    (dict(spacing=(1.0, 0.0, 1.0)), drr.DRR_ERR_INVALID_ARG, "spacing"),
+    (dict(spacing=(1.0, float("nan"), 1.0)), drr.DRR_ERR_INVALID_ARG, "spacing"),
+    (dict(origin=(0.0, float("inf"), 0.0)), drr.DRR_ERR_INVALID_ARG, "origin"),
+    (dict(K=[500.0, 0, 99.5, 1.0, 500.0, 99.5, 0, 0, 1]), drr.DRR_ERR_INVALID_ARG, "triangular"),
+    (dict(K=[0.0, 0, 99.5, 0, 500.0, 99.5, 0, 0, 1]), drr.DRR_ERR_INVALID_ARG, "invertible"),
+    (dict(K=[500.0, 0, float("nan"), 0, 500.0, 99.5, 0, 0, 1]), drr.DRR_ERR_INVALID_ARG, "finite"),
+    (dict(B=-1), drr.DRR_ERR_INVALID_ARG, ">= 0"),
+    (dict(B=70000), drr.DRR_ERR_UNSUPPORTED, "views"),
+    (dict(H=65535 * 16 + 1), drr.DRR_ERR_UNSUPPORTED, "rows"),
+    (dict(n_samples=0), drr.DRR_ERR_INVALID_ARG, "n_samples"),
+    (dict(n_samples=(1 << 20) + 1), drr.DRR_ERR_INVALID_ARG, "n_samples"),
+    (dict(density_factor=float("inf")), drr.DRR_ERR_INVALID_ARG, "density_factor"),
+    (dict(mode=2), drr.DRR_ERR_INVALID_ARG, "mode"),
+    (dict(dtype=7), drr.DRR_ERR_INVALID_ARG, "dtype"),
+    (dict(layout=5), drr.DRR_ERR_INVALID_ARG, "layout"),
+    (dict(vol=0), drr.DRR_ERR_INVALID_ARG, "vol"),
+    (dict(vol=FAKE + 2), drr.DRR_ERR_INVALID_ARG, "vol"),       # fp32 volume, 2-byte aligned
+    (dict(Rt=0), drr.DRR_ERR_INVALID_ARG, "Rt"),
+    (dict(Rt=FAKE + 1), drr.DRR_ERR_INVALID_ARG, "Rt"),
+    (dict(out=0), drr.DRR_ERR_INVALID_ARG, "out"),
+    (dict(out=FAKE + 6), drr.DRR_ERR_INVALID_ARG, "out"),
+]
+
+
+@pytest.mark.parametrize("kw,status,word", RENDER_BAD)
+def test_render_rejects_bad_arguments(kw, status, word):
+    with pytest.raises(drr.DrrError) as e:
+        _render(**kw)
+    assert e.value.status == status
+    assert word in drr.drr_get_last_error()
+
+
+ADJOINT_BAD = [
+    (dict(dims=(16, 0, 16)), drr.DRR_ERR_INVALID_ARG),
+    (dict(n_samples=-3), drr.DRR_ERR_INVALID_ARG),
+    (dict(grad_out=0), drr.DRR_ERR_INVALID_ARG),
+    (dict(grad_vol=0), drr.DRR_ERR_INVALID_ARG),
+    (dict(mode=drr.DRR_MODE_BEER_LAMBERT, fwd_out=0), drr.DRR_ERR_INVALID_ARG),
+    (dict(grad_vol=FAKE + (1 << 20)), drr.DRR_ERR_INVALID_ARG),    # overlaps grad_out
+    (dict(K=[500.0, 0, 99.5, 0, 500.0, 99.5, 0.5, 0, 1]), drr.DRR_ERR_INVALID_ARG),
+    (dict(mode=-1), drr.DRR_ERR_INVALID_ARG),
+]
+
+
+@pytest.mark.parametrize("kw,status", ADJOINT_BAD)
+def test_adjoint_rejects_bad_arguments(kw, status):
+    with pytest.raises(drr.DrrError) as e:
+        _adjoint(**kw)
+    assert e.value.status == status
+
+
+def test_raw_adjoint_does_not_need_the_forward_image():
+    # fwd_out may be NULL in RAW mode: only an empty batch keeps this off the device
+    _adjoint(fwd_out=None, B=0)
+
+
+@pytest.mark.parametrize("which", ["B", "H", "W"])
+def test_empty_batch_or_image_is_a_no_op(which):
+    # nothing to launch: succeeds even with NULL buffers
+    _render(**{which: 0, "vol": None, "out": None, "Rt": None})
+    _adjoint(**{which: 0, "grad_out": None, "grad_vol": None, "Rt": None, "fwd_out": None})
+    assert drr.drr_get_last_error() == ""
+
+
+def test_prepared_bytes():
+    assert drr.drr_prepared_bytes((256, 256, 256), drr.DRR_F32, drr.DRR_LAYOUT_LINEAR) == 4 * 256 ** 3
+    assert drr.drr_prepared_bytes((256, 256, 256), drr.DRR_BF16, drr.DRR_LAYOUT_LINEAR) == 2 * 256 ** 3
+    assert drr.drr_prepared_bytes((5, 6, 7), drr.DRR_F32, drr.DRR_LAYOUT_PADDED) == 4 * 7 * 8 * 9
+    assert drr.drr_prepared_bytes((5, 6, 7), drr.DRR_BF16, drr.DRR_LAYOUT_PADDED) == 2 * 7 * 8 * 9
+    assert drr.drr_prepared_bytes((1, 6, 7), drr.DRR_F32, drr.DRR_LAYOUT_PADDED) == 0
+    assert drr.drr_prepared_bytes((5, 6, 7), 3, drr.DRR_LAYOUT_PADDED) == 0
+    assert drr.drr_prepared_bytes((2048, 2048, 1024), drr.DRR_F32, drr.DRR_LAYOUT_LINEAR) == 0
+
+
+PREPARE_BAD = [
+    (dict(dims=(16, 16, 1)), drr.DRR_ERR_INVALID_ARG),
+    (dict(dtype=4), drr.DRR_ERR_INVALID_ARG),
+    (dict(layout=9), drr.DRR_ERR_INVALID_ARG),
+    (dict(src=0), drr.DRR_ERR_INVALID_ARG),
+    (dict(dst=0), drr.DRR_ERR_INVALID_ARG),
+    (dict(dst_bytes=100), drr.DRR_ERR_INVALID_ARG),
+    (dict(dst=FAKE + 64), drr.DRR_ERR_INVALID_ARG),      # overlaps src
+    (dict(src=FAKE + 2), drr.DRR_ERR_INVALID_ARG),       # misaligned
+    (dict(dims=(2048, 2048, 1024)), drr.DRR_ERR_UNSUPPORTED),
+]
+
+
+@pytest.mark.parametrize("kw,status", PREPARE_BAD)
+def test_prepare_rejects_bad_arguments(kw, status):
+    args = dict(src=FAKE, dims=DIMS, dtype=drr.DRR_BF16, layout=drr.DRR_LAYOUT_PADDED,
+                dst=FAKE + (1 << 24), dst_bytes=1 << 24, stream=0)
+    args.update(kw)
+    with pytest.raises(drr.DrrError) as e:
+        drr.drr_prepare_volume(**args)
+    assert e.value.status == status
+
+
+def test_binding_refuses_host_tensors_for_device_arguments():
+    torch = pytest.importorskip("torch")
+    with pytest.raises(TypeError):
+        _render(out=torch.zeros(2, 8, 8))
+
+
+def test_binding_fails_loudly_without_the_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(drr, "_lib", None)
+    monkeypatch.setattr(drr, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError, match="no CPU fallback"):
+        drr.lib()

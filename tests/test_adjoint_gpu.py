@@ -1,0 +1,118 @@
+"""GPU adjoint parity: the volume-gradient scatter against the fp64 oracle
+adjoint, and the dot-product identity <A x, y> = <x, A^T y> (TorchTomo page,
+"Discrete Adjoint and Learned Primal-Dual") between the GPU forward and the
+GPU adjoint.
+
+Tolerances.  No page fixes one for the adjoint; the bar of the forward
+(1e-4) is kept, read for a scatter whose voxels sum many random-sign terms
+(so per-voxel relative error is meaningless where they cancel): normwise
+max |gpu - oracle| / max |oracle| <= 1e-4 and relative L2 error <= 1e-4.
+Dot-product residual |<Ax, y> - <x, A^T y>| / (||Ax|| ||y||) <= 1e-5 (fp32
+sums of up to ~10^9 terms; the oracle itself meets 1e-12, see the pins).
+"""
+import numpy as np
+import pytest
+
+import oracle
+from cone_beam_ct_b200 import workloads as wl
+from tests.gpu_helpers import F32, LINEAR, PADDED, gpu_adjoint, gpu_forward
+
+pytestmark = pytest.mark.gpu
+TOL_ADJ, TOL_DOT = 1e-4, 1e-5
+
+
+@pytest.fixture(scope="module")
+def cuda():
+    torch = pytest.importorskip("torch")
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    return torch
+
+
+def assert_adjoint_parity(got, ref, what=""):
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    scale = np.max(np.abs(ref))
+    assert scale > 0
+    norm = np.max(np.abs(got - ref)) / scale
+    l2 = np.linalg.norm(got - ref) / np.linalg.norm(ref)
+    assert norm <= TOL_ADJ and l2 <= TOL_ADJ, f"{what}: normwise {norm:.3g}, L2 {l2:.3g}"
+
+
+def _oracle_adjoint(w, go, mode, nthreads=8):
+    return oracle.adjoint(w.dims, w.spacing, w.origin, w.K, w.Rt, w.H, w.W, w.n_samples,
+                          w.density_factor, mode, go, vol=w.vol, nthreads=nthreads)
+
+
+@pytest.mark.parametrize("seed", [201, 202, 203])
+@pytest.mark.parametrize("mode", [wl.MODE_RAW, wl.MODE_BEER_LAMBERT])
+def test_small_ragged_adjoint(cuda, seed, mode):
+    w = wl.small_random_case(seed)
+    go = np.random.default_rng(seed).standard_normal((w.B, w.H, w.W)).astype(np.float32)
+    fwd = gpu_forward(w, layout=PADDED, dtype=F32, mode=mode) if mode else None
+    got = gpu_adjoint(w, go, mode=mode, fwd_out=fwd)
+    assert_adjoint_parity(got, _oracle_adjoint(w, go, mode), what=f"seed {seed} mode {mode}")
+
+
+def _dot_residual(w, x, y, layout):
+    Ax = gpu_forward(w, layout=layout, dtype=F32, mode=wl.MODE_RAW, vol=x).astype(np.float64)
+    ATy = gpu_adjoint(w, y, mode=wl.MODE_RAW).astype(np.float64)
+    lhs = float(np.dot(Ax.reshape(-1), y.reshape(-1).astype(np.float64)))
+    rhs = float(np.dot(x.reshape(-1).astype(np.float64), ATy.reshape(-1)))
+    return abs(lhs - rhs) / (np.linalg.norm(Ax) * np.linalg.norm(y.astype(np.float64)))
+
+
+@pytest.mark.parametrize("layout", [LINEAR, PADDED])
+def test_dot_product_identity_small(cuda, layout):
+    w = wl.small_random_case(204)
+    rng = np.random.default_rng(5)
+    nx, ny, nz = w.dims
+    x = rng.uniform(0, 1, (nz, ny, nx)).astype(np.float32)
+    y = rng.standard_normal((w.B, w.H, w.W)).astype(np.float32)
+    assert _dot_residual(w, x, y, layout) <= TOL_DOT
+
+
+def test_adjoint_accumulates_and_skips_zero_gradient(cuda):
+    import torch
+    from cone_beam_ct_b200 import drr
+    w = wl.small_random_case(205)
+    go = np.random.default_rng(1).standard_normal((w.B, w.H, w.W)).astype(np.float32)
+    once = gpu_adjoint(w, go, mode=wl.MODE_RAW)
+    Rt = torch.from_numpy(w.Rt.reshape(-1, 12).copy()).cuda()
+    g = torch.from_numpy(once).cuda()
+    drr.drr_render_adjoint(w.dims, w.spacing, w.origin, w.K, Rt, w.B, w.H, w.W, w.n_samples,
+                           w.density_factor, wl.MODE_RAW, torch.from_numpy(go).cuda(), None, g)
+    torch.cuda.synchronize()
+    assert np.allclose(g.cpu().numpy(), 2 * once, rtol=1e-5, atol=1e-6 * np.abs(once).max())
+    zero = gpu_adjoint(w, np.zeros_like(go), mode=wl.MODE_RAW)
+    assert np.all(zero == 0.0)
+
+
+@pytest.mark.slow
+def test_config5_full_adjoint_and_dot_product(cuda):
+    w = wl.make_config(5)
+    got = gpu_adjoint(w, w.grad_out, mode=w.mode)
+    ref = _oracle_adjoint(w, w.grad_out, w.mode, nthreads=16)
+    assert_adjoint_parity(got, ref, what="config 5")
+    rng = np.random.default_rng(55)
+    nx, ny, nz = w.dims
+    x = rng.uniform(0, 1, (nz, ny, nx)).astype(np.float32)
+    y = rng.standard_normal((w.B, w.H, w.W)).astype(np.float32)
+    assert _dot_residual(w, x, y, PADDED) <= TOL_DOT
+
+
+@pytest.mark.slow
+def test_config3_geometry_adjoint(cuda):
+    # the 1024^2 x 512 C-arm geometry with an fp32 gradient volume: the dot-product
+    # identity at full size, and the oracle on a sparse upstream gradient (2000 rays)
+    w = wl.make_config(3)
+    rng = np.random.default_rng(33)
+    nx, ny, nz = w.dims
+    x = rng.uniform(0, 1, (nz, ny, nx)).astype(np.float32)
+    y = rng.standard_normal((w.B, w.H, w.W)).astype(np.float32)
+    assert _dot_residual(w, x, y, PADDED) <= TOL_DOT
+    sparse = np.zeros((w.B, w.H, w.W), np.float32)
+    ids = rng.choice(w.rays, size=2000, replace=False)
+    sparse.reshape(-1)[ids] = rng.standard_normal(2000).astype(np.float32)
+    got = gpu_adjoint(w, sparse, mode=wl.MODE_RAW)
+    ref = _oracle_adjoint(w, sparse, wl.MODE_RAW)
+    assert_adjoint_parity(got, ref, what="config 3 sparse")

@@ -34,8 +34,8 @@ MUTANTS = {
     "adjoint without dt": (
         "double scale = go * density_factor * dt;", "double scale = go * density_factor;"),
     "adjoint i/j transposed": (
-        "grad_vol[(kk * g.n[1] + jj) * g.n[0] + ii] += scale * w;",
-        "grad_vol[(kk * g.n[1] + ii) * g.n[0] + jj] += scale * w;"),
+        "grad[(kk * g->n[1] + jj) * g->n[0] + ii] += scale * w;",
+        "grad[(kk * g->n[1] + ii) * g->n[0] + jj] += scale * w;"),
     "no clamp of t0 at the camera": ("*t0 = t_near > 0.0 ? t_near : 0.0;", "*t0 = t_near;"),
     "half-pixel shift": (
         "double u = (double)(rc % job->W), v = (double)(rc / job->W);",
