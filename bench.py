@@ -41,7 +41,7 @@ FLUSH_BYTES = 256 << 20
 def parse_args():
     p = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--steps", type=int, default=100)
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--config", type=int, default=2, choices=[1, 2, 3, 4],
@@ -102,7 +102,7 @@ def physical_gpu(ordinal):
 
 
 class ClockSampler:
-    """nvidia-smi sampled every 200 ms during the timed region."""
+    """nvidia-smi sampled every 100 ms during the timed region."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -116,7 +116,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
@@ -203,11 +203,15 @@ def traffic_for(kernel, workload_name):
     entry = table.get(kernel, {}).get(workload_name)
     if not entry:
         return None
-    src = os.path.join(ROOT, entry["source"])
-    if not os.path.exists(src):
+    digest = hashlib.sha256()
+    for src in entry["sources"]:
+        full = os.path.join(ROOT, src)
+        if not os.path.exists(full):
+            return None
+        digest.update(open(full, "rb").read())
+    if digest.hexdigest()[:16] != entry["sources_sha256_16"]:
         return None
-    digest = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-    return entry["dram_bytes_per_launch"] if digest == entry["source_sha256_16"] else None
+    return entry["dram_bytes_per_launch"]
 
 
 # ---------------------------------------------------------------------------
@@ -263,7 +267,7 @@ def cpu_baseline(w):
     import oracle
     oracle.build()
     cores = len(os.sched_getaffinity(0))
-    views = min(w.B, 16)
+    views = min(w.B, 64)
     Rt = w.Rt[:views]
     t0 = time.perf_counter()
     oracle.render(w.vol, w.dims, w.spacing, w.origin, w.K, Rt, w.H, w.W, w.n_samples,

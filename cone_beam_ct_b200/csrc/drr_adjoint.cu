@@ -6,9 +6,9 @@
 // read, with g = grad_out * density_factor * dt per ray, times exp(-I) =
 // 1 - out in Beer-Lambert mode (the derivative of 1 - exp(-I)).  This is the
 // backward kernel of the fused renderer (FlashDRR page, "Train vs. Eval
-// Dynamics").  Same launch shape and ray setup as the forward; the sample
-// positions and weights use the forward's linear-layout (clamped) arithmetic,
-// so the adjoint is the transpose of that forward up to fp32 rounding.
+// Dynamics").  Same launch shape, ray setup and 32.32 sample positions as the
+// forward on the linear layout, so its weights are the forward's weights and
+// the adjoint is that forward's transpose up to fp32 rounding.
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -32,24 +32,18 @@ adjoint_kernel(const float* __restrict__ Rt, const float* __restrict__ grad_out,
     float go = grad_out[pix];
     if (MODE == 1) go *= 1.0f - fwd_out[pix];
     Ray ray;
-    if (go == 0.0f || !ray_setup(sv, g, (float)c, (float)r, ray)) return;
+    if (go == 0.0f || !ray_setup(sv, g, (double)c, (double)r, 0.0, ray)) return;
     const float scale = go * (g.density_factor * ray.dt);
-    float p0[3];
-#pragma unroll
-    for (int k = 0; k < 3; ++k) p0[k] = fmaf(0.5f, ray.S[k], ray.P[k]);
     const int row = g.row, slice = g.slice;
-    const float hx = g.hi_clamp[0], hy = g.hi_clamp[1], hz = g.hi_clamp[2];
-    float fi = 0.0f;
+    long long qx = ray.q0[0], qy = ray.q0[1], qz = ray.q0[2];
+    const long long sx = ray.s[0], sy = ray.s[1], sz = ray.s[2];
 #pragma unroll 2
-    for (int i = 0; i < g.N; ++i, fi += 1.0f) {
-        const float qx = fminf(fmaxf(fmaf(fi, ray.S[0], p0[0]), 0.0f), hx);
-        const float qy = fminf(fmaxf(fmaf(fi, ray.S[1], p0[1]), 0.0f), hy);
-        const float qz = fminf(fmaxf(fmaf(fi, ray.S[2], p0[2]), 0.0f), hz);
-        int ix, iy, iz;
-        const float fx = qx - floor_small(qx, ix);
-        const float fy = qy - floor_small(qy, iy);
-        const float fz = qz - floor_small(qz, iz);
-        float* base = grad + (iz * slice + iy * row + ix);
+    for (int i = 0; i < g.N; ++i) {
+        const float fx = fix_frac(qx), fy = fix_frac(qy), fz = fix_frac(qz);
+        float* base = grad + (fix_cell(qz) * slice + fix_cell(qy) * row + fix_cell(qx));
+        qx += sx;
+        qy += sy;
+        qz += sz;
         const float wz1 = scale * fz, wz0 = scale * (1.0f - fz);
         const float w01 = wz0 * fy, w00 = wz0 * (1.0f - fy);
         const float w11 = wz1 * fy, w10 = wz1 * (1.0f - fy);

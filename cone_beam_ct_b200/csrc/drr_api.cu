@@ -97,18 +97,21 @@ void fill_geom(drr::Geom& g, const int dims[3], const float spacing[3], const fl
     g.slice = (dims[0] + pad) * (dims[1] + pad);
     for (int a = 0; a < 3; ++a) {
         g.hi[a] = (float)(dims[a] - 1);
-        g.hi_clamp[a] = std::nextafter(g.hi[a], 0.0f);
-        g.inv_sp[a] = (float)(1.0 / (double)spacing[a]);
+        // largest 32.32 sample coordinate whose 8 corners are stored: cell <= n-2
+        // for the linear layout, cell <= n (inside the zero border) for the padded one
+        const long long cells = layout == DRR_LAYOUT_PADDED ? dims[a] + 1 : dims[a] - 1;
+        g.lim[a] = cells * (1LL << 32) - 1;
+        g.spacing[a] = spacing[a];
         g.origin[a] = origin[a];
     }
-    // inverse of the upper-triangular K in double
+    // inverse of the upper-triangular K, in double
     const double k0 = K[0], k1 = K[1], k2 = K[2], k4 = K[4], k5 = K[5], k8 = K[8];
-    g.kinv[0] = (float)(1.0 / k0);
-    g.kinv[1] = (float)(-k1 / (k0 * k4));
-    g.kinv[2] = (float)((k1 * k5 - k2 * k4) / (k0 * k4 * k8));
-    g.kinv[3] = (float)(1.0 / k4);
-    g.kinv[4] = (float)(-k5 / (k4 * k8));
-    g.kinv[5] = (float)(1.0 / k8);
+    g.kinv[0] = 1.0 / k0;
+    g.kinv[1] = -k1 / (k0 * k4);
+    g.kinv[2] = (k1 * k5 - k2 * k4) / (k0 * k4 * k8);
+    g.kinv[3] = 1.0 / k4;
+    g.kinv[4] = -k5 / (k4 * k8);
+    g.kinv[5] = 1.0 / k8;
     g.B = B;
     g.H = H;
     g.W = W;

@@ -9,17 +9,12 @@
 // materialised in memory: the fused design the FlashDRR page credits for its
 // near-constant footprint ("Memory Scaling").
 //
-// Two storage layouts:
-//  * PADDED: the volume sits inside a one-voxel zero border, so the border
-//    *is* the zero padding and the loop needs no clamps.  Memory safety comes
-//    from a per-ray check: samples are fma(i, S, Q0) and fma rounding is
-//    monotone in i, so if the first and the last sample lie inside the padded
-//    box, every sample does.
-//  * LINEAR: the caller's plain array; each sample is clamped into
-//    [0, n-1) per axis before the floor.  Inside the voxel-centre box that is
-//    the same interpolant (the upper corner at n-1 gets weight 0 either way);
-//    outside it, which only rounding at the box faces can reach, the result
-//    differs from zero padding by O(ulp).
+// Two storage layouts, one loop: the caller's linear array, or the array
+// inside a one-voxel zero border (drr_prepare_volume).  Sample positions are
+// 32.32 fixed point (drr_internal.cuh), clipped per ray so that every corner
+// read stays inside the stored volume; inside the voxel-centre box the linear
+// layout's upper corner at n-1 is reached with weight 1 - 2^-32 instead of
+// through the border, an O(2^-32) difference.
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -62,62 +57,23 @@ __device__ __forceinline__ float trilinear_at(const T* __restrict__ base, int ro
     return fmaf(fz, c1 - c0, c0);
 }
 
-// Sum of the N samples of one ray in the padded layout.  Returns false if the
-// ray's samples would leave the padded box (only possible for non-finite or
-// absurd geometry); the caller then treats the ray as a miss.
+// Sum of the N samples of one ray.  Every sample lies in [0, g.lim] per axis
+// (ray_setup), so the 8 corners of every sample lie inside the stored volume:
+// for the linear layout lim < (n-1) * 2^32 (cell <= n-2), for the padded one
+// lim < (n+1) * 2^32 (cell <= n, inside the zero border).
 template <typename T>
-__device__ __forceinline__ bool march_padded(const T* __restrict__ vol, const Geom& g,
-                                             const Ray& ray, float& sum) {
-    float q0[3], ql[3];
-    const float last = (float)(g.N - 1);
-    const float lim[3] = {(float)(g.nx + 1), (float)(g.ny + 1), (float)(g.nz + 1)};
-    bool inside = true;
-#pragma unroll
-    for (int k = 0; k < 3; ++k) {
-        q0[k] = fmaf(0.5f, ray.S[k], ray.P[k] + 1.0f);      // padded coordinate of sample 0
-        ql[k] = fmaf(last, ray.S[k], q0[k]);                // ... of sample N-1
-        inside = inside && q0[k] >= 0.0f && q0[k] < lim[k] && ql[k] >= 0.0f && ql[k] < lim[k];
-    }
-    if (!inside) return false;
+__device__ __forceinline__ float march(const T* __restrict__ vol, const Geom& g, const Ray& ray) {
     const int row = g.row, slice = g.slice;
-    float acc = 0.0f, fi = 0.0f;
+    long long qx = ray.q0[0], qy = ray.q0[1], qz = ray.q0[2];
+    const long long sx = ray.s[0], sy = ray.s[1], sz = ray.s[2];
+    float acc = 0.0f;
 #pragma unroll 4
-    for (int i = 0; i < g.N; ++i, fi += 1.0f) {
-        const float qx = fmaf(fi, ray.S[0], q0[0]);
-        const float qy = fmaf(fi, ray.S[1], q0[1]);
-        const float qz = fmaf(fi, ray.S[2], q0[2]);
-        int ix, iy, iz;
-        const float fx = qx - floor_small(qx, ix);
-        const float fy = qy - floor_small(qy, iy);
-        const float fz = qz - floor_small(qz, iz);
-        const int idx = iz * slice + iy * row + ix;
-        acc += trilinear_at(vol + idx, row, slice, fx, fy, fz);
-    }
-    sum = acc;
-    return true;
-}
-
-// Sum of the N samples of one ray in the caller's linear layout (clamped).
-template <typename T>
-__device__ __forceinline__ float march_linear(const T* __restrict__ vol, const Geom& g,
-                                              const Ray& ray) {
-    float p0[3];
-#pragma unroll
-    for (int k = 0; k < 3; ++k) p0[k] = fmaf(0.5f, ray.S[k], ray.P[k]);
-    const int row = g.row, slice = g.slice;
-    const float hx = g.hi_clamp[0], hy = g.hi_clamp[1], hz = g.hi_clamp[2];
-    float acc = 0.0f, fi = 0.0f;
-#pragma unroll 4
-    for (int i = 0; i < g.N; ++i, fi += 1.0f) {
-        const float qx = fminf(fmaxf(fmaf(fi, ray.S[0], p0[0]), 0.0f), hx);
-        const float qy = fminf(fmaxf(fmaf(fi, ray.S[1], p0[1]), 0.0f), hy);
-        const float qz = fminf(fmaxf(fmaf(fi, ray.S[2], p0[2]), 0.0f), hz);
-        int ix, iy, iz;
-        const float fx = qx - floor_small(qx, ix);
-        const float fy = qy - floor_small(qy, iy);
-        const float fz = qz - floor_small(qz, iz);
-        const int idx = iz * slice + iy * row + ix;
-        acc += trilinear_at(vol + idx, row, slice, fx, fy, fz);
+    for (int i = 0; i < g.N; ++i) {
+        const int idx = fix_cell(qz) * slice + fix_cell(qy) * row + fix_cell(qx);
+        acc += trilinear_at(vol + idx, row, slice, fix_frac(qx), fix_frac(qy), fix_frac(qz));
+        qx += sx;
+        qy += sy;
+        qz += sz;
     }
     return acc;
 }
@@ -135,17 +91,9 @@ forward_kernel(const T* __restrict__ vol, const float* __restrict__ Rt, float* _
     if (r >= g.H || c >= g.W) return;
     Ray ray;
     float result = 0.0f;
-    if (ray_setup(sv, g, (float)c, (float)r, ray)) {
-        float sum = 0.0f;
-        bool ok = true;
-        if (PADDED)
-            ok = march_padded(vol, g, ray, sum);
-        else
-            sum = march_linear(vol, g, ray);
-        if (ok) {
-            const float I = (g.density_factor * ray.dt) * sum;
-            result = (MODE == 1) ? -expm1f(-I) : I;
-        }
+    if (ray_setup(sv, g, (double)c, (double)r, PADDED ? 1.0 : 0.0, ray)) {
+        const float I = (g.density_factor * ray.dt) * march(vol, g, ray);
+        result = (MODE == 1) ? -expm1f(-I) : I;
     }
     out[((size_t)b * g.H + r) * g.W + c] = result;
 }

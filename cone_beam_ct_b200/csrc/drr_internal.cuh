@@ -27,99 +27,127 @@ struct Geom {
     int nx, ny, nz;          // logical volume dims
     int row, slice;          // element strides of j and k in the stored layout
     float hi[3];             // n - 1 per axis: the voxel-centre box is [0, hi]
-    float hi_clamp[3];       // largest float below n - 1 (linear-layout clamp)
-    float inv_sp[3];         // 1 / spacing
-    float origin[3];         // world mm of voxel 0's centre
-    float kinv[6];           // K^-1 = [k0 k1 k2; 0 k3 k4; 0 0 k5]
+    long long lim[3];        // largest 32.32 sample coordinate the stored layout allows
+    double spacing[3];       // voxel size, mm
+    double origin[3];        // world mm of voxel 0's centre
+    double kinv[6];          // K^-1 = [k0 k1 k2; 0 k3 k4; 0 0 k5], from fp64 on the host
     int B, H, W, N;
     float density_factor;
 };
 
-// Per-view quantities, computed once per CTA from the view's [R|t]:
+// Per-view quantities, computed once per CTA from the view's [R|t], in fp64
+// (the pose is widened from fp32; the camera sits hundreds of voxels from
+// the volume, so fp32 here would cost ~1e-4 voxel of sample position):
 //   A = R^T K^-1  (pixel (u, v, 1) -> world direction, unnormalised)
 //   C = (-R^T t - origin) / spacing  (camera centre in IJK)
 struct View {
-    float A[9];
-    float C[3];
+    double A[9];
+    double C[3];
 };
 
 __device__ __forceinline__ void view_setup(const float* __restrict__ Rt12, const Geom& g,
                                            View& v) {
-    float R[9], t[3];
+    double R[9], t[3];
 #pragma unroll
     for (int r = 0; r < 3; ++r) {
 #pragma unroll
-        for (int c = 0; c < 3; ++c) R[3 * r + c] = Rt12[4 * r + c];
-        t[r] = Rt12[4 * r + 3];
+        for (int c = 0; c < 3; ++c) R[3 * r + c] = (double)Rt12[4 * r + c];
+        t[r] = (double)Rt12[4 * r + 3];
     }
-    const float i00 = g.kinv[0], i01 = g.kinv[1], i02 = g.kinv[2];
-    const float i11 = g.kinv[3], i12 = g.kinv[4], i22 = g.kinv[5];
+    const double i00 = g.kinv[0], i01 = g.kinv[1], i02 = g.kinv[2];
+    const double i11 = g.kinv[3], i12 = g.kinv[4], i22 = g.kinv[5];
 #pragma unroll
     for (int a = 0; a < 3; ++a) {
         // column a of R is row a of R^T
-        const float r0 = R[a], r1 = R[3 + a], r2 = R[6 + a];
+        const double r0 = R[a], r1 = R[3 + a], r2 = R[6 + a];
         v.A[3 * a + 0] = r0 * i00;
-        v.A[3 * a + 1] = fmaf(r0, i01, r1 * i11);
-        v.A[3 * a + 2] = fmaf(r0, i02, fmaf(r1, i12, r2 * i22));
-        const float cw = -fmaf(r0, t[0], fmaf(r1, t[1], r2 * t[2]));
-        v.C[a] = (cw - g.origin[a]) * g.inv_sp[a];
+        v.A[3 * a + 1] = r0 * i01 + r1 * i11;
+        v.A[3 * a + 2] = r0 * i02 + r1 * i12 + r2 * i22;
+        const double cw = -(r0 * t[0] + r1 * t[1] + r2 * t[2]);
+        v.C[a] = (cw - g.origin[a]) / g.spacing[a];
     }
 }
 
-// One ray, clipped and discretised: sample i sits at P + (i + 1/2) * S in
-// IJK coordinates; dt is the sample spacing in world mm.
+// One ray, clipped and discretised.  Sample positions are 32.32 fixed point
+// per axis (high word: the cell index, low word: the fraction), advanced by
+// exact integer adds: sample i sits at q0 + i * s.  An fp32 position would
+// carry ~1e-5 voxel of rounding at coordinates ~256, which a ray grazing a
+// sharp edge turns into ~1e-4 of its integral; here the positions are exact
+// to ~1e-9 voxel and the fraction handed to the interpolation to 2^-23.
+// Because positions are exactly linear in i, keeping the first and the last
+// sample inside [0, lim] keeps every sample inside: that is the whole memory-
+// safety argument of the sample loops.
 struct Ray {
-    float P[3];
-    float S[3];
+    long long q0[3];
+    long long s[3];
     float dt;
 };
 
+constexpr double kFix = 4294967296.0;           // 2^32
+
+// fraction of a 32.32 coordinate as a float in [0, 1), from its top 23 bits
+__device__ __forceinline__ float fix_frac(long long q) {
+    const unsigned lo = (unsigned)(unsigned long long)q;
+    return __uint_as_float(0x3F800000u | (lo >> 9)) - 1.0f;
+}
+
+__device__ __forceinline__ int fix_cell(long long q) { return (int)(q >> 32); }
+
 // Returns false for a miss (or a ray whose geometry is not finite).
-__device__ __forceinline__ bool ray_setup(const View& v, const Geom& g, float u, float w,
-                                          Ray& ray) {
-    float a[3], d[3];
+//   offset     added to the IJK coordinates (1 for the zero-bordered layout)
+//   g.lim[k]   largest allowed 32.32 coordinate along axis k; the smallest is
+//              0.  Samples that rounding pushes past [0, lim] are pulled back
+//              by a few 2^-32 voxel.
+__device__ __forceinline__ bool ray_setup(const View& v, const Geom& g, double u, double w,
+                                          double offset, Ray& ray) {
+    double a[3], d[3];
 #pragma unroll
-    for (int k = 0; k < 3; ++k) a[k] = fmaf(v.A[3 * k], u, fmaf(v.A[3 * k + 1], w, v.A[3 * k + 2]));
-    const float n2 = fmaf(a[0], a[0], fmaf(a[1], a[1], a[2] * a[2]));
-    const float rn = 1.0f / sqrtf(n2);
-    float t_near = -INFINITY, t_far = INFINITY;
+    for (int k = 0; k < 3; ++k) a[k] = v.A[3 * k] * u + v.A[3 * k + 1] * w + v.A[3 * k + 2];
+    const double rn = 1.0 / sqrt(a[0] * a[0] + a[1] * a[1] + a[2] * a[2]);
+    double t_near = -INFINITY, t_far = INFINITY;
     bool ok = true;
 #pragma unroll
     for (int k = 0; k < 3; ++k) {
-        d[k] = a[k] * rn * g.inv_sp[k];
-        const float c = v.C[k];
+        d[k] = a[k] * rn / g.spacing[k];
+        const double c = v.C[k];
         ok = ok && isfinite(d[k]) && isfinite(c);
-        if (d[k] != 0.0f) {
-            const float inv = 1.0f / d[k];
-            const float ta = (0.0f - c) * inv;
-            const float tb = (g.hi[k] - c) * inv;
-            t_near = fmaxf(t_near, fminf(ta, tb));
-            t_far = fminf(t_far, fmaxf(ta, tb));
+        if (d[k] != 0.0) {
+            const double ta = (0.0 - c) / d[k];
+            const double tb = ((double)g.hi[k] - c) / d[k];
+            t_near = fmax(t_near, fmin(ta, tb));
+            t_far = fmin(t_far, fmax(ta, tb));
         } else {
             // parallel to this slab: inside (planes included) or a miss
-            ok = ok && (c >= 0.0f) && (c <= g.hi[k]);
+            ok = ok && (c >= 0.0) && (c <= (double)g.hi[k]);
         }
     }
-    const float t0 = fmaxf(t_near, 0.0f);
-    const float t1 = t_far;
+    const double t0 = fmax(t_near, 0.0);
+    const double t1 = t_far;
     if (!ok || !(t1 > t0) || !isfinite(t1)) return false;
-    const float dt = (t1 - t0) / (float)g.N;
+    const double dt = (t1 - t0) / (double)g.N;
+    const double tm = t0 + 0.5 * dt;                 // parameter of sample 0
+    const long long last = g.N - 1;
 #pragma unroll
     for (int k = 0; k < 3; ++k) {
-        ray.P[k] = fmaf(t0, d[k], v.C[k]);
-        ray.S[k] = dt * d[k];
+        const double first_d = v.C[k] + tm * d[k] + offset;
+        const double end_d = first_d + (double)last * dt * d[k];
+        // inside the box these are < 2^22; anything far outside is absurd geometry
+        if (!(fabs(first_d) < 16777216.0 && fabs(end_d) < 16777216.0)) return false;
+        // + 2^8: fix_frac truncates to 23 bits, so this makes it round to nearest
+        long long first = __double2ll_rn(first_d * kFix) + 256;
+        long long step = __double2ll_rn(dt * d[k] * kFix);
+        long long end = first + last * step;
+        const long long lim = g.lim[k];
+        if (first < 0 || first > lim || end < 0 || end > lim) {
+            first = min(max(first, 0LL), lim);
+            end = min(max(end, 0LL), lim);
+            step = last > 0 ? (end - first) / last : 0;   // truncation keeps q0 + last*s in range
+        }
+        ray.q0[k] = first;
+        ray.s[k] = step;
     }
-    ray.dt = dt;
+    ray.dt = (float)dt;
     return true;
-}
-
-// floor(x) for 0 <= x < 2^22 with full-rate FP32 ops only: adding 1.5 * 2^23
-// with round-down leaves floor(x) in the low mantissa bits.
-__device__ __forceinline__ float floor_small(float x, int& xi) {
-    const float kMagic = 12582912.0f;            // 1.5 * 2^23, bit pattern 0x4B400000
-    const float t = __fadd_rd(x, kMagic);
-    xi = __float_as_int(t) - 0x4B400000;
-    return t - kMagic;                           // exact
 }
 
 // Pixel of this thread inside a kTileW x kTileH tile (warps are 8 x 4).

@@ -50,7 +50,7 @@ def test_small_ragged_fp32(cuda, case, layout, mode):
     w = wl.small_random_case(**CASES[case])
     got = gpu_forward(w, layout=layout, dtype=F32, mode=mode)
     ref = _oracle(w, mode=mode)
-    assert np.count_nonzero(ref) > 0.2 * ref.size
+    assert np.count_nonzero(ref) > 0.05 * ref.size
     assert_parity(got, ref, TOL_F32, what=f"case {case}")
     # misses are exact zeros on both sides
     assert np.all(got[ref == 0.0] == 0.0)
