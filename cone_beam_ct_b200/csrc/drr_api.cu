@@ -45,9 +45,21 @@ constexpr int kMaxRows = 65535 * drr::kTileH;
 constexpr int64_t kMaxElements = (int64_t(1) << 31) - 1;
 constexpr int kMaxDim = (1 << 22) - 4;   // keeps padded coordinates inside the exact floor range
 
+bool known_layout(int layout) {
+    return layout == DRR_LAYOUT_LINEAR || layout == DRR_LAYOUT_PADDED ||
+           layout == DRR_LAYOUT_CORNERS;
+}
+
 int64_t stored_elements(const int dims[3], int layout) {
+    if (layout == DRR_LAYOUT_CORNERS)
+        return (int64_t)(dims[0] - 1) * (dims[1] - 1) * (dims[2] - 1) * 8;
     const int pad = layout == DRR_LAYOUT_PADDED ? 2 : 0;
     return (int64_t)(dims[0] + pad) * (dims[1] + pad) * (dims[2] + pad);
+}
+
+size_t layout_alignment(int layout, int dtype) {
+    if (layout == DRR_LAYOUT_CORNERS) return 16;
+    return dtype == DRR_F32 ? 4 : 2;
 }
 
 drr_status check_volume(const int dims[3], const float spacing[3], const float origin[3]) {
@@ -92,13 +104,19 @@ void fill_geom(drr::Geom& g, const int dims[3], const float spacing[3], const fl
     g.nx = dims[0];
     g.ny = dims[1];
     g.nz = dims[2];
-    const int pad = layout == DRR_LAYOUT_PADDED ? 2 : 0;
-    g.row = dims[0] + pad;
-    g.slice = (dims[0] + pad) * (dims[1] + pad);
+    if (layout == DRR_LAYOUT_CORNERS) {           // strides of cells, 8 elements each
+        g.row = dims[0] - 1;
+        g.slice = (dims[0] - 1) * (dims[1] - 1);
+    } else {
+        const int pad = layout == DRR_LAYOUT_PADDED ? 2 : 0;
+        g.row = dims[0] + pad;
+        g.slice = (dims[0] + pad) * (dims[1] + pad);
+    }
     for (int a = 0; a < 3; ++a) {
         g.hi[a] = (float)(dims[a] - 1);
         // largest 32.32 sample coordinate whose 8 corners are stored: cell <= n-2
-        // for the linear layout, cell <= n (inside the zero border) for the padded one
+        // for the linear and corner layouts, cell <= n (inside the zero border)
+        // for the padded one
         const long long cells = layout == DRR_LAYOUT_PADDED ? dims[a] + 1 : dims[a] - 1;
         g.lim[a] = cells * (1LL << 32) - 1;
         g.spacing[a] = spacing[a];
@@ -137,7 +155,7 @@ DRR_API size_t drr_prepared_bytes(const int dims[3], drr_dtype dtype, drr_layout
     for (int a = 0; a < 3; ++a)
         if (dims[a] < 2 || dims[a] > kMaxDim) return 0;
     if (dtype != DRR_F32 && dtype != DRR_BF16) return 0;
-    if (layout != DRR_LAYOUT_LINEAR && layout != DRR_LAYOUT_PADDED) return 0;
+    if (!known_layout(layout)) return 0;
     const int64_t n = stored_elements(dims, layout);
     if (n > kMaxElements) return 0;
     return (size_t)n * (dtype == DRR_F32 ? 4 : 2);
@@ -151,12 +169,12 @@ DRR_API drr_status drr_prepare_volume(const float* src, const int dims[3], drr_d
         if (dims[a] < 2 || dims[a] > kMaxDim)
             return fail(DRR_ERR_INVALID_ARG, "dims[%d] = %d must be in [2, %d]", a, dims[a], kMaxDim);
     if (dtype != DRR_F32 && dtype != DRR_BF16) return fail(DRR_ERR_INVALID_ARG, "unknown dtype %d", dtype);
-    if (layout != DRR_LAYOUT_LINEAR && layout != DRR_LAYOUT_PADDED)
-        return fail(DRR_ERR_INVALID_ARG, "unknown layout %d", layout);
+    if (!known_layout(layout)) return fail(DRR_ERR_INVALID_ARG, "unknown layout %d", layout);
     const size_t need = drr_prepared_bytes(dims, dtype, layout);
     if (need == 0) return fail(DRR_ERR_UNSUPPORTED, "volume too large (max 2^31 - 1 stored elements)");
     if (!src || !dst) return fail(DRR_ERR_INVALID_ARG, "src and dst must be non-NULL");
-    if (!aligned(src, 4) || !aligned(dst, 4)) return fail(DRR_ERR_INVALID_ARG, "src and dst must be 4-byte aligned");
+    if (!aligned(src, 4) || !aligned(dst, layout == DRR_LAYOUT_CORNERS ? 16 : 4))
+        return fail(DRR_ERR_INVALID_ARG, "src must be 4-byte aligned, dst 4-byte (16-byte for DRR_LAYOUT_CORNERS)");
     if (dst_bytes < need)
         return fail(DRR_ERR_INVALID_ARG, "dst holds %zu bytes, %zu needed", dst_bytes, need);
     const size_t src_bytes = (size_t)dims[0] * dims[1] * dims[2] * 4;
@@ -176,13 +194,13 @@ DRR_API drr_status drr_render(const void* vol, drr_dtype dtype, drr_layout layou
     st = check_rays(K, Rt, B, H, W, n_samples, density_factor, mode);
     if (st != DRR_OK) return st;
     if (dtype != DRR_F32 && dtype != DRR_BF16) return fail(DRR_ERR_INVALID_ARG, "unknown dtype %d", dtype);
-    if (layout != DRR_LAYOUT_LINEAR && layout != DRR_LAYOUT_PADDED)
-        return fail(DRR_ERR_INVALID_ARG, "unknown layout %d", layout);
+    if (!known_layout(layout)) return fail(DRR_ERR_INVALID_ARG, "unknown layout %d", layout);
     if (stored_elements(dims, layout) > kMaxElements)
         return fail(DRR_ERR_UNSUPPORTED, "volume too large (max 2^31 - 1 stored elements)");
     if ((int64_t)B * H * W == 0) return ok();   // empty batch or image: nothing to do
-    if (!vol || !aligned(vol, dtype == DRR_F32 ? 4 : 2))
-        return fail(DRR_ERR_INVALID_ARG, "vol must be a non-NULL, element-aligned device pointer");
+    if (!vol || !aligned(vol, layout_alignment(layout, dtype)))
+        return fail(DRR_ERR_INVALID_ARG, "vol must be a non-NULL device pointer aligned to %zu bytes",
+                    layout_alignment(layout, dtype));
     if (!out || !aligned(out, 4)) return fail(DRR_ERR_INVALID_ARG, "out must be a non-NULL, 4-byte aligned device pointer");
     drr::Geom g;
     fill_geom(g, dims, spacing, origin, K, B, H, W, n_samples, density_factor, layout);

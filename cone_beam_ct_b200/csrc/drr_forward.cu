@@ -78,7 +78,66 @@ __device__ __forceinline__ float march(const T* __restrict__ vol, const Geom& g,
     return acc;
 }
 
-template <typename T, bool PADDED, int MODE>
+// The 8 corner voxels of one cell in the corner-replicated layout, in the
+// order a + 2b + 4c of corner (a, b, c): two 16-byte loads for fp32 ...
+__device__ __forceinline__ void load_corners(const float* __restrict__ p, float v[8]) {
+    const float4 lo = __ldg(reinterpret_cast<const float4*>(p));
+    const float4 hi = __ldg(reinterpret_cast<const float4*>(p) + 1);
+    v[0] = lo.x;
+    v[1] = lo.y;
+    v[2] = lo.z;
+    v[3] = lo.w;
+    v[4] = hi.x;
+    v[5] = hi.y;
+    v[6] = hi.z;
+    v[7] = hi.w;
+}
+
+// ... and one for bf16 (element 2m in the low half of word m; widening is exact).
+__device__ __forceinline__ void load_corners(const uint16_t* __restrict__ p, float v[8]) {
+    const uint4 w = __ldg(reinterpret_cast<const uint4*>(p));
+    v[0] = __uint_as_float(w.x << 16);
+    v[1] = __uint_as_float(w.x & 0xFFFF0000u);
+    v[2] = __uint_as_float(w.y << 16);
+    v[3] = __uint_as_float(w.y & 0xFFFF0000u);
+    v[4] = __uint_as_float(w.z << 16);
+    v[5] = __uint_as_float(w.z & 0xFFFF0000u);
+    v[6] = __uint_as_float(w.w << 16);
+    v[7] = __uint_as_float(w.w & 0xFFFF0000u);
+}
+
+// Sum of the N samples of one ray in the corner-replicated layout: one cell
+// record per sample, the same lerps (and so the same result, bit for bit) as
+// trilinear_at on the linear layout.  Cells stay in [0, n-2] (g.lim as for
+// the linear layout), inside the stored records.
+template <typename T>
+__device__ __forceinline__ float march_corners(const T* __restrict__ vol, const Geom& g,
+                                               const Ray& ray) {
+    const int row = g.row, slice = g.slice;      // cell strides
+    long long qx = ray.q0[0], qy = ray.q0[1], qz = ray.q0[2];
+    const long long sx = ray.s[0], sy = ray.s[1], sz = ray.s[2];
+    float acc = 0.0f;
+#pragma unroll 4
+    for (int i = 0; i < g.N; ++i) {
+        const int cell = fix_cell(qz) * slice + fix_cell(qy) * row + fix_cell(qx);
+        float v[8];
+        load_corners(vol + (size_t)cell * 8, v);
+        const float fx = fix_frac(qx), fy = fix_frac(qy), fz = fix_frac(qz);
+        const float c00 = fmaf(fx, v[1] - v[0], v[0]);
+        const float c10 = fmaf(fx, v[3] - v[2], v[2]);
+        const float c01 = fmaf(fx, v[5] - v[4], v[4]);
+        const float c11 = fmaf(fx, v[7] - v[6], v[6]);
+        const float c0 = fmaf(fy, c10 - c00, c00);
+        const float c1 = fmaf(fy, c11 - c01, c01);
+        acc += fmaf(fz, c1 - c0, c0);
+        qx += sx;
+        qy += sy;
+        qz += sz;
+    }
+    return acc;
+}
+
+template <typename T, int LAYOUT, int MODE>
 __global__ void __launch_bounds__(kThreads)
 forward_kernel(const T* __restrict__ vol, const float* __restrict__ Rt, float* __restrict__ out,
                const Geom g) {
@@ -91,35 +150,40 @@ forward_kernel(const T* __restrict__ vol, const float* __restrict__ Rt, float* _
     if (r >= g.H || c >= g.W) return;
     Ray ray;
     float result = 0.0f;
-    if (ray_setup(sv, g, (double)c, (double)r, PADDED ? 1.0 : 0.0, ray)) {
-        const float I = (g.density_factor * ray.dt) * march(vol, g, ray);
+    if (ray_setup(sv, g, (double)c, (double)r, LAYOUT == 1 ? 1.0 : 0.0, ray)) {
+        const float sum = LAYOUT == 2 ? march_corners(vol, g, ray) : march(vol, g, ray);
+        const float I = (g.density_factor * ray.dt) * sum;
         result = (MODE == 1) ? -expm1f(-I) : I;
     }
     out[((size_t)b * g.H + r) * g.W + c] = result;
 }
 
-template <typename T, bool PADDED>
+template <typename T, int LAYOUT>
 cudaError_t launch_typed(const void* vol, const Geom& g, const float* Rt, int mode, float* out,
                          cudaStream_t stream) {
     const dim3 grid((g.W + kTileW - 1) / kTileW, (g.H + kTileH - 1) / kTileH, g.B);
     const T* v = static_cast<const T*>(vol);
     if (mode == 1)
-        forward_kernel<T, PADDED, 1><<<grid, kThreads, 0, stream>>>(v, Rt, out, g);
+        forward_kernel<T, LAYOUT, 1><<<grid, kThreads, 0, stream>>>(v, Rt, out, g);
     else
-        forward_kernel<T, PADDED, 0><<<grid, kThreads, 0, stream>>>(v, Rt, out, g);
+        forward_kernel<T, LAYOUT, 0><<<grid, kThreads, 0, stream>>>(v, Rt, out, g);
     return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t launch_layout(const void* vol, int layout, const Geom& g, const float* Rt, int mode,
+                          float* out, cudaStream_t stream) {
+    if (layout == 2) return launch_typed<T, 2>(vol, g, Rt, mode, out, stream);
+    if (layout == 1) return launch_typed<T, 1>(vol, g, Rt, mode, out, stream);
+    return launch_typed<T, 0>(vol, g, Rt, mode, out, stream);
 }
 
 }  // namespace
 
 cudaError_t launch_forward(const void* vol, int dtype, int layout, const Geom& g,
                            const float* Rt, int mode, float* out, cudaStream_t stream) {
-    const bool padded = layout == 1;
-    if (dtype == 0)
-        return padded ? launch_typed<float, true>(vol, g, Rt, mode, out, stream)
-                      : launch_typed<float, false>(vol, g, Rt, mode, out, stream);
-    return padded ? launch_typed<uint16_t, true>(vol, g, Rt, mode, out, stream)
-                  : launch_typed<uint16_t, false>(vol, g, Rt, mode, out, stream);
+    if (dtype == 0) return launch_layout<float>(vol, layout, g, Rt, mode, out, stream);
+    return launch_layout<uint16_t>(vol, layout, g, Rt, mode, out, stream);
 }
 
 }  // namespace drr

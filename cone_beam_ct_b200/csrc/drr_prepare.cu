@@ -4,7 +4,8 @@
 // nanodrr's page, "Benchmarks": mixed precision; here storage only, the
 // arithmetic stays fp32).  The padded layout surrounds the volume with a
 // one-voxel zero border, which is exactly the zero padding of the trilinear
-// interpolation.  Plain grid-stride loops: a one-off HBM-bound copy.
+// interpolation.  The corner-replicated layout stores every cell's 8 corner
+// voxels together.  Plain grid-stride loops: a one-off HBM-bound copy.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -51,6 +52,44 @@ __global__ void to_padded(const float* __restrict__ src, T* __restrict__ dst, in
     }
 }
 
+// Corner-replicated layout: record m = cell (i, j, k) holds the 8 voxels
+// src[k+c][j+b][i+a] in the order a + 2b + 4c, written as one (bf16) or two
+// (fp32) 16-byte stores.
+__device__ __forceinline__ void store_corners(float* dst, const float v[8]) {
+    float4* d = reinterpret_cast<float4*>(dst);
+    d[0] = make_float4(v[0], v[1], v[2], v[3]);
+    d[1] = make_float4(v[4], v[5], v[6], v[7]);
+}
+
+__device__ __forceinline__ void store_corners(uint16_t* dst, const float v[8]) {
+    unsigned w[4];
+#pragma unroll
+    for (int m = 0; m < 4; ++m)
+        w[m] = (unsigned)store_value<uint16_t>(v[2 * m]) |
+               ((unsigned)store_value<uint16_t>(v[2 * m + 1]) << 16);
+    *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+template <typename T>
+__global__ void to_corners(const float* __restrict__ src, T* __restrict__ dst, int nx, int ny,
+                           int nz) {
+    const int cx = nx - 1, cy = ny - 1;
+    const int64_t n = (int64_t)cx * cy * (nz - 1);
+    for (int64_t m = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; m < n;
+         m += (int64_t)gridDim.x * blockDim.x) {
+        const int i = (int)(m % cx);
+        const int j = (int)((m / cx) % cy);
+        const int k = (int)(m / ((int64_t)cx * cy));
+        const float* p = src + (((int64_t)k * ny + j) * nx + i);
+        const int64_t sy = nx, sz = (int64_t)nx * ny;
+        float v[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+            v[c] = __ldg(p + ((c & 1) ? 1 : 0) + ((c & 2) ? sy : 0) + ((c & 4) ? sz : 0));
+        store_corners(dst + m * 8, v);
+    }
+}
+
 int grid_for(int64_t n) {
     int64_t blocks = (n + 255) / 256;
     const int64_t cap = 148 * 16;   // enough CTAs to fill every SM; the loops stride
@@ -68,6 +107,14 @@ cudaError_t launch_prepare(const float* src, int nx, int ny, int nz, int dtype, 
         else
             to_linear<uint16_t><<<grid_for(n), 256, 0, stream>>>(src, static_cast<uint16_t*>(dst),
                                                                  n);
+    } else if (layout == 2) {
+        const int64_t n = (int64_t)(nx - 1) * (ny - 1) * (nz - 1);
+        if (dtype == 0)
+            to_corners<float><<<grid_for(n), 256, 0, stream>>>(src, static_cast<float*>(dst), nx,
+                                                               ny, nz);
+        else
+            to_corners<uint16_t><<<grid_for(n), 256, 0, stream>>>(
+                src, static_cast<uint16_t*>(dst), nx, ny, nz);
     } else {
         const int64_t n = (int64_t)(nx + 2) * (ny + 2) * (nz + 2);
         if (dtype == 0)

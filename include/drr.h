@@ -90,9 +90,16 @@ typedef enum {
     /* vol[k][j][i] exactly as the caller holds it (float32 or bfloat16). */
     DRR_LAYOUT_LINEAR = 0,
     /* vol[k+1][j+1][i+1] inside a one-voxel zero border: dims (nx+2, ny+2,
-       nz+2).  Written by drr_prepare_volume.  The border is the zero padding
-       of the interpolation, so the sample loop needs no clamping. */
-    DRR_LAYOUT_PADDED = 1
+       nz+2).  Written by drr_prepare_volume. */
+    DRR_LAYOUT_PADDED = 1,
+    /* Corner-replicated: for every cell (i, j, k) in [0, nx-2] x [0, ny-2] x
+       [0, nz-2] (cell index (k*(ny-1) + j)*(nx-1) + i) its 8 corner voxels
+       vol[k+c][j+b][i+a] stored contiguously in the order a + 2b + 4c: 8
+       elements, 16 bytes (bf16) or 32 bytes (fp32) per cell, 16-byte
+       aligned.  Written by drr_prepare_volume.  One sample of the forward
+       then reads its 8 voxels with one (bf16) or two (fp32) 16-byte loads
+       instead of 8 scalar gathers; the price is 8x the storage. */
+    DRR_LAYOUT_CORNERS = 2
 } drr_layout;
 
 /* Forward projection.
@@ -109,8 +116,9 @@ typedef enum {
  *   density_factor  finite scale of the integral.
  *   mode        DRR_MODE_RAW or DRR_MODE_BEER_LAMBERT.
  *   out         DEVICE float[B*H*W], overwritten.
- * Limits: the volume (with its border, for PADDED) must hold fewer than
- * 2^31 elements; B*H*W < 2^40.
+ * Limits: the stored volume must hold fewer than 2^31 elements (PADDED:
+ * with its border; CORNERS: 8 per cell); B*H*W < 2^40.  A CORNERS volume
+ * must be 16-byte aligned.
  */
 DRR_API drr_status drr_render(const void *vol, drr_dtype dtype, drr_layout layout,
                               const int dims[3], const float spacing[3], const float origin[3],
@@ -145,7 +153,8 @@ DRR_API size_t drr_prepared_bytes(const int dims[3], drr_dtype dtype, drr_layout
  *   src         DEVICE float32 [nz][ny][nx].
  *   dst         DEVICE, at least drr_prepared_bytes(dims, dtype, layout)
  *               bytes (dst_bytes says how many are available); must not
- *               overlap src.  Every byte of the prepared volume is written.
+ *               overlap src; 16-byte aligned for DRR_LAYOUT_CORNERS.  Every
+ *               byte of the prepared volume is written.
  * bf16 conversion rounds to nearest even.  Done once per volume (or once per
  * update of the volume), not per render. */
 DRR_API drr_status drr_prepare_volume(const float *src, const int dims[3], drr_dtype dtype,

@@ -5,7 +5,8 @@ import numpy as np
 
 from cone_beam_ct_b200 import drr
 
-LINEAR, PADDED = drr.DRR_LAYOUT_LINEAR, drr.DRR_LAYOUT_PADDED
+LINEAR, PADDED, CORNERS = drr.DRR_LAYOUT_LINEAR, drr.DRR_LAYOUT_PADDED, drr.DRR_LAYOUT_CORNERS
+LAYOUTS = (LINEAR, PADDED, CORNERS)
 F32, BF16 = drr.DRR_F32, drr.DRR_BF16
 
 

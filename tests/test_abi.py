@@ -99,6 +99,7 @@ RENDER_BAD = [
     (dict(Rt=0), drr.DRR_ERR_INVALID_ARG, "Rt"),
     (dict(Rt=FAKE + 1), drr.DRR_ERR_INVALID_ARG, "Rt"),
     (dict(out=0), drr.DRR_ERR_INVALID_ARG, "out"),
+    (dict(layout=drr.DRR_LAYOUT_CORNERS, vol=FAKE + 4), drr.DRR_ERR_INVALID_ARG, "16 bytes"),
     (dict(out=FAKE + 6), drr.DRR_ERR_INVALID_ARG, "out"),
 ]
 
@@ -151,6 +152,10 @@ def test_prepared_bytes():
     assert drr.drr_prepared_bytes((1, 6, 7), drr.DRR_F32, drr.DRR_LAYOUT_PADDED) == 0
     assert drr.drr_prepared_bytes((5, 6, 7), 3, drr.DRR_LAYOUT_PADDED) == 0
     assert drr.drr_prepared_bytes((2048, 2048, 1024), drr.DRR_F32, drr.DRR_LAYOUT_LINEAR) == 0
+    assert drr.drr_prepared_bytes((5, 6, 7), drr.DRR_F32, drr.DRR_LAYOUT_CORNERS) == 4 * 8 * 4 * 5 * 6
+    assert drr.drr_prepared_bytes((5, 6, 7), drr.DRR_BF16, drr.DRR_LAYOUT_CORNERS) == 2 * 8 * 4 * 5 * 6
+    assert drr.drr_prepared_bytes((640, 640, 640), drr.DRR_BF16, drr.DRR_LAYOUT_CORNERS) == 2 * 8 * 639 ** 3
+    assert drr.drr_prepared_bytes((660, 660, 660), drr.DRR_BF16, drr.DRR_LAYOUT_CORNERS) == 0
 
 
 PREPARE_BAD = [
@@ -162,6 +167,7 @@ PREPARE_BAD = [
     (dict(dst_bytes=100), drr.DRR_ERR_INVALID_ARG),
     (dict(dst=FAKE + 64), drr.DRR_ERR_INVALID_ARG),      # overlaps src
     (dict(src=FAKE + 2), drr.DRR_ERR_INVALID_ARG),       # misaligned
+    (dict(layout=drr.DRR_LAYOUT_CORNERS, dst=FAKE + (1 << 24) + 8), drr.DRR_ERR_INVALID_ARG),
     (dict(dims=(2048, 2048, 1024)), drr.DRR_ERR_UNSUPPORTED),
 ]
 

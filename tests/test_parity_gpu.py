@@ -16,8 +16,8 @@ import pytest
 
 import oracle
 from cone_beam_ct_b200 import workloads as wl
-from tests.gpu_helpers import (BF16, F32, LINEAR, PADDED, assert_parity, bf16_values,
-                               gpu_forward)
+from tests.gpu_helpers import (BF16, CORNERS, F32, LAYOUTS, LINEAR, PADDED, assert_parity,
+                               bf16_values, gpu_forward)
 
 pytestmark = pytest.mark.gpu
 TOL_F32, TOL_BF16 = 1e-4, 1e-2
@@ -44,7 +44,7 @@ CASES = [dict(seed=101), dict(seed=102, dims=(40, 9, 31), H=33, W=71, n_samples=
 
 
 @pytest.mark.parametrize("case", range(len(CASES)))
-@pytest.mark.parametrize("layout", [LINEAR, PADDED])
+@pytest.mark.parametrize("layout", LAYOUTS)
 @pytest.mark.parametrize("mode", [wl.MODE_RAW, wl.MODE_BEER_LAMBERT])
 def test_small_ragged_fp32(cuda, case, layout, mode):
     w = wl.small_random_case(**CASES[case])
@@ -57,7 +57,7 @@ def test_small_ragged_fp32(cuda, case, layout, mode):
 
 
 @pytest.mark.parametrize("case", range(len(CASES)))
-@pytest.mark.parametrize("layout", [LINEAR, PADDED])
+@pytest.mark.parametrize("layout", LAYOUTS)
 def test_small_ragged_bf16(cuda, case, layout):
     w = wl.small_random_case(**CASES[case])
     got = gpu_forward(w, layout=layout, dtype=BF16, mode=wl.MODE_RAW)
@@ -66,21 +66,30 @@ def test_small_ragged_bf16(cuda, case, layout):
     assert_parity(got, _oracle(w, mode=wl.MODE_RAW), TOL_BF16, what="vs oracle on fp32 values")
 
 
-@pytest.mark.parametrize("layout", [LINEAR, PADDED])
+@pytest.mark.parametrize("layout", LAYOUTS)
 def test_config1_full_image(cuda, layout):
     w = wl.make_config(1)
     got = gpu_forward(w, layout=layout)
     assert_parity(got, _oracle(w), TOL_F32, what="config 1")
 
 
+_CFG2 = {}
+
+
+def _config2_oracle(mode):
+    if mode not in _CFG2:
+        w = wl.make_config(2)
+        _CFG2[mode] = (w, _oracle(w, mode=mode))
+    return _CFG2[mode]
+
+
 @pytest.mark.slow
-@pytest.mark.parametrize("layout", [LINEAR, PADDED])
-def test_config2_full_image(cuda, layout):
-    w = wl.make_config(2)
-    got = gpu_forward(w, layout=layout)
-    for mode in (wl.MODE_BEER_LAMBERT, wl.MODE_RAW):
-        g = got if mode == w.mode else gpu_forward(w, layout=layout, mode=mode)
-        assert_parity(g, _oracle(w, mode=mode), TOL_F32, what=f"config 2 mode {mode}")
+@pytest.mark.parametrize("layout", LAYOUTS)
+@pytest.mark.parametrize("mode", [wl.MODE_BEER_LAMBERT, wl.MODE_RAW])
+def test_config2_full_image(cuda, layout, mode):
+    w, ref = _config2_oracle(mode)
+    assert_parity(gpu_forward(w, layout=layout, mode=mode), ref, TOL_F32,
+                  what=f"config 2 layout {layout} mode {mode}")
 
 
 def _sampled_ids(w, n, seed):
@@ -101,9 +110,10 @@ def _sampled_oracle(w, ids, vol=None, mode=None):
 
 
 @pytest.mark.slow
-def test_config3_bf16_sampled(cuda):
+@pytest.mark.parametrize("layout", [PADDED, CORNERS])
+def test_config3_bf16_sampled(cuda, layout):
     w = wl.make_config(3)
-    got = gpu_forward(w, layout=PADDED, dtype=BF16).reshape(-1)
+    got = gpu_forward(w, layout=layout, dtype=BF16).reshape(-1)
     ids = _sampled_ids(w, 40000, 3)
     assert_parity(got[ids], _sampled_oracle(w, ids, vol=bf16_values(w.vol)), TOL_F32,
                   what="config 3 vs oracle on bf16 values")
@@ -115,17 +125,20 @@ def test_config3_bf16_sampled(cuda):
 @pytest.mark.slow
 def test_config4_hbm_sampled(cuda):
     w = wl.make_config(4)
-    for layout in (LINEAR, PADDED):
+    ids = _sampled_ids(w, 30000, 4)
+    ref = _sampled_oracle(w, ids)
+    for layout in LAYOUTS:
         got = gpu_forward(w, layout=layout).reshape(-1)
-        ids = _sampled_ids(w, 30000, 4)
-        assert_parity(got[ids], _sampled_oracle(w, ids), TOL_F32, what=f"config 4 layout {layout}")
+        assert_parity(got[ids], ref, TOL_F32, what=f"config 4 layout {layout}")
 
 
-def test_linear_and_padded_layouts_agree(cuda):
+def test_layouts_agree(cuda):
     w = wl.small_random_case(105, H=64, W=64)
-    a = gpu_forward(w, layout=LINEAR, dtype=F32)
-    b = gpu_forward(w, layout=PADDED, dtype=F32)
-    assert_parity(a, b, 1e-5, what="linear vs padded")
+    for dtype in (F32, BF16):
+        a = gpu_forward(w, layout=LINEAR, dtype=dtype)
+        # same positions, fractions and lerps: the corner layout is bit-identical
+        assert np.array_equal(a, gpu_forward(w, layout=CORNERS, dtype=dtype))
+        assert_parity(a, gpu_forward(w, layout=PADDED, dtype=dtype), 1e-5, what="linear vs padded")
 
 
 def test_forward_is_deterministic(cuda):
@@ -143,7 +156,7 @@ def test_camera_inside_volume_and_axis_parallel_rays(cuda):
     Rt[1, :, 3] = [0.0, 0.0, 30.0]
     K = wl.intrinsics(12.0, 12.0, 9.0, 10.0)
     w.K, w.Rt = K, Rt
-    for layout in (LINEAR, PADDED):
+    for layout in LAYOUTS:
         got = gpu_forward(w, layout=layout, mode=wl.MODE_RAW)
         assert_parity(got, _oracle(w, mode=wl.MODE_RAW), TOL_F32, what="inside/axis")
 
@@ -153,7 +166,7 @@ def test_non_finite_pose_gives_zero_image(cuda):
     Rt = w.Rt.copy()
     Rt[1, 0, 0] = np.nan
     Rt[2, 2, 3] = np.inf
-    for layout in (LINEAR, PADDED):
+    for layout in LAYOUTS:
         got = gpu_forward(w, layout=layout, Rt=Rt)
         assert np.all(got[1] == 0.0) and np.all(got[2] == 0.0)
         assert_parity(got[0], _oracle(w, Rt=w.Rt[:1])[0], TOL_F32)
@@ -188,19 +201,24 @@ def test_prepare_layouts_round_trip(cuda):
     nx, ny, nz = w.dims
     for dtype, np_t, conv in ((F32, np.float32, lambda a: a),
                               (BF16, np.uint16, lambda a: oracle.bf16_to_float(a))):
-        for layout in (LINEAR, PADDED):
+        expect = w.vol if dtype == F32 else bf16_values(w.vol)
+        for layout in LAYOUTS:
             nbytes = drr.drr_prepared_bytes(w.dims, dtype, layout)
             buf = torch.full((nbytes,), 0xAB, dtype=torch.uint8, device="cuda")
             drr.drr_prepare_volume(v, w.dims, dtype, layout, buf)
             torch.cuda.synchronize()
             a = conv(buf.cpu().numpy().view(np_t))
             if layout == LINEAR:
-                vals = a.reshape(nz, ny, nx)
-            else:
+                assert np.array_equal(a.reshape(nz, ny, nx), expect)
+            elif layout == PADDED:
                 p = a.reshape(nz + 2, ny + 2, nx + 2)
-                vals = p[1:-1, 1:-1, 1:-1]
+                assert np.array_equal(p[1:-1, 1:-1, 1:-1], expect)
                 border = p.copy()
                 border[1:-1, 1:-1, 1:-1] = 0
                 assert np.all(border == 0)
-            expect = w.vol if dtype == F32 else bf16_values(w.vol)
-            assert np.array_equal(vals, expect)
+            else:
+                rec = a.reshape(nz - 1, ny - 1, nx - 1, 8)
+                for corner in range(8):
+                    da, db, dc = corner & 1, (corner >> 1) & 1, corner >> 2
+                    assert np.array_equal(rec[..., corner],
+                                          expect[dc:nz - 1 + dc, db:ny - 1 + db, da:nx - 1 + da])
