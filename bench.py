@@ -60,6 +60,23 @@ def dist_env():
     return world, rank, local
 
 
+def max_over_ranks(values, device):
+    """Element-wise max of a list of floats over all ranks (identity when no
+    process group is running).  Every rank must call it, in the same order."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.cpu()]
+
+
+def job_throughput(world, units_per_rank_step, steps, max_ms):
+    """Whole-job rate: the units every rank processed over the slowest rank's
+    time (weak scaling: each rank runs its own replica of the workload)."""
+    return world * units_per_rank_step * steps / (max_ms * 1e-3)
+
+
 # ---------------------------------------------------------------------------
 # workload description
 
@@ -359,17 +376,12 @@ def run_ours(args):
     per = np.array([[ev[s][i].elapsed_time(ev[s][i + 1]) for i in range(4)]
                     for s in range(args.steps)])          # ms: prepare, forward, zero, adjoint
     step_ms = per.sum(axis=1)
-    total_ms = float(step_ms.sum())
-    kern_ms = per.mean(axis=0)
-    if world > 1:
-        t = torch.tensor([total_ms] + list(kern_ms), dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(t[0])
-        kern_ms = t[1:].cpu().numpy()
+    red = max_over_ranks([float(step_ms.sum())] + list(per.mean(axis=0)), dev)
+    total_ms, kern_ms = red[0], np.array(red[1:])
     ms_per_step = total_ms / args.steps
     samples = w.samples
-    value = world * samples * args.steps / (total_ms * 1e-3) / 1e9
-    fps = world * w.B * args.steps / (total_ms * 1e-3)
+    value = job_throughput(world, samples, args.steps, total_ms) / 1e9
+    fps = job_throughput(world, w.B, args.steps, total_ms)
 
     # e2e through the public API with pinned host buffers
     e2e = None
@@ -400,14 +412,10 @@ def run_ours(args):
             e2e_step()
         e1.record(stream)
         torch.cuda.synchronize()
-        e2e_ms = e0.elapsed_time(e1)
-        if world > 1:
-            t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-            e2e_ms = float(t[0])
+        e2e_ms = max_over_ranks([e0.elapsed_time(e1)], dev)[0]
         h2d = h_vol.numel() * 4 + h_Rt.numel() * 4 + h_go.numel() * 4
         d2h = h_out.numel() * 4 + h_grad.numel() * 4
-        e2e = {"value": world * samples * args.steps / (e2e_ms * 1e-3) / 1e9,
+        e2e = {"value": job_throughput(world, samples, args.steps, e2e_ms) / 1e9,
                "unit": "Gsamples/s", "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "ms_per_step": e2e_ms / args.steps,
                "note": "includes the 256 MiB L2 flush write before each step"}
