@@ -48,6 +48,8 @@ def parse_args():
                    help="workload (default 2: 256^3 fp32, 64 views 200x200, 256 samples)")
     p.add_argument("--layout", choices=["padded", "corners", "linear"], default="corners",
                    help="volume layout drr_prepare_volume writes for the forward")
+    p.add_argument("--texture", action="store_true",
+                   help="also time the texture-trilinear comparison forward (libdrr_texture.so)")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     return p.parse_args()
@@ -300,6 +302,37 @@ def cpu_baseline(w):
             "sample": f"first {views} of {w.B} views, forward + adjoint (fp64), {dt:.1f} s"}
 
 
+def texture_comparison(torch, w, vol32, Rt, exact_out):
+    """Forward through the texture units (8-bit interpolation weights) on the
+    same workload: kernel time (best of 5) and its difference from the exact
+    forward's image (which the parity tests pin to the oracle)."""
+    from cone_beam_ct_b200 import texture
+    res = {}
+    stream = torch.cuda.current_stream()
+    for texel, name in ((texture.TEXEL_F32, "fp32 texels"), (texture.TEXEL_F16, "fp16 texels")):
+        tv = texture.TextureVolume(vol32, w.dims, texel)
+        out = torch.empty_like(exact_out)
+        times = []
+        for _ in range(6):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            tv.render(w.spacing, w.origin, w.K, Rt, w.B, w.H, w.W, w.n_samples, w.density_factor,
+                      w.mode, out, stream=stream)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            times.append(e0.elapsed_time(e1))
+        tv.close()
+        ref = exact_out.double()
+        scale = ref.abs().max().item()
+        diff = (out.double() - ref).abs()
+        big = ref.abs() >= 1e-2 * scale
+        ms = min(times[1:])
+        res[name] = {"ms": ms, "gsamples_s": w.samples / (ms * 1e-3) / 1e9,
+                     "normwise_vs_exact": diff.max().item() / scale,
+                     "per_pixel_vs_exact": (diff[big] / ref.abs()[big]).max().item()}
+    return res
+
+
 def run_ours(args):
     import torch
     from cone_beam_ct_b200 import drr
@@ -449,6 +482,10 @@ def run_ours(args):
     adj_roof = roof("adjoint_kernel", adj_ms, adj_bytes, "adjoint_kernel", wname)
     dominant = adj_roof if adj_ms >= fwd_ms else fwd_roof
 
+    tex = None
+    if args.texture:
+        tex = texture_comparison(torch, w, vol32, Rt, out)
+
     base = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         base = cpu_baseline(w)
@@ -470,6 +507,7 @@ def run_ours(args):
         "roofline": dominant,
         "cpu_baseline": base,
         "e2e": e2e,
+        "texture_comparison": tex,
         "gpu_launches": 3 * args.steps,
         "clocks": clocks,
         "bracket_ms": bracket[0].elapsed_time(bracket[1]),

@@ -16,6 +16,8 @@ PROBE_LIB = os.path.join(HERE, "libdrr_probe.so")
 SOURCES = ["drr_api.cu", "drr_forward.cu", "drr_adjoint.cu", "drr_prepare.cu"]
 HEADERS = ["drr_internal.cuh"]
 PROBE_SOURCES = ["drr_probe.cu"]
+TEXTURE_LIB = os.path.join(HERE, "libdrr_texture.so")
+TEXTURE_SOURCES = ["drr_texture.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-fvisibility=hidden",
          "-shared", "-cudart", "shared"]
@@ -32,7 +34,7 @@ def _stale(lib, sources, headers):
         return True
     t = os.path.getmtime(lib)
     deps = [os.path.join(CSRC, f) for f in sources + headers]
-    deps += [os.path.join(INCLUDE, h) for h in ("drr.h", "drr_probe.h")]
+    deps += [os.path.join(INCLUDE, h) for h in ("drr.h", "drr_probe.h", "drr_texture.h")]
     return any(os.path.getmtime(d) > t for d in deps)
 
 
@@ -46,12 +48,15 @@ def _nvcc_shared(lib, sources, verbose_ptxas):
 
 
 def build(force: bool = False, verbose_ptxas: bool = False) -> str:
-    """Build libdrr.so (the ray-march) and libdrr_probe.so (the bench's L2
-    bandwidth probe); returns the path of libdrr.so."""
+    """Build libdrr.so (the ray-march), libdrr_probe.so (the bench's L2
+    bandwidth probe) and libdrr_texture.so (the texture-trilinear
+    comparison); returns the path of libdrr.so."""
     if force or _stale(LIB, SOURCES, HEADERS):
         _nvcc_shared(LIB, SOURCES, verbose_ptxas)
     if force or _stale(PROBE_LIB, PROBE_SOURCES, []):
         _nvcc_shared(PROBE_LIB, PROBE_SOURCES, verbose_ptxas)
+    if force or _stale(TEXTURE_LIB, TEXTURE_SOURCES, HEADERS):
+        _nvcc_shared(TEXTURE_LIB, TEXTURE_SOURCES, verbose_ptxas)
     return LIB
 
 

@@ -10,7 +10,6 @@
 #include <cstdarg>
 #include <cstdint>
 #include <cstdio>
-#include <cstring>
 
 #include "../../include/drr.h"
 #include "drr_internal.cuh"
@@ -97,46 +96,6 @@ drr_status check_rays(const float K[9], const float* Rt, int B, int H, int W, in
     return DRR_OK;
 }
 
-void fill_geom(drr::Geom& g, const int dims[3], const float spacing[3], const float origin[3],
-               const float K[9], int B, int H, int W, int n_samples, float density_factor,
-               int layout) {
-    std::memset(&g, 0, sizeof(g));
-    g.nx = dims[0];
-    g.ny = dims[1];
-    g.nz = dims[2];
-    if (layout == DRR_LAYOUT_CORNERS) {           // strides of cells, 8 elements each
-        g.row = dims[0] - 1;
-        g.slice = (dims[0] - 1) * (dims[1] - 1);
-    } else {
-        const int pad = layout == DRR_LAYOUT_PADDED ? 2 : 0;
-        g.row = dims[0] + pad;
-        g.slice = (dims[0] + pad) * (dims[1] + pad);
-    }
-    for (int a = 0; a < 3; ++a) {
-        g.hi[a] = (float)(dims[a] - 1);
-        // largest 32.32 sample coordinate whose 8 corners are stored: cell <= n-2
-        // for the linear and corner layouts, cell <= n (inside the zero border)
-        // for the padded one
-        const long long cells = layout == DRR_LAYOUT_PADDED ? dims[a] + 1 : dims[a] - 1;
-        g.lim[a] = cells * (1LL << 32) - 1;
-        g.spacing[a] = spacing[a];
-        g.origin[a] = origin[a];
-    }
-    // inverse of the upper-triangular K, in double
-    const double k0 = K[0], k1 = K[1], k2 = K[2], k4 = K[4], k5 = K[5], k8 = K[8];
-    g.kinv[0] = 1.0 / k0;
-    g.kinv[1] = -k1 / (k0 * k4);
-    g.kinv[2] = (k1 * k5 - k2 * k4) / (k0 * k4 * k8);
-    g.kinv[3] = 1.0 / k4;
-    g.kinv[4] = -k5 / (k4 * k8);
-    g.kinv[5] = 1.0 / k8;
-    g.B = B;
-    g.H = H;
-    g.W = W;
-    g.N = n_samples;
-    g.density_factor = density_factor;
-}
-
 bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
     const uintptr_t pa = reinterpret_cast<uintptr_t>(a), pb = reinterpret_cast<uintptr_t>(b);
     return pa < pb + nb && pb < pa + na;
@@ -203,7 +162,7 @@ DRR_API drr_status drr_render(const void* vol, drr_dtype dtype, drr_layout layou
                     layout_alignment(layout, dtype));
     if (!out || !aligned(out, 4)) return fail(DRR_ERR_INVALID_ARG, "out must be a non-NULL, 4-byte aligned device pointer");
     drr::Geom g;
-    fill_geom(g, dims, spacing, origin, K, B, H, W, n_samples, density_factor, layout);
+    drr::fill_geom(g, dims, spacing, origin, K, B, H, W, n_samples, density_factor, layout);
     return cuda_status(drr::launch_forward(vol, dtype, layout, g, Rt, mode, out,
                                            static_cast<cudaStream_t>(stream)),
                        "drr_render launch");
@@ -233,7 +192,7 @@ DRR_API drr_status drr_render_adjoint(const int dims[3], const float spacing[3],
         (mode == DRR_MODE_BEER_LAMBERT && overlaps(grad_vol, vbytes, fwd_out, ibytes)))
         return fail(DRR_ERR_INVALID_ARG, "grad_vol overlaps an image buffer");
     drr::Geom g;
-    fill_geom(g, dims, spacing, origin, K, B, H, W, n_samples, density_factor, DRR_LAYOUT_LINEAR);
+    drr::fill_geom(g, dims, spacing, origin, K, B, H, W, n_samples, density_factor, DRR_LAYOUT_LINEAR);
     return cuda_status(drr::launch_adjoint(g, Rt, mode, grad_out, fwd_out, grad_vol,
                                            static_cast<cudaStream_t>(stream)),
                        "drr_render_adjoint launch");

@@ -161,7 +161,51 @@ __device__ __forceinline__ void tile_pixel(int& r, int& c) {
 }
 
 // ---------------------------------------------------------------------------
-// host-side launchers (defined in the .cu files)
+// host side
+
+// Kernel parameter block from validated host arguments.  layout: 0 linear,
+// 1 zero-bordered, 2 corner-replicated (include/drr.h).  K^-1 of the upper
+// triangular K in double.
+inline void fill_geom(Geom& g, const int dims[3], const float spacing[3], const float origin[3],
+                      const float K[9], int B, int H, int W, int n_samples, float density_factor,
+                      int layout) {
+    g = Geom{};
+    g.nx = dims[0];
+    g.ny = dims[1];
+    g.nz = dims[2];
+    if (layout == 2) {                      // strides of cells, 8 elements each
+        g.row = dims[0] - 1;
+        g.slice = (dims[0] - 1) * (dims[1] - 1);
+    } else {
+        const int pad = layout == 1 ? 2 : 0;
+        g.row = dims[0] + pad;
+        g.slice = (dims[0] + pad) * (dims[1] + pad);
+    }
+    for (int a = 0; a < 3; ++a) {
+        g.hi[a] = (float)(dims[a] - 1);
+        // largest 32.32 sample coordinate whose 8 corners are stored: cell <= n-2
+        // for the linear and corner layouts, cell <= n (inside the zero border)
+        // for the bordered one
+        const long long cells = layout == 1 ? dims[a] + 1 : dims[a] - 1;
+        g.lim[a] = cells * (1LL << 32) - 1;
+        g.spacing[a] = spacing[a];
+        g.origin[a] = origin[a];
+    }
+    const double k0 = K[0], k1 = K[1], k2 = K[2], k4 = K[4], k5 = K[5], k8 = K[8];
+    g.kinv[0] = 1.0 / k0;
+    g.kinv[1] = -k1 / (k0 * k4);
+    g.kinv[2] = (k1 * k5 - k2 * k4) / (k0 * k4 * k8);
+    g.kinv[3] = 1.0 / k4;
+    g.kinv[4] = -k5 / (k4 * k8);
+    g.kinv[5] = 1.0 / k8;
+    g.B = B;
+    g.H = H;
+    g.W = W;
+    g.N = n_samples;
+    g.density_factor = density_factor;
+}
+
+// launchers (defined in the .cu files)
 
 cudaError_t launch_forward(const void* vol, int dtype, int layout, const Geom& g,
                            const float* Rt, int mode, float* out, cudaStream_t stream);

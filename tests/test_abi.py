@@ -53,9 +53,17 @@ def test_probe_library_exports_its_declared_symbol():
     assert exported_names(PROBE_LIB) == set(names)
 
 
+def test_texture_library_exports_its_declared_symbols():
+    from cone_beam_ct_b200 import texture
+    texture.lib()
+    names = declared_names(os.path.join(ROOT, "include", "drr_texture.h"), "DRR_TEX_API")
+    assert names == sorted(texture.EXPORTED)
+    assert exported_names(texture.LIB_PATH) == set(names)
+
+
 def test_every_header_is_covered():
     headers = sorted(f for f in os.listdir(os.path.join(ROOT, "include")) if f.endswith(".h"))
-    assert headers == ["drr.h", "drr_probe.h"]
+    assert headers == ["drr.h", "drr_probe.h", "drr_texture.h"]
 
 
 def _render(**kw):
