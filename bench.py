@@ -363,6 +363,8 @@ def run_ours(args):
     out = torch.empty((w.B, w.H, w.W), dtype=torch.float32, device=dev)
     grad = torch.empty((nz, ny, nx), dtype=torch.float32, device=dev)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    ws_bytes = drr.drr_adjoint_workspace_bytes(w.dims, w.B)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
     fwd_needed = w.mode == wl.MODE_BEER_LAMBERT
 
@@ -379,9 +381,9 @@ def run_ours(args):
         grad.zero_()
         if events:
             events[3].record(stream)
-        drr.drr_render_adjoint(w.dims, w.spacing, w.origin, w.K, Rt, w.B, w.H, w.W, w.n_samples,
-                               w.density_factor, w.mode, grad_out, out if fwd_needed else None,
-                               grad, stream=stream)
+        drr.drr_render_adjoint_ws(w.dims, w.spacing, w.origin, w.K, Rt, w.B, w.H, w.W,
+                                  w.n_samples, w.density_factor, w.mode, grad_out,
+                                  out if fwd_needed else None, grad, ws, ws_bytes, stream=stream)
         if events:
             events[4].record(stream)
 
@@ -508,7 +510,7 @@ def run_ours(args):
         "cpu_baseline": base,
         "e2e": e2e,
         "texture_comparison": tex,
-        "gpu_launches": 3 * args.steps,
+        "gpu_launches": 7 * args.steps,   # prepare, forward, plan, zero, 2 adjoint paths, gather
         "clocks": clocks,
         "bracket_ms": bracket[0].elapsed_time(bracket[1]),
     }

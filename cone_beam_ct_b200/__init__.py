@@ -14,9 +14,11 @@ from .drr import (  # noqa: F401
     DRR_MODE_RAW,
     DrrError,
     drr_abi_version,
+    drr_adjoint_workspace_bytes,
     drr_get_last_error,
     drr_prepare_volume,
     drr_prepared_bytes,
     drr_render,
     drr_render_adjoint,
+    drr_render_adjoint_ws,
 )

@@ -30,6 +30,17 @@
 //    atomics share sectors.
 // Measured alternatives (shared-memory windows flushed with coalesced global
 // atomics; no pending block; no phases) were slower on every workload.
+//
+// With a workspace (drr_render_adjoint_ws), views whose rays are much closer
+// than a voxel ("dense": where a 16-pixel tile spans fewer than 8 voxels at
+// the volume centre) accumulate instead into corner records: for every cell
+// its 8 corner sums, contiguous (32 bytes, one L2 sector).  A ray keeps the
+// record of its current cell pending in registers and flushes it, when it
+// changes cell, with two 16-byte vector atomics -- the L2 executes a vector
+// atomic at the same rate as a scalar one, so this carries 4x the payload
+// per operation.  A gather pass then adds each voxel's 8 record entries into
+// the gradient volume.  Sparse views gain nothing from records (their
+// records would miss L2) and keep the direct path above.
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -81,37 +92,118 @@ __device__ __forceinline__ void slide(int d, float* __restrict__ grad, const int
     cell[AX] += d;
 }
 
-template <int MODE>
+// Is a 16-pixel tile at pixel (u0, v0) narrower than 8 voxels where its rays
+// cross the volume centre?  (NaN geometry: no.)
+__device__ __forceinline__ bool dense_tile(const View& v, const Geom& g, double u0, double v0) {
+    double c2 = 0.0, n0 = 0.0, n1 = 0.0, dot = 0.0;
+    for (int k = 0; k < 3; ++k) {
+        const double d0 = v.A[3 * k] * u0 + v.A[3 * k + 1] * v0 + v.A[3 * k + 2];
+        const double d1 = d0 + v.A[3 * k] * (double)kTileW;
+        const double off = (v.C[k] - 0.5 * g.hi[k]) * g.spacing[k];   // camera to centre, mm
+        c2 += off * off;
+        n0 += d0 * d0;
+        n1 += d1 * d1;
+        dot += d0 * d1;
+    }
+    const double ang = acos(fmin(1.0, fmax(-1.0, dot / sqrt(n0 * n1))));
+    const double min_sp = fmin(g.spacing[0], fmin(g.spacing[1], g.spacing[2]));
+    return (sqrt(c2) * ang / min_sp) < 8.0;
+}
+
+// Flush a pending corner record: two 16-byte vector atomics into one sector.
+__device__ __forceinline__ void flush_record(float* __restrict__ rec, int cell, const float a[8]) {
+    float4* p = reinterpret_cast<float4*>(rec + (size_t)cell * 8);
+    atomicAdd(p, make_float4(a[0], a[1], a[2], a[3]));
+    atomicAdd(p + 1, make_float4(a[4], a[5], a[6], a[7]));
+}
+
+// Workspace layout (drr_render_adjoint_ws): a 256-byte aligned header of
+// ints -- [0] "some view is dense", [1 + b] "view b is dense" -- then the
+// corner records, 8 floats per cell, cell = (k * (ny-1) + j) * (nx-1) + i.
+struct Workspace {
+    int* flags;        // NULL: no workspace, every view takes the direct path
+    float* rec;
+};
+
+// Which views accumulate into records: one CTA loops over the views, so
+// that flags[0] ("some view is dense") is written once, after all of them.
+__global__ void __launch_bounds__(256) plan_views(const float* __restrict__ Rt, const Geom g,
+                                                  int* __restrict__ flags) {
+    __shared__ int any;
+    if (threadIdx.x == 0) any = 0;
+    __syncthreads();
+    int mine = 0;
+    for (int b = threadIdx.x; b < g.B; b += blockDim.x) {
+        View v;
+        view_setup(Rt + 12 * (size_t)b, g, v);
+        // a view is judged by its first tile: every tile subtends nearly the
+        // same angle (the pixel pitch is constant across the detector)
+        const int dense = dense_tile(v, g, 0.0, 0.0) ? 1 : 0;
+        flags[1 + b] = dense;
+        mine |= dense;
+    }
+    if (mine) atomicOr(&any, 1);
+    __syncthreads();
+    if (threadIdx.x == 0) flags[0] = any;
+}
+
+// Zero the records when some view will use them.
+__global__ void zero_records(const int* __restrict__ flags, float4* __restrict__ rec, int64_t n4) {
+    if (flags[0] == 0) return;
+    const float4 z = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    for (int64_t m = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; m < n4;
+         m += (int64_t)gridDim.x * blockDim.x)
+        rec[m] = z;
+}
+
+// grad[k][j][i] += the 8 record entries of voxel (i, j, k): entry a + 2b + 4c of
+// cell (i - a, j - b, k - c), for the cells that exist.
+__global__ void gather_records(const int* __restrict__ flags, const float* __restrict__ rec,
+                               float* __restrict__ grad, int nx, int ny, int nz) {
+    if (flags[0] == 0) return;
+    const int64_t n = (int64_t)nx * ny * nz;
+    const int64_t cr = nx - 1, cs = (int64_t)(nx - 1) * (ny - 1);
+    for (int64_t m = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; m < n;
+         m += (int64_t)gridDim.x * blockDim.x) {
+        const int i = (int)(m % nx);
+        const int j = (int)((m / nx) % ny);
+        const int k = (int)(m / ((int64_t)nx * ny));
+        float s = 0.0f;
+#pragma unroll
+        for (int corner = 0; corner < 8; ++corner) {
+            const int ci = i - (corner & 1), cj = j - ((corner >> 1) & 1), ck = k - (corner >> 2);
+            if (ci >= 0 && cj >= 0 && ck >= 0 && ci < nx - 1 && cj < ny - 1 && ck < nz - 1)
+                s += __ldg(rec + (ck * cs + cj * cr + ci) * 8 + corner);
+        }
+        grad[m] += s;
+    }
+}
+
+// RECORDS = false: the direct path, for every view without a workspace, or
+// for the views the plan left sparse; RECORDS = true: the views the plan
+// marked dense.  Both are launched; a CTA whose view belongs to the other
+// path returns at once (a uniform exit before any barrier).
+template <int MODE, bool RECORDS>
 __global__ void __launch_bounds__(kThreads)
 adjoint_kernel(const float* __restrict__ Rt, const float* __restrict__ grad_out,
-               const float* __restrict__ fwd_out, float* __restrict__ grad, const Geom g) {
+               const float* __restrict__ fwd_out, float* __restrict__ grad, const Geom g,
+               const Workspace ws) {
     __shared__ View sv;
     __shared__ int s_dense;
     const int b = blockIdx.z;
     const int tid = threadIdx.x;
+    const bool view_dense = ws.flags != nullptr && ws.flags[1 + b] != 0;
+    if (view_dense != RECORDS) return;
     if (tid == 0) {
         view_setup(Rt + 12 * (size_t)b, g, sv);
-        // tile width in voxels where its rays cross the volume centre
-        const double u0 = blockIdx.x * kTileW, v0 = blockIdx.y * kTileH;
-        double c2 = 0.0, n0 = 0.0, n1 = 0.0, dot = 0.0;
-        for (int k = 0; k < 3; ++k) {
-            const double d0 = sv.A[3 * k] * u0 + sv.A[3 * k + 1] * v0 + sv.A[3 * k + 2];
-            const double d1 = d0 + sv.A[3 * k] * (double)kTileW;
-            const double off = (sv.C[k] - 0.5 * g.hi[k]) * g.spacing[k];   // camera to centre, mm
-            c2 += off * off;
-            n0 += d0 * d0;
-            n1 += d1 * d1;
-            dot += d0 * d1;
-        }
-        const double ang = acos(fmin(1.0, fmax(-1.0, dot / sqrt(n0 * n1))));
-        const double min_sp = fmin(g.spacing[0], fmin(g.spacing[1], g.spacing[2]));
-        s_dense = (sqrt(c2) * ang / min_sp) < 8.0 ? 1 : 0;   // NaN geometry: not dense
+        s_dense = dense_tile(sv, g, blockIdx.x * kTileW, blockIdx.y * kTileH) ? 1 : 0;
     }
     __syncthreads();
+    constexpr bool records = RECORDS;
 
     int r, c;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    if (s_dense) {
+    if (s_dense || records) {
         // spread: the 32 lanes of a warp cover the whole 16 x 16 tile (bijective)
         c = blockIdx.x * kTileW + (lane & 7) * 2 + (warp & 1);
         r = blockIdx.y * kTileH + (lane >> 3) * 4 + (warp >> 1);
@@ -130,6 +222,44 @@ adjoint_kernel(const float* __restrict__ Rt, const float* __restrict__ grad_out,
     // phase: this warp starts at sample `start` and wraps round to 0
     const int ph = (warp + blockIdx.x * 3 + blockIdx.y * 5 + blockIdx.z) & 7;
     const int start = (int)(((long long)g.N * ph) >> 3);
+
+    if constexpr (records) {
+        // cells stay in [0, n-2] per axis (linear-layout lim), inside the records
+        const int cr = g.nx - 1, cs = (g.nx - 1) * (g.ny - 1);
+        float p[8];
+        for (int pass = 0; pass < 2; ++pass) {
+            const int i0 = pass == 0 ? start : 0;
+            const int i1 = pass == 0 ? g.N : start;
+            if (i0 >= i1) continue;
+            long long qx = ray.q0[0] + (long long)i0 * ray.s[0];
+            long long qy = ray.q0[1] + (long long)i0 * ray.s[1];
+            long long qz = ray.q0[2] + (long long)i0 * ray.s[2];
+            int pc = -1;
+            for (int i = i0; i < i1; ++i) {
+                const int rc = fix_cell(qz) * cs + fix_cell(qy) * cr + fix_cell(qx);
+                const float fx = fix_frac(qx), fy = fix_frac(qy), fz = fix_frac(qz);
+                qx += ray.s[0];
+                qy += ray.s[1];
+                qz += ray.s[2];
+                const float wz1 = scale * fz, wz0 = scale * (1.0f - fz);
+                const float w00 = wz0 * (1.0f - fy), w01 = wz0 * fy;
+                const float w10 = wz1 * (1.0f - fy), w11 = wz1 * fy;
+                const float gx = 1.0f - fx;
+                const float w[8] = {w00 * gx, w00 * fx, w01 * gx, w01 * fx,
+                                    w10 * gx, w10 * fx, w11 * gx, w11 * fx};
+                if (rc != pc) {
+                    if (pc >= 0) flush_record(ws.rec, pc, p);
+                    pc = rc;
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) p[k] = w[k];
+                } else {
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) p[k] += w[k];
+                }
+            }
+            flush_record(ws.rec, pc, p);
+        }
+    } else {
     int cell[3];
     float a[8];
     for (int pass = 0; pass < 2; ++pass) {
@@ -179,17 +309,46 @@ adjoint_kernel(const float* __restrict__ Rt, const float* __restrict__ grad_out,
         }
         flush_block(grad, st, cell, a);
     }
+    }   // direct path
 }
 
 }  // namespace
 
+size_t adjoint_workspace_header(int B) {
+    return ((size_t)(1 + B) * sizeof(int) + 255) / 256 * 256;
+}
+
+size_t adjoint_workspace_bytes(int nx, int ny, int nz, int B) {
+    return adjoint_workspace_header(B) + (size_t)(nx - 1) * (ny - 1) * (nz - 1) * 8 * sizeof(float);
+}
+
 cudaError_t launch_adjoint(const Geom& g, const float* Rt, int mode, const float* grad_out,
-                           const float* fwd_out, float* grad_vol, cudaStream_t stream) {
+                           const float* fwd_out, float* grad_vol, void* workspace,
+                           cudaStream_t stream) {
     const dim3 grid((g.W + kTileW - 1) / kTileW, (g.H + kTileH - 1) / kTileH, g.B);
+    Workspace ws{nullptr, nullptr};
+    const int64_t n_rec4 = (int64_t)(g.nx - 1) * (g.ny - 1) * (g.nz - 1) * 2;   // float4 per record: 2
+    const int fill_grid = 148 * 8;
+    if (workspace) {
+        ws.flags = static_cast<int*>(workspace);
+        ws.rec = reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                          adjoint_workspace_header(g.B));
+        plan_views<<<1, 256, 0, stream>>>(Rt, g, ws.flags);
+        zero_records<<<fill_grid, 256, 0, stream>>>(ws.flags, reinterpret_cast<float4*>(ws.rec),
+                                                    n_rec4);
+    }
     if (mode == 1)
-        adjoint_kernel<1><<<grid, kThreads, 0, stream>>>(Rt, grad_out, fwd_out, grad_vol, g);
+        adjoint_kernel<1, false><<<grid, kThreads, 0, stream>>>(Rt, grad_out, fwd_out, grad_vol, g, ws);
     else
-        adjoint_kernel<0><<<grid, kThreads, 0, stream>>>(Rt, grad_out, fwd_out, grad_vol, g);
+        adjoint_kernel<0, false><<<grid, kThreads, 0, stream>>>(Rt, grad_out, fwd_out, grad_vol, g, ws);
+    if (workspace) {
+        if (mode == 1)
+            adjoint_kernel<1, true><<<grid, kThreads, 0, stream>>>(Rt, grad_out, fwd_out, grad_vol, g, ws);
+        else
+            adjoint_kernel<0, true><<<grid, kThreads, 0, stream>>>(Rt, grad_out, fwd_out, grad_vol, g, ws);
+    }
+    if (workspace)
+        gather_records<<<fill_grid, 256, 0, stream>>>(ws.flags, ws.rec, grad_vol, g.nx, g.ny, g.nz);
     return cudaGetLastError();
 }
 

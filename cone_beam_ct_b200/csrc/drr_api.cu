@@ -168,11 +168,15 @@ DRR_API drr_status drr_render(const void* vol, drr_dtype dtype, drr_layout layou
                        "drr_render launch");
 }
 
-DRR_API drr_status drr_render_adjoint(const int dims[3], const float spacing[3],
-                                      const float origin[3], const float K[9], const float* Rt,
-                                      int B, int H, int W, int n_samples, float density_factor,
-                                      drr_mode mode, const float* grad_out, const float* fwd_out,
-                                      float* grad_vol, void* stream) {
+}  // extern "C"
+
+namespace {
+
+drr_status render_adjoint(const int dims[3], const float spacing[3], const float origin[3],
+                          const float K[9], const float* Rt, int B, int H, int W, int n_samples,
+                          float density_factor, int mode, const float* grad_out,
+                          const float* fwd_out, float* grad_vol, bool with_ws, void* workspace,
+                          size_t workspace_bytes, void* stream) {
     drr_status st = check_volume(dims, spacing, origin);
     if (st != DRR_OK) return st;
     st = check_rays(K, Rt, B, H, W, n_samples, density_factor, mode);
@@ -191,11 +195,54 @@ DRR_API drr_status drr_render_adjoint(const int dims[3], const float spacing[3],
     if (overlaps(grad_vol, vbytes, grad_out, ibytes) ||
         (mode == DRR_MODE_BEER_LAMBERT && overlaps(grad_vol, vbytes, fwd_out, ibytes)))
         return fail(DRR_ERR_INVALID_ARG, "grad_vol overlaps an image buffer");
+    if (with_ws) {
+        const size_t need = drr::adjoint_workspace_bytes(dims[0], dims[1], dims[2], B);
+        if (!workspace || !aligned(workspace, 256))
+            return fail(DRR_ERR_INVALID_ARG, "workspace must be a non-NULL, 256-byte aligned device pointer");
+        if (workspace_bytes < need)
+            return fail(DRR_ERR_INVALID_ARG, "workspace holds %zu bytes, %zu needed", workspace_bytes, need);
+        if (overlaps(workspace, need, grad_vol, vbytes) || overlaps(workspace, need, grad_out, ibytes) ||
+            (mode == DRR_MODE_BEER_LAMBERT && overlaps(workspace, need, fwd_out, ibytes)) ||
+            overlaps(workspace, need, Rt, (size_t)B * 12 * sizeof(float)))
+            return fail(DRR_ERR_INVALID_ARG, "workspace overlaps another buffer");
+    }
     drr::Geom g;
     drr::fill_geom(g, dims, spacing, origin, K, B, H, W, n_samples, density_factor, DRR_LAYOUT_LINEAR);
     return cuda_status(drr::launch_adjoint(g, Rt, mode, grad_out, fwd_out, grad_vol,
+                                           with_ws ? workspace : nullptr,
                                            static_cast<cudaStream_t>(stream)),
                        "drr_render_adjoint launch");
+}
+
+}  // namespace
+
+extern "C" {
+
+DRR_API drr_status drr_render_adjoint(const int dims[3], const float spacing[3],
+                                      const float origin[3], const float K[9], const float* Rt,
+                                      int B, int H, int W, int n_samples, float density_factor,
+                                      drr_mode mode, const float* grad_out, const float* fwd_out,
+                                      float* grad_vol, void* stream) {
+    return render_adjoint(dims, spacing, origin, K, Rt, B, H, W, n_samples, density_factor, mode,
+                          grad_out, fwd_out, grad_vol, false, nullptr, 0, stream);
+}
+
+DRR_API size_t drr_adjoint_workspace_bytes(const int dims[3], int B) {
+    if (!dims || B < 0 || B > kMaxViews) return 0;
+    for (int a = 0; a < 3; ++a)
+        if (dims[a] < 2 || dims[a] > kMaxDim) return 0;
+    if (stored_elements(dims, DRR_LAYOUT_LINEAR) > kMaxElements) return 0;
+    return drr::adjoint_workspace_bytes(dims[0], dims[1], dims[2], B);
+}
+
+DRR_API drr_status drr_render_adjoint_ws(const int dims[3], const float spacing[3],
+                                         const float origin[3], const float K[9], const float* Rt,
+                                         int B, int H, int W, int n_samples, float density_factor,
+                                         drr_mode mode, const float* grad_out, const float* fwd_out,
+                                         float* grad_vol, void* workspace, size_t workspace_bytes,
+                                         void* stream) {
+    return render_adjoint(dims, spacing, origin, K, Rt, B, H, W, n_samples, density_factor, mode,
+                          grad_out, fwd_out, grad_vol, true, workspace, workspace_bytes, stream);
 }
 
 }  // extern "C"

@@ -210,7 +210,9 @@ inline void fill_geom(Geom& g, const int dims[3], const float spacing[3], const 
 cudaError_t launch_forward(const void* vol, int dtype, int layout, const Geom& g,
                            const float* Rt, int mode, float* out, cudaStream_t stream);
 cudaError_t launch_adjoint(const Geom& g, const float* Rt, int mode, const float* grad_out,
-                           const float* fwd_out, float* grad_vol, cudaStream_t stream);
+                           const float* fwd_out, float* grad_vol, void* workspace,
+                           cudaStream_t stream);
+size_t adjoint_workspace_bytes(int nx, int ny, int nz, int B);
 cudaError_t launch_prepare(const float* src, int nx, int ny, int nz, int dtype, int layout,
                            void* dst, cudaStream_t stream);
 

@@ -20,7 +20,8 @@ DRR_F32, DRR_BF16 = 0, 1
 DRR_LAYOUT_LINEAR, DRR_LAYOUT_PADDED, DRR_LAYOUT_CORNERS = 0, 1, 2
 
 # names exported by libdrr.so (include/drr.h)
-EXPORTED = ("drr_render", "drr_render_adjoint", "drr_prepared_bytes", "drr_prepare_volume",
+EXPORTED = ("drr_render", "drr_render_adjoint", "drr_render_adjoint_ws",
+            "drr_adjoint_workspace_bytes", "drr_prepared_bytes", "drr_prepare_volume",
             "drr_get_last_error", "drr_abi_version")
 
 
@@ -53,6 +54,12 @@ def lib():
     L.drr_render_adjoint.argtypes = [_i3, _f3, _f3, _f9, _vp, _c.c_int, _c.c_int, _c.c_int,
                                      _c.c_int, _c.c_float, _c.c_int, _vp, _vp, _vp, _vp]
     L.drr_render_adjoint.restype = _c.c_int
+    L.drr_render_adjoint_ws.argtypes = [_i3, _f3, _f3, _f9, _vp, _c.c_int, _c.c_int, _c.c_int,
+                                        _c.c_int, _c.c_float, _c.c_int, _vp, _vp, _vp, _vp,
+                                        _c.c_size_t, _vp]
+    L.drr_render_adjoint_ws.restype = _c.c_int
+    L.drr_adjoint_workspace_bytes.argtypes = [_i3, _c.c_int]
+    L.drr_adjoint_workspace_bytes.restype = _c.c_size_t
     L.drr_prepared_bytes.argtypes = [_i3, _c.c_int, _c.c_int]
     L.drr_prepared_bytes.restype = _c.c_size_t
     L.drr_prepare_volume.argtypes = [_vp, _i3, _c.c_int, _c.c_int, _vp, _c.c_size_t, _vp]
@@ -150,3 +157,22 @@ def drr_render_adjoint(dims, spacing, origin, K, Rt, B, H, W, n_samples, density
                                     _dev(grad_out, "grad_out", True),
                                     _dev(fwd_out, "fwd_out", True),
                                     _dev(grad_vol, "grad_vol", True), _stream(stream)))
+
+
+def drr_adjoint_workspace_bytes(dims, B):
+    return int(lib().drr_adjoint_workspace_bytes(_i3v(dims), int(B)))
+
+
+def drr_render_adjoint_ws(dims, spacing, origin, K, Rt, B, H, W, n_samples, density_factor, mode,
+                          grad_out, fwd_out, grad_vol, workspace, workspace_bytes=None,
+                          stream=None):
+    if workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    _check(lib().drr_render_adjoint_ws(_i3v(dims), _f3v(spacing), _f3v(origin), _f9v(K),
+                                       _dev(Rt, "Rt", True), int(B), int(H), int(W),
+                                       int(n_samples), float(density_factor), int(mode),
+                                       _dev(grad_out, "grad_out", True),
+                                       _dev(fwd_out, "fwd_out", True),
+                                       _dev(grad_vol, "grad_vol", True),
+                                       _dev(workspace, "workspace", True), int(workspace_bytes),
+                                       _stream(stream)))

@@ -145,6 +145,33 @@ DRR_API drr_status drr_render_adjoint(const int dims[3], const float spacing[3],
                                       drr_mode mode, const float *grad_out, const float *fwd_out,
                                       float *grad_vol, void *stream);
 
+/* Bytes of the workspace drr_render_adjoint_ws needs for a volume of dims
+ * and B views (0 if the arguments are invalid): a 256-byte header of view
+ * flags plus one 32-byte corner record per cell, (nx-1)(ny-1)(nz-1) of them
+ * (about 8x the fp32 volume). */
+DRR_API size_t drr_adjoint_workspace_bytes(const int dims[3], int B);
+
+/* drr_render_adjoint with a caller-provided workspace, for speed: views
+ * whose rays are much closer than a voxel (a 16-pixel tile spanning fewer
+ * than 8 voxels at the volume centre) accumulate into per-cell corner
+ * records with 16-byte vector atomics, which a final pass adds into
+ * grad_vol; other views scatter into grad_vol directly, as in
+ * drr_render_adjoint.  Same result up to fp32 summation order.
+ *   workspace        DEVICE, 256-byte aligned, at least
+ *                    drr_adjoint_workspace_bytes(dims, B) bytes; its content
+ *                    on entry is ignored and on return is unspecified; must
+ *                    not overlap any other buffer of the call.
+ *   workspace_bytes  bytes available at workspace.
+ * Calls that share one workspace must not overlap on the GPU (same stream,
+ * or ordered by events).  Other arguments as drr_render_adjoint. */
+DRR_API drr_status drr_render_adjoint_ws(const int dims[3], const float spacing[3],
+                                         const float origin[3], const float K[9],
+                                         const float *Rt, int B, int H, int W, int n_samples,
+                                         float density_factor, drr_mode mode,
+                                         const float *grad_out, const float *fwd_out,
+                                         float *grad_vol, void *workspace,
+                                         size_t workspace_bytes, void *stream);
+
 /* Bytes that drr_prepare_volume writes for this volume, dtype and layout
  * (0 if the arguments are invalid or the volume is too large). */
 DRR_API size_t drr_prepared_bytes(const int dims[3], drr_dtype dtype, drr_layout layout);

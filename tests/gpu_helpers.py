@@ -44,7 +44,10 @@ def gpu_forward(w, layout=PADDED, dtype=None, mode=None, vol=None, Rt=None):
     return out.cpu().numpy()
 
 
-def gpu_adjoint(w, grad_out, mode=None, fwd_out=None):
+def gpu_adjoint(w, grad_out, mode=None, fwd_out=None, workspace=False):
+    """Volume gradient through drr_render_adjoint, or drr_render_adjoint_ws
+    with a fresh workspace (filled with garbage first: its content on entry
+    must not matter)."""
     import torch
     mode = w.mode if mode is None else mode
     _, Rt_d = device_inputs(w, vol=np.zeros((1,), np.float32))
@@ -54,8 +57,14 @@ def gpu_adjoint(w, grad_out, mode=None, fwd_out=None):
         fo = torch.from_numpy(np.ascontiguousarray(fwd_out, dtype=np.float32)).cuda()
     nx, ny, nz = w.dims
     grad = torch.zeros((nz, ny, nx), dtype=torch.float32, device="cuda")
-    drr.drr_render_adjoint(w.dims, w.spacing, w.origin, w.K, Rt_d, w.B, w.H, w.W, w.n_samples,
-                           w.density_factor, mode, go, fo, grad)
+    if workspace:
+        nbytes = drr.drr_adjoint_workspace_bytes(w.dims, w.B)
+        ws = torch.full((nbytes,), 0x7F, dtype=torch.uint8, device="cuda")
+        drr.drr_render_adjoint_ws(w.dims, w.spacing, w.origin, w.K, Rt_d, w.B, w.H, w.W,
+                                  w.n_samples, w.density_factor, mode, go, fo, grad, ws)
+    else:
+        drr.drr_render_adjoint(w.dims, w.spacing, w.origin, w.K, Rt_d, w.B, w.H, w.W,
+                               w.n_samples, w.density_factor, mode, go, fo, grad)
     torch.cuda.synchronize()
     return grad.cpu().numpy()
 

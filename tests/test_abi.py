@@ -139,6 +139,45 @@ def test_adjoint_rejects_bad_arguments(kw, status):
     assert e.value.status == status
 
 
+WS = FAKE + (1 << 30)
+WS_BYTES = 1 << 28
+
+
+def _adjoint_ws(**kw):
+    args = dict(dims=DIMS, spacing=SP, origin=ORG, K=K_OK, Rt=FAKE, B=2, H=8, W=8,
+                n_samples=16, density_factor=1.0, mode=drr.DRR_MODE_RAW,
+                grad_out=FAKE + (1 << 20), fwd_out=None, grad_vol=FAKE + (1 << 24),
+                workspace=WS, workspace_bytes=WS_BYTES, stream=0)
+    args.update(kw)
+    return drr.drr_render_adjoint_ws(**args)
+
+
+WS_BAD = [
+    (dict(workspace=0), "workspace"),
+    (dict(workspace=WS + 16), "aligned"),
+    (dict(workspace_bytes=100), "needed"),
+    (dict(workspace=FAKE + (1 << 24)), "overlaps"),          # on grad_vol
+    (dict(n_samples=0), "n_samples"),
+]
+
+
+@pytest.mark.parametrize("kw,word", WS_BAD)
+def test_workspace_adjoint_rejects_bad_arguments(kw, word):
+    with pytest.raises(drr.DrrError) as e:
+        _adjoint_ws(**kw)
+    assert e.value.status == drr.DRR_ERR_INVALID_ARG
+    assert word in drr.drr_get_last_error()
+
+
+def test_workspace_bytes():
+    # 256-byte header of view flags, then 32 bytes per cell
+    assert drr.drr_adjoint_workspace_bytes((16, 16, 16), 2) == 256 + 15 ** 3 * 32
+    assert drr.drr_adjoint_workspace_bytes((256, 256, 256), 64) == 512 + 255 ** 3 * 32
+    assert drr.drr_adjoint_workspace_bytes((1, 16, 16), 2) == 0
+    assert drr.drr_adjoint_workspace_bytes((16, 16, 16), -1) == 0
+    _adjoint_ws(B=0, workspace=None, grad_out=None, grad_vol=None, Rt=None)   # empty: no-op
+
+
 def test_raw_adjoint_does_not_need_the_forward_image():
     # fwd_out may be NULL in RAW mode: only an empty batch keeps this off the device
     _adjoint(fwd_out=None, B=0)

@@ -45,17 +45,48 @@ def _oracle_adjoint(w, go, mode, nthreads=8):
 
 @pytest.mark.parametrize("seed", [201, 202, 203])
 @pytest.mark.parametrize("mode", [wl.MODE_RAW, wl.MODE_BEER_LAMBERT])
-def test_small_ragged_adjoint(cuda, seed, mode):
+@pytest.mark.parametrize("workspace", [False, True])
+def test_small_ragged_adjoint(cuda, seed, mode, workspace):
     w = wl.small_random_case(seed)
     go = np.random.default_rng(seed).standard_normal((w.B, w.H, w.W)).astype(np.float32)
     fwd = gpu_forward(w, layout=PADDED, dtype=F32, mode=mode) if mode else None
-    got = gpu_adjoint(w, go, mode=mode, fwd_out=fwd)
+    got = gpu_adjoint(w, go, mode=mode, fwd_out=fwd, workspace=workspace)
     assert_adjoint_parity(got, _oracle_adjoint(w, go, mode), what=f"seed {seed} mode {mode}")
 
 
-def _dot_residual(w, x, y, layout):
+# rays much closer than a voxel (a 16-pixel tile spans ~2.5 voxels): these
+# views take the corner-record path of drr_render_adjoint_ws
+DENSE = dict(dims=(23, 17, 29), H=150, W=170, n_samples=40)
+
+
+@pytest.mark.parametrize("seed", [211, 212])
+@pytest.mark.parametrize("mode", [wl.MODE_RAW, wl.MODE_BEER_LAMBERT])
+def test_dense_views_take_the_record_path(cuda, seed, mode):
+    w = wl.small_random_case(seed, **DENSE)
+    go = np.random.default_rng(seed).standard_normal((w.B, w.H, w.W)).astype(np.float32)
+    fwd = gpu_forward(w, layout=PADDED, dtype=F32, mode=mode) if mode else None
+    ref = _oracle_adjoint(w, go, mode)
+    for workspace in (False, True):
+        got = gpu_adjoint(w, go, mode=mode, fwd_out=fwd, workspace=workspace)
+        assert_adjoint_parity(got, ref, what=f"dense seed {seed} workspace {workspace}")
+
+
+def test_record_path_dot_product_identity(cuda):
+    w = wl.small_random_case(213, **DENSE)
+    rng = np.random.default_rng(7)
+    nx, ny, nz = w.dims
+    x = rng.uniform(0, 1, (nz, ny, nx)).astype(np.float32)
+    y = rng.standard_normal((w.B, w.H, w.W)).astype(np.float32)
+    Ax = gpu_forward(w, layout=LINEAR, dtype=F32, mode=wl.MODE_RAW, vol=x).astype(np.float64)
+    ATy = gpu_adjoint(w, y, mode=wl.MODE_RAW, workspace=True).astype(np.float64)
+    lhs = float(np.dot(Ax.reshape(-1), y.reshape(-1).astype(np.float64)))
+    rhs = float(np.dot(x.reshape(-1).astype(np.float64), ATy.reshape(-1)))
+    assert abs(lhs - rhs) / (np.linalg.norm(Ax) * np.linalg.norm(y.astype(np.float64))) <= TOL_DOT
+
+
+def _dot_residual(w, x, y, layout, workspace=False):
     Ax = gpu_forward(w, layout=layout, dtype=F32, mode=wl.MODE_RAW, vol=x).astype(np.float64)
-    ATy = gpu_adjoint(w, y, mode=wl.MODE_RAW).astype(np.float64)
+    ATy = gpu_adjoint(w, y, mode=wl.MODE_RAW, workspace=workspace).astype(np.float64)
     lhs = float(np.dot(Ax.reshape(-1), y.reshape(-1).astype(np.float64)))
     rhs = float(np.dot(x.reshape(-1).astype(np.float64), ATy.reshape(-1)))
     return abs(lhs - rhs) / (np.linalg.norm(Ax) * np.linalg.norm(y.astype(np.float64)))
@@ -90,9 +121,10 @@ def test_adjoint_accumulates_and_skips_zero_gradient(cuda):
 @pytest.mark.slow
 def test_config5_full_adjoint_and_dot_product(cuda):
     w = wl.make_config(5)
-    got = gpu_adjoint(w, w.grad_out, mode=w.mode)
     ref = _oracle_adjoint(w, w.grad_out, w.mode, nthreads=16)
-    assert_adjoint_parity(got, ref, what="config 5")
+    for workspace in (False, True):
+        got = gpu_adjoint(w, w.grad_out, mode=w.mode, workspace=workspace)
+        assert_adjoint_parity(got, ref, what=f"config 5 workspace {workspace}")
     rng = np.random.default_rng(55)
     nx, ny, nz = w.dims
     x = rng.uniform(0, 1, (nz, ny, nx)).astype(np.float32)
@@ -110,9 +142,11 @@ def test_config3_geometry_adjoint(cuda):
     x = rng.uniform(0, 1, (nz, ny, nx)).astype(np.float32)
     y = rng.standard_normal((w.B, w.H, w.W)).astype(np.float32)
     assert _dot_residual(w, x, y, PADDED) <= TOL_DOT
+    assert _dot_residual(w, x, y, PADDED, workspace=True) <= TOL_DOT
     sparse = np.zeros((w.B, w.H, w.W), np.float32)
     ids = rng.choice(w.rays, size=2000, replace=False)
     sparse.reshape(-1)[ids] = rng.standard_normal(2000).astype(np.float32)
-    got = gpu_adjoint(w, sparse, mode=wl.MODE_RAW)
     ref = _oracle_adjoint(w, sparse, wl.MODE_RAW)
-    assert_adjoint_parity(got, ref, what="config 3 sparse")
+    for workspace in (False, True):
+        got = gpu_adjoint(w, sparse, mode=wl.MODE_RAW, workspace=workspace)
+        assert_adjoint_parity(got, ref, what=f"config 3 sparse upstream, workspace {workspace}")
