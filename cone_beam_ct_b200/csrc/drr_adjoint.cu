@@ -44,9 +44,19 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "drr_internal.cuh"
 
 namespace drr {
+
+// Built-in scratch of drr_render_adjoint_noalloc, for callers that may not
+// allocate device memory.  It is part of the library's device image: every
+// GPU that loads the library holds these bytes until the process exits.
+// Host code must not use this name as an address (on the host it is only a
+// stand-in); noalloc_scratch() below fetches the device address.
+static __device__ __align__(256) unsigned char noalloc_scratch_bytes[kNoAllocScratchBytes];
+
 namespace {
 
 // 8 corner sums of a pending block at cell (x, y, z); a[k] belongs to corner
@@ -312,6 +322,29 @@ adjoint_kernel(const float* __restrict__ Rt, const float* __restrict__ grad_out,
     }   // direct path
 }
 
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[kMaxDevices] = {};
+
+// Device address of the built-in scratch on the current device, looked up
+// once per device (the first call on a device does it; that call should
+// come before any stream capture).
+cudaError_t noalloc_scratch(void** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_addr[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, noalloc_scratch_bytes);
+        if (e != cudaSuccess) return e;
+        g_noalloc_addr[dev] = p;
+    }
+    *out = g_noalloc_addr[dev];
+    return cudaSuccess;
+}
+
 }  // namespace
 
 size_t adjoint_workspace_header(int B) {
@@ -350,6 +383,14 @@ cudaError_t launch_adjoint(const Geom& g, const float* Rt, int mode, const float
     if (workspace)
         gather_records<<<fill_grid, 256, 0, stream>>>(ws.flags, ws.rec, grad_vol, g.nx, g.ny, g.nz);
     return cudaGetLastError();
+}
+
+cudaError_t launch_adjoint_noalloc(const Geom& g, const float* Rt, int mode, const float* grad_out,
+                                   const float* fwd_out, float* grad_vol, cudaStream_t stream) {
+    void* scratch = nullptr;
+    const cudaError_t e = noalloc_scratch(&scratch);
+    if (e != cudaSuccess) return e;
+    return launch_adjoint(g, Rt, mode, grad_out, fwd_out, grad_vol, scratch, stream);
 }
 
 }  // namespace drr

@@ -245,4 +245,44 @@ DRR_API drr_status drr_render_adjoint_ws(const int dims[3], const float spacing[
                           grad_out, fwd_out, grad_vol, true, workspace, workspace_bytes, stream);
 }
 
+// Adjoint for callers that may not allocate device memory (see include/drr.h):
+// the workspace of drr_render_adjoint_ws comes from the library's built-in
+// scratch instead of the caller.  No allocation happens here or below.
+DRR_API drr_status drr_render_adjoint_noalloc(const int dims[3], const float spacing[3],
+                                              const float origin[3], const float K[9],
+                                              const float* Rt, int B, int H, int W,
+                                              int n_samples, float density_factor, drr_mode mode,
+                                              const float* grad_out, const float* fwd_out,
+                                              float* grad_vol, void* stream) {
+    drr_status st = check_volume(dims, spacing, origin);
+    if (st != DRR_OK) return st;
+    st = check_rays(K, Rt, B, H, W, n_samples, density_factor, mode);
+    if (st != DRR_OK) return st;
+    if (stored_elements(dims, DRR_LAYOUT_LINEAR) > kMaxElements)
+        return fail(DRR_ERR_UNSUPPORTED, "volume too large (max 2^31 - 1 elements)");
+    const size_t need = drr::adjoint_workspace_bytes(dims[0], dims[1], dims[2], B);
+    if (need > drr::kNoAllocScratchBytes)
+        return fail(DRR_ERR_UNSUPPORTED,
+                    "this volume and view count need %zu bytes of scratch; the built-in scratch "
+                    "holds %zu (use drr_render_adjoint_ws with a workspace of your own)",
+                    need, drr::kNoAllocScratchBytes);
+    const int64_t npix = (int64_t)B * H * W;
+    if (npix == 0) return ok();
+    if (!grad_out || !aligned(grad_out, 4))
+        return fail(DRR_ERR_INVALID_ARG, "grad_out must be a non-NULL, 4-byte aligned device pointer");
+    if (mode == DRR_MODE_BEER_LAMBERT && (!fwd_out || !aligned(fwd_out, 4)))
+        return fail(DRR_ERR_INVALID_ARG, "fwd_out is required in Beer-Lambert mode");
+    if (!grad_vol || !aligned(grad_vol, 4))
+        return fail(DRR_ERR_INVALID_ARG, "grad_vol must be a non-NULL, 4-byte aligned device pointer");
+    const size_t vbytes = (size_t)dims[0] * dims[1] * dims[2] * 4, ibytes = (size_t)npix * 4;
+    if (overlaps(grad_vol, vbytes, grad_out, ibytes) ||
+        (mode == DRR_MODE_BEER_LAMBERT && overlaps(grad_vol, vbytes, fwd_out, ibytes)))
+        return fail(DRR_ERR_INVALID_ARG, "grad_vol overlaps an image buffer");
+    drr::Geom g;
+    drr::fill_geom(g, dims, spacing, origin, K, B, H, W, n_samples, density_factor, DRR_LAYOUT_LINEAR);
+    return cuda_status(drr::launch_adjoint_noalloc(g, Rt, mode, grad_out, fwd_out, grad_vol,
+                                                   static_cast<cudaStream_t>(stream)),
+                       "drr_render_adjoint_noalloc");
+}
+
 }  // extern "C"

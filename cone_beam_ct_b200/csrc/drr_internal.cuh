@@ -213,6 +213,11 @@ cudaError_t launch_adjoint(const Geom& g, const float* Rt, int mode, const float
                            const float* fwd_out, float* grad_vol, void* workspace,
                            cudaStream_t stream);
 size_t adjoint_workspace_bytes(int nx, int ny, int nz, int B);
+
+// Size of the built-in scratch of the allocation-free adjoint (32 MiB).
+constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;
+cudaError_t launch_adjoint_noalloc(const Geom& g, const float* Rt, int mode, const float* grad_out,
+                                   const float* fwd_out, float* grad_vol, cudaStream_t stream);
 cudaError_t launch_prepare(const float* src, int nx, int ny, int nz, int dtype, int layout,
                            void* dst, cudaStream_t stream);
 

@@ -172,6 +172,40 @@ DRR_API drr_status drr_render_adjoint_ws(const int dims[3], const float spacing[
                                          float *grad_vol, void *workspace,
                                          size_t workspace_bytes, void *stream);
 
+/* Size of the scratch built into the library for drr_render_adjoint_noalloc. */
+#define DRR_NOALLOC_SCRATCH_BYTES (32u << 20)
+
+/* drr_render_adjoint_ws without a caller-provided workspace, for callers
+ * that may not allocate device memory: code running under a memory manager
+ * that owns all of the device's memory (a framework's caching allocator, a
+ * server with fixed per-model budgets), or a real-time loop in which an
+ * allocation, which can synchronise the device, is not allowed.  The pages
+ * this library follows have no counterpart of this call; it exists only for
+ * such callers.
+ *   - The workspace is a scratch array built into the library's device
+ *     image, DRR_NOALLOC_SCRATCH_BYTES (32 MiB) in size.  Every GPU that
+ *     loads the library holds it until the process exits.
+ *   - Volumes and view counts whose workspace
+ *     (drr_adjoint_workspace_bytes(dims, B)) exceeds that size are rejected
+ *     with DRR_ERR_UNSUPPORTED before anything runs (about 100^3 voxels at
+ *     most); use drr_render_adjoint_ws for larger ones.
+ *   - Nothing is allocated: no cudaMalloc, cudaFree or allocating library
+ *     call.  The first call on a device looks up the scratch's device
+ *     address (once per device, with that device current); make that first
+ *     call before any stream capture.
+ *   - All calls share the one scratch array, which keeps the last call's
+ *     contents; each call re-initialises what it reads.  Calls that overlap
+ *     on the GPU (different streams without ordering, or several host
+ *     threads) race on it: serialise them.
+ * Arguments and result as drr_render_adjoint. */
+DRR_API drr_status drr_render_adjoint_noalloc(const int dims[3], const float spacing[3],
+                                              const float origin[3], const float K[9],
+                                              const float *Rt, int B, int H, int W,
+                                              int n_samples, float density_factor,
+                                              drr_mode mode, const float *grad_out,
+                                              const float *fwd_out, float *grad_vol,
+                                              void *stream);
+
 /* Bytes that drr_prepare_volume writes for this volume, dtype and layout
  * (0 if the arguments are invalid or the volume is too large). */
 DRR_API size_t drr_prepared_bytes(const int dims[3], drr_dtype dtype, drr_layout layout);

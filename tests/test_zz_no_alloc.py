@@ -1,0 +1,88 @@
+"""The allocation-free adjoint (drr_render_adjoint_noalloc), for callers that
+may not allocate device memory -- code under a memory manager that owns the
+whole device, or a real-time loop where an allocation could synchronise the
+device.  Its workspace is the library's built-in 32 MiB scratch, shared by
+every call.  It must match the ordinary adjoint (same tolerance as the
+other adjoint tests), call after call: the scratch keeps the previous call's
+contents, so a second call shows that each call re-initialises what it
+reads.  This file is collected last so that a failure here leaves every
+other test already run; it also passes on its own in a fresh process."""
+import numpy as np
+import pytest
+
+from cone_beam_ct_b200 import workloads as wl
+
+pytestmark = pytest.mark.gpu
+TOL_ADJ = 1e-4
+
+
+@pytest.fixture(scope="module")
+def cuda():
+    torch = pytest.importorskip("torch")
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    from cone_beam_ct_b200 import drr
+    drr.lib()
+    return torch
+
+
+def _inputs(torch, w, seed):
+    go = np.random.default_rng(seed).standard_normal((w.B, w.H, w.W)).astype(np.float32)
+    return (torch.from_numpy(np.ascontiguousarray(w.Rt.reshape(-1, 12))).cuda(),
+            torch.from_numpy(go).cuda())
+
+
+def _adjoint(torch, w, Rt, go, noalloc):
+    from cone_beam_ct_b200 import drr
+    nx, ny, nz = w.dims
+    grad = torch.zeros((nz, ny, nx), dtype=torch.float32, device="cuda")
+    fn = drr.drr_render_adjoint_noalloc if noalloc else drr.drr_render_adjoint
+    fn(w.dims, w.spacing, w.origin, w.K, Rt, w.B, w.H, w.W, w.n_samples, w.density_factor,
+       wl.MODE_RAW, go, None, grad)
+    torch.cuda.synchronize()
+    return grad.cpu().numpy().astype(np.float64)
+
+
+def _close(got, ref, what):
+    scale = np.max(np.abs(ref))
+    norm = np.max(np.abs(got - ref)) / scale
+    l2 = np.linalg.norm(got - ref) / np.linalg.norm(ref)
+    assert norm <= TOL_ADJ and l2 <= TOL_ADJ, f"{what}: normwise {norm:.3g}, L2 {l2:.3g}"
+
+
+# dense views (rays much closer than a voxel) use the scratch's corner records;
+# sparse views use it only for the view flags
+CASES = {
+    "dense": dict(seed=301, dims=(23, 17, 29), H=150, W=170, n_samples=40),
+    "dense, near the size limit": dict(seed=302, dims=(96, 96, 90), B=2, H=400, W=400,
+                                        n_samples=64),
+    "sparse": dict(seed=303),
+}
+
+
+@pytest.mark.parametrize("name", sorted(CASES))
+def test_noalloc_matches_the_ordinary_adjoint_twice_in_a_row(cuda, name):
+    from cone_beam_ct_b200 import drr
+    w = wl.small_random_case(**CASES[name])
+    assert drr.drr_adjoint_workspace_bytes(w.dims, w.B) <= drr.DRR_NOALLOC_SCRATCH_BYTES
+    Rt, go = _inputs(cuda, w, 7)
+    ref = _adjoint(cuda, w, Rt, go, noalloc=False)
+    assert np.max(np.abs(ref)) > 0
+    for call in (1, 2):
+        _close(_adjoint(cuda, w, Rt, go, noalloc=True), ref, f"{name}, call {call}")
+
+
+def test_noalloc_rejects_volumes_beyond_its_scratch(cuda):
+    from cone_beam_ct_b200 import drr
+    w = wl.small_random_case(304, dims=(128, 128, 128))
+    assert drr.drr_adjoint_workspace_bytes(w.dims, w.B) > drr.DRR_NOALLOC_SCRATCH_BYTES
+    Rt, go = _inputs(cuda, w, 8)
+    nx, ny, nz = w.dims
+    grad = cuda.zeros((nz, ny, nx), dtype=cuda.float32, device="cuda")
+    with pytest.raises(drr.DrrError) as e:
+        drr.drr_render_adjoint_noalloc(w.dims, w.spacing, w.origin, w.K, Rt, w.B, w.H, w.W,
+                                       w.n_samples, w.density_factor, wl.MODE_RAW, go, None,
+                                       grad)
+    assert e.value.status == drr.DRR_ERR_UNSUPPORTED
+    assert "built-in scratch" in drr.drr_get_last_error()
+    cuda.cuda.synchronize()
+    assert cuda.count_nonzero(grad).item() == 0
