@@ -34,11 +34,12 @@
 // With a workspace (drr_render_adjoint_ws), views whose rays are much closer
 // than a voxel ("dense": where a 16-pixel tile spans fewer than 8 voxels at
 // the volume centre) accumulate instead into corner records: for every cell
-// its 8 corner sums, contiguous (32 bytes, one L2 sector).  A ray keeps the
-// record of its current cell pending in registers and flushes it, when it
-// changes cell, with two 16-byte vector atomics -- the L2 executes a vector
-// atomic at the same rate as a scalar one, so this carries 4x the payload
-// per operation.  A gather pass then adds each voxel's 8 record entries into
+// its 8 corner sums, contiguous (32 bytes, one L2 sector).  A 2 x 2 bundle
+// of neighbouring rays keeps the records of its current cells pending in
+// registers and flushes one, when the bundle leaves that cell, with two
+// 16-byte vector atomics -- the L2 executes a vector atomic at the same rate
+// as a scalar one, so this carries 4x the payload per operation, and the
+// bundle flushes once where its rays would have flushed up to four times.  A gather pass then adds each voxel's 8 record entries into
 // the gradient volume.  Sparse views gain nothing from records (their
 // records would miss L2) and keep the direct path above.
 #include <cuda_runtime.h>
@@ -189,11 +190,10 @@ __global__ void gather_records(const int* __restrict__ flags, const float* __res
     }
 }
 
-// RECORDS = false: the direct path, for every view without a workspace, or
-// for the views the plan left sparse; RECORDS = true: the views the plan
-// marked dense.  Both are launched; a CTA whose view belongs to the other
-// path returns at once (a uniform exit before any barrier).
-template <int MODE, bool RECORDS>
+// The direct path: every view without a workspace, or the views the plan
+// left sparse (a CTA of a dense view returns at once -- a uniform exit before
+// any barrier -- since records_kernel handles it).
+template <int MODE>
 __global__ void __launch_bounds__(kThreads)
 adjoint_kernel(const float* __restrict__ Rt, const float* __restrict__ grad_out,
                const float* __restrict__ fwd_out, float* __restrict__ grad, const Geom g,
@@ -202,18 +202,16 @@ adjoint_kernel(const float* __restrict__ Rt, const float* __restrict__ grad_out,
     __shared__ int s_dense;
     const int b = blockIdx.z;
     const int tid = threadIdx.x;
-    const bool view_dense = ws.flags != nullptr && ws.flags[1 + b] != 0;
-    if (view_dense != RECORDS) return;
+    if (ws.flags != nullptr && ws.flags[1 + b] != 0) return;
     if (tid == 0) {
         view_setup(Rt + 12 * (size_t)b, g, sv);
         s_dense = dense_tile(sv, g, blockIdx.x * kTileW, blockIdx.y * kTileH) ? 1 : 0;
     }
     __syncthreads();
-    constexpr bool records = RECORDS;
 
     int r, c;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    if (s_dense || records) {
+    if (s_dense) {
         // spread: the 32 lanes of a warp cover the whole 16 x 16 tile (bijective)
         c = blockIdx.x * kTileW + (lane & 7) * 2 + (warp & 1);
         r = blockIdx.y * kTileH + (lane >> 3) * 4 + (warp >> 1);
@@ -233,43 +231,6 @@ adjoint_kernel(const float* __restrict__ Rt, const float* __restrict__ grad_out,
     const int ph = (warp + blockIdx.x * 3 + blockIdx.y * 5 + blockIdx.z) & 7;
     const int start = (int)(((long long)g.N * ph) >> 3);
 
-    if constexpr (records) {
-        // cells stay in [0, n-2] per axis (linear-layout lim), inside the records
-        const int cr = g.nx - 1, cs = (g.nx - 1) * (g.ny - 1);
-        float p[8];
-        for (int pass = 0; pass < 2; ++pass) {
-            const int i0 = pass == 0 ? start : 0;
-            const int i1 = pass == 0 ? g.N : start;
-            if (i0 >= i1) continue;
-            long long qx = ray.q0[0] + (long long)i0 * ray.s[0];
-            long long qy = ray.q0[1] + (long long)i0 * ray.s[1];
-            long long qz = ray.q0[2] + (long long)i0 * ray.s[2];
-            int pc = -1;
-            for (int i = i0; i < i1; ++i) {
-                const int rc = fix_cell(qz) * cs + fix_cell(qy) * cr + fix_cell(qx);
-                const float fx = fix_frac(qx), fy = fix_frac(qy), fz = fix_frac(qz);
-                qx += ray.s[0];
-                qy += ray.s[1];
-                qz += ray.s[2];
-                const float wz1 = scale * fz, wz0 = scale * (1.0f - fz);
-                const float w00 = wz0 * (1.0f - fy), w01 = wz0 * fy;
-                const float w10 = wz1 * (1.0f - fy), w11 = wz1 * fy;
-                const float gx = 1.0f - fx;
-                const float w[8] = {w00 * gx, w00 * fx, w01 * gx, w01 * fx,
-                                    w10 * gx, w10 * fx, w11 * gx, w11 * fx};
-                if (rc != pc) {
-                    if (pc >= 0) flush_record(ws.rec, pc, p);
-                    pc = rc;
-#pragma unroll
-                    for (int k = 0; k < 8; ++k) p[k] = w[k];
-                } else {
-#pragma unroll
-                    for (int k = 0; k < 8; ++k) p[k] += w[k];
-                }
-            }
-            flush_record(ws.rec, pc, p);
-        }
-    } else {
     int cell[3];
     float a[8];
     for (int pass = 0; pass < 2; ++pass) {
@@ -319,7 +280,120 @@ adjoint_kernel(const float* __restrict__ Rt, const float* __restrict__ grad_out,
         }
         flush_block(grad, st, cell, a);
     }
-    }   // direct path
+}
+
+// Record path for the views the plan marked dense.  A CTA covers a 32 x 32
+// pixel tile; each thread owns a 2 x 2 bundle of neighbouring rays (less than
+// half a voxel across where this path runs) and two pending record slots,
+// home to the bundle's upper and lower pair.  A ray adds its sample to any
+// slot already holding its cell, else flushes its home slot and takes it
+// over, so a bundle that moves together flushes once per cell instead of
+// once per ray.  Bundle positions are spread over the tile (stride 2 x 4 of
+// the 16 x 16 thread grid) as on the direct path, and warps start at
+// different phases of the ray.
+constexpr int kBundle = 2;                       // rays per bundle side
+constexpr int kBundleRays = kBundle * kBundle;
+constexpr int kSlots = 2;
+constexpr int kRecTile = kTileW * kBundle;       // 32 x 32 pixels per CTA
+
+template <int MODE>
+__global__ void __launch_bounds__(kThreads)
+records_kernel(const float* __restrict__ Rt, const float* __restrict__ grad_out,
+               const float* __restrict__ fwd_out, const Geom g, const Workspace ws) {
+    __shared__ View sv;
+    const int b = blockIdx.z;
+    if (ws.flags[1 + b] == 0) return;            // sparse view: adjoint_kernel's
+    if (threadIdx.x == 0) view_setup(Rt + 12 * (size_t)b, g, sv);
+    __syncthreads();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int px = (lane & 7) * 2 + (warp & 1), py = (lane >> 3) * 4 + (warp >> 1);
+    const int c0 = blockIdx.x * kRecTile + px * kBundle, r0 = blockIdx.y * kRecTile + py * kBundle;
+
+    bool act[kBundleRays];
+    float scale[kBundleRays];
+    long long q[kBundleRays][3], s[kBundleRays][3];
+#pragma unroll
+    for (int k = 0; k < kBundleRays; ++k) {
+        const int c = c0 + (k % kBundle), r = r0 + (k / kBundle);
+        act[k] = false;
+        scale[k] = 0.0f;
+#pragma unroll
+        for (int a = 0; a < 3; ++a) q[k][a] = s[k][a] = 0;
+        if (r >= g.H || c >= g.W) continue;
+        const size_t pix = ((size_t)b * g.H + r) * g.W + c;
+        float go = grad_out[pix];
+        if (MODE == 1) go *= 1.0f - fwd_out[pix];
+        Ray ray;
+        if (go == 0.0f || !ray_setup(sv, g, (double)c, (double)r, 0.0, ray)) continue;
+        act[k] = true;
+        scale[k] = go * (g.density_factor * ray.dt);
+#pragma unroll
+        for (int a = 0; a < 3; ++a) {
+            q[k][a] = ray.q0[a];
+            s[k][a] = ray.s[a];
+        }
+    }
+    // cells stay in [0, n-2] per axis (linear-layout lim), inside the records
+    const int cr = g.nx - 1, cs = (g.nx - 1) * (g.ny - 1);
+    float p[kSlots][8];
+    int pc[kSlots];
+    const int ph = (warp + blockIdx.x * 3 + blockIdx.y * 5 + blockIdx.z) & 7;
+    const int start = (int)(((long long)g.N * ph) >> 3);
+    for (int pass = 0; pass < 2; ++pass) {
+        const int i0 = pass == 0 ? start : 0;
+        const int i1 = pass == 0 ? g.N : start;
+        if (i0 >= i1) continue;
+#pragma unroll
+        for (int h = 0; h < kSlots; ++h) pc[h] = -1;
+        long long qq[kBundleRays][3];
+#pragma unroll
+        for (int k = 0; k < kBundleRays; ++k)
+#pragma unroll
+            for (int a = 0; a < 3; ++a) qq[k][a] = q[k][a] + (long long)i0 * s[k][a];
+        for (int i = i0; i < i1; ++i) {
+#pragma unroll
+            for (int k = 0; k < kBundleRays; ++k) {
+                if (!act[k]) continue;
+                const int cell = fix_cell(qq[k][2]) * cs + fix_cell(qq[k][1]) * cr + fix_cell(qq[k][0]);
+                const float fx = fix_frac(qq[k][0]), fy = fix_frac(qq[k][1]), fz = fix_frac(qq[k][2]);
+#pragma unroll
+                for (int a = 0; a < 3; ++a) qq[k][a] += s[k][a];
+                const float wz1 = scale[k] * fz, wz0 = scale[k] * (1.0f - fz);
+                const float w00 = wz0 * (1.0f - fy), w01 = wz0 * fy;
+                const float w10 = wz1 * (1.0f - fy), w11 = wz1 * fy;
+                const float gx = 1.0f - fx;
+                const float w[8] = {w00 * gx, w00 * fx, w01 * gx, w01 * fx,
+                                    w10 * gx, w10 * fx, w11 * gx, w11 * fx};
+                const int home = k / kBundle;      // rays 0, 1 -> slot 0; rays 2, 3 -> slot 1
+                const int other = 1 - home;
+                if (pc[home] == cell) {
+#pragma unroll
+                    for (int h = 0; h < kSlots; ++h)
+                        if (h == home)
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) p[h][e] += w[e];
+                } else if (pc[other] == cell) {
+#pragma unroll
+                    for (int h = 0; h < kSlots; ++h)
+                        if (h == other)
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) p[h][e] += w[e];
+                } else {
+#pragma unroll
+                    for (int h = 0; h < kSlots; ++h) {
+                        if (h != home) continue;
+                        if (pc[h] >= 0) flush_record(ws.rec, pc[h], p[h]);
+                        pc[h] = cell;
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) p[h][e] = w[e];
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int h = 0; h < kSlots; ++h)
+            if (pc[h] >= 0) flush_record(ws.rec, pc[h], p[h]);
+    }
 }
 
 constexpr int kMaxDevices = 64;
@@ -371,14 +445,15 @@ cudaError_t launch_adjoint(const Geom& g, const float* Rt, int mode, const float
                                                     n_rec4);
     }
     if (mode == 1)
-        adjoint_kernel<1, false><<<grid, kThreads, 0, stream>>>(Rt, grad_out, fwd_out, grad_vol, g, ws);
+        adjoint_kernel<1><<<grid, kThreads, 0, stream>>>(Rt, grad_out, fwd_out, grad_vol, g, ws);
     else
-        adjoint_kernel<0, false><<<grid, kThreads, 0, stream>>>(Rt, grad_out, fwd_out, grad_vol, g, ws);
+        adjoint_kernel<0><<<grid, kThreads, 0, stream>>>(Rt, grad_out, fwd_out, grad_vol, g, ws);
     if (workspace) {
+        const dim3 rgrid((g.W + kRecTile - 1) / kRecTile, (g.H + kRecTile - 1) / kRecTile, g.B);
         if (mode == 1)
-            adjoint_kernel<1, true><<<grid, kThreads, 0, stream>>>(Rt, grad_out, fwd_out, grad_vol, g, ws);
+            records_kernel<1><<<rgrid, kThreads, 0, stream>>>(Rt, grad_out, fwd_out, g, ws);
         else
-            adjoint_kernel<0, true><<<grid, kThreads, 0, stream>>>(Rt, grad_out, fwd_out, grad_vol, g, ws);
+            records_kernel<0><<<rgrid, kThreads, 0, stream>>>(Rt, grad_out, fwd_out, g, ws);
     }
     if (workspace)
         gather_records<<<fill_grid, 256, 0, stream>>>(ws.flags, ws.rec, grad_vol, g.nx, g.ny, g.nz);
