@@ -188,8 +188,11 @@ def measured_peaks():
 
 
 def l2_read_peak_gbs(torch, nbytes):
-    """L2 read bandwidth over a buffer of ``nbytes`` (the prepared volume's
-    size), best of 5 launches of libdrr_probe.so, in GB/s."""
+    """L2 read bandwidth over a buffer of ``nbytes`` (the volume's size), best
+    of 6 launches of libdrr_probe.so, in GB/s.  Each launch streams the buffer
+    enough times to read about 8 GB: shorter launches under-read the peak
+    (measured on B200 over 32 MiB: 14.8 TB/s at 0.6 GB per launch, 17.6 at
+    2 GB, 18.7 at 8 GB)."""
     import ctypes
     lib = ctypes.CDLL(os.path.join(ROOT, "cone_beam_ct_b200", "libdrr_probe.so"))
     lib.drr_probe_l2_read.argtypes = [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int,
@@ -199,7 +202,7 @@ def l2_read_peak_gbs(torch, nbytes):
     buf = torch.ones(n16 * 4, dtype=torch.float32, device="cuda")
     sink = torch.zeros(1, dtype=torch.float32, device="cuda")
     stream = torch.cuda.current_stream()
-    reps = 20
+    reps = max(20, -(-8_000_000_000 // (n16 * 16)))
     best = 0.0
     for _ in range(6):
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)

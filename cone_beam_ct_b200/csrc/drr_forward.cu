@@ -78,38 +78,68 @@ __device__ __forceinline__ float march(const T* __restrict__ vol, const Geom& g,
     return acc;
 }
 
-// The 8 corner voxels of one cell in the corner-replicated layout, in the
-// order a + 2b + 4c of corner (a, b, c): two 16-byte loads for fp32 ...
-__device__ __forceinline__ void load_corners(const float* __restrict__ p, float v[8]) {
-    const float4 lo = __ldg(reinterpret_cast<const float4*>(p));
-    const float4 hi = __ldg(reinterpret_cast<const float4*>(p) + 1);
-    v[0] = lo.x;
-    v[1] = lo.y;
-    v[2] = lo.z;
-    v[3] = lo.w;
-    v[4] = hi.x;
-    v[5] = hi.y;
-    v[6] = hi.z;
-    v[7] = hi.w;
+// One sample in the corner-replicated layout.  A cell record holds corner
+// (a, b, c) -- voxel (i + a, j + b, k + c) -- at element 4a + 2b + c, so that
+// the pairs the x lerps take side by side, (b, c) = (0, 0), (0, 1) and
+// (1, 0), (1, 1), are adjacent: the 7 lerps then run as 3 packed fp32x2
+// steps (sm_100's FFMA2, one instruction for two lanes of fp32 work) and one
+// scalar one.  Each lane computes exactly what trilinear_at computes (b - a
+// as fma(a, -1, b), which rounds once like the subtraction), so the corner
+// layout gives the linear layout's bits.
+__device__ __forceinline__ float lerp_pairs(float2 lo0, float2 lo1, float2 d0, float2 d1,
+                                            float fx, float fy, float fz) {
+    // d0, d1: the x differences hi - lo of the two pairs
+    const float2 f2 = make_float2(fx, fx);
+    const float2 x0 = __ffma2_rn(f2, d0, lo0);                 // (c00, c01): y = 0, z = 0 / 1
+    const float2 x1 = __ffma2_rn(f2, d1, lo1);                 // (c10, c11): y = 1
+    const float2 m1 = make_float2(-1.0f, -1.0f);
+    const float2 y = __ffma2_rn(make_float2(fy, fy), __ffma2_rn(x0, m1, x1), x0);   // (c0, c1)
+    return fmaf(fz, y.y - y.x, y.x);
 }
 
-// ... and one for bf16 (element 2m in the low half of word m; widening is exact).
-__device__ __forceinline__ void load_corners(const uint16_t* __restrict__ p, float v[8]) {
-    const uint4 w = __ldg(reinterpret_cast<const uint4*>(p));
-    v[0] = __uint_as_float(w.x << 16);
-    v[1] = __uint_as_float(w.x & 0xFFFF0000u);
-    v[2] = __uint_as_float(w.y << 16);
-    v[3] = __uint_as_float(w.y & 0xFFFF0000u);
-    v[4] = __uint_as_float(w.z << 16);
-    v[5] = __uint_as_float(w.z & 0xFFFF0000u);
-    v[6] = __uint_as_float(w.w << 16);
-    v[7] = __uint_as_float(w.w & 0xFFFF0000u);
+__device__ __forceinline__ float sample_corners(const float* __restrict__ p, float fx, float fy,
+                                                float fz) {
+    const float4 lo = __ldg(reinterpret_cast<const float4*>(p));       // a = 0
+    const float4 hi = __ldg(reinterpret_cast<const float4*>(p) + 1);   // a = 1
+    const float2 m1 = make_float2(-1.0f, -1.0f);
+    const float2 lo0 = make_float2(lo.x, lo.y), lo1 = make_float2(lo.z, lo.w);
+    const float2 d0 = __ffma2_rn(lo0, m1, make_float2(hi.x, hi.y));
+    const float2 d1 = __ffma2_rn(lo1, m1, make_float2(hi.z, hi.w));
+    return lerp_pairs(lo0, lo1, d0, d1, fx, fy, fz);
 }
+
+// bf16 voxels: element 2m in the low half of word m.  Widening a bf16 to fp32
+// is exact (its bits in the high half), so the low corners are widened with a
+// shift or a mask; the x differences take the high corners as bf16 operands
+// of sm_100's mixed-precision subtraction (sub.f32.bf16: the bf16 operand is
+// widened exactly, the difference rounded once -- the fp32 subtraction's
+// result).
+__device__ __forceinline__ float sub_bf16_f32(unsigned short a, float c) {
+    float d;
+    asm("sub.rn.f32.bf16 %0, %1, %2;" : "=f"(d) : "h"(a), "f"(c));
+    return d;
+}
+
+__device__ __forceinline__ float sample_corners(const uint16_t* __restrict__ p, float fx, float fy,
+                                                float fz) {
+    const uint4 w = __ldg(reinterpret_cast<const uint4*>(p));
+    const float2 lo0 = make_float2(__uint_as_float(w.x << 16), __uint_as_float(w.x & 0xFFFF0000u));
+    const float2 lo1 = make_float2(__uint_as_float(w.y << 16), __uint_as_float(w.y & 0xFFFF0000u));
+    const float2 d0 = make_float2(sub_bf16_f32((unsigned short)w.z, lo0.x),
+                                  sub_bf16_f32((unsigned short)(w.z >> 16), lo0.y));
+    const float2 d1 = make_float2(sub_bf16_f32((unsigned short)w.w, lo1.x),
+                                  sub_bf16_f32((unsigned short)(w.w >> 16), lo1.y));
+    return lerp_pairs(lo0, lo1, d0, d1, fx, fy, fz);
+}
+
+// Unroll of the corner-layout sample loop: the largest that ptxas compiles
+// without spilling for each element type under the kernel's launch bounds.
+template <typename T>
+constexpr int kCornerUnroll = sizeof(T) == 2 ? 2 : 4;
 
 // Sum of the N samples of one ray in the corner-replicated layout: one cell
-// record per sample, the same lerps (and so the same result, bit for bit) as
-// trilinear_at on the linear layout.  Cells stay in [0, n-2] (g.lim as for
-// the linear layout), inside the stored records.
+// record per sample.  Cells stay in [0, n-2] (g.lim as for the linear
+// layout), inside the stored records.
 template <typename T>
 __device__ __forceinline__ float march_corners(const T* __restrict__ vol, const Geom& g,
                                                const Ray& ray) {
@@ -117,19 +147,10 @@ __device__ __forceinline__ float march_corners(const T* __restrict__ vol, const 
     long long qx = ray.q0[0], qy = ray.q0[1], qz = ray.q0[2];
     const long long sx = ray.s[0], sy = ray.s[1], sz = ray.s[2];
     float acc = 0.0f;
-#pragma unroll 4
+#pragma unroll(kCornerUnroll<T>)
     for (int i = 0; i < g.N; ++i) {
         const int cell = fix_cell(qz) * slice + fix_cell(qy) * row + fix_cell(qx);
-        float v[8];
-        load_corners(vol + (size_t)cell * 8, v);
-        const float fx = fix_frac(qx), fy = fix_frac(qy), fz = fix_frac(qz);
-        const float c00 = fmaf(fx, v[1] - v[0], v[0]);
-        const float c10 = fmaf(fx, v[3] - v[2], v[2]);
-        const float c01 = fmaf(fx, v[5] - v[4], v[4]);
-        const float c11 = fmaf(fx, v[7] - v[6], v[6]);
-        const float c0 = fmaf(fy, c10 - c00, c00);
-        const float c1 = fmaf(fy, c11 - c01, c01);
-        acc += fmaf(fz, c1 - c0, c0);
+        acc += sample_corners(vol + (size_t)cell * 8, fix_frac(qx), fix_frac(qy), fix_frac(qz));
         qx += sx;
         qy += sy;
         qz += sz;

@@ -217,8 +217,9 @@ def test_prepare_layouts_round_trip(cuda):
                 border[1:-1, 1:-1, 1:-1] = 0
                 assert np.all(border == 0)
             else:
+                # corner (a, b, c) of cell (i, j, k) at element 4a + 2b + c
                 rec = a.reshape(nz - 1, ny - 1, nx - 1, 8)
-                for corner in range(8):
-                    da, db, dc = corner & 1, (corner >> 1) & 1, corner >> 2
-                    assert np.array_equal(rec[..., corner],
+                for e in range(8):
+                    da, db, dc = e >> 2, (e >> 1) & 1, e & 1
+                    assert np.array_equal(rec[..., e],
                                           expect[dc:nz - 1 + dc, db:ny - 1 + db, da:nx - 1 + da])
