@@ -9,6 +9,7 @@ from .oracle import (  # noqa: F401
     bf16_to_float,
     build,
     load,
+    pose_grad,
     ray,
     render,
     render_rays,

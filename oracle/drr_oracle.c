@@ -38,6 +38,15 @@
  *     mode (the derivative of 1 - exp(-I)); I is the oracle's own forward.
  *  7. bf16 storage: round-to-nearest-even of the fp32 bit pattern to the
  *     upper 16 bits (the IEEE rounding rule, written out).
+ *  8. Pose gradient (flashdrr.rendering API docs, VolumeRaycaster: rendering
+ *     is differentiable with respect to the view matrices): dL/d[R|t], the
+ *     12 entries of each view's world-to-camera matrix taken as free
+ *     variables, L = sum over pixels of grad_out * image.  Chain rule
+ *     through every step above: d = R^T q / |R^T q|, C = -R^T t, the IJK
+ *     map, the clip (t0 and t1 move with the plane each one lies on; t0
+ *     pinned at 0 has no derivative), the sample positions
+ *     t_i = t0 + (i + 1/2)(t1 - t0)/N, the trilinear interpolant (its
+ *     gradient inside the cell of each sample) and the factor dt.
  *
  * Rays are independent, so the forward may run rays on several threads;
  * every ray is still summed sequentially, so the result does not depend on
@@ -380,6 +389,167 @@ int oracle_adjoint(const float *vol, const int dims[3], const double spacing[3],
         for (int64_t m = 0; m < nvox; ++m) grad_vol[m] += bufs[t][m];
         free(bufs[t]);
     }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* pose gradient                                                             */
+
+/* Gradient of the zero-padded trilinear interpolant at p, inside the cell
+ * floor(p): d/dp_a of sum_corners w(f) v. */
+static void trilinear_grad(const float *vol, const grid_t *g, const double p[3], double gr[3]) {
+    double fl[3], f[3];
+    int64_t i0[3];
+    for (int a = 0; a < 3; ++a) {
+        fl[a] = floor(p[a]);
+        f[a] = p[a] - fl[a];
+        i0[a] = (int64_t)fl[a];
+        gr[a] = 0.0;
+    }
+    for (int dk = 0; dk < 2; ++dk)
+        for (int dj = 0; dj < 2; ++dj)
+            for (int di = 0; di < 2; ++di) {
+                double v = voxel(vol, g, i0[0] + di, i0[1] + dj, i0[2] + dk);
+                double wx = di ? f[0] : 1.0 - f[0], sx = di ? 1.0 : -1.0;
+                double wy = dj ? f[1] : 1.0 - f[1], sy = dj ? 1.0 : -1.0;
+                double wz = dk ? f[2] : 1.0 - f[2], sz = dk ? 1.0 : -1.0;
+                gr[0] += sx * wy * wz * v;
+                gr[1] += wx * sy * wz * v;
+                gr[2] += wx * wy * sz * v;
+            }
+}
+
+/* dI/d[R|t] of one ray, grad12[4r + c] for R[r][c] (c < 3) and t[r] (c = 3).
+ * Returns the integral I (0 and a zero gradient on a miss). */
+static double ray_pose_grad(const float *vol, const grid_t *g, const double K[9],
+                            const double Rt[12], double u, double v, int n_samples,
+                            double density_factor, double grad12[12]) {
+    for (int m = 0; m < 12; ++m) grad12[m] = 0.0;
+    double Cijk[3], dijk[3], t0, t1;
+    if (!ray_in_volume(g, K, Rt, u, v, Cijk, dijk, &t0, &t1)) return 0.0;
+    /* the camera ray again, with the pieces the derivatives need */
+    double q[3], a[3], n2 = 0.0;
+    q[2] = 1.0 / K[8];
+    q[1] = (v - K[5] * q[2]) / K[4];
+    q[0] = (u - K[1] * q[1] - K[2] * q[2]) / K[0];
+    for (int c = 0; c < 3; ++c) {
+        a[c] = 0.0;
+        for (int r = 0; r < 3; ++r) a[c] += Rt[4 * r + c] * q[r];
+        n2 += a[c] * a[c];
+    }
+    const double nrm = sqrt(n2);
+    double dw[3];
+    for (int c = 0; c < 3; ++c) dw[c] = a[c] / nrm;
+    /* which plane each end of the clip lies on: the axis that attains t_near
+     * (the largest entry parameter) and t_far (the smallest exit one) */
+    int ax0 = -1, ax1 = -1;
+    double t_near = -INFINITY, t_far = INFINITY;
+    for (int k = 0; k < 3; ++k) {
+        if (dijk[k] == 0.0) continue;
+        double tA = (0.0 - Cijk[k]) / dijk[k];
+        double tB = ((double)(g->n[k] - 1) - Cijk[k]) / dijk[k];
+        double tmin = tA < tB ? tA : tB, tmax = tA < tB ? tB : tA;
+        if (tmin > t_near) { t_near = tmin; ax0 = k; }
+        if (tmax < t_far) { t_far = tmax; ax1 = k; }
+    }
+    const int pinned0 = !(t_near > 0.0);   /* t0 = 0: the camera is inside the box */
+    const double dt = (t1 - t0) / (double)n_samples;
+    for (int m = 0; m < 12; ++m) {
+        const int r = m / 4, c = m % 4;
+        /* derivatives of the world camera centre and unit direction */
+        double dC[3] = {0.0, 0.0, 0.0}, dd[3] = {0.0, 0.0, 0.0};
+        if (c == 3) {
+            /* C_w = -R^T t: dC_w[k]/dt[r] = -R[r][k]; d does not depend on t */
+            for (int k = 0; k < 3; ++k) dC[k] = -Rt[4 * r + k];
+        } else {
+            /* dC_w[k]/dR[r][c] = -t[r] if k == c */
+            dC[c] = -Rt[4 * r + 3];
+            /* da/dR[r][c] = q[r] e_c; d(a/|a|) = (I - dw dw^T) da / |a| */
+            for (int k = 0; k < 3; ++k)
+                dd[k] = ((k == c ? 1.0 : 0.0) - dw[k] * dw[c]) * q[r] / nrm;
+        }
+        /* to IJK */
+        for (int k = 0; k < 3; ++k) {
+            dC[k] /= g->spacing[k];
+            dd[k] /= g->spacing[k];
+        }
+        /* a clip plane x_k = P gives t = (P - C_k) / d_k */
+        double dt0 = 0.0, dt1 = 0.0;
+        if (!pinned0) dt0 = -(dC[ax0] + t0 * dd[ax0]) / dijk[ax0];
+        dt1 = -(dC[ax1] + t1 * dd[ax1]) / dijk[ax1];
+        const double ddt = (dt1 - dt0) / (double)n_samples;
+        double sum = 0.0, dsum = 0.0;
+        for (int i = 0; i < n_samples; ++i) {
+            const double ti = t0 + ((double)i + 0.5) * dt;
+            const double dti = dt0 + ((double)i + 0.5) * ddt;
+            double p[3], gr[3];
+            for (int k = 0; k < 3; ++k) p[k] = Cijk[k] + ti * dijk[k];
+            sum += trilinear(vol, g, p);
+            trilinear_grad(vol, g, p, gr);
+            for (int k = 0; k < 3; ++k) dsum += gr[k] * (dC[k] + dti * dijk[k] + ti * dd[k]);
+        }
+        grad12[m] = density_factor * (ddt * sum + dt * dsum);
+    }
+    double dt2;
+    return ray_integral(vol, g, K, Rt, u, v, n_samples, density_factor, &dt2);
+}
+
+typedef struct {
+    const float *vol;
+    const grid_t *g;
+    const double *K, *Rt;
+    int B, H, W, n_samples, mode, stride, first;
+    double density_factor;
+    const double *grad_out;
+    double *grad_Rt;
+} pose_job_t;
+
+static void *pose_worker(void *arg) {
+    pose_job_t *j = (pose_job_t *)arg;
+    for (int b = j->first; b < j->B; b += j->stride) {
+        double acc[12] = {0.0};
+        for (int r = 0; r < j->H; ++r)
+            for (int c = 0; c < j->W; ++c) {
+                double go = j->grad_out[((int64_t)b * j->H + r) * j->W + c];
+                if (go == 0.0) continue;
+                double g12[12];
+                double I = ray_pose_grad(j->vol, j->g, j->K, j->Rt + 12 * b, c, r, j->n_samples,
+                                         j->density_factor, g12);
+                /* Beer-Lambert: d(1 - exp(-I))/dI = exp(-I) */
+                double w = go * (j->mode == ORACLE_BEER_LAMBERT ? exp(-I) : 1.0);
+                for (int m = 0; m < 12; ++m) acc[m] += w * g12[m];
+            }
+        for (int m = 0; m < 12; ++m) j->grad_Rt[12 * b + m] += acc[m];
+    }
+    return NULL;
+}
+
+/* Pose gradient: grad_Rt[b][4r + c] += sum over the pixels of view b of
+ * grad_out * d image / d Rt[b][r][c].  Views run on up to nthreads threads;
+ * each view is summed sequentially, so the result does not depend on the
+ * thread count. */
+int oracle_pose_grad(const float *vol, const int dims[3], const double spacing[3],
+                     const double origin[3], const double K[9], const double *Rt, int B,
+                     int H, int W, int n_samples, double density_factor, int mode,
+                     const double *grad_out, double *grad_Rt, int nthreads) {
+    grid_t g;
+    if (make_grid(dims, spacing, origin, &g) || B < 0 || H < 0 || W < 0 || n_samples < 1)
+        return -1;
+    if (nthreads > B) nthreads = B;
+    if (nthreads > 64) nthreads = 64;
+    if (nthreads < 1) nthreads = 1;
+    pthread_t tid[64];
+    int running[64];
+    pose_job_t jobs[64];
+    for (int t = 0; t < nthreads; ++t) {
+        pose_job_t j = {vol, &g, K, Rt, B, H, W, n_samples, mode, nthreads, t, density_factor,
+                        grad_out, grad_Rt};
+        jobs[t] = j;
+        running[t] = nthreads > 1 && pthread_create(&tid[t], NULL, pose_worker, &jobs[t]) == 0;
+        if (!running[t]) pose_worker(&jobs[t]);
+    }
+    for (int t = 0; t < nthreads; ++t)
+        if (running[t]) pthread_join(tid[t], NULL);
     return 0;
 }
 

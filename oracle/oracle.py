@@ -42,6 +42,10 @@ def load():
                                    _c.c_int, _c.c_int, _c.c_int, _c.c_double, _c.c_int, _f64p,
                                    _f64p, _c.c_int]
     lib.oracle_adjoint.restype = _c.c_int
+    lib.oracle_pose_grad.argtypes = [_f32p, _i32p, _f64p, _f64p, _f64p, _f64p, _c.c_int,
+                                     _c.c_int, _c.c_int, _c.c_int, _c.c_double, _c.c_int,
+                                     _f64p, _f64p, _c.c_int]
+    lib.oracle_pose_grad.restype = _c.c_int
     lib.oracle_round_bf16.argtypes = [_f32p, _u16p, _c.c_int64]
     lib.oracle_round_bf16.restype = None
     lib.oracle_bf16_to_float.argtypes = [_u16p, _f32p, _c.c_int64]
@@ -131,6 +135,23 @@ def adjoint(dims, spacing, origin, K, Rt, H, W, n_samples, density_factor, mode,
     assert rc == 0, "oracle_adjoint rejected its arguments"
     nx, ny, nz = (int(x) for x in dims)
     return grad.reshape(nz, ny, nx)
+
+
+def pose_grad(vol, dims, spacing, origin, K, Rt, H, W, n_samples, density_factor, mode,
+              grad_out, nthreads=1):
+    """grad_Rt[b][r][c] (float64, B x 3 x 4) = sum over the pixels of view b of
+    grad_out * d image / d Rt[b][r][c] (the 12 matrix entries taken as free
+    variables; times exp(-I) in Beer-Lambert)."""
+    dims, spacing, origin, K, Rt = _geom(dims, spacing, origin, K, Rt)
+    B = Rt.shape[0]
+    go = np.ascontiguousarray(grad_out, dtype=np.float64).reshape(-1)
+    assert go.size == B * H * W
+    out = np.zeros(B * 12, dtype=np.float64)
+    v = _vol(vol, dims)
+    rc = load().oracle_pose_grad(v, dims, spacing, origin, K, Rt.reshape(-1), B, H, W,
+                                 n_samples, density_factor, mode, go, out, int(nthreads))
+    assert rc == 0, "oracle_pose_grad rejected its arguments"
+    return out.reshape(B, 3, 4)
 
 
 def round_bf16(x):

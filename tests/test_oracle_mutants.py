@@ -51,6 +51,25 @@ MUTANTS = {
         " if (j >= g->n[1]) j = g->n[1] - 1; if (k >= g->n[2]) k = g->n[2] - 1;"),
     "spacing ignored in the direction": ("dijk[a] = d[a] / g->spacing[a];", "dijk[a] = d[a];"),
     "bf16 truncation instead of rounding": ("bits += 0x7fffu + lsb;", "(void)lsb;"),
+    "pose gradient without the derivative of dt": (
+        "grad12[m] = density_factor * (ddt * sum + dt * dsum);",
+        "grad12[m] = density_factor * (dt * dsum);"),
+    "pose gradient without the unit-length projection": (
+        "dd[k] = ((k == c ? 1.0 : 0.0) - dw[k] * dw[c]) * q[r] / nrm;",
+        "dd[k] = (k == c ? 1.0 : 0.0) * q[r] / nrm;"),
+    "pose gradient exit-plane sign": (
+        "dt1 = -(dC[ax1] + t1 * dd[ax1]) / dijk[ax1];", "dt1 = (dC[ax1] + t1 * dd[ax1]) / dijk[ax1];"),
+    "pose gradient entry point moving inside the box": (
+        "if (!pinned0) dt0 = -(dC[ax0] + t0 * dd[ax0]) / dijk[ax0];",
+        "if (ax0 >= 0) dt0 = -(dC[ax0] + t0 * dd[ax0]) / dijk[ax0];"),
+    "pose gradient y-derivative sign": (
+        "double wy = dj ? f[1] : 1.0 - f[1], sy = dj ? 1.0 : -1.0;",
+        "double wy = dj ? f[1] : 1.0 - f[1], sy = dj ? -1.0 : 1.0;"),
+    "pose gradient without exp(-I) in Beer-Lambert": (
+        "double w = go * (j->mode == ORACLE_BEER_LAMBERT ? exp(-I) : 1.0);", "double w = go;"),
+    "pose gradient translation sign": (
+        "for (int k = 0; k < 3; ++k) dC[k] = -Rt[4 * r + k];",
+        "for (int k = 0; k < 3; ++k) dC[k] = Rt[4 * r + k];"),
 }
 
 
@@ -66,7 +85,9 @@ def test_pins_catch_mutant(name, tmp_path):
     subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-o", str(lib),
                            str(c_file), "-lm", "-lpthread"])
     env = dict(os.environ, DRR_ORACLE_LIB=str(lib))
-    r = subprocess.run([sys.executable, "-m", "pytest", os.path.join(ROOT, "tests",
-                        "test_oracle_pins.py"), "-q", "-x", "-p", "no:cacheprovider"],
+    r = subprocess.run([sys.executable, "-m", "pytest",
+                        os.path.join(ROOT, "tests", "test_oracle_pins.py"),
+                        os.path.join(ROOT, "tests", "test_oracle_pose_pins.py"),
+                        "-q", "-x", "-p", "no:cacheprovider"],
                        env=env, cwd=ROOT, capture_output=True, text=True, timeout=600)
     assert r.returncode != 0, f"mutant '{name}' passed every pin:\n{r.stdout[-2000:]}"
