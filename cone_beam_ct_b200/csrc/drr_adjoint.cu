@@ -34,14 +34,16 @@
 // With a workspace (drr_render_adjoint_ws), views whose rays are much closer
 // than a voxel ("dense": where a 16-pixel tile spans fewer than 8 voxels at
 // the volume centre) accumulate instead into corner records: for every cell
-// its 8 corner sums, contiguous (32 bytes, one L2 sector).  A 2 x 2 bundle
+// its 8 corner sums, contiguous (32 bytes, one L2 sector).  A 3 x 2 bundle
 // of neighbouring rays keeps the records of its current cells pending in
 // registers and flushes one, when the bundle leaves that cell, with two
 // 16-byte vector atomics -- the L2 executes a vector atomic at the same rate
 // as a scalar one, so this carries 4x the payload per operation, and the
-// bundle flushes once where its rays would have flushed up to four times.  A gather pass then adds each voxel's 8 record entries into
-// the gradient volume.  Sparse views gain nothing from records (their
-// records would miss L2) and keep the direct path above.
+// bundle flushes once where its rays would have flushed up to six times.  A
+// gather pass then adds each voxel's 8 record entries into the gradient
+// volume.  Sparse views gain nothing from records (measured: the records
+// path ran 12-20 ms against the direct path's 9.3 on the 256^3 / 200^2
+// workload) and keep the direct path above.
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -282,24 +284,27 @@ adjoint_kernel(const float* __restrict__ Rt, const float* __restrict__ grad_out,
     }
 }
 
-// Record path for the views the plan marked dense.  A CTA covers a 32 x 32
-// pixel tile; each thread owns a 2 x 2 bundle of neighbouring rays (less than
-// half a voxel across where this path runs) and two pending record slots,
-// home to the bundle's upper and lower pair.  A ray adds its sample to any
-// slot already holding its cell, else flushes its home slot and takes it
-// over, so a bundle that moves together flushes once per cell instead of
-// once per ray.  A warp's bundles are neighbours (an 8 x 4 block of them)
-// and warps start at one of 16 phases of the ray.  (Measured on the
-// 1024^2 x 512 C-arm workload: neighbouring bundles beat bundles spread over
-// the tile, 7.1 vs 7.8 ms; 8, 16 or 32 phases are within 0.3 %, none is 2 %
-// slower.)
-constexpr int kBundle = 2;                       // rays per bundle side
-constexpr int kBundleRays = kBundle * kBundle;
+// Record path for the views the plan marked dense.  A CTA covers a 48 x 32
+// pixel tile; each thread owns a 3 x 2 bundle of neighbouring rays (less than
+// a voxel across where this path runs) and two pending record slots, home to
+// the bundle's upper and lower row.  A ray adds its sample to any slot
+// already holding its cell, else flushes its home slot and takes it over, so
+// a bundle that moves together flushes once per cell instead of once per
+// ray.  A warp's bundles are neighbours (an 8 x 4 block of them) and warps
+// start at one of 16 phases of the ray.  Measured on the 1024^2 x 512 and
+// 2048^2 x 256 C-arm workloads (B200): neighbouring bundles beat bundles
+// spread over the tile (7.1 vs 7.8 ms); 3 x 2 bundles flush 11 % less than
+// 2 x 2 (0.26 against 0.30 flushes per ray-sample) and run 3 % / 8 % faster;
+// a least-recently-used slot choice flushes less still but its extra
+// branches doubled the issued instructions; packed fp32x2 weights saturate
+// the FMA pipe instead.
+constexpr int kBundleX = 3, kBundleY = 2;        // rays per bundle, across and down
+constexpr int kBundleRays = kBundleX * kBundleY;
 constexpr int kSlots = 2;
-constexpr int kRecTile = kTileW * kBundle;       // 32 x 32 pixels per CTA
+constexpr int kRecTileW = 16 * kBundleX, kRecTileH = 16 * kBundleY;   // 48 x 32 pixels per CTA
 
 template <int MODE>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 2)
 records_kernel(const float* __restrict__ Rt, const float* __restrict__ grad_out,
                const float* __restrict__ fwd_out, const Geom g, const Workspace ws) {
     __shared__ View sv;
@@ -310,14 +315,18 @@ records_kernel(const float* __restrict__ Rt, const float* __restrict__ grad_out,
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     // a warp's 32 bundles form an 8 x 4 block of the 16 x 16 bundle grid
     const int px = (warp & 1) * 8 + (lane & 7), py = (warp >> 1) * 4 + (lane >> 3);
-    const int c0 = blockIdx.x * kRecTile + px * kBundle, r0 = blockIdx.y * kRecTile + py * kBundle;
+    const int c0 = blockIdx.x * kRecTileW + px * kBundleX, r0 = blockIdx.y * kRecTileH + py * kBundleY;
+    const int ph = (warp + blockIdx.x * 3 + blockIdx.y * 5 + blockIdx.z) & 15;   // 16 phases
+    const int start = (int)(((long long)g.N * ph) >> 4);
 
+    // per ray: its position at the current sample (32.32) and step; the start
+    // of the second pass is recovered from the position after the first
     bool act[kBundleRays];
     float scale[kBundleRays];
     long long q[kBundleRays][3], s[kBundleRays][3];
 #pragma unroll
     for (int k = 0; k < kBundleRays; ++k) {
-        const int c = c0 + (k % kBundle), r = r0 + (k / kBundle);
+        const int c = c0 + (k % kBundleX), r = r0 + (k / kBundleX);
         act[k] = false;
         scale[k] = 0.0f;
 #pragma unroll
@@ -332,42 +341,41 @@ records_kernel(const float* __restrict__ Rt, const float* __restrict__ grad_out,
         scale[k] = go * (g.density_factor * ray.dt);
 #pragma unroll
         for (int a = 0; a < 3; ++a) {
-            q[k][a] = ray.q0[a];
             s[k][a] = ray.s[a];
+            q[k][a] = ray.q0[a] + (long long)start * ray.s[a];
         }
     }
     // cells stay in [0, n-2] per axis (linear-layout lim), inside the records
     const int cr = g.nx - 1, cs = (g.nx - 1) * (g.ny - 1);
     float p[kSlots][8];
     int pc[kSlots];
-    const int ph = (warp + blockIdx.x * 3 + blockIdx.y * 5 + blockIdx.z) & 15;   // 16 phases
-    const int start = (int)(((long long)g.N * ph) >> 4);
     for (int pass = 0; pass < 2; ++pass) {
         const int i0 = pass == 0 ? start : 0;
         const int i1 = pass == 0 ? g.N : start;
+        if (pass == 1) {                         // back to sample 0: q0 = q(N) - N * s
+#pragma unroll
+            for (int k = 0; k < kBundleRays; ++k)
+#pragma unroll
+                for (int a = 0; a < 3; ++a) q[k][a] -= (long long)g.N * s[k][a];
+        }
         if (i0 >= i1) continue;
 #pragma unroll
         for (int h = 0; h < kSlots; ++h) pc[h] = -1;
-        long long qq[kBundleRays][3];
-#pragma unroll
-        for (int k = 0; k < kBundleRays; ++k)
-#pragma unroll
-            for (int a = 0; a < 3; ++a) qq[k][a] = q[k][a] + (long long)i0 * s[k][a];
         for (int i = i0; i < i1; ++i) {
 #pragma unroll
             for (int k = 0; k < kBundleRays; ++k) {
                 if (!act[k]) continue;
-                const int cell = fix_cell(qq[k][2]) * cs + fix_cell(qq[k][1]) * cr + fix_cell(qq[k][0]);
-                const float fx = fix_frac(qq[k][0]), fy = fix_frac(qq[k][1]), fz = fix_frac(qq[k][2]);
+                const int cell = fix_cell(q[k][2]) * cs + fix_cell(q[k][1]) * cr + fix_cell(q[k][0]);
+                const float fx = fix_frac(q[k][0]), fy = fix_frac(q[k][1]), fz = fix_frac(q[k][2]);
 #pragma unroll
-                for (int a = 0; a < 3; ++a) qq[k][a] += s[k][a];
+                for (int a = 0; a < 3; ++a) q[k][a] += s[k][a];
                 const float wz1 = scale[k] * fz, wz0 = scale[k] * (1.0f - fz);
                 const float w00 = wz0 * (1.0f - fy), w01 = wz0 * fy;
                 const float w10 = wz1 * (1.0f - fy), w11 = wz1 * fy;
                 const float gx = 1.0f - fx;
                 const float w[8] = {w00 * gx, w00 * fx, w01 * gx, w01 * fx,
                                     w10 * gx, w10 * fx, w11 * gx, w11 * fx};
-                const int home = k / kBundle;      // rays 0, 1 -> slot 0; rays 2, 3 -> slot 1
+                const int home = k / kBundleX;   // upper row -> slot 0, lower row -> slot 1
                 const int other = 1 - home;
                 if (pc[home] == cell) {
 #pragma unroll
@@ -452,7 +460,7 @@ cudaError_t launch_adjoint(const Geom& g, const float* Rt, int mode, const float
     else
         adjoint_kernel<0><<<grid, kThreads, 0, stream>>>(Rt, grad_out, fwd_out, grad_vol, g, ws);
     if (workspace) {
-        const dim3 rgrid((g.W + kRecTile - 1) / kRecTile, (g.H + kRecTile - 1) / kRecTile, g.B);
+        const dim3 rgrid((g.W + kRecTileW - 1) / kRecTileW, (g.H + kRecTileH - 1) / kRecTileH, g.B);
         if (mode == 1)
             records_kernel<1><<<rgrid, kThreads, 0, stream>>>(Rt, grad_out, fwd_out, g, ws);
         else

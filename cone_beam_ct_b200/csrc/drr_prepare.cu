@@ -53,7 +53,7 @@ __global__ void to_padded(const float* __restrict__ src, T* __restrict__ dst, in
 }
 
 // Corner-replicated layout: record m = cell (i, j, k) holds the 8 voxels
-// src[k+c][j+b][i+a] in the order 4a + 2b + c, written as one (bf16) or two
+// src[k+c][j+b][i+a] in the order a + 2b + 4c, written as one (bf16) or two
 // (fp32) 16-byte stores.
 __device__ __forceinline__ void store_corners(float* dst, const float v[8]) {
     float4* d = reinterpret_cast<float4*>(dst);
@@ -82,11 +82,11 @@ __global__ void to_corners(const float* __restrict__ src, T* __restrict__ dst, i
         const int k = (int)(m / ((int64_t)cx * cy));
         const float* p = src + (((int64_t)k * ny + j) * nx + i);
         const int64_t sy = nx, sz = (int64_t)nx * ny;
-        // corner (a, b, c) at element 4a + 2b + c
+        // corner (a, b, c) at element a + 2b + 4c
         float v[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e)
-            v[e] = __ldg(p + ((e & 4) ? 1 : 0) + ((e & 2) ? sy : 0) + ((e & 1) ? sz : 0));
+            v[e] = __ldg(p + ((e & 1) ? 1 : 0) + ((e & 2) ? sy : 0) + ((e & 4) ? sz : 0));
         store_corners(dst + m * 8, v);
     }
 }

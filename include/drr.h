@@ -94,7 +94,7 @@ typedef enum {
     DRR_LAYOUT_PADDED = 1,
     /* Corner-replicated: for every cell (i, j, k) in [0, nx-2] x [0, ny-2] x
        [0, nz-2] (cell index (k*(ny-1) + j)*(nx-1) + i) its 8 corner voxels
-       vol[k+c][j+b][i+a] stored contiguously in the order 4a + 2b + c: 8
+       vol[k+c][j+b][i+a] stored contiguously in the order a + 2b + 4c: 8
        elements, 16 bytes (bf16) or 32 bytes (fp32) per cell, 16-byte
        aligned.  Written by drr_prepare_volume.  One sample of the forward
        then reads its 8 voxels with one (bf16) or two (fp32) 16-byte loads

@@ -217,9 +217,9 @@ def test_prepare_layouts_round_trip(cuda):
                 border[1:-1, 1:-1, 1:-1] = 0
                 assert np.all(border == 0)
             else:
-                # corner (a, b, c) of cell (i, j, k) at element 4a + 2b + c
+                # corner (a, b, c) of cell (i, j, k) at element a + 2b + 4c
                 rec = a.reshape(nz - 1, ny - 1, nx - 1, 8)
                 for e in range(8):
-                    da, db, dc = e >> 2, (e >> 1) & 1, e & 1
+                    da, db, dc = e & 1, (e >> 1) & 1, e >> 2
                     assert np.array_equal(rec[..., e],
                                           expect[dc:nz - 1 + dc, db:ny - 1 + db, da:nx - 1 + da])
