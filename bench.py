@@ -54,6 +54,8 @@ def parse_args():
                    help="volume layout drr_prepare_volume writes for the forward")
     p.add_argument("--texture", action="store_true",
                    help="also time the texture-trilinear comparison forward (libdrr_texture.so)")
+    p.add_argument("--pose", action="store_true",
+                   help="also time the pose gradient (drr_render_pose_grad) on the same workload")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     return p.parse_args()
@@ -361,6 +363,39 @@ def texture_comparison(torch, w, vol32, Rt, exact_out):
     return res
 
 
+def pose_timing(torch, w, prep, dtype, layout, Rt, grad_out, out, elem, l2_peak, hbm_peak,
+                vol_fits_l2):
+    """The pose gradient on the same workload (not part of the step): kernel
+    time (median of 10, L2 flushed before each) and its gather roofline, the
+    forward's 8 voxel reads per sample."""
+    from cone_beam_ct_b200 import drr
+    from cone_beam_ct_b200 import workloads as wl
+    stream = torch.cuda.current_stream()
+    g = torch.zeros((w.B, 12), dtype=torch.float32, device=out.device)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=out.device)
+    fwd = out if w.mode == wl.MODE_BEER_LAMBERT else None
+    times = []
+    for m in range(13):
+        flush.fill_(m & 0xFF)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        drr.drr_render_pose_grad(prep, dtype, layout, w.dims, w.spacing, w.origin, w.K, Rt, w.B,
+                                 w.H, w.W, w.n_samples, w.density_factor, w.mode, grad_out, fwd,
+                                 g, stream=stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if m >= 3:
+            times.append(e0.elapsed_time(e1))
+    ms = statistics.median(times)
+    nbytes = 8 * elem * w.samples
+    achieved = nbytes / (ms * 1e-3) / 1e9
+    bound, peak = ("l2", l2_peak) if vol_fits_l2 and l2_peak else ("hbm", hbm_peak)
+    return {"ms": ms, "gsamples_s": w.samples / (ms * 1e-3) / 1e9,
+            "roofline": {"kernel": "pose_kernel", "bound": bound, "achieved": achieved,
+                         "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                         "algorithmic_bytes_per_launch": int(nbytes)}}
+
+
 def run_ours(args):
     import torch
     from cone_beam_ct_b200 import drr
@@ -512,6 +547,11 @@ def run_ours(args):
     adj_roof = roof("adjoint_kernel", adj_ms, adj_bytes, "adjoint_kernel", wname)
     dominant = adj_roof if adj_ms >= fwd_ms else fwd_roof
 
+    pose = None
+    if args.pose:
+        pose = pose_timing(torch, w, prep, dtype, layout, Rt, grad_out, out, elem, l2_peak,
+                           hbm_peak, vol_fits_l2)
+
     tex = None
     if args.texture:
         tex = texture_comparison(torch, w, vol32, Rt, out)
@@ -538,6 +578,7 @@ def run_ours(args):
         "cpu_baseline": base,
         "e2e": e2e,
         "texture_comparison": tex,
+        "pose_gradient": pose,
         "gpu_launches": 7 * args.steps,   # prepare, forward, plan, zero, 2 adjoint paths, gather
         "clocks": clocks,
         "bracket_ms": bracket[0].elapsed_time(bracket[1]),

@@ -1,7 +1,8 @@
 """B200-native cone-beam DRR ray-marcher (forward projection and its adjoint).
 
 The compute path is libdrr.so (hand-written sm_100a CUDA behind the C ABI of
-include/drr.h); ``cone_beam_ct_b200.drr`` binds it with the same names.
+include/drr.h): the forward ray-march, its volume adjoint and its pose
+gradient; ``cone_beam_ct_b200.drr`` binds it with the same names.
 ``cone_beam_ct_b200.workloads`` makes seeded synthetic inputs.
 """
 from .drr import (  # noqa: F401
@@ -20,5 +21,7 @@ from .drr import (  # noqa: F401
     drr_prepared_bytes,
     drr_render,
     drr_render_adjoint,
+    drr_render_adjoint_noalloc,
     drr_render_adjoint_ws,
+    drr_render_pose_grad,
 )

@@ -123,8 +123,10 @@ __device__ __forceinline__ float sample_corners(const uint16_t* __restrict__ p, 
     // a = 0 corners of rows (b, c) = (0, 0), (0, 1) and (1, 0), (1, 1),
     // widened by a byte permute (low half to high, zeros below) that runs on
     // the integer pipe rather than the FMA pipe a shift may be issued to
-    const float2 lo0 = make_float2(__uint_as_float(w.x << 16), __uint_as_float(w.z << 16));
-    const float2 lo1 = make_float2(__uint_as_float(w.y << 16), __uint_as_float(w.w << 16));
+    const float2 lo0 = make_float2(__uint_as_float(__byte_perm(w.x, 0u, 0x1044)),
+                                   __uint_as_float(__byte_perm(w.z, 0u, 0x1044)));
+    const float2 lo1 = make_float2(__uint_as_float(__byte_perm(w.y, 0u, 0x1044)),
+                                   __uint_as_float(__byte_perm(w.w, 0u, 0x1044)));
     const float2 d0 = make_float2(sub_bf16_f32((unsigned short)(w.x >> 16), lo0.x),
                                   sub_bf16_f32((unsigned short)(w.z >> 16), lo0.y));
     const float2 d1 = make_float2(sub_bf16_f32((unsigned short)(w.y >> 16), lo1.x),

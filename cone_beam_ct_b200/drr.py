@@ -21,8 +21,8 @@ DRR_LAYOUT_LINEAR, DRR_LAYOUT_PADDED, DRR_LAYOUT_CORNERS = 0, 1, 2
 
 # names exported by libdrr.so (include/drr.h)
 EXPORTED = ("drr_render", "drr_render_adjoint", "drr_render_adjoint_ws",
-            "drr_adjoint_workspace_bytes", "drr_render_adjoint_noalloc", "drr_prepared_bytes",
-            "drr_prepare_volume", "drr_get_last_error", "drr_abi_version")
+            "drr_adjoint_workspace_bytes", "drr_render_adjoint_noalloc", "drr_render_pose_grad",
+            "drr_prepared_bytes", "drr_prepare_volume", "drr_get_last_error", "drr_abi_version")
 DRR_NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
@@ -63,6 +63,10 @@ def lib():
                                              _c.c_int, _c.c_int, _c.c_float, _c.c_int, _vp, _vp,
                                              _vp, _vp]
     L.drr_render_adjoint_noalloc.restype = _c.c_int
+    L.drr_render_pose_grad.argtypes = [_vp, _c.c_int, _c.c_int, _i3, _f3, _f3, _f9, _vp,
+                                       _c.c_int, _c.c_int, _c.c_int, _c.c_int, _c.c_float,
+                                       _c.c_int, _vp, _vp, _vp, _vp]
+    L.drr_render_pose_grad.restype = _c.c_int
     L.drr_adjoint_workspace_bytes.argtypes = [_i3, _c.c_int]
     L.drr_adjoint_workspace_bytes.restype = _c.c_size_t
     L.drr_prepared_bytes.argtypes = [_i3, _c.c_int, _c.c_int]
@@ -162,6 +166,17 @@ def drr_render_adjoint(dims, spacing, origin, K, Rt, B, H, W, n_samples, density
                                     _dev(grad_out, "grad_out", True),
                                     _dev(fwd_out, "fwd_out", True),
                                     _dev(grad_vol, "grad_vol", True), _stream(stream)))
+
+
+def drr_render_pose_grad(vol, dtype, layout, dims, spacing, origin, K, Rt, B, H, W, n_samples,
+                         density_factor, mode, grad_out, fwd_out, grad_Rt, stream=None):
+    _check(lib().drr_render_pose_grad(_dev(vol, "vol", True), int(dtype), int(layout), _i3v(dims),
+                                      _f3v(spacing), _f3v(origin), _f9v(K), _dev(Rt, "Rt", True),
+                                      int(B), int(H), int(W), int(n_samples),
+                                      float(density_factor), int(mode),
+                                      _dev(grad_out, "grad_out", True),
+                                      _dev(fwd_out, "fwd_out", True),
+                                      _dev(grad_Rt, "grad_Rt", True), _stream(stream)))
 
 
 def drr_adjoint_workspace_bytes(dims, B):

@@ -206,6 +206,37 @@ DRR_API drr_status drr_render_adjoint_noalloc(const int dims[3], const float spa
                                               const float *fwd_out, float *grad_vol,
                                               void *stream);
 
+/* Pose gradient: dL/d[R|t] of L = sum(grad_out * out), per view, for the
+ * registration use of a differentiable renderer (flashdrr.rendering API
+ * docs, VolumeRaycaster: rendering is differentiable with respect to the
+ * view matrices; FlashDRR page, 2D/3D registration).  The 12 entries of
+ * each view's world-to-camera matrix are taken as free variables of the ray
+ * as written: direction R^T K^-1 (u, v, 1) normalised, centre -R^T t.
+ * Along rotations (dR = R [w]x) this equals the derivative of any rotation
+ * parameterisation; off the rotation group it is the derivative of these
+ * formulas (R^T, not R^-1).  The chain rule runs through the clip (each end
+ * moves with the box plane it lies on; an entry point at the camera, when
+ * the camera is inside the box, does not move), the sample positions, the
+ * gradient of the trilinear interpolant inside each sample's cell and dt.
+ *   vol, dtype, layout  the forward's volume (any layout).
+ *   grad_out    DEVICE float[B*H*W], upstream gradient dL/d(out).
+ *   fwd_out     DEVICE float[B*H*W], the Beer-Lambert image (required in
+ *               DRR_MODE_BEER_LAMBERT, where each ray's term is scaled by
+ *               exp(-I) = 1 - out; may be NULL in DRR_MODE_RAW).
+ *   grad_Rt     DEVICE float[B*12], row-major like Rt, ACCUMULATED into (zero
+ *               it first for a plain gradient); must not overlap Rt or the
+ *               images.  Per-ray terms are formed in fp64 and summed per CTA
+ *               in fp64, then added with fp32 atomics (order not
+ *               deterministic: the last bits may differ between runs).
+ * Other arguments as drr_render. */
+DRR_API drr_status drr_render_pose_grad(const void *vol, drr_dtype dtype, drr_layout layout,
+                                        const int dims[3], const float spacing[3],
+                                        const float origin[3], const float K[9],
+                                        const float *Rt, int B, int H, int W, int n_samples,
+                                        float density_factor, drr_mode mode,
+                                        const float *grad_out, const float *fwd_out,
+                                        float *grad_Rt, void *stream);
+
 /* Bytes that drr_prepare_volume writes for this volume, dtype and layout
  * (0 if the arguments are invalid or the volume is too large). */
 DRR_API size_t drr_prepared_bytes(const int dims[3], drr_dtype dtype, drr_layout layout);

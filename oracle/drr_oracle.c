@@ -78,14 +78,18 @@ static int make_grid(const int dims[3], const double spacing[3],
     return 0;
 }
 
-/* Step 1: ray of pixel centre (u, v) in world coordinates. */
-static void camera_ray(const double K[9], const double Rt[12], double u, double v,
-                       double C[3], double d[3]) {
-    /* back substitution of K q = (u, v, 1), K = [k0 k1 k2; 0 k4 k5; 0 0 k8] */
-    double q[3];
+/* Back substitution of K q = (u, v, 1), K = [k0 k1 k2; 0 k4 k5; 0 0 k8]. */
+static void back_substitute(const double K[9], double u, double v, double q[3]) {
     q[2] = 1.0 / K[8];
     q[1] = (v - K[5] * q[2]) / K[4];
     q[0] = (u - K[1] * q[1] - K[2] * q[2]) / K[0];
+}
+
+/* Step 1: ray of pixel centre (u, v) in world coordinates. */
+static void camera_ray(const double K[9], const double Rt[12], double u, double v,
+                       double C[3], double d[3]) {
+    double q[3];
+    back_substitute(K, u, v, q);
     double norm2 = 0.0;
     for (int a = 0; a < 3; ++a) {
         /* (R^T q)_a = sum_r R[r][a] q[r]; (R^T t)_a likewise */
@@ -429,9 +433,7 @@ static double ray_pose_grad(const float *vol, const grid_t *g, const double K[9]
     if (!ray_in_volume(g, K, Rt, u, v, Cijk, dijk, &t0, &t1)) return 0.0;
     /* the camera ray again, with the pieces the derivatives need */
     double q[3], a[3], n2 = 0.0;
-    q[2] = 1.0 / K[8];
-    q[1] = (v - K[5] * q[2]) / K[4];
-    q[0] = (u - K[1] * q[1] - K[2] * q[2]) / K[0];
+    back_substitute(K, u, v, q);
     for (int c = 0; c < 3; ++c) {
         a[c] = 0.0;
         for (int r = 0; r < 3; ++r) a[c] += Rt[4 * r + c] * q[r];

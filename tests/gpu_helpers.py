@@ -95,3 +95,39 @@ def assert_parity(got, ref, tol, floor=1e-2, what=""):
     norm, rel = parity_errors(got, ref, floor)
     assert norm <= tol and rel <= tol, f"{what}: normwise {norm:.3g}, per-element {rel:.3g} > {tol}"
     return norm, rel
+
+
+def gpu_pose_grad(w, grad_out, layout=LINEAR, dtype=F32, mode=None, fwd_out=None, accumulate=None):
+    """dL/d[R|t] (B x 3 x 4) through drr_render_pose_grad; ``accumulate`` is an
+    initial value of grad_Rt (zeros by default)."""
+    import torch
+    mode = w.mode if mode is None else mode
+    v32, Rt_d = device_inputs(w)
+    src = prepared(v32, w.dims, dtype, layout)
+    go = torch.from_numpy(np.ascontiguousarray(grad_out, dtype=np.float32)).cuda()
+    fo = None
+    if fwd_out is not None:
+        fo = torch.from_numpy(np.ascontiguousarray(fwd_out, dtype=np.float32)).cuda()
+    init = np.zeros((w.B, 12), np.float32) if accumulate is None else accumulate.reshape(w.B, 12)
+    g = torch.from_numpy(np.ascontiguousarray(init, dtype=np.float32)).cuda()
+    drr.drr_render_pose_grad(src, dtype, layout, w.dims, w.spacing, w.origin, w.K, Rt_d, w.B,
+                             w.H, w.W, w.n_samples, w.density_factor, mode, go, fo, g)
+    torch.cuda.synchronize()
+    return g.cpu().numpy().reshape(w.B, 3, 4)
+
+
+def assert_pose_parity(got, ref, tol, what=""):
+    """Per view, the rotation block and the translation column (different
+    units) each within tol of the oracle, normwise: max|got - ref| / max|ref|."""
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    assert np.all(np.isfinite(got)), f"{what}: non-finite pose gradient"
+    worst = 0.0
+    for b in range(ref.shape[0]):
+        for sl in (np.s_[:, :3], np.s_[:, 3]):
+            scale = np.max(np.abs(ref[b][sl]))
+            err = np.max(np.abs(got[b][sl] - ref[b][sl])) / scale if scale > 0 else np.max(
+                np.abs(got[b][sl]))
+            worst = max(worst, err)
+    assert worst <= tol, f"{what}: pose gradient normwise error {worst:.3g} > {tol}"
+    return worst

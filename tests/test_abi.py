@@ -191,6 +191,43 @@ def test_empty_batch_or_image_is_a_no_op(which):
     assert drr.drr_get_last_error() == ""
 
 
+def _pose(**kw):
+    args = dict(vol=FAKE, dtype=drr.DRR_F32, layout=drr.DRR_LAYOUT_LINEAR, dims=DIMS, spacing=SP,
+                origin=ORG, K=K_OK, Rt=FAKE + (1 << 26), B=2, H=8, W=8, n_samples=16,
+                density_factor=1.0, mode=drr.DRR_MODE_RAW, grad_out=FAKE + (1 << 20),
+                fwd_out=FAKE + (1 << 21), grad_Rt=FAKE + (1 << 27), stream=0)
+    args.update(kw)
+    return drr.drr_render_pose_grad(**args)
+
+
+POSE_BAD = [
+    (dict(dims=(16, 1, 16)), drr.DRR_ERR_INVALID_ARG, "dims"),
+    (dict(mode=3), drr.DRR_ERR_INVALID_ARG, "mode"),
+    (dict(layout=9), drr.DRR_ERR_INVALID_ARG, "layout"),
+    (dict(vol=0), drr.DRR_ERR_INVALID_ARG, "vol"),
+    (dict(layout=drr.DRR_LAYOUT_CORNERS, vol=FAKE + 8), drr.DRR_ERR_INVALID_ARG, "16 bytes"),
+    (dict(grad_out=0), drr.DRR_ERR_INVALID_ARG, "grad_out"),
+    (dict(mode=drr.DRR_MODE_BEER_LAMBERT, fwd_out=0), drr.DRR_ERR_INVALID_ARG, "fwd_out"),
+    (dict(grad_Rt=0), drr.DRR_ERR_INVALID_ARG, "grad_Rt"),
+    (dict(grad_Rt=FAKE + (1 << 26) + 8), drr.DRR_ERR_INVALID_ARG, "overlaps"),   # on Rt
+    (dict(grad_Rt=FAKE + (1 << 20) + 4), drr.DRR_ERR_INVALID_ARG, "overlaps"),   # on grad_out
+    (dict(n_samples=0), drr.DRR_ERR_INVALID_ARG, "n_samples"),
+]
+
+
+@pytest.mark.parametrize("kw,status,word", POSE_BAD)
+def test_pose_gradient_rejects_bad_arguments(kw, status, word):
+    with pytest.raises(drr.DrrError) as e:
+        _pose(**kw)
+    assert e.value.status == status
+    assert word in drr.drr_get_last_error()
+
+
+def test_pose_gradient_empty_batch_is_a_no_op():
+    _pose(B=0, vol=None, grad_out=None, fwd_out=None, grad_Rt=None, Rt=None)
+    assert drr.drr_get_last_error() == ""
+
+
 def test_prepared_bytes():
     assert drr.drr_prepared_bytes((256, 256, 256), drr.DRR_F32, drr.DRR_LAYOUT_LINEAR) == 4 * 256 ** 3
     assert drr.drr_prepared_bytes((256, 256, 256), drr.DRR_BF16, drr.DRR_LAYOUT_LINEAR) == 2 * 256 ** 3
