@@ -37,6 +37,7 @@ import numpy as np
 
 MODE_RAW = 0
 MODE_BEER_LAMBERT = 1
+MODE_ALPHA = 2
 
 DTYPE_F32 = 0
 DTYPE_BF16 = 1

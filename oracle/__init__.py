@@ -9,6 +9,8 @@ from .oracle import (  # noqa: F401
     bf16_to_float,
     build,
     load,
+    poisson_noise,
+    poisson_noise_backward,
     pose_grad,
     ray,
     render,

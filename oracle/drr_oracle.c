@@ -38,6 +38,20 @@
  *     mode (the derivative of 1 - exp(-I)); I is the oracle's own forward.
  *  7. bf16 storage: round-to-nearest-even of the fp32 bit pattern to the
  *     upper 16 bits (the IEEE rounding rule, written out).
+ *  9. Front-to-back alpha compositing, the over operator (flashdrr.rendering
+ *     API docs, VolumeRaycaster.__init__: use_beer_lambert = False, with
+ *     density_factor scaling the intensities before integration), read as
+ *     the emission-absorption sum: sample i has opacity
+ *     a_i = 1 - exp(-density_factor * mu_i * dt) and colour mu_i; with
+ *     T_0 = 1 and T_{i+1} = T_i (1 - a_i) the image is C = sum T_i a_i mu_i,
+ *     summed front (camera side) to back.  Its volume gradient is the
+ *     reverse-mode derivative of that recurrence, accumulated back to front.
+ * 10. Gaussian-Poisson surrogate (flashdrr.rendering API docs,
+ *     VolumeRaycaster.apply_poisson): transmission T' = clamp(T + sqrt(T/i0) z,
+ *     0, 1) with z ~ N(0, 1) given; here applied to a Beer-Lambert image
+ *     1 - T (so T = 1 - image) and returning 1 - T'; its derivative with
+ *     respect to the image is 1 + z / (2 sqrt(T i0)) where the clamp is
+ *     inactive (0 < T + sqrt(T/i0) z < 1, T > 0), else 0.
  *  8. Pose gradient (flashdrr.rendering API docs, VolumeRaycaster: rendering
  *     is differentiable with respect to the view matrices): dL/d[R|t], the
  *     12 entries of each view's world-to-camera matrix taken as free
@@ -60,6 +74,7 @@
 
 #define ORACLE_RAW 0
 #define ORACLE_BEER_LAMBERT 1
+#define ORACLE_ALPHA 2
 
 typedef struct {
     int64_t n[3];         /* nx, ny, nz; i is the fastest index */
@@ -180,6 +195,25 @@ static double apply_mode(double I, int mode) {
     return mode == ORACLE_BEER_LAMBERT ? -expm1(-I) : I;
 }
 
+/* Step 9 for one ray: the front-to-back over operator (0 on a miss). */
+static double ray_alpha(const float *vol, const grid_t *g, const double K[9],
+                        const double Rt[12], double u, double v, int n_samples,
+                        double density_factor) {
+    double C[3], d[3], t0, t1;
+    if (!ray_in_volume(g, K, Rt, u, v, C, d, &t0, &t1)) return 0.0;
+    double dt = (t1 - t0) / (double)n_samples;
+    double T = 1.0, out = 0.0;
+    for (int i = 0; i < n_samples; ++i) {
+        double t = t0 + ((double)i + 0.5) * dt;
+        double p[3] = {C[0] + t * d[0], C[1] + t * d[1], C[2] + t * d[2]};
+        double mu = trilinear(vol, g, p);
+        double a = -expm1(-density_factor * mu * dt);
+        out += T * a * mu;
+        T *= 1.0 - a;
+    }
+    return out;
+}
+
 /* ------------------------------------------------------------------------ */
 /* forward over a list of rays, threaded over contiguous chunks of rays      */
 
@@ -201,6 +235,11 @@ static void *fwd_worker(void *arg) {
         int64_t id = job->ray_ids ? job->ray_ids[n] : n;
         int64_t b = id / hw, rc = id % hw;
         double u = (double)(rc % job->W), v = (double)(rc / job->W);
+        if (job->mode == ORACLE_ALPHA) {
+            job->out[n] = ray_alpha(job->vol, job->g, job->K, job->Rt + 12 * b, u, v,
+                                    job->n_samples, job->density_factor);
+            continue;
+        }
         double dt;
         double I = ray_integral(job->vol, job->g, job->K, job->Rt + 12 * b, u, v,
                                 job->n_samples, job->density_factor, &dt);
@@ -284,6 +323,63 @@ int oracle_trilinear(const float *vol, const int dims[3], const double *p, int64
     return 0;
 }
 
+/* grad += go * w_corner * m at the 8 in-range corners of p. */
+static void scatter(const grid_t *g, const double p[3], double m, double *grad) {
+    double fl[3], f[3];
+    int64_t i0[3];
+    for (int a = 0; a < 3; ++a) {
+        fl[a] = floor(p[a]);
+        f[a] = p[a] - fl[a];
+        i0[a] = (int64_t)fl[a];
+    }
+    for (int dk = 0; dk < 2; ++dk)
+        for (int dj = 0; dj < 2; ++dj)
+            for (int di = 0; di < 2; ++di) {
+                int64_t ii = i0[0] + di, jj = i0[1] + dj, kk = i0[2] + dk;
+                if (ii < 0 || jj < 0 || kk < 0 || ii >= g->n[0] || jj >= g->n[1] || kk >= g->n[2])
+                    continue;
+                double w = (di ? f[0] : 1.0 - f[0]) * (dj ? f[1] : 1.0 - f[1]) *
+                           (dk ? f[2] : 1.0 - f[2]);
+                grad[(kk * g->n[1] + jj) * g->n[0] + ii] += m * w;
+            }
+}
+
+/* Step 9's volume gradient for one ray, by reverse-mode differentiation of
+ * the recurrence C += T_i a_i mu_i, T_{i+1} = T_i (1 - a_i), with
+ * a_i = 1 - exp(-s mu_i), s = density_factor * dt: going back to front with
+ * Tbar = dC/dT_{i+1} (0 after the last sample),
+ *   abar_i  = go T_i mu_i - Tbar T_i
+ *   mubar_i = go T_i a_i + abar_i s (1 - a_i)
+ *   Tbar    <- go a_i mu_i + Tbar (1 - a_i)   (= dC/dT_i)
+ * and mubar_i scattered with the trilinear weights of sample i. */
+static void alpha_ray_adjoint(const float *vol, const grid_t *g, const double C[3],
+                              const double d[3], double t0, double dt, int n_samples,
+                              double density_factor, double go, double *grad) {
+    double *mu = (double *)malloc(sizeof(double) * 3 * (size_t)n_samples);
+    if (!mu) return;
+    double *a = mu + n_samples, *T = a + n_samples;
+    const double s = density_factor * dt;
+    double Tr = 1.0;
+    for (int i = 0; i < n_samples; ++i) {
+        double t = t0 + ((double)i + 0.5) * dt;
+        double p[3] = {C[0] + t * d[0], C[1] + t * d[1], C[2] + t * d[2]};
+        mu[i] = trilinear(vol, g, p);
+        a[i] = -expm1(-s * mu[i]);
+        T[i] = Tr;
+        Tr *= 1.0 - a[i];
+    }
+    double Tbar = 0.0;
+    for (int i = n_samples - 1; i >= 0; --i) {
+        double abar = go * T[i] * mu[i] - Tbar * T[i];
+        double mubar = go * T[i] * a[i] + abar * s * (1.0 - a[i]);
+        Tbar = go * a[i] * mu[i] + Tbar * (1.0 - a[i]);
+        double t = t0 + ((double)i + 0.5) * dt;
+        double p[3] = {C[0] + t * d[0], C[1] + t * d[1], C[2] + t * d[2]};
+        scatter(g, p, mubar, grad);
+    }
+    free(mu);
+}
+
 /* Adjoint of one view: grad[k][j][i] += sum over its rays and samples of
  * g * w_corner, accumulated in order. */
 static void adjoint_view(const float *vol, const grid_t *g, const double K[9],
@@ -297,6 +393,10 @@ static void adjoint_view(const float *vol, const grid_t *g, const double K[9],
             if (go == 0.0) continue;   /* contributes exactly nothing */
             if (!ray_in_volume(g, K, Rt, c, r, C, d, &t0, &t1)) continue;
             double dt = (t1 - t0) / (double)n_samples;
+            if (mode == ORACLE_ALPHA) {
+                alpha_ray_adjoint(vol, g, C, d, t0, dt, n_samples, density_factor, go, grad);
+                continue;
+            }
             double scale = go * density_factor * dt;
             if (mode == ORACLE_BEER_LAMBERT) {
                 double dt2;
@@ -359,7 +459,7 @@ int oracle_adjoint(const float *vol, const int dims[3], const double spacing[3],
     grid_t g;
     if (make_grid(dims, spacing, origin, &g) || B < 0 || H < 0 || W < 0 || n_samples < 1)
         return -1;
-    if (mode == ORACLE_BEER_LAMBERT && vol == NULL) return -1;
+    if ((mode == ORACLE_BEER_LAMBERT || mode == ORACLE_ALPHA) && vol == NULL) return -1;
     if (nthreads > B) nthreads = B;
     if (nthreads > 64) nthreads = 64;
     if (nthreads < 1) nthreads = 1;
@@ -537,6 +637,7 @@ int oracle_pose_grad(const float *vol, const int dims[3], const double spacing[3
     grid_t g;
     if (make_grid(dims, spacing, origin, &g) || B < 0 || H < 0 || W < 0 || n_samples < 1)
         return -1;
+    if (mode != ORACLE_RAW && mode != ORACLE_BEER_LAMBERT) return -1;
     if (nthreads > B) nthreads = B;
     if (nthreads > 64) nthreads = 64;
     if (nthreads < 1) nthreads = 1;
@@ -552,6 +653,37 @@ int oracle_pose_grad(const float *vol, const int dims[3], const double spacing[3
     }
     for (int t = 0; t < nthreads; ++t)
         if (running[t]) pthread_join(tid[t], NULL);
+    return 0;
+}
+
+/* Step 10: out[m] = 1 - clamp(T + sqrt(T / i0) z[m], 0, 1), T = 1 - image[m]. */
+int oracle_poisson_noise(const double *image, const double *z, double i0, double *out,
+                         int64_t n) {
+    if (!(i0 > 0.0)) return -1;
+    for (int64_t m = 0; m < n; ++m) {
+        double T = 1.0 - image[m];
+        double Tn = T > 0.0 ? T + sqrt(T / i0) * z[m] : T;
+        if (Tn < 0.0) Tn = 0.0;
+        if (Tn > 1.0) Tn = 1.0;
+        out[m] = 1.0 - Tn;
+    }
+    return 0;
+}
+
+/* Its derivative: grad_image[m] = grad_out[m] * (1 + z / (2 sqrt(T i0))) where
+ * 0 < T + sqrt(T / i0) z < 1 and T > 0, else 0. */
+int oracle_poisson_noise_backward(const double *image, const double *z, double i0,
+                                  const double *grad_out, double *grad_image, int64_t n) {
+    if (!(i0 > 0.0)) return -1;
+    for (int64_t m = 0; m < n; ++m) {
+        double T = 1.0 - image[m];
+        double slope = 0.0;
+        if (T > 0.0) {
+            double Tn = T + sqrt(T / i0) * z[m];
+            if (Tn > 0.0 && Tn < 1.0) slope = 1.0 + z[m] / (2.0 * sqrt(T * i0));
+        }
+        grad_image[m] = grad_out[m] * slope;
+    }
     return 0;
 }
 

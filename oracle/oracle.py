@@ -46,6 +46,11 @@ def load():
                                      _c.c_int, _c.c_int, _c.c_int, _c.c_double, _c.c_int,
                                      _f64p, _f64p, _c.c_int]
     lib.oracle_pose_grad.restype = _c.c_int
+    lib.oracle_poisson_noise.argtypes = [_f64p, _f64p, _c.c_double, _f64p, _c.c_int64]
+    lib.oracle_poisson_noise.restype = _c.c_int
+    lib.oracle_poisson_noise_backward.argtypes = [_f64p, _f64p, _c.c_double, _f64p, _f64p,
+                                                  _c.c_int64]
+    lib.oracle_poisson_noise_backward.restype = _c.c_int
     lib.oracle_round_bf16.argtypes = [_f32p, _u16p, _c.c_int64]
     lib.oracle_round_bf16.restype = None
     lib.oracle_bf16_to_float.argtypes = [_u16p, _f32p, _c.c_int64]
@@ -119,7 +124,9 @@ def trilinear(vol, dims, points):
 
 def adjoint(dims, spacing, origin, K, Rt, H, W, n_samples, density_factor, mode, grad_out,
             vol=None, nthreads=1):
-    """grad_vol[k][j][i] (float64) = A^T grad_out (times exp(-I) in Beer-Lambert)."""
+    """grad_vol[k][j][i] (float64) = A^T grad_out (times exp(-I) in Beer-Lambert);
+    in alpha mode (2) the volume gradient of the over-operator image, which
+    needs vol."""
     dims, spacing, origin, K, Rt = _geom(dims, spacing, origin, K, Rt)
     B = Rt.shape[0]
     go = np.ascontiguousarray(grad_out, dtype=np.float64).reshape(-1)
@@ -152,6 +159,31 @@ def pose_grad(vol, dims, spacing, origin, K, Rt, H, W, n_samples, density_factor
                                  n_samples, density_factor, mode, go, out, int(nthreads))
     assert rc == 0, "oracle_pose_grad rejected its arguments"
     return out.reshape(B, 3, 4)
+
+
+def poisson_noise(image, z, i0):
+    """1 - clamp(T + sqrt(T / i0) z, 0, 1) with T = 1 - image (float64)."""
+    img = np.ascontiguousarray(image, dtype=np.float64)
+    zz = np.ascontiguousarray(z, dtype=np.float64)
+    assert zz.shape == img.shape
+    out = np.empty_like(img)
+    rc = load().oracle_poisson_noise(img.reshape(-1), zz.reshape(-1), float(i0), out.reshape(-1),
+                                     img.size)
+    assert rc == 0, "oracle_poisson_noise rejected its arguments"
+    return out
+
+
+def poisson_noise_backward(image, z, i0, grad_out):
+    """d/d(image) of poisson_noise, times grad_out (float64)."""
+    img = np.ascontiguousarray(image, dtype=np.float64)
+    zz = np.ascontiguousarray(z, dtype=np.float64)
+    go = np.ascontiguousarray(grad_out, dtype=np.float64)
+    assert zz.shape == img.shape == go.shape
+    gi = np.empty_like(img)
+    rc = load().oracle_poisson_noise_backward(img.reshape(-1), zz.reshape(-1), float(i0),
+                                              go.reshape(-1), gi.reshape(-1), img.size)
+    assert rc == 0, "oracle_poisson_noise_backward rejected its arguments"
+    return gi
 
 
 def round_bf16(x):

@@ -67,6 +67,23 @@ MUTANTS = {
         "double wy = dj ? f[1] : 1.0 - f[1], sy = dj ? -1.0 : 1.0;"),
     "pose gradient without exp(-I) in Beer-Lambert": (
         "double w = go * (j->mode == ORACLE_BEER_LAMBERT ? exp(-I) : 1.0);", "double w = go;"),
+    "alpha colour 1 instead of the intensity": ("out += T * a * mu;", "out += T * a;"),
+    "alpha opacity without dt": (
+        "double a = -expm1(-density_factor * mu * dt);", "double a = -expm1(-density_factor * mu);"),
+    "alpha transmittance not updated": ("T *= 1.0 - a;\n    }\n    return out;",
+                                        "(void)T;\n    }\n    return out;"),
+    "alpha adjoint transmittance term dropped": (
+        "double abar = go * T[i] * mu[i] - Tbar * T[i];", "double abar = go * T[i] * mu[i];"),
+    "alpha adjoint direct term dropped": (
+        "double mubar = go * T[i] * a[i] + abar * s * (1.0 - a[i]);",
+        "double mubar = abar * s * (1.0 - a[i]);"),
+    "noise scale sqrt(T i0) instead of sqrt(T / i0)": (
+        "double Tn = T > 0.0 ? T + sqrt(T / i0) * z[m] : T;",
+        "double Tn = T > 0.0 ? T + sqrt(T * i0) * z[m] : T;"),
+    "noise without the upper clamp": ("        if (Tn > 1.0) Tn = 1.0;\n", ""),
+    "noise derivative without the 1/2": (
+        "if (Tn > 0.0 && Tn < 1.0) slope = 1.0 + z[m] / (2.0 * sqrt(T * i0));",
+        "if (Tn > 0.0 && Tn < 1.0) slope = 1.0 + z[m] / sqrt(T * i0);"),
     "pose gradient translation sign": (
         "for (int k = 0; k < 3; ++k) dC[k] = -Rt[4 * r + k];",
         "for (int k = 0; k < 3; ++k) dC[k] = Rt[4 * r + k];"),
@@ -88,6 +105,7 @@ def test_pins_catch_mutant(name, tmp_path):
     r = subprocess.run([sys.executable, "-m", "pytest",
                         os.path.join(ROOT, "tests", "test_oracle_pins.py"),
                         os.path.join(ROOT, "tests", "test_oracle_pose_pins.py"),
+                        os.path.join(ROOT, "tests", "test_oracle_alpha_noise_pins.py"),
                         "-q", "-x", "-p", "no:cacheprovider"],
                        env=env, cwd=ROOT, capture_output=True, text=True, timeout=600)
     assert r.returncode != 0, f"mutant '{name}' passed every pin:\n{r.stdout[-2000:]}"
