@@ -173,6 +173,9 @@ static double trilinear(const float *vol, const grid_t *g, const double p[3]) {
     return s;
 }
 
+/* Step 4: parameter of sample i, the midpoint of the i-th of N equal parts. */
+static double sample_t(double t0, double dt, int i) { return t0 + ((double)i + 0.5) * dt; }
+
 /* Steps 4-5 for one ray: returns the integral I (0 on a miss). */
 static double ray_integral(const float *vol, const grid_t *g, const double K[9],
                            const double Rt[12], double u, double v, int n_samples,
@@ -183,7 +186,7 @@ static double ray_integral(const float *vol, const grid_t *g, const double K[9],
     double dt = (t1 - t0) / (double)n_samples;
     double sum = 0.0;
     for (int i = 0; i < n_samples; ++i) {
-        double t = t0 + ((double)i + 0.5) * dt;
+        double t = sample_t(t0, dt, i);
         double p[3] = {C[0] + t * d[0], C[1] + t * d[1], C[2] + t * d[2]};
         sum += trilinear(vol, g, p);
     }
@@ -204,7 +207,7 @@ static double ray_alpha(const float *vol, const grid_t *g, const double K[9],
     double dt = (t1 - t0) / (double)n_samples;
     double T = 1.0, out = 0.0;
     for (int i = 0; i < n_samples; ++i) {
-        double t = t0 + ((double)i + 0.5) * dt;
+        double t = sample_t(t0, dt, i);
         double p[3] = {C[0] + t * d[0], C[1] + t * d[1], C[2] + t * d[2]};
         double mu = trilinear(vol, g, p);
         double a = -expm1(-density_factor * mu * dt);
@@ -361,7 +364,7 @@ static void alpha_ray_adjoint(const float *vol, const grid_t *g, const double C[
     const double s = density_factor * dt;
     double Tr = 1.0;
     for (int i = 0; i < n_samples; ++i) {
-        double t = t0 + ((double)i + 0.5) * dt;
+        double t = sample_t(t0, dt, i);
         double p[3] = {C[0] + t * d[0], C[1] + t * d[1], C[2] + t * d[2]};
         mu[i] = trilinear(vol, g, p);
         a[i] = -expm1(-s * mu[i]);
@@ -373,7 +376,7 @@ static void alpha_ray_adjoint(const float *vol, const grid_t *g, const double C[
         double abar = go * T[i] * mu[i] - Tbar * T[i];
         double mubar = go * T[i] * a[i] + abar * s * (1.0 - a[i]);
         Tbar = go * a[i] * mu[i] + Tbar * (1.0 - a[i]);
-        double t = t0 + ((double)i + 0.5) * dt;
+        double t = sample_t(t0, dt, i);
         double p[3] = {C[0] + t * d[0], C[1] + t * d[1], C[2] + t * d[2]};
         scatter(g, p, mubar, grad);
     }
@@ -404,7 +407,7 @@ static void adjoint_view(const float *vol, const grid_t *g, const double K[9],
                 scale *= exp(-I);
             }
             for (int i = 0; i < n_samples; ++i) {
-                double t = t0 + ((double)i + 0.5) * dt;
+                double t = sample_t(t0, dt, i);
                 double p[3] = {C[0] + t * d[0], C[1] + t * d[1], C[2] + t * d[2]};
                 double fl[3], f[3];
                 int64_t i0[3];
@@ -582,7 +585,7 @@ static double ray_pose_grad(const float *vol, const grid_t *g, const double K[9]
         const double ddt = (dt1 - dt0) / (double)n_samples;
         double sum = 0.0, dsum = 0.0;
         for (int i = 0; i < n_samples; ++i) {
-            const double ti = t0 + ((double)i + 0.5) * dt;
+            const double ti = sample_t(t0, dt, i);
             const double dti = dt0 + ((double)i + 0.5) * ddt;
             double p[3], gr[3];
             for (int k = 0; k < 3; ++k) p[k] = Cijk[k] + ti * dijk[k];

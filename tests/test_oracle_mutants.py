@@ -21,8 +21,7 @@ MUTANTS = {
         "(di ? 1.0 - f[0] : f[0]) * (dj ? f[1] : 1.0 - f[1]) *\n"
         "                           (dk ? f[2] : 1.0 - f[2]);\n                s += w"),
     "left-endpoint instead of midpoint samples": (
-        "double t = t0 + ((double)i + 0.5) * dt;\n        double p[3]",
-        "double t = t0 + ((double)i) * dt;\n        double p[3]"),
+        "return t0 + ((double)i + 0.5) * dt;", "return t0 + ((double)i) * dt;"),
     "camera centre sign": ("C[a] = -ca;", "C[a] = ca;"),
     "direction not normalised": ("for (int a = 0; a < 3; ++a) d[a] *= inv;", "(void)inv;"),
     "R instead of R^T": ("da += Rt[4 * r + a] * q[r];", "da += Rt[4 * a + r] * q[r];"),
