@@ -56,6 +56,9 @@ def parse_args():
                    help="also time the texture-trilinear comparison forward (libdrr_texture.so)")
     p.add_argument("--pose", action="store_true",
                    help="also time the pose gradient (drr_render_pose_grad) on the same workload")
+    p.add_argument("--alpha", action="store_true",
+                   help="also time alpha compositing (forward and volume gradient) and the "
+                        "Gaussian-Poisson surrogate on the same workload")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     return p.parse_args()
@@ -396,6 +399,72 @@ def pose_timing(torch, w, prep, dtype, layout, Rt, grad_out, out, elem, l2_peak,
                          "algorithmic_bytes_per_launch": int(nbytes)}}
 
 
+def _median_ms(torch, fn, reps=10, flush=None):
+    stream = torch.cuda.current_stream()
+    times = []
+    for m in range(reps + 3):
+        if flush is not None:
+            flush.fill_(m & 0xFF)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if m >= 3:
+            times.append(e0.elapsed_time(e1))
+    return statistics.median(times)
+
+
+def alpha_timing(torch, w, vol32, prep, dtype, layout, Rt, grad_out, elem, l2_peak, hbm_peak,
+                 vol_fits_l2):
+    """Alpha compositing on the same workload (forward from the prepared
+    volume, volume gradient from it when it is linear or corner records),
+    and the surrogate on its image: median of 10, L2 flushed before each."""
+    from cone_beam_ct_b200 import drr
+    dev = vol32.device
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    out = torch.empty((w.B, w.H, w.W), dtype=torch.float32, device=dev)
+    grad = torch.zeros((w.dims[2], w.dims[1], w.dims[0]), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def fwd():
+        drr.drr_render(prep, dtype, layout, w.dims, w.spacing, w.origin, w.K, Rt, w.B, w.H, w.W,
+                       w.n_samples, w.density_factor, drr.DRR_MODE_ALPHA, out, stream=stream)
+
+    def adj():
+        drr.drr_render_alpha_adjoint(prep, dtype, layout, w.dims, w.spacing, w.origin, w.K, Rt,
+                                     w.B, w.H, w.W, w.n_samples, w.density_factor, grad_out, out,
+                                     grad, stream=stream)
+
+    fwd_ms = _median_ms(torch, fwd, flush=flush)
+    adj_ms = _median_ms(torch, adj, flush=flush) if layout != drr.DRR_LAYOUT_PADDED else None
+    bound, peak = ("l2", l2_peak) if vol_fits_l2 and l2_peak else ("hbm", hbm_peak)
+
+    def roof(kernel, ms, nbytes):
+        a = nbytes / (ms * 1e-3) / 1e9
+        return {"kernel": kernel, "bound": bound, "achieved": a, "peak": peak, "unit": "GB/s",
+                "frac": a / peak, "algorithmic_bytes_per_launch": int(nbytes)}
+
+    z = torch.randn((w.B, w.H, w.W), dtype=torch.float32, device=dev,
+                    generator=torch.Generator(device=dev).manual_seed(5))
+    noisy = torch.empty_like(out)
+    gi = torch.empty_like(out)
+    n = out.numel()
+    noise_ms = _median_ms(torch, lambda: drr.drr_poisson_noise(out, z, 1e4, noisy, stream=stream))
+    noise_bwd_ms = _median_ms(torch, lambda: drr.drr_poisson_noise_backward(
+        out, z, 1e4, grad_out, gi, stream=stream))
+    res = {"forward": {"ms": fwd_ms, "gsamples_s": w.samples / (fwd_ms * 1e-3) / 1e9,
+                       "roofline": roof("forward_kernel<alpha>", fwd_ms, 8 * elem * w.samples)},
+           "density_factor": w.density_factor,
+           "surrogate": {"ms": noise_ms, "backward_ms": noise_bwd_ms,
+                         "hbm_gbs": 12 * n / (noise_ms * 1e-3) / 1e9,
+                         "backward_hbm_gbs": 16 * n / (noise_bwd_ms * 1e-3) / 1e9}}
+    if adj_ms is not None:
+        res["adjoint"] = {"ms": adj_ms, "gsamples_s": w.samples / (adj_ms * 1e-3) / 1e9,
+                          "roofline": roof("alpha_adjoint_kernel", adj_ms, 32 * w.samples)}
+    return res
+
+
 def run_ours(args):
     import torch
     from cone_beam_ct_b200 import drr
@@ -552,6 +621,11 @@ def run_ours(args):
         pose = pose_timing(torch, w, prep, dtype, layout, Rt, grad_out, out, elem, l2_peak,
                            hbm_peak, vol_fits_l2)
 
+    alpha = None
+    if args.alpha:
+        alpha = alpha_timing(torch, w, vol32, prep, dtype, layout, Rt, grad_out, elem, l2_peak,
+                             hbm_peak, vol_fits_l2)
+
     tex = None
     if args.texture:
         tex = texture_comparison(torch, w, vol32, Rt, out)
@@ -579,6 +653,7 @@ def run_ours(args):
         "e2e": e2e,
         "texture_comparison": tex,
         "pose_gradient": pose,
+        "alpha_compositing": alpha,
         "gpu_launches": 7 * args.steps,   # prepare, forward, plan, zero, 2 adjoint paths, gather
         "clocks": clocks,
         "bracket_ms": bracket[0].elapsed_time(bracket[1]),

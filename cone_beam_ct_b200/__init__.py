@@ -11,16 +11,20 @@ from .drr import (  # noqa: F401
     DRR_LAYOUT_CORNERS,
     DRR_LAYOUT_LINEAR,
     DRR_LAYOUT_PADDED,
+    DRR_MODE_ALPHA,
     DRR_MODE_BEER_LAMBERT,
     DRR_MODE_RAW,
     DrrError,
     drr_abi_version,
     drr_adjoint_workspace_bytes,
     drr_get_last_error,
+    drr_poisson_noise,
+    drr_poisson_noise_backward,
     drr_prepare_volume,
     drr_prepared_bytes,
     drr_render,
     drr_render_adjoint,
+    drr_render_alpha_adjoint,
     drr_render_adjoint_noalloc,
     drr_render_adjoint_ws,
     drr_render_pose_grad,

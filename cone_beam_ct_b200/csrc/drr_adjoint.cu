@@ -50,6 +50,7 @@
 #include <mutex>
 
 #include "drr_internal.cuh"
+#include "drr_sample.cuh"
 
 namespace drr {
 
@@ -407,6 +408,87 @@ records_kernel(const float* __restrict__ Rt, const float* __restrict__ grad_out,
     }
 }
 
+// Volume gradient of the alpha-composited image (front to back, the over
+// operator; see march_alpha in drr_forward.cu): C = sum_i T_i a_i mu_i with
+// a_i = 1 - exp(-s mu_i), s = density_factor * dt, T_{i+1} = T_i (1 - a_i).
+// dC/dmu_i has a closed form in quantities known when sample i is reached
+// front to back:
+//   dC/dmu_i = T_i (s (1 - a_i) mu_i + a_i) - s (C - C_i),
+// C_i = sum_{k <= i} T_k a_k mu_k, C the ray's image value (fwd_out) -- the
+// later samples see sample i's absorption through T.  The kernel reads the
+// volume (linear or corner layout: the forward's own sample values), walks
+// each ray once, front to back (no phases: T is sequential), and scatters
+// grad_out * dC/dmu_i * w_corner through the pending 2 x 2 x 2 block of the
+// direct path into the fp32 linear gradient volume.
+template <typename T, int LAYOUT>
+__global__ void __launch_bounds__(kThreads)
+alpha_adjoint_kernel(const T* __restrict__ vol, const float* __restrict__ Rt,
+                     const float* __restrict__ grad_out, const float* __restrict__ fwd_out,
+                     float* __restrict__ grad, const Geom g, int grad_row, int grad_slice) {
+    __shared__ View sv;
+    const int b = blockIdx.z;
+    if (threadIdx.x == 0) view_setup(Rt + 12 * (size_t)b, g, sv);
+    __syncthreads();
+    int r, c;
+    tile_pixel(r, c);
+    if (r >= g.H || c >= g.W) return;
+    const size_t pix = ((size_t)b * g.H + r) * g.W + c;
+    const float go = grad_out[pix];
+    Ray ray;
+    if (go == 0.0f || !ray_setup(sv, g, (double)c, (double)r, 0.0, ray)) return;
+    const float Cray = fwd_out[pix];
+    const float s = g.density_factor * ray.dt;
+    const int st[3] = {1, grad_row, grad_slice};
+    long long qx = ray.q0[0], qy = ray.q0[1], qz = ray.q0[2];
+    int cell[3] = {fix_cell(qx), fix_cell(qy), fix_cell(qz)};
+    float a8[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) a8[k] = 0.0f;
+    float Ci = 0.0f, Tr = 1.0f;
+    for (int i = 0; i < g.N; ++i) {
+        const int cx = fix_cell(qx), cy = fix_cell(qy), cz = fix_cell(qz);
+        const float fx = fix_frac(qx), fy = fix_frac(qy), fz = fix_frac(qz);
+        // the forward's sample value, bit for bit
+        const float mu = LAYOUT == 2
+                             ? sample_corners(vol + (size_t)(cz * g.slice + cy * g.row + cx) * 8, fx, fy, fz)
+                             : trilinear_at(vol + (cz * g.slice + cy * g.row + cx), g.row, g.slice, fx, fy, fz);
+        const float a = -expm1f(-s * mu);
+        Ci = fmaf(Tr * a, mu, Ci);
+        const float dmu = Tr * fmaf(s * (1.0f - a), mu, a) - s * (Cray - Ci);
+        Tr *= 1.0f - a;
+        const float scale = go * dmu;
+        const int dx = cx - cell[0], dy = cy - cell[1], dz = cz - cell[2];
+        if (dx < -1 || dx > 1 || dy < -1 || dy > 1 || dz < -1 || dz > 1) {
+            flush_block(grad, st, cell, a8);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) a8[k] = 0.0f;
+            cell[0] = cx;
+            cell[1] = cy;
+            cell[2] = cz;
+        } else {
+            slide<0>(dx, grad, st, cell, a8);
+            slide<1>(dy, grad, st, cell, a8);
+            slide<2>(dz, grad, st, cell, a8);
+        }
+        const float wz1 = scale * fz, wz0 = scale * (1.0f - fz);
+        const float w00 = wz0 * (1.0f - fy), w01 = wz0 * fy;
+        const float w10 = wz1 * (1.0f - fy), w11 = wz1 * fy;
+        const float gx = 1.0f - fx;
+        a8[0] += w00 * gx;
+        a8[1] += w00 * fx;
+        a8[2] += w01 * gx;
+        a8[3] += w01 * fx;
+        a8[4] += w10 * gx;
+        a8[5] += w10 * fx;
+        a8[6] += w11 * gx;
+        a8[7] += w11 * fx;
+        qx += ray.s[0];
+        qy += ray.s[1];
+        qz += ray.s[2];
+    }
+    flush_block(grad, st, cell, a8);
+}
+
 constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mu;
 void* g_noalloc_addr[kMaxDevices] = {};
@@ -468,6 +550,26 @@ cudaError_t launch_adjoint(const Geom& g, const float* Rt, int mode, const float
     }
     if (workspace)
         gather_records<<<fill_grid, 256, 0, stream>>>(ws.flags, ws.rec, grad_vol, g.nx, g.ny, g.nz);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_alpha_adjoint(const void* vol, int dtype, int layout, const Geom& g,
+                                 const float* Rt, const float* grad_out, const float* fwd_out,
+                                 float* grad_vol, cudaStream_t stream) {
+    const dim3 grid((g.W + kTileW - 1) / kTileW, (g.H + kTileH - 1) / kTileH, g.B);
+    const int grow = g.nx, gslice = g.nx * g.ny;
+    if (dtype == 0 && layout == 2)
+        alpha_adjoint_kernel<float, 2><<<grid, kThreads, 0, stream>>>(
+            static_cast<const float*>(vol), Rt, grad_out, fwd_out, grad_vol, g, grow, gslice);
+    else if (dtype == 0)
+        alpha_adjoint_kernel<float, 0><<<grid, kThreads, 0, stream>>>(
+            static_cast<const float*>(vol), Rt, grad_out, fwd_out, grad_vol, g, grow, gslice);
+    else if (layout == 2)
+        alpha_adjoint_kernel<uint16_t, 2><<<grid, kThreads, 0, stream>>>(
+            static_cast<const uint16_t*>(vol), Rt, grad_out, fwd_out, grad_vol, g, grow, gslice);
+    else
+        alpha_adjoint_kernel<uint16_t, 0><<<grid, kThreads, 0, stream>>>(
+            static_cast<const uint16_t*>(vol), Rt, grad_out, fwd_out, grad_vol, g, grow, gslice);
     return cudaGetLastError();
 }
 

@@ -74,7 +74,7 @@ drr_status check_volume(const int dims[3], const float spacing[3], const float o
 }
 
 drr_status check_rays(const float K[9], const float* Rt, int B, int H, int W, int n_samples,
-                      float density_factor, int mode) {
+                      float density_factor, int mode, bool alpha_ok = false) {
     if (!K) return fail(DRR_ERR_INVALID_ARG, "K must be a non-NULL host array of 9 floats");
     for (int m = 0; m < 9; ++m)
         if (!std::isfinite(K[m])) return fail(DRR_ERR_INVALID_ARG, "K[%d] is not finite", m);
@@ -89,7 +89,11 @@ drr_status check_rays(const float K[9], const float* Rt, int B, int H, int W, in
     if (n_samples < 1 || n_samples > kMaxSamples)
         return fail(DRR_ERR_INVALID_ARG, "n_samples = %d must be in [1, %d]", n_samples, kMaxSamples);
     if (!std::isfinite(density_factor)) return fail(DRR_ERR_INVALID_ARG, "density_factor must be finite");
-    if (mode != DRR_MODE_RAW && mode != DRR_MODE_BEER_LAMBERT)
+    if (mode == DRR_MODE_ALPHA && !alpha_ok)
+        return fail(DRR_ERR_UNSUPPORTED,
+                    "DRR_MODE_ALPHA is not linear in the volume: its gradient needs the volume "
+                    "(drr_render_alpha_adjoint); the pose gradient does not support it");
+    if (mode != DRR_MODE_RAW && mode != DRR_MODE_BEER_LAMBERT && mode != DRR_MODE_ALPHA)
         return fail(DRR_ERR_INVALID_ARG, "unknown mode %d", mode);
     if ((int64_t)B * H * W > 0 && (!Rt || !aligned(Rt, 4)))
         return fail(DRR_ERR_INVALID_ARG, "Rt must be a non-NULL, 4-byte aligned device pointer");
@@ -150,7 +154,7 @@ DRR_API drr_status drr_render(const void* vol, drr_dtype dtype, drr_layout layou
                               void* stream) {
     drr_status st = check_volume(dims, spacing, origin);
     if (st != DRR_OK) return st;
-    st = check_rays(K, Rt, B, H, W, n_samples, density_factor, mode);
+    st = check_rays(K, Rt, B, H, W, n_samples, density_factor, mode, true);
     if (st != DRR_OK) return st;
     if (dtype != DRR_F32 && dtype != DRR_BF16) return fail(DRR_ERR_INVALID_ARG, "unknown dtype %d", dtype);
     if (!known_layout(layout)) return fail(DRR_ERR_INVALID_ARG, "unknown layout %d", layout);
@@ -323,6 +327,84 @@ DRR_API drr_status drr_render_pose_grad(const void* vol, drr_dtype dtype, drr_la
     return cuda_status(drr::launch_pose_grad(vol, dtype, layout, g, Rt, mode, grad_out, fwd_out,
                                              grad_Rt, static_cast<cudaStream_t>(stream)),
                        "drr_render_pose_grad launch");
+}
+
+}  // extern "C"
+
+extern "C" {
+
+DRR_API drr_status drr_render_alpha_adjoint(const void* vol, drr_dtype dtype, drr_layout layout,
+                                            const int dims[3], const float spacing[3],
+                                            const float origin[3], const float K[9],
+                                            const float* Rt, int B, int H, int W, int n_samples,
+                                            float density_factor, const float* grad_out,
+                                            const float* fwd_out, float* grad_vol, void* stream) {
+    drr_status st = check_volume(dims, spacing, origin);
+    if (st != DRR_OK) return st;
+    st = check_rays(K, Rt, B, H, W, n_samples, density_factor, DRR_MODE_ALPHA, true);
+    if (st != DRR_OK) return st;
+    if (dtype != DRR_F32 && dtype != DRR_BF16) return fail(DRR_ERR_INVALID_ARG, "unknown dtype %d", dtype);
+    if (!known_layout(layout)) return fail(DRR_ERR_INVALID_ARG, "unknown layout %d", layout);
+    if (layout == DRR_LAYOUT_PADDED)
+        return fail(DRR_ERR_UNSUPPORTED, "the alpha adjoint reads DRR_LAYOUT_LINEAR or DRR_LAYOUT_CORNERS volumes");
+    if (stored_elements(dims, layout) > kMaxElements)
+        return fail(DRR_ERR_UNSUPPORTED, "volume too large (max 2^31 - 1 stored elements)");
+    const int64_t npix = (int64_t)B * H * W;
+    if (npix == 0) return ok();
+    if (!vol || !aligned(vol, layout_alignment(layout, dtype)))
+        return fail(DRR_ERR_INVALID_ARG, "vol must be a non-NULL device pointer aligned to %zu bytes",
+                    layout_alignment(layout, dtype));
+    if (!grad_out || !aligned(grad_out, 4))
+        return fail(DRR_ERR_INVALID_ARG, "grad_out must be a non-NULL, 4-byte aligned device pointer");
+    if (!fwd_out || !aligned(fwd_out, 4))
+        return fail(DRR_ERR_INVALID_ARG, "fwd_out (the alpha image) is required");
+    if (!grad_vol || !aligned(grad_vol, 4))
+        return fail(DRR_ERR_INVALID_ARG, "grad_vol must be a non-NULL, 4-byte aligned device pointer");
+    const size_t vbytes = (size_t)dims[0] * dims[1] * dims[2] * 4, ibytes = (size_t)npix * 4;
+    const size_t sbytes = (size_t)stored_elements(dims, layout) * (dtype == DRR_F32 ? 4 : 2);
+    if (overlaps(grad_vol, vbytes, grad_out, ibytes) || overlaps(grad_vol, vbytes, fwd_out, ibytes) ||
+        overlaps(grad_vol, vbytes, vol, sbytes))
+        return fail(DRR_ERR_INVALID_ARG, "grad_vol overlaps another buffer");
+    drr::Geom g;
+    drr::fill_geom(g, dims, spacing, origin, K, B, H, W, n_samples, density_factor, layout);
+    return cuda_status(drr::launch_alpha_adjoint(vol, dtype, layout, g, Rt, grad_out, fwd_out,
+                                                 grad_vol, static_cast<cudaStream_t>(stream)),
+                       "drr_render_alpha_adjoint launch");
+}
+
+DRR_API drr_status drr_poisson_noise(const float* image, const float* z, float i0, float* out,
+                                     int64_t n, void* stream) {
+    if (!(i0 > 0.0f) || !std::isfinite(i0))
+        return fail(DRR_ERR_INVALID_ARG, "i0 must be finite and > 0");
+    if (n < 0) return fail(DRR_ERR_INVALID_ARG, "n must be >= 0");
+    if (n == 0) return ok();
+    if (!image || !z || !out || !aligned(image, 4) || !aligned(z, 4) || !aligned(out, 4))
+        return fail(DRR_ERR_INVALID_ARG, "image, z and out must be non-NULL, 4-byte aligned device pointers");
+    const size_t bytes = (size_t)n * 4;
+    if ((out != image && overlaps(out, bytes, image, bytes)) || overlaps(out, bytes, z, bytes))
+        return fail(DRR_ERR_INVALID_ARG, "out overlaps z or part of image (it may be image itself)");
+    return cuda_status(drr::launch_poisson_noise(image, z, i0, out, n, static_cast<cudaStream_t>(stream)),
+                       "drr_poisson_noise launch");
+}
+
+DRR_API drr_status drr_poisson_noise_backward(const float* image, const float* z, float i0,
+                                              const float* grad_out, float* grad_image, int64_t n,
+                                              void* stream) {
+    if (!(i0 > 0.0f) || !std::isfinite(i0))
+        return fail(DRR_ERR_INVALID_ARG, "i0 must be finite and > 0");
+    if (n < 0) return fail(DRR_ERR_INVALID_ARG, "n must be >= 0");
+    if (n == 0) return ok();
+    if (!image || !z || !grad_out || !grad_image || !aligned(image, 4) || !aligned(z, 4) ||
+        !aligned(grad_out, 4) || !aligned(grad_image, 4))
+        return fail(DRR_ERR_INVALID_ARG,
+                    "image, z, grad_out and grad_image must be non-NULL, 4-byte aligned device pointers");
+    const size_t bytes = (size_t)n * 4;
+    if (overlaps(grad_image, bytes, image, bytes) || overlaps(grad_image, bytes, z, bytes) ||
+        (grad_image != grad_out && overlaps(grad_image, bytes, grad_out, bytes)))
+        return fail(DRR_ERR_INVALID_ARG, "grad_image overlaps image, z or part of grad_out");
+    return cuda_status(drr::launch_poisson_noise_backward(image, z, i0, grad_out, grad_image, n,
+                                                          static_cast<cudaStream_t>(stream)),
+                       "drr_poisson_noise_backward launch");
 }
 
 }  // extern "C"

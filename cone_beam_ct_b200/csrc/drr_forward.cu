@@ -5,12 +5,14 @@
 // then n_samples midpoint samples of the zero-padded trilinear interpolant,
 // summed in fp32, then I = density_factor * dt * sum written raw or as
 // 1 - exp(-I) (flashdrr.rendering API docs, VolumeRaycaster.__init__:
-// ray_samples, density_factor, use_beer_lambert).  Nothing per sample is
+// ray_samples, density_factor, use_beer_lambert), or composited front to
+// back (use_beer_lambert = False; march_alpha below).  Nothing per sample is
 // materialised in memory: the fused design the FlashDRR page credits for its
 // near-constant footprint ("Memory Scaling").
 //
-// Two storage layouts, one loop: the caller's linear array, or the array
-// inside a one-voxel zero border (drr_prepare_volume).  Sample positions are
+// Three storage layouts (include/drr.h): the caller's linear array, the
+// array inside a one-voxel zero border, or corner records (drr_sample.cuh
+// reads one sample from each).  Sample positions are
 // 32.32 fixed point (drr_internal.cuh), clipped per ray so that every corner
 // read stays inside the stored volume; inside the voxel-centre box the linear
 // layout's upper corner at n-1 is reached with weight 1 - 2^-32 instead of
@@ -19,43 +21,10 @@
 #include <stdint.h>
 
 #include "drr_internal.cuh"
+#include "drr_sample.cuh"
 
 namespace drr {
 namespace {
-
-template <typename T>
-__device__ __forceinline__ float load_voxel(const T* p);
-
-template <>
-__device__ __forceinline__ float load_voxel<float>(const float* p) {
-    return __ldg(p);
-}
-
-// bf16 voxels are stored as their 16-bit patterns; widening to fp32 is exact.
-template <>
-__device__ __forceinline__ float load_voxel<uint16_t>(const uint16_t* p) {
-    return __uint_as_float(((uint32_t)__ldg(reinterpret_cast<const unsigned short*>(p))) << 16);
-}
-
-template <typename T>
-__device__ __forceinline__ float trilinear_at(const T* __restrict__ base, int row, int slice,
-                                              float fx, float fy, float fz) {
-    const float v000 = load_voxel(base);
-    const float v100 = load_voxel(base + 1);
-    const float v010 = load_voxel(base + row);
-    const float v110 = load_voxel(base + row + 1);
-    const float v001 = load_voxel(base + slice);
-    const float v101 = load_voxel(base + slice + 1);
-    const float v011 = load_voxel(base + slice + row);
-    const float v111 = load_voxel(base + slice + row + 1);
-    const float c00 = fmaf(fx, v100 - v000, v000);
-    const float c10 = fmaf(fx, v110 - v010, v010);
-    const float c01 = fmaf(fx, v101 - v001, v001);
-    const float c11 = fmaf(fx, v111 - v011, v011);
-    const float c0 = fmaf(fy, c10 - c00, c00);
-    const float c1 = fmaf(fy, c11 - c01, c01);
-    return fmaf(fz, c1 - c0, c0);
-}
 
 // Sum of the N samples of one ray.  Every sample lies in [0, g.lim] per axis
 // (ray_setup), so the 8 corners of every sample lie inside the stored volume:
@@ -76,67 +45,6 @@ __device__ __forceinline__ float march(const T* __restrict__ vol, const Geom& g,
         qz += sz;
     }
     return acc;
-}
-
-// One sample in the corner-replicated layout.  A cell record holds corner
-// (a, b, c) -- voxel (i + a, j + b, k + c) -- at element a + 2b + 4c.
-//
-// fp32 records: two 16-byte loads (the corners with c = 0, then c = 1) and
-// scalar lerps.  This path is bound by memory latency; a record order with
-// a as the slowest index (which lets packed lerps start without moves) ran
-// slower here (B200, 512^3 fp32 volume: 5.1 against 4.0 ms; 256^3: 3.07
-// against 2.96 ms).
-__device__ __forceinline__ float sample_corners(const float* __restrict__ p, float fx, float fy,
-                                                float fz) {
-    const float4 lo = __ldg(reinterpret_cast<const float4*>(p));       // c = 0: 000 100 010 110
-    const float4 hi = __ldg(reinterpret_cast<const float4*>(p) + 1);   // c = 1
-    const float c00 = fmaf(fx, lo.y - lo.x, lo.x);
-    const float c10 = fmaf(fx, lo.w - lo.z, lo.z);
-    const float c01 = fmaf(fx, hi.y - hi.x, hi.x);
-    const float c11 = fmaf(fx, hi.w - hi.z, hi.z);
-    const float c0 = fmaf(fy, c10 - c00, c00);
-    const float c1 = fmaf(fy, c11 - c01, c01);
-    return fmaf(fz, c1 - c0, c0);
-}
-
-// bf16 records: one 16-byte load, element 2m in the low half of word m, so
-// word m holds the x pair (a = 0, 1) of corner row m = b + 2c.  Widening a
-// bf16 to fp32 is exact (its bits in the high half): the a = 0 corners are
-// widened with a shift; the x differences take the a = 1 corners as bf16
-// operands of sm_100's mixed-precision subtraction (sub.f32.bf16 widens its
-// bf16 operand exactly and rounds the difference once: the fp32
-// subtraction's result).  The 7 lerps then run as 3 packed fp32x2 steps
-// (sm_100's FFMA2, one instruction for two lanes of fp32 work) on the row
-// pairs (c = 0, c = 1) at b = 0 and b = 1, and one scalar step.  Each lane
-// computes exactly what trilinear_at computes (b - a as fma(a, -1, b), which
-// rounds once like the subtraction), so the corner layout gives the linear
-// layout's bits.
-__device__ __forceinline__ float sub_bf16_f32(unsigned short a, float c) {
-    float d;
-    asm("sub.rn.f32.bf16 %0, %1, %2;" : "=f"(d) : "h"(a), "f"(c));
-    return d;
-}
-
-__device__ __forceinline__ float sample_corners(const uint16_t* __restrict__ p, float fx, float fy,
-                                                float fz) {
-    const uint4 w = __ldg(reinterpret_cast<const uint4*>(p));
-    // a = 0 corners of rows (b, c) = (0, 0), (0, 1) and (1, 0), (1, 1),
-    // widened by a byte permute (low half to high, zeros below) that runs on
-    // the integer pipe rather than the FMA pipe a shift may be issued to
-    const float2 lo0 = make_float2(__uint_as_float(__byte_perm(w.x, 0u, 0x1044)),
-                                   __uint_as_float(__byte_perm(w.z, 0u, 0x1044)));
-    const float2 lo1 = make_float2(__uint_as_float(__byte_perm(w.y, 0u, 0x1044)),
-                                   __uint_as_float(__byte_perm(w.w, 0u, 0x1044)));
-    const float2 d0 = make_float2(sub_bf16_f32((unsigned short)(w.x >> 16), lo0.x),
-                                  sub_bf16_f32((unsigned short)(w.z >> 16), lo0.y));
-    const float2 d1 = make_float2(sub_bf16_f32((unsigned short)(w.y >> 16), lo1.x),
-                                  sub_bf16_f32((unsigned short)(w.w >> 16), lo1.y));
-    const float2 f2 = make_float2(fx, fx);
-    const float2 x0 = __ffma2_rn(f2, d0, lo0);                 // (c00, c01): b = 0, c = 0 / 1
-    const float2 x1 = __ffma2_rn(f2, d1, lo1);                 // (c10, c11): b = 1
-    const float2 m1 = make_float2(-1.0f, -1.0f);
-    const float2 y = __ffma2_rn(make_float2(fy, fy), __ffma2_rn(x0, m1, x1), x0);   // (c0, c1)
-    return fmaf(fz, y.y - y.x, y.x);
 }
 
 // Unroll of the corner-layout sample loop: the largest that ptxas compiles
@@ -165,6 +73,35 @@ __device__ __forceinline__ float march_corners(const T* __restrict__ vol, const 
     return acc;
 }
 
+// Front-to-back alpha compositing of one ray (the over operator; flashdrr
+// rendering API docs, VolumeRaycaster.__init__, use_beer_lambert = False),
+// read as the emission-absorption sum: sample i has opacity
+// a_i = 1 - exp(-s mu_i), s = density_factor * dt, and colour mu_i;
+// C = sum_i T_i a_i mu_i with T_0 = 1, T_{i+1} = T_i (1 - a_i).  The same
+// samples and interpolation as the integral; a_i by expm1f, which keeps its
+// relative accuracy for the small opacities of thin samples.
+template <typename T, int LAYOUT>
+__device__ __forceinline__ float march_alpha(const T* __restrict__ vol, const Geom& g,
+                                             const Ray& ray, float s) {
+    const int row = g.row, slice = g.slice;
+    long long qx = ray.q0[0], qy = ray.q0[1], qz = ray.q0[2];
+    const long long sx = ray.s[0], sy = ray.s[1], sz = ray.s[2];
+    float C = 0.0f, Tr = 1.0f;
+    for (int i = 0; i < g.N; ++i) {
+        const int cell = fix_cell(qz) * slice + fix_cell(qy) * row + fix_cell(qx);
+        const float fx = fix_frac(qx), fy = fix_frac(qy), fz = fix_frac(qz);
+        const float mu = LAYOUT == 2 ? sample_corners(vol + (size_t)cell * 8, fx, fy, fz)
+                                     : trilinear_at(vol + cell, row, slice, fx, fy, fz);
+        const float a = -expm1f(-s * mu);
+        C = fmaf(Tr * a, mu, C);
+        Tr *= 1.0f - a;
+        qx += sx;
+        qy += sy;
+        qz += sz;
+    }
+    return C;
+}
+
 template <typename T, int LAYOUT, int MODE>
 __global__ void __launch_bounds__(kThreads)
 forward_kernel(const T* __restrict__ vol, const float* __restrict__ Rt, float* __restrict__ out,
@@ -179,9 +116,13 @@ forward_kernel(const T* __restrict__ vol, const float* __restrict__ Rt, float* _
     Ray ray;
     float result = 0.0f;
     if (ray_setup(sv, g, (double)c, (double)r, LAYOUT == 1 ? 1.0 : 0.0, ray)) {
-        const float sum = LAYOUT == 2 ? march_corners(vol, g, ray) : march(vol, g, ray);
-        const float I = (g.density_factor * ray.dt) * sum;
-        result = (MODE == 1) ? -expm1f(-I) : I;
+        if (MODE == 2) {
+            result = march_alpha<T, LAYOUT>(vol, g, ray, g.density_factor * ray.dt);
+        } else {
+            const float sum = LAYOUT == 2 ? march_corners(vol, g, ray) : march(vol, g, ray);
+            const float I = (g.density_factor * ray.dt) * sum;
+            result = (MODE == 1) ? -expm1f(-I) : I;
+        }
     }
     out[((size_t)b * g.H + r) * g.W + c] = result;
 }
@@ -191,7 +132,9 @@ cudaError_t launch_typed(const void* vol, const Geom& g, const float* Rt, int mo
                          cudaStream_t stream) {
     const dim3 grid((g.W + kTileW - 1) / kTileW, (g.H + kTileH - 1) / kTileH, g.B);
     const T* v = static_cast<const T*>(vol);
-    if (mode == 1)
+    if (mode == 2)
+        forward_kernel<T, LAYOUT, 2><<<grid, kThreads, 0, stream>>>(v, Rt, out, g);
+    else if (mode == 1)
         forward_kernel<T, LAYOUT, 1><<<grid, kThreads, 0, stream>>>(v, Rt, out, g);
     else
         forward_kernel<T, LAYOUT, 0><<<grid, kThreads, 0, stream>>>(v, Rt, out, g);

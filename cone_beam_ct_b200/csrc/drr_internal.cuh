@@ -220,6 +220,14 @@ cudaError_t launch_adjoint_noalloc(const Geom& g, const float* Rt, int mode, con
                                    const float* fwd_out, float* grad_vol, cudaStream_t stream);
 cudaError_t launch_prepare(const float* src, int nx, int ny, int nz, int dtype, int layout,
                            void* dst, cudaStream_t stream);
+cudaError_t launch_alpha_adjoint(const void* vol, int dtype, int layout, const Geom& g,
+                                 const float* Rt, const float* grad_out, const float* fwd_out,
+                                 float* grad_vol, cudaStream_t stream);
+cudaError_t launch_poisson_noise(const float* image, const float* z, float i0, float* out,
+                                 int64_t n, cudaStream_t stream);
+cudaError_t launch_poisson_noise_backward(const float* image, const float* z, float i0,
+                                          const float* grad_out, float* grad_image, int64_t n,
+                                          cudaStream_t stream);
 cudaError_t launch_pose_grad(const void* vol, int dtype, int layout, const Geom& g,
                              const float* Rt, int mode, const float* grad_out,
                              const float* fwd_out, float* grad_Rt, cudaStream_t stream);

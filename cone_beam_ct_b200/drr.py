@@ -15,13 +15,14 @@ import numpy as np
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libdrr.so")
 
 DRR_OK, DRR_ERR_INVALID_ARG, DRR_ERR_UNSUPPORTED, DRR_ERR_CUDA = 0, 1, 2, 3
-DRR_MODE_RAW, DRR_MODE_BEER_LAMBERT = 0, 1
+DRR_MODE_RAW, DRR_MODE_BEER_LAMBERT, DRR_MODE_ALPHA = 0, 1, 2
 DRR_F32, DRR_BF16 = 0, 1
 DRR_LAYOUT_LINEAR, DRR_LAYOUT_PADDED, DRR_LAYOUT_CORNERS = 0, 1, 2
 
 # names exported by libdrr.so (include/drr.h)
 EXPORTED = ("drr_render", "drr_render_adjoint", "drr_render_adjoint_ws",
             "drr_adjoint_workspace_bytes", "drr_render_adjoint_noalloc", "drr_render_pose_grad",
+            "drr_render_alpha_adjoint", "drr_poisson_noise", "drr_poisson_noise_backward",
             "drr_prepared_bytes", "drr_prepare_volume", "drr_get_last_error", "drr_abi_version")
 DRR_NOALLOC_SCRATCH_BYTES = 32 << 20
 
@@ -67,6 +68,14 @@ def lib():
                                        _c.c_int, _c.c_int, _c.c_int, _c.c_int, _c.c_float,
                                        _c.c_int, _vp, _vp, _vp, _vp]
     L.drr_render_pose_grad.restype = _c.c_int
+    L.drr_render_alpha_adjoint.argtypes = [_vp, _c.c_int, _c.c_int, _i3, _f3, _f3, _f9, _vp,
+                                           _c.c_int, _c.c_int, _c.c_int, _c.c_int, _c.c_float,
+                                           _vp, _vp, _vp, _vp]
+    L.drr_render_alpha_adjoint.restype = _c.c_int
+    L.drr_poisson_noise.argtypes = [_vp, _vp, _c.c_float, _vp, _c.c_int64, _vp]
+    L.drr_poisson_noise.restype = _c.c_int
+    L.drr_poisson_noise_backward.argtypes = [_vp, _vp, _c.c_float, _vp, _vp, _c.c_int64, _vp]
+    L.drr_poisson_noise_backward.restype = _c.c_int
     L.drr_adjoint_workspace_bytes.argtypes = [_i3, _c.c_int]
     L.drr_adjoint_workspace_bytes.restype = _c.c_size_t
     L.drr_prepared_bytes.argtypes = [_i3, _c.c_int, _c.c_int]
@@ -177,6 +186,31 @@ def drr_render_pose_grad(vol, dtype, layout, dims, spacing, origin, K, Rt, B, H,
                                       _dev(grad_out, "grad_out", True),
                                       _dev(fwd_out, "fwd_out", True),
                                       _dev(grad_Rt, "grad_Rt", True), _stream(stream)))
+
+
+def drr_render_alpha_adjoint(vol, dtype, layout, dims, spacing, origin, K, Rt, B, H, W,
+                             n_samples, density_factor, grad_out, fwd_out, grad_vol, stream=None):
+    _check(lib().drr_render_alpha_adjoint(_dev(vol, "vol", True), int(dtype), int(layout),
+                                          _i3v(dims), _f3v(spacing), _f3v(origin), _f9v(K),
+                                          _dev(Rt, "Rt", True), int(B), int(H), int(W),
+                                          int(n_samples), float(density_factor),
+                                          _dev(grad_out, "grad_out", True),
+                                          _dev(fwd_out, "fwd_out", True),
+                                          _dev(grad_vol, "grad_vol", True), _stream(stream)))
+
+
+def drr_poisson_noise(image, z, i0, out, n=None, stream=None):
+    n = image.numel() if n is None else n
+    _check(lib().drr_poisson_noise(_dev(image, "image", True), _dev(z, "z", True), float(i0),
+                                   _dev(out, "out", True), int(n), _stream(stream)))
+
+
+def drr_poisson_noise_backward(image, z, i0, grad_out, grad_image, n=None, stream=None):
+    n = image.numel() if n is None else n
+    _check(lib().drr_poisson_noise_backward(_dev(image, "image", True), _dev(z, "z", True),
+                                            float(i0), _dev(grad_out, "grad_out", True),
+                                            _dev(grad_image, "grad_image", True), int(n),
+                                            _stream(stream)))
 
 
 def drr_adjoint_workspace_bytes(dims, B):

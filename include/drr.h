@@ -58,6 +58,7 @@
 #define DRR_H
 
 #include <stddef.h>
+#include <stdint.h>
 
 #ifdef __cplusplus
 extern "C" {
@@ -78,7 +79,15 @@ typedef enum {
 
 typedef enum {
     DRR_MODE_RAW = 0,          /* out = I */
-    DRR_MODE_BEER_LAMBERT = 1  /* out = 1 - exp(-I), evaluated as -expm1(-I) */
+    DRR_MODE_BEER_LAMBERT = 1, /* out = 1 - exp(-I), evaluated as -expm1(-I) */
+    /* Front-to-back alpha compositing, the over operator (flashdrr.rendering
+       API docs, VolumeRaycaster.__init__: use_beer_lambert = False), read as
+       the emission-absorption sum: sample i has opacity
+       a_i = 1 - exp(-density_factor * mu_i * dt) and colour mu_i, and
+       out = sum_i T_i a_i mu_i with T_0 = 1, T_{i+1} = T_i (1 - a_i), summed
+       from the camera side.  drr_render only; its volume gradient is
+       drr_render_alpha_adjoint (it is not linear in the volume). */
+    DRR_MODE_ALPHA = 2
 } drr_mode;
 
 typedef enum {
@@ -114,7 +123,7 @@ typedef enum {
  *               nothing to do, DRR_OK); B <= 65535.
  *   n_samples   samples per ray, 1 <= n_samples <= 1048576.
  *   density_factor  finite scale of the integral.
- *   mode        DRR_MODE_RAW or DRR_MODE_BEER_LAMBERT.
+ *   mode        DRR_MODE_RAW, DRR_MODE_BEER_LAMBERT or DRR_MODE_ALPHA.
  *   out         DEVICE float[B*H*W], overwritten.
  * Limits: the stored volume must hold fewer than 2^31 elements (PADDED:
  * with its border; CORNERS: 8 per cell); B*H*W < 2^40.  A CORNERS volume
@@ -137,7 +146,8 @@ DRR_API drr_status drr_render(const void *vol, drr_dtype dtype, drr_layout layou
  *               into with atomic adds (zero it first for a plain gradient).
  *               The order of the atomic adds is not deterministic, so results
  *               may differ between runs in the last bits.
- * Other arguments as drr_render.  grad_vol must not overlap the images.
+ * Other arguments as drr_render; mode DRR_MODE_ALPHA is DRR_ERR_UNSUPPORTED
+ * here (see drr_render_alpha_adjoint).  grad_vol must not overlap the images.
  */
 DRR_API drr_status drr_render_adjoint(const int dims[3], const float spacing[3],
                                       const float origin[3], const float K[9], const float *Rt,
@@ -236,6 +246,47 @@ DRR_API drr_status drr_render_pose_grad(const void *vol, drr_dtype dtype, drr_la
                                         float density_factor, drr_mode mode,
                                         const float *grad_out, const float *fwd_out,
                                         float *grad_Rt, void *stream);
+
+/* Volume gradient of a DRR_MODE_ALPHA image: grad_vol += d(sum grad_out *
+ * out)/d vol.  With C_i the composite up to and including sample i and C the
+ * ray's image value, dC/dmu_i = T_i (s (1 - a_i) mu_i + a_i) - s (C - C_i),
+ * s = density_factor * dt; each sample's value is scattered with its
+ * trilinear weights.  One pass per ray, front to back.
+ *   vol, dtype, layout  the forward's volume: DRR_LAYOUT_LINEAR or
+ *               DRR_LAYOUT_CORNERS (DRR_LAYOUT_PADDED: DRR_ERR_UNSUPPORTED).
+ *   grad_out    DEVICE float[B*H*W], upstream gradient dL/d(out).
+ *   fwd_out     DEVICE float[B*H*W], the alpha image of this volume and these
+ *               poses (drr_render with DRR_MODE_ALPHA), required.
+ *   grad_vol    DEVICE float32 [nz][ny][nx], ACCUMULATED into (atomic adds,
+ *               order not deterministic); must not overlap the other buffers.
+ * Other arguments as drr_render. */
+DRR_API drr_status drr_render_alpha_adjoint(const void *vol, drr_dtype dtype, drr_layout layout,
+                                            const int dims[3], const float spacing[3],
+                                            const float origin[3], const float K[9],
+                                            const float *Rt, int B, int H, int W, int n_samples,
+                                            float density_factor, const float *grad_out,
+                                            const float *fwd_out, float *grad_vol, void *stream);
+
+/* Gaussian-Poisson surrogate of shot noise (flashdrr.rendering API docs,
+ * VolumeRaycaster.apply_poisson) on a Beer-Lambert image: with transmission
+ * T = 1 - image, T' = clamp(T + sqrt(T / i0) z, 0, 1) and out = 1 - T'.
+ *   image   DEVICE float[n], a Beer-Lambert image (values in [0, 1]).
+ *   z       DEVICE float[n], standard normal draws (the caller's generator).
+ *   i0      mean photon count at the source, finite and > 0.
+ *   out     DEVICE float[n]; may be image itself (in place), must not
+ *           overlap z or only part of image.
+ * n == 0 is a no-op. */
+DRR_API drr_status drr_poisson_noise(const float *image, const float *z, float i0, float *out,
+                                     int64_t n, void *stream);
+
+/* Its derivative: grad_image = grad_out * (1 + z / (2 sqrt(T i0))) where the
+ * clamp is inactive (0 < T + sqrt(T / i0) z < 1, T > 0), else 0.
+ *   grad_image  DEVICE float[n], overwritten; may be grad_out itself, must not
+ *               overlap image or z.
+ * Other arguments as drr_poisson_noise. */
+DRR_API drr_status drr_poisson_noise_backward(const float *image, const float *z, float i0,
+                                              const float *grad_out, float *grad_image,
+                                              int64_t n, void *stream);
 
 /* Bytes that drr_prepare_volume writes for this volume, dtype and layout
  * (0 if the arguments are invalid or the volume is too large). */

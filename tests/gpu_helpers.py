@@ -131,3 +131,18 @@ def assert_pose_parity(got, ref, tol, what=""):
             worst = max(worst, err)
     assert worst <= tol, f"{what}: pose gradient normwise error {worst:.3g} > {tol}"
     return worst
+
+
+def gpu_alpha_adjoint(w, grad_out, fwd_out, layout=LINEAR, dtype=F32):
+    """Volume gradient of the alpha image through drr_render_alpha_adjoint."""
+    import torch
+    v32, Rt_d = device_inputs(w)
+    src = prepared(v32, w.dims, dtype, layout)
+    go = torch.from_numpy(np.ascontiguousarray(grad_out, dtype=np.float32)).cuda()
+    fo = torch.from_numpy(np.ascontiguousarray(fwd_out, dtype=np.float32)).cuda()
+    nx, ny, nz = w.dims
+    grad = torch.zeros((nz, ny, nx), dtype=torch.float32, device="cuda")
+    drr.drr_render_alpha_adjoint(src, dtype, layout, w.dims, w.spacing, w.origin, w.K, Rt_d, w.B,
+                                 w.H, w.W, w.n_samples, w.density_factor, go, fo, grad)
+    torch.cuda.synchronize()
+    return grad.cpu().numpy()

@@ -99,7 +99,7 @@ RENDER_BAD = [
     (dict(n_samples=0), drr.DRR_ERR_INVALID_ARG, "n_samples"),
     (dict(n_samples=(1 << 20) + 1), drr.DRR_ERR_INVALID_ARG, "n_samples"),
     (dict(density_factor=float("inf")), drr.DRR_ERR_INVALID_ARG, "density_factor"),
-    (dict(mode=2), drr.DRR_ERR_INVALID_ARG, "mode"),
+    (dict(mode=3), drr.DRR_ERR_INVALID_ARG, "mode"),
     (dict(dtype=7), drr.DRR_ERR_INVALID_ARG, "dtype"),
     (dict(layout=5), drr.DRR_ERR_INVALID_ARG, "layout"),
     (dict(vol=0), drr.DRR_ERR_INVALID_ARG, "vol"),
@@ -129,6 +129,7 @@ ADJOINT_BAD = [
     (dict(grad_vol=FAKE + (1 << 20)), drr.DRR_ERR_INVALID_ARG),    # overlaps grad_out
     (dict(K=[500.0, 0, 99.5, 0, 500.0, 99.5, 0.5, 0, 1]), drr.DRR_ERR_INVALID_ARG),
     (dict(mode=-1), drr.DRR_ERR_INVALID_ARG),
+    (dict(mode=drr.DRR_MODE_ALPHA), drr.DRR_ERR_UNSUPPORTED),      # needs the volume
 ]
 
 
@@ -212,6 +213,7 @@ POSE_BAD = [
     (dict(grad_Rt=FAKE + (1 << 26) + 8), drr.DRR_ERR_INVALID_ARG, "overlaps"),   # on Rt
     (dict(grad_Rt=FAKE + (1 << 20) + 4), drr.DRR_ERR_INVALID_ARG, "overlaps"),   # on grad_out
     (dict(n_samples=0), drr.DRR_ERR_INVALID_ARG, "n_samples"),
+    (dict(mode=drr.DRR_MODE_ALPHA), drr.DRR_ERR_UNSUPPORTED, "pose gradient"),
 ]
 
 
@@ -226,6 +228,65 @@ def test_pose_gradient_rejects_bad_arguments(kw, status, word):
 def test_pose_gradient_empty_batch_is_a_no_op():
     _pose(B=0, vol=None, grad_out=None, fwd_out=None, grad_Rt=None, Rt=None)
     assert drr.drr_get_last_error() == ""
+
+
+def _alpha_adjoint(**kw):
+    args = dict(vol=FAKE, dtype=drr.DRR_F32, layout=drr.DRR_LAYOUT_LINEAR, dims=DIMS, spacing=SP,
+                origin=ORG, K=K_OK, Rt=FAKE + (1 << 26), B=2, H=8, W=8, n_samples=16,
+                density_factor=1.0, grad_out=FAKE + (1 << 20), fwd_out=FAKE + (1 << 21),
+                grad_vol=FAKE + (1 << 24), stream=0)
+    args.update(kw)
+    return drr.drr_render_alpha_adjoint(**args)
+
+
+ALPHA_BAD = [
+    (dict(layout=drr.DRR_LAYOUT_PADDED), drr.DRR_ERR_UNSUPPORTED, "LINEAR"),
+    (dict(fwd_out=0), drr.DRR_ERR_INVALID_ARG, "alpha image"),
+    (dict(grad_out=0), drr.DRR_ERR_INVALID_ARG, "grad_out"),
+    (dict(grad_vol=0), drr.DRR_ERR_INVALID_ARG, "grad_vol"),
+    (dict(vol=0), drr.DRR_ERR_INVALID_ARG, "vol"),
+    (dict(grad_vol=FAKE), drr.DRR_ERR_INVALID_ARG, "overlaps"),        # on the volume
+    (dict(dims=(16, 16, 0)), drr.DRR_ERR_INVALID_ARG, "dims"),
+]
+
+
+@pytest.mark.parametrize("kw,status,word", ALPHA_BAD)
+def test_alpha_adjoint_rejects_bad_arguments(kw, status, word):
+    with pytest.raises(drr.DrrError) as e:
+        _alpha_adjoint(**kw)
+    assert e.value.status == status
+    assert word in drr.drr_get_last_error()
+
+
+NOISE_BAD = [
+    (dict(i0=0.0), "i0"),
+    (dict(i0=float("inf")), "i0"),
+    (dict(n=-1), "n must"),
+    (dict(z=0), "non-NULL"),
+    (dict(out=FAKE + 4), "overlaps"),          # part of image
+    (dict(out=FAKE + (1 << 20)), "overlaps"),  # z
+]
+
+
+@pytest.mark.parametrize("kw,word", NOISE_BAD)
+def test_noise_rejects_bad_arguments(kw, word):
+    args = dict(image=FAKE, z=FAKE + (1 << 20), i0=100.0, out=FAKE + (1 << 21), n=1000, stream=0)
+    args.update(kw)
+    with pytest.raises(drr.DrrError) as e:
+        drr.drr_poisson_noise(**args)
+    assert e.value.status == drr.DRR_ERR_INVALID_ARG
+    assert word in drr.drr_get_last_error()
+
+
+def test_noise_backward_rejects_bad_arguments():
+    args = dict(image=FAKE, z=FAKE + (1 << 20), i0=100.0, grad_out=FAKE + (1 << 21),
+                grad_image=FAKE + (1 << 22), n=1000, stream=0)
+    for kw in (dict(i0=-1.0), dict(grad_image=FAKE + 8), dict(grad_out=0)):
+        with pytest.raises(drr.DrrError) as e:
+            drr.drr_poisson_noise_backward(**dict(args, **kw))
+        assert e.value.status == drr.DRR_ERR_INVALID_ARG
+    drr.drr_poisson_noise(FAKE, FAKE, 1.0, FAKE, n=0, stream=0)           # empty: no-op
+    drr.drr_poisson_noise_backward(FAKE, FAKE, 1.0, FAKE, FAKE, n=0, stream=0)
 
 
 def test_prepared_bytes():
