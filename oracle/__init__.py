@@ -15,6 +15,8 @@ from .oracle import (  # noqa: F401
     ray,
     render,
     render_rays,
+    render_siddon,
     round_bf16,
+    siddon_adjoint,
     trilinear,
 )

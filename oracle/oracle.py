@@ -51,6 +51,13 @@ def load():
     lib.oracle_poisson_noise_backward.argtypes = [_f64p, _f64p, _c.c_double, _f64p, _f64p,
                                                   _c.c_int64]
     lib.oracle_poisson_noise_backward.restype = _c.c_int
+    lib.oracle_render_siddon.argtypes = [_f32p, _i32p, _f64p, _f64p, _f64p, _f64p, _c.c_int,
+                                         _c.c_int, _c.c_int, _c.c_double, _c.c_int, _f64p]
+    lib.oracle_render_siddon.restype = _c.c_int
+    lib.oracle_siddon_adjoint.argtypes = [_c.c_void_p, _i32p, _f64p, _f64p, _f64p, _f64p,
+                                          _c.c_int, _c.c_int, _c.c_int, _c.c_double, _c.c_int,
+                                          _f64p, _f64p]
+    lib.oracle_siddon_adjoint.restype = _c.c_int
     lib.oracle_round_bf16.argtypes = [_f32p, _u16p, _c.c_int64]
     lib.oracle_round_bf16.restype = None
     lib.oracle_bf16_to_float.argtypes = [_u16p, _f32p, _c.c_int64]
@@ -184,6 +191,33 @@ def poisson_noise_backward(image, z, i0, grad_out):
                                               go.reshape(-1), gi.reshape(-1), img.size)
     assert rc == 0, "oracle_poisson_noise_backward rejected its arguments"
     return gi
+
+
+def render_siddon(vol, dims, spacing, origin, K, Rt, H, W, density_factor, mode):
+    """Cell-constant (Siddon) image out[b][r][c] (float64), RAW or Beer-Lambert."""
+    dims, spacing, origin, K, Rt = _geom(dims, spacing, origin, K, Rt)
+    B = Rt.shape[0]
+    out = np.zeros(B * H * W, dtype=np.float64)
+    rc = load().oracle_render_siddon(_vol(vol, dims), dims, spacing, origin, K, Rt.reshape(-1),
+                                     B, H, W, density_factor, mode, out)
+    assert rc == 0, "oracle_render_siddon rejected its arguments"
+    return out.reshape(B, H, W)
+
+
+def siddon_adjoint(dims, spacing, origin, K, Rt, H, W, density_factor, mode, grad_out, vol=None):
+    """Backprojection of the cell-constant model (float64 [nz][ny][nx])."""
+    dims, spacing, origin, K, Rt = _geom(dims, spacing, origin, K, Rt)
+    B = Rt.shape[0]
+    go = np.ascontiguousarray(grad_out, dtype=np.float64).reshape(-1)
+    assert go.size == B * H * W
+    grad = np.zeros(int(np.prod(dims)), dtype=np.float64)
+    keep = _vol(vol, dims) if vol is not None else None
+    rc = load().oracle_siddon_adjoint(None if keep is None else keep.ctypes.data, dims, spacing,
+                                      origin, K, Rt.reshape(-1), B, H, W, density_factor, mode,
+                                      go, grad)
+    assert rc == 0, "oracle_siddon_adjoint rejected its arguments"
+    nx, ny, nz = (int(x) for x in dims)
+    return grad.reshape(nz, ny, nx)
 
 
 def round_bf16(x):

@@ -83,6 +83,17 @@ MUTANTS = {
     "noise derivative without the 1/2": (
         "if (Tn > 0.0 && Tn < 1.0) slope = 1.0 + z[m] / (2.0 * sqrt(T * i0));",
         "if (Tn > 0.0 && Tn < 1.0) slope = 1.0 + z[m] / sqrt(T * i0);"),
+    "siddon cell by floor instead of the nearest centre": (
+        "int64_t k = (int64_t)floor(p[a] + 0.5);", "int64_t k = (int64_t)floor(p[a]);"),
+    "siddon box of voxel centres instead of cells": (
+        "double lo = -0.5, hi = (double)g->n[a] - 0.5;", "double lo = 0.0, hi = (double)(g->n[a] - 1);"),
+    "siddon crossings unsorted": (
+        "qsort(ts + 1, (size_t)(m - 1), sizeof(double), cmp_double);", "(void)cmp_double;"),
+    "siddon last interior plane missed": (
+        "for (int64_t k = 0; k + 1 < g->n[a]; ++k) {", "for (int64_t k = 0; k + 2 < g->n[a]; ++k) {"),
+    "siddon backprojection without density_factor": (
+        "double scale = go * density_factor;\n                if (mode == ORACLE_BEER_LAMBERT)\n                    scale *= exp(-ray_siddon",
+        "double scale = go;\n                if (mode == ORACLE_BEER_LAMBERT)\n                    scale *= exp(-ray_siddon"),
     "pose gradient translation sign": (
         "for (int k = 0; k < 3; ++k) dC[k] = -Rt[4 * r + k];",
         "for (int k = 0; k < 3; ++k) dC[k] = Rt[4 * r + k];"),
@@ -105,6 +116,7 @@ def test_pins_catch_mutant(name, tmp_path):
                         os.path.join(ROOT, "tests", "test_oracle_pins.py"),
                         os.path.join(ROOT, "tests", "test_oracle_pose_pins.py"),
                         os.path.join(ROOT, "tests", "test_oracle_alpha_noise_pins.py"),
+                        os.path.join(ROOT, "tests", "test_oracle_siddon_pins.py"),
                         "-q", "-x", "-p", "no:cacheprovider"],
                        env=env, cwd=ROOT, capture_output=True, text=True, timeout=600)
     assert r.returncode != 0, f"mutant '{name}' passed every pin:\n{r.stdout[-2000:]}"
