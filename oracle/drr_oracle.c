@@ -130,17 +130,19 @@ static void camera_ray(const double K[9], const double Rt[12], double u, double 
     for (int a = 0; a < 3; ++a) d[a] *= inv;
 }
 
-/* Steps 2-3: ray in IJK and its clipped parameter range; returns 1 on hit. */
-static int ray_in_volume(const grid_t *g, const double K[9], const double Rt[12],
-                         double u, double v, double Cijk[3], double dijk[3],
-                         double *t0, double *t1) {
+/* Steps 2-3: ray in IJK, clipped to the box [lo, lo + n - 1 + 2 pad] per
+ * axis with lo = -pad (pad 0: the voxel centres; 1/2: the cells of the
+ * cell-constant model); returns 1 on a hit. */
+static int ray_in_box(const grid_t *g, const double K[9], const double Rt[12], double u,
+                      double v, double pad, double Cijk[3], double dijk[3], double *t0,
+                      double *t1) {
     double C[3], d[3];
     camera_ray(K, Rt, u, v, C, d);
     double t_near = -INFINITY, t_far = INFINITY;
     for (int a = 0; a < 3; ++a) {
         Cijk[a] = (C[a] - g->origin[a]) / g->spacing[a];
         dijk[a] = d[a] / g->spacing[a];
-        double lo = 0.0, hi = (double)(g->n[a] - 1);
+        double lo = 0.0 - pad, hi = (double)(g->n[a] - 1) + pad;
         if (dijk[a] == 0.0) {
             if (Cijk[a] < lo || Cijk[a] > hi) return 0;
             continue;
@@ -155,6 +157,11 @@ static int ray_in_volume(const grid_t *g, const double K[9], const double Rt[12]
     *t0 = t_near > 0.0 ? t_near : 0.0;
     *t1 = t_far;
     return (*t1 > *t0) ? 1 : 0;
+}
+
+static int ray_in_volume(const grid_t *g, const double K[9], const double Rt[12], double u,
+                         double v, double Cijk[3], double dijk[3], double *t0, double *t1) {
+    return ray_in_box(g, K, Rt, u, v, 0.0, Cijk, dijk, t0, t1);
 }
 
 static double voxel(const float *vol, const grid_t *g, int64_t i, int64_t j, int64_t k) {
@@ -674,27 +681,7 @@ int oracle_pose_grad(const float *vol, const int dims[3], const double spacing[3
 /* The ray clipped to the cells' box [-1/2, n - 1/2]; returns 1 on a hit. */
 static int ray_in_cells(const grid_t *g, const double K[9], const double Rt[12], double u,
                         double v, double Cijk[3], double dijk[3], double *t0, double *t1) {
-    double C[3], d[3];
-    camera_ray(K, Rt, u, v, C, d);
-    double t_near = -INFINITY, t_far = INFINITY;
-    for (int a = 0; a < 3; ++a) {
-        Cijk[a] = (C[a] - g->origin[a]) / g->spacing[a];
-        dijk[a] = d[a] / g->spacing[a];
-        double lo = -0.5, hi = (double)g->n[a] - 0.5;
-        if (dijk[a] == 0.0) {
-            if (Cijk[a] < lo || Cijk[a] > hi) return 0;
-            continue;
-        }
-        double tA = (lo - Cijk[a]) / dijk[a];
-        double tB = (hi - Cijk[a]) / dijk[a];
-        double tmin = tA < tB ? tA : tB;
-        double tmax = tA < tB ? tB : tA;
-        if (tmin > t_near) t_near = tmin;
-        if (tmax < t_far) t_far = tmax;
-    }
-    *t0 = t_near > 0.0 ? t_near : 0.0;
-    *t1 = t_far;
-    return (*t1 > *t0) ? 1 : 0;
+    return ray_in_box(g, K, Rt, u, v, 0.5, Cijk, dijk, t0, t1);
 }
 
 static int cmp_double(const void *a, const void *b) {

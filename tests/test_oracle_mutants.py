@@ -26,7 +26,8 @@ MUTANTS = {
     "direction not normalised": ("for (int a = 0; a < 3; ++a) d[a] *= inv;", "(void)inv;"),
     "R instead of R^T": ("da += Rt[4 * r + a] * q[r];", "da += Rt[4 * a + r] * q[r];"),
     "box [0, n] instead of [0, n-1]": (
-        "double lo = 0.0, hi = (double)(g->n[a] - 1);", "double lo = 0.0, hi = (double)(g->n[a]);"),
+        "double lo = 0.0 - pad, hi = (double)(g->n[a] - 1) + pad;",
+        "double lo = 0.0 - pad, hi = (double)(g->n[a]) + pad;"),
     "Beer-Lambert as exp(-I)": (
         "return mode == ORACLE_BEER_LAMBERT ? -expm1(-I) : I;",
         "return mode == ORACLE_BEER_LAMBERT ? exp(-I) : I;"),
@@ -86,7 +87,8 @@ MUTANTS = {
     "siddon cell by floor instead of the nearest centre": (
         "int64_t k = (int64_t)floor(p[a] + 0.5);", "int64_t k = (int64_t)floor(p[a]);"),
     "siddon box of voxel centres instead of cells": (
-        "double lo = -0.5, hi = (double)g->n[a] - 0.5;", "double lo = 0.0, hi = (double)(g->n[a] - 1);"),
+        "return ray_in_box(g, K, Rt, u, v, 0.5, Cijk, dijk, t0, t1);",
+        "return ray_in_box(g, K, Rt, u, v, 0.0, Cijk, dijk, t0, t1);"),
     "siddon crossings unsorted": (
         "qsort(ts + 1, (size_t)(m - 1), sizeof(double), cmp_double);", "(void)cmp_double;"),
     "siddon last interior plane missed": (
