@@ -59,6 +59,9 @@ def parse_args():
     p.add_argument("--alpha", action="store_true",
                    help="also time alpha compositing (forward and volume gradient) and the "
                         "Gaussian-Poisson surrogate on the same workload")
+    p.add_argument("--siddon", action="store_true",
+                   help="also time the cell-constant (Siddon) projector and backprojection on "
+                        "the same workload (fp32 linear volume)")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     return p.parse_args()
@@ -465,6 +468,71 @@ def alpha_timing(torch, w, vol32, prep, dtype, layout, Rt, grad_out, elem, l2_pe
     return res
 
 
+def siddon_pieces(w):
+    """Cells crossed per ray, summed over the workload (the Siddon walk's unit
+    of work): |entry cell - exit cell| summed over the axes, plus one, for every
+    ray that hits the cells' box -- geometry only, in numpy fp64."""
+    K = np.asarray(w.K, np.float64)
+    u, v = np.meshgrid(np.arange(w.W, dtype=np.float64), np.arange(w.H, dtype=np.float64))
+    pix = np.stack([u.ravel(), v.ravel(), np.ones(u.size)])
+    q = np.linalg.solve(K, pix)
+    n = np.asarray(w.dims, np.float64)
+    sp = np.asarray(w.spacing, np.float64)
+    total = 0
+    for b in range(w.B):
+        Rt = np.asarray(w.Rt[b], np.float64).reshape(3, 4)
+        R, t = Rt[:, :3], Rt[:, 3]
+        a = R.T @ q
+        d = (a / np.linalg.norm(a, axis=0)) / sp[:, None]
+        C = ((-R.T @ t) - np.asarray(w.origin, np.float64)) / sp
+        with np.errstate(divide="ignore", invalid="ignore"):
+            ta = (-0.5 - C[:, None]) / d
+            tb = (n[:, None] - 0.5 - C[:, None]) / d
+        tn = np.nanmax(np.where(np.isfinite(ta), np.minimum(ta, tb), -np.inf), axis=0)
+        tf = np.nanmin(np.where(np.isfinite(ta), np.maximum(ta, tb), np.inf), axis=0)
+        t0 = np.maximum(tn, 0.0)
+        hit = tf > t0
+        p0 = C[:, None] + t0 * d
+        p1 = C[:, None] + tf * d
+        c0 = np.clip(np.floor(p0 + 0.5), 0, n[:, None] - 1)
+        c1 = np.clip(np.floor(p1 + 0.5), 0, n[:, None] - 1)
+        total += int(np.sum((np.abs(c1 - c0).sum(axis=0) + 1)[hit]))
+    return total
+
+
+def siddon_timing(torch, w, vol32, Rt, grad_out, l2_peak, hbm_peak):
+    """The cell-constant projector and its backprojection on the same
+    workload: median of 10 with L2 flushed before each, per cell crossed."""
+    from cone_beam_ct_b200 import drr
+    from cone_beam_ct_b200 import workloads as wl
+    dev = vol32.device
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    out = torch.empty((w.B, w.H, w.W), dtype=torch.float32, device=dev)
+    grad = torch.zeros((w.dims[2], w.dims[1], w.dims[0]), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+    mode = w.mode if w.mode != wl.MODE_ALPHA else wl.MODE_RAW
+    fwd_ms = _median_ms(torch, lambda: drr.drr_render_siddon(
+        vol32, drr.DRR_F32, w.dims, w.spacing, w.origin, w.K, Rt, w.B, w.H, w.W,
+        w.density_factor, mode, out, stream=stream), flush=flush)
+    adj_ms = _median_ms(torch, lambda: drr.drr_render_siddon_adjoint(
+        w.dims, w.spacing, w.origin, w.K, Rt, w.B, w.H, w.W, w.density_factor, mode, grad_out,
+        out, grad, stream=stream), flush=flush)
+    pieces = siddon_pieces(w)
+    fits = w.dims[0] * w.dims[1] * w.dims[2] * 4 < L2_BYTES
+    bound, peak = ("l2", l2_peak) if fits and l2_peak else ("hbm", hbm_peak)
+
+    def roof(kernel, ms):
+        a = 4 * pieces / (ms * 1e-3) / 1e9      # one fp32 voxel read (or atomic add) per cell
+        return {"kernel": kernel, "bound": bound, "achieved": a, "peak": peak, "unit": "GB/s",
+                "frac": a / peak, "algorithmic_bytes_per_launch": 4 * pieces}
+
+    return {"cells_crossed": pieces, "volume": "fp32, linear",
+            "forward": {"ms": fwd_ms, "gcells_s": pieces / (fwd_ms * 1e-3) / 1e9,
+                        "roofline": roof("siddon_forward_kernel", fwd_ms)},
+            "adjoint": {"ms": adj_ms, "gcells_s": pieces / (adj_ms * 1e-3) / 1e9,
+                        "roofline": roof("siddon_adjoint_kernel", adj_ms)}}
+
+
 def run_ours(args):
     import torch
     from cone_beam_ct_b200 import drr
@@ -621,6 +689,10 @@ def run_ours(args):
         pose = pose_timing(torch, w, prep, dtype, layout, Rt, grad_out, out, elem, l2_peak,
                            hbm_peak, vol_fits_l2)
 
+    siddon = None
+    if args.siddon:
+        siddon = siddon_timing(torch, w, vol32, Rt, grad_out, l2_peak, hbm_peak)
+
     alpha = None
     if args.alpha:
         alpha = alpha_timing(torch, w, vol32, prep, dtype, layout, Rt, grad_out, elem, l2_peak,
@@ -654,6 +726,7 @@ def run_ours(args):
         "texture_comparison": tex,
         "pose_gradient": pose,
         "alpha_compositing": alpha,
+        "siddon": siddon,
         "gpu_launches": 7 * args.steps,   # prepare, forward, plan, zero, 2 adjoint paths, gather
         "clocks": clocks,
         "bracket_ms": bracket[0].elapsed_time(bracket[1]),

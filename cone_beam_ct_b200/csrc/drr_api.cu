@@ -408,3 +408,64 @@ DRR_API drr_status drr_poisson_noise_backward(const float* image, const float* z
 }
 
 }  // extern "C"
+
+extern "C" {
+
+DRR_API drr_status drr_render_siddon(const void* vol, drr_dtype dtype, const int dims[3],
+                                     const float spacing[3], const float origin[3],
+                                     const float K[9], const float* Rt, int B, int H, int W,
+                                     float density_factor, drr_mode mode, float* out,
+                                     void* stream) {
+    if (mode == DRR_MODE_ALPHA)
+        return fail(DRR_ERR_UNSUPPORTED, "the cell-constant projector writes DRR_MODE_RAW or DRR_MODE_BEER_LAMBERT");
+    drr_status st = check_volume(dims, spacing, origin);
+    if (st != DRR_OK) return st;
+    st = check_rays(K, Rt, B, H, W, 1, density_factor, mode);
+    if (st != DRR_OK) return st;
+    if (dtype != DRR_F32 && dtype != DRR_BF16) return fail(DRR_ERR_INVALID_ARG, "unknown dtype %d", dtype);
+    if (stored_elements(dims, DRR_LAYOUT_LINEAR) > kMaxElements)
+        return fail(DRR_ERR_UNSUPPORTED, "volume too large (max 2^31 - 1 elements)");
+    if ((int64_t)B * H * W == 0) return ok();
+    if (!vol || !aligned(vol, dtype == DRR_F32 ? 4 : 2))
+        return fail(DRR_ERR_INVALID_ARG, "vol must be a non-NULL, aligned device pointer");
+    if (!out || !aligned(out, 4)) return fail(DRR_ERR_INVALID_ARG, "out must be a non-NULL, 4-byte aligned device pointer");
+    drr::Geom g;
+    drr::fill_geom(g, dims, spacing, origin, K, B, H, W, 1, density_factor, DRR_LAYOUT_LINEAR);
+    return cuda_status(drr::launch_siddon(vol, dtype, g, Rt, mode, out, static_cast<cudaStream_t>(stream)),
+                       "drr_render_siddon launch");
+}
+
+DRR_API drr_status drr_render_siddon_adjoint(const int dims[3], const float spacing[3],
+                                             const float origin[3], const float K[9],
+                                             const float* Rt, int B, int H, int W,
+                                             float density_factor, drr_mode mode,
+                                             const float* grad_out, const float* fwd_out,
+                                             float* grad_vol, void* stream) {
+    if (mode == DRR_MODE_ALPHA)
+        return fail(DRR_ERR_UNSUPPORTED, "the cell-constant projector writes DRR_MODE_RAW or DRR_MODE_BEER_LAMBERT");
+    drr_status st = check_volume(dims, spacing, origin);
+    if (st != DRR_OK) return st;
+    st = check_rays(K, Rt, B, H, W, 1, density_factor, mode);
+    if (st != DRR_OK) return st;
+    if (stored_elements(dims, DRR_LAYOUT_LINEAR) > kMaxElements)
+        return fail(DRR_ERR_UNSUPPORTED, "volume too large (max 2^31 - 1 elements)");
+    const int64_t npix = (int64_t)B * H * W;
+    if (npix == 0) return ok();
+    if (!grad_out || !aligned(grad_out, 4))
+        return fail(DRR_ERR_INVALID_ARG, "grad_out must be a non-NULL, 4-byte aligned device pointer");
+    if (mode == DRR_MODE_BEER_LAMBERT && (!fwd_out || !aligned(fwd_out, 4)))
+        return fail(DRR_ERR_INVALID_ARG, "fwd_out is required in Beer-Lambert mode");
+    if (!grad_vol || !aligned(grad_vol, 4))
+        return fail(DRR_ERR_INVALID_ARG, "grad_vol must be a non-NULL, 4-byte aligned device pointer");
+    const size_t vbytes = (size_t)dims[0] * dims[1] * dims[2] * 4, ibytes = (size_t)npix * 4;
+    if (overlaps(grad_vol, vbytes, grad_out, ibytes) ||
+        (mode == DRR_MODE_BEER_LAMBERT && overlaps(grad_vol, vbytes, fwd_out, ibytes)))
+        return fail(DRR_ERR_INVALID_ARG, "grad_vol overlaps an image buffer");
+    drr::Geom g;
+    drr::fill_geom(g, dims, spacing, origin, K, B, H, W, 1, density_factor, DRR_LAYOUT_LINEAR);
+    return cuda_status(drr::launch_siddon_adjoint(g, Rt, mode, grad_out, fwd_out, grad_vol,
+                                                  static_cast<cudaStream_t>(stream)),
+                       "drr_render_siddon_adjoint launch");
+}
+
+}  // extern "C"

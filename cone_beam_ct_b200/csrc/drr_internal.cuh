@@ -228,6 +228,10 @@ cudaError_t launch_poisson_noise(const float* image, const float* z, float i0, f
 cudaError_t launch_poisson_noise_backward(const float* image, const float* z, float i0,
                                           const float* grad_out, float* grad_image, int64_t n,
                                           cudaStream_t stream);
+cudaError_t launch_siddon(const void* vol, int dtype, const Geom& g, const float* Rt, int mode,
+                          float* out, cudaStream_t stream);
+cudaError_t launch_siddon_adjoint(const Geom& g, const float* Rt, int mode, const float* grad_out,
+                                  const float* fwd_out, float* grad_vol, cudaStream_t stream);
 cudaError_t launch_pose_grad(const void* vol, int dtype, int layout, const Geom& g,
                              const float* Rt, int mode, const float* grad_out,
                              const float* fwd_out, float* grad_Rt, cudaStream_t stream);

@@ -23,6 +23,7 @@ DRR_LAYOUT_LINEAR, DRR_LAYOUT_PADDED, DRR_LAYOUT_CORNERS = 0, 1, 2
 EXPORTED = ("drr_render", "drr_render_adjoint", "drr_render_adjoint_ws",
             "drr_adjoint_workspace_bytes", "drr_render_adjoint_noalloc", "drr_render_pose_grad",
             "drr_render_alpha_adjoint", "drr_poisson_noise", "drr_poisson_noise_backward",
+            "drr_render_siddon", "drr_render_siddon_adjoint",
             "drr_prepared_bytes", "drr_prepare_volume", "drr_get_last_error", "drr_abi_version")
 DRR_NOALLOC_SCRATCH_BYTES = 32 << 20
 
@@ -76,6 +77,12 @@ def lib():
     L.drr_poisson_noise.restype = _c.c_int
     L.drr_poisson_noise_backward.argtypes = [_vp, _vp, _c.c_float, _vp, _vp, _c.c_int64, _vp]
     L.drr_poisson_noise_backward.restype = _c.c_int
+    L.drr_render_siddon.argtypes = [_vp, _c.c_int, _i3, _f3, _f3, _f9, _vp, _c.c_int, _c.c_int,
+                                    _c.c_int, _c.c_float, _c.c_int, _vp, _vp]
+    L.drr_render_siddon.restype = _c.c_int
+    L.drr_render_siddon_adjoint.argtypes = [_i3, _f3, _f3, _f9, _vp, _c.c_int, _c.c_int,
+                                            _c.c_int, _c.c_float, _c.c_int, _vp, _vp, _vp, _vp]
+    L.drr_render_siddon_adjoint.restype = _c.c_int
     L.drr_adjoint_workspace_bytes.argtypes = [_i3, _c.c_int]
     L.drr_adjoint_workspace_bytes.restype = _c.c_size_t
     L.drr_prepared_bytes.argtypes = [_i3, _c.c_int, _c.c_int]
@@ -211,6 +218,24 @@ def drr_poisson_noise_backward(image, z, i0, grad_out, grad_image, n=None, strea
                                             float(i0), _dev(grad_out, "grad_out", True),
                                             _dev(grad_image, "grad_image", True), int(n),
                                             _stream(stream)))
+
+
+def drr_render_siddon(vol, dtype, dims, spacing, origin, K, Rt, B, H, W, density_factor, mode,
+                      out, stream=None):
+    _check(lib().drr_render_siddon(_dev(vol, "vol", True), int(dtype), _i3v(dims), _f3v(spacing),
+                                   _f3v(origin), _f9v(K), _dev(Rt, "Rt", True), int(B), int(H),
+                                   int(W), float(density_factor), int(mode),
+                                   _dev(out, "out", True), _stream(stream)))
+
+
+def drr_render_siddon_adjoint(dims, spacing, origin, K, Rt, B, H, W, density_factor, mode,
+                              grad_out, fwd_out, grad_vol, stream=None):
+    _check(lib().drr_render_siddon_adjoint(_i3v(dims), _f3v(spacing), _f3v(origin), _f9v(K),
+                                           _dev(Rt, "Rt", True), int(B), int(H), int(W),
+                                           float(density_factor), int(mode),
+                                           _dev(grad_out, "grad_out", True),
+                                           _dev(fwd_out, "fwd_out", True),
+                                           _dev(grad_vol, "grad_vol", True), _stream(stream)))
 
 
 def drr_adjoint_workspace_bytes(dims, B):

@@ -288,6 +288,36 @@ DRR_API drr_status drr_poisson_noise_backward(const float *image, const float *z
                                               const float *grad_out, float *grad_image,
                                               int64_t n, void *stream);
 
+/* The cell-constant (Siddon) projector (diffct page, Features: project()
+ * and backproject() form an exact adjoint pair for the cell-constant Siddon
+ * model): a second discretisation of the same line integral.  Voxel
+ * (i, j, k) is the cube of side one voxel centred on (i, j, k) in IJK, with
+ * the constant value vol[k][j][i]; a ray's image is density_factor times the
+ * exact integral of that piecewise-constant function along the ray (the sum
+ * over the cells it crosses of chord length in mm times value), clipped to
+ * the cells' box [-1/2, n - 1/2] per axis (t0 = max(t_near, 0)), written raw
+ * or as 1 - exp(-I).  No samples: n_samples does not apply.
+ *   vol     DEVICE, DRR_LAYOUT_LINEAR only, fp32 or bf16.
+ *   mode    DRR_MODE_RAW or DRR_MODE_BEER_LAMBERT (DRR_MODE_ALPHA:
+ *           DRR_ERR_UNSUPPORTED).
+ * Other arguments as drr_render. */
+DRR_API drr_status drr_render_siddon(const void *vol, drr_dtype dtype, const int dims[3],
+                                     const float spacing[3], const float origin[3],
+                                     const float K[9], const float *Rt, int B, int H, int W,
+                                     float density_factor, drr_mode mode, float *out,
+                                     void *stream);
+
+/* Its exact adjoint (the matched backprojection): grad_vol += each ray's
+ * grad_out * density_factor (times exp(-I) = 1 - fwd_out in Beer-Lambert)
+ * times its chord length in every cell it crosses; fp32 atomic adds, order
+ * not deterministic.  Arguments as drr_render_adjoint without n_samples. */
+DRR_API drr_status drr_render_siddon_adjoint(const int dims[3], const float spacing[3],
+                                             const float origin[3], const float K[9],
+                                             const float *Rt, int B, int H, int W,
+                                             float density_factor, drr_mode mode,
+                                             const float *grad_out, const float *fwd_out,
+                                             float *grad_vol, void *stream);
+
 /* Bytes that drr_prepare_volume writes for this volume, dtype and layout
  * (0 if the arguments are invalid or the volume is too large). */
 DRR_API size_t drr_prepared_bytes(const int dims[3], drr_dtype dtype, drr_layout layout);

@@ -146,3 +146,32 @@ def gpu_alpha_adjoint(w, grad_out, fwd_out, layout=LINEAR, dtype=F32):
                                  w.H, w.W, w.n_samples, w.density_factor, go, fo, grad)
     torch.cuda.synchronize()
     return grad.cpu().numpy()
+
+
+def gpu_siddon(w, dtype=F32, mode=None, vol=None):
+    """Cell-constant image through drr_render_siddon (linear volume)."""
+    import torch
+    mode = w.mode if mode is None else mode
+    v32, Rt_d = device_inputs(w, vol)
+    src = prepared(v32, w.dims, dtype, LINEAR)
+    out = torch.full((w.B, w.H, w.W), float("nan"), dtype=torch.float32, device="cuda")
+    drr.drr_render_siddon(src, dtype, w.dims, w.spacing, w.origin, w.K, Rt_d, w.B, w.H, w.W,
+                          w.density_factor, mode, out)
+    torch.cuda.synchronize()
+    return out.cpu().numpy()
+
+
+def gpu_siddon_adjoint(w, grad_out, mode=None, fwd_out=None):
+    import torch
+    mode = w.mode if mode is None else mode
+    _, Rt_d = device_inputs(w, vol=np.zeros((1,), np.float32))
+    go = torch.from_numpy(np.ascontiguousarray(grad_out, dtype=np.float32)).cuda()
+    fo = None
+    if fwd_out is not None:
+        fo = torch.from_numpy(np.ascontiguousarray(fwd_out, dtype=np.float32)).cuda()
+    nx, ny, nz = w.dims
+    grad = torch.zeros((nz, ny, nx), dtype=torch.float32, device="cuda")
+    drr.drr_render_siddon_adjoint(w.dims, w.spacing, w.origin, w.K, Rt_d, w.B, w.H, w.W,
+                                  w.density_factor, mode, go, fo, grad)
+    torch.cuda.synchronize()
+    return grad.cpu().numpy()

@@ -289,6 +289,43 @@ def test_noise_backward_rejects_bad_arguments():
     drr.drr_poisson_noise_backward(FAKE, FAKE, 1.0, FAKE, FAKE, n=0, stream=0)
 
 
+SIDDON_BAD = [
+    (dict(mode=drr.DRR_MODE_ALPHA), drr.DRR_ERR_UNSUPPORTED, "RAW"),
+    (dict(mode=5), drr.DRR_ERR_INVALID_ARG, "mode"),
+    (dict(dtype=4), drr.DRR_ERR_INVALID_ARG, "dtype"),
+    (dict(vol=0), drr.DRR_ERR_INVALID_ARG, "vol"),
+    (dict(out=0), drr.DRR_ERR_INVALID_ARG, "out"),
+    (dict(dims=(16, 1, 16)), drr.DRR_ERR_INVALID_ARG, "dims"),
+    (dict(density_factor=float("nan")), drr.DRR_ERR_INVALID_ARG, "density_factor"),
+]
+
+
+@pytest.mark.parametrize("kw,status,word", SIDDON_BAD)
+def test_siddon_rejects_bad_arguments(kw, status, word):
+    args = dict(vol=FAKE, dtype=drr.DRR_F32, dims=DIMS, spacing=SP, origin=ORG, K=K_OK, Rt=FAKE,
+                B=2, H=8, W=8, density_factor=1.0, mode=drr.DRR_MODE_RAW, out=FAKE + (1 << 20),
+                stream=0)
+    args.update(kw)
+    with pytest.raises(drr.DrrError) as e:
+        drr.drr_render_siddon(**args)
+    assert e.value.status == status
+    assert word in drr.drr_get_last_error()
+
+
+def test_siddon_adjoint_rejects_bad_arguments():
+    args = dict(dims=DIMS, spacing=SP, origin=ORG, K=K_OK, Rt=FAKE, B=2, H=8, W=8,
+                density_factor=1.0, mode=drr.DRR_MODE_RAW, grad_out=FAKE + (1 << 20),
+                fwd_out=None, grad_vol=FAKE + (1 << 24), stream=0)
+    for kw, status in ((dict(grad_out=0), drr.DRR_ERR_INVALID_ARG),
+                       (dict(mode=drr.DRR_MODE_BEER_LAMBERT), drr.DRR_ERR_INVALID_ARG),
+                       (dict(grad_vol=FAKE + (1 << 20) + 4), drr.DRR_ERR_INVALID_ARG),
+                       (dict(mode=drr.DRR_MODE_ALPHA), drr.DRR_ERR_UNSUPPORTED)):
+        with pytest.raises(drr.DrrError) as e:
+            drr.drr_render_siddon_adjoint(**dict(args, **kw))
+        assert e.value.status == status
+    drr.drr_render_siddon_adjoint(**dict(args, B=0, grad_out=None, grad_vol=None))   # no-op
+
+
 def test_prepared_bytes():
     assert drr.drr_prepared_bytes((256, 256, 256), drr.DRR_F32, drr.DRR_LAYOUT_LINEAR) == 4 * 256 ** 3
     assert drr.drr_prepared_bytes((256, 256, 256), drr.DRR_BF16, drr.DRR_LAYOUT_LINEAR) == 2 * 256 ** 3
