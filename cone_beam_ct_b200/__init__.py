@@ -24,7 +24,9 @@ from .drr import (  # noqa: F401
     drr_prepared_bytes,
     drr_render,
     drr_render_adjoint,
+    drr_render_adjoint_batched,
     drr_render_alpha_adjoint,
+    drr_render_batched,
     drr_render_adjoint_noalloc,
     drr_render_adjoint_ws,
     drr_render_pose_grad,

@@ -203,11 +203,13 @@ adjoint_kernel(const float* __restrict__ Rt, const float* __restrict__ grad_out,
                const Workspace ws) {
     __shared__ View sv;
     __shared__ int s_dense;
-    const int b = blockIdx.z;
+    const int b = blockIdx.z;                    // output image (view x channel)
     const int tid = threadIdx.x;
     if (ws.flags != nullptr && ws.flags[1 + b] != 0) return;
+    const BatchItem it = batch_item(g, b);
+    grad += it.slot * g.vstride;                 // this volume-channel's gradient
     if (tid == 0) {
-        view_setup(Rt + 12 * (size_t)b, g, sv);
+        view_setup(Rt + 12 * (size_t)it.pose, g, sv);
         s_dense = dense_tile(sv, g, blockIdx.x * kTileW, blockIdx.y * kTileH) ? 1 : 0;
     }
     __syncthreads();

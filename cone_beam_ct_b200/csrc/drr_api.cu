@@ -469,3 +469,119 @@ DRR_API drr_status drr_render_siddon_adjoint(const int dims[3], const float spac
 }
 
 }  // extern "C"
+
+namespace {
+
+// The batch rule of VolumeRaycaster.forward: n_views view matrices for
+// n_vols volumes of `channels` channels; n_views == 1 is broadcast to every
+// volume, else n_views must be a multiple of n_vols (views_per_vol of them
+// per volume, consecutive).  Output images: n_out x channels.
+drr_status batch_shape(int n_vols, int channels, int n_views, int* n_out, int* per_vol,
+                       int* broadcast) {
+    if (n_vols < 0 || channels < 0 || n_views < 0)
+        return fail(DRR_ERR_INVALID_ARG, "n_vols, channels and n_views must be >= 0");
+    if (n_vols == 0 || channels == 0 || n_views == 0) {
+        *n_out = 0;
+        *per_vol = 1;
+        *broadcast = 0;
+        return DRR_OK;
+    }
+    if (n_views == 1 && n_vols > 1) {
+        *n_out = n_vols;
+        *per_vol = 1;
+        *broadcast = 1;
+    } else if (n_views % n_vols == 0) {
+        *n_out = n_views;
+        *per_vol = n_views / n_vols;
+        *broadcast = 0;
+    } else {
+        return fail(DRR_ERR_INVALID_ARG,
+                    "n_views = %d must be 1 or a multiple of n_vols = %d", n_views, n_vols);
+    }
+    if ((int64_t)*n_out * channels > kMaxViews)
+        return fail(DRR_ERR_UNSUPPORTED, "n_out * channels = %lld exceeds %d images per call",
+                    (long long)*n_out * channels, kMaxViews);
+    return DRR_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+DRR_API drr_status drr_render_batched(const void* vols, drr_dtype dtype, drr_layout layout,
+                                      const int dims[3], const float spacing[3],
+                                      const float origin[3], const float K[9], const float* Rt,
+                                      int n_vols, int channels, int n_views, int H, int W,
+                                      int n_samples, float density_factor, drr_mode mode,
+                                      float* out, void* stream) {
+    int n_out = 0, per_vol = 1, bcast = 0;
+    drr_status st = batch_shape(n_vols, channels, n_views, &n_out, &per_vol, &bcast);
+    if (st != DRR_OK) return st;
+    st = check_volume(dims, spacing, origin);
+    if (st != DRR_OK) return st;
+    const int images = n_out * channels;
+    st = check_rays(K, Rt, images, H, W, n_samples, density_factor, mode, true);
+    if (st != DRR_OK) return st;
+    if (dtype != DRR_F32 && dtype != DRR_BF16) return fail(DRR_ERR_INVALID_ARG, "unknown dtype %d", dtype);
+    if (!known_layout(layout)) return fail(DRR_ERR_INVALID_ARG, "unknown layout %d", layout);
+    if (stored_elements(dims, layout) > kMaxElements)
+        return fail(DRR_ERR_UNSUPPORTED, "volume too large (max 2^31 - 1 stored elements)");
+    if ((int64_t)images * H * W == 0) return ok();
+    if (!vols || !aligned(vols, layout_alignment(layout, dtype)))
+        return fail(DRR_ERR_INVALID_ARG, "vols must be a non-NULL device pointer aligned to %zu bytes",
+                    layout_alignment(layout, dtype));
+    if (!out || !aligned(out, 4)) return fail(DRR_ERR_INVALID_ARG, "out must be a non-NULL, 4-byte aligned device pointer");
+    drr::Geom g;
+    drr::fill_geom(g, dims, spacing, origin, K, images, H, W, n_samples, density_factor, layout);
+    g.C = channels;
+    g.views_per_vol = per_vol;
+    g.broadcast = bcast;
+    g.vstride = stored_elements(dims, layout);
+    return cuda_status(drr::launch_forward(vols, dtype, layout, g, Rt, mode, out,
+                                           static_cast<cudaStream_t>(stream)),
+                       "drr_render_batched launch");
+}
+
+DRR_API drr_status drr_render_adjoint_batched(const int dims[3], const float spacing[3],
+                                              const float origin[3], const float K[9],
+                                              const float* Rt, int n_vols, int channels,
+                                              int n_views, int H, int W, int n_samples,
+                                              float density_factor, drr_mode mode,
+                                              const float* grad_out, const float* fwd_out,
+                                              float* grad_vols, void* stream) {
+    int n_out = 0, per_vol = 1, bcast = 0;
+    drr_status st = batch_shape(n_vols, channels, n_views, &n_out, &per_vol, &bcast);
+    if (st != DRR_OK) return st;
+    st = check_volume(dims, spacing, origin);
+    if (st != DRR_OK) return st;
+    const int images = n_out * channels;
+    st = check_rays(K, Rt, images, H, W, n_samples, density_factor, mode);
+    if (st != DRR_OK) return st;
+    if (stored_elements(dims, DRR_LAYOUT_LINEAR) > kMaxElements)
+        return fail(DRR_ERR_UNSUPPORTED, "volume too large (max 2^31 - 1 elements)");
+    const int64_t npix = (int64_t)images * H * W;
+    if (npix == 0) return ok();
+    if (!grad_out || !aligned(grad_out, 4))
+        return fail(DRR_ERR_INVALID_ARG, "grad_out must be a non-NULL, 4-byte aligned device pointer");
+    if (mode == DRR_MODE_BEER_LAMBERT && (!fwd_out || !aligned(fwd_out, 4)))
+        return fail(DRR_ERR_INVALID_ARG, "fwd_out is required in Beer-Lambert mode");
+    if (!grad_vols || !aligned(grad_vols, 4))
+        return fail(DRR_ERR_INVALID_ARG, "grad_vols must be a non-NULL, 4-byte aligned device pointer");
+    const int64_t nvox = (int64_t)dims[0] * dims[1] * dims[2];
+    const size_t vbytes = (size_t)nvox * n_vols * channels * 4, ibytes = (size_t)npix * 4;
+    if (overlaps(grad_vols, vbytes, grad_out, ibytes) ||
+        (mode == DRR_MODE_BEER_LAMBERT && overlaps(grad_vols, vbytes, fwd_out, ibytes)))
+        return fail(DRR_ERR_INVALID_ARG, "grad_vols overlaps an image buffer");
+    drr::Geom g;
+    drr::fill_geom(g, dims, spacing, origin, K, images, H, W, n_samples, density_factor,
+                   DRR_LAYOUT_LINEAR);
+    g.C = channels;
+    g.views_per_vol = per_vol;
+    g.broadcast = bcast;
+    g.vstride = nvox;
+    return cuda_status(drr::launch_adjoint(g, Rt, mode, grad_out, fwd_out, grad_vols, nullptr,
+                                           static_cast<cudaStream_t>(stream)),
+                       "drr_render_adjoint_batched launch");
+}
+
+}  // extern "C"

@@ -104,11 +104,13 @@ __device__ __forceinline__ float march_alpha(const T* __restrict__ vol, const Ge
 
 template <typename T, int LAYOUT, int MODE>
 __global__ void __launch_bounds__(kThreads)
-forward_kernel(const T* __restrict__ vol, const float* __restrict__ Rt, float* __restrict__ out,
-               const Geom g) {
+forward_kernel(const T* __restrict__ vol_base, const float* __restrict__ Rt,
+               float* __restrict__ out, const Geom g) {
     __shared__ View sv;
-    const int b = blockIdx.z;
-    if (threadIdx.x == 0) view_setup(Rt + 12 * (size_t)b, g, sv);
+    const int b = blockIdx.z;                    // output image (view x channel)
+    const BatchItem it = batch_item(g, b);
+    const T* __restrict__ vol = vol_base + it.slot * g.vstride;
+    if (threadIdx.x == 0) view_setup(Rt + 12 * (size_t)it.pose, g, sv);
     __syncthreads();
     int r, c;
     tile_pixel(r, c);

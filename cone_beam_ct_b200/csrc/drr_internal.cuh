@@ -33,7 +33,33 @@ struct Geom {
     double kinv[6];          // K^-1 = [k0 k1 k2; 0 k3 k4; 0 0 k5], from fp64 on the host
     int B, H, W, N;
     float density_factor;
+    // Batches of volumes and channels (VolumeRaycaster.forward's (B, C, D,
+    // H, W) volumes and N = B * views_per_vol view matrices, N == 1
+    // broadcast): grid z = output view n times C plus channel ch; view n
+    // uses pose n (pose 0 when broadcast) and volume n / views_per_vol
+    // (volume n when broadcast); volume v, channel ch starts vstride
+    // elements after the previous one.  One volume of one channel: C = 1,
+    // views_per_vol = B, no broadcast.
+    int C;
+    int views_per_vol;
+    int broadcast;
+    long long vstride;
 };
+
+// Pose, volume-channel slot and output image of grid z.
+struct BatchItem {
+    int pose;         // row of Rt
+    long long slot;   // volume * C + channel
+};
+
+__device__ __forceinline__ BatchItem batch_item(const Geom& g, int z) {
+    const int n = z / g.C, ch = z - n * g.C;
+    BatchItem it;
+    it.pose = g.broadcast ? 0 : n;
+    const int v = g.broadcast ? n : n / g.views_per_vol;
+    it.slot = (long long)v * g.C + ch;
+    return it;
+}
 
 // Per-view quantities, computed once per CTA from the view's [R|t], in fp64
 // (the pose is widened from fp32; the camera sits hundreds of voxels from
@@ -203,6 +229,10 @@ inline void fill_geom(Geom& g, const int dims[3], const float spacing[3], const 
     g.W = W;
     g.N = n_samples;
     g.density_factor = density_factor;
+    g.C = 1;
+    g.views_per_vol = B > 0 ? B : 1;
+    g.broadcast = 0;
+    g.vstride = 0;
 }
 
 // launchers (defined in the .cu files)

@@ -23,7 +23,8 @@ DRR_LAYOUT_LINEAR, DRR_LAYOUT_PADDED, DRR_LAYOUT_CORNERS = 0, 1, 2
 EXPORTED = ("drr_render", "drr_render_adjoint", "drr_render_adjoint_ws",
             "drr_adjoint_workspace_bytes", "drr_render_adjoint_noalloc", "drr_render_pose_grad",
             "drr_render_alpha_adjoint", "drr_poisson_noise", "drr_poisson_noise_backward",
-            "drr_render_siddon", "drr_render_siddon_adjoint",
+            "drr_render_siddon", "drr_render_siddon_adjoint", "drr_render_batched",
+            "drr_render_adjoint_batched",
             "drr_prepared_bytes", "drr_prepare_volume", "drr_get_last_error", "drr_abi_version")
 DRR_NOALLOC_SCRATCH_BYTES = 32 << 20
 
@@ -83,6 +84,14 @@ def lib():
     L.drr_render_siddon_adjoint.argtypes = [_i3, _f3, _f3, _f9, _vp, _c.c_int, _c.c_int,
                                             _c.c_int, _c.c_float, _c.c_int, _vp, _vp, _vp, _vp]
     L.drr_render_siddon_adjoint.restype = _c.c_int
+    L.drr_render_batched.argtypes = [_vp, _c.c_int, _c.c_int, _i3, _f3, _f3, _f9, _vp,
+                                     _c.c_int, _c.c_int, _c.c_int, _c.c_int, _c.c_int, _c.c_int,
+                                     _c.c_float, _c.c_int, _vp, _vp]
+    L.drr_render_batched.restype = _c.c_int
+    L.drr_render_adjoint_batched.argtypes = [_i3, _f3, _f3, _f9, _vp, _c.c_int, _c.c_int,
+                                             _c.c_int, _c.c_int, _c.c_int, _c.c_int, _c.c_float,
+                                             _c.c_int, _vp, _vp, _vp, _vp]
+    L.drr_render_adjoint_batched.restype = _c.c_int
     L.drr_adjoint_workspace_bytes.argtypes = [_i3, _c.c_int]
     L.drr_adjoint_workspace_bytes.restype = _c.c_size_t
     L.drr_prepared_bytes.argtypes = [_i3, _c.c_int, _c.c_int]
@@ -236,6 +245,27 @@ def drr_render_siddon_adjoint(dims, spacing, origin, K, Rt, B, H, W, density_fac
                                            _dev(grad_out, "grad_out", True),
                                            _dev(fwd_out, "fwd_out", True),
                                            _dev(grad_vol, "grad_vol", True), _stream(stream)))
+
+
+def drr_render_batched(vols, dtype, layout, dims, spacing, origin, K, Rt, n_vols, channels,
+                       n_views, H, W, n_samples, density_factor, mode, out, stream=None):
+    _check(lib().drr_render_batched(_dev(vols, "vols", True), int(dtype), int(layout), _i3v(dims),
+                                    _f3v(spacing), _f3v(origin), _f9v(K), _dev(Rt, "Rt", True),
+                                    int(n_vols), int(channels), int(n_views), int(H), int(W),
+                                    int(n_samples), float(density_factor), int(mode),
+                                    _dev(out, "out", True), _stream(stream)))
+
+
+def drr_render_adjoint_batched(dims, spacing, origin, K, Rt, n_vols, channels, n_views, H, W,
+                               n_samples, density_factor, mode, grad_out, fwd_out, grad_vols,
+                               stream=None):
+    _check(lib().drr_render_adjoint_batched(_i3v(dims), _f3v(spacing), _f3v(origin), _f9v(K),
+                                            _dev(Rt, "Rt", True), int(n_vols), int(channels),
+                                            int(n_views), int(H), int(W), int(n_samples),
+                                            float(density_factor), int(mode),
+                                            _dev(grad_out, "grad_out", True),
+                                            _dev(fwd_out, "fwd_out", True),
+                                            _dev(grad_vols, "grad_vols", True), _stream(stream)))
 
 
 def drr_adjoint_workspace_bytes(dims, B):

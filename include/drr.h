@@ -318,6 +318,42 @@ DRR_API drr_status drr_render_siddon_adjoint(const int dims[3], const float spac
                                              const float *grad_out, const float *fwd_out,
                                              float *grad_vol, void *stream);
 
+/* Batches of volumes, channels and views (flashdrr.rendering API docs,
+ * VolumeRaycaster.forward: vol of shape (B, C, D, H, W) and view matrices of
+ * shape (N, 4, 4) with N = B * views_per_vol, N == 1 broadcast to B; output
+ * (N, C, H, W)).
+ *   vols      DEVICE: n_vols * channels volumes of one geometry, each in
+ *             `layout` and `dtype` (drr_prepared_bytes(dims, dtype, layout)
+ *             bytes each), back to back: volume v, channel ch at slot
+ *             v * channels + ch.
+ *   Rt        DEVICE float[n_views * 12]: n_views == 1 renders that pose of
+ *             every volume (n_out = n_vols); otherwise n_views must be a
+ *             multiple of n_vols, and views v * views_per_vol ...
+ *             (v + 1) * views_per_vol - 1 see volume v (n_out = n_views,
+ *             views_per_vol = n_views / n_vols).
+ *   out       DEVICE float[n_out * channels * H * W], image (n, ch) at
+ *             n * channels + ch.
+ * n_out * channels <= 65535.  Other arguments and modes as drr_render. */
+DRR_API drr_status drr_render_batched(const void *vols, drr_dtype dtype, drr_layout layout,
+                                      const int dims[3], const float spacing[3],
+                                      const float origin[3], const float K[9], const float *Rt,
+                                      int n_vols, int channels, int n_views, int H, int W,
+                                      int n_samples, float density_factor, drr_mode mode,
+                                      float *out, void *stream);
+
+/* Adjoint of drr_render_batched (RAW or Beer-Lambert): grad_vols, DEVICE
+ * float32 [n_vols * channels][nz][ny][nx] (linear), ACCUMULATED into; each
+ * image's gradient goes to the volume-channel it was rendered from.  Uses
+ * the direct scatter path (no workspace).  Other arguments as
+ * drr_render_adjoint and drr_render_batched. */
+DRR_API drr_status drr_render_adjoint_batched(const int dims[3], const float spacing[3],
+                                              const float origin[3], const float K[9],
+                                              const float *Rt, int n_vols, int channels,
+                                              int n_views, int H, int W, int n_samples,
+                                              float density_factor, drr_mode mode,
+                                              const float *grad_out, const float *fwd_out,
+                                              float *grad_vols, void *stream);
+
 /* Bytes that drr_prepare_volume writes for this volume, dtype and layout
  * (0 if the arguments are invalid or the volume is too large). */
 DRR_API size_t drr_prepared_bytes(const int dims[3], drr_dtype dtype, drr_layout layout);

@@ -6,6 +6,8 @@ never imports it and shares no code with it.
 """
 from .oracle import (  # noqa: F401
     adjoint,
+    adjoint_batched,
+    batch_map,
     bf16_to_float,
     build,
     load,
@@ -14,6 +16,7 @@ from .oracle import (  # noqa: F401
     pose_grad,
     ray,
     render,
+    render_batched,
     render_rays,
     render_siddon,
     round_bf16,

@@ -220,6 +220,51 @@ def siddon_adjoint(dims, spacing, origin, K, Rt, H, W, density_factor, mode, gra
     return grad.reshape(nz, ny, nx)
 
 
+def batch_map(n_vols, channels, n_views):
+    """The batch rule written out (VolumeRaycaster.forward: N = B *
+    views_per_vol view matrices, N == 1 broadcast to B): a list of
+    (output view n, pose row, volume v) for every output view."""
+    if n_views == 1 and n_vols > 1:
+        return [(n, 0, n) for n in range(n_vols)]
+    assert n_views % n_vols == 0, "n_views must be 1 or a multiple of n_vols"
+    per = n_views // n_vols
+    return [(n, n, n // per) for n in range(n_views)]
+
+
+def render_batched(vols, dims, spacing, origin, K, Rt, n_views, H, W, n_samples, density_factor,
+                   mode, nthreads=None):
+    """vols[v][ch] (n_vols x C x nz x ny x nx) -> out[n][ch][r][c] (float64),
+    each image rendered alone by render()."""
+    vols = np.asarray(vols)
+    n_vols, C = vols.shape[0], vols.shape[1]
+    Rt = np.asarray(Rt).reshape(-1, 12)
+    items = batch_map(n_vols, C, n_views)
+    out = np.zeros((len(items), C, H, W))
+    for n, pose, v in items:
+        for ch in range(C):
+            out[n, ch] = render(vols[v, ch], dims, spacing, origin, K, Rt[pose:pose + 1], H, W,
+                                n_samples, density_factor, mode, nthreads)[0]
+    return out
+
+
+def adjoint_batched(dims, spacing, origin, K, Rt, n_vols, n_views, H, W, n_samples,
+                    density_factor, mode, grad_out, vols=None, nthreads=1):
+    """grad_vols[v][ch] (float64) = sum over the images rendered from (v, ch)
+    of their adjoints (adjoint() of each image alone)."""
+    go = np.asarray(grad_out, np.float64)
+    C = go.shape[1]
+    Rt = np.asarray(Rt).reshape(-1, 12)
+    nx, ny, nz = (int(x) for x in dims)
+    grads = np.zeros((n_vols, C, nz, ny, nx))
+    for n, pose, v in batch_map(n_vols, C, n_views):
+        for ch in range(C):
+            grads[v, ch] += adjoint(dims, spacing, origin, K, Rt[pose:pose + 1], H, W, n_samples,
+                                    density_factor, mode, go[n, ch][None],
+                                    vol=None if vols is None else np.asarray(vols)[v, ch],
+                                    nthreads=nthreads)
+    return grads
+
+
 def round_bf16(x):
     """bf16 bit patterns (uint16) of float32 values, round-to-nearest-even."""
     a = np.ascontiguousarray(x, dtype=np.float32)

@@ -326,6 +326,29 @@ def test_siddon_adjoint_rejects_bad_arguments():
     drr.drr_render_siddon_adjoint(**dict(args, B=0, grad_out=None, grad_vol=None))   # no-op
 
 
+def test_batched_rejects_bad_arguments():
+    args = dict(vols=FAKE, dtype=drr.DRR_F32, layout=drr.DRR_LAYOUT_LINEAR, dims=DIMS, spacing=SP,
+                origin=ORG, K=K_OK, Rt=FAKE + (1 << 26), n_vols=2, channels=3, n_views=4, H=8, W=8,
+                n_samples=16, density_factor=1.0, mode=drr.DRR_MODE_RAW, out=FAKE + (1 << 20),
+                stream=0)
+    for kw, status, word in ((dict(n_views=3), drr.DRR_ERR_INVALID_ARG, "multiple"),
+                             (dict(channels=-1), drr.DRR_ERR_INVALID_ARG, ">= 0"),
+                             (dict(channels=20000), drr.DRR_ERR_UNSUPPORTED, "images"),
+                             (dict(vols=0), drr.DRR_ERR_INVALID_ARG, "vols"),
+                             (dict(out=0), drr.DRR_ERR_INVALID_ARG, "out")):
+        with pytest.raises(drr.DrrError) as e:
+            drr.drr_render_batched(**dict(args, **kw))
+        assert e.value.status == status and word in drr.drr_get_last_error()
+    drr.drr_render_batched(**dict(args, channels=0, vols=None, out=None))   # empty: no-op
+    adj = dict(dims=DIMS, spacing=SP, origin=ORG, K=K_OK, Rt=FAKE, n_vols=2, channels=1,
+               n_views=1, H=8, W=8, n_samples=16, density_factor=1.0, mode=drr.DRR_MODE_RAW,
+               grad_out=FAKE + (1 << 20), fwd_out=None, grad_vols=FAKE + (1 << 24), stream=0)
+    for kw in (dict(grad_out=0), dict(n_views=5), dict(mode=drr.DRR_MODE_BEER_LAMBERT),
+               dict(grad_vols=FAKE + (1 << 20) + 4)):
+        with pytest.raises(drr.DrrError):
+            drr.drr_render_adjoint_batched(**dict(adj, **kw))
+
+
 def test_prepared_bytes():
     assert drr.drr_prepared_bytes((256, 256, 256), drr.DRR_F32, drr.DRR_LAYOUT_LINEAR) == 4 * 256 ** 3
     assert drr.drr_prepared_bytes((256, 256, 256), drr.DRR_BF16, drr.DRR_LAYOUT_LINEAR) == 2 * 256 ** 3

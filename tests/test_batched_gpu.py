@@ -1,0 +1,108 @@
+"""GPU parity of the batched forward and adjoint (drr_render_batched /
+drr_render_adjoint_batched) against the oracle's batch rule
+(tests/test_oracle_batch_pins.py): volumes x channels x views with the
+views grouped per volume, and one view broadcast to every volume.  Each
+image carries the single-image tolerances (forward 1e-4 normwise and per
+pixel; adjoint 1e-4 normwise and L2, per volume-channel), and the batched
+pair passes the dot-product identity at 1e-5.
+"""
+import numpy as np
+import pytest
+
+import oracle
+from cone_beam_ct_b200 import drr
+from cone_beam_ct_b200 import workloads as wl
+from tests.gpu_helpers import CORNERS, F32, LAYOUTS, LINEAR, PADDED, assert_parity
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def cuda():
+    torch = pytest.importorskip("torch")
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    return torch
+
+
+def _batch(n_vols, C, n_views, seed):
+    w = wl.small_random_case(seed, B=n_views)
+    nx, ny, nz = w.dims
+    vols = np.random.default_rng(seed).uniform(0.0, 0.05, (n_vols, C, nz, ny, nx)).astype(np.float32)
+    return w, vols
+
+
+def _gpu_batched(w, vols, n_views, layout, mode):
+    import torch
+    n_vols, C = vols.shape[:2]
+    v32 = torch.from_numpy(vols).cuda()
+    per = drr.drr_prepared_bytes(w.dims, F32, layout)
+    if layout == LINEAR:
+        src = v32
+    else:
+        src = torch.empty(n_vols * C * per, dtype=torch.uint8, device="cuda")
+        for s in range(n_vols * C):
+            drr.drr_prepare_volume(v32.view(n_vols * C, -1)[s], w.dims, F32, layout,
+                                   src[s * per:(s + 1) * per], per)
+    Rt = torch.from_numpy(np.ascontiguousarray(w.Rt.reshape(-1, 12))).cuda()
+    n_out = n_vols if (n_views == 1 and n_vols > 1) else n_views
+    out = torch.full((n_out, C, w.H, w.W), float("nan"), device="cuda")
+    drr.drr_render_batched(src, F32, layout, w.dims, w.spacing, w.origin, w.K, Rt, n_vols, C,
+                           n_views, w.H, w.W, w.n_samples, w.density_factor, mode, out)
+    torch.cuda.synchronize()
+    return out.cpu().numpy()
+
+
+def _gpu_adjoint_batched(w, n_vols, C, n_views, go, mode, fwd=None):
+    import torch
+    nx, ny, nz = w.dims
+    Rt = torch.from_numpy(np.ascontiguousarray(w.Rt.reshape(-1, 12))).cuda()
+    g = torch.zeros((n_vols, C, nz, ny, nx), device="cuda")
+    fo = None if fwd is None else torch.from_numpy(np.ascontiguousarray(fwd, np.float32)).cuda()
+    drr.drr_render_adjoint_batched(w.dims, w.spacing, w.origin, w.K, Rt, n_vols, C, n_views, w.H,
+                                   w.W, w.n_samples, w.density_factor, mode,
+                                   torch.from_numpy(np.ascontiguousarray(go, np.float32)).cuda(),
+                                   fo, g)
+    torch.cuda.synchronize()
+    return g.cpu().numpy()
+
+
+@pytest.mark.parametrize("n_vols,C,n_views", [(2, 3, 4), (3, 2, 1), (1, 2, 3)])
+@pytest.mark.parametrize("layout", LAYOUTS)
+def test_batched_forward(cuda, n_vols, C, n_views, layout):
+    w, vols = _batch(n_vols, C, n_views, 601 + n_views)
+    got = _gpu_batched(w, vols, n_views, layout, wl.MODE_BEER_LAMBERT)
+    ref = oracle.render_batched(vols, w.dims, w.spacing, w.origin, w.K, w.Rt, n_views, w.H, w.W,
+                                w.n_samples, w.density_factor, wl.MODE_BEER_LAMBERT)
+    assert got.shape == ref.shape
+    for n in range(ref.shape[0]):
+        for ch in range(C):
+            assert_parity(got[n, ch], ref[n, ch], 1e-4, what=f"image ({n}, {ch})")
+
+
+@pytest.mark.parametrize("n_vols,C,n_views", [(2, 3, 4), (3, 2, 1)])
+@pytest.mark.parametrize("mode", [wl.MODE_RAW, wl.MODE_BEER_LAMBERT])
+def test_batched_adjoint(cuda, n_vols, C, n_views, mode):
+    w, vols = _batch(n_vols, C, n_views, 611 + n_views)
+    n_out = n_vols if (n_views == 1 and n_vols > 1) else n_views
+    go = np.random.default_rng(5).standard_normal((n_out, C, w.H, w.W)).astype(np.float32)
+    fwd = _gpu_batched(w, vols, n_views, PADDED, mode) if mode else None
+    got = _gpu_adjoint_batched(w, n_vols, C, n_views, go, mode, fwd)
+    ref = oracle.adjoint_batched(w.dims, w.spacing, w.origin, w.K, w.Rt, n_vols, n_views, w.H,
+                                 w.W, w.n_samples, w.density_factor, mode, go, vols=vols,
+                                 nthreads=4)
+    for v in range(n_vols):
+        for ch in range(C):
+            r = ref[v, ch]
+            g = got[v, ch].astype(np.float64)
+            assert np.max(np.abs(g - r)) <= 1e-4 * np.max(np.abs(r))
+            assert np.linalg.norm(g - r) <= 1e-4 * np.linalg.norm(r)
+
+
+def test_batched_dot_product_identity(cuda):
+    w, x = _batch(2, 2, 6, 621)
+    y = np.random.default_rng(9).standard_normal((6, 2, w.H, w.W)).astype(np.float32)
+    Ax = _gpu_batched(w, x, 6, LINEAR, wl.MODE_RAW).astype(np.float64)
+    ATy = _gpu_adjoint_batched(w, 2, 2, 6, y, wl.MODE_RAW).astype(np.float64)
+    lhs = float(np.sum(Ax * y.astype(np.float64)))
+    rhs = float(np.sum(x.astype(np.float64) * ATy))
+    assert abs(lhs - rhs) <= 1e-5 * np.linalg.norm(Ax) * np.linalg.norm(y.astype(np.float64))

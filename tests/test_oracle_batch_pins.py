@@ -1,0 +1,70 @@
+"""Pins of the oracle's batch rule (CPU): VolumeRaycaster.forward's volumes
+(B, C, D, H, W) and view matrices (N, 4, 4), N = B * views_per_vol, N == 1
+broadcast to B, output (N, C, H, W) (flashdrr.rendering API docs).
+
+Each volume-channel is a constant with its own value, so every output image
+is that value times density_factor times the box chord (tests/pin_math.py):
+an image shows by its value which volume and channel, and by its chords
+which pose, it was rendered from -- checked against the rule as the page
+states it, written here without the oracle's helper.
+"""
+import numpy as np
+import pytest
+
+import oracle
+from cone_beam_ct_b200 import workloads as wl
+from tests import pin_math as pm
+
+
+def _case(n_vols, C, n_views, seed):
+    w = wl.small_random_case(seed, dims=(9, 8, 10), B=n_views, H=6, W=7, n_samples=11)
+    Rt = np.array(w.Rt, np.float64).reshape(-1, 3, 4)
+    for b in range(Rt.shape[0]):
+        U, _, Vt = np.linalg.svd(Rt[b, :, :3])
+        Rt[b, :, :3] = U @ Vt
+    vals = np.array([[0.01 * (1 + v + 10 * ch) for ch in range(C)] for v in range(n_vols)],
+                    np.float32)
+    nx, ny, nz = w.dims
+    vols = np.broadcast_to(vals[:, :, None, None, None], (n_vols, C, nz, ny, nx)).copy()
+    return w, Rt, vols, vals
+
+
+@pytest.mark.parametrize("n_vols,C,n_views", [(2, 3, 4), (3, 1, 1), (1, 2, 3), (2, 2, 2)])
+def test_batch_rule_by_constant_volumes(n_vols, C, n_views):
+    w, Rt, vols, vals = _case(n_vols, C, n_views, 81 + n_views)
+    out = oracle.render_batched(vols, w.dims, w.spacing, w.origin, w.K, Rt, n_views, w.H, w.W,
+                                w.n_samples, w.density_factor, wl.MODE_RAW)
+    n_out = n_vols if (n_views == 1 and n_vols > 1) else n_views
+    assert out.shape == (n_out, C, w.H, w.W)
+    lo = np.asarray(w.origin, np.float64)
+    hi = lo + (np.asarray(w.dims) - 1) * np.asarray(w.spacing, np.float64)
+    for n in range(n_out):
+        pose = 0 if n_views == 1 else n
+        vol = n if (n_views == 1 and n_vols > 1) else n // (n_views // n_vols)
+        for r in range(w.H):
+            for c in range(w.W):
+                C0, d = pm.world_ray(w.K, Rt[pose].reshape(-1), c, r)
+                ch_ = pm.box_chord(C0, d, lo, hi)
+                chord = 0.0 if ch_ is None else ch_[1] - ch_[0]
+                for ch in range(C):
+                    expect = w.density_factor * float(vals[vol, ch]) * chord
+                    assert abs(out[n, ch, r, c] - expect) <= 1e-12 + 1e-9 * expect
+
+
+def test_batch_rule_rejects_a_view_count_that_does_not_divide():
+    with pytest.raises(AssertionError):
+        oracle.batch_map(2, 1, 3)
+
+
+def test_batched_adjoint_is_the_transpose_of_the_batched_forward():
+    w, Rt, _, _ = _case(2, 2, 4, 91)
+    rng = np.random.default_rng(3)
+    nx, ny, nz = w.dims
+    x = rng.uniform(0, 1, (2, 2, nz, ny, nx)).astype(np.float32)
+    y = rng.standard_normal((4, 2, w.H, w.W))
+    Ax = oracle.render_batched(x, w.dims, w.spacing, w.origin, w.K, Rt, 4, w.H, w.W, w.n_samples,
+                               w.density_factor, wl.MODE_RAW)
+    ATy = oracle.adjoint_batched(w.dims, w.spacing, w.origin, w.K, Rt, 2, 4, w.H, w.W,
+                                 w.n_samples, w.density_factor, wl.MODE_RAW, y)
+    lhs, rhs = np.sum(Ax * y), np.sum(x.astype(np.float64) * ATy)
+    assert abs(lhs - rhs) <= 1e-12 * np.linalg.norm(Ax) * np.linalg.norm(y)
