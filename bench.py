@@ -333,7 +333,7 @@ def cpu_baseline(w):
         done += oracle_on_rays(w, view, rows, cores)
     dt = time.perf_counter() - t0
     return {"value": done / dt / 1e9, "unit": "Gsamples/s", "cores": cores, "kind": "oracle",
-            "sample": f"every {k}th detector row of all {w.B} views ({done:.3g} ray-samples), "
+            "sample": f"every {k}-th detector row of all {w.B} views ({done:.3g} ray-samples), "
                       f"fp64 forward threaded over rays + fp64 adjoint on one thread, "
                       f"{dt:.1f} s"}
 
