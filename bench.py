@@ -50,7 +50,7 @@ def parse_args():
     p.add_argument("--config", type=int, default=3, choices=[1, 2, 3, 4],
                    help="workload (default 3: 256^3 bf16, 4 views 1024x1024, 512 samples, "
                         "the size the throughput target is quoted at)")
-    p.add_argument("--layout", choices=["padded", "corners", "linear"], default="corners",
+    p.add_argument("--layout", choices=["padded", "corners", "quads", "linear"], default="corners",
                    help="volume layout drr_prepare_volume writes for the forward")
     p.add_argument("--texture", action="store_true",
                    help="also time the texture-trilinear comparison forward (libdrr_texture.so)")
@@ -228,16 +228,17 @@ def l2_read_peak_gbs(torch, nbytes):
     return best
 
 
-def traffic_for(kernel, workload_name):
+def traffic_for(kernel, workload_name, layout_name):
     """DRAM bytes per launch from a committed ncu summary, if it was taken on
-    the current source of the kernel (else None)."""
+    the current source of the kernel and, for a kernel that reads the
+    volume, in the same layout (else None)."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
         table = json.load(f)
     entry = table.get(kernel, {}).get(workload_name)
-    if not entry:
+    if not entry or entry.get("layout", layout_name) != layout_name:
         return None
     digest = hashlib.sha256()
     for src in entry["sources"]:
@@ -551,7 +552,7 @@ def run_ours(args):
 
     w = workload(args.config)
     layout = {"padded": drr.DRR_LAYOUT_PADDED, "corners": drr.DRR_LAYOUT_CORNERS,
-              "linear": drr.DRR_LAYOUT_LINEAR}[args.layout]
+              "quads": drr.DRR_LAYOUT_QUADS, "linear": drr.DRR_LAYOUT_LINEAR}[args.layout]
     dtype = drr.DRR_BF16 if w.dtype == wl.DTYPE_BF16 else drr.DRR_F32
     elem = 2 if dtype == drr.DRR_BF16 else 4
     nx, ny, nz = w.dims
@@ -677,7 +678,7 @@ def run_ours(args):
                 "unit": "GB/s", "frac": achieved / peak, "peak_source": src,
                 "frac_of_hbm": achieved / hbm_peak,
                 "algorithmic_bytes_per_launch": int(nbytes), "ms_per_launch": ms,
-                "traffic": traffic_for(kernel_key, wname)}
+                "traffic": traffic_for(kernel_key, wname, args.layout)}
 
     wname = config_block(w, args.config, "")["workload"]
     fwd_roof = roof("forward_kernel", fwd_ms, fwd_bytes, "forward_kernel", wname)

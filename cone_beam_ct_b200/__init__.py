@@ -11,6 +11,7 @@ from .drr import (  # noqa: F401
     DRR_LAYOUT_CORNERS,
     DRR_LAYOUT_LINEAR,
     DRR_LAYOUT_PADDED,
+    DRR_LAYOUT_QUADS,
     DRR_MODE_ALPHA,
     DRR_MODE_BEER_LAMBERT,
     DRR_MODE_RAW,

@@ -451,9 +451,10 @@ alpha_adjoint_kernel(const T* __restrict__ vol, const float* __restrict__ Rt,
         const int cx = fix_cell(qx), cy = fix_cell(qy), cz = fix_cell(qz);
         const float fx = fix_frac(qx), fy = fix_frac(qy), fz = fix_frac(qz);
         // the forward's sample value, bit for bit
-        const float mu = LAYOUT == 2
-                             ? sample_corners(vol + (size_t)(cz * g.slice + cy * g.row + cx) * 8, fx, fy, fz)
-                             : trilinear_at(vol + (cz * g.slice + cy * g.row + cx), g.row, g.slice, fx, fy, fz);
+        const int at = cz * g.slice + cy * g.row + cx;
+        const float mu = LAYOUT == 2   ? sample_corners(vol + (size_t)at * 8, fx, fy, fz)
+                         : LAYOUT == 3 ? sample_quads(vol + (size_t)at * 4, g.slice, fx, fy, fz)
+                                       : trilinear_at(vol + at, g.row, g.slice, fx, fy, fz);
         const float a = -expm1f(-s * mu);
         Ci = fmaf(Tr * a, mu, Ci);
         const float dmu = Tr * fmaf(s * (1.0f - a), mu, a) - s * (Cray - Ci);
@@ -560,6 +561,15 @@ cudaError_t launch_alpha_adjoint(const void* vol, int dtype, int layout, const G
                                  float* grad_vol, cudaStream_t stream) {
     const dim3 grid((g.W + kTileW - 1) / kTileW, (g.H + kTileH - 1) / kTileH, g.B);
     const int grow = g.nx, gslice = g.nx * g.ny;
+    if (layout == 3) {
+        if (dtype == 0)
+            alpha_adjoint_kernel<float, 3><<<grid, kThreads, 0, stream>>>(
+                static_cast<const float*>(vol), Rt, grad_out, fwd_out, grad_vol, g, grow, gslice);
+        else
+            alpha_adjoint_kernel<uint16_t, 3><<<grid, kThreads, 0, stream>>>(
+                static_cast<const uint16_t*>(vol), Rt, grad_out, fwd_out, grad_vol, g, grow, gslice);
+        return cudaGetLastError();
+    }
     if (dtype == 0 && layout == 2)
         alpha_adjoint_kernel<float, 2><<<grid, kThreads, 0, stream>>>(
             static_cast<const float*>(vol), Rt, grad_out, fwd_out, grad_vol, g, grow, gslice);

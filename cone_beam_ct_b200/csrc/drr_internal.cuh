@@ -190,7 +190,7 @@ __device__ __forceinline__ void tile_pixel(int& r, int& c) {
 // host side
 
 // Kernel parameter block from validated host arguments.  layout: 0 linear,
-// 1 zero-bordered, 2 corner-replicated (include/drr.h).  K^-1 of the upper
+// 1 zero-bordered, 2 corner records, 3 xy quads (include/drr.h).  K^-1 of the upper
 // triangular K in double.
 inline void fill_geom(Geom& g, const int dims[3], const float spacing[3], const float origin[3],
                       const float K[9], int B, int H, int W, int n_samples, float density_factor,
@@ -199,7 +199,7 @@ inline void fill_geom(Geom& g, const int dims[3], const float spacing[3], const 
     g.nx = dims[0];
     g.ny = dims[1];
     g.nz = dims[2];
-    if (layout == 2) {                      // strides of cells, 8 elements each
+    if (layout == 2 || layout == 3) {       // strides of cells (8 elements) or quads (4)
         g.row = dims[0] - 1;
         g.slice = (dims[0] - 1) * (dims[1] - 1);
     } else {
@@ -210,8 +210,8 @@ inline void fill_geom(Geom& g, const int dims[3], const float spacing[3], const 
     for (int a = 0; a < 3; ++a) {
         g.hi[a] = (float)(dims[a] - 1);
         // largest 32.32 sample coordinate whose 8 corners are stored: cell <= n-2
-        // for the linear and corner layouts, cell <= n (inside the zero border)
-        // for the bordered one
+        // for the linear, corner and quad layouts, cell <= n (inside the zero
+        // border) for the bordered one
         const long long cells = layout == 1 ? dims[a] + 1 : dims[a] - 1;
         g.lim[a] = cells * (1LL << 32) - 1;
         g.spacing[a] = spacing[a];

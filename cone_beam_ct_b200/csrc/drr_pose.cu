@@ -53,6 +53,10 @@ __device__ __forceinline__ void cell_corners(const T* __restrict__ vol, const Ge
                 v[2 * m + 1] = __uint_as_float(words[m] & 0xFFFF0000u);
             }
         }
+    } else if (LAYOUT == 3) {
+        const T* p = vol + (size_t)(cz * g.slice + cy * g.row + cx) * 4;
+        load_quad(p, v);
+        load_quad(p + 4 * (size_t)g.slice, v + 4);
     } else {
         const T* p = vol + (cz * g.slice + cy * g.row + cx);
 #pragma unroll
@@ -295,6 +299,7 @@ template <typename T>
 cudaError_t launch_layout(const void* vol, int layout, const Geom& g, const float* Rt, int mode,
                           const float* grad_out, const float* fwd_out, float* grad_Rt,
                           cudaStream_t stream) {
+    if (layout == 3) return launch_typed<T, 3>(vol, g, Rt, mode, grad_out, fwd_out, grad_Rt, stream);
     if (layout == 2) return launch_typed<T, 2>(vol, g, Rt, mode, grad_out, fwd_out, grad_Rt, stream);
     if (layout == 1) return launch_typed<T, 1>(vol, g, Rt, mode, grad_out, fwd_out, grad_Rt, stream);
     return launch_typed<T, 0>(vol, g, Rt, mode, grad_out, fwd_out, grad_Rt, stream);

@@ -91,6 +91,32 @@ __global__ void to_corners(const float* __restrict__ src, T* __restrict__ dst, i
     }
 }
 
+// xy-quad layout: quad m = (i, j, k) holds src[k][j+b][i+a] in the order
+// a + 2b, one 16-byte (fp32) or 8-byte (bf16) store.
+template <typename T>
+__global__ void to_quads(const float* __restrict__ src, T* __restrict__ dst, int nx, int ny,
+                         int nz) {
+    const int qx = nx - 1, qy = ny - 1;
+    const int64_t n = (int64_t)qx * qy * nz;
+    for (int64_t m = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; m < n;
+         m += (int64_t)gridDim.x * blockDim.x) {
+        const int i = (int)(m % qx);
+        const int j = (int)((m / qx) % qy);
+        const int64_t k = m / ((int64_t)qx * qy);
+        const float* p = src + (k * ny + j) * nx + i;
+        const float v[4] = {__ldg(p), __ldg(p + 1), __ldg(p + nx), __ldg(p + nx + 1)};
+        if constexpr (sizeof(T) == 4) {
+            reinterpret_cast<float4*>(dst)[m] = make_float4(v[0], v[1], v[2], v[3]);
+        } else {
+            const unsigned w0 = (unsigned)store_value<uint16_t>(v[0]) |
+                                ((unsigned)store_value<uint16_t>(v[1]) << 16);
+            const unsigned w1 = (unsigned)store_value<uint16_t>(v[2]) |
+                                ((unsigned)store_value<uint16_t>(v[3]) << 16);
+            reinterpret_cast<uint2*>(dst)[m] = make_uint2(w0, w1);
+        }
+    }
+}
+
 int grid_for(int64_t n) {
     int64_t blocks = (n + 255) / 256;
     const int64_t cap = 148 * 16;   // enough CTAs to fill every SM; the loops stride
@@ -108,6 +134,14 @@ cudaError_t launch_prepare(const float* src, int nx, int ny, int nz, int dtype, 
         else
             to_linear<uint16_t><<<grid_for(n), 256, 0, stream>>>(src, static_cast<uint16_t*>(dst),
                                                                  n);
+    } else if (layout == 3) {
+        const int64_t n = (int64_t)(nx - 1) * (ny - 1) * nz;
+        if (dtype == 0)
+            to_quads<float><<<grid_for(n), 256, 0, stream>>>(src, static_cast<float*>(dst), nx, ny,
+                                                             nz);
+        else
+            to_quads<uint16_t><<<grid_for(n), 256, 0, stream>>>(src, static_cast<uint16_t*>(dst),
+                                                                nx, ny, nz);
     } else if (layout == 2) {
         const int64_t n = (int64_t)(nx - 1) * (ny - 1) * (nz - 1);
         if (dtype == 0)

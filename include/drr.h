@@ -108,7 +108,14 @@ typedef enum {
        aligned.  Written by drr_prepare_volume.  One sample of the forward
        then reads its 8 voxels with one (bf16) or two (fp32) 16-byte loads
        instead of 8 scalar gathers; the price is 8x the storage. */
-    DRR_LAYOUT_CORNERS = 2
+    DRR_LAYOUT_CORNERS = 2,
+    /* xy quads: for every (i, j, k) in [0, nx-2] x [0, ny-2] x [0, nz-1]
+       (quad index (k*(ny-1) + j)*(nx-1) + i) the 4 voxels vol[k][j+b][i+a]
+       stored contiguously in the order a + 2b: 4 elements, 8 bytes (bf16) or
+       16 bytes (fp32), 16-byte aligned.  Written by drr_prepare_volume.  A
+       sample reads two quads (slices k and k+1); 4x the storage, half of the
+       corner records'. */
+    DRR_LAYOUT_QUADS = 3
 } drr_layout;
 
 /* Forward projection.

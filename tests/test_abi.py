@@ -108,6 +108,7 @@ RENDER_BAD = [
     (dict(Rt=FAKE + 1), drr.DRR_ERR_INVALID_ARG, "Rt"),
     (dict(out=0), drr.DRR_ERR_INVALID_ARG, "out"),
     (dict(layout=drr.DRR_LAYOUT_CORNERS, vol=FAKE + 4), drr.DRR_ERR_INVALID_ARG, "16 bytes"),
+    (dict(layout=drr.DRR_LAYOUT_QUADS, vol=FAKE + 8), drr.DRR_ERR_INVALID_ARG, "16 bytes"),
     (dict(out=FAKE + 6), drr.DRR_ERR_INVALID_ARG, "out"),
 ]
 
@@ -361,6 +362,10 @@ def test_prepared_bytes():
     assert drr.drr_prepared_bytes((5, 6, 7), drr.DRR_BF16, drr.DRR_LAYOUT_CORNERS) == 2 * 8 * 4 * 5 * 6
     assert drr.drr_prepared_bytes((640, 640, 640), drr.DRR_BF16, drr.DRR_LAYOUT_CORNERS) == 2 * 8 * 639 ** 3
     assert drr.drr_prepared_bytes((660, 660, 660), drr.DRR_BF16, drr.DRR_LAYOUT_CORNERS) == 0
+    assert drr.drr_prepared_bytes((5, 6, 7), drr.DRR_F32, drr.DRR_LAYOUT_QUADS) == 4 * 4 * 4 * 5 * 7
+    assert drr.drr_prepared_bytes((5, 6, 7), drr.DRR_BF16, drr.DRR_LAYOUT_QUADS) == 2 * 4 * 4 * 5 * 7
+    assert drr.drr_prepared_bytes((1024, 1024, 512), drr.DRR_F32, drr.DRR_LAYOUT_QUADS) == \
+        4 * 4 * 1023 * 1023 * 512
 
 
 PREPARE_BAD = [
@@ -373,6 +378,7 @@ PREPARE_BAD = [
     (dict(dst=FAKE + 64), drr.DRR_ERR_INVALID_ARG),      # overlaps src
     (dict(src=FAKE + 2), drr.DRR_ERR_INVALID_ARG),       # misaligned
     (dict(layout=drr.DRR_LAYOUT_CORNERS, dst=FAKE + (1 << 24) + 8), drr.DRR_ERR_INVALID_ARG),
+    (dict(layout=drr.DRR_LAYOUT_QUADS, dst=FAKE + (1 << 24) + 8), drr.DRR_ERR_INVALID_ARG),
     (dict(dims=(2048, 2048, 1024)), drr.DRR_ERR_UNSUPPORTED),
 ]
 

@@ -16,7 +16,7 @@ import pytest
 
 import oracle
 from cone_beam_ct_b200 import workloads as wl
-from tests.gpu_helpers import (BF16, CORNERS, F32, LAYOUTS, LINEAR, PADDED, assert_parity,
+from tests.gpu_helpers import (BF16, CORNERS, F32, LAYOUTS, LINEAR, PADDED, QUADS, assert_parity,
                                bf16_values, gpu_forward)
 
 pytestmark = pytest.mark.gpu
@@ -136,8 +136,9 @@ def test_layouts_agree(cuda):
     w = wl.small_random_case(105, H=64, W=64)
     for dtype in (F32, BF16):
         a = gpu_forward(w, layout=LINEAR, dtype=dtype)
-        # same positions, fractions and lerps: the corner layout is bit-identical
+        # same positions, fractions and lerps: corner records and quads are bit-identical
         assert np.array_equal(a, gpu_forward(w, layout=CORNERS, dtype=dtype))
+        assert np.array_equal(a, gpu_forward(w, layout=QUADS, dtype=dtype))
         assert_parity(a, gpu_forward(w, layout=PADDED, dtype=dtype), 1e-5, what="linear vs padded")
 
 
@@ -216,6 +217,12 @@ def test_prepare_layouts_round_trip(cuda):
                 border = p.copy()
                 border[1:-1, 1:-1, 1:-1] = 0
                 assert np.all(border == 0)
+            elif layout == QUADS:
+                # voxel (i + a, j + b, k) of quad (i, j, k) at element a + 2b
+                rec = a.reshape(nz, ny - 1, nx - 1, 4)
+                for e in range(4):
+                    da, db = e & 1, e >> 1
+                    assert np.array_equal(rec[..., e], expect[:, db:ny - 1 + db, da:nx - 1 + da])
             else:
                 # corner (a, b, c) of cell (i, j, k) at element a + 2b + 4c
                 rec = a.reshape(nz - 1, ny - 1, nx - 1, 8)
