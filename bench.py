@@ -2,8 +2,9 @@
 """Throughput of the cone-beam DRR hot path on B200 (one JSON line on stdout).
 
 A step is one pass of the whole path over one batch of synthetic input:
-prepare the volume (fp32 -> corner-record layout, bf16 for the bf16
-workload), forward ray-march of every view, zero the gradient volume,
+prepare the volume (fp32 -> corner records or xy quads, whichever the
+workload's forward runs faster in; bf16 for the bf16 workload), forward
+ray-march of every view, zero the gradient volume,
 adjoint scatter of an N(0,1) upstream gradient (with a workspace, so that
 dense views take the corner-record path).  The default workload is the
 256^3 bf16 volume seen by 4 C-arm views of 1024x1024 pixels with 512
@@ -50,8 +51,10 @@ def parse_args():
     p.add_argument("--config", type=int, default=3, choices=[1, 2, 3, 4],
                    help="workload (default 3: 256^3 bf16, 4 views 1024x1024, 512 samples, "
                         "the size the throughput target is quoted at)")
-    p.add_argument("--layout", choices=["padded", "corners", "quads", "linear"], default="corners",
-                   help="volume layout drr_prepare_volume writes for the forward")
+    p.add_argument("--layout", choices=["auto", "padded", "corners", "quads", "linear"],
+                   default="auto",
+                   help="volume layout drr_prepare_volume writes for the forward (auto: the "
+                        "faster one measured for the workload, AUTO_LAYOUT)")
     p.add_argument("--texture", action="store_true",
                    help="also time the texture-trilinear comparison forward (libdrr_texture.so)")
     p.add_argument("--pose", action="store_true",
@@ -93,6 +96,15 @@ def job_throughput(world, units_per_rank_step, steps, max_ms):
 
 # ---------------------------------------------------------------------------
 # workload description
+
+# The layout each workload's forward runs fastest in on B200: corner records
+# (one load per sample) where dense rays reuse them in L1, xy quads (half the
+# footprint) where sparse views re-read an fp32 volume from DRAM.  Forward
+# times measured: 256^3 fp32 seen by 64 views of 200^2, quads 2.17 / corners
+# 2.96 ms; 256^3 bf16 seen by 4 views of 1024^2, corners 2.87 / quads 3.88 ms;
+# 512^3 fp32 seen by 2 views of 2048^2, corners 3.97 / quads 4.49 ms.
+AUTO_LAYOUT = {1: "corners", 2: "quads", 3: "corners", 4: "corners"}
+
 
 def workload(cfg):
     from cone_beam_ct_b200 import workloads as wl
@@ -422,8 +434,9 @@ def _median_ms(torch, fn, reps=10, flush=None):
 def alpha_timing(torch, w, vol32, prep, dtype, layout, Rt, grad_out, elem, l2_peak, hbm_peak,
                  vol_fits_l2):
     """Alpha compositing on the same workload (forward from the prepared
-    volume, volume gradient from it when it is linear or corner records),
-    and the surrogate on its image: median of 10, L2 flushed before each."""
+    volume; volume gradient from it, with and without a workspace, unless it
+    is zero-bordered), and the surrogate on its image: median of 10, L2
+    flushed before each."""
     from cone_beam_ct_b200 import drr
     dev = vol32.device
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
@@ -435,13 +448,23 @@ def alpha_timing(torch, w, vol32, prep, dtype, layout, Rt, grad_out, elem, l2_pe
         drr.drr_render(prep, dtype, layout, w.dims, w.spacing, w.origin, w.K, Rt, w.B, w.H, w.W,
                        w.n_samples, w.density_factor, drr.DRR_MODE_ALPHA, out, stream=stream)
 
-    def adj():
-        drr.drr_render_alpha_adjoint(prep, dtype, layout, w.dims, w.spacing, w.origin, w.K, Rt,
-                                     w.B, w.H, w.W, w.n_samples, w.density_factor, grad_out, out,
-                                     grad, stream=stream)
+    ws = torch.empty(drr.drr_adjoint_workspace_bytes(w.dims, w.B), dtype=torch.uint8, device=dev)
+
+    def adj(workspace):
+        if workspace:
+            drr.drr_render_alpha_adjoint_ws(prep, dtype, layout, w.dims, w.spacing, w.origin, w.K,
+                                            Rt, w.B, w.H, w.W, w.n_samples, w.density_factor,
+                                            grad_out, out, grad, ws, stream=stream)
+        else:
+            drr.drr_render_alpha_adjoint(prep, dtype, layout, w.dims, w.spacing, w.origin, w.K,
+                                         Rt, w.B, w.H, w.W, w.n_samples, w.density_factor,
+                                         grad_out, out, grad, stream=stream)
 
     fwd_ms = _median_ms(torch, fwd, flush=flush)
-    adj_ms = _median_ms(torch, adj, flush=flush) if layout != drr.DRR_LAYOUT_PADDED else None
+    adj_ms = direct_ms = None
+    if layout != drr.DRR_LAYOUT_PADDED:
+        adj_ms = _median_ms(torch, lambda: adj(True), flush=flush)
+        direct_ms = _median_ms(torch, lambda: adj(False), flush=flush)
     bound, peak = ("l2", l2_peak) if vol_fits_l2 and l2_peak else ("hbm", hbm_peak)
 
     def roof(kernel, ms, nbytes):
@@ -465,7 +488,9 @@ def alpha_timing(torch, w, vol32, prep, dtype, layout, Rt, grad_out, elem, l2_pe
                          "backward_hbm_gbs": 16 * n / (noise_bwd_ms * 1e-3) / 1e9}}
     if adj_ms is not None:
         res["adjoint"] = {"ms": adj_ms, "gsamples_s": w.samples / (adj_ms * 1e-3) / 1e9,
-                          "roofline": roof("alpha_adjoint_kernel", adj_ms, 32 * w.samples)}
+                          "roofline": roof("alpha adjoint (with a workspace)", adj_ms,
+                                           32 * w.samples),
+                          "without_workspace_ms": direct_ms}
     return res
 
 
@@ -551,6 +576,8 @@ def run_ours(args):
     drr.lib()
 
     w = workload(args.config)
+    if args.layout == "auto":
+        args.layout = AUTO_LAYOUT[args.config]
     layout = {"padded": drr.DRR_LAYOUT_PADDED, "corners": drr.DRR_LAYOUT_CORNERS,
               "quads": drr.DRR_LAYOUT_QUADS, "linear": drr.DRR_LAYOUT_LINEAR}[args.layout]
     dtype = drr.DRR_BF16 if w.dtype == wl.DTYPE_BF16 else drr.DRR_F32

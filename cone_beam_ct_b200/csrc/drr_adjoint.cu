@@ -130,6 +130,11 @@ __device__ __forceinline__ void flush_record(float* __restrict__ rec, int cell, 
     atomicAdd(p, make_float4(a[0], a[1], a[2], a[3]));
     atomicAdd(p + 1, make_float4(a[4], a[5], a[6], a[7]));
 }
+__device__ __forceinline__ void flush_record(float* __restrict__ rec, int cell, const float2 a[4]) {
+    float4* p = reinterpret_cast<float4*>(rec + (size_t)cell * 8);
+    atomicAdd(p, make_float4(a[0].x, a[0].y, a[1].x, a[1].y));
+    atomicAdd(p + 1, make_float4(a[2].x, a[2].y, a[3].x, a[3].y));
+}
 
 // Workspace layout (drr_render_adjoint_ws): a 256-byte aligned header of
 // ints -- [0] "some view is dense", [1 + b] "view b is dense" -- then the
@@ -299,8 +304,12 @@ adjoint_kernel(const float* __restrict__ Rt, const float* __restrict__ grad_out,
 // spread over the tile (7.1 vs 7.8 ms); 3 x 2 bundles flush 11 % less than
 // 2 x 2 (0.26 against 0.30 flushes per ray-sample) and run 3 % / 8 % faster;
 // a least-recently-used slot choice flushes less still but its extra
-// branches doubled the issued instructions; packed fp32x2 weights saturate
-// the FMA pipe instead.
+// branches doubled the issued instructions.  Letting a miss share the home
+// slot's add (two divergent paths instead of three) took 7.12 to 6.65 ms at
+// 1024^2 x 512, and packed fp32x2 weights and sums then 6.55 ms; summing
+// the 8 trilinear moments instead of the 8 weights (fewer multiplies per
+// sample, converted at flush) was slower (6.83 ms), and a third, victim slot much
+// slower (8.6 ms, spills; 11.0 ms at 149 registers and 1 CTA per SM).
 constexpr int kBundleX = 3, kBundleY = 2;        // rays per bundle, across and down
 constexpr int kBundleRays = kBundleX * kBundleY;
 constexpr int kSlots = 2;
@@ -350,7 +359,7 @@ records_kernel(const float* __restrict__ Rt, const float* __restrict__ grad_out,
     }
     // cells stay in [0, n-2] per axis (linear-layout lim), inside the records
     const int cr = g.nx - 1, cs = (g.nx - 1) * (g.ny - 1);
-    float p[kSlots][8];
+    float2 p[kSlots][4];
     int pc[kSlots];
     for (int pass = 0; pass < 2; ++pass) {
         const int i0 = pass == 0 ? start : 0;
@@ -375,31 +384,34 @@ records_kernel(const float* __restrict__ Rt, const float* __restrict__ grad_out,
                 const float wz1 = scale[k] * fz, wz0 = scale[k] * (1.0f - fz);
                 const float w00 = wz0 * (1.0f - fy), w01 = wz0 * fy;
                 const float w10 = wz1 * (1.0f - fy), w11 = wz1 * fy;
-                const float gx = 1.0f - fx;
-                const float w[8] = {w00 * gx, w00 * fx, w01 * gx, w01 * fx,
-                                    w10 * gx, w10 * fx, w11 * gx, w11 * fx};
+                // corner pairs (a = 0, 1) as packed fp32x2: 4 FMUL2 and 4 FADD2
+                const float2 fxp = make_float2(1.0f - fx, fx);
+                const float2 w[4] = {__fmul2_rn(make_float2(w00, w00), fxp),
+                                     __fmul2_rn(make_float2(w01, w01), fxp),
+                                     __fmul2_rn(make_float2(w10, w10), fxp),
+                                     __fmul2_rn(make_float2(w11, w11), fxp)};
                 const int home = k / kBundleX;   // upper row -> slot 0, lower row -> slot 1
                 const int other = 1 - home;
-                if (pc[home] == cell) {
-#pragma unroll
-                    for (int h = 0; h < kSlots; ++h)
-                        if (h == home)
-#pragma unroll
-                            for (int e = 0; e < 8; ++e) p[h][e] += w[e];
-                } else if (pc[other] == cell) {
+                // two paths, not three: a miss flushes and clears the home
+                // slot, then shares the home slot's add
+                if (pc[other] == cell && pc[home] != cell) {
 #pragma unroll
                     for (int h = 0; h < kSlots; ++h)
                         if (h == other)
 #pragma unroll
-                            for (int e = 0; e < 8; ++e) p[h][e] += w[e];
+                            for (int e = 0; e < 4; ++e) p[h][e] = __fadd2_rn(p[h][e], w[e]);
                 } else {
 #pragma unroll
                     for (int h = 0; h < kSlots; ++h) {
                         if (h != home) continue;
-                        if (pc[h] >= 0) flush_record(ws.rec, pc[h], p[h]);
-                        pc[h] = cell;
+                        if (pc[h] != cell) {
+                            if (pc[h] >= 0) flush_record(ws.rec, pc[h], p[h]);
+                            pc[h] = cell;
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) p[h][e] = w[e];
+                            for (int e = 0; e < 4; ++e) p[h][e] = make_float2(0.0f, 0.0f);
+                        }
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) p[h][e] = __fadd2_rn(p[h][e], w[e]);
                     }
                 }
             }
@@ -426,9 +438,11 @@ template <typename T, int LAYOUT>
 __global__ void __launch_bounds__(kThreads)
 alpha_adjoint_kernel(const T* __restrict__ vol, const float* __restrict__ Rt,
                      const float* __restrict__ grad_out, const float* __restrict__ fwd_out,
-                     float* __restrict__ grad, const Geom g, int grad_row, int grad_slice) {
+                     float* __restrict__ grad, const Geom g, int grad_row, int grad_slice,
+                     const int* __restrict__ flags) {
     __shared__ View sv;
     const int b = blockIdx.z;
+    if (flags && flags[1 + b]) return;           // dense view: alpha_records_kernel's
     if (threadIdx.x == 0) view_setup(Rt + 12 * (size_t)b, g, sv);
     __syncthreads();
     int r, c;
@@ -490,6 +504,115 @@ alpha_adjoint_kernel(const T* __restrict__ vol, const float* __restrict__ Rt,
         qz += ray.s[2];
     }
     flush_block(grad, st, cell, a8);
+}
+
+// Record path of the alpha gradient for the views the plan marked dense: the
+// per-sample factor of alpha_adjoint_kernel, accumulated like records_kernel.
+// Each thread owns a 2 x 2 bundle of neighbouring rays (a CTA a 32 x 32 pixel
+// tile) and two record slots, home to the bundle's rows; every ray carries
+// its own T and C_i front to back, so there are no phases.  2 x 2 rather
+// than 3 x 2: each ray also holds its sampling and compositing state.
+constexpr int kAlphaBundle = 2;                          // rays per bundle, across and down
+constexpr int kAlphaTile = 16 * kAlphaBundle;            // 32 x 32 pixels per CTA
+
+template <typename T, int LAYOUT>
+__global__ void __launch_bounds__(kThreads, 2)
+alpha_records_kernel(const T* __restrict__ vol, const float* __restrict__ Rt,
+                     const float* __restrict__ grad_out, const float* __restrict__ fwd_out,
+                     const Geom g, const Workspace ws) {
+    constexpr int kRays = kAlphaBundle * kAlphaBundle;
+    __shared__ View sv;
+    const int b = blockIdx.z;
+    if (ws.flags[1 + b] == 0) return;            // sparse view: alpha_adjoint_kernel's
+    if (threadIdx.x == 0) view_setup(Rt + 12 * (size_t)b, g, sv);
+    __syncthreads();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int px = (warp & 1) * 8 + (lane & 7), py = (warp >> 1) * 4 + (lane >> 3);
+    const int c0 = blockIdx.x * kAlphaTile + px * kAlphaBundle;
+    const int r0 = blockIdx.y * kAlphaTile + py * kAlphaBundle;
+
+    bool act[kRays];
+    float go[kRays], sa[kRays], Cray[kRays], Ci[kRays], Tr[kRays];
+    long long q[kRays][3], s[kRays][3];
+#pragma unroll
+    for (int k = 0; k < kRays; ++k) {
+        const int c = c0 + (k % kAlphaBundle), r = r0 + (k / kAlphaBundle);
+        act[k] = false;
+        go[k] = sa[k] = Cray[k] = Ci[k] = 0.0f;
+        Tr[k] = 1.0f;
+#pragma unroll
+        for (int a = 0; a < 3; ++a) q[k][a] = s[k][a] = 0;
+        if (r >= g.H || c >= g.W) continue;
+        const size_t pix = ((size_t)b * g.H + r) * g.W + c;
+        go[k] = grad_out[pix];
+        Ray ray;
+        if (go[k] == 0.0f || !ray_setup(sv, g, (double)c, (double)r, 0.0, ray)) continue;
+        act[k] = true;
+        Cray[k] = fwd_out[pix];
+        sa[k] = g.density_factor * ray.dt;
+#pragma unroll
+        for (int a = 0; a < 3; ++a) {
+            s[k][a] = ray.s[a];
+            q[k][a] = ray.q0[a];
+        }
+    }
+    // cells stay in [0, n-2] per axis (lim as for the linear layout), inside the records
+    const int cr = g.nx - 1, cs = (g.nx - 1) * (g.ny - 1);
+    float p[kSlots][8];
+    int pc[kSlots];
+#pragma unroll
+    for (int h = 0; h < kSlots; ++h) pc[h] = -1;
+    for (int i = 0; i < g.N; ++i) {
+#pragma unroll
+        for (int k = 0; k < kRays; ++k) {
+            if (!act[k]) continue;
+            const int cx = fix_cell(q[k][0]), cy = fix_cell(q[k][1]), cz = fix_cell(q[k][2]);
+            const float fx = fix_frac(q[k][0]), fy = fix_frac(q[k][1]), fz = fix_frac(q[k][2]);
+#pragma unroll
+            for (int a = 0; a < 3; ++a) q[k][a] += s[k][a];
+            // the forward's sample value, bit for bit
+            const int at = cz * g.slice + cy * g.row + cx;
+            const float mu = LAYOUT == 2   ? sample_corners(vol + (size_t)at * 8, fx, fy, fz)
+                             : LAYOUT == 3 ? sample_quads(vol + (size_t)at * 4, g.slice, fx, fy, fz)
+                                           : trilinear_at(vol + at, g.row, g.slice, fx, fy, fz);
+            const float a = -expm1f(-sa[k] * mu);
+            Ci[k] = fmaf(Tr[k] * a, mu, Ci[k]);
+            const float dmu = Tr[k] * fmaf(sa[k] * (1.0f - a), mu, a) - sa[k] * (Cray[k] - Ci[k]);
+            Tr[k] *= 1.0f - a;
+            const float scale = go[k] * dmu;
+            const int cell = cz * cs + cy * cr + cx;
+            const float wz1 = scale * fz, wz0 = scale * (1.0f - fz);
+            const float w00 = wz0 * (1.0f - fy), w01 = wz0 * fy;
+            const float w10 = wz1 * (1.0f - fy), w11 = wz1 * fy;
+            const float gx = 1.0f - fx;
+            const float w[8] = {w00 * gx, w00 * fx, w01 * gx, w01 * fx,
+                                w10 * gx, w10 * fx, w11 * gx, w11 * fx};
+            const int home = k / kAlphaBundle, other = 1 - home;
+            if (pc[other] == cell && pc[home] != cell) {
+#pragma unroll
+                for (int h = 0; h < kSlots; ++h)
+                    if (h == other)
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) p[h][e] += w[e];
+            } else {
+#pragma unroll
+                for (int h = 0; h < kSlots; ++h) {
+                    if (h != home) continue;
+                    if (pc[h] != cell) {
+                        if (pc[h] >= 0) flush_record(ws.rec, pc[h], p[h]);
+                        pc[h] = cell;
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) p[h][e] = 0.0f;
+                    }
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) p[h][e] += w[e];
+                }
+            }
+        }
+    }
+#pragma unroll
+    for (int h = 0; h < kSlots; ++h)
+        if (pc[h] >= 0) flush_record(ws.rec, pc[h], p[h]);
 }
 
 constexpr int kMaxDevices = 64;
@@ -556,32 +679,47 @@ cudaError_t launch_adjoint(const Geom& g, const float* Rt, int mode, const float
     return cudaGetLastError();
 }
 
+template <typename T, int LAYOUT>
+void alpha_kernels(const void* vol, const Geom& g, const float* Rt, const float* grad_out,
+                   const float* fwd_out, float* grad_vol, const Workspace& ws,
+                   cudaStream_t stream) {
+    const T* v = static_cast<const T*>(vol);
+    const dim3 grid((g.W + kTileW - 1) / kTileW, (g.H + kTileH - 1) / kTileH, g.B);
+    alpha_adjoint_kernel<T, LAYOUT><<<grid, kThreads, 0, stream>>>(
+        v, Rt, grad_out, fwd_out, grad_vol, g, g.nx, g.nx * g.ny, ws.flags);
+    if (ws.flags) {
+        const dim3 rgrid((g.W + kAlphaTile - 1) / kAlphaTile, (g.H + kAlphaTile - 1) / kAlphaTile,
+                         g.B);
+        alpha_records_kernel<T, LAYOUT><<<rgrid, kThreads, 0, stream>>>(v, Rt, grad_out, fwd_out,
+                                                                         g, ws);
+    }
+}
+
 cudaError_t launch_alpha_adjoint(const void* vol, int dtype, int layout, const Geom& g,
                                  const float* Rt, const float* grad_out, const float* fwd_out,
-                                 float* grad_vol, cudaStream_t stream) {
-    const dim3 grid((g.W + kTileW - 1) / kTileW, (g.H + kTileH - 1) / kTileH, g.B);
-    const int grow = g.nx, gslice = g.nx * g.ny;
-    if (layout == 3) {
-        if (dtype == 0)
-            alpha_adjoint_kernel<float, 3><<<grid, kThreads, 0, stream>>>(
-                static_cast<const float*>(vol), Rt, grad_out, fwd_out, grad_vol, g, grow, gslice);
-        else
-            alpha_adjoint_kernel<uint16_t, 3><<<grid, kThreads, 0, stream>>>(
-                static_cast<const uint16_t*>(vol), Rt, grad_out, fwd_out, grad_vol, g, grow, gslice);
-        return cudaGetLastError();
+                                 float* grad_vol, void* workspace, cudaStream_t stream) {
+    Workspace ws{nullptr, nullptr};
+    const int fill_grid = 148 * 8;
+    if (workspace) {
+        ws.flags = static_cast<int*>(workspace);
+        ws.rec = reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                          adjoint_workspace_header(g.B));
+        const int64_t n_rec4 = (int64_t)(g.nx - 1) * (g.ny - 1) * (g.nz - 1) * 2;
+        plan_views<<<1, 256, 0, stream>>>(Rt, g, ws.flags);
+        zero_records<<<fill_grid, 256, 0, stream>>>(ws.flags, reinterpret_cast<float4*>(ws.rec),
+                                                    n_rec4);
     }
-    if (dtype == 0 && layout == 2)
-        alpha_adjoint_kernel<float, 2><<<grid, kThreads, 0, stream>>>(
-            static_cast<const float*>(vol), Rt, grad_out, fwd_out, grad_vol, g, grow, gslice);
-    else if (dtype == 0)
-        alpha_adjoint_kernel<float, 0><<<grid, kThreads, 0, stream>>>(
-            static_cast<const float*>(vol), Rt, grad_out, fwd_out, grad_vol, g, grow, gslice);
-    else if (layout == 2)
-        alpha_adjoint_kernel<uint16_t, 2><<<grid, kThreads, 0, stream>>>(
-            static_cast<const uint16_t*>(vol), Rt, grad_out, fwd_out, grad_vol, g, grow, gslice);
-    else
-        alpha_adjoint_kernel<uint16_t, 0><<<grid, kThreads, 0, stream>>>(
-            static_cast<const uint16_t*>(vol), Rt, grad_out, fwd_out, grad_vol, g, grow, gslice);
+    if (dtype == 0) {
+        if (layout == 3) alpha_kernels<float, 3>(vol, g, Rt, grad_out, fwd_out, grad_vol, ws, stream);
+        else if (layout == 2) alpha_kernels<float, 2>(vol, g, Rt, grad_out, fwd_out, grad_vol, ws, stream);
+        else alpha_kernels<float, 0>(vol, g, Rt, grad_out, fwd_out, grad_vol, ws, stream);
+    } else {
+        if (layout == 3) alpha_kernels<uint16_t, 3>(vol, g, Rt, grad_out, fwd_out, grad_vol, ws, stream);
+        else if (layout == 2) alpha_kernels<uint16_t, 2>(vol, g, Rt, grad_out, fwd_out, grad_vol, ws, stream);
+        else alpha_kernels<uint16_t, 0>(vol, g, Rt, grad_out, fwd_out, grad_vol, ws, stream);
+    }
+    if (workspace)
+        gather_records<<<fill_grid, 256, 0, stream>>>(ws.flags, ws.rec, grad_vol, g.nx, g.ny, g.nz);
     return cudaGetLastError();
 }
 

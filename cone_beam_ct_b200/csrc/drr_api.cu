@@ -334,12 +334,16 @@ DRR_API drr_status drr_render_pose_grad(const void* vol, drr_dtype dtype, drr_la
 
 extern "C" {
 
-DRR_API drr_status drr_render_alpha_adjoint(const void* vol, drr_dtype dtype, drr_layout layout,
-                                            const int dims[3], const float spacing[3],
-                                            const float origin[3], const float K[9],
-                                            const float* Rt, int B, int H, int W, int n_samples,
-                                            float density_factor, const float* grad_out,
-                                            const float* fwd_out, float* grad_vol, void* stream) {
+}  // extern "C"
+
+namespace {
+
+drr_status render_alpha_adjoint(const void* vol, drr_dtype dtype, drr_layout layout,
+                                const int dims[3], const float spacing[3], const float origin[3],
+                                const float K[9], const float* Rt, int B, int H, int W,
+                                int n_samples, float density_factor, const float* grad_out,
+                                const float* fwd_out, float* grad_vol, bool with_ws,
+                                void* workspace, size_t workspace_bytes, void* stream) {
     drr_status st = check_volume(dims, spacing, origin);
     if (st != DRR_OK) return st;
     st = check_rays(K, Rt, B, H, W, n_samples, density_factor, DRR_MODE_ALPHA, true);
@@ -366,11 +370,51 @@ DRR_API drr_status drr_render_alpha_adjoint(const void* vol, drr_dtype dtype, dr
     if (overlaps(grad_vol, vbytes, grad_out, ibytes) || overlaps(grad_vol, vbytes, fwd_out, ibytes) ||
         overlaps(grad_vol, vbytes, vol, sbytes))
         return fail(DRR_ERR_INVALID_ARG, "grad_vol overlaps another buffer");
+    if (with_ws) {
+        const size_t need = drr::adjoint_workspace_bytes(dims[0], dims[1], dims[2], B);
+        if (!workspace || !aligned(workspace, 256))
+            return fail(DRR_ERR_INVALID_ARG, "workspace must be a non-NULL, 256-byte aligned device pointer");
+        if (workspace_bytes < need)
+            return fail(DRR_ERR_INVALID_ARG, "workspace holds %zu bytes, %zu needed", workspace_bytes, need);
+        if (overlaps(workspace, need, grad_vol, vbytes) || overlaps(workspace, need, grad_out, ibytes) ||
+            overlaps(workspace, need, fwd_out, ibytes) || overlaps(workspace, need, vol, sbytes) ||
+            overlaps(workspace, need, Rt, (size_t)B * 12 * sizeof(float)))
+            return fail(DRR_ERR_INVALID_ARG, "workspace overlaps another buffer");
+    }
     drr::Geom g;
     drr::fill_geom(g, dims, spacing, origin, K, B, H, W, n_samples, density_factor, layout);
     return cuda_status(drr::launch_alpha_adjoint(vol, dtype, layout, g, Rt, grad_out, fwd_out,
-                                                 grad_vol, static_cast<cudaStream_t>(stream)),
+                                                 grad_vol, with_ws ? workspace : nullptr,
+                                                 static_cast<cudaStream_t>(stream)),
                        "drr_render_alpha_adjoint launch");
+}
+
+}  // namespace
+
+extern "C" {
+
+DRR_API drr_status drr_render_alpha_adjoint(const void* vol, drr_dtype dtype, drr_layout layout,
+                                            const int dims[3], const float spacing[3],
+                                            const float origin[3], const float K[9],
+                                            const float* Rt, int B, int H, int W, int n_samples,
+                                            float density_factor, const float* grad_out,
+                                            const float* fwd_out, float* grad_vol, void* stream) {
+    return render_alpha_adjoint(vol, dtype, layout, dims, spacing, origin, K, Rt, B, H, W,
+                                n_samples, density_factor, grad_out, fwd_out, grad_vol, false,
+                                nullptr, 0, stream);
+}
+
+DRR_API drr_status drr_render_alpha_adjoint_ws(const void* vol, drr_dtype dtype, drr_layout layout,
+                                               const int dims[3], const float spacing[3],
+                                               const float origin[3], const float K[9],
+                                               const float* Rt, int B, int H, int W,
+                                               int n_samples, float density_factor,
+                                               const float* grad_out, const float* fwd_out,
+                                               float* grad_vol, void* workspace,
+                                               size_t workspace_bytes, void* stream) {
+    return render_alpha_adjoint(vol, dtype, layout, dims, spacing, origin, K, Rt, B, H, W,
+                                n_samples, density_factor, grad_out, fwd_out, grad_vol, true,
+                                workspace, workspace_bytes, stream);
 }
 
 DRR_API drr_status drr_poisson_noise(const float* image, const float* z, float i0, float* out,

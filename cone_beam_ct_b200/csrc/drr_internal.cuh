@@ -250,9 +250,11 @@ cudaError_t launch_adjoint_noalloc(const Geom& g, const float* Rt, int mode, con
                                    const float* fwd_out, float* grad_vol, cudaStream_t stream);
 cudaError_t launch_prepare(const float* src, int nx, int ny, int nz, int dtype, int layout,
                            void* dst, cudaStream_t stream);
+// workspace: NULL (every view on the direct path) or the layout of
+// adjoint_workspace_bytes (dense views accumulate into corner records)
 cudaError_t launch_alpha_adjoint(const void* vol, int dtype, int layout, const Geom& g,
                                  const float* Rt, const float* grad_out, const float* fwd_out,
-                                 float* grad_vol, cudaStream_t stream);
+                                 float* grad_vol, void* workspace, cudaStream_t stream);
 cudaError_t launch_poisson_noise(const float* image, const float* z, float i0, float* out,
                                  int64_t n, cudaStream_t stream);
 cudaError_t launch_poisson_noise_backward(const float* image, const float* z, float i0,

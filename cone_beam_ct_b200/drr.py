@@ -22,7 +22,7 @@ DRR_LAYOUT_LINEAR, DRR_LAYOUT_PADDED, DRR_LAYOUT_CORNERS, DRR_LAYOUT_QUADS = 0, 
 # names exported by libdrr.so (include/drr.h)
 EXPORTED = ("drr_render", "drr_render_adjoint", "drr_render_adjoint_ws",
             "drr_adjoint_workspace_bytes", "drr_render_adjoint_noalloc", "drr_render_pose_grad",
-            "drr_render_alpha_adjoint", "drr_poisson_noise", "drr_poisson_noise_backward",
+            "drr_render_alpha_adjoint", "drr_render_alpha_adjoint_ws", "drr_poisson_noise", "drr_poisson_noise_backward",
             "drr_render_siddon", "drr_render_siddon_adjoint", "drr_render_batched",
             "drr_render_adjoint_batched",
             "drr_prepared_bytes", "drr_prepare_volume", "drr_get_last_error", "drr_abi_version")
@@ -74,6 +74,10 @@ def lib():
                                            _c.c_int, _c.c_int, _c.c_int, _c.c_int, _c.c_float,
                                            _vp, _vp, _vp, _vp]
     L.drr_render_alpha_adjoint.restype = _c.c_int
+    L.drr_render_alpha_adjoint_ws.argtypes = [_vp, _c.c_int, _c.c_int, _i3, _f3, _f3, _f9, _vp,
+                                              _c.c_int, _c.c_int, _c.c_int, _c.c_int, _c.c_float,
+                                              _vp, _vp, _vp, _vp, _c.c_size_t, _vp]
+    L.drr_render_alpha_adjoint_ws.restype = _c.c_int
     L.drr_poisson_noise.argtypes = [_vp, _vp, _c.c_float, _vp, _c.c_int64, _vp]
     L.drr_poisson_noise.restype = _c.c_int
     L.drr_poisson_noise_backward.argtypes = [_vp, _vp, _c.c_float, _vp, _vp, _c.c_int64, _vp]
@@ -213,6 +217,22 @@ def drr_render_alpha_adjoint(vol, dtype, layout, dims, spacing, origin, K, Rt, B
                                           _dev(grad_out, "grad_out", True),
                                           _dev(fwd_out, "fwd_out", True),
                                           _dev(grad_vol, "grad_vol", True), _stream(stream)))
+
+
+def drr_render_alpha_adjoint_ws(vol, dtype, layout, dims, spacing, origin, K, Rt, B, H, W,
+                                n_samples, density_factor, grad_out, fwd_out, grad_vol, workspace,
+                                workspace_bytes=None, stream=None):
+    if workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    _check(lib().drr_render_alpha_adjoint_ws(_dev(vol, "vol", True), int(dtype), int(layout),
+                                             _i3v(dims), _f3v(spacing), _f3v(origin), _f9v(K),
+                                             _dev(Rt, "Rt", True), int(B), int(H), int(W),
+                                             int(n_samples), float(density_factor),
+                                             _dev(grad_out, "grad_out", True),
+                                             _dev(fwd_out, "fwd_out", True),
+                                             _dev(grad_vol, "grad_vol", True),
+                                             _dev(workspace, "workspace", True),
+                                             int(workspace_bytes), _stream(stream)))
 
 
 def drr_poisson_noise(image, z, i0, out, n=None, stream=None):

@@ -259,8 +259,9 @@ DRR_API drr_status drr_render_pose_grad(const void *vol, drr_dtype dtype, drr_la
  * ray's image value, dC/dmu_i = T_i (s (1 - a_i) mu_i + a_i) - s (C - C_i),
  * s = density_factor * dt; each sample's value is scattered with its
  * trilinear weights.  One pass per ray, front to back.
- *   vol, dtype, layout  the forward's volume: DRR_LAYOUT_LINEAR or
- *               DRR_LAYOUT_CORNERS (DRR_LAYOUT_PADDED: DRR_ERR_UNSUPPORTED).
+ *   vol, dtype, layout  the forward's volume: DRR_LAYOUT_LINEAR,
+ *               DRR_LAYOUT_CORNERS or DRR_LAYOUT_QUADS (DRR_LAYOUT_PADDED:
+ *               DRR_ERR_UNSUPPORTED).
  *   grad_out    DEVICE float[B*H*W], upstream gradient dL/d(out).
  *   fwd_out     DEVICE float[B*H*W], the alpha image of this volume and these
  *               poses (drr_render with DRR_MODE_ALPHA), required.
@@ -273,6 +274,27 @@ DRR_API drr_status drr_render_alpha_adjoint(const void *vol, drr_dtype dtype, dr
                                             const float *Rt, int B, int H, int W, int n_samples,
                                             float density_factor, const float *grad_out,
                                             const float *fwd_out, float *grad_vol, void *stream);
+
+/* drr_render_alpha_adjoint with a caller-provided workspace, for speed:
+ * views whose rays are much closer than a voxel (the test of
+ * drr_render_adjoint_ws) accumulate into per-cell corner records, which a
+ * final pass adds into grad_vol; other views scatter directly.  Same result
+ * up to fp32 summation order.
+ *   workspace        DEVICE, 256-byte aligned, at least
+ *                    drr_adjoint_workspace_bytes(dims, B) bytes; content on
+ *                    entry ignored, on return unspecified; must not overlap
+ *                    any other buffer of the call.
+ *   workspace_bytes  bytes available at workspace.
+ * Calls that share one workspace must not overlap on the GPU.  Other
+ * arguments as drr_render_alpha_adjoint. */
+DRR_API drr_status drr_render_alpha_adjoint_ws(const void *vol, drr_dtype dtype, drr_layout layout,
+                                               const int dims[3], const float spacing[3],
+                                               const float origin[3], const float K[9],
+                                               const float *Rt, int B, int H, int W,
+                                               int n_samples, float density_factor,
+                                               const float *grad_out, const float *fwd_out,
+                                               float *grad_vol, void *workspace,
+                                               size_t workspace_bytes, void *stream);
 
 /* Gaussian-Poisson surrogate of shot noise (flashdrr.rendering API docs,
  * VolumeRaycaster.apply_poisson) on a Beer-Lambert image: with transmission

@@ -134,8 +134,9 @@ def assert_pose_parity(got, ref, tol, what=""):
     return worst
 
 
-def gpu_alpha_adjoint(w, grad_out, fwd_out, layout=LINEAR, dtype=F32):
-    """Volume gradient of the alpha image through drr_render_alpha_adjoint."""
+def gpu_alpha_adjoint(w, grad_out, fwd_out, layout=LINEAR, dtype=F32, workspace=False):
+    """Volume gradient of the alpha image through drr_render_alpha_adjoint, or
+    drr_render_alpha_adjoint_ws with a fresh workspace filled with garbage."""
     import torch
     v32, Rt_d = device_inputs(w)
     src = prepared(v32, w.dims, dtype, layout)
@@ -143,8 +144,15 @@ def gpu_alpha_adjoint(w, grad_out, fwd_out, layout=LINEAR, dtype=F32):
     fo = torch.from_numpy(np.ascontiguousarray(fwd_out, dtype=np.float32)).cuda()
     nx, ny, nz = w.dims
     grad = torch.zeros((nz, ny, nx), dtype=torch.float32, device="cuda")
-    drr.drr_render_alpha_adjoint(src, dtype, layout, w.dims, w.spacing, w.origin, w.K, Rt_d, w.B,
-                                 w.H, w.W, w.n_samples, w.density_factor, go, fo, grad)
+    if workspace:
+        nbytes = drr.drr_adjoint_workspace_bytes(w.dims, w.B)
+        ws = torch.full((nbytes,), 0x7F, dtype=torch.uint8, device="cuda")
+        drr.drr_render_alpha_adjoint_ws(src, dtype, layout, w.dims, w.spacing, w.origin, w.K,
+                                        Rt_d, w.B, w.H, w.W, w.n_samples, w.density_factor, go,
+                                        fo, grad, ws)
+    else:
+        drr.drr_render_alpha_adjoint(src, dtype, layout, w.dims, w.spacing, w.origin, w.K, Rt_d,
+                                     w.B, w.H, w.W, w.n_samples, w.density_factor, go, fo, grad)
     torch.cuda.synchronize()
     return grad.cpu().numpy()
 

@@ -259,6 +259,40 @@ def test_alpha_adjoint_rejects_bad_arguments(kw, status, word):
     assert word in drr.drr_get_last_error()
 
 
+def _alpha_adjoint_ws(**kw):
+    args = dict(vol=FAKE, dtype=drr.DRR_F32, layout=drr.DRR_LAYOUT_LINEAR, dims=DIMS, spacing=SP,
+                origin=ORG, K=K_OK, Rt=FAKE + (1 << 26), B=2, H=8, W=8, n_samples=16,
+                density_factor=1.0, grad_out=FAKE + (1 << 20), fwd_out=FAKE + (1 << 21),
+                grad_vol=FAKE + (1 << 24), workspace=WS, workspace_bytes=WS_BYTES, stream=0)
+    args.update(kw)
+    return drr.drr_render_alpha_adjoint_ws(**args)
+
+
+ALPHA_WS_BAD = [
+    (dict(workspace=0), drr.DRR_ERR_INVALID_ARG, "workspace"),
+    (dict(workspace=WS + 16), drr.DRR_ERR_INVALID_ARG, "aligned"),
+    (dict(workspace_bytes=100), drr.DRR_ERR_INVALID_ARG, "needed"),
+    (dict(workspace=FAKE), drr.DRR_ERR_INVALID_ARG, "overlaps"),             # on the volume
+    (dict(workspace=FAKE + (1 << 21)), drr.DRR_ERR_INVALID_ARG, "overlaps"),  # on fwd_out
+    (dict(layout=drr.DRR_LAYOUT_PADDED), drr.DRR_ERR_UNSUPPORTED, "LINEAR"),
+    (dict(fwd_out=0), drr.DRR_ERR_INVALID_ARG, "alpha image"),
+]
+
+
+@pytest.mark.parametrize("kw,status,word", ALPHA_WS_BAD)
+def test_alpha_adjoint_ws_rejects_bad_arguments(kw, status, word):
+    with pytest.raises(drr.DrrError) as e:
+        _alpha_adjoint_ws(**kw)
+    assert e.value.status == status
+    assert word in drr.drr_get_last_error()
+
+
+def test_alpha_adjoint_ws_empty_batch_is_a_no_op():
+    _alpha_adjoint_ws(B=0, vol=None, workspace=None, grad_out=None, fwd_out=None, grad_vol=None,
+                      Rt=None)
+    assert drr.drr_get_last_error() == ""
+
+
 NOISE_BAD = [
     (dict(i0=0.0), "i0"),
     (dict(i0=float("inf")), "i0"),

@@ -1,7 +1,7 @@
 """GPU parity of front-to-back alpha compositing (DRR_MODE_ALPHA: drr_render
-and drr_render_alpha_adjoint) and of the Gaussian-Poisson surrogate
-(drr_poisson_noise and its backward) against the pinned fp64 oracle
-(tests/test_oracle_alpha_noise_pins.py).
+and drr_render_alpha_adjoint, with or without a workspace) and of the
+Gaussian-Poisson surrogate (drr_poisson_noise and its backward) against the
+pinned fp64 oracle (tests/test_oracle_alpha_noise_pins.py).
 
 Tolerances, read from the arithmetic (no page fixes one): the alpha image
 composites in fp32 -- a transmittance product and a running sum over N
@@ -88,6 +88,38 @@ def test_alpha_adjoint_small_ragged(cuda, seed, layout, dtype):
     _assert_adjoint(got, ref, f"seed {seed} layout {layout} dtype {dtype}")
 
 
+# rays much closer than a voxel (the geometry of the adjoint's record-path
+# tests): with a workspace these views take alpha_records_kernel
+DENSE = dict(dims=(23, 17, 29), H=150, W=170, n_samples=40)
+
+
+@pytest.mark.parametrize("layout,dtype", [(LINEAR, F32), (CORNERS, BF16), (QUADS, F32),
+                                          (QUADS, BF16)])
+def test_alpha_adjoint_dense_views_take_the_record_path(cuda, layout, dtype):
+    w = wl.small_random_case(421, **DENSE)
+    w.density_factor = 25.0
+    go = np.random.default_rng(421).standard_normal((w.B, w.H, w.W)).astype(np.float32)
+    fwd = gpu_forward(w, layout=layout, dtype=dtype, mode=ALPHA)
+    vol = bf16_values(w.vol) if dtype == BF16 else w.vol
+    ref = oracle.adjoint(w.dims, w.spacing, w.origin, w.K, w.Rt, w.H, w.W, w.n_samples,
+                         w.density_factor, ALPHA, go, vol=vol, nthreads=8)
+    for workspace in (False, True):
+        got = gpu_alpha_adjoint(w, go, fwd, layout=layout, dtype=dtype, workspace=workspace)
+        _assert_adjoint(got, ref, f"dense layout {layout} dtype {dtype} workspace {workspace}")
+
+
+def test_alpha_adjoint_workspace_on_sparse_views(cuda):
+    # views the plan leaves sparse still go through the direct kernel
+    w = wl.small_random_case(422)
+    w.density_factor = 25.0
+    go = np.random.default_rng(422).standard_normal((w.B, w.H, w.W)).astype(np.float32)
+    fwd = gpu_forward(w, layout=CORNERS, dtype=F32, mode=ALPHA)
+    ref = oracle.adjoint(w.dims, w.spacing, w.origin, w.K, w.Rt, w.H, w.W, w.n_samples,
+                         w.density_factor, ALPHA, go, vol=w.vol, nthreads=8)
+    got = gpu_alpha_adjoint(w, go, fwd, layout=CORNERS, dtype=F32, workspace=True)
+    _assert_adjoint(got, ref, "sparse views with a workspace")
+
+
 @pytest.mark.slow
 def test_alpha_adjoint_config3_sparse_upstream(cuda):
     w = wl.make_config(3)
@@ -97,10 +129,11 @@ def test_alpha_adjoint_config3_sparse_upstream(cuda):
     ids = rng.choice(w.rays, size=3000, replace=False)
     go.reshape(-1)[ids] = rng.standard_normal(3000).astype(np.float32)
     fwd = gpu_forward(w, layout=CORNERS, dtype=BF16, mode=ALPHA)
-    got = gpu_alpha_adjoint(w, go, fwd, layout=CORNERS, dtype=BF16)
     ref = oracle.adjoint(w.dims, w.spacing, w.origin, w.K, w.Rt, w.H, w.W, w.n_samples,
                          w.density_factor, ALPHA, go, vol=bf16_values(w.vol), nthreads=4)
-    _assert_adjoint(got, ref, "config 3, 3000 rays")
+    for workspace in (False, True):
+        got = gpu_alpha_adjoint(w, go, fwd, layout=CORNERS, dtype=BF16, workspace=workspace)
+        _assert_adjoint(got, ref, f"config 3, 3000 rays, workspace {workspace}")
 
 
 def _noise_inputs(n, seed):
