@@ -512,6 +512,10 @@ alpha_adjoint_kernel(const T* __restrict__ vol, const float* __restrict__ Rt,
 // tile) and two record slots, home to the bundle's rows; every ray carries
 // its own T and C_i front to back, so there are no phases.  2 x 2 rather
 // than 3 x 2: each ray also holds its sampling and compositing state.
+// Measured on the 256^3 bf16 volume seen by 4 views of 1024^2, 512 samples:
+// 12.0 ms against 31.4 for the direct path; 3 x 2 bundles 13.4 ms (spills
+// at 128 registers) or 19.6 ms (148 registers, 1 CTA per SM); packed fp32x2
+// weights 12.1 ms.
 constexpr int kAlphaBundle = 2;                          // rays per bundle, across and down
 constexpr int kAlphaTile = 16 * kAlphaBundle;            // 32 x 32 pixels per CTA
 
