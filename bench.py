@@ -65,6 +65,10 @@ def parse_args():
     p.add_argument("--siddon", action="store_true",
                    help="also time the cell-constant (Siddon) projector and backprojection on "
                         "the same workload (fp32 linear volume)")
+    p.add_argument("--batched", action="store_true",
+                   help="also time the batched forward and adjoint: the workload's views split "
+                        "one per volume over as many volumes (drr_render_batched, "
+                        "drr_render_adjoint_batched_ws)")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     return p.parse_args()
@@ -494,6 +498,61 @@ def alpha_timing(torch, w, vol32, prep, dtype, layout, Rt, grad_out, elem, l2_pe
     return res
 
 
+def batched_timing(torch, w, vol32, dtype, layout, Rt, grad_out, elem, l2_peak, hbm_peak,
+                   vol_fits_l2):
+    """Batches on the same workload: its B views split one per volume over B
+    volumes (the phantom scaled by 1 + v/10 for volume v), one channel, in
+    the bench's layout and dtype; the batched forward (Beer-Lambert) and the
+    batched adjoint with a workspace (records per volume): median of 10, L2
+    flushed before each.  Same ray-samples as the step; B volumes to read and
+    B gradient volumes to scatter into instead of one."""
+    from cone_beam_ct_b200 import drr
+    from cone_beam_ct_b200 import workloads as wl
+    dev = vol32.device
+    n_vols = w.B
+    nx, ny, nz = w.dims
+    per = drr.drr_prepared_bytes(w.dims, dtype, layout)
+    vols = torch.empty(n_vols * per, dtype=torch.uint8, device=dev)
+    for v in range(n_vols):
+        drr.drr_prepare_volume((vol32 * (1.0 + 0.1 * v)).contiguous(), w.dims, dtype, layout,
+                               vols[v * per:(v + 1) * per], per)
+    out = torch.empty((w.B, 1, w.H, w.W), dtype=torch.float32, device=dev)
+    grads = torch.zeros((n_vols, 1, nz, ny, nx), dtype=torch.float32, device=dev)
+    ws = torch.empty(drr.drr_adjoint_batched_workspace_bytes(w.dims, n_vols, 1, w.B),
+                     dtype=torch.uint8, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    mode = w.mode
+
+    def fwd():
+        drr.drr_render_batched(vols, dtype, layout, w.dims, w.spacing, w.origin, w.K, Rt, n_vols,
+                               1, w.B, w.H, w.W, w.n_samples, w.density_factor, mode, out,
+                               stream=stream)
+
+    def adj():
+        drr.drr_render_adjoint_batched_ws(w.dims, w.spacing, w.origin, w.K, Rt, n_vols, 1, w.B,
+                                          w.H, w.W, w.n_samples, w.density_factor, mode,
+                                          grad_out, out if mode == wl.MODE_BEER_LAMBERT else None,
+                                          grads, ws, stream=stream)
+
+    fwd_ms = _median_ms(torch, fwd, flush=flush)
+    adj_ms = _median_ms(torch, adj, flush=flush)
+    bound, peak = ("l2", l2_peak) if vol_fits_l2 and l2_peak else ("hbm", hbm_peak)
+
+    def roof(kernel, ms, nbytes):
+        a = nbytes / (ms * 1e-3) / 1e9
+        return {"kernel": kernel, "bound": bound, "achieved": a, "peak": peak, "unit": "GB/s",
+                "frac": a / peak, "algorithmic_bytes_per_launch": int(nbytes)}
+
+    return {"n_vols": n_vols, "channels": 1, "n_views": w.B,
+            "forward": {"ms": fwd_ms, "gsamples_s": w.samples / (fwd_ms * 1e-3) / 1e9,
+                        "roofline": roof("forward_kernel (batched)", fwd_ms,
+                                         8 * elem * w.samples)},
+            "adjoint": {"ms": adj_ms, "gsamples_s": w.samples / (adj_ms * 1e-3) / 1e9,
+                        "roofline": roof("adjoint (batched, with a workspace)", adj_ms,
+                                         32 * w.samples)}}
+
+
 def siddon_pieces(w):
     """Cells crossed per ray, summed over the workload (the Siddon walk's unit
     of work): |entry cell - exit cell| summed over the axes, plus one, for every
@@ -726,6 +785,11 @@ def run_ours(args):
         alpha = alpha_timing(torch, w, vol32, prep, dtype, layout, Rt, grad_out, elem, l2_peak,
                              hbm_peak, vol_fits_l2)
 
+    batched = None
+    if args.batched:
+        batched = batched_timing(torch, w, vol32, dtype, layout, Rt, grad_out, elem, l2_peak,
+                                 hbm_peak, vol_fits_l2)
+
     tex = None
     if args.texture:
         tex = texture_comparison(torch, w, vol32, Rt, out)
@@ -755,6 +819,7 @@ def run_ours(args):
         "pose_gradient": pose,
         "alpha_compositing": alpha,
         "siddon": siddon,
+        "batched": batched,
         "gpu_launches": 7 * args.steps,   # prepare, forward, plan, zero, 2 adjoint paths, gather
         "clocks": clocks,
         "bracket_ms": bracket[0].elapsed_time(bracket[1]),

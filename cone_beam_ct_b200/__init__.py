@@ -17,6 +17,7 @@ from .drr import (  # noqa: F401
     DRR_MODE_RAW,
     DrrError,
     drr_abi_version,
+    drr_adjoint_batched_workspace_bytes,
     drr_adjoint_workspace_bytes,
     drr_get_last_error,
     drr_poisson_noise,
@@ -26,6 +27,7 @@ from .drr import (  # noqa: F401
     drr_render,
     drr_render_adjoint,
     drr_render_adjoint_batched,
+    drr_render_adjoint_batched_ws,
     drr_render_alpha_adjoint,
     drr_render_alpha_adjoint_ws,
     drr_render_batched,

@@ -137,11 +137,13 @@ __device__ __forceinline__ void flush_record(float* __restrict__ rec, int cell, 
 }
 
 // Workspace layout (drr_render_adjoint_ws): a 256-byte aligned header of
-// ints -- [0] "some view is dense", [1 + b] "view b is dense" -- then the
-// corner records, 8 floats per cell, cell = (k * (ny-1) + j) * (nx-1) + i.
+// ints -- [0] "some view is dense", [1 + b] "view b is dense" (b: output
+// image) -- then the corner records of each volume-channel slot, 8 floats per
+// cell, cell = (k * (ny-1) + j) * (nx-1) + i.
 struct Workspace {
     int* flags;        // NULL: no workspace, every view takes the direct path
-    float* rec;
+    float* rec;        // records of volume-channel slot 0; slot s at rec + s * rec_stride
+    long long rec_stride;
 };
 
 // Which views accumulate into records: one CTA loops over the views, so
@@ -154,7 +156,7 @@ __global__ void __launch_bounds__(256) plan_views(const float* __restrict__ Rt, 
     int mine = 0;
     for (int b = threadIdx.x; b < g.B; b += blockDim.x) {
         View v;
-        view_setup(Rt + 12 * (size_t)b, g, v);
+        view_setup(Rt + 12 * (size_t)batch_item(g, b).pose, g, v);
         // a view is judged by its first tile: every tile subtends nearly the
         // same angle (the pixel pitch is constant across the detector)
         const int dense = dense_tile(v, g, 0.0, 0.0) ? 1 : 0;
@@ -176,23 +178,29 @@ __global__ void zero_records(const int* __restrict__ flags, float4* __restrict__
 }
 
 // grad[k][j][i] += the 8 record entries of voxel (i, j, k): entry a + 2b + 4c of
-// cell (i - a, j - b, k - c), for the cells that exist.
+// cell (i - a, j - b, k - c), for the cells that exist; for every
+// volume-channel slot (slot s: gradient s * nx*ny*nz elements on, records
+// s * rec_stride floats on).
 __global__ void gather_records(const int* __restrict__ flags, const float* __restrict__ rec,
-                               float* __restrict__ grad, int nx, int ny, int nz) {
+                               long long rec_stride, float* __restrict__ grad, int nx, int ny,
+                               int nz, int slots) {
     if (flags[0] == 0) return;
-    const int64_t n = (int64_t)nx * ny * nz;
+    const int64_t nvox = (int64_t)nx * ny * nz;
+    const int64_t n = nvox * slots;
     const int64_t cr = nx - 1, cs = (int64_t)(nx - 1) * (ny - 1);
     for (int64_t m = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; m < n;
          m += (int64_t)gridDim.x * blockDim.x) {
-        const int i = (int)(m % nx);
-        const int j = (int)((m / nx) % ny);
-        const int k = (int)(m / ((int64_t)nx * ny));
+        const int64_t slot = m / nvox, v = m - slot * nvox;
+        const float* r = rec + slot * rec_stride;
+        const int i = (int)(v % nx);
+        const int j = (int)((v / nx) % ny);
+        const int k = (int)(v / ((int64_t)nx * ny));
         float s = 0.0f;
 #pragma unroll
         for (int corner = 0; corner < 8; ++corner) {
             const int ci = i - (corner & 1), cj = j - ((corner >> 1) & 1), ck = k - (corner >> 2);
             if (ci >= 0 && cj >= 0 && ck >= 0 && ci < nx - 1 && cj < ny - 1 && ck < nz - 1)
-                s += __ldg(rec + (ck * cs + cj * cr + ci) * 8 + corner);
+                s += __ldg(r + (ck * cs + cj * cr + ci) * 8 + corner);
         }
         grad[m] += s;
     }
@@ -298,7 +306,7 @@ adjoint_kernel(const float* __restrict__ Rt, const float* __restrict__ grad_out,
 // the bundle's upper and lower row.  A ray adds its sample to any slot
 // already holding its cell, else flushes its home slot and takes it over, so
 // a bundle that moves together flushes once per cell instead of once per
-// ray.  A warp's bundles are neighbours (an 8 x 4 block of them) and warps
+// ray.  A warp's bundles are neighbours (a 4 x 8 block of them) and warps
 // start at one of 16 phases of the ray.  Measured on the 1024^2 x 512 and
 // 2048^2 x 256 C-arm workloads (B200): neighbouring bundles beat bundles
 // spread over the tile (7.1 vs 7.8 ms); 3 x 2 bundles flush 11 % less than
@@ -322,11 +330,14 @@ records_kernel(const float* __restrict__ Rt, const float* __restrict__ grad_out,
     __shared__ View sv;
     const int b = blockIdx.z;
     if (ws.flags[1 + b] == 0) return;            // sparse view: adjoint_kernel's
-    if (threadIdx.x == 0) view_setup(Rt + 12 * (size_t)b, g, sv);
+    const BatchItem it = batch_item(g, b);
+    float* const rec = ws.rec + it.slot * ws.rec_stride;   // this volume-channel's records
+    if (threadIdx.x == 0) view_setup(Rt + 12 * (size_t)it.pose, g, sv);
     __syncthreads();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    // a warp's 32 bundles form an 8 x 4 block of the 16 x 16 bundle grid
-    const int px = (warp & 1) * 8 + (lane & 7), py = (warp >> 1) * 4 + (lane >> 3);
+    // a warp's 32 bundles form a 4 x 8 block of the 16 x 16 bundle grid (12 x
+    // 16 rays; 8 x 4 bundles, 24 x 8 rays, measured 1 % slower)
+    const int px = (warp & 3) * 4 + (lane & 3), py = (warp >> 2) * 8 + (lane >> 2);
     const int c0 = blockIdx.x * kRecTileW + px * kBundleX, r0 = blockIdx.y * kRecTileH + py * kBundleY;
     const int ph = (warp + blockIdx.x * 3 + blockIdx.y * 5 + blockIdx.z) & 15;   // 16 phases
     const int start = (int)(((long long)g.N * ph) >> 4);
@@ -405,7 +416,7 @@ records_kernel(const float* __restrict__ Rt, const float* __restrict__ grad_out,
                     for (int h = 0; h < kSlots; ++h) {
                         if (h != home) continue;
                         if (pc[h] != cell) {
-                            if (pc[h] >= 0) flush_record(ws.rec, pc[h], p[h]);
+                            if (pc[h] >= 0) flush_record(rec, pc[h], p[h]);
                             pc[h] = cell;
 #pragma unroll
                             for (int e = 0; e < 4; ++e) p[h][e] = make_float2(0.0f, 0.0f);
@@ -418,7 +429,7 @@ records_kernel(const float* __restrict__ Rt, const float* __restrict__ grad_out,
         }
 #pragma unroll
         for (int h = 0; h < kSlots; ++h)
-            if (pc[h] >= 0) flush_record(ws.rec, pc[h], p[h]);
+            if (pc[h] >= 0) flush_record(rec, pc[h], p[h]);
     }
 }
 
@@ -648,21 +659,25 @@ size_t adjoint_workspace_header(int B) {
     return ((size_t)(1 + B) * sizeof(int) + 255) / 256 * 256;
 }
 
-size_t adjoint_workspace_bytes(int nx, int ny, int nz, int B) {
-    return adjoint_workspace_header(B) + (size_t)(nx - 1) * (ny - 1) * (nz - 1) * 8 * sizeof(float);
+size_t adjoint_workspace_bytes(int nx, int ny, int nz, int B, int slots) {
+    return adjoint_workspace_header(B) +
+           (size_t)(nx - 1) * (ny - 1) * (nz - 1) * 8 * sizeof(float) * (size_t)slots;
 }
 
 cudaError_t launch_adjoint(const Geom& g, const float* Rt, int mode, const float* grad_out,
                            const float* fwd_out, float* grad_vol, void* workspace,
                            cudaStream_t stream) {
     const dim3 grid((g.W + kTileW - 1) / kTileW, (g.H + kTileH - 1) / kTileH, g.B);
-    Workspace ws{nullptr, nullptr};
-    const int64_t n_rec4 = (int64_t)(g.nx - 1) * (g.ny - 1) * (g.nz - 1) * 2;   // float4 per record: 2
+    Workspace ws{nullptr, nullptr, 0};
+    const int slots = batch_slots(g);
+    const long long cells = (long long)(g.nx - 1) * (g.ny - 1) * (g.nz - 1);
+    const int64_t n_rec4 = cells * 2 * slots;    // float4 per record: 2
     const int fill_grid = 148 * 8;
     if (workspace) {
         ws.flags = static_cast<int*>(workspace);
         ws.rec = reinterpret_cast<float*>(static_cast<char*>(workspace) +
                                           adjoint_workspace_header(g.B));
+        ws.rec_stride = cells * 8;
         plan_views<<<1, 256, 0, stream>>>(Rt, g, ws.flags);
         zero_records<<<fill_grid, 256, 0, stream>>>(ws.flags, reinterpret_cast<float4*>(ws.rec),
                                                     n_rec4);
@@ -679,7 +694,8 @@ cudaError_t launch_adjoint(const Geom& g, const float* Rt, int mode, const float
             records_kernel<0><<<rgrid, kThreads, 0, stream>>>(Rt, grad_out, fwd_out, g, ws);
     }
     if (workspace)
-        gather_records<<<fill_grid, 256, 0, stream>>>(ws.flags, ws.rec, grad_vol, g.nx, g.ny, g.nz);
+        gather_records<<<fill_grid, 256, 0, stream>>>(ws.flags, ws.rec, ws.rec_stride, grad_vol,
+                                                      g.nx, g.ny, g.nz, slots);
     return cudaGetLastError();
 }
 
@@ -702,12 +718,13 @@ void alpha_kernels(const void* vol, const Geom& g, const float* Rt, const float*
 cudaError_t launch_alpha_adjoint(const void* vol, int dtype, int layout, const Geom& g,
                                  const float* Rt, const float* grad_out, const float* fwd_out,
                                  float* grad_vol, void* workspace, cudaStream_t stream) {
-    Workspace ws{nullptr, nullptr};
+    Workspace ws{nullptr, nullptr, 0};
     const int fill_grid = 148 * 8;
     if (workspace) {
         ws.flags = static_cast<int*>(workspace);
         ws.rec = reinterpret_cast<float*>(static_cast<char*>(workspace) +
                                           adjoint_workspace_header(g.B));
+        ws.rec_stride = (long long)(g.nx - 1) * (g.ny - 1) * (g.nz - 1) * 8;
         const int64_t n_rec4 = (int64_t)(g.nx - 1) * (g.ny - 1) * (g.nz - 1) * 2;
         plan_views<<<1, 256, 0, stream>>>(Rt, g, ws.flags);
         zero_records<<<fill_grid, 256, 0, stream>>>(ws.flags, reinterpret_cast<float4*>(ws.rec),
@@ -723,7 +740,8 @@ cudaError_t launch_alpha_adjoint(const void* vol, int dtype, int layout, const G
         else alpha_kernels<uint16_t, 0>(vol, g, Rt, grad_out, fwd_out, grad_vol, ws, stream);
     }
     if (workspace)
-        gather_records<<<fill_grid, 256, 0, stream>>>(ws.flags, ws.rec, grad_vol, g.nx, g.ny, g.nz);
+        gather_records<<<fill_grid, 256, 0, stream>>>(ws.flags, ws.rec, ws.rec_stride, grad_vol,
+                                                      g.nx, g.ny, g.nz, 1);
     return cudaGetLastError();
 }
 

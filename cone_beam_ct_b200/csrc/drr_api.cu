@@ -587,13 +587,16 @@ DRR_API drr_status drr_render_batched(const void* vols, drr_dtype dtype, drr_lay
                        "drr_render_batched launch");
 }
 
-DRR_API drr_status drr_render_adjoint_batched(const int dims[3], const float spacing[3],
-                                              const float origin[3], const float K[9],
-                                              const float* Rt, int n_vols, int channels,
-                                              int n_views, int H, int W, int n_samples,
-                                              float density_factor, drr_mode mode,
-                                              const float* grad_out, const float* fwd_out,
-                                              float* grad_vols, void* stream) {
+}  // extern "C"
+
+namespace {
+
+drr_status render_adjoint_batched(const int dims[3], const float spacing[3], const float origin[3],
+                                  const float K[9], const float* Rt, int n_vols, int channels,
+                                  int n_views, int H, int W, int n_samples, float density_factor,
+                                  drr_mode mode, const float* grad_out, const float* fwd_out,
+                                  float* grad_vols, bool with_ws, void* workspace,
+                                  size_t workspace_bytes, void* stream) {
     int n_out = 0, per_vol = 1, bcast = 0;
     drr_status st = batch_shape(n_vols, channels, n_views, &n_out, &per_vol, &bcast);
     if (st != DRR_OK) return st;
@@ -617,6 +620,18 @@ DRR_API drr_status drr_render_adjoint_batched(const int dims[3], const float spa
     if (overlaps(grad_vols, vbytes, grad_out, ibytes) ||
         (mode == DRR_MODE_BEER_LAMBERT && overlaps(grad_vols, vbytes, fwd_out, ibytes)))
         return fail(DRR_ERR_INVALID_ARG, "grad_vols overlaps an image buffer");
+    if (with_ws) {
+        const size_t need =
+            drr::adjoint_workspace_bytes(dims[0], dims[1], dims[2], images, n_vols * channels);
+        if (!workspace || !aligned(workspace, 256))
+            return fail(DRR_ERR_INVALID_ARG, "workspace must be a non-NULL, 256-byte aligned device pointer");
+        if (workspace_bytes < need)
+            return fail(DRR_ERR_INVALID_ARG, "workspace holds %zu bytes, %zu needed", workspace_bytes, need);
+        if (overlaps(workspace, need, grad_vols, vbytes) || overlaps(workspace, need, grad_out, ibytes) ||
+            (mode == DRR_MODE_BEER_LAMBERT && overlaps(workspace, need, fwd_out, ibytes)) ||
+            overlaps(workspace, need, Rt, (size_t)n_views * 12 * sizeof(float)))
+            return fail(DRR_ERR_INVALID_ARG, "workspace overlaps another buffer");
+    }
     drr::Geom g;
     drr::fill_geom(g, dims, spacing, origin, K, images, H, W, n_samples, density_factor,
                    DRR_LAYOUT_LINEAR);
@@ -624,9 +639,53 @@ DRR_API drr_status drr_render_adjoint_batched(const int dims[3], const float spa
     g.views_per_vol = per_vol;
     g.broadcast = bcast;
     g.vstride = nvox;
-    return cuda_status(drr::launch_adjoint(g, Rt, mode, grad_out, fwd_out, grad_vols, nullptr,
+    return cuda_status(drr::launch_adjoint(g, Rt, mode, grad_out, fwd_out, grad_vols,
+                                           with_ws ? workspace : nullptr,
                                            static_cast<cudaStream_t>(stream)),
                        "drr_render_adjoint_batched launch");
+}
+
+}  // namespace
+
+extern "C" {
+
+DRR_API drr_status drr_render_adjoint_batched(const int dims[3], const float spacing[3],
+                                              const float origin[3], const float K[9],
+                                              const float* Rt, int n_vols, int channels,
+                                              int n_views, int H, int W, int n_samples,
+                                              float density_factor, drr_mode mode,
+                                              const float* grad_out, const float* fwd_out,
+                                              float* grad_vols, void* stream) {
+    return render_adjoint_batched(dims, spacing, origin, K, Rt, n_vols, channels, n_views, H, W,
+                                  n_samples, density_factor, mode, grad_out, fwd_out, grad_vols,
+                                  false, nullptr, 0, stream);
+}
+
+DRR_API size_t drr_adjoint_batched_workspace_bytes(const int dims[3], int n_vols, int channels,
+                                                   int n_views) {
+    if (!dims) return 0;
+    for (int a = 0; a < 3; ++a)
+        if (dims[a] < 2 || dims[a] > kMaxDim) return 0;
+    if (stored_elements(dims, DRR_LAYOUT_LINEAR) > kMaxElements) return 0;
+    if (n_vols < 1 || channels < 1 || n_views < 1) return 0;
+    if (!(n_views == 1 || n_views % n_vols == 0)) return 0;
+    const int64_t n_out = n_views == 1 ? n_vols : n_views;
+    if (n_out * channels > kMaxViews) return 0;
+    return drr::adjoint_workspace_bytes(dims[0], dims[1], dims[2], (int)(n_out * channels),
+                                        n_vols * channels);
+}
+
+DRR_API drr_status drr_render_adjoint_batched_ws(const int dims[3], const float spacing[3],
+                                                 const float origin[3], const float K[9],
+                                                 const float* Rt, int n_vols, int channels,
+                                                 int n_views, int H, int W, int n_samples,
+                                                 float density_factor, drr_mode mode,
+                                                 const float* grad_out, const float* fwd_out,
+                                                 float* grad_vols, void* workspace,
+                                                 size_t workspace_bytes, void* stream) {
+    return render_adjoint_batched(dims, spacing, origin, K, Rt, n_vols, channels, n_views, H, W,
+                                  n_samples, density_factor, mode, grad_out, fwd_out, grad_vols,
+                                  true, workspace, workspace_bytes, stream);
 }
 
 }  // extern "C"

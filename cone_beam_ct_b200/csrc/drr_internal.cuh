@@ -52,6 +52,12 @@ struct BatchItem {
     long long slot;   // volume * C + channel
 };
 
+// Number of volume-channel slots a batched call touches.
+__host__ __device__ __forceinline__ int batch_slots(const Geom& g) {
+    const int n_out = g.B / g.C;
+    return (g.broadcast ? n_out : n_out / g.views_per_vol) * g.C;
+}
+
 __device__ __forceinline__ BatchItem batch_item(const Geom& g, int z) {
     const int n = z / g.C, ch = z - n * g.C;
     BatchItem it;
@@ -242,7 +248,7 @@ cudaError_t launch_forward(const void* vol, int dtype, int layout, const Geom& g
 cudaError_t launch_adjoint(const Geom& g, const float* Rt, int mode, const float* grad_out,
                            const float* fwd_out, float* grad_vol, void* workspace,
                            cudaStream_t stream);
-size_t adjoint_workspace_bytes(int nx, int ny, int nz, int B);
+size_t adjoint_workspace_bytes(int nx, int ny, int nz, int B, int slots = 1);
 
 // Size of the built-in scratch of the allocation-free adjoint (32 MiB).
 constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;

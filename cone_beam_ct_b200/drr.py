@@ -24,7 +24,8 @@ EXPORTED = ("drr_render", "drr_render_adjoint", "drr_render_adjoint_ws",
             "drr_adjoint_workspace_bytes", "drr_render_adjoint_noalloc", "drr_render_pose_grad",
             "drr_render_alpha_adjoint", "drr_render_alpha_adjoint_ws", "drr_poisson_noise", "drr_poisson_noise_backward",
             "drr_render_siddon", "drr_render_siddon_adjoint", "drr_render_batched",
-            "drr_render_adjoint_batched",
+            "drr_render_adjoint_batched", "drr_adjoint_batched_workspace_bytes",
+            "drr_render_adjoint_batched_ws",
             "drr_prepared_bytes", "drr_prepare_volume", "drr_get_last_error", "drr_abi_version")
 DRR_NOALLOC_SCRATCH_BYTES = 32 << 20
 
@@ -98,6 +99,11 @@ def lib():
     L.drr_render_adjoint_batched.restype = _c.c_int
     L.drr_adjoint_workspace_bytes.argtypes = [_i3, _c.c_int]
     L.drr_adjoint_workspace_bytes.restype = _c.c_size_t
+    L.drr_adjoint_batched_workspace_bytes.argtypes = [_i3, _c.c_int, _c.c_int, _c.c_int]
+    L.drr_adjoint_batched_workspace_bytes.restype = _c.c_size_t
+    L.drr_render_adjoint_batched_ws.argtypes = (L.drr_render_adjoint_batched.argtypes[:-1] +
+                                                [_vp, _c.c_size_t, _vp])
+    L.drr_render_adjoint_batched_ws.restype = _c.c_int
     L.drr_prepared_bytes.argtypes = [_i3, _c.c_int, _c.c_int]
     L.drr_prepared_bytes.restype = _c.c_size_t
     L.drr_prepare_volume.argtypes = [_vp, _i3, _c.c_int, _c.c_int, _vp, _c.c_size_t, _vp]
@@ -290,6 +296,27 @@ def drr_render_adjoint_batched(dims, spacing, origin, K, Rt, n_vols, channels, n
 
 def drr_adjoint_workspace_bytes(dims, B):
     return int(lib().drr_adjoint_workspace_bytes(_i3v(dims), int(B)))
+
+
+def drr_adjoint_batched_workspace_bytes(dims, n_vols, channels, n_views):
+    return int(lib().drr_adjoint_batched_workspace_bytes(_i3v(dims), int(n_vols), int(channels),
+                                                         int(n_views)))
+
+
+def drr_render_adjoint_batched_ws(dims, spacing, origin, K, Rt, n_vols, channels, n_views, H, W,
+                                  n_samples, density_factor, mode, grad_out, fwd_out, grad_vols,
+                                  workspace, workspace_bytes=None, stream=None):
+    if workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    _check(lib().drr_render_adjoint_batched_ws(_i3v(dims), _f3v(spacing), _f3v(origin), _f9v(K),
+                                               _dev(Rt, "Rt", True), int(n_vols), int(channels),
+                                               int(n_views), int(H), int(W), int(n_samples),
+                                               float(density_factor), int(mode),
+                                               _dev(grad_out, "grad_out", True),
+                                               _dev(fwd_out, "fwd_out", True),
+                                               _dev(grad_vols, "grad_vols", True),
+                                               _dev(workspace, "workspace", True),
+                                               int(workspace_bytes), _stream(stream)))
 
 
 def drr_render_adjoint_ws(dims, spacing, origin, K, Rt, B, H, W, n_samples, density_factor, mode,

@@ -373,8 +373,8 @@ DRR_API drr_status drr_render_batched(const void *vols, drr_dtype dtype, drr_lay
 /* Adjoint of drr_render_batched (RAW or Beer-Lambert): grad_vols, DEVICE
  * float32 [n_vols * channels][nz][ny][nx] (linear), ACCUMULATED into; each
  * image's gradient goes to the volume-channel it was rendered from.  Uses
- * the direct scatter path (no workspace).  Other arguments as
- * drr_render_adjoint and drr_render_batched. */
+ * the direct scatter path (no workspace; see drr_render_adjoint_batched_ws).
+ * Other arguments as drr_render_adjoint and drr_render_batched. */
 DRR_API drr_status drr_render_adjoint_batched(const int dims[3], const float spacing[3],
                                               const float origin[3], const float K[9],
                                               const float *Rt, int n_vols, int channels,
@@ -382,6 +382,36 @@ DRR_API drr_status drr_render_adjoint_batched(const int dims[3], const float spa
                                               float density_factor, drr_mode mode,
                                               const float *grad_out, const float *fwd_out,
                                               float *grad_vols, void *stream);
+
+/* Bytes of the workspace drr_render_adjoint_batched_ws needs (0 if the
+ * arguments are invalid): a 256-byte aligned header of one int per output
+ * image plus one, then the corner records (32 bytes per cell,
+ * (nx-1)(ny-1)(nz-1) cells) of each of the n_vols * channels
+ * volume-channels. */
+DRR_API size_t drr_adjoint_batched_workspace_bytes(const int dims[3], int n_vols, int channels,
+                                                   int n_views);
+
+/* drr_render_adjoint_batched with a caller-provided workspace, for speed:
+ * images whose rays are much closer than a voxel (the test of
+ * drr_render_adjoint_ws) accumulate into the corner records of their
+ * volume-channel, which a final pass adds into grad_vols; other images
+ * scatter directly.  Same result up to fp32 summation order.
+ *   workspace        DEVICE, 256-byte aligned, at least
+ *                    drr_adjoint_batched_workspace_bytes(dims, n_vols,
+ *                    channels, n_views) bytes; content on entry ignored, on
+ *                    return unspecified; must not overlap any other buffer
+ *                    of the call.
+ *   workspace_bytes  bytes available at workspace.
+ * Calls that share one workspace must not overlap on the GPU.  Other
+ * arguments as drr_render_adjoint_batched. */
+DRR_API drr_status drr_render_adjoint_batched_ws(const int dims[3], const float spacing[3],
+                                                 const float origin[3], const float K[9],
+                                                 const float *Rt, int n_vols, int channels,
+                                                 int n_views, int H, int W, int n_samples,
+                                                 float density_factor, drr_mode mode,
+                                                 const float *grad_out, const float *fwd_out,
+                                                 float *grad_vols, void *workspace,
+                                                 size_t workspace_bytes, void *stream);
 
 /* Bytes that drr_prepare_volume writes for this volume, dtype and layout
  * (0 if the arguments are invalid or the volume is too large). */

@@ -384,6 +384,45 @@ def test_batched_rejects_bad_arguments():
             drr.drr_render_adjoint_batched(**dict(adj, **kw))
 
 
+def test_batched_workspace_bytes():
+    # header: one int per output image plus one, rounded to 256 bytes; then 32 bytes per
+    # cell for each of the n_vols * channels volume-channels
+    assert drr.drr_adjoint_batched_workspace_bytes((16, 16, 16), 2, 3, 4) == 256 + 6 * 15 ** 3 * 32
+    assert drr.drr_adjoint_batched_workspace_bytes((16, 16, 16), 2, 3, 1) == 256 + 6 * 15 ** 3 * 32
+    assert drr.drr_adjoint_batched_workspace_bytes((16, 16, 16), 1, 1, 64) == \
+        drr.drr_adjoint_workspace_bytes((16, 16, 16), 64)
+    assert drr.drr_adjoint_batched_workspace_bytes((16, 16, 16), 2, 3, 3) == 0   # 3 % 2 != 0
+    assert drr.drr_adjoint_batched_workspace_bytes((16, 16, 16), 0, 3, 4) == 0
+    assert drr.drr_adjoint_batched_workspace_bytes((1, 16, 16), 2, 3, 4) == 0
+    assert drr.drr_adjoint_batched_workspace_bytes((16, 16, 16), 1, 2, 40000) == 0
+
+
+def _adjoint_batched_ws(**kw):
+    args = dict(dims=DIMS, spacing=SP, origin=ORG, K=K_OK, Rt=FAKE, n_vols=2, channels=1,
+                n_views=2, H=8, W=8, n_samples=16, density_factor=1.0, mode=drr.DRR_MODE_RAW,
+                grad_out=FAKE + (1 << 20), fwd_out=None, grad_vols=FAKE + (1 << 24),
+                workspace=WS, workspace_bytes=WS_BYTES, stream=0)
+    args.update(kw)
+    return drr.drr_render_adjoint_batched_ws(**args)
+
+
+BATCHED_WS_BAD = [
+    (dict(workspace=0), "workspace"),
+    (dict(workspace=WS + 64), "aligned"),
+    (dict(workspace_bytes=1000), "needed"),
+    (dict(workspace=FAKE + (1 << 24)), "overlaps"),          # on grad_vols
+    (dict(n_views=3), "multiple"),
+]
+
+
+@pytest.mark.parametrize("kw,word", BATCHED_WS_BAD)
+def test_batched_workspace_adjoint_rejects_bad_arguments(kw, word):
+    with pytest.raises(drr.DrrError) as e:
+        _adjoint_batched_ws(**kw)
+    assert e.value.status == drr.DRR_ERR_INVALID_ARG
+    assert word in drr.drr_get_last_error()
+
+
 def test_prepared_bytes():
     assert drr.drr_prepared_bytes((256, 256, 256), drr.DRR_F32, drr.DRR_LAYOUT_LINEAR) == 4 * 256 ** 3
     assert drr.drr_prepared_bytes((256, 256, 256), drr.DRR_BF16, drr.DRR_LAYOUT_LINEAR) == 2 * 256 ** 3

@@ -71,6 +71,37 @@ def test_dense_views_take_the_record_path(cuda, seed, mode):
         assert_adjoint_parity(got, ref, what=f"dense seed {seed} workspace {workspace}")
 
 
+def _mixed_case(seed):
+    """DENSE geometry with its last view moved 4x farther: one call whose plan
+    sends two views to the record path and one to the direct path."""
+    w = wl.small_random_case(seed, **DENSE)
+    Rt = w.Rt.copy()
+    Rt[2, :, 3] *= 4.0
+    w.Rt = Rt
+    return w
+
+
+def test_mixed_dense_and_sparse_views_in_one_call(cuda):
+    import torch
+    from cone_beam_ct_b200 import drr
+    w = _mixed_case(214)
+    go = np.random.default_rng(214).standard_normal((w.B, w.H, w.W)).astype(np.float32)
+    ref = _oracle_adjoint(w, go, wl.MODE_RAW)
+    Rt = torch.from_numpy(np.ascontiguousarray(w.Rt.reshape(-1, 12))).cuda()
+    nx, ny, nz = w.dims
+    grad = torch.zeros((nz, ny, nx), dtype=torch.float32, device="cuda")
+    ws = torch.full((drr.drr_adjoint_workspace_bytes(w.dims, w.B),), 0x7F, dtype=torch.uint8,
+                    device="cuda")
+    drr.drr_render_adjoint_ws(w.dims, w.spacing, w.origin, w.K, Rt, w.B, w.H, w.W, w.n_samples,
+                              w.density_factor, wl.MODE_RAW, torch.from_numpy(go).cuda(), None,
+                              grad, ws)
+    torch.cuda.synchronize()
+    # white-box: the plan's view flags at the head of the workspace
+    flags = ws[:4 * (1 + w.B)].cpu().numpy().view(np.int32)
+    assert flags.tolist() == [1, 1, 1, 0]
+    assert_adjoint_parity(grad.cpu().numpy(), ref, what="mixed dense and sparse views")
+
+
 def test_record_path_dot_product_identity(cuda):
     w = wl.small_random_case(213, **DENSE)
     rng = np.random.default_rng(7)

@@ -108,6 +108,22 @@ def test_alpha_adjoint_dense_views_take_the_record_path(cuda, layout, dtype):
         _assert_adjoint(got, ref, f"dense layout {layout} dtype {dtype} workspace {workspace}")
 
 
+def test_alpha_adjoint_mixed_dense_and_sparse_views(cuda):
+    # the dense geometry with its last view moved 4x farther: two views on the
+    # record path, one on the direct path, in one call
+    w = wl.small_random_case(423, **DENSE)
+    Rt = w.Rt.copy()
+    Rt[2, :, 3] *= 4.0
+    w.Rt = Rt
+    w.density_factor = 25.0
+    go = np.random.default_rng(423).standard_normal((w.B, w.H, w.W)).astype(np.float32)
+    fwd = gpu_forward(w, layout=QUADS, dtype=F32, mode=ALPHA)
+    ref = oracle.adjoint(w.dims, w.spacing, w.origin, w.K, w.Rt, w.H, w.W, w.n_samples,
+                         w.density_factor, ALPHA, go, vol=w.vol, nthreads=8)
+    got = gpu_alpha_adjoint(w, go, fwd, layout=QUADS, dtype=F32, workspace=True)
+    _assert_adjoint(got, ref, "mixed dense and sparse views")
+
+
 def test_alpha_adjoint_workspace_on_sparse_views(cuda):
     # views the plan leaves sparse still go through the direct kernel
     w = wl.small_random_case(422)

@@ -1,5 +1,5 @@
 """GPU parity of the batched forward and adjoint (drr_render_batched /
-drr_render_adjoint_batched) against the oracle's batch rule
+drr_render_adjoint_batched, with or without a workspace) against the oracle's batch rule
 (tests/test_oracle_batch_pins.py): volumes x channels x views with the
 views grouped per volume, and one view broadcast to every volume.  Each
 image carries the single-image tolerances (forward 1e-4 normwise and per
@@ -52,16 +52,22 @@ def _gpu_batched(w, vols, n_views, layout, mode):
     return out.cpu().numpy()
 
 
-def _gpu_adjoint_batched(w, n_vols, C, n_views, go, mode, fwd=None):
+def _gpu_adjoint_batched(w, n_vols, C, n_views, go, mode, fwd=None, workspace=False):
     import torch
     nx, ny, nz = w.dims
     Rt = torch.from_numpy(np.ascontiguousarray(w.Rt.reshape(-1, 12))).cuda()
     g = torch.zeros((n_vols, C, nz, ny, nx), device="cuda")
     fo = None if fwd is None else torch.from_numpy(np.ascontiguousarray(fwd, np.float32)).cuda()
-    drr.drr_render_adjoint_batched(w.dims, w.spacing, w.origin, w.K, Rt, n_vols, C, n_views, w.H,
-                                   w.W, w.n_samples, w.density_factor, mode,
-                                   torch.from_numpy(np.ascontiguousarray(go, np.float32)).cuda(),
-                                   fo, g)
+    go_d = torch.from_numpy(np.ascontiguousarray(go, np.float32)).cuda()
+    if workspace:
+        nbytes = drr.drr_adjoint_batched_workspace_bytes(w.dims, n_vols, C, n_views)
+        ws = torch.full((nbytes,), 0x7F, dtype=torch.uint8, device="cuda")   # garbage on entry
+        drr.drr_render_adjoint_batched_ws(w.dims, w.spacing, w.origin, w.K, Rt, n_vols, C, n_views,
+                                          w.H, w.W, w.n_samples, w.density_factor, mode, go_d, fo,
+                                          g, ws)
+    else:
+        drr.drr_render_adjoint_batched(w.dims, w.spacing, w.origin, w.K, Rt, n_vols, C, n_views,
+                                       w.H, w.W, w.n_samples, w.density_factor, mode, go_d, fo, g)
     torch.cuda.synchronize()
     return g.cpu().numpy()
 
@@ -96,6 +102,49 @@ def test_batched_adjoint(cuda, n_vols, C, n_views, mode):
             g = got[v, ch].astype(np.float64)
             assert np.max(np.abs(g - r)) <= 1e-4 * np.max(np.abs(r))
             assert np.linalg.norm(g - r) <= 1e-4 * np.linalg.norm(r)
+
+
+def _assert_batched_adjoint(got, ref, what):
+    for v in range(ref.shape[0]):
+        for ch in range(ref.shape[1]):
+            r = ref[v, ch]
+            g = got[v, ch].astype(np.float64)
+            assert np.max(np.abs(g - r)) <= 1e-4 * np.max(np.abs(r)), f"{what} ({v}, {ch})"
+            assert np.linalg.norm(g - r) <= 1e-4 * np.linalg.norm(r), f"{what} ({v}, {ch})"
+
+
+# rays much closer than a voxel (as in the adjoint's record-path tests): with
+# a workspace every image takes the record path of its volume-channel
+DENSE = dict(dims=(23, 17, 29), H=150, W=170, n_samples=40)
+
+
+@pytest.mark.parametrize("n_vols,C,n_views", [(2, 2, 4), (3, 1, 1)])
+@pytest.mark.parametrize("mode", [wl.MODE_RAW, wl.MODE_BEER_LAMBERT])
+def test_batched_adjoint_with_workspace_dense_views(cuda, n_vols, C, n_views, mode):
+    seed = 631 + n_views
+    w = wl.small_random_case(seed, B=n_views, **DENSE)
+    nx, ny, nz = w.dims
+    vols = np.random.default_rng(seed).uniform(0.0, 0.05, (n_vols, C, nz, ny, nx)).astype(np.float32)
+    n_out = n_vols if (n_views == 1 and n_vols > 1) else n_views
+    go = np.random.default_rng(6).standard_normal((n_out, C, w.H, w.W)).astype(np.float32)
+    fwd = _gpu_batched(w, vols, n_views, PADDED, mode) if mode else None
+    ref = oracle.adjoint_batched(w.dims, w.spacing, w.origin, w.K, w.Rt, n_vols, n_views, w.H,
+                                 w.W, w.n_samples, w.density_factor, mode, go, vols=vols,
+                                 nthreads=8)
+    for workspace in (False, True):
+        got = _gpu_adjoint_batched(w, n_vols, C, n_views, go, mode, fwd, workspace=workspace)
+        _assert_batched_adjoint(got, ref, f"workspace {workspace}")
+
+
+def test_batched_adjoint_with_workspace_sparse_views(cuda):
+    # the plan leaves these images on the direct path
+    w, vols = _batch(2, 3, 4, 641)
+    go = np.random.default_rng(7).standard_normal((4, 3, w.H, w.W)).astype(np.float32)
+    ref = oracle.adjoint_batched(w.dims, w.spacing, w.origin, w.K, w.Rt, 2, 4, w.H, w.W,
+                                 w.n_samples, w.density_factor, wl.MODE_RAW, go, vols=vols,
+                                 nthreads=4)
+    got = _gpu_adjoint_batched(w, 2, 3, 4, go, wl.MODE_RAW, workspace=True)
+    _assert_batched_adjoint(got, ref, "sparse, workspace")
 
 
 def test_batched_dot_product_identity(cuda):
