@@ -46,8 +46,11 @@ def texture_forward(w, texel, Rt=None):
 
 
 def _record(name, texel, norm, rel):
-    os.makedirs("gpurun_out", exist_ok=True)
-    with open(os.path.join("gpurun_out", "texture_errors.jsonl"), "a") as f:
+    """Append the measured errors to the file DRR_TEXTURE_ERRORS names, if set."""
+    path = os.environ.get("DRR_TEXTURE_ERRORS")
+    if not path:
+        return
+    with open(path, "a") as f:
         f.write(json.dumps({"case": name, "texel": texel, "normwise": norm, "per_pixel": rel}) + "\n")
 
 
