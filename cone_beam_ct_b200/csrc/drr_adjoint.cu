@@ -180,29 +180,31 @@ __global__ void zero_records(const int* __restrict__ flags, float4* __restrict__
 // grad[k][j][i] += the 8 record entries of voxel (i, j, k): entry a + 2b + 4c of
 // cell (i - a, j - b, k - c), for the cells that exist; for every
 // volume-channel slot (slot s: gradient s * nx*ny*nz elements on, records
-// s * rec_stride floats on).
+// s * rec_stride floats on).  A CTA takes whole x rows, so the row's (j, k)
+// and slot come from one division per row, not three 64-bit ones per voxel.
 __global__ void gather_records(const int* __restrict__ flags, const float* __restrict__ rec,
                                long long rec_stride, float* __restrict__ grad, int nx, int ny,
                                int nz, int slots) {
     if (flags[0] == 0) return;
-    const int64_t nvox = (int64_t)nx * ny * nz;
-    const int64_t n = nvox * slots;
-    const int64_t cr = nx - 1, cs = (int64_t)(nx - 1) * (ny - 1);
-    for (int64_t m = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; m < n;
-         m += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t slot = m / nvox, v = m - slot * nvox;
-        const float* r = rec + slot * rec_stride;
-        const int i = (int)(v % nx);
-        const int j = (int)((v / nx) % ny);
-        const int k = (int)(v / ((int64_t)nx * ny));
-        float s = 0.0f;
+    const int rows = ny * nz;                    // x rows per slot (nx*ny*nz < 2^31)
+    const long long total = (long long)rows * slots;
+    const int cr = nx - 1, cs = (nx - 1) * (ny - 1);
+    for (long long row = blockIdx.x; row < total; row += gridDim.x) {
+        const int slot = (int)(row / rows);
+        const int rr = (int)(row - (long long)slot * rows);
+        const int k = rr / ny, j = rr - k * ny;
+        const float* __restrict__ r = rec + slot * rec_stride;
+        float* __restrict__ gr = grad + row * nx;
+        for (int i = threadIdx.x; i < nx; i += blockDim.x) {
+            float s = 0.0f;
 #pragma unroll
-        for (int corner = 0; corner < 8; ++corner) {
-            const int ci = i - (corner & 1), cj = j - ((corner >> 1) & 1), ck = k - (corner >> 2);
-            if (ci >= 0 && cj >= 0 && ck >= 0 && ci < nx - 1 && cj < ny - 1 && ck < nz - 1)
-                s += __ldg(r + (ck * cs + cj * cr + ci) * 8 + corner);
+            for (int corner = 0; corner < 8; ++corner) {
+                const int ci = i - (corner & 1), cj = j - ((corner >> 1) & 1), ck = k - (corner >> 2);
+                if (ci >= 0 && cj >= 0 && ck >= 0 && ci < nx - 1 && cj < ny - 1 && ck < nz - 1)
+                    s += __ldg(r + (size_t)(ck * cs + cj * cr + ci) * 8 + corner);
+            }
+            gr[i] += s;
         }
-        grad[m] += s;
     }
 }
 
