@@ -41,7 +41,8 @@
 // as a scalar one, so this carries 4x the payload per operation, and the
 // bundle flushes once where its rays would have flushed up to six times.  A
 // gather pass then adds each voxel's 8 record entries into the gradient
-// volume.  Sparse views gain nothing from records (measured: the records
+// volume.  The alpha gradient and batched calls (records per volume-channel)
+// take the same path.  Sparse views gain nothing from records (measured: the records
 // path ran 12-20 ms against the direct path's 9.3 on the 256^3 / 200^2
 // workload) and keep the direct path above.
 #include <cuda_runtime.h>
@@ -443,10 +444,10 @@ records_kernel(const float* __restrict__ Rt, const float* __restrict__ grad_out,
 //   dC/dmu_i = T_i (s (1 - a_i) mu_i + a_i) - s (C - C_i),
 // C_i = sum_{k <= i} T_k a_k mu_k, C the ray's image value (fwd_out) -- the
 // later samples see sample i's absorption through T.  The kernel reads the
-// volume (linear or corner layout: the forward's own sample values), walks
-// each ray once, front to back (no phases: T is sequential), and scatters
-// grad_out * dC/dmu_i * w_corner through the pending 2 x 2 x 2 block of the
-// direct path into the fp32 linear gradient volume.
+// volume (linear, corner or quad layout: the forward's own sample values),
+// walks each ray once, front to back (no phases: T is sequential), and
+// scatters grad_out * dC/dmu_i * w_corner through the pending 2 x 2 x 2
+// block of the direct path into the fp32 linear gradient volume.
 template <typename T, int LAYOUT>
 __global__ void __launch_bounds__(kThreads)
 alpha_adjoint_kernel(const T* __restrict__ vol, const float* __restrict__ Rt,

@@ -5,7 +5,7 @@
 // Zero-padded trilinear interpolation (the grid_sample path of flashdrr's
 // VolumeRaycaster): 8 corner voxels, 7 lerps a + f (b - a), x first, then y,
 // then z.  Every layout evaluates the same lerps in the same order, so the
-// three layouts give the same bits.
+// layouts give the same bits.
 #pragma once
 
 #include <cuda_runtime.h>
