@@ -28,6 +28,7 @@ import argparse
 import hashlib
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -246,10 +247,24 @@ def l2_read_peak_gbs(torch, nbytes):
     return best
 
 
+def code_digest(paths):
+    """First 16 hex digits of the SHA-256 of the sources' code: comments
+    removed and whitespace collapsed, so that a comment edit does not count as
+    a change of the kernel."""
+    digest = hashlib.sha256()
+    for src in paths:
+        with open(os.path.join(ROOT, src)) as f:
+            text = f.read()
+        text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", " ", text)
+        digest.update(" ".join(text.split()).encode())
+    return digest.hexdigest()[:16]
+
+
 def traffic_for(kernel, workload_name, layout_name):
     """DRAM bytes per launch from a committed ncu summary, if it was taken on
-    the current source of the kernel and, for a kernel that reads the
-    volume, in the same layout (else None)."""
+    the current code of the kernel and, for a kernel that reads the volume,
+    in the same layout (else None)."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
@@ -258,13 +273,9 @@ def traffic_for(kernel, workload_name, layout_name):
     entry = table.get(kernel, {}).get(workload_name)
     if not entry or entry.get("layout", layout_name) != layout_name:
         return None
-    digest = hashlib.sha256()
-    for src in entry["sources"]:
-        full = os.path.join(ROOT, src)
-        if not os.path.exists(full):
-            return None
-        digest.update(open(full, "rb").read())
-    if digest.hexdigest()[:16] != entry["sources_sha256_16"]:
+    if not all(os.path.exists(os.path.join(ROOT, src)) for src in entry["sources"]):
+        return None
+    if code_digest(entry["sources"]) != entry["code_sha256_16"]:
         return None
     return entry["dram_bytes_per_launch"]
 

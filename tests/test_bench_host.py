@@ -1,7 +1,7 @@
 """Host logic of bench.py that needs no GPU: the per-workload layout choice
 and the lookup of committed DRAM-traffic figures (taken only when the kernel
-sources and, for the forward, the layout are those the figure was measured
-on)."""
+code -- comments aside -- and, for the forward, the layout are those the
+figure was measured on)."""
 import json
 
 import bench
@@ -13,15 +13,13 @@ def test_auto_layout_covers_every_bench_workload():
 
 
 def _entry(tmp_path, monkeypatch, layout="corners", digest=None):
-    src = tmp_path / "k.cu"
-    src.write_text("kernel source")
-    import hashlib
-    d = hashlib.sha256(b"kernel source").hexdigest()[:16] if digest is None else digest
-    table = {"forward_kernel": {"w": {"sources": ["k.cu"], "sources_sha256_16": d,
+    (tmp_path / "k.cu").write_text("int f(int x) { return x + 1; }  // add one\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    d = bench.code_digest(["k.cu"]) if digest is None else digest
+    table = {"forward_kernel": {"w": {"sources": ["k.cu"], "code_sha256_16": d,
                                       "dram_bytes_per_launch": 123, "layout": layout}}}
     (tmp_path / "profiles").mkdir()
     (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(table))
-    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
 
 
 def test_traffic_is_taken_for_the_same_source_and_layout(tmp_path, monkeypatch):
@@ -36,9 +34,20 @@ def test_traffic_is_null_for_another_layout_or_workload(tmp_path, monkeypatch):
     assert bench.traffic_for("adjoint_kernel", "w", "corners") is None
 
 
-def test_traffic_is_null_once_the_source_changed(tmp_path, monkeypatch):
+def test_traffic_is_null_once_the_code_changed(tmp_path, monkeypatch):
     _entry(tmp_path, monkeypatch, digest="0" * 16)
     assert bench.traffic_for("forward_kernel", "w", "corners") is None
+    _entry_dir = tmp_path / "second"
+    _entry_dir.mkdir()
+    _entry(_entry_dir, monkeypatch)
+    (_entry_dir / "k.cu").write_text("int f(int x) { return x + 2; }\n")
+    assert bench.traffic_for("forward_kernel", "w", "corners") is None
+
+
+def test_a_comment_edit_keeps_the_traffic(tmp_path, monkeypatch):
+    _entry(tmp_path, monkeypatch)
+    (tmp_path / "k.cu").write_text("// adds one\nint f(int x)\n{\n    return x + 1;  /* one */\n}\n")
+    assert bench.traffic_for("forward_kernel", "w", "corners") == 123
 
 
 def test_committed_traffic_names_the_bench_workloads():
