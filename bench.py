@@ -69,9 +69,10 @@ def parse_args():
                    help="also time the cell-constant (Siddon) projector and backprojection on "
                         "the same workload (fp32 linear volume)")
     p.add_argument("--batched", action="store_true",
-                   help="also time the batched forward and adjoint: the workload's views split "
-                        "one per volume over as many volumes (drr_render_batched, "
-                        "drr_render_adjoint_batched_ws)")
+                   help="also time the batched forward, adjoint and pose gradient: the "
+                        "workload's views split one per volume over as many volumes "
+                        "(drr_render_batched, drr_render_adjoint_batched_ws, "
+                        "drr_render_pose_grad_batched)")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     return p.parse_args()
@@ -515,9 +516,9 @@ def batched_timing(torch, w, vol32, dtype, layout, Rt, grad_out, elem, l2_peak, 
                    vol_fits_l2):
     """Batches on the same workload: its B views split one per volume over B
     volumes (the phantom scaled by 1 + v/10 for volume v), one channel, in
-    the bench's layout and dtype; the batched forward (Beer-Lambert) and the
-    batched adjoint with a workspace (records per volume): median of 10, L2
-    flushed before each.  Same ray-samples as the step; B volumes to read and
+    the bench's layout and dtype; the batched forward (Beer-Lambert), the
+    batched adjoint with a workspace (records per volume) and the batched
+    pose gradient: median of 10, L2 flushed before each.  Same ray-samples as the step; B volumes to read and
     B gradient volumes to scatter into instead of one."""
     from cone_beam_ct_b200 import drr
     from cone_beam_ct_b200 import workloads as wl
@@ -548,8 +549,18 @@ def batched_timing(torch, w, vol32, dtype, layout, Rt, grad_out, elem, l2_peak, 
                                           grad_out, out if mode == wl.MODE_BEER_LAMBERT else None,
                                           grads, ws, stream=stream)
 
+    grad_Rt = torch.zeros((w.B, 12), dtype=torch.float32, device=dev)
+
+    def pose():
+        drr.drr_render_pose_grad_batched(vols, dtype, layout, w.dims, w.spacing, w.origin, w.K,
+                                         Rt, n_vols, 1, w.B, w.H, w.W, w.n_samples,
+                                         w.density_factor, mode, grad_out,
+                                         out if mode == wl.MODE_BEER_LAMBERT else None, grad_Rt,
+                                         stream=stream)
+
     fwd_ms = _median_ms(torch, fwd, flush=flush)
     adj_ms = _median_ms(torch, adj, flush=flush)
+    pose_ms = _median_ms(torch, pose, flush=flush)
     bound, peak = ("l2", l2_peak) if vol_fits_l2 and l2_peak else ("hbm", hbm_peak)
 
     def roof(kernel, ms, nbytes):
@@ -558,6 +569,9 @@ def batched_timing(torch, w, vol32, dtype, layout, Rt, grad_out, elem, l2_peak, 
                 "frac": a / peak, "algorithmic_bytes_per_launch": int(nbytes)}
 
     return {"n_vols": n_vols, "channels": 1, "n_views": w.B,
+            "pose_gradient": {"ms": pose_ms, "gsamples_s": w.samples / (pose_ms * 1e-3) / 1e9,
+                              "roofline": roof("pose_kernel (batched)", pose_ms,
+                                               8 * elem * w.samples)},
             "forward": {"ms": fwd_ms, "gsamples_s": w.samples / (fwd_ms * 1e-3) / 1e9,
                         "roofline": roof("forward_kernel (batched)", fwd_ms,
                                          8 * elem * w.samples)},

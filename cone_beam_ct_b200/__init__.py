@@ -34,6 +34,7 @@ from .drr import (  # noqa: F401
     drr_render_adjoint_noalloc,
     drr_render_adjoint_ws,
     drr_render_pose_grad,
+    drr_render_pose_grad_batched,
     drr_render_siddon,
     drr_render_siddon_adjoint,
 )

@@ -587,6 +587,53 @@ DRR_API drr_status drr_render_batched(const void* vols, drr_dtype dtype, drr_lay
                        "drr_render_batched launch");
 }
 
+DRR_API drr_status drr_render_pose_grad_batched(const void* vols, drr_dtype dtype,
+                                                drr_layout layout, const int dims[3],
+                                                const float spacing[3], const float origin[3],
+                                                const float K[9], const float* Rt, int n_vols,
+                                                int channels, int n_views, int H, int W,
+                                                int n_samples, float density_factor,
+                                                drr_mode mode, const float* grad_out,
+                                                const float* fwd_out, float* grad_Rt,
+                                                void* stream) {
+    int n_out = 0, per_vol = 1, bcast = 0;
+    drr_status st = batch_shape(n_vols, channels, n_views, &n_out, &per_vol, &bcast);
+    if (st != DRR_OK) return st;
+    st = check_volume(dims, spacing, origin);
+    if (st != DRR_OK) return st;
+    const int images = n_out * channels;
+    st = check_rays(K, Rt, images, H, W, n_samples, density_factor, mode);
+    if (st != DRR_OK) return st;
+    if (dtype != DRR_F32 && dtype != DRR_BF16) return fail(DRR_ERR_INVALID_ARG, "unknown dtype %d", dtype);
+    if (!known_layout(layout)) return fail(DRR_ERR_INVALID_ARG, "unknown layout %d", layout);
+    if (stored_elements(dims, layout) > kMaxElements)
+        return fail(DRR_ERR_UNSUPPORTED, "volume too large (max 2^31 - 1 stored elements)");
+    const int64_t npix = (int64_t)images * H * W;
+    if (npix == 0) return ok();
+    if (!vols || !aligned(vols, layout_alignment(layout, dtype)))
+        return fail(DRR_ERR_INVALID_ARG, "vols must be a non-NULL device pointer aligned to %zu bytes",
+                    layout_alignment(layout, dtype));
+    if (!grad_out || !aligned(grad_out, 4))
+        return fail(DRR_ERR_INVALID_ARG, "grad_out must be a non-NULL, 4-byte aligned device pointer");
+    if (mode == DRR_MODE_BEER_LAMBERT && (!fwd_out || !aligned(fwd_out, 4)))
+        return fail(DRR_ERR_INVALID_ARG, "fwd_out is required in Beer-Lambert mode");
+    if (!grad_Rt || !aligned(grad_Rt, 4))
+        return fail(DRR_ERR_INVALID_ARG, "grad_Rt must be a non-NULL, 4-byte aligned device pointer");
+    const size_t gbytes = (size_t)n_views * 12 * sizeof(float), ibytes = (size_t)npix * 4;
+    if (overlaps(grad_Rt, gbytes, grad_out, ibytes) || overlaps(grad_Rt, gbytes, Rt, gbytes) ||
+        (mode == DRR_MODE_BEER_LAMBERT && overlaps(grad_Rt, gbytes, fwd_out, ibytes)))
+        return fail(DRR_ERR_INVALID_ARG, "grad_Rt overlaps another buffer");
+    drr::Geom g;
+    drr::fill_geom(g, dims, spacing, origin, K, images, H, W, n_samples, density_factor, layout);
+    g.C = channels;
+    g.views_per_vol = per_vol;
+    g.broadcast = bcast;
+    g.vstride = stored_elements(dims, layout);
+    return cuda_status(drr::launch_pose_grad(vols, dtype, layout, g, Rt, mode, grad_out, fwd_out,
+                                             grad_Rt, static_cast<cudaStream_t>(stream)),
+                       "drr_render_pose_grad_batched launch");
+}
+
 }  // extern "C"
 
 namespace {

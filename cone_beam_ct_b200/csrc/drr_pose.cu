@@ -20,7 +20,9 @@
 // add per entry and CTA.  grad mu is the gradient of the trilinear
 // interpolant inside each sample's cell, from the same 8 corners the
 // forward reads, so the loop is the forward's gather with about twice its
-// arithmetic.
+// arithmetic.  Batched calls (volumes x channels x views, the forward's
+// batch rule) map each image to its pose and volume-channel; images that
+// share a pose add into the same 12 entries.
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -196,17 +198,24 @@ __device__ __forceinline__ void pose_terms(const Clip& k, const Geom& g, const f
 // spills a little) instead of 96 and 2 CTAs; measured on B200 at 1024^2 x
 // 512: 4.78 against 5.80 ms (before the packed bf16 sample and the unroll,
 // which brought it to 4.18 ms).
-template <typename T, int LAYOUT, int MODE>
+// BATCH: images map to poses and volume-channels by the batch rule (a
+// separate instantiation, so that the single-volume kernel carries none of
+// its registers).
+template <typename T, int LAYOUT, int MODE, bool BATCH>
 __global__ void __launch_bounds__(kThreads, 3)
-pose_kernel(const T* __restrict__ vol, const float* __restrict__ Rt,
+pose_kernel(const T* __restrict__ vol_base, const float* __restrict__ Rt,
             const float* __restrict__ grad_out, const float* __restrict__ fwd_out,
             float* __restrict__ grad_Rt, const Geom g) {
     __shared__ View sv;
     __shared__ float sR[12];
     __shared__ double red[kThreads / 32][12];
-    const int b = blockIdx.z;
-    if (threadIdx.x == 0) view_setup(Rt + 12 * (size_t)b, g, sv);
-    if (threadIdx.x < 12) sR[threadIdx.x] = Rt[12 * (size_t)b + threadIdx.x];
+    const int b = blockIdx.z;                    // output image (view x channel)
+    const T* __restrict__ vol = BATCH ? vol_base + batch_item(g, b).slot * g.vstride : vol_base;
+    {
+        const int pose = BATCH ? batch_item(g, b).pose : b;
+        if (threadIdx.x == 0) view_setup(Rt + 12 * (size_t)pose, g, sv);
+        if (threadIdx.x < 12) sR[threadIdx.x] = Rt[12 * (size_t)pose + threadIdx.x];
+    }
     __syncthreads();
     int r, c;
     tile_pixel(r, c);
@@ -278,7 +287,8 @@ pose_kernel(const T* __restrict__ vol, const float* __restrict__ Rt,
         double x = 0.0;
 #pragma unroll
         for (int w = 0; w < kThreads / 32; ++w) x += red[w][threadIdx.x];
-        if (x != 0.0) atomicAdd(grad_Rt + 12 * (size_t)b + threadIdx.x, (float)x);
+        const int pose = BATCH ? batch_item(g, blockIdx.z).pose : (int)blockIdx.z;
+        if (x != 0.0) atomicAdd(grad_Rt + 12 * (size_t)pose + threadIdx.x, (float)x);
     }
 }
 
@@ -288,10 +298,18 @@ cudaError_t launch_typed(const void* vol, const Geom& g, const float* Rt, int mo
                          cudaStream_t stream) {
     const dim3 grid((g.W + kTileW - 1) / kTileW, (g.H + kTileH - 1) / kTileH, g.B);
     const T* v = static_cast<const T*>(vol);
-    if (mode == 1)
-        pose_kernel<T, LAYOUT, 1><<<grid, kThreads, 0, stream>>>(v, Rt, grad_out, fwd_out, grad_Rt, g);
-    else
-        pose_kernel<T, LAYOUT, 0><<<grid, kThreads, 0, stream>>>(v, Rt, grad_out, fwd_out, grad_Rt, g);
+    const bool batch = g.C != 1 || g.broadcast || g.views_per_vol != g.B;
+    if (batch) {
+        if (mode == 1)
+            pose_kernel<T, LAYOUT, 1, true><<<grid, kThreads, 0, stream>>>(v, Rt, grad_out, fwd_out, grad_Rt, g);
+        else
+            pose_kernel<T, LAYOUT, 0, true><<<grid, kThreads, 0, stream>>>(v, Rt, grad_out, fwd_out, grad_Rt, g);
+    } else {
+        if (mode == 1)
+            pose_kernel<T, LAYOUT, 1, false><<<grid, kThreads, 0, stream>>>(v, Rt, grad_out, fwd_out, grad_Rt, g);
+        else
+            pose_kernel<T, LAYOUT, 0, false><<<grid, kThreads, 0, stream>>>(v, Rt, grad_out, fwd_out, grad_Rt, g);
+    }
     return cudaGetLastError();
 }
 

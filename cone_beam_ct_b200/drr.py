@@ -25,6 +25,7 @@ EXPORTED = ("drr_render", "drr_render_adjoint", "drr_render_adjoint_ws",
             "drr_render_alpha_adjoint", "drr_render_alpha_adjoint_ws", "drr_poisson_noise", "drr_poisson_noise_backward",
             "drr_render_siddon", "drr_render_siddon_adjoint", "drr_render_batched",
             "drr_render_adjoint_batched", "drr_adjoint_batched_workspace_bytes",
+            "drr_render_pose_grad_batched",
             "drr_render_adjoint_batched_ws",
             "drr_prepared_bytes", "drr_prepare_volume", "drr_get_last_error", "drr_abi_version")
 DRR_NOALLOC_SCRATCH_BYTES = 32 << 20
@@ -71,6 +72,11 @@ def lib():
                                        _c.c_int, _c.c_int, _c.c_int, _c.c_int, _c.c_float,
                                        _c.c_int, _vp, _vp, _vp, _vp]
     L.drr_render_pose_grad.restype = _c.c_int
+    L.drr_render_pose_grad_batched.argtypes = [_vp, _c.c_int, _c.c_int, _i3, _f3, _f3, _f9, _vp,
+                                               _c.c_int, _c.c_int, _c.c_int, _c.c_int, _c.c_int,
+                                               _c.c_int, _c.c_float, _c.c_int, _vp, _vp, _vp,
+                                               _vp]
+    L.drr_render_pose_grad_batched.restype = _c.c_int
     L.drr_render_alpha_adjoint.argtypes = [_vp, _c.c_int, _c.c_int, _i3, _f3, _f3, _f9, _vp,
                                            _c.c_int, _c.c_int, _c.c_int, _c.c_int, _c.c_float,
                                            _vp, _vp, _vp, _vp]
@@ -212,6 +218,19 @@ def drr_render_pose_grad(vol, dtype, layout, dims, spacing, origin, K, Rt, B, H,
                                       _dev(grad_out, "grad_out", True),
                                       _dev(fwd_out, "fwd_out", True),
                                       _dev(grad_Rt, "grad_Rt", True), _stream(stream)))
+
+
+def drr_render_pose_grad_batched(vols, dtype, layout, dims, spacing, origin, K, Rt, n_vols,
+                                 channels, n_views, H, W, n_samples, density_factor, mode,
+                                 grad_out, fwd_out, grad_Rt, stream=None):
+    _check(lib().drr_render_pose_grad_batched(_dev(vols, "vols", True), int(dtype), int(layout),
+                                              _i3v(dims), _f3v(spacing), _f3v(origin), _f9v(K),
+                                              _dev(Rt, "Rt", True), int(n_vols), int(channels),
+                                              int(n_views), int(H), int(W), int(n_samples),
+                                              float(density_factor), int(mode),
+                                              _dev(grad_out, "grad_out", True),
+                                              _dev(fwd_out, "fwd_out", True),
+                                              _dev(grad_Rt, "grad_Rt", True), _stream(stream)))
 
 
 def drr_render_alpha_adjoint(vol, dtype, layout, dims, spacing, origin, K, Rt, B, H, W,

@@ -254,6 +254,21 @@ DRR_API drr_status drr_render_pose_grad(const void *vol, drr_dtype dtype, drr_la
                                         const float *grad_out, const float *fwd_out,
                                         float *grad_Rt, void *stream);
 
+/* Pose gradient of drr_render_batched (RAW or Beer-Lambert): grad_Rt, DEVICE
+ * float[n_views * 12], ACCUMULATED into; each image adds its terms to the
+ * pose it was rendered from (with n_views == 1, every volume's image adds to
+ * pose 0).  vols, Rt, grad_out and fwd_out as drr_render_batched and
+ * drr_render_adjoint_batched; other arguments as drr_render_pose_grad. */
+DRR_API drr_status drr_render_pose_grad_batched(const void *vols, drr_dtype dtype,
+                                                drr_layout layout, const int dims[3],
+                                                const float spacing[3], const float origin[3],
+                                                const float K[9], const float *Rt, int n_vols,
+                                                int channels, int n_views, int H, int W,
+                                                int n_samples, float density_factor,
+                                                drr_mode mode, const float *grad_out,
+                                                const float *fwd_out, float *grad_Rt,
+                                                void *stream);
+
 /* Volume gradient of a DRR_MODE_ALPHA image: grad_vol += d(sum grad_out *
  * out)/d vol.  With C_i the composite up to and including sample i and C the
  * ray's image value, dC/dmu_i = T_i (s (1 - a_i) mu_i + a_i) - s (C - C_i),

@@ -14,6 +14,7 @@ from .oracle import (  # noqa: F401
     poisson_noise,
     poisson_noise_backward,
     pose_grad,
+    pose_grad_batched,
     ray,
     render,
     render_batched,

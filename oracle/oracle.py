@@ -265,6 +265,24 @@ def adjoint_batched(dims, spacing, origin, K, Rt, n_vols, n_views, H, W, n_sampl
     return grads
 
 
+def pose_grad_batched(vols, dims, spacing, origin, K, Rt, n_views, H, W, n_samples,
+                      density_factor, mode, grad_out, nthreads=1):
+    """grad_Rt[p] (float64, n_views x 3 x 4) = sum over the images rendered
+    with pose p of their pose gradients (pose_grad() of each image alone,
+    with the volume-channel it was rendered from)."""
+    vols = np.asarray(vols)
+    n_vols, C = vols.shape[0], vols.shape[1]
+    go = np.asarray(grad_out, np.float64)
+    Rt = np.asarray(Rt).reshape(-1, 12)
+    out = np.zeros((Rt.shape[0], 3, 4))
+    for n, pose, v in batch_map(n_vols, C, n_views):
+        for ch in range(C):
+            out[pose] += pose_grad(vols[v, ch], dims, spacing, origin, K, Rt[pose:pose + 1], H, W,
+                                   n_samples, density_factor, mode, go[n, ch][None],
+                                   nthreads=nthreads)[0]
+    return out
+
+
 def round_bf16(x):
     """bf16 bit patterns (uint16) of float32 values, round-to-nearest-even."""
     a = np.ascontiguousarray(x, dtype=np.float32)

@@ -423,6 +423,39 @@ def test_batched_workspace_adjoint_rejects_bad_arguments(kw, word):
     assert word in drr.drr_get_last_error()
 
 
+def _pose_batched(**kw):
+    args = dict(vols=FAKE, dtype=drr.DRR_F32, layout=drr.DRR_LAYOUT_LINEAR, dims=DIMS, spacing=SP,
+                origin=ORG, K=K_OK, Rt=FAKE + (1 << 26), n_vols=2, channels=2, n_views=4, H=8,
+                W=8, n_samples=16, density_factor=1.0, mode=drr.DRR_MODE_RAW,
+                grad_out=FAKE + (1 << 20), fwd_out=None, grad_Rt=FAKE + (1 << 27), stream=0)
+    args.update(kw)
+    return drr.drr_render_pose_grad_batched(**args)
+
+
+POSE_BATCHED_BAD = [
+    (dict(n_views=3), drr.DRR_ERR_INVALID_ARG, "multiple"),
+    (dict(mode=drr.DRR_MODE_ALPHA), drr.DRR_ERR_UNSUPPORTED, "pose gradient"),
+    (dict(mode=drr.DRR_MODE_BEER_LAMBERT), drr.DRR_ERR_INVALID_ARG, "fwd_out"),
+    (dict(grad_Rt=0), drr.DRR_ERR_INVALID_ARG, "grad_Rt"),
+    (dict(grad_Rt=FAKE + (1 << 26)), drr.DRR_ERR_INVALID_ARG, "overlaps"),   # on Rt
+    (dict(vols=0), drr.DRR_ERR_INVALID_ARG, "vols"),
+    (dict(layout=drr.DRR_LAYOUT_QUADS, vols=FAKE + 8), drr.DRR_ERR_INVALID_ARG, "16 bytes"),
+]
+
+
+@pytest.mark.parametrize("kw,status,word", POSE_BATCHED_BAD)
+def test_batched_pose_gradient_rejects_bad_arguments(kw, status, word):
+    with pytest.raises(drr.DrrError) as e:
+        _pose_batched(**kw)
+    assert e.value.status == status
+    assert word in drr.drr_get_last_error()
+
+
+def test_batched_pose_gradient_empty_batch_is_a_no_op():
+    _pose_batched(channels=0, vols=None, grad_out=None, grad_Rt=None)
+    assert drr.drr_get_last_error() == ""
+
+
 def test_prepared_bytes():
     assert drr.drr_prepared_bytes((256, 256, 256), drr.DRR_F32, drr.DRR_LAYOUT_LINEAR) == 4 * 256 ** 3
     assert drr.drr_prepared_bytes((256, 256, 256), drr.DRR_BF16, drr.DRR_LAYOUT_LINEAR) == 2 * 256 ** 3

@@ -1,5 +1,6 @@
-"""GPU parity of the batched forward and adjoint (drr_render_batched /
-drr_render_adjoint_batched, with or without a workspace) against the oracle's batch rule
+"""GPU parity of the batched forward, adjoint and pose gradient
+(drr_render_batched / drr_render_adjoint_batched, with or without a
+workspace / drr_render_pose_grad_batched) against the oracle's batch rule
 (tests/test_oracle_batch_pins.py): volumes x channels x views with the
 views grouped per volume, and one view broadcast to every volume.  Each
 image carries the single-image tolerances (forward 1e-4 normwise and per
@@ -12,7 +13,8 @@ import pytest
 import oracle
 from cone_beam_ct_b200 import drr
 from cone_beam_ct_b200 import workloads as wl
-from tests.gpu_helpers import CORNERS, F32, LAYOUTS, LINEAR, PADDED, assert_parity
+from tests.gpu_helpers import (BF16, CORNERS, F32, LAYOUTS, LINEAR, PADDED, QUADS, assert_parity,
+                               assert_pose_parity, bf16_values)
 
 pytestmark = pytest.mark.gpu
 
@@ -155,3 +157,43 @@ def test_batched_dot_product_identity(cuda):
     lhs = float(np.sum(Ax * y.astype(np.float64)))
     rhs = float(np.sum(x.astype(np.float64) * ATy))
     assert abs(lhs - rhs) <= 1e-5 * np.linalg.norm(Ax) * np.linalg.norm(y.astype(np.float64))
+
+
+def _prepared_batch(vols, dims, dtype, layout):
+    import torch
+    n_vols, C = vols.shape[:2]
+    v32 = torch.from_numpy(np.ascontiguousarray(vols)).cuda()
+    per = drr.drr_prepared_bytes(dims, dtype, layout)
+    src = torch.empty(n_vols * C * per, dtype=torch.uint8, device="cuda")
+    for s in range(n_vols * C):
+        drr.drr_prepare_volume(v32.view(n_vols * C, -1)[s], dims, dtype, layout,
+                               src[s * per:(s + 1) * per], per)
+    return src
+
+
+@pytest.mark.parametrize("n_vols,C,n_views,mode", [(2, 2, 4, wl.MODE_RAW),
+                                                   (3, 2, 1, wl.MODE_BEER_LAMBERT)])
+@pytest.mark.parametrize("layout,dtype", [(CORNERS, F32), (QUADS, BF16)])
+def test_batched_pose_gradient(cuda, n_vols, C, n_views, mode, layout, dtype):
+    # (3, 2, 1): one pose broadcast to three volumes, six images add into it
+    import torch
+    w, vols = _batch(n_vols, C, n_views, 651 + n_views)
+    n_out = n_vols if (n_views == 1 and n_vols > 1) else n_views
+    go = np.random.default_rng(8).standard_normal((n_out, C, w.H, w.W)).astype(np.float32)
+    ref_vols = bf16_values(vols) if dtype == BF16 else vols
+    ref = oracle.pose_grad_batched(ref_vols, w.dims, w.spacing, w.origin, w.K, w.Rt, n_views, w.H,
+                                   w.W, w.n_samples, w.density_factor, mode, go, nthreads=8)
+    src = _prepared_batch(vols, w.dims, dtype, layout)
+    Rt = torch.from_numpy(np.ascontiguousarray(w.Rt.reshape(-1, 12))).cuda()
+    fo = None
+    if mode == wl.MODE_BEER_LAMBERT:
+        fo = torch.full((n_out, C, w.H, w.W), float("nan"), device="cuda")
+        drr.drr_render_batched(src, dtype, layout, w.dims, w.spacing, w.origin, w.K, Rt, n_vols, C,
+                               n_views, w.H, w.W, w.n_samples, w.density_factor, mode, fo)
+    g = torch.zeros((n_views, 12), device="cuda")
+    drr.drr_render_pose_grad_batched(src, dtype, layout, w.dims, w.spacing, w.origin, w.K, Rt,
+                                     n_vols, C, n_views, w.H, w.W, w.n_samples, w.density_factor,
+                                     mode, torch.from_numpy(go).cuda(), fo, g)
+    torch.cuda.synchronize()
+    assert_pose_parity(g.cpu().numpy().reshape(-1, 3, 4), ref, 1e-4,
+                       what=f"batched ({n_vols}, {C}, {n_views}) layout {layout} dtype {dtype}")

@@ -68,3 +68,37 @@ def test_batched_adjoint_is_the_transpose_of_the_batched_forward():
                                  w.n_samples, w.density_factor, wl.MODE_RAW, y)
     lhs, rhs = np.sum(Ax * y), np.sum(x.astype(np.float64) * ATy)
     assert abs(lhs - rhs) <= 1e-12 * np.linalg.norm(Ax) * np.linalg.norm(y)
+
+
+@pytest.mark.parametrize("n_vols,C,n_views,mode", [(2, 2, 4, wl.MODE_RAW), (3, 1, 1, wl.MODE_BEER_LAMBERT)])
+def test_batched_pose_gradient_matches_finite_differences_of_the_batched_render(n_vols, C, n_views,
+                                                                                mode):
+    # random volume-channels, so that images of one pose differ; central
+    # differences of sum(go * render_batched) in each pose entry.  With one
+    # pose broadcast to every volume, all images add into pose 0.
+    w, Rt, _, _ = _case(n_vols, C, n_views, 95 + n_views)
+    nx, ny, nz = w.dims
+    rng = np.random.default_rng(11 + n_views)
+    vols = rng.uniform(0.0, 0.05, (n_vols, C, nz, ny, nx)).astype(np.float32)
+    n_out = n_vols if (n_views == 1 and n_vols > 1) else n_views
+    go = rng.standard_normal((n_out, C, w.H, w.W))
+    g = oracle.pose_grad_batched(vols, w.dims, w.spacing, w.origin, w.K, Rt, n_views, w.H, w.W,
+                                 w.n_samples, w.density_factor, mode, go)
+    assert g.shape == (Rt.shape[0], 3, 4)
+
+    def objective(R):
+        return np.sum(go * oracle.render_batched(vols, w.dims, w.spacing, w.origin, w.K, R,
+                                                 n_views, w.H, w.W, w.n_samples,
+                                                 w.density_factor, mode))
+
+    for p in range(Rt.shape[0]):
+        fd = np.zeros((3, 4))
+        for r in range(3):
+            for c in range(4):
+                h = 1e-5 if c == 3 else 1e-7
+                Rp, Rm = Rt.copy(), Rt.copy()
+                Rp[p, r, c] += h
+                Rm[p, r, c] -= h
+                fd[r, c] = (objective(Rp) - objective(Rm)) / (2 * h)
+        assert np.max(np.abs(g[p, :, :3] - fd[:, :3])) <= 1e-6 * np.max(np.abs(fd[:, :3]))
+        assert np.max(np.abs(g[p, :, 3] - fd[:, 3])) <= 1e-5 * np.max(np.abs(fd[:, 3]))
