@@ -543,10 +543,15 @@ static void trilinear_grad(const float *vol, const grid_t *g, const double p[3],
 }
 
 /* dI/d[R|t] of one ray, grad12[4r + c] for R[r][c] (c < 3) and t[r] (c = 3).
- * Returns the integral I (0 and a zero gradient on a miss). */
+ * Returns the integral I (0 and a zero gradient on a miss).  In alpha mode
+ * the derivative is of the composite C = sum_i T_i a_i mu_i instead (the
+ * value returned is then C): each parameter's tangent is carried through the
+ * front-to-back recurrence step by step -- dmu_i from the moved sample, ds =
+ * density_factor * d(dt), da_i = (1 - a_i)(ds mu_i + s dmu_i), dC += dT_i a_i
+ * mu_i + T_i da_i mu_i + T_i a_i dmu_i, dT_{i+1} = dT_i (1 - a_i) - T_i da_i. */
 static double ray_pose_grad(const float *vol, const grid_t *g, const double K[9],
                             const double Rt[12], double u, double v, int n_samples,
-                            double density_factor, double grad12[12]) {
+                            double density_factor, int mode, double grad12[12]) {
     for (int m = 0; m < 12; ++m) grad12[m] = 0.0;
     double Cijk[3], dijk[3], t0, t1;
     if (!ray_in_volume(g, K, Rt, u, v, Cijk, dijk, &t0, &t1)) return 0.0;
@@ -599,6 +604,26 @@ static double ray_pose_grad(const float *vol, const grid_t *g, const double K[9]
         if (!pinned0) dt0 = -(dC[ax0] + t0 * dd[ax0]) / dijk[ax0];
         dt1 = -(dC[ax1] + t1 * dd[ax1]) / dijk[ax1];
         const double ddt = (dt1 - dt0) / (double)n_samples;
+        if (mode == ORACLE_ALPHA) {
+            const double s = density_factor * dt, ds = density_factor * ddt;
+            double T = 1.0, dT = 0.0, dCv = 0.0;
+            for (int i = 0; i < n_samples; ++i) {
+                const double ti = sample_t(t0, dt, i);
+                const double dti = dt0 + ((double)i + 0.5) * ddt;
+                double p[3], gr[3], dmu = 0.0;
+                for (int k = 0; k < 3; ++k) p[k] = Cijk[k] + ti * dijk[k];
+                const double mu = trilinear(vol, g, p);
+                trilinear_grad(vol, g, p, gr);
+                for (int k = 0; k < 3; ++k) dmu += gr[k] * (dC[k] + dti * dijk[k] + ti * dd[k]);
+                const double a = -expm1(-s * mu);
+                const double da = (1.0 - a) * (ds * mu + s * dmu);
+                dCv += dT * a * mu + T * da * mu + T * a * dmu;
+                dT = dT * (1.0 - a) - T * da;
+                T *= 1.0 - a;
+            }
+            grad12[m] = dCv;
+            continue;
+        }
         double sum = 0.0, dsum = 0.0;
         for (int i = 0; i < n_samples; ++i) {
             const double ti = sample_t(t0, dt, i);
@@ -611,6 +636,7 @@ static double ray_pose_grad(const float *vol, const grid_t *g, const double K[9]
         }
         grad12[m] = density_factor * (ddt * sum + dt * dsum);
     }
+    if (mode == ORACLE_ALPHA) return ray_alpha(vol, g, K, Rt, u, v, n_samples, density_factor);
     double dt2;
     return ray_integral(vol, g, K, Rt, u, v, n_samples, density_factor, &dt2);
 }
@@ -635,7 +661,7 @@ static void *pose_worker(void *arg) {
                 if (go == 0.0) continue;
                 double g12[12];
                 double I = ray_pose_grad(j->vol, j->g, j->K, j->Rt + 12 * b, c, r, j->n_samples,
-                                         j->density_factor, g12);
+                                         j->density_factor, j->mode, g12);
                 /* Beer-Lambert: d(1 - exp(-I))/dI = exp(-I) */
                 double w = go * (j->mode == ORACLE_BEER_LAMBERT ? exp(-I) : 1.0);
                 for (int m = 0; m < 12; ++m) acc[m] += w * g12[m];
@@ -646,7 +672,8 @@ static void *pose_worker(void *arg) {
 }
 
 /* Pose gradient: grad_Rt[b][4r + c] += sum over the pixels of view b of
- * grad_out * d image / d Rt[b][r][c].  Views run on up to nthreads threads;
+ * grad_out * d image / d Rt[b][r][c] (RAW, Beer-Lambert or alpha image).
+ * Views run on up to nthreads threads;
  * each view is summed sequentially, so the result does not depend on the
  * thread count. */
 int oracle_pose_grad(const float *vol, const int dims[3], const double spacing[3],
@@ -656,7 +683,7 @@ int oracle_pose_grad(const float *vol, const int dims[3], const double spacing[3
     grid_t g;
     if (make_grid(dims, spacing, origin, &g) || B < 0 || H < 0 || W < 0 || n_samples < 1)
         return -1;
-    if (mode != ORACLE_RAW && mode != ORACLE_BEER_LAMBERT) return -1;
+    if (mode != ORACLE_RAW && mode != ORACLE_BEER_LAMBERT && mode != ORACLE_ALPHA) return -1;
     if (nthreads > B) nthreads = B;
     if (nthreads > 64) nthreads = 64;
     if (nthreads < 1) nthreads = 1;

@@ -155,7 +155,8 @@ def pose_grad(vol, dims, spacing, origin, K, Rt, H, W, n_samples, density_factor
               grad_out, nthreads=1):
     """grad_Rt[b][r][c] (float64, B x 3 x 4) = sum over the pixels of view b of
     grad_out * d image / d Rt[b][r][c] (the 12 matrix entries taken as free
-    variables; times exp(-I) in Beer-Lambert)."""
+    variables; times exp(-I) in Beer-Lambert; of the composite in alpha
+    mode)."""
     dims, spacing, origin, K, Rt = _geom(dims, spacing, origin, K, Rt)
     B = Rt.shape[0]
     go = np.ascontiguousarray(grad_out, dtype=np.float64).reshape(-1)

@@ -51,6 +51,12 @@ MUTANTS = {
         " if (j >= g->n[1]) j = g->n[1] - 1; if (k >= g->n[2]) k = g->n[2] - 1;"),
     "spacing ignored in the direction": ("dijk[a] = d[a] / g->spacing[a];", "dijk[a] = d[a];"),
     "bf16 truncation instead of rounding": ("bits += 0x7fffu + lsb;", "(void)lsb;"),
+    "alpha pose gradient without the transmittance tangent": (
+        "dCv += dT * a * mu + T * da * mu + T * a * dmu;",
+        "dCv += T * da * mu + T * a * dmu;"),
+    "alpha pose gradient without the step-length tangent": (
+        "const double da = (1.0 - a) * (ds * mu + s * dmu);",
+        "const double da = (1.0 - a) * (s * dmu);"),
     "pose gradient without the derivative of dt": (
         "grad12[m] = density_factor * (ddt * sum + dt * dsum);",
         "grad12[m] = density_factor * (dt * dsum);"),

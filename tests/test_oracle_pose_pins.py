@@ -75,6 +75,24 @@ def test_pose_gradient_matches_finite_differences(seed, mode):
         assert np.max(np.abs(g[b, :, 3] - fd[b, :, 3])) <= 1e-5 * np.max(np.abs(fd[b, :, 3]))
 
 
+@pytest.mark.parametrize("seed", [14, 15])
+def test_alpha_pose_gradient_matches_finite_differences(seed):
+    # the composite C = sum T_i a_i mu_i (alpha mode) is smooth in the pose
+    # between sample-crossings of voxel faces, like the line integral; a large
+    # density_factor keeps the opacities far from the linear regime
+    w = _case(seed)
+    w.density_factor = 30.0
+    Rt = w.Rt.astype(np.float64).reshape(-1, 3, 4)
+    go = np.random.default_rng(seed).standard_normal((w.B, w.H, w.W))
+    g = _pose_grad(w, Rt, go, wl.MODE_ALPHA)
+    fd = _fd_pose_grad(w, Rt, go, wl.MODE_ALPHA)
+    for b in range(w.B):
+        assert np.max(np.abs(g[b, :, :3] - fd[b, :, :3])) <= 1e-6 * np.max(np.abs(fd[b, :, :3]))
+        assert np.max(np.abs(g[b, :, 3] - fd[b, :, 3])) <= 1e-5 * np.max(np.abs(fd[b, :, 3]))
+    # and it is not the line integral's gradient
+    assert np.max(np.abs(g - _pose_grad(w, Rt, go, RAW))) > 1e-3 * np.max(np.abs(g))
+
+
 def test_pose_gradient_camera_inside_the_volume():
     # camera at the volume centre: every ray starts at t0 = 0
     w = _case(21, B=1, H=11, W=10)
