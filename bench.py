@@ -452,9 +452,9 @@ def _median_ms(torch, fn, reps=10, flush=None):
 def alpha_timing(torch, w, vol32, prep, dtype, layout, Rt, grad_out, elem, l2_peak, hbm_peak,
                  vol_fits_l2):
     """Alpha compositing on the same workload (forward from the prepared
-    volume; volume gradient from it, with and without a workspace, unless it
-    is zero-bordered), and the surrogate on its image: median of 10, L2
-    flushed before each."""
+    volume; its pose gradient; its volume gradient, with and without a
+    workspace, unless the volume is zero-bordered), and the surrogate on its
+    image: median of 10, L2 flushed before each."""
     from cone_beam_ct_b200 import drr
     dev = vol32.device
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
@@ -478,7 +478,15 @@ def alpha_timing(torch, w, vol32, prep, dtype, layout, Rt, grad_out, elem, l2_pe
                                          Rt, w.B, w.H, w.W, w.n_samples, w.density_factor,
                                          grad_out, out, grad, stream=stream)
 
+    grad_Rt = torch.zeros((w.B, 12), dtype=torch.float32, device=dev)
+
+    def pose():
+        drr.drr_render_pose_grad(prep, dtype, layout, w.dims, w.spacing, w.origin, w.K, Rt, w.B,
+                                 w.H, w.W, w.n_samples, w.density_factor, drr.DRR_MODE_ALPHA,
+                                 grad_out, out, grad_Rt, stream=stream)
+
     fwd_ms = _median_ms(torch, fwd, flush=flush)
+    pose_ms = _median_ms(torch, pose, flush=flush)
     adj_ms = direct_ms = None
     if layout != drr.DRR_LAYOUT_PADDED:
         adj_ms = _median_ms(torch, lambda: adj(True), flush=flush)
@@ -500,6 +508,9 @@ def alpha_timing(torch, w, vol32, prep, dtype, layout, Rt, grad_out, elem, l2_pe
         out, z, 1e4, grad_out, gi, stream=stream))
     res = {"forward": {"ms": fwd_ms, "gsamples_s": w.samples / (fwd_ms * 1e-3) / 1e9,
                        "roofline": roof("forward_kernel<alpha>", fwd_ms, 8 * elem * w.samples)},
+           "pose_gradient": {"ms": pose_ms, "gsamples_s": w.samples / (pose_ms * 1e-3) / 1e9,
+                             "roofline": roof("pose_kernel<alpha>", pose_ms,
+                                              8 * elem * w.samples)},
            "density_factor": w.density_factor,
            "surrogate": {"ms": noise_ms, "backward_ms": noise_bwd_ms,
                          "hbm_gbs": 12 * n / (noise_ms * 1e-3) / 1e9,

@@ -93,7 +93,7 @@ drr_status check_rays(const float K[9], const float* Rt, int B, int H, int W, in
     if (mode == DRR_MODE_ALPHA && !alpha_ok)
         return fail(DRR_ERR_UNSUPPORTED,
                     "DRR_MODE_ALPHA is not linear in the volume: its gradient needs the volume "
-                    "(drr_render_alpha_adjoint); the pose gradient does not support it");
+                    "(drr_render_alpha_adjoint)");
     if (mode != DRR_MODE_RAW && mode != DRR_MODE_BEER_LAMBERT && mode != DRR_MODE_ALPHA)
         return fail(DRR_ERR_INVALID_ARG, "unknown mode %d", mode);
     if ((int64_t)B * H * W > 0 && (!Rt || !aligned(Rt, 4)))
@@ -302,7 +302,7 @@ DRR_API drr_status drr_render_pose_grad(const void* vol, drr_dtype dtype, drr_la
                                         float* grad_Rt, void* stream) {
     drr_status st = check_volume(dims, spacing, origin);
     if (st != DRR_OK) return st;
-    st = check_rays(K, Rt, B, H, W, n_samples, density_factor, mode);
+    st = check_rays(K, Rt, B, H, W, n_samples, density_factor, mode, true);
     if (st != DRR_OK) return st;
     if (dtype != DRR_F32 && dtype != DRR_BF16) return fail(DRR_ERR_INVALID_ARG, "unknown dtype %d", dtype);
     if (!known_layout(layout)) return fail(DRR_ERR_INVALID_ARG, "unknown layout %d", layout);
@@ -315,13 +315,13 @@ DRR_API drr_status drr_render_pose_grad(const void* vol, drr_dtype dtype, drr_la
                     layout_alignment(layout, dtype));
     if (!grad_out || !aligned(grad_out, 4))
         return fail(DRR_ERR_INVALID_ARG, "grad_out must be a non-NULL, 4-byte aligned device pointer");
-    if (mode == DRR_MODE_BEER_LAMBERT && (!fwd_out || !aligned(fwd_out, 4)))
-        return fail(DRR_ERR_INVALID_ARG, "fwd_out is required in Beer-Lambert mode");
+    if (mode != DRR_MODE_RAW && (!fwd_out || !aligned(fwd_out, 4)))
+        return fail(DRR_ERR_INVALID_ARG, "fwd_out is required in Beer-Lambert and alpha mode");
     if (!grad_Rt || !aligned(grad_Rt, 4))
         return fail(DRR_ERR_INVALID_ARG, "grad_Rt must be a non-NULL, 4-byte aligned device pointer");
     const size_t gbytes = (size_t)B * 12 * sizeof(float), ibytes = (size_t)npix * 4;
     if (overlaps(grad_Rt, gbytes, grad_out, ibytes) || overlaps(grad_Rt, gbytes, Rt, gbytes) ||
-        (mode == DRR_MODE_BEER_LAMBERT && overlaps(grad_Rt, gbytes, fwd_out, ibytes)))
+        (mode != DRR_MODE_RAW && overlaps(grad_Rt, gbytes, fwd_out, ibytes)))
         return fail(DRR_ERR_INVALID_ARG, "grad_Rt overlaps another buffer");
     drr::Geom g;
     drr::fill_geom(g, dims, spacing, origin, K, B, H, W, n_samples, density_factor, layout);
@@ -602,7 +602,7 @@ DRR_API drr_status drr_render_pose_grad_batched(const void* vols, drr_dtype dtyp
     st = check_volume(dims, spacing, origin);
     if (st != DRR_OK) return st;
     const int images = n_out * channels;
-    st = check_rays(K, Rt, images, H, W, n_samples, density_factor, mode);
+    st = check_rays(K, Rt, images, H, W, n_samples, density_factor, mode, true);
     if (st != DRR_OK) return st;
     if (dtype != DRR_F32 && dtype != DRR_BF16) return fail(DRR_ERR_INVALID_ARG, "unknown dtype %d", dtype);
     if (!known_layout(layout)) return fail(DRR_ERR_INVALID_ARG, "unknown layout %d", layout);
@@ -615,13 +615,13 @@ DRR_API drr_status drr_render_pose_grad_batched(const void* vols, drr_dtype dtyp
                     layout_alignment(layout, dtype));
     if (!grad_out || !aligned(grad_out, 4))
         return fail(DRR_ERR_INVALID_ARG, "grad_out must be a non-NULL, 4-byte aligned device pointer");
-    if (mode == DRR_MODE_BEER_LAMBERT && (!fwd_out || !aligned(fwd_out, 4)))
-        return fail(DRR_ERR_INVALID_ARG, "fwd_out is required in Beer-Lambert mode");
+    if (mode != DRR_MODE_RAW && (!fwd_out || !aligned(fwd_out, 4)))
+        return fail(DRR_ERR_INVALID_ARG, "fwd_out is required in Beer-Lambert and alpha mode");
     if (!grad_Rt || !aligned(grad_Rt, 4))
         return fail(DRR_ERR_INVALID_ARG, "grad_Rt must be a non-NULL, 4-byte aligned device pointer");
     const size_t gbytes = (size_t)n_views * 12 * sizeof(float), ibytes = (size_t)npix * 4;
     if (overlaps(grad_Rt, gbytes, grad_out, ibytes) || overlaps(grad_Rt, gbytes, Rt, gbytes) ||
-        (mode == DRR_MODE_BEER_LAMBERT && overlaps(grad_Rt, gbytes, fwd_out, ibytes)))
+        (mode != DRR_MODE_RAW && overlaps(grad_Rt, gbytes, fwd_out, ibytes)))
         return fail(DRR_ERR_INVALID_ARG, "grad_Rt overlaps another buffer");
     drr::Geom g;
     drr::fill_geom(g, dims, spacing, origin, K, images, H, W, n_samples, density_factor, layout);

@@ -85,8 +85,9 @@ typedef enum {
        the emission-absorption sum: sample i has opacity
        a_i = 1 - exp(-density_factor * mu_i * dt) and colour mu_i, and
        out = sum_i T_i a_i mu_i with T_0 = 1, T_{i+1} = T_i (1 - a_i), summed
-       from the camera side.  drr_render only; its volume gradient is
-       drr_render_alpha_adjoint (it is not linear in the volume). */
+       from the camera side.  Its volume gradient is drr_render_alpha_adjoint
+       (it is not linear in the volume); drr_render_pose_grad(_batched) take
+       it too. */
     DRR_MODE_ALPHA = 2
 } drr_mode;
 
@@ -235,11 +236,15 @@ DRR_API drr_status drr_render_adjoint_noalloc(const int dims[3], const float spa
  * moves with the box plane it lies on; an entry point at the camera, when
  * the camera is inside the box, does not move), the sample positions, the
  * gradient of the trilinear interpolant inside each sample's cell and dt.
+ * In DRR_MODE_ALPHA each sample's gradient is weighted by dC/dmu_i (see
+ * drr_render_alpha_adjoint) and dt enters through the opacities as well:
+ * dC/ds = sum_i T_i mu_i^2 (1 - a_i) - mu_i (C - C_i), s = density_factor dt.
  *   vol, dtype, layout  the forward's volume (any layout).
  *   grad_out    DEVICE float[B*H*W], upstream gradient dL/d(out).
- *   fwd_out     DEVICE float[B*H*W], the Beer-Lambert image (required in
- *               DRR_MODE_BEER_LAMBERT, where each ray's term is scaled by
- *               exp(-I) = 1 - out; may be NULL in DRR_MODE_RAW).
+ *   fwd_out     DEVICE float[B*H*W], the forward's image: required in
+ *               DRR_MODE_BEER_LAMBERT (each ray's term is scaled by
+ *               exp(-I) = 1 - out) and in DRR_MODE_ALPHA (the composite C
+ *               of each ray); may be NULL in DRR_MODE_RAW.
  *   grad_Rt     DEVICE float[B*12], row-major like Rt, ACCUMULATED into (zero
  *               it first for a plain gradient); must not overlap Rt or the
  *               images.  Per-ray terms are formed in fp64 and summed per CTA
@@ -254,7 +259,7 @@ DRR_API drr_status drr_render_pose_grad(const void *vol, drr_dtype dtype, drr_la
                                         const float *grad_out, const float *fwd_out,
                                         float *grad_Rt, void *stream);
 
-/* Pose gradient of drr_render_batched (RAW or Beer-Lambert): grad_Rt, DEVICE
+/* Pose gradient of drr_render_batched (any mode): grad_Rt, DEVICE
  * float[n_views * 12], ACCUMULATED into; each image adds its terms to the
  * pose it was rendered from (with n_views == 1, every volume's image adds to
  * pose 0).  vols, Rt, grad_out and fwd_out as drr_render_batched and

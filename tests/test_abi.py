@@ -214,7 +214,7 @@ POSE_BAD = [
     (dict(grad_Rt=FAKE + (1 << 26) + 8), drr.DRR_ERR_INVALID_ARG, "overlaps"),   # on Rt
     (dict(grad_Rt=FAKE + (1 << 20) + 4), drr.DRR_ERR_INVALID_ARG, "overlaps"),   # on grad_out
     (dict(n_samples=0), drr.DRR_ERR_INVALID_ARG, "n_samples"),
-    (dict(mode=drr.DRR_MODE_ALPHA), drr.DRR_ERR_UNSUPPORTED, "pose gradient"),
+    (dict(mode=drr.DRR_MODE_ALPHA, fwd_out=0), drr.DRR_ERR_INVALID_ARG, "alpha"),
 ]
 
 
@@ -434,7 +434,7 @@ def _pose_batched(**kw):
 
 POSE_BATCHED_BAD = [
     (dict(n_views=3), drr.DRR_ERR_INVALID_ARG, "multiple"),
-    (dict(mode=drr.DRR_MODE_ALPHA), drr.DRR_ERR_UNSUPPORTED, "pose gradient"),
+    (dict(mode=drr.DRR_MODE_ALPHA), drr.DRR_ERR_INVALID_ARG, "fwd_out"),
     (dict(mode=drr.DRR_MODE_BEER_LAMBERT), drr.DRR_ERR_INVALID_ARG, "fwd_out"),
     (dict(grad_Rt=0), drr.DRR_ERR_INVALID_ARG, "grad_Rt"),
     (dict(grad_Rt=FAKE + (1 << 26)), drr.DRR_ERR_INVALID_ARG, "overlaps"),   # on Rt

@@ -172,7 +172,8 @@ def _prepared_batch(vols, dims, dtype, layout):
 
 
 @pytest.mark.parametrize("n_vols,C,n_views,mode", [(2, 2, 4, wl.MODE_RAW),
-                                                   (3, 2, 1, wl.MODE_BEER_LAMBERT)])
+                                                   (3, 2, 1, wl.MODE_BEER_LAMBERT),
+                                                   (2, 1, 2, wl.MODE_ALPHA)])
 @pytest.mark.parametrize("layout,dtype", [(CORNERS, F32), (QUADS, BF16)])
 def test_batched_pose_gradient(cuda, n_vols, C, n_views, mode, layout, dtype):
     # (3, 2, 1): one pose broadcast to three volumes, six images add into it
@@ -186,7 +187,7 @@ def test_batched_pose_gradient(cuda, n_vols, C, n_views, mode, layout, dtype):
     src = _prepared_batch(vols, w.dims, dtype, layout)
     Rt = torch.from_numpy(np.ascontiguousarray(w.Rt.reshape(-1, 12))).cuda()
     fo = None
-    if mode == wl.MODE_BEER_LAMBERT:
+    if mode != wl.MODE_RAW:
         fo = torch.full((n_out, C, w.H, w.W), float("nan"), device="cuda")
         drr.drr_render_batched(src, dtype, layout, w.dims, w.spacing, w.origin, w.K, Rt, n_vols, C,
                                n_views, w.H, w.W, w.n_samples, w.density_factor, mode, fo)

@@ -1,4 +1,5 @@
-"""GPU parity of the pose gradient dL/d[R|t] (drr_render_pose_grad) against
+"""GPU parity of the pose gradient dL/d[R|t] (drr_render_pose_grad; line
+integral, Beer-Lambert and alpha composite) against
 the fp64 oracle's, which tests/test_oracle_pose_pins.py pins to finite
 differences and to a constant-volume closed form.
 
@@ -16,8 +17,8 @@ import pytest
 
 import oracle
 from cone_beam_ct_b200 import workloads as wl
-from tests.gpu_helpers import (BF16, CORNERS, F32, LAYOUTS, LINEAR, PADDED, assert_pose_parity,
-                               bf16_values, gpu_forward, gpu_pose_grad)
+from tests.gpu_helpers import (BF16, CORNERS, F32, LAYOUTS, LINEAR, PADDED, QUADS,
+                               assert_pose_parity, bf16_values, gpu_forward, gpu_pose_grad)
 
 pytestmark = pytest.mark.gpu
 TOL = 1e-4
@@ -54,6 +55,36 @@ def test_pose_gradient_bf16_volume(cuda, layout):
     got = gpu_pose_grad(w, go, layout=layout, dtype=BF16, mode=wl.MODE_RAW)
     ref = _oracle(w, go, wl.MODE_RAW, vol=bf16_values(w.vol))
     assert_pose_parity(got, ref, TOL, what=f"bf16 layout {layout}")
+
+
+@pytest.mark.parametrize("seed", [311, 312])
+@pytest.mark.parametrize("layout,dtype", [(LINEAR, F32), (PADDED, F32), (CORNERS, BF16),
+                                          (QUADS, F32)])
+def test_alpha_pose_gradient_small_ragged(cuda, seed, layout, dtype):
+    # the composite's pose gradient: samples weighted by dC/dmu_i, dt through
+    # the opacities; opacities far from the linear regime
+    w = wl.small_random_case(seed)
+    w.density_factor = 30.0
+    go = np.random.default_rng(seed).standard_normal((w.B, w.H, w.W)).astype(np.float32)
+    fwd = gpu_forward(w, layout=layout, dtype=dtype, mode=wl.MODE_ALPHA)
+    got = gpu_pose_grad(w, go, layout=layout, dtype=dtype, mode=wl.MODE_ALPHA, fwd_out=fwd)
+    vol = bf16_values(w.vol) if dtype == BF16 else None
+    ref = _oracle(w, go, wl.MODE_ALPHA, vol=vol)
+    assert_pose_parity(got, ref, TOL, what=f"alpha seed {seed} layout {layout} dtype {dtype}")
+
+
+@pytest.mark.slow
+def test_alpha_pose_gradient_config3_sparse_upstream(cuda):
+    w = wl.make_config(3)
+    w.density_factor = 10.0
+    rng = np.random.default_rng(37)
+    go = np.zeros((w.B, w.H, w.W), np.float32)
+    ids = rng.choice(w.rays, size=2000, replace=False)
+    go.reshape(-1)[ids] = rng.standard_normal(2000).astype(np.float32)
+    fwd = gpu_forward(w, layout=CORNERS, dtype=BF16, mode=wl.MODE_ALPHA)
+    got = gpu_pose_grad(w, go, layout=CORNERS, dtype=BF16, mode=wl.MODE_ALPHA, fwd_out=fwd)
+    ref = _oracle(w, go, wl.MODE_ALPHA, vol=bf16_values(w.vol), nthreads=4)
+    assert_pose_parity(got, ref, TOL, what="alpha, config 3, 2000 rays")
 
 
 def test_pose_gradient_camera_inside_the_volume(cuda):
