@@ -29,6 +29,7 @@ from .drr import (  # noqa: F401
     drr_render_adjoint_batched,
     drr_render_adjoint_batched_ws,
     drr_render_alpha_adjoint,
+    drr_render_alpha_adjoint_batched,
     drr_render_alpha_adjoint_ws,
     drr_render_batched,
     drr_render_adjoint_noalloc,

@@ -448,16 +448,26 @@ records_kernel(const float* __restrict__ Rt, const float* __restrict__ grad_out,
 // walks each ray once, front to back (no phases: T is sequential), and
 // scatters grad_out * dC/dmu_i * w_corner through the pending 2 x 2 x 2
 // block of the direct path into the fp32 linear gradient volume.
-template <typename T, int LAYOUT>
+template <typename T, int LAYOUT, bool BATCH>
 __global__ void __launch_bounds__(kThreads)
-alpha_adjoint_kernel(const T* __restrict__ vol, const float* __restrict__ Rt,
+alpha_adjoint_kernel(const T* __restrict__ vol_base, const float* __restrict__ Rt,
                      const float* __restrict__ grad_out, const float* __restrict__ fwd_out,
                      float* __restrict__ grad, const Geom g, int grad_row, int grad_slice,
                      const int* __restrict__ flags) {
     __shared__ View sv;
-    const int b = blockIdx.z;
+    const int b = blockIdx.z;                    // output image (view x channel)
     if (flags && flags[1 + b]) return;           // dense view: alpha_records_kernel's
-    if (threadIdx.x == 0) view_setup(Rt + 12 * (size_t)b, g, sv);
+    // batches (a separate instantiation, so that single-volume calls carry
+    // none of its registers): the image's pose and volume-channel
+    const T* __restrict__ vol = vol_base;
+    int pose = b;
+    if constexpr (BATCH) {
+        const BatchItem it = batch_item(g, b);
+        vol += it.slot * g.vstride;
+        grad += it.slot * ((long long)g.nx * g.ny * g.nz);
+        pose = it.pose;
+    }
+    if (threadIdx.x == 0) view_setup(Rt + 12 * (size_t)pose, g, sv);
     __syncthreads();
     int r, c;
     tile_pixel(r, c);
@@ -535,14 +545,17 @@ constexpr int kAlphaTile = 16 * kAlphaBundle;            // 32 x 32 pixels per C
 
 template <typename T, int LAYOUT>
 __global__ void __launch_bounds__(kThreads, 2)
-alpha_records_kernel(const T* __restrict__ vol, const float* __restrict__ Rt,
+alpha_records_kernel(const T* __restrict__ vol_base, const float* __restrict__ Rt,
                      const float* __restrict__ grad_out, const float* __restrict__ fwd_out,
                      const Geom g, const Workspace ws) {
     constexpr int kRays = kAlphaBundle * kAlphaBundle;
     __shared__ View sv;
     const int b = blockIdx.z;
     if (ws.flags[1 + b] == 0) return;            // sparse view: alpha_adjoint_kernel's
-    if (threadIdx.x == 0) view_setup(Rt + 12 * (size_t)b, g, sv);
+    const BatchItem it = batch_item(g, b);
+    const T* __restrict__ vol = vol_base + it.slot * g.vstride;
+    float* const rec = ws.rec + it.slot * ws.rec_stride;   // this volume-channel's records
+    if (threadIdx.x == 0) view_setup(Rt + 12 * (size_t)it.pose, g, sv);
     __syncthreads();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int px = (warp & 1) * 8 + (lane & 7), py = (warp >> 1) * 4 + (lane >> 3);
@@ -617,7 +630,7 @@ alpha_records_kernel(const T* __restrict__ vol, const float* __restrict__ Rt,
                 for (int h = 0; h < kSlots; ++h) {
                     if (h != home) continue;
                     if (pc[h] != cell) {
-                        if (pc[h] >= 0) flush_record(ws.rec, pc[h], p[h]);
+                        if (pc[h] >= 0) flush_record(rec, pc[h], p[h]);
                         pc[h] = cell;
 #pragma unroll
                         for (int e = 0; e < 8; ++e) p[h][e] = 0.0f;
@@ -630,7 +643,7 @@ alpha_records_kernel(const T* __restrict__ vol, const float* __restrict__ Rt,
     }
 #pragma unroll
     for (int h = 0; h < kSlots; ++h)
-        if (pc[h] >= 0) flush_record(ws.rec, pc[h], p[h]);
+        if (pc[h] >= 0) flush_record(rec, pc[h], p[h]);
 }
 
 constexpr int kMaxDevices = 64;
@@ -708,8 +721,12 @@ void alpha_kernels(const void* vol, const Geom& g, const float* Rt, const float*
                    cudaStream_t stream) {
     const T* v = static_cast<const T*>(vol);
     const dim3 grid((g.W + kTileW - 1) / kTileW, (g.H + kTileH - 1) / kTileH, g.B);
-    alpha_adjoint_kernel<T, LAYOUT><<<grid, kThreads, 0, stream>>>(
-        v, Rt, grad_out, fwd_out, grad_vol, g, g.nx, g.nx * g.ny, ws.flags);
+    if (g.C != 1 || g.broadcast || g.views_per_vol != g.B)
+        alpha_adjoint_kernel<T, LAYOUT, true><<<grid, kThreads, 0, stream>>>(
+            v, Rt, grad_out, fwd_out, grad_vol, g, g.nx, g.nx * g.ny, ws.flags);
+    else
+        alpha_adjoint_kernel<T, LAYOUT, false><<<grid, kThreads, 0, stream>>>(
+            v, Rt, grad_out, fwd_out, grad_vol, g, g.nx, g.nx * g.ny, ws.flags);
     if (ws.flags) {
         const dim3 rgrid((g.W + kAlphaTile - 1) / kAlphaTile, (g.H + kAlphaTile - 1) / kAlphaTile,
                          g.B);
@@ -723,12 +740,13 @@ cudaError_t launch_alpha_adjoint(const void* vol, int dtype, int layout, const G
                                  float* grad_vol, void* workspace, cudaStream_t stream) {
     Workspace ws{nullptr, nullptr, 0};
     const int fill_grid = 148 * 8;
+    const int slots = batch_slots(g);
     if (workspace) {
         ws.flags = static_cast<int*>(workspace);
         ws.rec = reinterpret_cast<float*>(static_cast<char*>(workspace) +
                                           adjoint_workspace_header(g.B));
         ws.rec_stride = (long long)(g.nx - 1) * (g.ny - 1) * (g.nz - 1) * 8;
-        const int64_t n_rec4 = (int64_t)(g.nx - 1) * (g.ny - 1) * (g.nz - 1) * 2;
+        const int64_t n_rec4 = (int64_t)(g.nx - 1) * (g.ny - 1) * (g.nz - 1) * 2 * slots;
         plan_views<<<1, 256, 0, stream>>>(Rt, g, ws.flags);
         zero_records<<<fill_grid, 256, 0, stream>>>(ws.flags, reinterpret_cast<float4*>(ws.rec),
                                                     n_rec4);
@@ -744,7 +762,7 @@ cudaError_t launch_alpha_adjoint(const void* vol, int dtype, int layout, const G
     }
     if (workspace)
         gather_records<<<fill_grid, 256, 0, stream>>>(ws.flags, ws.rec, ws.rec_stride, grad_vol,
-                                                      g.nx, g.ny, g.nz, 1);
+                                                      g.nx, g.ny, g.nz, slots);
     return cudaGetLastError();
 }
 

@@ -338,15 +338,23 @@ extern "C" {
 
 namespace {
 
+drr_status batch_shape(int n_vols, int channels, int n_views, int* n_out, int* per_vol,
+                       int* broadcast);
+
 drr_status render_alpha_adjoint(const void* vol, drr_dtype dtype, drr_layout layout,
                                 const int dims[3], const float spacing[3], const float origin[3],
-                                const float K[9], const float* Rt, int B, int H, int W,
-                                int n_samples, float density_factor, const float* grad_out,
-                                const float* fwd_out, float* grad_vol, bool with_ws,
-                                void* workspace, size_t workspace_bytes, void* stream) {
-    drr_status st = check_volume(dims, spacing, origin);
+                                const float K[9], const float* Rt, int n_vols, int channels,
+                                int n_views, int H, int W, int n_samples, float density_factor,
+                                const float* grad_out, const float* fwd_out, float* grad_vol,
+                                bool with_ws, void* workspace, size_t workspace_bytes,
+                                void* stream) {
+    int n_out = 0, per_vol = 1, bcast = 0;
+    drr_status st = batch_shape(n_vols, channels, n_views, &n_out, &per_vol, &bcast);
     if (st != DRR_OK) return st;
-    st = check_rays(K, Rt, B, H, W, n_samples, density_factor, DRR_MODE_ALPHA, true);
+    st = check_volume(dims, spacing, origin);
+    if (st != DRR_OK) return st;
+    const int images = n_out * channels;
+    st = check_rays(K, Rt, images, H, W, n_samples, density_factor, DRR_MODE_ALPHA, true);
     if (st != DRR_OK) return st;
     if (dtype != DRR_F32 && dtype != DRR_BF16) return fail(DRR_ERR_INVALID_ARG, "unknown dtype %d", dtype);
     if (!known_layout(layout)) return fail(DRR_ERR_INVALID_ARG, "unknown layout %d", layout);
@@ -354,7 +362,7 @@ drr_status render_alpha_adjoint(const void* vol, drr_dtype dtype, drr_layout lay
         return fail(DRR_ERR_UNSUPPORTED, "the alpha adjoint reads DRR_LAYOUT_LINEAR, _CORNERS or _QUADS volumes");
     if (stored_elements(dims, layout) > kMaxElements)
         return fail(DRR_ERR_UNSUPPORTED, "volume too large (max 2^31 - 1 stored elements)");
-    const int64_t npix = (int64_t)B * H * W;
+    const int64_t npix = (int64_t)images * H * W;
     if (npix == 0) return ok();
     if (!vol || !aligned(vol, layout_alignment(layout, dtype)))
         return fail(DRR_ERR_INVALID_ARG, "vol must be a non-NULL device pointer aligned to %zu bytes",
@@ -365,24 +373,29 @@ drr_status render_alpha_adjoint(const void* vol, drr_dtype dtype, drr_layout lay
         return fail(DRR_ERR_INVALID_ARG, "fwd_out (the alpha image) is required");
     if (!grad_vol || !aligned(grad_vol, 4))
         return fail(DRR_ERR_INVALID_ARG, "grad_vol must be a non-NULL, 4-byte aligned device pointer");
-    const size_t vbytes = (size_t)dims[0] * dims[1] * dims[2] * 4, ibytes = (size_t)npix * 4;
-    const size_t sbytes = (size_t)stored_elements(dims, layout) * (dtype == DRR_F32 ? 4 : 2);
+    const int slots = n_vols * channels;
+    const size_t vbytes = (size_t)dims[0] * dims[1] * dims[2] * 4 * slots, ibytes = (size_t)npix * 4;
+    const size_t sbytes = (size_t)stored_elements(dims, layout) * (dtype == DRR_F32 ? 4 : 2) * slots;
     if (overlaps(grad_vol, vbytes, grad_out, ibytes) || overlaps(grad_vol, vbytes, fwd_out, ibytes) ||
         overlaps(grad_vol, vbytes, vol, sbytes))
         return fail(DRR_ERR_INVALID_ARG, "grad_vol overlaps another buffer");
     if (with_ws) {
-        const size_t need = drr::adjoint_workspace_bytes(dims[0], dims[1], dims[2], B);
+        const size_t need = drr::adjoint_workspace_bytes(dims[0], dims[1], dims[2], images, slots);
         if (!workspace || !aligned(workspace, 256))
             return fail(DRR_ERR_INVALID_ARG, "workspace must be a non-NULL, 256-byte aligned device pointer");
         if (workspace_bytes < need)
             return fail(DRR_ERR_INVALID_ARG, "workspace holds %zu bytes, %zu needed", workspace_bytes, need);
         if (overlaps(workspace, need, grad_vol, vbytes) || overlaps(workspace, need, grad_out, ibytes) ||
             overlaps(workspace, need, fwd_out, ibytes) || overlaps(workspace, need, vol, sbytes) ||
-            overlaps(workspace, need, Rt, (size_t)B * 12 * sizeof(float)))
+            overlaps(workspace, need, Rt, (size_t)n_views * 12 * sizeof(float)))
             return fail(DRR_ERR_INVALID_ARG, "workspace overlaps another buffer");
     }
     drr::Geom g;
-    drr::fill_geom(g, dims, spacing, origin, K, B, H, W, n_samples, density_factor, layout);
+    drr::fill_geom(g, dims, spacing, origin, K, images, H, W, n_samples, density_factor, layout);
+    g.C = channels;
+    g.views_per_vol = per_vol;
+    g.broadcast = bcast;
+    g.vstride = stored_elements(dims, layout);
     return cuda_status(drr::launch_alpha_adjoint(vol, dtype, layout, g, Rt, grad_out, fwd_out,
                                                  grad_vol, with_ws ? workspace : nullptr,
                                                  static_cast<cudaStream_t>(stream)),
@@ -399,7 +412,7 @@ DRR_API drr_status drr_render_alpha_adjoint(const void* vol, drr_dtype dtype, dr
                                             const float* Rt, int B, int H, int W, int n_samples,
                                             float density_factor, const float* grad_out,
                                             const float* fwd_out, float* grad_vol, void* stream) {
-    return render_alpha_adjoint(vol, dtype, layout, dims, spacing, origin, K, Rt, B, H, W,
+    return render_alpha_adjoint(vol, dtype, layout, dims, spacing, origin, K, Rt, 1, 1, B, H, W,
                                 n_samples, density_factor, grad_out, fwd_out, grad_vol, false,
                                 nullptr, 0, stream);
 }
@@ -412,9 +425,24 @@ DRR_API drr_status drr_render_alpha_adjoint_ws(const void* vol, drr_dtype dtype,
                                                const float* grad_out, const float* fwd_out,
                                                float* grad_vol, void* workspace,
                                                size_t workspace_bytes, void* stream) {
-    return render_alpha_adjoint(vol, dtype, layout, dims, spacing, origin, K, Rt, B, H, W,
+    return render_alpha_adjoint(vol, dtype, layout, dims, spacing, origin, K, Rt, 1, 1, B, H, W,
                                 n_samples, density_factor, grad_out, fwd_out, grad_vol, true,
                                 workspace, workspace_bytes, stream);
+}
+
+DRR_API drr_status drr_render_alpha_adjoint_batched(const void* vols, drr_dtype dtype,
+                                                    drr_layout layout, const int dims[3],
+                                                    const float spacing[3], const float origin[3],
+                                                    const float K[9], const float* Rt,
+                                                    int n_vols, int channels, int n_views, int H,
+                                                    int W, int n_samples, float density_factor,
+                                                    const float* grad_out, const float* fwd_out,
+                                                    float* grad_vols, void* workspace,
+                                                    size_t workspace_bytes, void* stream) {
+    return render_alpha_adjoint(vols, dtype, layout, dims, spacing, origin, K, Rt, n_vols,
+                                channels, n_views, H, W, n_samples, density_factor, grad_out,
+                                fwd_out, grad_vols, workspace != nullptr, workspace,
+                                workspace_bytes, stream);
 }
 
 DRR_API drr_status drr_poisson_noise(const float* image, const float* z, float i0, float* out,

@@ -25,7 +25,7 @@ EXPORTED = ("drr_render", "drr_render_adjoint", "drr_render_adjoint_ws",
             "drr_render_alpha_adjoint", "drr_render_alpha_adjoint_ws", "drr_poisson_noise", "drr_poisson_noise_backward",
             "drr_render_siddon", "drr_render_siddon_adjoint", "drr_render_batched",
             "drr_render_adjoint_batched", "drr_adjoint_batched_workspace_bytes",
-            "drr_render_pose_grad_batched",
+            "drr_render_pose_grad_batched", "drr_render_alpha_adjoint_batched",
             "drr_render_adjoint_batched_ws",
             "drr_prepared_bytes", "drr_prepare_volume", "drr_get_last_error", "drr_abi_version")
 DRR_NOALLOC_SCRATCH_BYTES = 32 << 20
@@ -85,6 +85,11 @@ def lib():
                                               _c.c_int, _c.c_int, _c.c_int, _c.c_int, _c.c_float,
                                               _vp, _vp, _vp, _vp, _c.c_size_t, _vp]
     L.drr_render_alpha_adjoint_ws.restype = _c.c_int
+    L.drr_render_alpha_adjoint_batched.argtypes = [_vp, _c.c_int, _c.c_int, _i3, _f3, _f3, _f9,
+                                                   _vp, _c.c_int, _c.c_int, _c.c_int, _c.c_int,
+                                                   _c.c_int, _c.c_int, _c.c_float, _vp, _vp, _vp,
+                                                   _vp, _c.c_size_t, _vp]
+    L.drr_render_alpha_adjoint_batched.restype = _c.c_int
     L.drr_poisson_noise.argtypes = [_vp, _vp, _c.c_float, _vp, _c.c_int64, _vp]
     L.drr_poisson_noise.restype = _c.c_int
     L.drr_poisson_noise_backward.argtypes = [_vp, _vp, _c.c_float, _vp, _vp, _c.c_int64, _vp]
@@ -258,6 +263,25 @@ def drr_render_alpha_adjoint_ws(vol, dtype, layout, dims, spacing, origin, K, Rt
                                              _dev(grad_vol, "grad_vol", True),
                                              _dev(workspace, "workspace", True),
                                              int(workspace_bytes), _stream(stream)))
+
+
+def drr_render_alpha_adjoint_batched(vols, dtype, layout, dims, spacing, origin, K, Rt, n_vols,
+                                     channels, n_views, H, W, n_samples, density_factor,
+                                     grad_out, fwd_out, grad_vols, workspace=None,
+                                     workspace_bytes=None, stream=None):
+    if workspace_bytes is None:
+        workspace_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().drr_render_alpha_adjoint_batched(_dev(vols, "vols", True), int(dtype),
+                                                  int(layout), _i3v(dims), _f3v(spacing),
+                                                  _f3v(origin), _f9v(K), _dev(Rt, "Rt", True),
+                                                  int(n_vols), int(channels), int(n_views),
+                                                  int(H), int(W), int(n_samples),
+                                                  float(density_factor),
+                                                  _dev(grad_out, "grad_out", True),
+                                                  _dev(fwd_out, "fwd_out", True),
+                                                  _dev(grad_vols, "grad_vols", True),
+                                                  _dev(workspace, "workspace", True),
+                                                  int(workspace_bytes), _stream(stream)))
 
 
 def drr_poisson_noise(image, z, i0, out, n=None, stream=None):

@@ -316,6 +316,25 @@ DRR_API drr_status drr_render_alpha_adjoint_ws(const void *vol, drr_dtype dtype,
                                                float *grad_vol, void *workspace,
                                                size_t workspace_bytes, void *stream);
 
+/* Volume gradient of a batched DRR_MODE_ALPHA render (drr_render_batched):
+ * grad_vols, DEVICE float32 [n_vols * channels][nz][ny][nx] (linear),
+ * ACCUMULATED into; each image's gradient goes to the volume-channel it was
+ * rendered from.  workspace: NULL (every image on the direct path) or at
+ * least drr_adjoint_batched_workspace_bytes(dims, n_vols, channels, n_views)
+ * bytes, 256-byte aligned (dense images accumulate into the corner records of
+ * their volume-channel).  vols, Rt, grad_out and fwd_out (the batched alpha
+ * image, required) as drr_render_batched; other arguments as
+ * drr_render_alpha_adjoint_ws. */
+DRR_API drr_status drr_render_alpha_adjoint_batched(const void *vols, drr_dtype dtype,
+                                                    drr_layout layout, const int dims[3],
+                                                    const float spacing[3], const float origin[3],
+                                                    const float K[9], const float *Rt,
+                                                    int n_vols, int channels, int n_views, int H,
+                                                    int W, int n_samples, float density_factor,
+                                                    const float *grad_out, const float *fwd_out,
+                                                    float *grad_vols, void *workspace,
+                                                    size_t workspace_bytes, void *stream);
+
 /* Gaussian-Poisson surrogate of shot noise (flashdrr.rendering API docs,
  * VolumeRaycaster.apply_poisson) on a Beer-Lambert image: with transmission
  * T = 1 - image, T' = clamp(T + sqrt(T / i0) z, 0, 1) and out = 1 - T'.

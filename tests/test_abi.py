@@ -456,6 +456,33 @@ def test_batched_pose_gradient_empty_batch_is_a_no_op():
     assert drr.drr_get_last_error() == ""
 
 
+def _alpha_batched(**kw):
+    args = dict(vols=FAKE, dtype=drr.DRR_F32, layout=drr.DRR_LAYOUT_CORNERS, dims=DIMS, spacing=SP,
+                origin=ORG, K=K_OK, Rt=FAKE + (1 << 26), n_vols=2, channels=1, n_views=2, H=8,
+                W=8, n_samples=16, density_factor=1.0, grad_out=FAKE + (1 << 27),
+                fwd_out=FAKE + (1 << 28), grad_vols=FAKE + (1 << 29), workspace=None, stream=0)
+    args.update(kw)
+    return drr.drr_render_alpha_adjoint_batched(**args)
+
+
+ALPHA_BATCHED_BAD = [
+    (dict(layout=drr.DRR_LAYOUT_PADDED), drr.DRR_ERR_UNSUPPORTED, "LINEAR"),
+    (dict(fwd_out=0), drr.DRR_ERR_INVALID_ARG, "alpha image"),
+    (dict(n_views=3), drr.DRR_ERR_INVALID_ARG, "multiple"),
+    (dict(grad_vols=FAKE), drr.DRR_ERR_INVALID_ARG, "overlaps"),          # on the volumes
+    (dict(workspace=WS, workspace_bytes=1000), drr.DRR_ERR_INVALID_ARG, "needed"),
+    (dict(workspace=WS + 64, workspace_bytes=WS_BYTES), drr.DRR_ERR_INVALID_ARG, "aligned"),
+]
+
+
+@pytest.mark.parametrize("kw,status,word", ALPHA_BATCHED_BAD)
+def test_batched_alpha_adjoint_rejects_bad_arguments(kw, status, word):
+    with pytest.raises(drr.DrrError) as e:
+        _alpha_batched(**kw)
+    assert e.value.status == status
+    assert word in drr.drr_get_last_error()
+
+
 def test_prepared_bytes():
     assert drr.drr_prepared_bytes((256, 256, 256), drr.DRR_F32, drr.DRR_LAYOUT_LINEAR) == 4 * 256 ** 3
     assert drr.drr_prepared_bytes((256, 256, 256), drr.DRR_BF16, drr.DRR_LAYOUT_LINEAR) == 2 * 256 ** 3

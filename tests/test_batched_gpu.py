@@ -198,3 +198,39 @@ def test_batched_pose_gradient(cuda, n_vols, C, n_views, mode, layout, dtype):
     torch.cuda.synchronize()
     assert_pose_parity(g.cpu().numpy().reshape(-1, 3, 4), ref, 1e-4,
                        what=f"batched ({n_vols}, {C}, {n_views}) layout {layout} dtype {dtype}")
+
+
+@pytest.mark.parametrize("n_vols,C,n_views", [(2, 2, 4), (3, 1, 1)])
+@pytest.mark.parametrize("layout,dtype", [(CORNERS, BF16), (QUADS, F32)])
+def test_batched_alpha_volume_gradient(cuda, n_vols, C, n_views, layout, dtype):
+    # dense geometry: with a workspace the images take the alpha record path of
+    # their volume-channel; without one, the direct path
+    import torch
+    seed = 661 + n_views
+    w = wl.small_random_case(seed, B=n_views, **DENSE)
+    w.density_factor = 25.0
+    nx, ny, nz = w.dims
+    vols = np.random.default_rng(seed).uniform(0.0, 0.05, (n_vols, C, nz, ny, nx)).astype(np.float32)
+    n_out = n_vols if (n_views == 1 and n_vols > 1) else n_views
+    go = np.random.default_rng(9).standard_normal((n_out, C, w.H, w.W)).astype(np.float32)
+    ref_vols = bf16_values(vols) if dtype == BF16 else vols
+    ref = oracle.adjoint_batched(w.dims, w.spacing, w.origin, w.K, w.Rt, n_vols, n_views, w.H,
+                                 w.W, w.n_samples, w.density_factor, wl.MODE_ALPHA, go,
+                                 vols=ref_vols, nthreads=8)
+    src = _prepared_batch(vols, w.dims, dtype, layout)
+    Rt = torch.from_numpy(np.ascontiguousarray(w.Rt.reshape(-1, 12))).cuda()
+    fo = torch.full((n_out, C, w.H, w.W), float("nan"), device="cuda")
+    drr.drr_render_batched(src, dtype, layout, w.dims, w.spacing, w.origin, w.K, Rt, n_vols, C,
+                           n_views, w.H, w.W, w.n_samples, w.density_factor, wl.MODE_ALPHA, fo)
+    go_d = torch.from_numpy(go).cuda()
+    for workspace in (False, True):
+        g = torch.zeros((n_vols, C, nz, ny, nx), device="cuda")
+        ws = None
+        if workspace:
+            ws = torch.full((drr.drr_adjoint_batched_workspace_bytes(w.dims, n_vols, C, n_views),),
+                            0x7F, dtype=torch.uint8, device="cuda")
+        drr.drr_render_alpha_adjoint_batched(src, dtype, layout, w.dims, w.spacing, w.origin, w.K,
+                                             Rt, n_vols, C, n_views, w.H, w.W, w.n_samples,
+                                             w.density_factor, go_d, fo, g, ws)
+        torch.cuda.synchronize()
+        _assert_batched_adjoint(g.cpu().numpy(), ref, f"alpha workspace {workspace}")

@@ -102,3 +102,30 @@ def test_batched_pose_gradient_matches_finite_differences_of_the_batched_render(
                 fd[r, c] = (objective(Rp) - objective(Rm)) / (2 * h)
         assert np.max(np.abs(g[p, :, :3] - fd[:, :3])) <= 1e-6 * np.max(np.abs(fd[:, :3]))
         assert np.max(np.abs(g[p, :, 3] - fd[:, 3])) <= 1e-5 * np.max(np.abs(fd[:, 3]))
+
+
+def test_batched_alpha_volume_gradient_matches_finite_differences():
+    # the alpha composite is not linear in the volume: its batched gradient
+    # (adjoint_batched in alpha mode, each image's gradient into its own
+    # volume-channel) against central differences of the batched alpha render
+    w, Rt, _, _ = _case(2, 2, 4, 97)
+    w.density_factor = 30.0
+    nx, ny, nz = w.dims
+    rng = np.random.default_rng(21)
+    vols = rng.uniform(0.0, 0.05, (2, 2, nz, ny, nx)).astype(np.float32)
+    go = rng.standard_normal((4, 2, w.H, w.W))
+    g = oracle.adjoint_batched(w.dims, w.spacing, w.origin, w.K, Rt, 2, 4, w.H, w.W, w.n_samples,
+                               w.density_factor, wl.MODE_ALPHA, go, vols=vols)
+    for _ in range(3):
+        delta = rng.standard_normal(vols.shape)
+        h = 1e-5
+        vp = (vols + h * delta).astype(np.float32)
+        vm = (vols - h * delta).astype(np.float32)
+        dv = vp.astype(np.float64) - vm.astype(np.float64)
+        fd = np.sum(go * (oracle.render_batched(vp, w.dims, w.spacing, w.origin, w.K, Rt, 4, w.H,
+                                                w.W, w.n_samples, w.density_factor,
+                                                wl.MODE_ALPHA) -
+                          oracle.render_batched(vm, w.dims, w.spacing, w.origin, w.K, Rt, 4, w.H,
+                                                w.W, w.n_samples, w.density_factor,
+                                                wl.MODE_ALPHA)))
+        assert abs(fd - np.sum(g * dv)) <= 1e-6 * np.sum(np.abs(g * dv))
