@@ -106,212 +106,150 @@ bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
     return pa < pb + nb && pb < pa + na;
 }
 
-}  // namespace
-
-extern "C" {
-
-DRR_API int drr_abi_version(void) { return 1; }
-
-DRR_API const char* drr_get_last_error(void) { return g_last_error; }
-
-DRR_API size_t drr_prepared_bytes(const int dims[3], drr_dtype dtype, drr_layout layout) {
-    if (!dims) return 0;
-    for (int a = 0; a < 3; ++a)
-        if (dims[a] < 2 || dims[a] > kMaxDim) return 0;
-    if (dtype != DRR_F32 && dtype != DRR_BF16) return 0;
-    if (!known_layout(layout)) return 0;
-    const int64_t n = stored_elements(dims, layout);
-    if (n > kMaxElements) return 0;
-    return (size_t)n * (dtype == DRR_F32 ? 4 : 2);
+// The batch rule of VolumeRaycaster.forward: n_views view matrices for
+// n_vols volumes of `channels` channels; n_views == 1 is broadcast to every
+// volume, else n_views must be a multiple of n_vols (views_per_vol of them
+// per volume, consecutive).  Output images: n_out x channels.
+drr_status batch_shape(int n_vols, int channels, int n_views, int* n_out, int* per_vol,
+                       int* broadcast) {
+    if (n_vols < 0 || channels < 0 || n_views < 0)
+        return fail(DRR_ERR_INVALID_ARG, "n_vols, channels and n_views must be >= 0");
+    if (n_vols == 0 || channels == 0 || n_views == 0) {
+        *n_out = 0;
+        *per_vol = 1;
+        *broadcast = 0;
+        return DRR_OK;
+    }
+    if (n_views == 1 && n_vols > 1) {
+        *n_out = n_vols;
+        *per_vol = 1;
+        *broadcast = 1;
+    } else if (n_views % n_vols == 0) {
+        *n_out = n_views;
+        *per_vol = n_views / n_vols;
+        *broadcast = 0;
+    } else {
+        return fail(DRR_ERR_INVALID_ARG,
+                    "n_views = %d must be 1 or a multiple of n_vols = %d", n_views, n_vols);
+    }
+    if ((int64_t)*n_out * channels > kMaxViews)
+        return fail(DRR_ERR_UNSUPPORTED, "%lld images (views x channels) exceed %d per call",
+                    (long long)*n_out * channels, kMaxViews);
+    return DRR_OK;
 }
 
-DRR_API drr_status drr_prepare_volume(const float* src, const int dims[3], drr_dtype dtype,
-                                      drr_layout layout, void* dst, size_t dst_bytes,
-                                      void* stream) {
-    if (!dims) return fail(DRR_ERR_INVALID_ARG, "dims must be non-NULL");
-    for (int a = 0; a < 3; ++a)
-        if (dims[a] < 2 || dims[a] > kMaxDim)
-            return fail(DRR_ERR_INVALID_ARG, "dims[%d] = %d must be in [2, %d]", a, dims[a], kMaxDim);
-    if (dtype != DRR_F32 && dtype != DRR_BF16) return fail(DRR_ERR_INVALID_ARG, "unknown dtype %d", dtype);
-    if (!known_layout(layout)) return fail(DRR_ERR_INVALID_ARG, "unknown layout %d", layout);
-    const size_t need = drr_prepared_bytes(dims, dtype, layout);
-    if (need == 0) return fail(DRR_ERR_UNSUPPORTED, "volume too large (max 2^31 - 1 stored elements)");
-    if (!src || !dst) return fail(DRR_ERR_INVALID_ARG, "src and dst must be non-NULL");
-    if (!aligned(src, 4) || !aligned(dst, layout_alignment(layout, DRR_F32)))
-        return fail(DRR_ERR_INVALID_ARG, "src must be 4-byte aligned, dst 4-byte (16-byte for DRR_LAYOUT_CORNERS and DRR_LAYOUT_QUADS)");
-    if (dst_bytes < need)
-        return fail(DRR_ERR_INVALID_ARG, "dst holds %zu bytes, %zu needed", dst_bytes, need);
-    const size_t src_bytes = (size_t)dims[0] * dims[1] * dims[2] * 4;
-    if (overlaps(src, src_bytes, dst, need)) return fail(DRR_ERR_INVALID_ARG, "src and dst overlap");
-    return cuda_status(drr::launch_prepare(src, dims[0], dims[1], dims[2], dtype, layout, dst,
-                                           static_cast<cudaStream_t>(stream)),
-                       "drr_prepare_volume launch");
-}
+// The implementations, over batches of volumes x channels x views; each
+// single-volume entry point is the case n_vols = channels = 1, n_views = B.
 
-DRR_API drr_status drr_render(const void* vol, drr_dtype dtype, drr_layout layout,
-                              const int dims[3], const float spacing[3], const float origin[3],
-                              const float K[9], const float* Rt, int B, int H, int W,
-                              int n_samples, float density_factor, drr_mode mode, float* out,
-                              void* stream) {
-    drr_status st = check_volume(dims, spacing, origin);
+drr_status render_batched(const void* vols, drr_dtype dtype, drr_layout layout, const int dims[3],
+                          const float spacing[3], const float origin[3], const float K[9],
+                          const float* Rt, int n_vols, int channels, int n_views, int H, int W,
+                          int n_samples, float density_factor, drr_mode mode, float* out,
+                          void* stream) {
+    int n_out = 0, per_vol = 1, bcast = 0;
+    drr_status st = batch_shape(n_vols, channels, n_views, &n_out, &per_vol, &bcast);
     if (st != DRR_OK) return st;
-    st = check_rays(K, Rt, B, H, W, n_samples, density_factor, mode, true);
+    st = check_volume(dims, spacing, origin);
+    if (st != DRR_OK) return st;
+    const int images = n_out * channels;
+    st = check_rays(K, Rt, images, H, W, n_samples, density_factor, mode, true);
     if (st != DRR_OK) return st;
     if (dtype != DRR_F32 && dtype != DRR_BF16) return fail(DRR_ERR_INVALID_ARG, "unknown dtype %d", dtype);
     if (!known_layout(layout)) return fail(DRR_ERR_INVALID_ARG, "unknown layout %d", layout);
     if (stored_elements(dims, layout) > kMaxElements)
         return fail(DRR_ERR_UNSUPPORTED, "volume too large (max 2^31 - 1 stored elements)");
-    if ((int64_t)B * H * W == 0) return ok();   // empty batch or image: nothing to do
-    if (!vol || !aligned(vol, layout_alignment(layout, dtype)))
-        return fail(DRR_ERR_INVALID_ARG, "vol must be a non-NULL device pointer aligned to %zu bytes",
+    if ((int64_t)images * H * W == 0) return ok();
+    if (!vols || !aligned(vols, layout_alignment(layout, dtype)))
+        return fail(DRR_ERR_INVALID_ARG, "vols must be a non-NULL device pointer aligned to %zu bytes",
                     layout_alignment(layout, dtype));
     if (!out || !aligned(out, 4)) return fail(DRR_ERR_INVALID_ARG, "out must be a non-NULL, 4-byte aligned device pointer");
     drr::Geom g;
-    drr::fill_geom(g, dims, spacing, origin, K, B, H, W, n_samples, density_factor, layout);
-    return cuda_status(drr::launch_forward(vol, dtype, layout, g, Rt, mode, out,
+    drr::fill_geom(g, dims, spacing, origin, K, images, H, W, n_samples, density_factor, layout);
+    g.C = channels;
+    g.views_per_vol = per_vol;
+    g.broadcast = bcast;
+    g.vstride = stored_elements(dims, layout);
+    return cuda_status(drr::launch_forward(vols, dtype, layout, g, Rt, mode, out,
                                            static_cast<cudaStream_t>(stream)),
                        "drr_render launch");
 }
 
-}  // extern "C"
-
-namespace {
-
-drr_status render_adjoint(const int dims[3], const float spacing[3], const float origin[3],
-                          const float K[9], const float* Rt, int B, int H, int W, int n_samples,
-                          float density_factor, int mode, const float* grad_out,
-                          const float* fwd_out, float* grad_vol, bool with_ws, void* workspace,
-                          size_t workspace_bytes, void* stream) {
-    drr_status st = check_volume(dims, spacing, origin);
+drr_status render_adjoint_batched(const int dims[3], const float spacing[3], const float origin[3],
+                                  const float K[9], const float* Rt, int n_vols, int channels,
+                                  int n_views, int H, int W, int n_samples, float density_factor,
+                                  drr_mode mode, const float* grad_out, const float* fwd_out,
+                                  float* grad_vols, bool with_ws, void* workspace,
+                                  size_t workspace_bytes, void* stream) {
+    int n_out = 0, per_vol = 1, bcast = 0;
+    drr_status st = batch_shape(n_vols, channels, n_views, &n_out, &per_vol, &bcast);
     if (st != DRR_OK) return st;
-    st = check_rays(K, Rt, B, H, W, n_samples, density_factor, mode);
+    st = check_volume(dims, spacing, origin);
+    if (st != DRR_OK) return st;
+    const int images = n_out * channels;
+    st = check_rays(K, Rt, images, H, W, n_samples, density_factor, mode);
     if (st != DRR_OK) return st;
     if (stored_elements(dims, DRR_LAYOUT_LINEAR) > kMaxElements)
         return fail(DRR_ERR_UNSUPPORTED, "volume too large (max 2^31 - 1 elements)");
-    const int64_t npix = (int64_t)B * H * W;
+    const int64_t npix = (int64_t)images * H * W;
     if (npix == 0) return ok();
     if (!grad_out || !aligned(grad_out, 4))
         return fail(DRR_ERR_INVALID_ARG, "grad_out must be a non-NULL, 4-byte aligned device pointer");
     if (mode == DRR_MODE_BEER_LAMBERT && (!fwd_out || !aligned(fwd_out, 4)))
         return fail(DRR_ERR_INVALID_ARG, "fwd_out is required in Beer-Lambert mode");
-    if (!grad_vol || !aligned(grad_vol, 4))
-        return fail(DRR_ERR_INVALID_ARG, "grad_vol must be a non-NULL, 4-byte aligned device pointer");
-    const size_t vbytes = (size_t)dims[0] * dims[1] * dims[2] * 4, ibytes = (size_t)npix * 4;
-    if (overlaps(grad_vol, vbytes, grad_out, ibytes) ||
-        (mode == DRR_MODE_BEER_LAMBERT && overlaps(grad_vol, vbytes, fwd_out, ibytes)))
-        return fail(DRR_ERR_INVALID_ARG, "grad_vol overlaps an image buffer");
+    if (!grad_vols || !aligned(grad_vols, 4))
+        return fail(DRR_ERR_INVALID_ARG, "grad_vols must be a non-NULL, 4-byte aligned device pointer");
+    const int64_t nvox = (int64_t)dims[0] * dims[1] * dims[2];
+    const size_t vbytes = (size_t)nvox * n_vols * channels * 4, ibytes = (size_t)npix * 4;
+    if (overlaps(grad_vols, vbytes, grad_out, ibytes) ||
+        (mode == DRR_MODE_BEER_LAMBERT && overlaps(grad_vols, vbytes, fwd_out, ibytes)))
+        return fail(DRR_ERR_INVALID_ARG, "grad_vols overlaps an image buffer");
     if (with_ws) {
-        const size_t need = drr::adjoint_workspace_bytes(dims[0], dims[1], dims[2], B);
+        const size_t need =
+            drr::adjoint_workspace_bytes(dims[0], dims[1], dims[2], images, n_vols * channels);
         if (!workspace || !aligned(workspace, 256))
             return fail(DRR_ERR_INVALID_ARG, "workspace must be a non-NULL, 256-byte aligned device pointer");
         if (workspace_bytes < need)
             return fail(DRR_ERR_INVALID_ARG, "workspace holds %zu bytes, %zu needed", workspace_bytes, need);
-        if (overlaps(workspace, need, grad_vol, vbytes) || overlaps(workspace, need, grad_out, ibytes) ||
+        if (overlaps(workspace, need, grad_vols, vbytes) || overlaps(workspace, need, grad_out, ibytes) ||
             (mode == DRR_MODE_BEER_LAMBERT && overlaps(workspace, need, fwd_out, ibytes)) ||
-            overlaps(workspace, need, Rt, (size_t)B * 12 * sizeof(float)))
+            overlaps(workspace, need, Rt, (size_t)n_views * 12 * sizeof(float)))
             return fail(DRR_ERR_INVALID_ARG, "workspace overlaps another buffer");
     }
     drr::Geom g;
-    drr::fill_geom(g, dims, spacing, origin, K, B, H, W, n_samples, density_factor, DRR_LAYOUT_LINEAR);
-    return cuda_status(drr::launch_adjoint(g, Rt, mode, grad_out, fwd_out, grad_vol,
+    drr::fill_geom(g, dims, spacing, origin, K, images, H, W, n_samples, density_factor,
+                   DRR_LAYOUT_LINEAR);
+    g.C = channels;
+    g.views_per_vol = per_vol;
+    g.broadcast = bcast;
+    g.vstride = nvox;
+    return cuda_status(drr::launch_adjoint(g, Rt, mode, grad_out, fwd_out, grad_vols,
                                            with_ws ? workspace : nullptr,
                                            static_cast<cudaStream_t>(stream)),
-                       "drr_render_adjoint launch");
+                       "drr_render_adjoint_batched launch");
 }
 
-}  // namespace
-
-extern "C" {
-
-DRR_API drr_status drr_render_adjoint(const int dims[3], const float spacing[3],
-                                      const float origin[3], const float K[9], const float* Rt,
-                                      int B, int H, int W, int n_samples, float density_factor,
-                                      drr_mode mode, const float* grad_out, const float* fwd_out,
-                                      float* grad_vol, void* stream) {
-    return render_adjoint(dims, spacing, origin, K, Rt, B, H, W, n_samples, density_factor, mode,
-                          grad_out, fwd_out, grad_vol, false, nullptr, 0, stream);
-}
-
-DRR_API size_t drr_adjoint_workspace_bytes(const int dims[3], int B) {
-    if (!dims || B < 0 || B > kMaxViews) return 0;
-    for (int a = 0; a < 3; ++a)
-        if (dims[a] < 2 || dims[a] > kMaxDim) return 0;
-    if (stored_elements(dims, DRR_LAYOUT_LINEAR) > kMaxElements) return 0;
-    return drr::adjoint_workspace_bytes(dims[0], dims[1], dims[2], B);
-}
-
-DRR_API drr_status drr_render_adjoint_ws(const int dims[3], const float spacing[3],
-                                         const float origin[3], const float K[9], const float* Rt,
-                                         int B, int H, int W, int n_samples, float density_factor,
-                                         drr_mode mode, const float* grad_out, const float* fwd_out,
-                                         float* grad_vol, void* workspace, size_t workspace_bytes,
-                                         void* stream) {
-    return render_adjoint(dims, spacing, origin, K, Rt, B, H, W, n_samples, density_factor, mode,
-                          grad_out, fwd_out, grad_vol, true, workspace, workspace_bytes, stream);
-}
-
-// Adjoint for callers that may not allocate device memory (see include/drr.h):
-// the workspace of drr_render_adjoint_ws comes from the library's built-in
-// scratch instead of the caller.  No allocation happens here or below.
-DRR_API drr_status drr_render_adjoint_noalloc(const int dims[3], const float spacing[3],
-                                              const float origin[3], const float K[9],
-                                              const float* Rt, int B, int H, int W,
-                                              int n_samples, float density_factor, drr_mode mode,
-                                              const float* grad_out, const float* fwd_out,
-                                              float* grad_vol, void* stream) {
-    drr_status st = check_volume(dims, spacing, origin);
+drr_status pose_grad_batched(const void* vols, drr_dtype dtype, drr_layout layout,
+                             const int dims[3], const float spacing[3], const float origin[3],
+                             const float K[9], const float* Rt, int n_vols, int channels,
+                             int n_views, int H, int W, int n_samples, float density_factor,
+                             drr_mode mode, const float* grad_out, const float* fwd_out,
+                             float* grad_Rt, void* stream) {
+    int n_out = 0, per_vol = 1, bcast = 0;
+    drr_status st = batch_shape(n_vols, channels, n_views, &n_out, &per_vol, &bcast);
     if (st != DRR_OK) return st;
-    st = check_rays(K, Rt, B, H, W, n_samples, density_factor, mode);
+    st = check_volume(dims, spacing, origin);
     if (st != DRR_OK) return st;
-    if (stored_elements(dims, DRR_LAYOUT_LINEAR) > kMaxElements)
-        return fail(DRR_ERR_UNSUPPORTED, "volume too large (max 2^31 - 1 elements)");
-    const size_t need = drr::adjoint_workspace_bytes(dims[0], dims[1], dims[2], B);
-    if (need > drr::kNoAllocScratchBytes)
-        return fail(DRR_ERR_UNSUPPORTED,
-                    "this volume and view count need %zu bytes of scratch; the built-in scratch "
-                    "holds %zu (use drr_render_adjoint_ws with a workspace of your own)",
-                    need, drr::kNoAllocScratchBytes);
-    const int64_t npix = (int64_t)B * H * W;
-    if (npix == 0) return ok();
-    if (!grad_out || !aligned(grad_out, 4))
-        return fail(DRR_ERR_INVALID_ARG, "grad_out must be a non-NULL, 4-byte aligned device pointer");
-    if (mode == DRR_MODE_BEER_LAMBERT && (!fwd_out || !aligned(fwd_out, 4)))
-        return fail(DRR_ERR_INVALID_ARG, "fwd_out is required in Beer-Lambert mode");
-    if (!grad_vol || !aligned(grad_vol, 4))
-        return fail(DRR_ERR_INVALID_ARG, "grad_vol must be a non-NULL, 4-byte aligned device pointer");
-    const size_t vbytes = (size_t)dims[0] * dims[1] * dims[2] * 4, ibytes = (size_t)npix * 4;
-    if (overlaps(grad_vol, vbytes, grad_out, ibytes) ||
-        (mode == DRR_MODE_BEER_LAMBERT && overlaps(grad_vol, vbytes, fwd_out, ibytes)))
-        return fail(DRR_ERR_INVALID_ARG, "grad_vol overlaps an image buffer");
-    drr::Geom g;
-    drr::fill_geom(g, dims, spacing, origin, K, B, H, W, n_samples, density_factor, DRR_LAYOUT_LINEAR);
-    return cuda_status(drr::launch_adjoint_noalloc(g, Rt, mode, grad_out, fwd_out, grad_vol,
-                                                   static_cast<cudaStream_t>(stream)),
-                       "drr_render_adjoint_noalloc");
-}
-
-}  // extern "C"
-
-extern "C" {
-
-DRR_API drr_status drr_render_pose_grad(const void* vol, drr_dtype dtype, drr_layout layout,
-                                        const int dims[3], const float spacing[3],
-                                        const float origin[3], const float K[9], const float* Rt,
-                                        int B, int H, int W, int n_samples, float density_factor,
-                                        drr_mode mode, const float* grad_out, const float* fwd_out,
-                                        float* grad_Rt, void* stream) {
-    drr_status st = check_volume(dims, spacing, origin);
-    if (st != DRR_OK) return st;
-    st = check_rays(K, Rt, B, H, W, n_samples, density_factor, mode, true);
+    const int images = n_out * channels;
+    st = check_rays(K, Rt, images, H, W, n_samples, density_factor, mode, true);
     if (st != DRR_OK) return st;
     if (dtype != DRR_F32 && dtype != DRR_BF16) return fail(DRR_ERR_INVALID_ARG, "unknown dtype %d", dtype);
     if (!known_layout(layout)) return fail(DRR_ERR_INVALID_ARG, "unknown layout %d", layout);
     if (stored_elements(dims, layout) > kMaxElements)
         return fail(DRR_ERR_UNSUPPORTED, "volume too large (max 2^31 - 1 stored elements)");
-    const int64_t npix = (int64_t)B * H * W;
+    const int64_t npix = (int64_t)images * H * W;
     if (npix == 0) return ok();
-    if (!vol || !aligned(vol, layout_alignment(layout, dtype)))
-        return fail(DRR_ERR_INVALID_ARG, "vol must be a non-NULL device pointer aligned to %zu bytes",
+    if (!vols || !aligned(vols, layout_alignment(layout, dtype)))
+        return fail(DRR_ERR_INVALID_ARG, "vols must be a non-NULL device pointer aligned to %zu bytes",
                     layout_alignment(layout, dtype));
     if (!grad_out || !aligned(grad_out, 4))
         return fail(DRR_ERR_INVALID_ARG, "grad_out must be a non-NULL, 4-byte aligned device pointer");
@@ -319,27 +257,20 @@ DRR_API drr_status drr_render_pose_grad(const void* vol, drr_dtype dtype, drr_la
         return fail(DRR_ERR_INVALID_ARG, "fwd_out is required in Beer-Lambert and alpha mode");
     if (!grad_Rt || !aligned(grad_Rt, 4))
         return fail(DRR_ERR_INVALID_ARG, "grad_Rt must be a non-NULL, 4-byte aligned device pointer");
-    const size_t gbytes = (size_t)B * 12 * sizeof(float), ibytes = (size_t)npix * 4;
+    const size_t gbytes = (size_t)n_views * 12 * sizeof(float), ibytes = (size_t)npix * 4;
     if (overlaps(grad_Rt, gbytes, grad_out, ibytes) || overlaps(grad_Rt, gbytes, Rt, gbytes) ||
         (mode != DRR_MODE_RAW && overlaps(grad_Rt, gbytes, fwd_out, ibytes)))
         return fail(DRR_ERR_INVALID_ARG, "grad_Rt overlaps another buffer");
     drr::Geom g;
-    drr::fill_geom(g, dims, spacing, origin, K, B, H, W, n_samples, density_factor, layout);
-    return cuda_status(drr::launch_pose_grad(vol, dtype, layout, g, Rt, mode, grad_out, fwd_out,
+    drr::fill_geom(g, dims, spacing, origin, K, images, H, W, n_samples, density_factor, layout);
+    g.C = channels;
+    g.views_per_vol = per_vol;
+    g.broadcast = bcast;
+    g.vstride = stored_elements(dims, layout);
+    return cuda_status(drr::launch_pose_grad(vols, dtype, layout, g, Rt, mode, grad_out, fwd_out,
                                              grad_Rt, static_cast<cudaStream_t>(stream)),
                        "drr_render_pose_grad launch");
 }
-
-}  // extern "C"
-
-extern "C" {
-
-}  // extern "C"
-
-namespace {
-
-drr_status batch_shape(int n_vols, int channels, int n_views, int* n_out, int* per_vol,
-                       int* broadcast);
 
 drr_status render_alpha_adjoint(const void* vol, drr_dtype dtype, drr_layout layout,
                                 const int dims[3], const float spacing[3], const float origin[3],
@@ -405,6 +336,195 @@ drr_status render_alpha_adjoint(const void* vol, drr_dtype dtype, drr_layout lay
 }  // namespace
 
 extern "C" {
+
+DRR_API int drr_abi_version(void) { return 1; }
+
+DRR_API const char* drr_get_last_error(void) { return g_last_error; }
+
+DRR_API size_t drr_prepared_bytes(const int dims[3], drr_dtype dtype, drr_layout layout) {
+    if (!dims) return 0;
+    for (int a = 0; a < 3; ++a)
+        if (dims[a] < 2 || dims[a] > kMaxDim) return 0;
+    if (dtype != DRR_F32 && dtype != DRR_BF16) return 0;
+    if (!known_layout(layout)) return 0;
+    const int64_t n = stored_elements(dims, layout);
+    if (n > kMaxElements) return 0;
+    return (size_t)n * (dtype == DRR_F32 ? 4 : 2);
+}
+
+DRR_API drr_status drr_prepare_volume(const float* src, const int dims[3], drr_dtype dtype,
+                                      drr_layout layout, void* dst, size_t dst_bytes,
+                                      void* stream) {
+    if (!dims) return fail(DRR_ERR_INVALID_ARG, "dims must be non-NULL");
+    for (int a = 0; a < 3; ++a)
+        if (dims[a] < 2 || dims[a] > kMaxDim)
+            return fail(DRR_ERR_INVALID_ARG, "dims[%d] = %d must be in [2, %d]", a, dims[a], kMaxDim);
+    if (dtype != DRR_F32 && dtype != DRR_BF16) return fail(DRR_ERR_INVALID_ARG, "unknown dtype %d", dtype);
+    if (!known_layout(layout)) return fail(DRR_ERR_INVALID_ARG, "unknown layout %d", layout);
+    const size_t need = drr_prepared_bytes(dims, dtype, layout);
+    if (need == 0) return fail(DRR_ERR_UNSUPPORTED, "volume too large (max 2^31 - 1 stored elements)");
+    if (!src || !dst) return fail(DRR_ERR_INVALID_ARG, "src and dst must be non-NULL");
+    if (!aligned(src, 4) || !aligned(dst, layout_alignment(layout, DRR_F32)))
+        return fail(DRR_ERR_INVALID_ARG, "src must be 4-byte aligned, dst 4-byte (16-byte for DRR_LAYOUT_CORNERS and DRR_LAYOUT_QUADS)");
+    if (dst_bytes < need)
+        return fail(DRR_ERR_INVALID_ARG, "dst holds %zu bytes, %zu needed", dst_bytes, need);
+    const size_t src_bytes = (size_t)dims[0] * dims[1] * dims[2] * 4;
+    if (overlaps(src, src_bytes, dst, need)) return fail(DRR_ERR_INVALID_ARG, "src and dst overlap");
+    return cuda_status(drr::launch_prepare(src, dims[0], dims[1], dims[2], dtype, layout, dst,
+                                           static_cast<cudaStream_t>(stream)),
+                       "drr_prepare_volume launch");
+}
+
+DRR_API drr_status drr_render(const void* vol, drr_dtype dtype, drr_layout layout,
+                              const int dims[3], const float spacing[3], const float origin[3],
+                              const float K[9], const float* Rt, int B, int H, int W,
+                              int n_samples, float density_factor, drr_mode mode, float* out,
+                              void* stream) {
+    return render_batched(vol, dtype, layout, dims, spacing, origin, K, Rt, 1, 1, B, H, W,
+                          n_samples, density_factor, mode, out, stream);
+}
+
+DRR_API drr_status drr_render_batched(const void* vols, drr_dtype dtype, drr_layout layout,
+                                      const int dims[3], const float spacing[3],
+                                      const float origin[3], const float K[9], const float* Rt,
+                                      int n_vols, int channels, int n_views, int H, int W,
+                                      int n_samples, float density_factor, drr_mode mode,
+                                      float* out, void* stream) {
+    return render_batched(vols, dtype, layout, dims, spacing, origin, K, Rt, n_vols, channels,
+                          n_views, H, W, n_samples, density_factor, mode, out, stream);
+}
+
+DRR_API drr_status drr_render_adjoint(const int dims[3], const float spacing[3],
+                                      const float origin[3], const float K[9], const float* Rt,
+                                      int B, int H, int W, int n_samples, float density_factor,
+                                      drr_mode mode, const float* grad_out, const float* fwd_out,
+                                      float* grad_vol, void* stream) {
+    return render_adjoint_batched(dims, spacing, origin, K, Rt, 1, 1, B, H, W, n_samples,
+                                  density_factor, mode, grad_out, fwd_out, grad_vol, false,
+                                  nullptr, 0, stream);
+}
+
+DRR_API size_t drr_adjoint_workspace_bytes(const int dims[3], int B) {
+    if (!dims || B < 0 || B > kMaxViews) return 0;
+    for (int a = 0; a < 3; ++a)
+        if (dims[a] < 2 || dims[a] > kMaxDim) return 0;
+    if (stored_elements(dims, DRR_LAYOUT_LINEAR) > kMaxElements) return 0;
+    return drr::adjoint_workspace_bytes(dims[0], dims[1], dims[2], B);
+}
+
+DRR_API drr_status drr_render_adjoint_ws(const int dims[3], const float spacing[3],
+                                         const float origin[3], const float K[9], const float* Rt,
+                                         int B, int H, int W, int n_samples, float density_factor,
+                                         drr_mode mode, const float* grad_out, const float* fwd_out,
+                                         float* grad_vol, void* workspace, size_t workspace_bytes,
+                                         void* stream) {
+    return render_adjoint_batched(dims, spacing, origin, K, Rt, 1, 1, B, H, W, n_samples,
+                                  density_factor, mode, grad_out, fwd_out, grad_vol, true,
+                                  workspace, workspace_bytes, stream);
+}
+
+// Adjoint for callers that may not allocate device memory (see include/drr.h):
+// the workspace of drr_render_adjoint_ws comes from the library's built-in
+// scratch instead of the caller.  No allocation happens here or below.
+DRR_API drr_status drr_render_adjoint_noalloc(const int dims[3], const float spacing[3],
+                                              const float origin[3], const float K[9],
+                                              const float* Rt, int B, int H, int W,
+                                              int n_samples, float density_factor, drr_mode mode,
+                                              const float* grad_out, const float* fwd_out,
+                                              float* grad_vol, void* stream) {
+    drr_status st = check_volume(dims, spacing, origin);
+    if (st != DRR_OK) return st;
+    st = check_rays(K, Rt, B, H, W, n_samples, density_factor, mode);
+    if (st != DRR_OK) return st;
+    if (stored_elements(dims, DRR_LAYOUT_LINEAR) > kMaxElements)
+        return fail(DRR_ERR_UNSUPPORTED, "volume too large (max 2^31 - 1 elements)");
+    const size_t need = drr::adjoint_workspace_bytes(dims[0], dims[1], dims[2], B);
+    if (need > drr::kNoAllocScratchBytes)
+        return fail(DRR_ERR_UNSUPPORTED,
+                    "this volume and view count need %zu bytes of scratch; the built-in scratch "
+                    "holds %zu (use drr_render_adjoint_ws with a workspace of your own)",
+                    need, drr::kNoAllocScratchBytes);
+    const int64_t npix = (int64_t)B * H * W;
+    if (npix == 0) return ok();
+    if (!grad_out || !aligned(grad_out, 4))
+        return fail(DRR_ERR_INVALID_ARG, "grad_out must be a non-NULL, 4-byte aligned device pointer");
+    if (mode == DRR_MODE_BEER_LAMBERT && (!fwd_out || !aligned(fwd_out, 4)))
+        return fail(DRR_ERR_INVALID_ARG, "fwd_out is required in Beer-Lambert mode");
+    if (!grad_vol || !aligned(grad_vol, 4))
+        return fail(DRR_ERR_INVALID_ARG, "grad_vol must be a non-NULL, 4-byte aligned device pointer");
+    const size_t vbytes = (size_t)dims[0] * dims[1] * dims[2] * 4, ibytes = (size_t)npix * 4;
+    if (overlaps(grad_vol, vbytes, grad_out, ibytes) ||
+        (mode == DRR_MODE_BEER_LAMBERT && overlaps(grad_vol, vbytes, fwd_out, ibytes)))
+        return fail(DRR_ERR_INVALID_ARG, "grad_vol overlaps an image buffer");
+    drr::Geom g;
+    drr::fill_geom(g, dims, spacing, origin, K, B, H, W, n_samples, density_factor, DRR_LAYOUT_LINEAR);
+    return cuda_status(drr::launch_adjoint_noalloc(g, Rt, mode, grad_out, fwd_out, grad_vol,
+                                                   static_cast<cudaStream_t>(stream)),
+                       "drr_render_adjoint_noalloc");
+}
+
+DRR_API drr_status drr_render_adjoint_batched(const int dims[3], const float spacing[3],
+                                              const float origin[3], const float K[9],
+                                              const float* Rt, int n_vols, int channels,
+                                              int n_views, int H, int W, int n_samples,
+                                              float density_factor, drr_mode mode,
+                                              const float* grad_out, const float* fwd_out,
+                                              float* grad_vols, void* stream) {
+    return render_adjoint_batched(dims, spacing, origin, K, Rt, n_vols, channels, n_views, H, W,
+                                  n_samples, density_factor, mode, grad_out, fwd_out, grad_vols,
+                                  false, nullptr, 0, stream);
+}
+
+DRR_API size_t drr_adjoint_batched_workspace_bytes(const int dims[3], int n_vols, int channels,
+                                                   int n_views) {
+    if (!dims) return 0;
+    for (int a = 0; a < 3; ++a)
+        if (dims[a] < 2 || dims[a] > kMaxDim) return 0;
+    if (stored_elements(dims, DRR_LAYOUT_LINEAR) > kMaxElements) return 0;
+    if (n_vols < 1 || channels < 1 || n_views < 1) return 0;
+    if (!(n_views == 1 || n_views % n_vols == 0)) return 0;
+    const int64_t n_out = n_views == 1 ? n_vols : n_views;
+    if (n_out * channels > kMaxViews) return 0;
+    return drr::adjoint_workspace_bytes(dims[0], dims[1], dims[2], (int)(n_out * channels),
+                                        n_vols * channels);
+}
+
+DRR_API drr_status drr_render_adjoint_batched_ws(const int dims[3], const float spacing[3],
+                                                 const float origin[3], const float K[9],
+                                                 const float* Rt, int n_vols, int channels,
+                                                 int n_views, int H, int W, int n_samples,
+                                                 float density_factor, drr_mode mode,
+                                                 const float* grad_out, const float* fwd_out,
+                                                 float* grad_vols, void* workspace,
+                                                 size_t workspace_bytes, void* stream) {
+    return render_adjoint_batched(dims, spacing, origin, K, Rt, n_vols, channels, n_views, H, W,
+                                  n_samples, density_factor, mode, grad_out, fwd_out, grad_vols,
+                                  true, workspace, workspace_bytes, stream);
+}
+
+DRR_API drr_status drr_render_pose_grad(const void* vol, drr_dtype dtype, drr_layout layout,
+                                        const int dims[3], const float spacing[3],
+                                        const float origin[3], const float K[9], const float* Rt,
+                                        int B, int H, int W, int n_samples, float density_factor,
+                                        drr_mode mode, const float* grad_out, const float* fwd_out,
+                                        float* grad_Rt, void* stream) {
+    return pose_grad_batched(vol, dtype, layout, dims, spacing, origin, K, Rt, 1, 1, B, H, W,
+                             n_samples, density_factor, mode, grad_out, fwd_out, grad_Rt, stream);
+}
+
+DRR_API drr_status drr_render_pose_grad_batched(const void* vols, drr_dtype dtype,
+                                                drr_layout layout, const int dims[3],
+                                                const float spacing[3], const float origin[3],
+                                                const float K[9], const float* Rt, int n_vols,
+                                                int channels, int n_views, int H, int W,
+                                                int n_samples, float density_factor,
+                                                drr_mode mode, const float* grad_out,
+                                                const float* fwd_out, float* grad_Rt,
+                                                void* stream) {
+    return pose_grad_batched(vols, dtype, layout, dims, spacing, origin, K, Rt, n_vols, channels,
+                             n_views, H, W, n_samples, density_factor, mode, grad_out, fwd_out,
+                             grad_Rt, stream);
+}
 
 DRR_API drr_status drr_render_alpha_adjoint(const void* vol, drr_dtype dtype, drr_layout layout,
                                             const int dims[3], const float spacing[3],
@@ -480,10 +600,6 @@ DRR_API drr_status drr_poisson_noise_backward(const float* image, const float* z
                        "drr_poisson_noise_backward launch");
 }
 
-}  // extern "C"
-
-extern "C" {
-
 DRR_API drr_status drr_render_siddon(const void* vol, drr_dtype dtype, const int dims[3],
                                      const float spacing[3], const float origin[3],
                                      const float K[9], const float* Rt, int B, int H, int W,
@@ -539,228 +655,6 @@ DRR_API drr_status drr_render_siddon_adjoint(const int dims[3], const float spac
     return cuda_status(drr::launch_siddon_adjoint(g, Rt, mode, grad_out, fwd_out, grad_vol,
                                                   static_cast<cudaStream_t>(stream)),
                        "drr_render_siddon_adjoint launch");
-}
-
-}  // extern "C"
-
-namespace {
-
-// The batch rule of VolumeRaycaster.forward: n_views view matrices for
-// n_vols volumes of `channels` channels; n_views == 1 is broadcast to every
-// volume, else n_views must be a multiple of n_vols (views_per_vol of them
-// per volume, consecutive).  Output images: n_out x channels.
-drr_status batch_shape(int n_vols, int channels, int n_views, int* n_out, int* per_vol,
-                       int* broadcast) {
-    if (n_vols < 0 || channels < 0 || n_views < 0)
-        return fail(DRR_ERR_INVALID_ARG, "n_vols, channels and n_views must be >= 0");
-    if (n_vols == 0 || channels == 0 || n_views == 0) {
-        *n_out = 0;
-        *per_vol = 1;
-        *broadcast = 0;
-        return DRR_OK;
-    }
-    if (n_views == 1 && n_vols > 1) {
-        *n_out = n_vols;
-        *per_vol = 1;
-        *broadcast = 1;
-    } else if (n_views % n_vols == 0) {
-        *n_out = n_views;
-        *per_vol = n_views / n_vols;
-        *broadcast = 0;
-    } else {
-        return fail(DRR_ERR_INVALID_ARG,
-                    "n_views = %d must be 1 or a multiple of n_vols = %d", n_views, n_vols);
-    }
-    if ((int64_t)*n_out * channels > kMaxViews)
-        return fail(DRR_ERR_UNSUPPORTED, "n_out * channels = %lld exceeds %d images per call",
-                    (long long)*n_out * channels, kMaxViews);
-    return DRR_OK;
-}
-
-}  // namespace
-
-extern "C" {
-
-DRR_API drr_status drr_render_batched(const void* vols, drr_dtype dtype, drr_layout layout,
-                                      const int dims[3], const float spacing[3],
-                                      const float origin[3], const float K[9], const float* Rt,
-                                      int n_vols, int channels, int n_views, int H, int W,
-                                      int n_samples, float density_factor, drr_mode mode,
-                                      float* out, void* stream) {
-    int n_out = 0, per_vol = 1, bcast = 0;
-    drr_status st = batch_shape(n_vols, channels, n_views, &n_out, &per_vol, &bcast);
-    if (st != DRR_OK) return st;
-    st = check_volume(dims, spacing, origin);
-    if (st != DRR_OK) return st;
-    const int images = n_out * channels;
-    st = check_rays(K, Rt, images, H, W, n_samples, density_factor, mode, true);
-    if (st != DRR_OK) return st;
-    if (dtype != DRR_F32 && dtype != DRR_BF16) return fail(DRR_ERR_INVALID_ARG, "unknown dtype %d", dtype);
-    if (!known_layout(layout)) return fail(DRR_ERR_INVALID_ARG, "unknown layout %d", layout);
-    if (stored_elements(dims, layout) > kMaxElements)
-        return fail(DRR_ERR_UNSUPPORTED, "volume too large (max 2^31 - 1 stored elements)");
-    if ((int64_t)images * H * W == 0) return ok();
-    if (!vols || !aligned(vols, layout_alignment(layout, dtype)))
-        return fail(DRR_ERR_INVALID_ARG, "vols must be a non-NULL device pointer aligned to %zu bytes",
-                    layout_alignment(layout, dtype));
-    if (!out || !aligned(out, 4)) return fail(DRR_ERR_INVALID_ARG, "out must be a non-NULL, 4-byte aligned device pointer");
-    drr::Geom g;
-    drr::fill_geom(g, dims, spacing, origin, K, images, H, W, n_samples, density_factor, layout);
-    g.C = channels;
-    g.views_per_vol = per_vol;
-    g.broadcast = bcast;
-    g.vstride = stored_elements(dims, layout);
-    return cuda_status(drr::launch_forward(vols, dtype, layout, g, Rt, mode, out,
-                                           static_cast<cudaStream_t>(stream)),
-                       "drr_render_batched launch");
-}
-
-DRR_API drr_status drr_render_pose_grad_batched(const void* vols, drr_dtype dtype,
-                                                drr_layout layout, const int dims[3],
-                                                const float spacing[3], const float origin[3],
-                                                const float K[9], const float* Rt, int n_vols,
-                                                int channels, int n_views, int H, int W,
-                                                int n_samples, float density_factor,
-                                                drr_mode mode, const float* grad_out,
-                                                const float* fwd_out, float* grad_Rt,
-                                                void* stream) {
-    int n_out = 0, per_vol = 1, bcast = 0;
-    drr_status st = batch_shape(n_vols, channels, n_views, &n_out, &per_vol, &bcast);
-    if (st != DRR_OK) return st;
-    st = check_volume(dims, spacing, origin);
-    if (st != DRR_OK) return st;
-    const int images = n_out * channels;
-    st = check_rays(K, Rt, images, H, W, n_samples, density_factor, mode, true);
-    if (st != DRR_OK) return st;
-    if (dtype != DRR_F32 && dtype != DRR_BF16) return fail(DRR_ERR_INVALID_ARG, "unknown dtype %d", dtype);
-    if (!known_layout(layout)) return fail(DRR_ERR_INVALID_ARG, "unknown layout %d", layout);
-    if (stored_elements(dims, layout) > kMaxElements)
-        return fail(DRR_ERR_UNSUPPORTED, "volume too large (max 2^31 - 1 stored elements)");
-    const int64_t npix = (int64_t)images * H * W;
-    if (npix == 0) return ok();
-    if (!vols || !aligned(vols, layout_alignment(layout, dtype)))
-        return fail(DRR_ERR_INVALID_ARG, "vols must be a non-NULL device pointer aligned to %zu bytes",
-                    layout_alignment(layout, dtype));
-    if (!grad_out || !aligned(grad_out, 4))
-        return fail(DRR_ERR_INVALID_ARG, "grad_out must be a non-NULL, 4-byte aligned device pointer");
-    if (mode != DRR_MODE_RAW && (!fwd_out || !aligned(fwd_out, 4)))
-        return fail(DRR_ERR_INVALID_ARG, "fwd_out is required in Beer-Lambert and alpha mode");
-    if (!grad_Rt || !aligned(grad_Rt, 4))
-        return fail(DRR_ERR_INVALID_ARG, "grad_Rt must be a non-NULL, 4-byte aligned device pointer");
-    const size_t gbytes = (size_t)n_views * 12 * sizeof(float), ibytes = (size_t)npix * 4;
-    if (overlaps(grad_Rt, gbytes, grad_out, ibytes) || overlaps(grad_Rt, gbytes, Rt, gbytes) ||
-        (mode != DRR_MODE_RAW && overlaps(grad_Rt, gbytes, fwd_out, ibytes)))
-        return fail(DRR_ERR_INVALID_ARG, "grad_Rt overlaps another buffer");
-    drr::Geom g;
-    drr::fill_geom(g, dims, spacing, origin, K, images, H, W, n_samples, density_factor, layout);
-    g.C = channels;
-    g.views_per_vol = per_vol;
-    g.broadcast = bcast;
-    g.vstride = stored_elements(dims, layout);
-    return cuda_status(drr::launch_pose_grad(vols, dtype, layout, g, Rt, mode, grad_out, fwd_out,
-                                             grad_Rt, static_cast<cudaStream_t>(stream)),
-                       "drr_render_pose_grad_batched launch");
-}
-
-}  // extern "C"
-
-namespace {
-
-drr_status render_adjoint_batched(const int dims[3], const float spacing[3], const float origin[3],
-                                  const float K[9], const float* Rt, int n_vols, int channels,
-                                  int n_views, int H, int W, int n_samples, float density_factor,
-                                  drr_mode mode, const float* grad_out, const float* fwd_out,
-                                  float* grad_vols, bool with_ws, void* workspace,
-                                  size_t workspace_bytes, void* stream) {
-    int n_out = 0, per_vol = 1, bcast = 0;
-    drr_status st = batch_shape(n_vols, channels, n_views, &n_out, &per_vol, &bcast);
-    if (st != DRR_OK) return st;
-    st = check_volume(dims, spacing, origin);
-    if (st != DRR_OK) return st;
-    const int images = n_out * channels;
-    st = check_rays(K, Rt, images, H, W, n_samples, density_factor, mode);
-    if (st != DRR_OK) return st;
-    if (stored_elements(dims, DRR_LAYOUT_LINEAR) > kMaxElements)
-        return fail(DRR_ERR_UNSUPPORTED, "volume too large (max 2^31 - 1 elements)");
-    const int64_t npix = (int64_t)images * H * W;
-    if (npix == 0) return ok();
-    if (!grad_out || !aligned(grad_out, 4))
-        return fail(DRR_ERR_INVALID_ARG, "grad_out must be a non-NULL, 4-byte aligned device pointer");
-    if (mode == DRR_MODE_BEER_LAMBERT && (!fwd_out || !aligned(fwd_out, 4)))
-        return fail(DRR_ERR_INVALID_ARG, "fwd_out is required in Beer-Lambert mode");
-    if (!grad_vols || !aligned(grad_vols, 4))
-        return fail(DRR_ERR_INVALID_ARG, "grad_vols must be a non-NULL, 4-byte aligned device pointer");
-    const int64_t nvox = (int64_t)dims[0] * dims[1] * dims[2];
-    const size_t vbytes = (size_t)nvox * n_vols * channels * 4, ibytes = (size_t)npix * 4;
-    if (overlaps(grad_vols, vbytes, grad_out, ibytes) ||
-        (mode == DRR_MODE_BEER_LAMBERT && overlaps(grad_vols, vbytes, fwd_out, ibytes)))
-        return fail(DRR_ERR_INVALID_ARG, "grad_vols overlaps an image buffer");
-    if (with_ws) {
-        const size_t need =
-            drr::adjoint_workspace_bytes(dims[0], dims[1], dims[2], images, n_vols * channels);
-        if (!workspace || !aligned(workspace, 256))
-            return fail(DRR_ERR_INVALID_ARG, "workspace must be a non-NULL, 256-byte aligned device pointer");
-        if (workspace_bytes < need)
-            return fail(DRR_ERR_INVALID_ARG, "workspace holds %zu bytes, %zu needed", workspace_bytes, need);
-        if (overlaps(workspace, need, grad_vols, vbytes) || overlaps(workspace, need, grad_out, ibytes) ||
-            (mode == DRR_MODE_BEER_LAMBERT && overlaps(workspace, need, fwd_out, ibytes)) ||
-            overlaps(workspace, need, Rt, (size_t)n_views * 12 * sizeof(float)))
-            return fail(DRR_ERR_INVALID_ARG, "workspace overlaps another buffer");
-    }
-    drr::Geom g;
-    drr::fill_geom(g, dims, spacing, origin, K, images, H, W, n_samples, density_factor,
-                   DRR_LAYOUT_LINEAR);
-    g.C = channels;
-    g.views_per_vol = per_vol;
-    g.broadcast = bcast;
-    g.vstride = nvox;
-    return cuda_status(drr::launch_adjoint(g, Rt, mode, grad_out, fwd_out, grad_vols,
-                                           with_ws ? workspace : nullptr,
-                                           static_cast<cudaStream_t>(stream)),
-                       "drr_render_adjoint_batched launch");
-}
-
-}  // namespace
-
-extern "C" {
-
-DRR_API drr_status drr_render_adjoint_batched(const int dims[3], const float spacing[3],
-                                              const float origin[3], const float K[9],
-                                              const float* Rt, int n_vols, int channels,
-                                              int n_views, int H, int W, int n_samples,
-                                              float density_factor, drr_mode mode,
-                                              const float* grad_out, const float* fwd_out,
-                                              float* grad_vols, void* stream) {
-    return render_adjoint_batched(dims, spacing, origin, K, Rt, n_vols, channels, n_views, H, W,
-                                  n_samples, density_factor, mode, grad_out, fwd_out, grad_vols,
-                                  false, nullptr, 0, stream);
-}
-
-DRR_API size_t drr_adjoint_batched_workspace_bytes(const int dims[3], int n_vols, int channels,
-                                                   int n_views) {
-    if (!dims) return 0;
-    for (int a = 0; a < 3; ++a)
-        if (dims[a] < 2 || dims[a] > kMaxDim) return 0;
-    if (stored_elements(dims, DRR_LAYOUT_LINEAR) > kMaxElements) return 0;
-    if (n_vols < 1 || channels < 1 || n_views < 1) return 0;
-    if (!(n_views == 1 || n_views % n_vols == 0)) return 0;
-    const int64_t n_out = n_views == 1 ? n_vols : n_views;
-    if (n_out * channels > kMaxViews) return 0;
-    return drr::adjoint_workspace_bytes(dims[0], dims[1], dims[2], (int)(n_out * channels),
-                                        n_vols * channels);
-}
-
-DRR_API drr_status drr_render_adjoint_batched_ws(const int dims[3], const float spacing[3],
-                                                 const float origin[3], const float K[9],
-                                                 const float* Rt, int n_vols, int channels,
-                                                 int n_views, int H, int W, int n_samples,
-                                                 float density_factor, drr_mode mode,
-                                                 const float* grad_out, const float* fwd_out,
-                                                 float* grad_vols, void* workspace,
-                                                 size_t workspace_bytes, void* stream) {
-    return render_adjoint_batched(dims, spacing, origin, K, Rt, n_vols, channels, n_views, H, W,
-                                  n_samples, density_factor, mode, grad_out, fwd_out, grad_vols,
-                                  true, workspace, workspace_bytes, stream);
 }
 
 }  // extern "C"
