@@ -248,6 +248,40 @@ def l2_read_peak_gbs(torch, nbytes):
     return best
 
 
+def l2_red_probe(torch, nbytes):
+    """The L2's fp32 reduction throughput over a buffer of ``nbytes`` (the
+    gradient volume's size), for each pattern of libdrr_probe.so's
+    drr_probe_l2_red: best of 4 launches of ~2 G values each.  Returns
+    {pattern: {"gvalues_s", "gsector_ops_s"}} or None."""
+    import ctypes
+    lib = ctypes.CDLL(os.path.join(ROOT, "cone_beam_ct_b200", "libdrr_probe.so"))
+    lib.drr_probe_l2_red.argtypes = [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int,
+                                     ctypes.c_int, ctypes.c_void_p]
+    lib.drr_probe_l2_red.restype = ctypes.c_int
+    n = max(8, (nbytes // 4) // 8 * 8)
+    buf = torch.zeros(n, dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream()
+    res = {}
+    # kind: (name, values per pass, sector operations per pass)
+    kinds = {0: ("scalar, 8 values per sector op", n, n // 8),
+             1: ("16-byte vector, 4 values per sector op", n, n // 4),
+             2: ("scalar, 1 value per sector op", n // 8, n // 8)}
+    for kind, (name, values, ops) in kinds.items():
+        reps = max(1, 2_000_000_000 // values)
+        best = 0.0
+        for _ in range(4):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            rc = lib.drr_probe_l2_red(buf.data_ptr(), n, reps, kind, stream.cuda_stream)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            if rc != 0:
+                return None
+            best = max(best, reps / (e0.elapsed_time(e1) * 1e-3))
+        res[name] = {"gvalues_s": best * values / 1e9, "gsector_ops_s": best * ops / 1e9}
+    return res
+
+
 def code_digest(paths):
     """First 16 hex digits of the SHA-256 of the sources' code: comments
     removed and whitespace collapsed, so that a comment edit does not count as
@@ -283,6 +317,11 @@ def traffic_for(kernel, workload_name, layout_name):
 
 # ---------------------------------------------------------------------------
 # the reference arm: the fp64 CPU oracle, timed on the host cores
+
+# the volume adjoint's launches, timed as one group; the record kernel (dense
+# views) dominates it
+ADJOINT_GROUP = ("volume adjoint: plan_views + zero_records + adjoint_kernel + records_kernel "
+                 "+ gather_records (records_kernel dominant)")
 
 REF_SAMPLES_PER_STEP = 4_000_000      # ray-samples per reference-arm step (~0.6 s of fp64 CPU)
 BASELINE_SAMPLES = 100_000_000        # ray-samples of the cpu_baseline sample (~15 s)
@@ -828,7 +867,15 @@ def run_ours(args):
 
     wname = config_block(w, args.config, "")["workload"]
     fwd_roof = roof("forward_kernel", fwd_ms, fwd_bytes, "forward_kernel", wname)
-    adj_roof = roof("adjoint_kernel", adj_ms, adj_bytes, "adjoint_kernel", wname)
+    adj_roof = roof(ADJOINT_GROUP, adj_ms, adj_bytes, "adjoint_kernel", wname)
+    # the ceiling of a scatter: the L2's fp32 reduction rate, measured beside
+    # the read-bandwidth fraction (8 fp32 values added per ray-sample)
+    red = l2_red_probe(torch, nx * ny * nz * 4)
+    if red:
+        best = max(v["gvalues_s"] for v in red.values())
+        adj_roof["red_probe"] = red
+        adj_roof["gvalues_s"] = 8 * samples / (adj_ms * 1e-3) / 1e9
+        adj_roof["frac_of_best_red_values"] = adj_roof["gvalues_s"] / best
     dominant = adj_roof if adj_ms >= fwd_ms else fwd_roof
 
     pose = None

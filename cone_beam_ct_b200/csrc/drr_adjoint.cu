@@ -646,13 +646,22 @@ alpha_records_kernel(const T* __restrict__ vol_base, const float* __restrict__ R
         if (pc[h] >= 0) flush_record(rec, pc[h], p[h]);
 }
 
+}  // namespace
+
+size_t adjoint_workspace_header(int B) {
+    return ((size_t)(1 + B) * sizeof(int) + 255) / 256 * 256;
+}
+
+namespace {
 constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mu;
 void* g_noalloc_addr[kMaxDevices] = {};
+}  // namespace
 
 // Device address of the built-in scratch on the current device, looked up
-// once per device (the first call on a device does it; that call should
-// come before any stream capture).
+// once per device with that device current (the first call on a device does
+// it; that call should come before any stream capture).  The cache holds for
+// the life of the process: a cudaDeviceReset in between leaves it stale.
 cudaError_t noalloc_scratch(void** out) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -667,12 +676,6 @@ cudaError_t noalloc_scratch(void** out) {
     }
     *out = g_noalloc_addr[dev];
     return cudaSuccess;
-}
-
-}  // namespace
-
-size_t adjoint_workspace_header(int B) {
-    return ((size_t)(1 + B) * sizeof(int) + 255) / 256 * 256;
 }
 
 size_t adjoint_workspace_bytes(int nx, int ny, int nz, int B, int slots) {
@@ -764,14 +767,6 @@ cudaError_t launch_alpha_adjoint(const void* vol, int dtype, int layout, const G
         gather_records<<<fill_grid, 256, 0, stream>>>(ws.flags, ws.rec, ws.rec_stride, grad_vol,
                                                       g.nx, g.ny, g.nz, slots);
     return cudaGetLastError();
-}
-
-cudaError_t launch_adjoint_noalloc(const Geom& g, const float* Rt, int mode, const float* grad_out,
-                                   const float* fwd_out, float* grad_vol, cudaStream_t stream) {
-    void* scratch = nullptr;
-    const cudaError_t e = noalloc_scratch(&scratch);
-    if (e != cudaSuccess) return e;
-    return launch_adjoint(g, Rt, mode, grad_out, fwd_out, grad_vol, scratch, stream);
 }
 
 }  // namespace drr

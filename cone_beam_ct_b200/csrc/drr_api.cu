@@ -14,6 +14,9 @@
 #include "../../include/drr.h"
 #include "drr_internal.cuh"
 
+static_assert(DRR_NOALLOC_SCRATCH_BYTES == drr::kNoAllocScratchBytes,
+              "the header's scratch size must be the library's");
+
 namespace {
 
 thread_local char g_last_error[512] = "";
@@ -174,11 +177,16 @@ drr_status render_batched(const void* vols, drr_dtype dtype, drr_layout layout, 
                        "drr_render launch");
 }
 
+// Where the adjoint's workspace comes from: none (every view on the direct
+// path), the caller's buffer, or the library's built-in scratch (the
+// allocation-free entry point).
+enum class Workspace { kNone, kCaller, kBuiltin };
+
 drr_status render_adjoint_batched(const int dims[3], const float spacing[3], const float origin[3],
                                   const float K[9], const float* Rt, int n_vols, int channels,
                                   int n_views, int H, int W, int n_samples, float density_factor,
                                   drr_mode mode, const float* grad_out, const float* fwd_out,
-                                  float* grad_vols, bool with_ws, void* workspace,
+                                  float* grad_vols, Workspace ws_kind, void* workspace,
                                   size_t workspace_bytes, void* stream) {
     int n_out = 0, per_vol = 1, bcast = 0;
     drr_status st = batch_shape(n_vols, channels, n_views, &n_out, &per_vol, &bcast);
@@ -203,9 +211,19 @@ drr_status render_adjoint_batched(const int dims[3], const float spacing[3], con
     if (overlaps(grad_vols, vbytes, grad_out, ibytes) ||
         (mode == DRR_MODE_BEER_LAMBERT && overlaps(grad_vols, vbytes, fwd_out, ibytes)))
         return fail(DRR_ERR_INVALID_ARG, "grad_vols overlaps an image buffer");
-    if (with_ws) {
-        const size_t need =
-            drr::adjoint_workspace_bytes(dims[0], dims[1], dims[2], images, n_vols * channels);
+    const size_t need =
+        drr::adjoint_workspace_bytes(dims[0], dims[1], dims[2], images, n_vols * channels);
+    if (ws_kind == Workspace::kBuiltin) {
+        // checked before the scratch's address is looked up, so that a call
+        // rejected here touches nothing on the device
+        if (need > drr::kNoAllocScratchBytes)
+            return fail(DRR_ERR_UNSUPPORTED,
+                        "this volume and view count need %zu bytes of scratch; the built-in "
+                        "scratch holds %zu (use drr_render_adjoint_ws with a workspace of your own)",
+                        need, drr::kNoAllocScratchBytes);
+        const cudaError_t e = drr::noalloc_scratch(&workspace);
+        if (e != cudaSuccess) return cuda_status(e, "drr_render_adjoint_noalloc scratch lookup");
+    } else if (ws_kind == Workspace::kCaller) {
         if (!workspace || !aligned(workspace, 256))
             return fail(DRR_ERR_INVALID_ARG, "workspace must be a non-NULL, 256-byte aligned device pointer");
         if (workspace_bytes < need)
@@ -223,7 +241,7 @@ drr_status render_adjoint_batched(const int dims[3], const float spacing[3], con
     g.broadcast = bcast;
     g.vstride = nvox;
     return cuda_status(drr::launch_adjoint(g, Rt, mode, grad_out, fwd_out, grad_vols,
-                                           with_ws ? workspace : nullptr,
+                                           ws_kind == Workspace::kNone ? nullptr : workspace,
                                            static_cast<cudaStream_t>(stream)),
                        "drr_render_adjoint_batched launch");
 }
@@ -400,8 +418,8 @@ DRR_API drr_status drr_render_adjoint(const int dims[3], const float spacing[3],
                                       drr_mode mode, const float* grad_out, const float* fwd_out,
                                       float* grad_vol, void* stream) {
     return render_adjoint_batched(dims, spacing, origin, K, Rt, 1, 1, B, H, W, n_samples,
-                                  density_factor, mode, grad_out, fwd_out, grad_vol, false,
-                                  nullptr, 0, stream);
+                                  density_factor, mode, grad_out, fwd_out, grad_vol,
+                                  Workspace::kNone, nullptr, 0, stream);
 }
 
 DRR_API size_t drr_adjoint_workspace_bytes(const int dims[3], int B) {
@@ -419,8 +437,8 @@ DRR_API drr_status drr_render_adjoint_ws(const int dims[3], const float spacing[
                                          float* grad_vol, void* workspace, size_t workspace_bytes,
                                          void* stream) {
     return render_adjoint_batched(dims, spacing, origin, K, Rt, 1, 1, B, H, W, n_samples,
-                                  density_factor, mode, grad_out, fwd_out, grad_vol, true,
-                                  workspace, workspace_bytes, stream);
+                                  density_factor, mode, grad_out, fwd_out, grad_vol,
+                                  Workspace::kCaller, workspace, workspace_bytes, stream);
 }
 
 // Adjoint for callers that may not allocate device memory (see include/drr.h):
@@ -432,35 +450,9 @@ DRR_API drr_status drr_render_adjoint_noalloc(const int dims[3], const float spa
                                               int n_samples, float density_factor, drr_mode mode,
                                               const float* grad_out, const float* fwd_out,
                                               float* grad_vol, void* stream) {
-    drr_status st = check_volume(dims, spacing, origin);
-    if (st != DRR_OK) return st;
-    st = check_rays(K, Rt, B, H, W, n_samples, density_factor, mode);
-    if (st != DRR_OK) return st;
-    if (stored_elements(dims, DRR_LAYOUT_LINEAR) > kMaxElements)
-        return fail(DRR_ERR_UNSUPPORTED, "volume too large (max 2^31 - 1 elements)");
-    const size_t need = drr::adjoint_workspace_bytes(dims[0], dims[1], dims[2], B);
-    if (need > drr::kNoAllocScratchBytes)
-        return fail(DRR_ERR_UNSUPPORTED,
-                    "this volume and view count need %zu bytes of scratch; the built-in scratch "
-                    "holds %zu (use drr_render_adjoint_ws with a workspace of your own)",
-                    need, drr::kNoAllocScratchBytes);
-    const int64_t npix = (int64_t)B * H * W;
-    if (npix == 0) return ok();
-    if (!grad_out || !aligned(grad_out, 4))
-        return fail(DRR_ERR_INVALID_ARG, "grad_out must be a non-NULL, 4-byte aligned device pointer");
-    if (mode == DRR_MODE_BEER_LAMBERT && (!fwd_out || !aligned(fwd_out, 4)))
-        return fail(DRR_ERR_INVALID_ARG, "fwd_out is required in Beer-Lambert mode");
-    if (!grad_vol || !aligned(grad_vol, 4))
-        return fail(DRR_ERR_INVALID_ARG, "grad_vol must be a non-NULL, 4-byte aligned device pointer");
-    const size_t vbytes = (size_t)dims[0] * dims[1] * dims[2] * 4, ibytes = (size_t)npix * 4;
-    if (overlaps(grad_vol, vbytes, grad_out, ibytes) ||
-        (mode == DRR_MODE_BEER_LAMBERT && overlaps(grad_vol, vbytes, fwd_out, ibytes)))
-        return fail(DRR_ERR_INVALID_ARG, "grad_vol overlaps an image buffer");
-    drr::Geom g;
-    drr::fill_geom(g, dims, spacing, origin, K, B, H, W, n_samples, density_factor, DRR_LAYOUT_LINEAR);
-    return cuda_status(drr::launch_adjoint_noalloc(g, Rt, mode, grad_out, fwd_out, grad_vol,
-                                                   static_cast<cudaStream_t>(stream)),
-                       "drr_render_adjoint_noalloc");
+    return render_adjoint_batched(dims, spacing, origin, K, Rt, 1, 1, B, H, W, n_samples,
+                                  density_factor, mode, grad_out, fwd_out, grad_vol,
+                                  Workspace::kBuiltin, nullptr, 0, stream);
 }
 
 DRR_API drr_status drr_render_adjoint_batched(const int dims[3], const float spacing[3],
@@ -472,7 +464,7 @@ DRR_API drr_status drr_render_adjoint_batched(const int dims[3], const float spa
                                               float* grad_vols, void* stream) {
     return render_adjoint_batched(dims, spacing, origin, K, Rt, n_vols, channels, n_views, H, W,
                                   n_samples, density_factor, mode, grad_out, fwd_out, grad_vols,
-                                  false, nullptr, 0, stream);
+                                  Workspace::kNone, nullptr, 0, stream);
 }
 
 DRR_API size_t drr_adjoint_batched_workspace_bytes(const int dims[3], int n_vols, int channels,
@@ -499,7 +491,7 @@ DRR_API drr_status drr_render_adjoint_batched_ws(const int dims[3], const float 
                                                  size_t workspace_bytes, void* stream) {
     return render_adjoint_batched(dims, spacing, origin, K, Rt, n_vols, channels, n_views, H, W,
                                   n_samples, density_factor, mode, grad_out, fwd_out, grad_vols,
-                                  true, workspace, workspace_bytes, stream);
+                                  Workspace::kCaller, workspace, workspace_bytes, stream);
 }
 
 DRR_API drr_status drr_render_pose_grad(const void* vol, drr_dtype dtype, drr_layout layout,

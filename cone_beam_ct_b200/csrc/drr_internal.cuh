@@ -252,8 +252,9 @@ size_t adjoint_workspace_bytes(int nx, int ny, int nz, int B, int slots = 1);
 
 // Size of the built-in scratch of the allocation-free adjoint (32 MiB).
 constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;
-cudaError_t launch_adjoint_noalloc(const Geom& g, const float* Rt, int mode, const float* grad_out,
-                                   const float* fwd_out, float* grad_vol, cudaStream_t stream);
+// Device address of that scratch on the current device (drr_adjoint.cu),
+// looked up once per device and cached for the life of the process.
+cudaError_t noalloc_scratch(void** out);
 cudaError_t launch_prepare(const float* src, int nx, int ny, int nz, int dtype, int layout,
                            void* dst, cudaStream_t stream);
 // workspace: NULL (every view on the direct path) or the layout of

@@ -1,7 +1,8 @@
-// drr_probe.cu -- L2 read-bandwidth probe for the gather roofline
-// (include/drr_probe.h).  Grid-stride float4 loads with the .cg cache
-// operator (cached in L2, not in L1), one persistent wave of CTAs (4 of 512
-// threads per SM).
+// drr_probe.cu -- the benchmark's probes (include/drr_probe.h): the L2 read
+// bandwidth of the gather roofline (grid-stride float4 loads with the .cg
+// cache operator, cached in L2, not in L1; one persistent wave of CTAs, 4 of
+// 512 threads per SM), and the L2's fp32 reduction (RED) throughput beside
+// which the adjoint's scatter is read.
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -32,7 +33,48 @@ __global__ void __launch_bounds__(512) l2_read(const float4* __restrict__ buf, s
     if (acc != acc) *sink = acc;   // never true for finite data
 }
 
+// fp32 reductions over an L2-resident buffer, one persistent wave; every pass
+// adds 1 to each float the pattern touches:
+//   kind 0  scalar, a warp's 32 lanes on 32 consecutive floats (each 32-byte
+//           sector receives one operation carrying 8 values)
+//   kind 1  16-byte vector, each lane on its own 32-byte record, two vector
+//           reductions per record (each sector receives two operations of 4
+//           values: the adjoint's corner-record flush)
+//   kind 2  scalar, each lane on the first float of its own sector (one
+//           operation carrying 1 value per sector: scattered adds)
+__global__ void __launch_bounds__(512) l2_red(float* __restrict__ buf, size_t n, int reps,
+                                              int kind) {
+    const size_t tid = blockIdx.x * (size_t)blockDim.x + threadIdx.x;
+    const size_t stride = (size_t)gridDim.x * blockDim.x;
+    for (int r = 0; r < reps; ++r) {
+        if (kind == 0) {
+            for (size_t m = tid; m < n; m += stride) atomicAdd(buf + m, 1.0f);
+        } else if (kind == 1) {
+            for (size_t m = tid; m < n / 8; m += stride) {
+                float4* p = reinterpret_cast<float4*>(buf + 8 * m);
+                atomicAdd(p, make_float4(1.0f, 1.0f, 1.0f, 1.0f));
+                atomicAdd(p + 1, make_float4(1.0f, 1.0f, 1.0f, 1.0f));
+            }
+        } else {
+            for (size_t m = tid; m < n / 8; m += stride) atomicAdd(buf + 8 * m, 1.0f);
+        }
+    }
+}
+
 }  // namespace
+
+extern "C" DRR_PROBE_API int drr_probe_l2_red(float* buf, size_t n_floats, int reps, int kind,
+                                              void* stream) {
+    if (!buf || n_floats < 8 || (n_floats % 8) != 0 || reps < 1 || kind < 0 || kind > 2 ||
+        (reinterpret_cast<uintptr_t>(buf) % 32) != 0)
+        return -1;
+    int dev = 0, sms = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (sms <= 0) sms = 148;
+    l2_red<<<sms * 4, 512, 0, static_cast<cudaStream_t>(stream)>>>(buf, n_floats, reps, kind);
+    return (int)cudaGetLastError();
+}
 
 extern "C" DRR_PROBE_API int drr_probe_l2_read(const void* buf, size_t n_vec16, int reps,
                                                float* sink, void* stream) {

@@ -210,7 +210,13 @@ DRR_API drr_status drr_render_adjoint_ws(const int dims[3], const float spacing[
  *   - Nothing is allocated: no cudaMalloc, cudaFree or allocating library
  *     call.  The first call on a device looks up the scratch's device
  *     address (once per device, with that device current); make that first
- *     call before any stream capture.
+ *     call before any stream capture.  The address is cached for the life
+ *     of the process: do not call cudaDeviceReset between calls (the cached
+ *     address would be stale).  The scratch used is the one of the device
+ *     current on the calling thread, so that device must be the one that
+ *     owns `stream` and the buffers.
+ *   - Argument checks are those of drr_render_adjoint_ws; a rejected call
+ *     touches nothing on the device.
  *   - All calls share the one scratch array, which keeps the last call's
  *     contents; each call re-initialises what it reads.  Calls that overlap
  *     on the GPU (different streams without ordering, or several host

@@ -49,7 +49,7 @@ def test_probe_library_exports_its_declared_symbol():
     import ctypes
     ctypes.CDLL(PROBE_LIB)
     names = declared_names(PROBE_HEADER, "DRR_PROBE_API")
-    assert names == ["drr_probe_l2_read"]
+    assert names == ["drr_probe_l2_read", "drr_probe_l2_red"]
     assert exported_names(PROBE_LIB) == set(names)
 
 
@@ -178,6 +178,51 @@ def test_workspace_bytes():
     assert drr.drr_adjoint_workspace_bytes((1, 16, 16), 2) == 0
     assert drr.drr_adjoint_workspace_bytes((16, 16, 16), -1) == 0
     _adjoint_ws(B=0, workspace=None, grad_out=None, grad_vol=None, Rt=None)   # empty: no-op
+
+
+def _adjoint_noalloc(**kw):
+    args = dict(dims=DIMS, spacing=SP, origin=ORG, K=K_OK, Rt=FAKE, B=2, H=8, W=8,
+                n_samples=16, density_factor=1.0, mode=drr.DRR_MODE_RAW,
+                grad_out=FAKE + (1 << 20), fwd_out=None, grad_vol=FAKE + (1 << 24), stream=0)
+    args.update(kw)
+    return drr.drr_render_adjoint_noalloc(**args)
+
+
+# every one of these is rejected before the built-in scratch's address is
+# looked up, so nothing touches a device
+NOALLOC_BAD = [
+    (dict(grad_out=0), drr.DRR_ERR_INVALID_ARG, "grad_out"),
+    (dict(grad_vol=FAKE + (1 << 24) + 2), drr.DRR_ERR_INVALID_ARG, "grad_vol"),
+    (dict(mode=drr.DRR_MODE_BEER_LAMBERT, fwd_out=None), drr.DRR_ERR_INVALID_ARG, "fwd_out"),
+    (dict(grad_vol=FAKE + (1 << 20) + 64), drr.DRR_ERR_INVALID_ARG, "overlaps"),
+    (dict(mode=drr.DRR_MODE_BEER_LAMBERT, fwd_out=FAKE + (1 << 24)), drr.DRR_ERR_INVALID_ARG,
+     "overlaps"),
+    (dict(mode=drr.DRR_MODE_ALPHA), drr.DRR_ERR_UNSUPPORTED, "ALPHA"),
+    (dict(n_samples=0), drr.DRR_ERR_INVALID_ARG, "n_samples"),
+    (dict(dims=(1, 16, 16)), drr.DRR_ERR_INVALID_ARG, "dims"),
+    (dict(dims=(128, 128, 128), grad_vol=FAKE + (1 << 32)), drr.DRR_ERR_UNSUPPORTED,
+     "built-in scratch"),
+]
+
+
+@pytest.mark.parametrize("kw,status,word", NOALLOC_BAD)
+def test_noalloc_adjoint_rejects_bad_arguments(kw, status, word):
+    with pytest.raises(drr.DrrError) as e:
+        _adjoint_noalloc(**kw)
+    assert e.value.status == status
+    assert word in drr.drr_get_last_error()
+
+
+def test_noalloc_adjoint_empty_batch_is_a_no_op():
+    _adjoint_noalloc(B=0, grad_out=None, grad_vol=None, Rt=None)
+    assert drr.drr_get_last_error() == ""
+
+
+def test_noalloc_scratch_size_is_the_headers():
+    m = re.search(r"#define\s+DRR_NOALLOC_SCRATCH_BYTES\s+\((\d+)u\s*<<\s*(\d+)\)",
+                  open(HEADER).read())
+    assert m, "DRR_NOALLOC_SCRATCH_BYTES not found in include/drr.h"
+    assert drr.DRR_NOALLOC_SCRATCH_BYTES == int(m.group(1)) << int(m.group(2))
 
 
 def test_raw_adjoint_does_not_need_the_forward_image():

@@ -15,7 +15,8 @@ import pytest
 
 import oracle
 from cone_beam_ct_b200 import workloads as wl
-from tests.gpu_helpers import F32, LINEAR, PADDED, gpu_adjoint, gpu_forward
+from tests.gpu_helpers import (BF16, CORNERS, F32, LINEAR, PADDED, bf16_values, gpu_adjoint,
+                               gpu_forward)
 
 pytestmark = pytest.mark.gpu
 TOL_ADJ, TOL_DOT = 1e-4, 1e-5
@@ -181,3 +182,35 @@ def test_config3_geometry_adjoint(cuda):
     for workspace in (False, True):
         got = gpu_adjoint(w, sparse, mode=wl.MODE_RAW, workspace=workspace)
         assert_adjoint_parity(got, ref, what=f"config 3 sparse upstream, workspace {workspace}")
+
+
+# A contiguous band of full detector rows at the 1024^2 x 512 C-arm geometry:
+# rows 472-567 of every view, so the band covers whole 32-row tiles of the
+# dense-view path and ragged ones at both ends, with every ray of it live.
+BAND_ROWS = slice(472, 568)
+
+
+def dense_band(w, seed):
+    go = np.zeros((w.B, w.H, w.W), np.float32)
+    rng = np.random.default_rng(seed)
+    n = BAND_ROWS.stop - BAND_ROWS.start
+    go[:, BAND_ROWS, :] = rng.standard_normal((w.B, n, w.W)).astype(np.float32)
+    return go
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("mode", [wl.MODE_RAW, wl.MODE_BEER_LAMBERT])
+def test_config3_dense_band_adjoint_as_timed(cuda, mode):
+    # the adjoint the throughput run times: 256^3 volume (bf16 corner records
+    # for the forward), 4 C-arm views of 1024^2, 512 samples, a dense N(0, 1)
+    # upstream gradient, drr_render_adjoint_ws; in Beer-Lambert mode fwd_out
+    # comes from the GPU forward and the oracle recomputes exp(-I) from the
+    # same bf16-rounded volume
+    w = wl.make_config(3)
+    go = dense_band(w, 330 + mode)
+    vb = bf16_values(w.vol)
+    fwd = gpu_forward(w, layout=CORNERS, dtype=BF16, mode=mode) if mode else None
+    ref = oracle.adjoint(w.dims, w.spacing, w.origin, w.K, w.Rt, w.H, w.W, w.n_samples,
+                         w.density_factor, mode, go, vol=vb, nthreads=4)
+    got = gpu_adjoint(w, go, mode=mode, fwd_out=fwd, workspace=True)
+    assert_adjoint_parity(got, ref, what=f"config 3 dense band, mode {mode}")

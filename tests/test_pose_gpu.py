@@ -133,3 +133,25 @@ def test_pose_gradient_config2_full(cuda):
     fwd = gpu_forward(w, layout=CORNERS, dtype=F32, mode=w.mode)
     got = gpu_pose_grad(w, go, layout=CORNERS, dtype=F32, mode=w.mode, fwd_out=fwd)
     assert_pose_parity(got, _oracle(w, go, w.mode, nthreads=8), TOL, what="config 2, 8 views")
+
+
+# 32 contiguous full detector rows of every view at the 1024^2 x 512 C-arm
+# geometry (rows 472-503: two ragged 16-row tiles around a whole one), every
+# ray live, so each CTA's reduction sums full tiles.
+POSE_BAND_ROWS = slice(472, 504)
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("mode", [wl.MODE_BEER_LAMBERT, wl.MODE_ALPHA])
+def test_pose_gradient_config3_dense_band(cuda, mode):
+    w = wl.make_config(3)
+    if mode == wl.MODE_ALPHA:
+        w.density_factor = 10.0
+    go = np.zeros((w.B, w.H, w.W), np.float32)
+    n = POSE_BAND_ROWS.stop - POSE_BAND_ROWS.start
+    go[:, POSE_BAND_ROWS, :] = np.random.default_rng(38 + mode).standard_normal(
+        (w.B, n, w.W)).astype(np.float32)
+    fwd = gpu_forward(w, layout=CORNERS, dtype=BF16, mode=mode)
+    got = gpu_pose_grad(w, go, layout=CORNERS, dtype=BF16, mode=mode, fwd_out=fwd)
+    ref = _oracle(w, go, mode, vol=bf16_values(w.vol), nthreads=4)
+    assert_pose_parity(got, ref, TOL, what=f"config 3 dense band, mode {mode}")

@@ -2,15 +2,23 @@
 may not allocate device memory -- code under a memory manager that owns the
 whole device, or a real-time loop where an allocation could synchronise the
 device.  Its workspace is the library's built-in 32 MiB scratch, shared by
-every call.  It must match the ordinary adjoint (same tolerance as the
-other adjoint tests), call after call: the scratch keeps the previous call's
-contents, so a second call shows that each call re-initialises what it
-reads.  This file is collected last so that a failure here leaves every
-other test already run; it also passes on its own in a fresh process."""
+every call.
+
+Each case runs the call twice in a row (the scratch keeps the previous
+call's contents, so the second call shows that each call re-initialises
+what it reads) and checks both results against the fp64 oracle's adjoint
+and against the ordinary workspace adjoint (drr_render_adjoint_ws), in the
+raw and the Beer-Lambert mode (where fwd_out, from the GPU forward, is
+read).  Tolerance: the other adjoint tests' (normwise max error and relative
+L2 error, each <= 1e-4).  This file is collected last so that a failure here
+leaves every other test already run; it also passes on its own in a fresh
+process."""
 import numpy as np
 import pytest
 
+import oracle
 from cone_beam_ct_b200 import workloads as wl
+from tests.gpu_helpers import F32, PADDED, gpu_forward
 
 pytestmark = pytest.mark.gpu
 TOL_ADJ = 1e-4
@@ -25,25 +33,32 @@ def cuda():
     return torch
 
 
-def _inputs(torch, w, seed):
+def _inputs(torch, w, seed, mode):
     go = np.random.default_rng(seed).standard_normal((w.B, w.H, w.W)).astype(np.float32)
-    return (torch.from_numpy(np.ascontiguousarray(w.Rt.reshape(-1, 12))).cuda(),
-            torch.from_numpy(go).cuda())
+    fwd = gpu_forward(w, layout=PADDED, dtype=F32, mode=mode) if mode else None
+    dev = lambda a: None if a is None else torch.from_numpy(np.ascontiguousarray(a)).cuda()
+    return dev(w.Rt.reshape(-1, 12)), dev(go), dev(fwd), go
 
 
-def _adjoint(torch, w, Rt, go, noalloc):
+def _adjoint(torch, w, Rt, go, fwd, mode, noalloc):
     from cone_beam_ct_b200 import drr
     nx, ny, nz = w.dims
     grad = torch.zeros((nz, ny, nx), dtype=torch.float32, device="cuda")
-    fn = drr.drr_render_adjoint_noalloc if noalloc else drr.drr_render_adjoint
-    fn(w.dims, w.spacing, w.origin, w.K, Rt, w.B, w.H, w.W, w.n_samples, w.density_factor,
-       wl.MODE_RAW, go, None, grad)
+    if noalloc:
+        drr.drr_render_adjoint_noalloc(w.dims, w.spacing, w.origin, w.K, Rt, w.B, w.H, w.W,
+                                       w.n_samples, w.density_factor, mode, go, fwd, grad)
+    else:
+        nbytes = drr.drr_adjoint_workspace_bytes(w.dims, w.B)
+        ws = torch.full((nbytes,), 0x7F, dtype=torch.uint8, device="cuda")
+        drr.drr_render_adjoint_ws(w.dims, w.spacing, w.origin, w.K, Rt, w.B, w.H, w.W,
+                                  w.n_samples, w.density_factor, mode, go, fwd, grad, ws)
     torch.cuda.synchronize()
     return grad.cpu().numpy().astype(np.float64)
 
 
 def _close(got, ref, what):
     scale = np.max(np.abs(ref))
+    assert scale > 0
     norm = np.max(np.abs(got - ref)) / scale
     l2 = np.linalg.norm(got - ref) / np.linalg.norm(ref)
     assert norm <= TOL_ADJ and l2 <= TOL_ADJ, f"{what}: normwise {norm:.3g}, L2 {l2:.3g}"
@@ -59,23 +74,28 @@ CASES = {
 }
 
 
+@pytest.mark.parametrize("mode", [wl.MODE_RAW, wl.MODE_BEER_LAMBERT])
 @pytest.mark.parametrize("name", sorted(CASES))
-def test_noalloc_matches_the_ordinary_adjoint_twice_in_a_row(cuda, name):
+def test_noalloc_matches_the_oracle_and_the_workspace_adjoint_twice_in_a_row(cuda, name, mode):
     from cone_beam_ct_b200 import drr
     w = wl.small_random_case(**CASES[name])
     assert drr.drr_adjoint_workspace_bytes(w.dims, w.B) <= drr.DRR_NOALLOC_SCRATCH_BYTES
-    Rt, go = _inputs(cuda, w, 7)
-    ref = _adjoint(cuda, w, Rt, go, noalloc=False)
-    assert np.max(np.abs(ref)) > 0
+    Rt, go, fwd, go_host = _inputs(cuda, w, 7, mode)
+    ref = oracle.adjoint(w.dims, w.spacing, w.origin, w.K, w.Rt, w.H, w.W, w.n_samples,
+                         w.density_factor, mode, go_host, vol=w.vol, nthreads=8)
+    with_ws = _adjoint(cuda, w, Rt, go, fwd, mode, noalloc=False)
+    _close(with_ws, ref, f"{name}, mode {mode}, workspace adjoint against the oracle")
     for call in (1, 2):
-        _close(_adjoint(cuda, w, Rt, go, noalloc=True), ref, f"{name}, call {call}")
+        got = _adjoint(cuda, w, Rt, go, fwd, mode, noalloc=True)
+        _close(got, ref, f"{name}, mode {mode}, call {call} against the oracle")
+        _close(got, with_ws, f"{name}, mode {mode}, call {call} against the workspace adjoint")
 
 
 def test_noalloc_rejects_volumes_beyond_its_scratch(cuda):
     from cone_beam_ct_b200 import drr
     w = wl.small_random_case(304, dims=(128, 128, 128))
     assert drr.drr_adjoint_workspace_bytes(w.dims, w.B) > drr.DRR_NOALLOC_SCRATCH_BYTES
-    Rt, go = _inputs(cuda, w, 8)
+    Rt, go, _, _ = _inputs(cuda, w, 8, wl.MODE_RAW)
     nx, ny, nz = w.dims
     grad = cuda.zeros((nz, ny, nx), dtype=cuda.float32, device="cuda")
     with pytest.raises(drr.DrrError) as e:
