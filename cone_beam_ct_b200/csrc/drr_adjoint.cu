@@ -40,9 +40,10 @@
 // 16-byte vector atomics -- the L2 executes a vector atomic at the same rate
 // as a scalar one, so this carries 4x the payload per operation, and the
 // bundle flushes once where its rays would have flushed up to six times.  A
-// gather pass then adds each voxel's 8 record entries into the gradient
-// volume.  The alpha gradient and batched calls (records per volume-channel)
-// take the same path.  Sparse views gain nothing from records (measured: the records
+// record sums the moments of its samples (records_kernel); a scatter pass
+// then turns each record into corner weights and adds them to the gradient
+// volume.  The alpha gradient (records of weights, added by a gather pass)
+// and batched calls (records per volume-channel) take the same path.  Sparse views gain nothing from records (measured: the records
 // path ran 12-20 ms against the direct path's 9.3 on the 256^3 / 200^2
 // workload) and keep the direct path above.
 #include <cuda_runtime.h>
@@ -176,6 +177,49 @@ __global__ void zero_records(const int* __restrict__ flags, float4* __restrict__
     for (int64_t m = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; m < n4;
          m += (int64_t)gridDim.x * blockDim.x)
         rec[m] = z;
+}
+
+// Records written as moments (records_kernel) into the gradient volume: each
+// cell's 8 moments become its 8 corner weights (per axis, the pair
+// (sum s g, sum s g f) becomes (sum s g (1 - f), sum s g f); x, then y, then
+// z), which are added to the cell's 8 corner voxels with atomic adds.  A CTA
+// takes whole x rows of cells (one division per row for (j, k) and the
+// volume-channel slot); consecutive threads hold consecutive cells, so each
+// of the 8 adds of a warp covers 32 consecutive voxels (4 or 5 L2 sectors).
+// Zero weights are skipped.
+__device__ __forceinline__ void moments_to_corner_weights(float v[8]) {
+#pragma unroll
+    for (int axis = 0; axis < 3; ++axis) {
+        const int st = 1 << axis;
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+            if ((e & st) == 0) v[e] -= v[e | st];
+    }
+}
+
+__global__ void scatter_records(const int* __restrict__ flags, const float* __restrict__ rec,
+                                long long rec_stride, float* __restrict__ grad, int nx, int ny,
+                                int nz, int slots) {
+    if (flags[0] == 0) return;
+    const int crow = nx - 1, rows = (ny - 1) * (nz - 1);    // cells per row, rows per slot
+    const long long total = (long long)rows * slots;
+    const long long nxy = (long long)nx * ny, nvox = nxy * nz;
+    for (long long row = blockIdx.x; row < total; row += gridDim.x) {
+        const int slot = (int)(row / rows);
+        const int rr = (int)(row - (long long)slot * rows);
+        const int k = rr / (ny - 1), j = rr - k * (ny - 1);
+        const float4* __restrict__ r =
+            reinterpret_cast<const float4*>(rec + slot * rec_stride + (long long)rr * crow * 8);
+        float* __restrict__ gr = grad + slot * nvox + k * nxy + (long long)j * nx;
+        for (int i = threadIdx.x; i < crow; i += blockDim.x) {
+            const float4 lo = __ldcs(r + 2 * i), hi = __ldcs(r + 2 * i + 1);
+            float v[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+            moments_to_corner_weights(v);
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+                if (v[e] != 0.0f) atomicAdd(gr + i + (e & 1) + ((e >> 1) & 1) * nx + (e >> 2) * nxy, v[e]);
+        }
+    }
 }
 
 // grad[k][j][i] += the 8 record entries of voxel (i, j, k): entry a + 2b + 4c of
@@ -321,6 +365,14 @@ adjoint_kernel(const float* __restrict__ Rt, const float* __restrict__ grad_out,
 // the 8 trilinear moments instead of the 8 weights (fewer multiplies per
 // sample, converted at flush) was slower (6.83 ms), and a third, victim slot much
 // slower (8.6 ms, spills; 11.0 ms at 149 registers and 1 CTA per SM).
+//
+// A record accumulates the moments of its samples, not their weights: for a
+// sample with fractions (fx, fy, fz) in its cell and ray scale s, entry
+// a + 2b + 4c adds s fx^a fy^b fz^c.  The 8 trilinear weights are a fixed
+// linear map of these (w_0 = 1 - f, w_1 = f per axis), applied once per
+// record by scatter_records after the scatter, so a sample costs one
+// multiply and three packed fp32x2 multiplies instead of the weights'
+// products.
 constexpr int kBundleX = 3, kBundleY = 2;        // rays per bundle, across and down
 constexpr int kBundleRays = kBundleX * kBundleY;
 constexpr int kSlots = 2;
@@ -395,15 +447,12 @@ records_kernel(const float* __restrict__ Rt, const float* __restrict__ grad_out,
                 const float fx = fix_frac(q[k][0]), fy = fix_frac(q[k][1]), fz = fix_frac(q[k][2]);
 #pragma unroll
                 for (int a = 0; a < 3; ++a) q[k][a] += s[k][a];
-                const float wz1 = scale[k] * fz, wz0 = scale[k] * (1.0f - fz);
-                const float w00 = wz0 * (1.0f - fy), w01 = wz0 * fy;
-                const float w10 = wz1 * (1.0f - fy), w11 = wz1 * fy;
-                // corner pairs (a = 0, 1) as packed fp32x2: 4 FMUL2 and 4 FADD2
-                const float2 fxp = make_float2(1.0f - fx, fx);
-                const float2 w[4] = {__fmul2_rn(make_float2(w00, w00), fxp),
-                                     __fmul2_rn(make_float2(w01, w01), fxp),
-                                     __fmul2_rn(make_float2(w10, w10), fxp),
-                                     __fmul2_rn(make_float2(w11, w11), fxp)};
+                // the sample's 8 moments s fx^a fy^b fz^c, as pairs (a = 0, 1):
+                // one FMUL and three packed FMUL2
+                const float2 mx = make_float2(scale[k], scale[k] * fx);
+                const float2 mxy = __fmul2_rn(mx, make_float2(fy, fy));
+                const float2 w[4] = {mx, mxy, __fmul2_rn(mx, make_float2(fz, fz)),
+                                     __fmul2_rn(mxy, make_float2(fz, fz))};
                 const int home = k / kBundleX;   // upper row -> slot 0, lower row -> slot 1
                 const int other = 1 - home;
                 // two paths, not three: a miss flushes and clears the home
@@ -711,10 +760,9 @@ cudaError_t launch_adjoint(const Geom& g, const float* Rt, int mode, const float
             records_kernel<1><<<rgrid, kThreads, 0, stream>>>(Rt, grad_out, fwd_out, g, ws);
         else
             records_kernel<0><<<rgrid, kThreads, 0, stream>>>(Rt, grad_out, fwd_out, g, ws);
+        scatter_records<<<fill_grid, 256, 0, stream>>>(ws.flags, ws.rec, ws.rec_stride, grad_vol,
+                                                       g.nx, g.ny, g.nz, slots);
     }
-    if (workspace)
-        gather_records<<<fill_grid, 256, 0, stream>>>(ws.flags, ws.rec, ws.rec_stride, grad_vol,
-                                                      g.nx, g.ny, g.nz, slots);
     return cudaGetLastError();
 }
 
