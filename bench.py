@@ -73,6 +73,16 @@ def parse_args():
                         "workload's views split one per volume over as many volumes "
                         "(drr_render_batched, drr_render_adjoint_batched_ws, "
                         "drr_render_pose_grad_batched)")
+    p.add_argument("--no-extras", action="store_true",
+                   help="skip the widened rows the default run also times (pose gradient, alpha "
+                        "compositing, Siddon pair, batches)")
+    p.add_argument("--no-configs", action="store_true",
+                   help="skip the other workloads' forward / adjoint timings (the configs block)")
+    p.add_argument("--partition", choices=["replicas", "views"], default="replicas",
+                   help="replicas (default): every rank runs the whole workload (weak scaling, no "
+                        "collective); views: one job's detector rows split over the ranks, the "
+                        "volume broadcast once, the gradient volume all-reduced every step "
+                        "(strong scaling)")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     return p.parse_args()
@@ -695,6 +705,80 @@ def siddon_timing(torch, w, vol32, Rt, grad_out, l2_peak, hbm_peak):
                         "roofline": roof("siddon_adjoint_kernel", adj_ms)}}
 
 
+# the workloads of the configs block: the other four, config 5 being the
+# adjoint of config 2's geometry (RAW, its own seeded N(0, 1) upstream)
+OTHER_CONFIGS = {3: (1, 2, 4, 5), 1: (2, 3, 4, 5), 2: (1, 3, 4, 5), 4: (1, 2, 3, 5)}
+
+
+def config_timing(torch, cfg, hbm_peak, l2_cache):
+    """Forward and adjoint (with a workspace) of one more workload, each the
+    median of 5 launches with L2 flushed before each, in the layout its
+    forward runs fastest in; Gsamples/s, DRR FPS and the gather-roofline
+    fraction (L2 read probe for a volume that fits in L2, else HBM)."""
+    from cone_beam_ct_b200 import drr
+    from cone_beam_ct_b200 import workloads as wl
+    w = workload(cfg)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    geom_cfg = 2 if cfg == 5 else cfg
+    lname = AUTO_LAYOUT[geom_cfg]
+    layout = {"corners": drr.DRR_LAYOUT_CORNERS, "quads": drr.DRR_LAYOUT_QUADS}[lname]
+    dtype = drr.DRR_BF16 if w.dtype == wl.DTYPE_BF16 else drr.DRR_F32
+    elem = 2 if dtype == drr.DRR_BF16 else 4
+    nx, ny, nz = w.dims
+    vol32 = torch.from_numpy(w.vol).to(dev)
+    Rt = torch.from_numpy(np.ascontiguousarray(w.Rt.reshape(-1, 12))).to(dev)
+    go = torch.from_numpy(w.grad_out).to(dev)
+    pbytes = drr.drr_prepared_bytes(w.dims, dtype, layout)
+    prep = torch.empty(pbytes, dtype=torch.uint8, device=dev)
+    drr.drr_prepare_volume(vol32, w.dims, dtype, layout, prep, pbytes)
+    out = torch.empty((w.B, w.H, w.W), dtype=torch.float32, device=dev)
+    grad = torch.zeros((nz, ny, nx), dtype=torch.float32, device=dev)
+    ws = torch.empty(drr.drr_adjoint_workspace_bytes(w.dims, w.B), dtype=torch.uint8, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    mode = w.mode
+
+    def fwd():
+        drr.drr_render(prep, dtype, layout, w.dims, w.spacing, w.origin, w.K, Rt, w.B, w.H, w.W,
+                       w.n_samples, w.density_factor, mode, out)
+
+    def adj():
+        drr.drr_render_adjoint_ws(w.dims, w.spacing, w.origin, w.K, Rt, w.B, w.H, w.W,
+                                  w.n_samples, w.density_factor, mode, go,
+                                  out if mode == wl.MODE_BEER_LAMBERT else None, grad, ws)
+
+    vol_bytes = nx * ny * nz * elem
+    fits = vol_bytes < L2_BYTES
+    if fits and vol_bytes not in l2_cache:
+        l2_cache[vol_bytes] = l2_read_peak_gbs(torch, vol_bytes)
+    bound, peak = ("l2", l2_cache[vol_bytes]) if fits and l2_cache.get(vol_bytes) else (
+        "hbm", hbm_peak)
+
+    def entry(name, ms, nbytes):
+        a = nbytes / (ms * 1e-3) / 1e9
+        return {"ms": ms, "gsamples_s": w.samples / (ms * 1e-3) / 1e9, "fps": w.B / (ms * 1e-3),
+                "roofline": {"kernel": name, "bound": bound, "achieved": a, "peak": peak,
+                             "unit": "GB/s", "frac": a / peak,
+                             "algorithmic_bytes_per_launch": int(nbytes)}}
+
+    res = {"workload": config_block(w, cfg, lname)["workload"], "layout": lname,
+           "samples": w.samples}
+    fwd()
+    if cfg != 5:
+        res["forward"] = entry("forward_kernel", _median_ms(torch, fwd, reps=5, flush=flush),
+                               8 * elem * w.samples)
+    res["adjoint"] = entry(ADJOINT_GROUP, _median_ms(torch, adj, reps=5, flush=flush),
+                           32 * w.samples)
+    if cfg == 5:
+        res["workload"] = (f"adjoint of the {nx}^3 / {w.B}-view {w.H}x{w.W} / "
+                           f"{w.n_samples}-sample geometry, N(0,1) upstream, RAW")
+    else:
+        step = res["forward"]["ms"] + res["adjoint"]["ms"]
+        res["forward_plus_adjoint"] = {"ms": step, "gsamples_s": w.samples / (step * 1e-3) / 1e9}
+    del prep, ws, grad, out, vol32, flush
+    torch.cuda.empty_cache()
+    return res
+
+
 def run_ours(args):
     import torch
     from cone_beam_ct_b200 import drr
@@ -878,24 +962,31 @@ def run_ours(args):
         adj_roof["frac_of_best_red_values"] = adj_roof["gvalues_s"] / best
     dominant = adj_roof if adj_ms >= fwd_ms else fwd_roof
 
+    extras = not args.no_extras
     pose = None
-    if args.pose:
+    if args.pose or extras:
         pose = pose_timing(torch, w, prep, dtype, layout, Rt, grad_out, out, elem, l2_peak,
                            hbm_peak, vol_fits_l2)
 
     siddon = None
-    if args.siddon:
+    if args.siddon or extras:
         siddon = siddon_timing(torch, w, vol32, Rt, grad_out, l2_peak, hbm_peak)
 
     alpha = None
-    if args.alpha:
+    if args.alpha or extras:
         alpha = alpha_timing(torch, w, vol32, prep, dtype, layout, Rt, grad_out, elem, l2_peak,
                              hbm_peak, vol_fits_l2)
 
     batched = None
-    if args.batched:
+    if args.batched or extras:
         batched = batched_timing(torch, w, vol32, dtype, layout, Rt, grad_out, elem, l2_peak,
                                  hbm_peak, vol_fits_l2)
+
+    configs = None
+    if not args.no_configs:
+        l2_cache = {vol_bytes: l2_peak} if vol_fits_l2 else {}
+        configs = {str(c): config_timing(torch, c, hbm_peak, l2_cache)
+                   for c in OTHER_CONFIGS[args.config]}
 
     tex = None
     if args.texture:
@@ -927,6 +1018,7 @@ def run_ours(args):
         "alpha_compositing": alpha,
         "siddon": siddon,
         "batched": batched,
+        "configs": configs,
         "gpu_launches": 7 * args.steps,   # prepare, forward, plan, zero, 2 adjoint paths, gather
         "clocks": clocks,
         "bracket_ms": bracket[0].elapsed_time(bracket[1]),
@@ -938,12 +1030,108 @@ def run_ours(args):
     return 0
 
 
+def run_partitioned(args):
+    """One job over all ranks (cone_beam_ct_b200.partition): rank r renders
+    and back-projects its share of the detector rows; the volume is broadcast
+    from rank 0 once, before timing; every step ends with one NCCL all-reduce
+    of the fp32 gradient volume.  value = the whole job's ray-samples per
+    second, timed as the max over ranks (strong scaling)."""
+    import datetime
+    import torch
+    import torch.distributed as dist
+    from cone_beam_ct_b200 import drr
+    from cone_beam_ct_b200 import partition as P
+    from cone_beam_ct_b200 import workloads as wl
+
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local if world > 1 else 0)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", torch.cuda.current_device())
+    drr.lib()
+    w = workload(args.config)
+    if args.layout == "auto":
+        args.layout = AUTO_LAYOUT[args.config]
+    layout = {"padded": drr.DRR_LAYOUT_PADDED, "corners": drr.DRR_LAYOUT_CORNERS,
+              "quads": drr.DRR_LAYOUT_QUADS, "linear": drr.DRR_LAYOUT_LINEAR}[args.layout]
+    dtype = drr.DRR_BF16 if w.dtype == wl.DTYPE_BF16 else drr.DRR_F32
+    nx, ny, nz = w.dims
+    part = P.Partition(w.B, w.H, w.W, world, rank)
+    # the volume lives on rank 0 and reaches the others by one broadcast
+    vol32 = (torch.from_numpy(w.vol).to(dev) if rank == 0 else
+             torch.empty((nz, ny, nx), dtype=torch.float32, device=dev))
+    P.broadcast_volume(vol32)
+    Rt = torch.from_numpy(np.ascontiguousarray(w.Rt.reshape(-1, 12))).to(dev)
+    go = torch.from_numpy(np.ascontiguousarray(
+        w.grad_out.reshape(-1)[part.local_slice()])).to(dev)
+    pbytes = drr.drr_prepared_bytes(w.dims, dtype, layout)
+    prep = torch.empty(pbytes, dtype=torch.uint8, device=dev)
+    out = torch.empty(max(1, part.rays), dtype=torch.float32, device=dev)
+    grad = torch.empty((nz, ny, nx), dtype=torch.float32, device=dev)
+    ws = torch.empty(drr.drr_adjoint_workspace_bytes(w.dims, w.B), dtype=torch.uint8,
+                     device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    fwd_needed = w.mode == wl.MODE_BEER_LAMBERT
+
+    def step():
+        drr.drr_prepare_volume(vol32, w.dims, dtype, layout, prep, pbytes, stream=stream)
+        P.render_partitioned(part, prep, dtype, layout, w.dims, w.spacing, w.origin, w.K, Rt,
+                             w.n_samples, w.density_factor, w.mode, out, stream=stream)
+        grad.zero_()
+        P.adjoint_partitioned(part, w.dims, w.spacing, w.origin, w.K, Rt, w.n_samples,
+                              w.density_factor, w.mode, go, out if fwd_needed else None, grad,
+                              workspace=ws, stream=stream)
+
+    for _ in range(max(args.warmup, 3)):
+        flush.fill_(1)
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    total = 0.0
+    with ClockSampler(physical_gpu(dev.index)) as clk:
+        for s in range(args.steps):
+            flush.fill_(s & 0xFF)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            step()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            total += e0.elapsed_time(e1)
+    if world > 1:
+        dist.barrier()
+    total_ms = max_over_ranks([total], dev)[0]
+    launches = 1 + 6 * len(part.segments)      # prepare; per call: forward, plan, zero, 3 adjoint
+    line = {
+        "metric": METRIC, "value": w.samples * args.steps / (total_ms * 1e-3) / 1e9,
+        "unit": "Gsamples/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "strong",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": dict(config_block(w, args.config, args.layout),
+                       parallelism=f"detector rows split over {world} ranks, volume replicated, "
+                                   "gradient all-reduced (NCCL) every step"),
+        "fps": w.B * args.steps / (total_ms * 1e-3),
+        "rows_per_rank": [P.Partition(w.B, w.H, w.W, world, r).rows for r in range(world)],
+        "e2e": None, "cpu_baseline": None, "gpu_launches": launches * args.steps,
+        "clocks": clk.summary(),
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
 def main():
     args = parse_args()
     if args.steps < 1 or args.warmup < 0:
         raise SystemExit("--steps must be >= 1 and --warmup >= 0")
     if args.impl == "reference":
         return run_reference(args)
+    if args.partition == "views":
+        return run_partitioned(args)
     return run_ours(args)
 
 
