@@ -17,6 +17,8 @@ SOURCES = ["drr_api.cu", "drr_forward.cu", "drr_adjoint.cu", "drr_prepare.cu", "
            "drr_siddon.cu"]
 HEADERS = ["drr_internal.cuh", "drr_sample.cuh"]
 PROBE_SOURCES = ["drr_probe.cu"]
+# the same sources with every gather and scatter range-checked (include/drr_debug.h)
+CHECKED_LIB = os.path.join(HERE, "libdrr_checked.so")
 TEXTURE_LIB = os.path.join(HERE, "libdrr_texture.so")
 TEXTURE_SOURCES = ["drr_texture.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -35,12 +37,14 @@ def _stale(lib, sources, headers):
         return True
     t = os.path.getmtime(lib)
     deps = [os.path.join(CSRC, f) for f in sources + headers]
-    deps += [os.path.join(INCLUDE, h) for h in ("drr.h", "drr_probe.h", "drr_texture.h")]
+    deps += [os.path.join(INCLUDE, h)
+             for h in ("drr.h", "drr_debug.h", "drr_probe.h", "drr_texture.h")]
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def _nvcc_shared(lib, sources, verbose_ptxas):
+def _nvcc_shared(lib, sources, verbose_ptxas, defines=()):
     cmd = [_nvcc()] + ARCH + FLAGS + ["-I", INCLUDE, "-o", lib + ".tmp"]
+    cmd += ["-D" + d for d in defines]
     if verbose_ptxas:
         cmd += ["-Xptxas", "-v"]
     cmd += [os.path.join(CSRC, f) for f in sources]
@@ -49,11 +53,14 @@ def _nvcc_shared(lib, sources, verbose_ptxas):
 
 
 def build(force: bool = False, verbose_ptxas: bool = False) -> str:
-    """Build libdrr.so (the ray-march), libdrr_probe.so (the bench's L2
-    bandwidth probe) and libdrr_texture.so (the texture-trilinear
-    comparison); returns the path of libdrr.so."""
+    """Build libdrr.so (the ray-march), libdrr_checked.so (the same with
+    every gather and scatter range-checked), libdrr_probe.so (the bench's
+    probes) and libdrr_texture.so (the texture-trilinear comparison);
+    returns the path of libdrr.so."""
     if force or _stale(LIB, SOURCES, HEADERS):
         _nvcc_shared(LIB, SOURCES, verbose_ptxas)
+    if force or _stale(CHECKED_LIB, SOURCES, HEADERS):
+        _nvcc_shared(CHECKED_LIB, SOURCES, verbose_ptxas, defines=("DRR_BOUNDS_CHECK",))
     if force or _stale(PROBE_LIB, PROBE_SOURCES, []):
         _nvcc_shared(PROBE_LIB, PROBE_SOURCES, verbose_ptxas)
     if force or _stale(TEXTURE_LIB, TEXTURE_SOURCES, HEADERS):

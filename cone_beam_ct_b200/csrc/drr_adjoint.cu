@@ -67,32 +67,37 @@ namespace {
 
 // 8 corner sums of a pending block at cell (x, y, z); a[k] belongs to corner
 // (k & 1, (k >> 1) & 1, k >> 2).
+// (n: elements of the gradient volume at grad, for the bounds-checked build)
 __device__ __forceinline__ void flush_block(float* __restrict__ grad, const int st[3],
-                                            const int cell[3], const float a[8]) {
-    float* p = grad + (cell[2] * st[2] + cell[1] * st[1] + cell[0]);
+                                            const int cell[3], const float a[8], long long n) {
+    const int base = cell[2] * st[2] + cell[1] * st[1] + cell[0];
+    float* p = grad + base;
 #pragma unroll
-    for (int k = 0; k < 8; ++k)
-        atomicAdd(p + ((k & 1) ? 1 : 0) + ((k & 2) ? st[1] : 0) + ((k & 4) ? st[2] : 0), a[k]);
+    for (int k = 0; k < 8; ++k) {
+        const int off = ((k & 1) ? 1 : 0) + ((k & 2) ? st[1] : 0) + ((k & 4) ? st[2] : 0);
+        if (in_bounds(base + off, 1, n)) atomicAdd(p + off, a[k]);
+    }
 }
 
 // Move the pending block one cell along axis AX (d = +1 or -1): flush the face
 // that leaves, slide the other face over, start the new face at zero.
 template <int AX>
 __device__ __forceinline__ void slide(int d, float* __restrict__ grad, const int st[3], int cell[3],
-                                      float a[8]) {
+                                      float a[8], long long nvox) {
     if (d == 0) return;
     const int side = d > 0 ? 0 : 1;                           // face that leaves
     constexpr int A = AX == 0 ? 1 : 0, B = AX == 2 ? 1 : 2;   // the other two axes, ascending
-    float* p = grad + (cell[2] * st[2] + cell[1] * st[1] + cell[0]) + (side ? st[AX] : 0);
+    const int base = (cell[2] * st[2] + cell[1] * st[1] + cell[0]) + (side ? st[AX] : 0);
+    float* p = grad + base;
     float v[4];
     int n = 0;
 #pragma unroll
     for (int k = 0; k < 8; ++k)
         if (((k >> AX) & 1) == 0) v[n++] = side ? a[k | (1 << AX)] : a[k];
-    atomicAdd(p, v[0]);
-    atomicAdd(p + st[A], v[1]);
-    atomicAdd(p + st[B], v[2]);
-    atomicAdd(p + st[A] + st[B], v[3]);
+    if (in_bounds(base, 1, nvox)) atomicAdd(p, v[0]);
+    if (in_bounds(base + st[A], 1, nvox)) atomicAdd(p + st[A], v[1]);
+    if (in_bounds(base + st[B], 1, nvox)) atomicAdd(p + st[B], v[2]);
+    if (in_bounds(base + st[A] + st[B], 1, nvox)) atomicAdd(p + st[A] + st[B], v[3]);
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
         if (((k >> AX) & 1) != 0) continue;
@@ -127,12 +132,17 @@ __device__ __forceinline__ bool dense_tile(const View& v, const Geom& g, double 
 }
 
 // Flush a pending corner record: two 16-byte vector atomics into one sector.
-__device__ __forceinline__ void flush_record(float* __restrict__ rec, int cell, const float a[8]) {
+// (n: floats of the record array at rec, for the bounds-checked build)
+__device__ __forceinline__ void flush_record(float* __restrict__ rec, int cell, const float a[8],
+                                             long long n) {
+    if (!in_bounds((long long)cell * 8, 8, n)) return;
     float4* p = reinterpret_cast<float4*>(rec + (size_t)cell * 8);
     atomicAdd(p, make_float4(a[0], a[1], a[2], a[3]));
     atomicAdd(p + 1, make_float4(a[4], a[5], a[6], a[7]));
 }
-__device__ __forceinline__ void flush_record(float* __restrict__ rec, int cell, const float2 a[4]) {
+__device__ __forceinline__ void flush_record(float* __restrict__ rec, int cell, const float2 a[4],
+                                             long long n) {
+    if (!in_bounds((long long)cell * 8, 8, n)) return;
     float4* p = reinterpret_cast<float4*>(rec + (size_t)cell * 8);
     atomicAdd(p, make_float4(a[0].x, a[0].y, a[1].x, a[1].y));
     atomicAdd(p + 1, make_float4(a[2].x, a[2].y, a[3].x, a[3].y));
@@ -212,12 +222,16 @@ __global__ void scatter_records(const int* __restrict__ flags, const float* __re
             reinterpret_cast<const float4*>(rec + slot * rec_stride + (long long)rr * crow * 8);
         float* __restrict__ gr = grad + slot * nvox + k * nxy + (long long)j * nx;
         for (int i = threadIdx.x; i < crow; i += blockDim.x) {
+            if (!in_bounds(((long long)rr * crow + i) * 8, 8, rec_stride)) continue;
             const float4 lo = __ldcs(r + 2 * i), hi = __ldcs(r + 2 * i + 1);
             float v[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
             moments_to_corner_weights(v);
 #pragma unroll
-            for (int e = 0; e < 8; ++e)
-                if (v[e] != 0.0f) atomicAdd(gr + i + (e & 1) + ((e >> 1) & 1) * nx + (e >> 2) * nxy, v[e]);
+            for (int e = 0; e < 8; ++e) {
+                const long long off = i + (e & 1) + ((e >> 1) & 1) * nx + (e >> 2) * nxy;
+                if (v[e] != 0.0f && in_bounds(k * nxy + (long long)j * nx + off, 1, nvox))
+                    atomicAdd(gr + off, v[e]);
+            }
         }
     }
 }
@@ -245,10 +259,12 @@ __global__ void gather_records(const int* __restrict__ flags, const float* __res
 #pragma unroll
             for (int corner = 0; corner < 8; ++corner) {
                 const int ci = i - (corner & 1), cj = j - ((corner >> 1) & 1), ck = k - (corner >> 2);
-                if (ci >= 0 && cj >= 0 && ck >= 0 && ci < nx - 1 && cj < ny - 1 && ck < nz - 1)
-                    s += __ldg(r + (size_t)(ck * cs + cj * cr + ci) * 8 + corner);
+                const long long off = (long long)(ck * cs + cj * cr + ci) * 8 + corner;
+                if (ci >= 0 && cj >= 0 && ck >= 0 && ci < nx - 1 && cj < ny - 1 && ck < nz - 1 &&
+                    in_bounds(off, 1, rec_stride))
+                    s += __ldg(r + off);
             }
-            gr[i] += s;
+            if (in_bounds((long long)rr * nx + i, 1, (long long)rows * nx)) gr[i] += s;
         }
     }
 }
@@ -267,6 +283,7 @@ adjoint_kernel(const float* __restrict__ Rt, const float* __restrict__ grad_out,
     const int tid = threadIdx.x;
     if (ws.flags != nullptr && ws.flags[1 + b] != 0) return;
     const BatchItem it = batch_item(g, b);
+    if (!in_bounds(it.slot * g.vstride, g.vstride, batch_slots(g) * g.vstride)) return;
     grad += it.slot * g.vstride;                 // this volume-channel's gradient
     if (tid == 0) {
         view_setup(Rt + 12 * (size_t)it.pose, g, sv);
@@ -285,6 +302,7 @@ adjoint_kernel(const float* __restrict__ Rt, const float* __restrict__ grad_out,
     }
     if (r >= g.H || c >= g.W) return;
     const size_t pix = ((size_t)b * g.H + r) * g.W + c;
+    if (!in_bounds(pix, 1, (long long)g.B * g.H * g.W)) return;
     float go = grad_out[pix];
     if (MODE == 1) go *= 1.0f - fwd_out[pix];
     Ray ray;
@@ -315,16 +333,16 @@ adjoint_kernel(const float* __restrict__ Rt, const float* __restrict__ grad_out,
             const int dx = cx - cell[0], dy = cy - cell[1], dz = cz - cell[2];
             if (dx < -1 || dx > 1 || dy < -1 || dy > 1 || dz < -1 || dz > 1) {
                 // a step of more than one cell: flush the whole block and restart
-                flush_block(grad, st, cell, a);
+                flush_block(grad, st, cell, a, g.vstride);
 #pragma unroll
                 for (int k = 0; k < 8; ++k) a[k] = 0.0f;
                 cell[0] = cx;
                 cell[1] = cy;
                 cell[2] = cz;
             } else {
-                slide<0>(dx, grad, st, cell, a);
-                slide<1>(dy, grad, st, cell, a);
-                slide<2>(dz, grad, st, cell, a);
+                slide<0>(dx, grad, st, cell, a, g.vstride);
+                slide<1>(dy, grad, st, cell, a, g.vstride);
+                slide<2>(dz, grad, st, cell, a, g.vstride);
             }
             const float fx = fix_frac(qx), fy = fix_frac(qy), fz = fix_frac(qz);
             const float wz1 = scale * fz, wz0 = scale * (1.0f - fz);
@@ -343,7 +361,7 @@ adjoint_kernel(const float* __restrict__ Rt, const float* __restrict__ grad_out,
             qy += ray.s[1];
             qz += ray.s[2];
         }
-        flush_block(grad, st, cell, a);
+        flush_block(grad, st, cell, a, g.vstride);
     }
 }
 
@@ -386,6 +404,7 @@ records_kernel(const float* __restrict__ Rt, const float* __restrict__ grad_out,
     const int b = blockIdx.z;
     if (ws.flags[1 + b] == 0) return;            // sparse view: adjoint_kernel's
     const BatchItem it = batch_item(g, b);
+    if (!in_bounds(it.slot * ws.rec_stride, ws.rec_stride, batch_slots(g) * ws.rec_stride)) return;
     float* const rec = ws.rec + it.slot * ws.rec_stride;   // this volume-channel's records
     if (threadIdx.x == 0) view_setup(Rt + 12 * (size_t)it.pose, g, sv);
     __syncthreads();
@@ -411,6 +430,7 @@ records_kernel(const float* __restrict__ Rt, const float* __restrict__ grad_out,
         for (int a = 0; a < 3; ++a) q[k][a] = s[k][a] = 0;
         if (r >= g.H || c >= g.W) continue;
         const size_t pix = ((size_t)b * g.H + r) * g.W + c;
+        if (!in_bounds(pix, 1, (long long)g.B * g.H * g.W)) continue;
         float go = grad_out[pix];
         if (MODE == 1) go *= 1.0f - fwd_out[pix];
         Ray ray;
@@ -468,7 +488,7 @@ records_kernel(const float* __restrict__ Rt, const float* __restrict__ grad_out,
                     for (int h = 0; h < kSlots; ++h) {
                         if (h != home) continue;
                         if (pc[h] != cell) {
-                            if (pc[h] >= 0) flush_record(rec, pc[h], p[h]);
+                            if (pc[h] >= 0) flush_record(rec, pc[h], p[h], ws.rec_stride);
                             pc[h] = cell;
 #pragma unroll
                             for (int e = 0; e < 4; ++e) p[h][e] = make_float2(0.0f, 0.0f);
@@ -481,7 +501,7 @@ records_kernel(const float* __restrict__ Rt, const float* __restrict__ grad_out,
         }
 #pragma unroll
         for (int h = 0; h < kSlots; ++h)
-            if (pc[h] >= 0) flush_record(rec, pc[h], p[h]);
+            if (pc[h] >= 0) flush_record(rec, pc[h], p[h], ws.rec_stride);
     }
 }
 
@@ -512,8 +532,12 @@ alpha_adjoint_kernel(const T* __restrict__ vol_base, const float* __restrict__ R
     int pose = b;
     if constexpr (BATCH) {
         const BatchItem it = batch_item(g, b);
+        const long long slots = batch_slots(g), nv = (long long)g.nx * g.ny * g.nz;
+        if (!in_bounds(it.slot * g.vstride, g.vstride, slots * g.vstride) ||
+            !in_bounds(it.slot * nv, nv, slots * nv))
+            return;
         vol += it.slot * g.vstride;
-        grad += it.slot * ((long long)g.nx * g.ny * g.nz);
+        grad += it.slot * nv;
         pose = it.pose;
     }
     if (threadIdx.x == 0) view_setup(Rt + 12 * (size_t)pose, g, sv);
@@ -522,12 +546,14 @@ alpha_adjoint_kernel(const T* __restrict__ vol_base, const float* __restrict__ R
     tile_pixel(r, c);
     if (r >= g.H || c >= g.W) return;
     const size_t pix = ((size_t)b * g.H + r) * g.W + c;
+    if (!in_bounds(pix, 1, (long long)g.B * g.H * g.W)) return;
     const float go = grad_out[pix];
     Ray ray;
     if (go == 0.0f || !ray_setup(sv, g, (double)c, (double)r, 0.0, ray)) return;
     const float Cray = fwd_out[pix];
     const float s = g.density_factor * ray.dt;
     const int st[3] = {1, grad_row, grad_slice};
+    const long long nvox = (long long)g.nx * g.ny * g.nz;
     long long qx = ray.q0[0], qy = ray.q0[1], qz = ray.q0[2];
     int cell[3] = {fix_cell(qx), fix_cell(qy), fix_cell(qz)};
     float a8[8];
@@ -539,9 +565,11 @@ alpha_adjoint_kernel(const T* __restrict__ vol_base, const float* __restrict__ R
         const float fx = fix_frac(qx), fy = fix_frac(qy), fz = fix_frac(qz);
         // the forward's sample value, bit for bit
         const int at = cz * g.slice + cy * g.row + cx;
-        const float mu = LAYOUT == 2   ? sample_corners(vol + (size_t)at * 8, fx, fy, fz)
-                         : LAYOUT == 3 ? sample_quads(vol + (size_t)at * 4, g.slice, fx, fy, fz)
-                                       : trilinear_at(vol + at, g.row, g.slice, fx, fy, fz);
+        const float mu =
+            !in_bounds(sample_offset<LAYOUT>(at), sample_extent<LAYOUT>(g), g.vstride) ? 0.0f
+            : LAYOUT == 2 ? sample_corners(vol + (size_t)at * 8, fx, fy, fz)
+            : LAYOUT == 3 ? sample_quads(vol + (size_t)at * 4, g.slice, fx, fy, fz)
+                          : trilinear_at(vol + at, g.row, g.slice, fx, fy, fz);
         const float a = -expm1f(-s * mu);
         Ci = fmaf(Tr * a, mu, Ci);
         const float dmu = Tr * fmaf(s * (1.0f - a), mu, a) - s * (Cray - Ci);
@@ -549,16 +577,16 @@ alpha_adjoint_kernel(const T* __restrict__ vol_base, const float* __restrict__ R
         const float scale = go * dmu;
         const int dx = cx - cell[0], dy = cy - cell[1], dz = cz - cell[2];
         if (dx < -1 || dx > 1 || dy < -1 || dy > 1 || dz < -1 || dz > 1) {
-            flush_block(grad, st, cell, a8);
+            flush_block(grad, st, cell, a8, nvox);
 #pragma unroll
             for (int k = 0; k < 8; ++k) a8[k] = 0.0f;
             cell[0] = cx;
             cell[1] = cy;
             cell[2] = cz;
         } else {
-            slide<0>(dx, grad, st, cell, a8);
-            slide<1>(dy, grad, st, cell, a8);
-            slide<2>(dz, grad, st, cell, a8);
+            slide<0>(dx, grad, st, cell, a8, nvox);
+            slide<1>(dy, grad, st, cell, a8, nvox);
+            slide<2>(dz, grad, st, cell, a8, nvox);
         }
         const float wz1 = scale * fz, wz0 = scale * (1.0f - fz);
         const float w00 = wz0 * (1.0f - fy), w01 = wz0 * fy;
@@ -576,7 +604,7 @@ alpha_adjoint_kernel(const T* __restrict__ vol_base, const float* __restrict__ R
         qy += ray.s[1];
         qz += ray.s[2];
     }
-    flush_block(grad, st, cell, a8);
+    flush_block(grad, st, cell, a8, nvox);
 }
 
 // Record path of the alpha gradient for the views the plan marked dense: the
@@ -602,6 +630,10 @@ alpha_records_kernel(const T* __restrict__ vol_base, const float* __restrict__ R
     const int b = blockIdx.z;
     if (ws.flags[1 + b] == 0) return;            // sparse view: alpha_adjoint_kernel's
     const BatchItem it = batch_item(g, b);
+    const long long slots = batch_slots(g);
+    if (!in_bounds(it.slot * g.vstride, g.vstride, slots * g.vstride) ||
+        !in_bounds(it.slot * ws.rec_stride, ws.rec_stride, slots * ws.rec_stride))
+        return;
     const T* __restrict__ vol = vol_base + it.slot * g.vstride;
     float* const rec = ws.rec + it.slot * ws.rec_stride;   // this volume-channel's records
     if (threadIdx.x == 0) view_setup(Rt + 12 * (size_t)it.pose, g, sv);
@@ -624,6 +656,7 @@ alpha_records_kernel(const T* __restrict__ vol_base, const float* __restrict__ R
         for (int a = 0; a < 3; ++a) q[k][a] = s[k][a] = 0;
         if (r >= g.H || c >= g.W) continue;
         const size_t pix = ((size_t)b * g.H + r) * g.W + c;
+        if (!in_bounds(pix, 1, (long long)g.B * g.H * g.W)) continue;
         go[k] = grad_out[pix];
         Ray ray;
         if (go[k] == 0.0f || !ray_setup(sv, g, (double)c, (double)r, 0.0, ray)) continue;
@@ -652,9 +685,11 @@ alpha_records_kernel(const T* __restrict__ vol_base, const float* __restrict__ R
             for (int a = 0; a < 3; ++a) q[k][a] += s[k][a];
             // the forward's sample value, bit for bit
             const int at = cz * g.slice + cy * g.row + cx;
-            const float mu = LAYOUT == 2   ? sample_corners(vol + (size_t)at * 8, fx, fy, fz)
-                             : LAYOUT == 3 ? sample_quads(vol + (size_t)at * 4, g.slice, fx, fy, fz)
-                                           : trilinear_at(vol + at, g.row, g.slice, fx, fy, fz);
+            const float mu =
+                !in_bounds(sample_offset<LAYOUT>(at), sample_extent<LAYOUT>(g), g.vstride) ? 0.0f
+                : LAYOUT == 2 ? sample_corners(vol + (size_t)at * 8, fx, fy, fz)
+                : LAYOUT == 3 ? sample_quads(vol + (size_t)at * 4, g.slice, fx, fy, fz)
+                              : trilinear_at(vol + at, g.row, g.slice, fx, fy, fz);
             const float a = -expm1f(-sa[k] * mu);
             Ci[k] = fmaf(Tr[k] * a, mu, Ci[k]);
             const float dmu = Tr[k] * fmaf(sa[k] * (1.0f - a), mu, a) - sa[k] * (Cray[k] - Ci[k]);
@@ -679,7 +714,7 @@ alpha_records_kernel(const T* __restrict__ vol_base, const float* __restrict__ R
                 for (int h = 0; h < kSlots; ++h) {
                     if (h != home) continue;
                     if (pc[h] != cell) {
-                        if (pc[h] >= 0) flush_record(rec, pc[h], p[h]);
+                        if (pc[h] >= 0) flush_record(rec, pc[h], p[h], ws.rec_stride);
                         pc[h] = cell;
 #pragma unroll
                         for (int e = 0; e < 8; ++e) p[h][e] = 0.0f;
@@ -692,7 +727,7 @@ alpha_records_kernel(const T* __restrict__ vol_base, const float* __restrict__ R
     }
 #pragma unroll
     for (int h = 0; h < kSlots; ++h)
-        if (pc[h] >= 0) flush_record(rec, pc[h], p[h]);
+        if (pc[h] >= 0) flush_record(rec, pc[h], p[h], ws.rec_stride);
 }
 
 }  // namespace
@@ -726,6 +761,8 @@ cudaError_t noalloc_scratch(void** out) {
     *out = g_noalloc_addr[dev];
     return cudaSuccess;
 }
+
+DRR_BOUNDS_READER(bounds_word_adjoint)
 
 size_t adjoint_workspace_bytes(int nx, int ny, int nz, int B, int slots) {
     return adjoint_workspace_header(B) +

@@ -12,6 +12,7 @@
 #include <cstdio>
 
 #include "../../include/drr.h"
+#include "../../include/drr_debug.h"
 #include "drr_internal.cuh"
 
 static_assert(DRR_NOALLOC_SCRATCH_BYTES == drr::kNoAllocScratchBytes,
@@ -354,6 +355,25 @@ drr_status render_alpha_adjoint(const void* vol, drr_dtype dtype, drr_layout lay
 }  // namespace
 
 extern "C" {
+
+#ifdef DRR_BOUNDS_CHECK
+DRR_API drr_status drr_debug_bounds_errors(unsigned long long* count, long long* first) {
+    if (!count || !first) return fail(DRR_ERR_INVALID_ARG, "count and first must be non-NULL");
+    cudaError_t (*const readers[])(drr::BoundsWord*) = {
+        drr::bounds_word_forward, drr::bounds_word_adjoint, drr::bounds_word_pose,
+        drr::bounds_word_siddon,  drr::bounds_word_prepare, drr::bounds_word_noise};
+    *count = 0;
+    *first = 0;
+    for (auto read : readers) {
+        drr::BoundsWord w{0ULL, 0LL};
+        const cudaError_t e = read(&w);
+        if (e != cudaSuccess) return cuda_status(e, "drr_debug_bounds_errors");
+        if (w.count && *count == 0) *first = w.first;
+        *count += w.count;
+    }
+    return ok();
+}
+#endif
 
 DRR_API int drr_abi_version(void) { return 1; }
 

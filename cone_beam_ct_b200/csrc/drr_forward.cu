@@ -39,7 +39,8 @@ __device__ __forceinline__ float march(const T* __restrict__ vol, const Geom& g,
 #pragma unroll 4
     for (int i = 0; i < g.N; ++i) {
         const int idx = fix_cell(qz) * slice + fix_cell(qy) * row + fix_cell(qx);
-        acc += trilinear_at(vol + idx, row, slice, fix_frac(qx), fix_frac(qy), fix_frac(qz));
+        if (in_bounds(idx, sample_extent<0>(g), g.vstride))
+            acc += trilinear_at(vol + idx, row, slice, fix_frac(qx), fix_frac(qy), fix_frac(qz));
         qx += sx;
         qy += sy;
         qz += sz;
@@ -65,7 +66,8 @@ __device__ __forceinline__ float march_corners(const T* __restrict__ vol, const 
 #pragma unroll(kCornerUnroll<T>)
     for (int i = 0; i < g.N; ++i) {
         const int cell = fix_cell(qz) * slice + fix_cell(qy) * row + fix_cell(qx);
-        acc += sample_corners(vol + (size_t)cell * 8, fix_frac(qx), fix_frac(qy), fix_frac(qz));
+        if (in_bounds(sample_offset<2>(cell), 8, g.vstride))
+            acc += sample_corners(vol + (size_t)cell * 8, fix_frac(qx), fix_frac(qy), fix_frac(qz));
         qx += sx;
         qy += sy;
         qz += sz;
@@ -90,9 +92,11 @@ __device__ __forceinline__ float march_alpha(const T* __restrict__ vol, const Ge
     for (int i = 0; i < g.N; ++i) {
         const int cell = fix_cell(qz) * slice + fix_cell(qy) * row + fix_cell(qx);
         const float fx = fix_frac(qx), fy = fix_frac(qy), fz = fix_frac(qz);
-        const float mu = LAYOUT == 2   ? sample_corners(vol + (size_t)cell * 8, fx, fy, fz)
-                         : LAYOUT == 3 ? sample_quads(vol + (size_t)cell * 4, slice, fx, fy, fz)
-                                       : trilinear_at(vol + cell, row, slice, fx, fy, fz);
+        const float mu =
+            !in_bounds(sample_offset<LAYOUT>(cell), sample_extent<LAYOUT>(g), g.vstride) ? 0.0f
+            : LAYOUT == 2 ? sample_corners(vol + (size_t)cell * 8, fx, fy, fz)
+            : LAYOUT == 3 ? sample_quads(vol + (size_t)cell * 4, slice, fx, fy, fz)
+                          : trilinear_at(vol + cell, row, slice, fx, fy, fz);
         const float a = -expm1f(-s * mu);
         C = fmaf(Tr * a, mu, C);
         Tr *= 1.0f - a;
@@ -121,7 +125,8 @@ __device__ __forceinline__ float march_quads(const T* __restrict__ vol, const Ge
 #pragma unroll 4
     for (int i = 0; i < g.N; ++i) {
         const int q = fix_cell(qz) * slice + fix_cell(qy) * row + fix_cell(qx);
-        acc += sample_quads(vol + (size_t)q * 4, slice, fix_frac(qx), fix_frac(qy), fix_frac(qz));
+        if (in_bounds(sample_offset<3>(q), sample_extent<3>(g), g.vstride))
+            acc += sample_quads(vol + (size_t)q * 4, slice, fix_frac(qx), fix_frac(qy), fix_frac(qz));
         qx += sx;
         qy += sy;
         qz += sz;
@@ -137,6 +142,7 @@ forward_kernel(const T* __restrict__ vol_base, const float* __restrict__ Rt,
     const int b = blockIdx.z;                    // output image (view x channel)
     const BatchItem it = batch_item(g, b);
     const T* __restrict__ vol = vol_base + it.slot * g.vstride;
+    if (!in_bounds(it.slot * g.vstride, g.vstride, batch_slots(g) * g.vstride)) return;
     if (threadIdx.x == 0) view_setup(Rt + 12 * (size_t)it.pose, g, sv);
     __syncthreads();
     int r, c;
@@ -155,7 +161,8 @@ forward_kernel(const T* __restrict__ vol_base, const float* __restrict__ Rt,
             result = (MODE == 1) ? -expm1f(-I) : I;
         }
     }
-    out[((size_t)b * g.H + r) * g.W + c] = result;
+    const long long pix = ((long long)b * g.H + r) * g.W + c;
+    if (in_bounds(pix, 1, (long long)g.B * g.H * g.W)) out[pix] = result;
 }
 
 template <typename T, int LAYOUT>
@@ -182,6 +189,8 @@ cudaError_t launch_layout(const void* vol, int layout, const Geom& g, const floa
 }
 
 }  // namespace
+
+DRR_BOUNDS_READER(bounds_word_forward)
 
 cudaError_t launch_forward(const void* vol, int dtype, int layout, const Geom& g,
                            const float* Rt, int mode, float* out, cudaStream_t stream) {

@@ -182,6 +182,57 @@ __device__ __forceinline__ bool ray_setup(const View& v, const Geom& g, double u
     return true;
 }
 
+// ---------------------------------------------------------------------------
+// Bounds-checked debug build.  Compiled with -DDRR_BOUNDS_CHECK (into
+// libdrr_checked.so), every gather and scatter of the kernels tests its
+// element range [off, off + len) against the extent n of the buffer (or of
+// the volume-channel slot) it addresses; an access outside is skipped (a
+// load reads 0) and counted in this translation unit's error word, with the
+// first offending offset.  drr_debug_bounds_errors (include/drr_debug.h)
+// reads and clears the words of every unit.  In the ordinary build the test
+// is the constant true and compiles away.
+struct BoundsWord {
+    unsigned long long count;
+    long long first;
+};
+
+#ifdef DRR_BOUNDS_CHECK
+static __device__ BoundsWord g_bounds_word;
+
+__device__ __forceinline__ bool in_bounds(long long off, long long len, long long n) {
+    if (off >= 0 && len >= 0 && off <= n - len) return true;
+    if (atomicAdd(&g_bounds_word.count, 1ULL) == 0ULL) g_bounds_word.first = off;
+    return false;
+}
+
+// Host: this unit's error word (read, then cleared); defined once per .cu
+// file that launches kernels, under the given name.
+#define DRR_BOUNDS_READER(name)                                                  \
+    cudaError_t name(BoundsWord* out) {                                          \
+        cudaError_t e = cudaMemcpyFromSymbol(out, g_bounds_word, sizeof(*out));  \
+        if (e != cudaSuccess) return e;                                          \
+        const BoundsWord zero{0ULL, 0LL};                                        \
+        return cudaMemcpyToSymbol(g_bounds_word, &zero, sizeof(zero));           \
+    }
+#else
+__device__ __forceinline__ constexpr bool in_bounds(long long, long long, long long) {
+    return true;
+}
+#define DRR_BOUNDS_READER(name)
+#endif
+
+// Elements one trilinear sample reads, from the offset of its cell's first
+// element, in each stored layout (0 linear, 1 zero-bordered, 2 corner
+// records, 3 xy quads), and that offset for cell index `cell`.
+template <int LAYOUT>
+__host__ __device__ __forceinline__ long long sample_extent(const Geom& g) {
+    return LAYOUT == 2 ? 8 : LAYOUT == 3 ? 4LL * g.slice + 4 : (long long)g.slice + g.row + 2;
+}
+template <int LAYOUT>
+__host__ __device__ __forceinline__ long long sample_offset(long long cell) {
+    return LAYOUT == 2 ? cell * 8 : LAYOUT == 3 ? cell * 4 : cell;
+}
+
 // Pixel of this thread inside a kTileW x kTileH tile (warps are 8 x 4).
 __device__ __forceinline__ void tile_pixel(int& r, int& c) {
     const int tid = threadIdx.x;
@@ -271,6 +322,16 @@ cudaError_t launch_siddon(const void* vol, int dtype, const Geom& g, const float
                           float* out, cudaStream_t stream);
 cudaError_t launch_siddon_adjoint(const Geom& g, const float* Rt, int mode, const float* grad_out,
                                   const float* fwd_out, float* grad_vol, cudaStream_t stream);
+// per-unit readers of the bounds-check error words (the checked build only)
+#ifdef DRR_BOUNDS_CHECK
+cudaError_t bounds_word_forward(BoundsWord* out);
+cudaError_t bounds_word_adjoint(BoundsWord* out);
+cudaError_t bounds_word_pose(BoundsWord* out);
+cudaError_t bounds_word_siddon(BoundsWord* out);
+cudaError_t bounds_word_prepare(BoundsWord* out);
+cudaError_t bounds_word_noise(BoundsWord* out);
+#endif
+
 cudaError_t launch_pose_grad(const void* vol, int dtype, int layout, const Geom& g,
                              const float* Rt, int mode, const float* grad_out,
                              const float* fwd_out, float* grad_Rt, cudaStream_t stream);

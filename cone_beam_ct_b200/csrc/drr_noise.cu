@@ -53,6 +53,9 @@ int grid_for_elements(int64_t n) {
 
 }  // namespace
 
+// (the elementwise loops index only [0, n): nothing to check)
+DRR_BOUNDS_READER(bounds_word_noise)
+
 cudaError_t launch_poisson_noise(const float* image, const float* z, float i0, float* out,
                                  int64_t n, cudaStream_t stream) {
     poisson_noise_kernel<<<grid_for_elements(n), 256, 0, stream>>>(image, z, i0, out, n);

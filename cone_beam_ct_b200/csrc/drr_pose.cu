@@ -39,6 +39,12 @@ __device__ __forceinline__ float widen(uint16_t v) { return __uint_as_float((uin
 template <typename T, int LAYOUT>
 __device__ __forceinline__ void cell_corners(const T* __restrict__ vol, const Geom& g, int cx,
                                              int cy, int cz, float v[8]) {
+    if (!in_bounds(sample_offset<LAYOUT>(cz * g.slice + cy * g.row + cx), sample_extent<LAYOUT>(g),
+                   g.vstride)) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) v[e] = 0.0f;
+        return;
+    }
     if (LAYOUT == 2) {
         const T* p = vol + (size_t)(cz * g.slice + cy * g.row + cx) * 8;
         if constexpr (sizeof(T) == 4) {
@@ -211,6 +217,9 @@ pose_kernel(const T* __restrict__ vol_base, const float* __restrict__ Rt,
     __shared__ double red[kThreads / 32][12];
     const int b = blockIdx.z;                    // output image (view x channel)
     const T* __restrict__ vol = BATCH ? vol_base + batch_item(g, b).slot * g.vstride : vol_base;
+    if (!in_bounds(BATCH ? batch_item(g, b).slot * g.vstride : 0, g.vstride,
+                   batch_slots(g) * g.vstride))
+        return;
     {
         const int pose = BATCH ? batch_item(g, b).pose : b;
         if (threadIdx.x == 0) view_setup(Rt + 12 * (size_t)pose, g, sv);
@@ -224,7 +233,7 @@ pose_kernel(const T* __restrict__ vol_base, const float* __restrict__ Rt,
     for (int e = 0; e < 12; ++e) acc[e] = 0.0;
     if (r < g.H && c < g.W) {
         const size_t pix = ((size_t)b * g.H + r) * g.W + c;
-        float go = grad_out[pix];
+        float go = in_bounds(pix, 1, (long long)g.B * g.H * g.W) ? grad_out[pix] : 0.0f;
         if (MODE == 1) go *= 1.0f - fwd_out[pix];           // d(1 - e^-I)/dI = e^-I
         Ray ray;
         if (go != 0.0f && ray_setup(sv, g, (double)c, (double)r, LAYOUT == 1 ? 1.0 : 0.0, ray)) {
@@ -244,8 +253,12 @@ pose_kernel(const T* __restrict__ vol_base, const float* __restrict__ Rt,
                 float val, gx, gy, gz;
                 if constexpr (LAYOUT == 2 && sizeof(T) == 2) {
                     const int cell = fix_cell(qz) * g.slice + fix_cell(qy) * g.row + fix_cell(qx);
-                    value_grad_bf16(reinterpret_cast<const uint16_t*>(vol) + (size_t)cell * 8, fx,
-                                    fy, fz, val, gx, gy, gz);
+                    if (in_bounds((long long)cell * 8, 8, g.vstride)) {
+                        value_grad_bf16(reinterpret_cast<const uint16_t*>(vol) + (size_t)cell * 8,
+                                        fx, fy, fz, val, gx, gy, gz);
+                    } else {
+                        val = gx = gy = gz = 0.0f;
+                    }
                 } else {
                     float v[8];
                     cell_corners<T, LAYOUT>(vol, g, fix_cell(qx), fix_cell(qy), fix_cell(qz), v);
@@ -319,7 +332,9 @@ pose_kernel(const T* __restrict__ vol_base, const float* __restrict__ Rt,
 #pragma unroll
         for (int w = 0; w < kThreads / 32; ++w) x += red[w][threadIdx.x];
         const int pose = BATCH ? batch_item(g, blockIdx.z).pose : (int)blockIdx.z;
-        if (x != 0.0) atomicAdd(grad_Rt + 12 * (size_t)pose + threadIdx.x, (float)x);
+        const long long poses = g.broadcast ? 1 : g.B / g.C;
+        if (x != 0.0 && in_bounds(12LL * pose + threadIdx.x, 1, 12 * poses))
+            atomicAdd(grad_Rt + 12 * (size_t)pose + threadIdx.x, (float)x);
     }
 }
 
@@ -356,6 +371,8 @@ cudaError_t launch_layout(const void* vol, int layout, const Geom& g, const floa
 }
 
 }  // namespace
+
+DRR_BOUNDS_READER(bounds_word_pose)
 
 cudaError_t launch_pose_grad(const void* vol, int dtype, int layout, const Geom& g,
                              const float* Rt, int mode, const float* grad_out,

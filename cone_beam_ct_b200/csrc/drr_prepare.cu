@@ -46,8 +46,10 @@ __global__ void to_padded(const float* __restrict__ src, T* __restrict__ dst, in
         const int j = (int)((m / px) % py);
         const int k = (int)(m / ((int64_t)px * py));
         float v = 0.0f;
-        if (i >= 1 && i <= nx && j >= 1 && j <= ny && k >= 1 && k <= nz)
-            v = __ldg(src + (((int64_t)(k - 1) * ny + (j - 1)) * nx + (i - 1)));
+        const int64_t at = ((int64_t)(k - 1) * ny + (j - 1)) * nx + (i - 1);
+        if (i >= 1 && i <= nx && j >= 1 && j <= ny && k >= 1 && k <= nz &&
+            in_bounds(at, 1, (int64_t)nx * ny * nz))
+            v = __ldg(src + at);
         dst[m] = store_value<T>(v);
     }
 }
@@ -80,13 +82,15 @@ __global__ void to_corners(const float* __restrict__ src, T* __restrict__ dst, i
         const int i = (int)(m % cx);
         const int j = (int)((m / cx) % cy);
         const int k = (int)(m / ((int64_t)cx * cy));
-        const float* p = src + (((int64_t)k * ny + j) * nx + i);
+        const int64_t at = ((int64_t)k * ny + j) * nx + i;
+        const float* p = src + at;
         const int64_t sy = nx, sz = (int64_t)nx * ny;
         // corner (a, b, c) at element a + 2b + 4c
         float v[8];
+        const bool ok = in_bounds(at, sz + sy + 2, sz * nz);
 #pragma unroll
         for (int e = 0; e < 8; ++e)
-            v[e] = __ldg(p + ((e & 1) ? 1 : 0) + ((e & 2) ? sy : 0) + ((e & 4) ? sz : 0));
+            v[e] = ok ? __ldg(p + ((e & 1) ? 1 : 0) + ((e & 2) ? sy : 0) + ((e & 4) ? sz : 0)) : 0.0f;
         store_corners(dst + m * 8, v);
     }
 }
@@ -104,7 +108,9 @@ __global__ void to_quads(const float* __restrict__ src, T* __restrict__ dst, int
         const int j = (int)((m / qx) % qy);
         const int64_t k = m / ((int64_t)qx * qy);
         const float* p = src + (k * ny + j) * nx + i;
-        const float v[4] = {__ldg(p), __ldg(p + 1), __ldg(p + nx), __ldg(p + nx + 1)};
+        const bool ok = in_bounds((k * ny + j) * nx + i, (int64_t)nx + 2, (int64_t)nx * ny * nz);
+        const float v[4] = {ok ? __ldg(p) : 0.0f, ok ? __ldg(p + 1) : 0.0f,
+                            ok ? __ldg(p + nx) : 0.0f, ok ? __ldg(p + nx + 1) : 0.0f};
         if constexpr (sizeof(T) == 4) {
             reinterpret_cast<float4*>(dst)[m] = make_float4(v[0], v[1], v[2], v[3]);
         } else {
@@ -124,6 +130,8 @@ int grid_for(int64_t n) {
 }
 
 }  // namespace
+
+DRR_BOUNDS_READER(bounds_word_prepare)
 
 cudaError_t launch_prepare(const float* src, int nx, int ny, int nz, int dtype, int layout,
                            void* dst, cudaStream_t stream) {

@@ -143,13 +143,15 @@ siddon_forward_kernel(const T* __restrict__ vol, const float* __restrict__ Rt,
             const int idx = k.idx;               // in the volume: checked before every step
             double len;
             const bool more = walk_step(g, k, len);
-            acc = fmaf((float)len, voxel_value(vol + idx), acc);
+            if (in_bounds(idx, 1, (long long)g.nx * g.ny * g.nz))
+                acc = fmaf((float)len, voxel_value(vol + idx), acc);
             if (!more) break;
         }
         const float I = g.density_factor * acc;
         result = MODE == 1 ? -expm1f(-I) : I;
     }
-    out[((size_t)b * g.H + r) * g.W + c] = result;
+    const long long pix = ((long long)b * g.H + r) * g.W + c;
+    if (in_bounds(pix, 1, (long long)g.B * g.H * g.W)) out[pix] = result;
 }
 
 template <int MODE>
@@ -164,6 +166,7 @@ siddon_adjoint_kernel(const float* __restrict__ Rt, const float* __restrict__ gr
     tile_pixel(r, c);
     if (r >= g.H || c >= g.W) return;
     const size_t pix = ((size_t)b * g.H + r) * g.W + c;
+    if (!in_bounds(pix, 1, (long long)g.B * g.H * g.W)) return;
     float go = grad_out[pix];
     if (MODE == 1) go *= 1.0f - fwd_out[pix];
     Walk k;
@@ -174,12 +177,15 @@ siddon_adjoint_kernel(const float* __restrict__ Rt, const float* __restrict__ gr
         const int idx = k.idx;
         double len;
         const bool more = walk_step(g, k, len);
-        if (len > 0.0) atomicAdd(grad + idx, scale * (float)len);
+        if (len > 0.0 && in_bounds(idx, 1, (long long)g.nx * g.ny * g.nz))
+            atomicAdd(grad + idx, scale * (float)len);
         if (!more) break;
     }
 }
 
 }  // namespace
+
+DRR_BOUNDS_READER(bounds_word_siddon)
 
 cudaError_t launch_siddon(const void* vol, int dtype, const Geom& g, const float* Rt, int mode,
                           float* out, cudaStream_t stream) {

@@ -13,6 +13,8 @@ import os
 import numpy as np
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libdrr.so")
+# the bounds-checked debug build of the same sources (include/drr_debug.h)
+CHECKED_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libdrr_checked.so")
 
 DRR_OK, DRR_ERR_INVALID_ARG, DRR_ERR_UNSUPPORTED, DRR_ERR_CUDA = 0, 1, 2, 3
 DRR_MODE_RAW, DRR_MODE_BEER_LAMBERT, DRR_MODE_ALPHA = 0, 1, 2
@@ -43,6 +45,17 @@ _vp = ctypes.c_void_p
 _i3 = ctypes.c_int * 3
 _f3 = ctypes.c_float * 3
 _f9 = ctypes.c_float * 9
+
+
+def use_library(path):
+    """Load ``path`` (for example CHECKED_LIB_PATH, the bounds-checked debug
+    build) in place of libdrr.so for every later call; returns the path that
+    was in use, so that a caller can switch back."""
+    global _lib, LIB_PATH
+    previous = LIB_PATH
+    LIB_PATH = path
+    _lib = None
+    return previous
 
 
 def lib():
@@ -123,6 +136,9 @@ def lib():
     L.drr_get_last_error.restype = _c.c_char_p
     L.drr_abi_version.argtypes = []
     L.drr_abi_version.restype = _c.c_int
+    if hasattr(L, "drr_debug_bounds_errors"):
+        L.drr_debug_bounds_errors.argtypes = [_c.POINTER(_c.c_ulonglong), _c.POINTER(_c.c_longlong)]
+        L.drr_debug_bounds_errors.restype = _c.c_int
     _lib = L
     return L
 
@@ -387,3 +403,15 @@ def drr_render_adjoint_noalloc(dims, spacing, origin, K, Rt, B, H, W, n_samples,
                                             _dev(grad_out, "grad_out", True),
                                             _dev(fwd_out, "fwd_out", True),
                                             _dev(grad_vol, "grad_vol", True), _stream(stream)))
+
+
+def drr_debug_bounds_errors():
+    """(count, first offset) of out-of-range accesses since the last call, from
+    the bounds-checked build (use_library(CHECKED_LIB_PATH)); the device
+    words are cleared.  Call after the work has completed."""
+    L = lib()
+    if not hasattr(L, "drr_debug_bounds_errors"):
+        raise RuntimeError(f"{LIB_PATH} is not the bounds-checked build")
+    count, first = _c.c_ulonglong(0), _c.c_longlong(0)
+    _check(L.drr_debug_bounds_errors(_c.byref(count), _c.byref(first)))
+    return int(count.value), int(first.value)

@@ -45,6 +45,23 @@ def test_library_exports_every_declared_symbol():
     assert drr.drr_abi_version() == 1
 
 
+def test_checked_library_exports_the_abi_and_its_debug_call():
+    checked = os.path.join(ROOT, "cone_beam_ct_b200", "libdrr_checked.so")
+    debug = declared_names(os.path.join(ROOT, "include", "drr_debug.h"))
+    assert debug == ["drr_debug_bounds_errors"]
+    assert exported_names(checked) == set(declared_names()) | set(debug)
+    assert "drr_debug_bounds_errors" not in exported_names(drr.LIB_PATH)
+
+
+def test_checked_library_debug_call_rejects_null_pointers():
+    import ctypes
+    L = ctypes.CDLL(os.path.join(ROOT, "cone_beam_ct_b200", "libdrr_checked.so"))
+    L.drr_debug_bounds_errors.argtypes = [ctypes.c_void_p, ctypes.c_void_p]
+    L.drr_get_last_error.restype = ctypes.c_char_p
+    assert L.drr_debug_bounds_errors(None, None) == drr.DRR_ERR_INVALID_ARG
+    assert b"non-NULL" in L.drr_get_last_error()
+
+
 def test_probe_library_exports_its_declared_symbol():
     import ctypes
     ctypes.CDLL(PROBE_LIB)
@@ -63,7 +80,7 @@ def test_texture_library_exports_its_declared_symbols():
 
 def test_every_header_is_covered():
     headers = sorted(f for f in os.listdir(os.path.join(ROOT, "include")) if f.endswith(".h"))
-    assert headers == ["drr.h", "drr_probe.h", "drr_texture.h"]
+    assert headers == ["drr.h", "drr_debug.h", "drr_probe.h", "drr_texture.h"]
 
 
 def _render(**kw):
