@@ -54,7 +54,7 @@ def parse_args():
     p.add_argument("--config", type=int, default=3, choices=[1, 2, 3, 4],
                    help="workload (default 3: 256^3 bf16, 4 views 1024x1024, 512 samples, "
                         "the size the throughput target is quoted at)")
-    p.add_argument("--layout", choices=["auto", "padded", "corners", "quads", "linear"],
+    p.add_argument("--layout", choices=["auto", "padded", "corners", "quads", "linear", "bricks"],
                    default="auto",
                    help="volume layout drr_prepare_volume writes for the forward (auto: the "
                         "faster one measured for the workload, AUTO_LAYOUT)")
@@ -116,12 +116,14 @@ def job_throughput(world, units_per_rank_step, steps, max_ms):
 # workload description
 
 # The layout each workload's forward runs fastest in on B200: corner records
-# (one load per sample) where dense rays reuse them in L1, xy quads (half the
-# footprint) where sparse views re-read an fp32 volume from DRAM.  Forward
-# times measured: 256^3 fp32 seen by 64 views of 200^2, quads 2.17 / corners
-# 2.96 ms; 256^3 bf16 seen by 4 views of 1024^2, corners 2.87 / quads 3.88 ms;
-# 512^3 fp32 seen by 2 views of 2048^2, corners 3.97 / quads 4.49 ms.
-AUTO_LAYOUT = {1: "corners", 2: "quads", 3: "corners", 4: "corners"}
+# (one 16-byte load per sample) where dense bf16 rays reuse them in L1, xy
+# quads (two loads, half the footprint) for the fp32 volumes.  Forward times
+# measured (ms): 256^3 fp32 seen by 64 views of 200^2: quads 2.00, bricks
+# 2.43, padded 2.96, corners 3.01, linear 3.95; 256^3 bf16 seen by 4 views of
+# 1024^2: corners 2.86, quads 3.86, bricks 4.78, padded 4.92, linear 6.27;
+# 512^3 fp32 seen by 2 views of 2048^2: quads 3.76, corners 3.97, bricks
+# 4.53, padded 4.71, linear 6.23.
+AUTO_LAYOUT = {1: "corners", 2: "quads", 3: "corners", 4: "quads"}
 
 
 def workload(cfg):
@@ -721,7 +723,8 @@ def config_timing(torch, cfg, hbm_peak, l2_cache):
     dev = torch.device("cuda", torch.cuda.current_device())
     geom_cfg = 2 if cfg == 5 else cfg
     lname = AUTO_LAYOUT[geom_cfg]
-    layout = {"corners": drr.DRR_LAYOUT_CORNERS, "quads": drr.DRR_LAYOUT_QUADS}[lname]
+    layout = {"corners": drr.DRR_LAYOUT_CORNERS, "quads": drr.DRR_LAYOUT_QUADS,
+              "bricks": drr.DRR_LAYOUT_BRICKS}[lname]
     dtype = drr.DRR_BF16 if w.dtype == wl.DTYPE_BF16 else drr.DRR_F32
     elem = 2 if dtype == drr.DRR_BF16 else 4
     nx, ny, nz = w.dims
@@ -799,7 +802,8 @@ def run_ours(args):
     if args.layout == "auto":
         args.layout = AUTO_LAYOUT[args.config]
     layout = {"padded": drr.DRR_LAYOUT_PADDED, "corners": drr.DRR_LAYOUT_CORNERS,
-              "quads": drr.DRR_LAYOUT_QUADS, "linear": drr.DRR_LAYOUT_LINEAR}[args.layout]
+              "quads": drr.DRR_LAYOUT_QUADS, "linear": drr.DRR_LAYOUT_LINEAR,
+              "bricks": drr.DRR_LAYOUT_BRICKS}[args.layout]
     dtype = drr.DRR_BF16 if w.dtype == wl.DTYPE_BF16 else drr.DRR_F32
     elem = 2 if dtype == drr.DRR_BF16 else 4
     nx, ny, nz = w.dims
@@ -1053,7 +1057,8 @@ def run_partitioned(args):
     if args.layout == "auto":
         args.layout = AUTO_LAYOUT[args.config]
     layout = {"padded": drr.DRR_LAYOUT_PADDED, "corners": drr.DRR_LAYOUT_CORNERS,
-              "quads": drr.DRR_LAYOUT_QUADS, "linear": drr.DRR_LAYOUT_LINEAR}[args.layout]
+              "quads": drr.DRR_LAYOUT_QUADS, "linear": drr.DRR_LAYOUT_LINEAR,
+              "bricks": drr.DRR_LAYOUT_BRICKS}[args.layout]
     dtype = drr.DRR_BF16 if w.dtype == wl.DTYPE_BF16 else drr.DRR_F32
     nx, ny, nz = w.dims
     part = P.Partition(w.B, w.H, w.W, world, rank)

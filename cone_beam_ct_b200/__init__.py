@@ -8,6 +8,7 @@ gradient; ``cone_beam_ct_b200.drr`` binds it with the same names.
 from .drr import (  # noqa: F401
     DRR_BF16,
     DRR_F32,
+    DRR_LAYOUT_BRICKS,
     DRR_LAYOUT_CORNERS,
     DRR_LAYOUT_LINEAR,
     DRR_LAYOUT_PADDED,

@@ -564,9 +564,10 @@ alpha_adjoint_kernel(const T* __restrict__ vol_base, const float* __restrict__ R
         const int cx = fix_cell(qx), cy = fix_cell(qy), cz = fix_cell(qz);
         const float fx = fix_frac(qx), fy = fix_frac(qy), fz = fix_frac(qz);
         // the forward's sample value, bit for bit
-        const int at = cz * g.slice + cy * g.row + cx;
+        const int at = cell_index<LAYOUT>(g, cx, cy, cz);
         const float mu =
             !in_bounds(sample_offset<LAYOUT>(at), sample_extent<LAYOUT>(g), g.vstride) ? 0.0f
+            : LAYOUT == 4 ? sample_brick(vol + at, fx, fy, fz)
             : LAYOUT == 2 ? sample_corners(vol + (size_t)at * 8, fx, fy, fz)
             : LAYOUT == 3 ? sample_quads(vol + (size_t)at * 4, g.slice, fx, fy, fz)
                           : trilinear_at(vol + at, g.row, g.slice, fx, fy, fz);
@@ -684,9 +685,10 @@ alpha_records_kernel(const T* __restrict__ vol_base, const float* __restrict__ R
 #pragma unroll
             for (int a = 0; a < 3; ++a) q[k][a] += s[k][a];
             // the forward's sample value, bit for bit
-            const int at = cz * g.slice + cy * g.row + cx;
+            const int at = cell_index<LAYOUT>(g, cx, cy, cz);
             const float mu =
                 !in_bounds(sample_offset<LAYOUT>(at), sample_extent<LAYOUT>(g), g.vstride) ? 0.0f
+                : LAYOUT == 4 ? sample_brick(vol + at, fx, fy, fz)
                 : LAYOUT == 2 ? sample_corners(vol + (size_t)at * 8, fx, fy, fz)
                 : LAYOUT == 3 ? sample_quads(vol + (size_t)at * 4, g.slice, fx, fy, fz)
                               : trilinear_at(vol + at, g.row, g.slice, fx, fy, fz);
@@ -840,11 +842,13 @@ cudaError_t launch_alpha_adjoint(const void* vol, int dtype, int layout, const G
                                                     n_rec4);
     }
     if (dtype == 0) {
-        if (layout == 3) alpha_kernels<float, 3>(vol, g, Rt, grad_out, fwd_out, grad_vol, ws, stream);
+        if (layout == 4) alpha_kernels<float, 4>(vol, g, Rt, grad_out, fwd_out, grad_vol, ws, stream);
+        else if (layout == 3) alpha_kernels<float, 3>(vol, g, Rt, grad_out, fwd_out, grad_vol, ws, stream);
         else if (layout == 2) alpha_kernels<float, 2>(vol, g, Rt, grad_out, fwd_out, grad_vol, ws, stream);
         else alpha_kernels<float, 0>(vol, g, Rt, grad_out, fwd_out, grad_vol, ws, stream);
     } else {
-        if (layout == 3) alpha_kernels<uint16_t, 3>(vol, g, Rt, grad_out, fwd_out, grad_vol, ws, stream);
+        if (layout == 4) alpha_kernels<uint16_t, 4>(vol, g, Rt, grad_out, fwd_out, grad_vol, ws, stream);
+        else if (layout == 3) alpha_kernels<uint16_t, 3>(vol, g, Rt, grad_out, fwd_out, grad_vol, ws, stream);
         else if (layout == 2) alpha_kernels<uint16_t, 2>(vol, g, Rt, grad_out, fwd_out, grad_vol, ws, stream);
         else alpha_kernels<uint16_t, 0>(vol, g, Rt, grad_out, fwd_out, grad_vol, ws, stream);
     }

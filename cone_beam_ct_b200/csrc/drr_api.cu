@@ -50,19 +50,24 @@ constexpr int kMaxDim = (1 << 22) - 4;   // keeps padded coordinates inside the 
 
 bool known_layout(int layout) {
     return layout == DRR_LAYOUT_LINEAR || layout == DRR_LAYOUT_PADDED ||
-           layout == DRR_LAYOUT_CORNERS || layout == DRR_LAYOUT_QUADS;
+           layout == DRR_LAYOUT_CORNERS || layout == DRR_LAYOUT_QUADS ||
+           layout == DRR_LAYOUT_BRICKS;
 }
 
 int64_t stored_elements(const int dims[3], int layout) {
     if (layout == DRR_LAYOUT_CORNERS)
         return (int64_t)(dims[0] - 1) * (dims[1] - 1) * (dims[2] - 1) * 8;
     if (layout == DRR_LAYOUT_QUADS) return (int64_t)(dims[0] - 1) * (dims[1] - 1) * dims[2] * 4;
+    if (layout == DRR_LAYOUT_BRICKS)
+        return (int64_t)drr::brick_count(dims[0]) * drr::brick_count(dims[1]) *
+               drr::brick_count(dims[2]) * drr::kBrickStride;
     const int pad = layout == DRR_LAYOUT_PADDED ? 2 : 0;
     return (int64_t)(dims[0] + pad) * (dims[1] + pad) * (dims[2] + pad);
 }
 
 size_t layout_alignment(int layout, int dtype) {
-    if (layout == DRR_LAYOUT_CORNERS || layout == DRR_LAYOUT_QUADS) return 16;
+    if (layout == DRR_LAYOUT_CORNERS || layout == DRR_LAYOUT_QUADS || layout == DRR_LAYOUT_BRICKS)
+        return 16;
     return dtype == DRR_F32 ? 4 : 2;
 }
 
@@ -309,7 +314,8 @@ drr_status render_alpha_adjoint(const void* vol, drr_dtype dtype, drr_layout lay
     if (dtype != DRR_F32 && dtype != DRR_BF16) return fail(DRR_ERR_INVALID_ARG, "unknown dtype %d", dtype);
     if (!known_layout(layout)) return fail(DRR_ERR_INVALID_ARG, "unknown layout %d", layout);
     if (layout == DRR_LAYOUT_PADDED)
-        return fail(DRR_ERR_UNSUPPORTED, "the alpha adjoint reads DRR_LAYOUT_LINEAR, _CORNERS or _QUADS volumes");
+        return fail(DRR_ERR_UNSUPPORTED,
+                    "the alpha adjoint reads DRR_LAYOUT_LINEAR, _CORNERS, _QUADS or _BRICKS volumes");
     if (stored_elements(dims, layout) > kMaxElements)
         return fail(DRR_ERR_UNSUPPORTED, "volume too large (max 2^31 - 1 stored elements)");
     const int64_t npix = (int64_t)images * H * W;
@@ -403,7 +409,7 @@ DRR_API drr_status drr_prepare_volume(const float* src, const int dims[3], drr_d
     if (need == 0) return fail(DRR_ERR_UNSUPPORTED, "volume too large (max 2^31 - 1 stored elements)");
     if (!src || !dst) return fail(DRR_ERR_INVALID_ARG, "src and dst must be non-NULL");
     if (!aligned(src, 4) || !aligned(dst, layout_alignment(layout, DRR_F32)))
-        return fail(DRR_ERR_INVALID_ARG, "src must be 4-byte aligned, dst 4-byte (16-byte for DRR_LAYOUT_CORNERS and DRR_LAYOUT_QUADS)");
+        return fail(DRR_ERR_INVALID_ARG, "src must be 4-byte aligned, dst 4-byte (16-byte for DRR_LAYOUT_CORNERS, _QUADS and _BRICKS)");
     if (dst_bytes < need)
         return fail(DRR_ERR_INVALID_ARG, "dst holds %zu bytes, %zu needed", dst_bytes, need);
     const size_t src_bytes = (size_t)dims[0] * dims[1] * dims[2] * 4;

@@ -75,6 +75,27 @@ __device__ __forceinline__ float march_corners(const T* __restrict__ vol, const 
     return acc;
 }
 
+// Sum of the N samples of one ray in the bricked layout: one brick per
+// sample, its 8 corners at constant offsets.  Cells stay in [0, n-2] (g.lim
+// as for the linear layout), inside the stored bricks.
+template <typename T>
+__device__ __forceinline__ float march_bricks(const T* __restrict__ vol, const Geom& g,
+                                              const Ray& ray) {
+    long long qx = ray.q0[0], qy = ray.q0[1], qz = ray.q0[2];
+    const long long sx = ray.s[0], sy = ray.s[1], sz = ray.s[2];
+    float acc = 0.0f;
+#pragma unroll 4
+    for (int i = 0; i < g.N; ++i) {
+        const int e = brick_element(g, fix_cell(qx), fix_cell(qy), fix_cell(qz));
+        if (in_bounds(e, sample_extent<4>(g), g.vstride))
+            acc += sample_brick(vol + e, fix_frac_fs(qx), fix_frac_fs(qy), fix_frac_fs(qz));
+        qx += sx;
+        qy += sy;
+        qz += sz;
+    }
+    return acc;
+}
+
 // Front-to-back alpha compositing of one ray (the over operator; flashdrr
 // rendering API docs, VolumeRaycaster.__init__, use_beer_lambert = False),
 // read as the emission-absorption sum: sample i has opacity
@@ -90,10 +111,11 @@ __device__ __forceinline__ float march_alpha(const T* __restrict__ vol, const Ge
     const long long sx = ray.s[0], sy = ray.s[1], sz = ray.s[2];
     float C = 0.0f, Tr = 1.0f;
     for (int i = 0; i < g.N; ++i) {
-        const int cell = fix_cell(qz) * slice + fix_cell(qy) * row + fix_cell(qx);
+        const int cell = cell_index<LAYOUT>(g, fix_cell(qx), fix_cell(qy), fix_cell(qz));
         const float fx = fix_frac(qx), fy = fix_frac(qy), fz = fix_frac(qz);
         const float mu =
             !in_bounds(sample_offset<LAYOUT>(cell), sample_extent<LAYOUT>(g), g.vstride) ? 0.0f
+            : LAYOUT == 4 ? sample_brick(vol + cell, fx, fy, fz)
             : LAYOUT == 2 ? sample_corners(vol + (size_t)cell * 8, fx, fy, fz)
             : LAYOUT == 3 ? sample_quads(vol + (size_t)cell * 4, slice, fx, fy, fz)
                           : trilinear_at(vol + cell, row, slice, fx, fy, fz);
@@ -126,7 +148,8 @@ __device__ __forceinline__ float march_quads(const T* __restrict__ vol, const Ge
     for (int i = 0; i < g.N; ++i) {
         const int q = fix_cell(qz) * slice + fix_cell(qy) * row + fix_cell(qx);
         if (in_bounds(sample_offset<3>(q), sample_extent<3>(g), g.vstride))
-            acc += sample_quads(vol + (size_t)q * 4, slice, fix_frac(qx), fix_frac(qy), fix_frac(qz));
+            acc += sample_quads(vol + (size_t)q * 4, slice, fix_frac_fs(qx), fix_frac_fs(qy),
+                                fix_frac_fs(qz));
         qx += sx;
         qy += sy;
         qz += sz;
@@ -156,6 +179,7 @@ forward_kernel(const T* __restrict__ vol_base, const float* __restrict__ Rt,
         } else {
             const float sum = LAYOUT == 2   ? march_corners(vol, g, ray)
                               : LAYOUT == 3 ? march_quads(vol, g, ray)
+                              : LAYOUT == 4 ? march_bricks(vol, g, ray)
                                             : march(vol, g, ray);
             const float I = (g.density_factor * ray.dt) * sum;
             result = (MODE == 1) ? -expm1f(-I) : I;
@@ -182,6 +206,7 @@ cudaError_t launch_typed(const void* vol, const Geom& g, const float* Rt, int mo
 template <typename T>
 cudaError_t launch_layout(const void* vol, int layout, const Geom& g, const float* Rt, int mode,
                           float* out, cudaStream_t stream) {
+    if (layout == 4) return launch_typed<T, 4>(vol, g, Rt, mode, out, stream);
     if (layout == 3) return launch_typed<T, 3>(vol, g, Rt, mode, out, stream);
     if (layout == 2) return launch_typed<T, 2>(vol, g, Rt, mode, out, stream);
     if (layout == 1) return launch_typed<T, 1>(vol, g, Rt, mode, out, stream);

@@ -123,6 +123,18 @@ __device__ __forceinline__ float fix_frac(long long q) {
     return __uint_as_float(0x3F800000u | (lo >> 9)) - 1.0f;
 }
 
+// The same value another way: a funnel shift of the pair (0x7F : lo) right
+// by 9 leaves lo's top 23 bits as a mantissa under the exponent of 1.0 (the
+// float 1 + f in one instruction), then the exact subtraction.  Bit for bit
+// fix_frac; which runs faster depends on the loop around it (B200: the
+// xy-quad forward 8-16 % and the brick forward 3 % faster with this one, the
+// corner-record forward 2-22 % and the record adjoint 1 % slower), so each
+// loop uses the one measured faster.
+__device__ __forceinline__ float fix_frac_fs(long long q) {
+    const unsigned lo = (unsigned)(unsigned long long)q;
+    return __uint_as_float(__funnelshift_r(lo, 0x7Fu, 9)) - 1.0f;
+}
+
 __device__ __forceinline__ int fix_cell(long long q) { return (int)(q >> 32); }
 
 // Returns false for a miss (or a ray whose geometry is not finite).
@@ -221,12 +233,49 @@ __device__ __forceinline__ constexpr bool in_bounds(long long, long long, long l
 #define DRR_BOUNDS_READER(name)
 #endif
 
+// Bricked layout (4): the cells in bricks of kBrick^3; brick (bx, by, bz)
+// stores the voxels (kBrick bx + lx, kBrick by + ly, kBrick bz + lz) for lx,
+// ly, lz in [0, kBrick] -- its cells' corners, the last plane of each axis
+// shared with the next brick (a one-voxel apron) -- x fastest, padded to
+// kBrickStride elements (a multiple of 16 bytes for fp32 and bf16).  A cell's
+// 8 corners then lie in one brick, at the constant offsets a + kBrickEdge b
+// + kBrickPlane c, and a brick (2.9 KB fp32) is one contiguous block.  Brick
+// (bx, by, bz) is number (bz * nby + by) * nbx + bx; in Geom, row = nbx and
+// slice = nbx * nby.
+constexpr int kBrick = 8;
+constexpr int kBrickEdge = kBrick + 1;
+constexpr int kBrickPlane = kBrickEdge * kBrickEdge;
+constexpr int kBrickStride = 736;          // 729 voxels, padded
+static_assert(kBrickStride >= kBrickPlane * kBrickEdge && kBrickStride % 8 == 0, "brick stride");
+
+// bricks along an axis of n voxels (n - 1 cells)
+__host__ __device__ __forceinline__ int brick_count(int n) { return (n - 1 + kBrick - 1) / kBrick; }
+
+// element of corner (0, 0, 0) of cell (cx, cy, cz) in the bricked layout
+__device__ __forceinline__ int brick_element(const Geom& g, int cx, int cy, int cz) {
+    const int brick = (cz >> 3) * g.slice + (cy >> 3) * g.row + (cx >> 3);
+    const int local = ((cz & 7) * kBrickEdge + (cy & 7)) * kBrickEdge + (cx & 7);
+    return brick * kBrickStride + local;
+}
+static_assert(kBrick == 8, "brick_element shifts by 3");
+
+// Index of cell (cx, cy, cz) in each stored layout (0 linear, 1 zero-bordered,
+// 2 corner records, 3 xy quads, 4 bricks): a cell, record or quad number,
+// or for bricks the element of its first corner.
+template <int LAYOUT>
+__device__ __forceinline__ int cell_index(const Geom& g, int cx, int cy, int cz) {
+    if constexpr (LAYOUT == 4) return brick_element(g, cx, cy, cz);
+    return cz * g.slice + cy * g.row + cx;
+}
+
 // Elements one trilinear sample reads, from the offset of its cell's first
-// element, in each stored layout (0 linear, 1 zero-bordered, 2 corner
-// records, 3 xy quads), and that offset for cell index `cell`.
+// element, in each stored layout, and that offset for cell index `cell`.
 template <int LAYOUT>
 __host__ __device__ __forceinline__ long long sample_extent(const Geom& g) {
-    return LAYOUT == 2 ? 8 : LAYOUT == 3 ? 4LL * g.slice + 4 : (long long)g.slice + g.row + 2;
+    return LAYOUT == 2   ? 8
+           : LAYOUT == 3 ? 4LL * g.slice + 4
+           : LAYOUT == 4 ? (long long)kBrickPlane + kBrickEdge + 2
+                         : (long long)g.slice + g.row + 2;
 }
 template <int LAYOUT>
 __host__ __device__ __forceinline__ long long sample_offset(long long cell) {
@@ -247,7 +296,7 @@ __device__ __forceinline__ void tile_pixel(int& r, int& c) {
 // host side
 
 // Kernel parameter block from validated host arguments.  layout: 0 linear,
-// 1 zero-bordered, 2 corner records, 3 xy quads (include/drr.h).  K^-1 of the upper
+// 1 zero-bordered, 2 corner records, 3 xy quads, 4 bricks (include/drr.h).  K^-1 of the upper
 // triangular K in double.
 inline void fill_geom(Geom& g, const int dims[3], const float spacing[3], const float origin[3],
                       const float K[9], int B, int H, int W, int n_samples, float density_factor,
@@ -259,6 +308,9 @@ inline void fill_geom(Geom& g, const int dims[3], const float spacing[3], const 
     if (layout == 2 || layout == 3) {       // strides of cells (8 elements) or quads (4)
         g.row = dims[0] - 1;
         g.slice = (dims[0] - 1) * (dims[1] - 1);
+    } else if (layout == 4) {               // bricks per row and per slice of bricks
+        g.row = brick_count(dims[0]);
+        g.slice = brick_count(dims[0]) * brick_count(dims[1]);
     } else {
         const int pad = layout == 1 ? 2 : 0;
         g.row = dims[0] + pad;

@@ -39,8 +39,8 @@ __device__ __forceinline__ float widen(uint16_t v) { return __uint_as_float((uin
 template <typename T, int LAYOUT>
 __device__ __forceinline__ void cell_corners(const T* __restrict__ vol, const Geom& g, int cx,
                                              int cy, int cz, float v[8]) {
-    if (!in_bounds(sample_offset<LAYOUT>(cz * g.slice + cy * g.row + cx), sample_extent<LAYOUT>(g),
-                   g.vstride)) {
+    if (!in_bounds(sample_offset<LAYOUT>(cell_index<LAYOUT>(g, cx, cy, cz)),
+                   sample_extent<LAYOUT>(g), g.vstride)) {
 #pragma unroll
         for (int e = 0; e < 8; ++e) v[e] = 0.0f;
         return;
@@ -61,6 +61,12 @@ __device__ __forceinline__ void cell_corners(const T* __restrict__ vol, const Ge
                 v[2 * m + 1] = __uint_as_float(words[m] & 0xFFFF0000u);
             }
         }
+    } else if (LAYOUT == 4) {
+        const T* p = vol + brick_element(g, cx, cy, cz);
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+            v[e] = widen(__ldg(p + ((e & 1) ? 1 : 0) + ((e & 2) ? kBrickEdge : 0) +
+                               ((e & 4) ? kBrickPlane : 0)));
     } else if (LAYOUT == 3) {
         const T* p = vol + (size_t)(cz * g.slice + cy * g.row + cx) * 4;
         load_quad(p, v);
@@ -364,6 +370,7 @@ template <typename T>
 cudaError_t launch_layout(const void* vol, int layout, const Geom& g, const float* Rt, int mode,
                           const float* grad_out, const float* fwd_out, float* grad_Rt,
                           cudaStream_t stream) {
+    if (layout == 4) return launch_typed<T, 4>(vol, g, Rt, mode, grad_out, fwd_out, grad_Rt, stream);
     if (layout == 3) return launch_typed<T, 3>(vol, g, Rt, mode, grad_out, fwd_out, grad_Rt, stream);
     if (layout == 2) return launch_typed<T, 2>(vol, g, Rt, mode, grad_out, fwd_out, grad_Rt, stream);
     if (layout == 1) return launch_typed<T, 1>(vol, g, Rt, mode, grad_out, fwd_out, grad_Rt, stream);

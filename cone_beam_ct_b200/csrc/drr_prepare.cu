@@ -129,6 +129,32 @@ int grid_for(int64_t n) {
     return (int)(blocks < cap ? (blocks > 0 ? blocks : 1) : cap);
 }
 
+// Bricked layout: element m of the output is element m % kBrickStride of
+// brick m / kBrickStride; a brick's elements past its (kBrick + 1)^3 voxels,
+// and voxels past the volume's edge, are zero.
+template <typename T>
+__global__ void to_bricks(const float* __restrict__ src, T* __restrict__ dst, int nx, int ny,
+                          int nz) {
+    const int nbx = brick_count(nx), nby = brick_count(ny);
+    const int64_t n = (int64_t)nbx * nby * brick_count(nz) * kBrickStride;
+    for (int64_t m = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; m < n;
+         m += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t brick = m / kBrickStride;
+        const int e = (int)(m - brick * kBrickStride);
+        float v = 0.0f;
+        if (e < kBrickPlane * kBrickEdge) {
+            const int lz = e / kBrickPlane, ly = (e / kBrickEdge) % kBrickEdge, lx = e % kBrickEdge;
+            const int bx = (int)(brick % nbx), by = (int)((brick / nbx) % nby);
+            const int bz = (int)(brick / ((int64_t)nbx * nby));
+            const int i = bx * kBrick + lx, j = by * kBrick + ly, k = bz * kBrick + lz;
+            const int64_t at = ((int64_t)k * ny + j) * nx + i;
+            if (i < nx && j < ny && k < nz && in_bounds(at, 1, (int64_t)nx * ny * nz))
+                v = __ldg(src + at);
+        }
+        dst[m] = store_value<T>(v);
+    }
+}
+
 }  // namespace
 
 DRR_BOUNDS_READER(bounds_word_prepare)
@@ -142,6 +168,15 @@ cudaError_t launch_prepare(const float* src, int nx, int ny, int nz, int dtype, 
         else
             to_linear<uint16_t><<<grid_for(n), 256, 0, stream>>>(src, static_cast<uint16_t*>(dst),
                                                                  n);
+    } else if (layout == 4) {
+        const int64_t n =
+            (int64_t)brick_count(nx) * brick_count(ny) * brick_count(nz) * kBrickStride;
+        if (dtype == 0)
+            to_bricks<float><<<grid_for(n), 256, 0, stream>>>(src, static_cast<float*>(dst), nx,
+                                                              ny, nz);
+        else
+            to_bricks<uint16_t><<<grid_for(n), 256, 0, stream>>>(src, static_cast<uint16_t*>(dst),
+                                                                 nx, ny, nz);
     } else if (layout == 3) {
         const int64_t n = (int64_t)(nx - 1) * (ny - 1) * nz;
         if (dtype == 0)

@@ -11,6 +11,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "drr_internal.cuh"
+
 namespace drr {
 namespace {
 
@@ -141,6 +143,15 @@ __device__ __forceinline__ float sample_quads(const T* __restrict__ p, int slice
     const float c0 = fmaf(fy, c10 - c00, c00);
     const float c1 = fmaf(fy, c11 - c01, c01);
     return fmaf(fz, c1 - c0, c0);
+}
+
+// One sample in the bricked layout: the 8 corners in one brick at constant
+// offsets (kBrickEdge voxels per row, kBrickPlane per plane); the linear
+// layout's loads and lerps.
+template <typename T>
+__device__ __forceinline__ float sample_brick(const T* __restrict__ p, float fx, float fy,
+                                              float fz) {
+    return trilinear_at(p, kBrickEdge, kBrickPlane, fx, fy, fz);
 }
 
 }  // namespace

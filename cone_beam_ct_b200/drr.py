@@ -20,6 +20,7 @@ DRR_OK, DRR_ERR_INVALID_ARG, DRR_ERR_UNSUPPORTED, DRR_ERR_CUDA = 0, 1, 2, 3
 DRR_MODE_RAW, DRR_MODE_BEER_LAMBERT, DRR_MODE_ALPHA = 0, 1, 2
 DRR_F32, DRR_BF16 = 0, 1
 DRR_LAYOUT_LINEAR, DRR_LAYOUT_PADDED, DRR_LAYOUT_CORNERS, DRR_LAYOUT_QUADS = 0, 1, 2, 3
+DRR_LAYOUT_BRICKS = 4
 
 # names exported by libdrr.so (include/drr.h)
 EXPORTED = ("drr_render", "drr_render_adjoint", "drr_render_adjoint_ws",

@@ -6,8 +6,8 @@ import numpy as np
 from cone_beam_ct_b200 import drr
 
 LINEAR, PADDED, CORNERS = drr.DRR_LAYOUT_LINEAR, drr.DRR_LAYOUT_PADDED, drr.DRR_LAYOUT_CORNERS
-QUADS = drr.DRR_LAYOUT_QUADS
-LAYOUTS = (LINEAR, PADDED, CORNERS, QUADS)
+QUADS, BRICKS = drr.DRR_LAYOUT_QUADS, drr.DRR_LAYOUT_BRICKS
+LAYOUTS = (LINEAR, PADDED, CORNERS, QUADS, BRICKS)
 F32, BF16 = drr.DRR_F32, drr.DRR_BF16
 
 

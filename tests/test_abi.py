@@ -561,6 +561,12 @@ def test_prepared_bytes():
     assert drr.drr_prepared_bytes((5, 6, 7), drr.DRR_BF16, drr.DRR_LAYOUT_QUADS) == 2 * 4 * 4 * 5 * 7
     assert drr.drr_prepared_bytes((1024, 1024, 512), drr.DRR_F32, drr.DRR_LAYOUT_QUADS) == \
         4 * 4 * 1023 * 1023 * 512
+    # bricks of 8^3 cells, 736 elements each: ceil((n - 1) / 8) per axis
+    assert drr.drr_prepared_bytes((256, 256, 256), drr.DRR_F32, drr.DRR_LAYOUT_BRICKS) == \
+        4 * 736 * 32 ** 3
+    assert drr.drr_prepared_bytes((9, 10, 17), drr.DRR_BF16, drr.DRR_LAYOUT_BRICKS) == \
+        2 * 736 * 1 * 2 * 2
+    assert drr.drr_prepared_bytes((2, 2, 2), drr.DRR_F32, drr.DRR_LAYOUT_BRICKS) == 4 * 736
 
 
 PREPARE_BAD = [
@@ -574,6 +580,7 @@ PREPARE_BAD = [
     (dict(src=FAKE + 2), drr.DRR_ERR_INVALID_ARG),       # misaligned
     (dict(layout=drr.DRR_LAYOUT_CORNERS, dst=FAKE + (1 << 24) + 8), drr.DRR_ERR_INVALID_ARG),
     (dict(layout=drr.DRR_LAYOUT_QUADS, dst=FAKE + (1 << 24) + 8), drr.DRR_ERR_INVALID_ARG),
+    (dict(layout=drr.DRR_LAYOUT_BRICKS, dst=FAKE + (1 << 24) + 8), drr.DRR_ERR_INVALID_ARG),
     (dict(dims=(2048, 2048, 1024)), drr.DRR_ERR_UNSUPPORTED),
 ]
 

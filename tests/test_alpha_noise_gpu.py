@@ -20,7 +20,7 @@ import pytest
 import oracle
 from cone_beam_ct_b200 import drr
 from cone_beam_ct_b200 import workloads as wl
-from tests.gpu_helpers import (BF16, CORNERS, F32, LAYOUTS, LINEAR, QUADS, assert_parity, bf16_values,
+from tests.gpu_helpers import (BF16, BRICKS, CORNERS, F32, LAYOUTS, LINEAR, QUADS, assert_parity, bf16_values,
                                gpu_alpha_adjoint, gpu_forward)
 
 pytestmark = pytest.mark.gpu
@@ -75,7 +75,8 @@ def test_alpha_forward_config2_views(cuda):
 
 @pytest.mark.parametrize("seed", [411, 412])
 @pytest.mark.parametrize("layout,dtype", [(LINEAR, F32), (CORNERS, F32), (QUADS, F32),
-                                          (LINEAR, BF16), (CORNERS, BF16), (QUADS, BF16)])
+                                          (BRICKS, F32), (LINEAR, BF16), (CORNERS, BF16),
+                                          (QUADS, BF16), (BRICKS, BF16)])
 def test_alpha_adjoint_small_ragged(cuda, seed, layout, dtype):
     w = wl.small_random_case(seed)
     w.density_factor = 25.0
@@ -94,7 +95,7 @@ DENSE = dict(dims=(23, 17, 29), H=150, W=170, n_samples=40)
 
 
 @pytest.mark.parametrize("layout,dtype", [(LINEAR, F32), (CORNERS, BF16), (QUADS, F32),
-                                          (QUADS, BF16)])
+                                          (QUADS, BF16), (BRICKS, F32)])
 def test_alpha_adjoint_dense_views_take_the_record_path(cuda, layout, dtype):
     w = wl.small_random_case(421, **DENSE)
     w.density_factor = 25.0

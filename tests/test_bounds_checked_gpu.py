@@ -72,7 +72,7 @@ def test_adjoints_and_pose_gradient_stay_in_bounds(checked, case):
                 H.gpu_pose_grad(w, go, layout=layout, dtype=dtype, mode=mode, fwd_out=fwd)
                 _clean(checked, f"pose gradient layout {layout} dtype {dtype} mode {mode}")
     alpha = H.gpu_forward(w, layout=H.LINEAR, dtype=H.F32, mode=wl.MODE_ALPHA)
-    for layout in (H.LINEAR, H.CORNERS, H.QUADS):
+    for layout in (H.LINEAR, H.CORNERS, H.QUADS, H.BRICKS):
         for workspace in (False, True):
             H.gpu_alpha_adjoint(w, go, alpha, layout=layout, dtype=H.F32, workspace=workspace)
             _clean(checked, f"alpha adjoint layout {layout} workspace {workspace}")

@@ -16,7 +16,7 @@ import pytest
 
 import oracle
 from cone_beam_ct_b200 import workloads as wl
-from tests.gpu_helpers import (BF16, CORNERS, F32, LAYOUTS, LINEAR, PADDED, QUADS, assert_parity,
+from tests.gpu_helpers import (BF16, BRICKS, CORNERS, F32, LAYOUTS, LINEAR, PADDED, QUADS, assert_parity,
                                bf16_values, gpu_forward)
 
 pytestmark = pytest.mark.gpu
@@ -217,6 +217,21 @@ def test_prepare_layouts_round_trip(cuda):
                 border = p.copy()
                 border[1:-1, 1:-1, 1:-1] = 0
                 assert np.all(border == 0)
+            elif layout == BRICKS:
+                # voxel (8bx + lx, 8by + ly, 8bz + lz) of brick (bx, by, bz) at element
+                # (lz * 9 + ly) * 9 + lx of a 736-element block, zero elsewhere
+                nb = [-(-(n - 1) // 8) for n in (nx, ny, nz)]
+                blocks = a.reshape(nb[2], nb[1], nb[0], 736)
+                assert np.all(blocks[..., 729:] == 0)
+                cube = blocks[..., :729].reshape(nb[2], nb[1], nb[0], 9, 9, 9)
+                full = np.zeros((8 * nb[2] + 1, 8 * nb[1] + 1, 8 * nb[0] + 1), a.dtype)
+                full[:nz, :ny, :nx] = expect
+                for bz in range(nb[2]):
+                    for by in range(nb[1]):
+                        for bx in range(nb[0]):
+                            assert np.array_equal(cube[bz, by, bx],
+                                                  full[8 * bz:8 * bz + 9, 8 * by:8 * by + 9,
+                                                       8 * bx:8 * bx + 9])
             elif layout == QUADS:
                 # voxel (i + a, j + b, k) of quad (i, j, k) at element a + 2b
                 rec = a.reshape(nz, ny - 1, nx - 1, 4)
