@@ -707,6 +707,29 @@ def siddon_timing(torch, w, vol32, Rt, grad_out, l2_peak, hbm_peak):
                         "roofline": roof("siddon_adjoint_kernel", adj_ms)}}
 
 
+def bricks_timing(torch, w, vol32, Rt, dtype, mode):
+    """The bricked layout's forward (drr_render) and the same with each frustum
+    layer staged in shared memory by bulk copies (drr_render_staged, the
+    measured comparison): median of 5 each, L2 flushed before each."""
+    from cone_beam_ct_b200 import drr
+    dev = vol32.device
+    nbytes = drr.drr_prepared_bytes(w.dims, dtype, drr.DRR_LAYOUT_BRICKS)
+    bricks = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    drr.drr_prepare_volume(vol32, w.dims, dtype, drr.DRR_LAYOUT_BRICKS, bricks, nbytes)
+    out = torch.empty((w.B, w.H, w.W), dtype=torch.float32, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    mode = 0 if mode == 2 else mode
+    plain = _median_ms(torch, lambda: drr.drr_render(
+        bricks, dtype, drr.DRR_LAYOUT_BRICKS, w.dims, w.spacing, w.origin, w.K, Rt, w.B, w.H,
+        w.W, w.n_samples, w.density_factor, mode, out), reps=5, flush=flush)
+    staged = _median_ms(torch, lambda: drr.drr_render_staged(
+        bricks, dtype, w.dims, w.spacing, w.origin, w.K, Rt, w.B, w.H, w.W, w.n_samples,
+        w.density_factor, mode, out), reps=5, flush=flush)
+    return {"bytes": nbytes, "forward_ms": plain, "staged_forward_ms": staged,
+            "gsamples_s": w.samples / (plain * 1e-3) / 1e9,
+            "staged_gsamples_s": w.samples / (staged * 1e-3) / 1e9}
+
+
 # the workloads of the configs block: the other four, config 5 being the
 # adjoint of config 2's geometry (RAW, its own seeded N(0, 1) upstream)
 OTHER_CONFIGS = {3: (1, 2, 4, 5), 1: (2, 3, 4, 5), 2: (1, 3, 4, 5), 4: (1, 2, 3, 5)}
@@ -771,6 +794,8 @@ def config_timing(torch, cfg, hbm_peak, l2_cache):
                                8 * elem * w.samples)
     res["adjoint"] = entry(ADJOINT_GROUP, _median_ms(torch, adj, reps=5, flush=flush),
                            32 * w.samples)
+    if cfg != 5:
+        res["bricks"] = bricks_timing(torch, w, vol32, Rt, dtype, mode)
     if cfg == 5:
         res["workload"] = (f"adjoint of the {nx}^3 / {w.B}-view {w.H}x{w.W} / "
                            f"{w.n_samples}-sample geometry, N(0,1) upstream, RAW")
@@ -992,6 +1017,10 @@ def run_ours(args):
         configs = {str(c): config_timing(torch, c, hbm_peak, l2_cache)
                    for c in OTHER_CONFIGS[args.config]}
 
+    bricks = None
+    if extras:
+        bricks = bricks_timing(torch, w, vol32, Rt, dtype, w.mode)
+
     tex = None
     if args.texture:
         tex = texture_comparison(torch, w, vol32, Rt, out)
@@ -1023,6 +1052,7 @@ def run_ours(args):
         "siddon": siddon,
         "batched": batched,
         "configs": configs,
+        "bricks": bricks,
         "gpu_launches": 7 * args.steps,   # prepare, forward, plan, zero, 2 adjoint paths, gather
         "clocks": clocks,
         "bracket_ms": bracket[0].elapsed_time(bracket[1]),

@@ -39,4 +39,5 @@ from .drr import (  # noqa: F401
     drr_render_pose_grad_batched,
     drr_render_siddon,
     drr_render_siddon_adjoint,
+    drr_render_staged,
 )

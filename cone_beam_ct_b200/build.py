@@ -13,8 +13,8 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 LIB = os.path.join(HERE, "libdrr.so")
 PROBE_LIB = os.path.join(HERE, "libdrr_probe.so")
-SOURCES = ["drr_api.cu", "drr_forward.cu", "drr_adjoint.cu", "drr_prepare.cu", "drr_pose.cu", "drr_noise.cu",
-           "drr_siddon.cu"]
+SOURCES = ["drr_api.cu", "drr_forward.cu", "drr_staged.cu", "drr_adjoint.cu", "drr_prepare.cu",
+           "drr_pose.cu", "drr_noise.cu", "drr_siddon.cu"]
 HEADERS = ["drr_internal.cuh", "drr_sample.cuh"]
 PROBE_SOURCES = ["drr_probe.cu"]
 # the same sources with every gather and scatter range-checked (include/drr_debug.h)

@@ -367,7 +367,8 @@ DRR_API drr_status drr_debug_bounds_errors(unsigned long long* count, long long*
     if (!count || !first) return fail(DRR_ERR_INVALID_ARG, "count and first must be non-NULL");
     cudaError_t (*const readers[])(drr::BoundsWord*) = {
         drr::bounds_word_forward, drr::bounds_word_adjoint, drr::bounds_word_pose,
-        drr::bounds_word_siddon,  drr::bounds_word_prepare, drr::bounds_word_noise};
+        drr::bounds_word_siddon,  drr::bounds_word_prepare, drr::bounds_word_noise,
+        drr::bounds_word_staged};
     *count = 0;
     *first = 0;
     for (auto read : readers) {
@@ -426,6 +427,35 @@ DRR_API drr_status drr_render(const void* vol, drr_dtype dtype, drr_layout layou
                               void* stream) {
     return render_batched(vol, dtype, layout, dims, spacing, origin, K, Rt, 1, 1, B, H, W,
                           n_samples, density_factor, mode, out, stream);
+}
+
+DRR_API drr_status drr_render_staged(const void* vol, drr_dtype dtype, const int dims[3],
+                                     const float spacing[3], const float origin[3],
+                                     const float K[9], const float* Rt, int B, int H, int W,
+                                     int n_samples, float density_factor, drr_mode mode,
+                                     float* out, void* stream) {
+    if (mode == DRR_MODE_ALPHA)
+        return fail(DRR_ERR_UNSUPPORTED,
+                    "drr_render_staged integrates (raw or Beer-Lambert); alpha compositing: drr_render");
+    drr_status st = check_volume(dims, spacing, origin);
+    if (st != DRR_OK) return st;
+    st = check_rays(K, Rt, B, H, W, n_samples, density_factor, mode);
+    if (st != DRR_OK) return st;
+    if (dtype != DRR_F32 && dtype != DRR_BF16) return fail(DRR_ERR_INVALID_ARG, "unknown dtype %d", dtype);
+    if (stored_elements(dims, DRR_LAYOUT_BRICKS) > kMaxElements)
+        return fail(DRR_ERR_UNSUPPORTED, "volume too large (max 2^31 - 1 stored elements)");
+    if ((int64_t)B * H * W == 0) return ok();
+    if (!vol || !aligned(vol, 16))
+        return fail(DRR_ERR_INVALID_ARG, "vol must be a non-NULL, 16-byte aligned device pointer");
+    if (!out || !aligned(out, 4))
+        return fail(DRR_ERR_INVALID_ARG, "out must be a non-NULL, 4-byte aligned device pointer");
+    drr::Geom g;
+    drr::fill_geom(g, dims, spacing, origin, K, B, H, W, n_samples, density_factor,
+                   DRR_LAYOUT_BRICKS);
+    g.vstride = stored_elements(dims, DRR_LAYOUT_BRICKS);
+    return cuda_status(drr::launch_forward_staged(vol, dtype, g, Rt, mode, out,
+                                                  static_cast<cudaStream_t>(stream)),
+                       "drr_render_staged launch");
 }
 
 DRR_API drr_status drr_render_batched(const void* vols, drr_dtype dtype, drr_layout layout,

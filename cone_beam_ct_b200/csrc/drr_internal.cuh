@@ -348,6 +348,10 @@ inline void fill_geom(Geom& g, const int dims[3], const float spacing[3], const 
 
 cudaError_t launch_forward(const void* vol, int dtype, int layout, const Geom& g,
                            const float* Rt, int mode, float* out, cudaStream_t stream);
+// the bricked layout's forward with each frustum layer's bricks staged in
+// shared memory by bulk copies (drr_staged.cu; raw and Beer-Lambert modes)
+cudaError_t launch_forward_staged(const void* vol, int dtype, const Geom& g, const float* Rt,
+                                  int mode, float* out, cudaStream_t stream);
 cudaError_t launch_adjoint(const Geom& g, const float* Rt, int mode, const float* grad_out,
                            const float* fwd_out, float* grad_vol, void* workspace,
                            cudaStream_t stream);
@@ -382,6 +386,7 @@ cudaError_t bounds_word_pose(BoundsWord* out);
 cudaError_t bounds_word_siddon(BoundsWord* out);
 cudaError_t bounds_word_prepare(BoundsWord* out);
 cudaError_t bounds_word_noise(BoundsWord* out);
+cudaError_t bounds_word_staged(BoundsWord* out);
 #endif
 
 cudaError_t launch_pose_grad(const void* vol, int dtype, int layout, const Geom& g,

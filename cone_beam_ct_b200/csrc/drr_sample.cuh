@@ -30,17 +30,27 @@ __device__ __forceinline__ float load_voxel<uint16_t>(const uint16_t* p) {
     return __uint_as_float(((uint32_t)__ldg(reinterpret_cast<const unsigned short*>(p))) << 16);
 }
 
-template <typename T>
+// A voxel read with an ordinary load, from any state space (__ldg is a
+// global-memory load: a shared-memory address is not valid for it).
+__device__ __forceinline__ float load_voxel_any(const float* p) { return *p; }
+__device__ __forceinline__ float load_voxel_any(const uint16_t* p) {
+    return __uint_as_float(((uint32_t)*p) << 16);
+}
+
+// GLOBAL: the volume is in global memory (read through the read-only path);
+// else anywhere, shared memory included.  The same lerps either way.
+template <typename T, bool GLOBAL = true>
 __device__ __forceinline__ float trilinear_at(const T* __restrict__ base, int row, int slice,
                                               float fx, float fy, float fz) {
-    const float v000 = load_voxel(base);
-    const float v100 = load_voxel(base + 1);
-    const float v010 = load_voxel(base + row);
-    const float v110 = load_voxel(base + row + 1);
-    const float v001 = load_voxel(base + slice);
-    const float v101 = load_voxel(base + slice + 1);
-    const float v011 = load_voxel(base + slice + row);
-    const float v111 = load_voxel(base + slice + row + 1);
+    auto ld = [](const T* p) { return GLOBAL ? load_voxel(p) : load_voxel_any(p); };
+    const float v000 = ld(base);
+    const float v100 = ld(base + 1);
+    const float v010 = ld(base + row);
+    const float v110 = ld(base + row + 1);
+    const float v001 = ld(base + slice);
+    const float v101 = ld(base + slice + 1);
+    const float v011 = ld(base + slice + row);
+    const float v111 = ld(base + slice + row + 1);
     const float c00 = fmaf(fx, v100 - v000, v000);
     const float c10 = fmaf(fx, v110 - v010, v010);
     const float c01 = fmaf(fx, v101 - v001, v001);
@@ -148,10 +158,10 @@ __device__ __forceinline__ float sample_quads(const T* __restrict__ p, int slice
 // One sample in the bricked layout: the 8 corners in one brick at constant
 // offsets (kBrickEdge voxels per row, kBrickPlane per plane); the linear
 // layout's loads and lerps.
-template <typename T>
+template <typename T, bool GLOBAL = true>
 __device__ __forceinline__ float sample_brick(const T* __restrict__ p, float fx, float fy,
                                               float fz) {
-    return trilinear_at(p, kBrickEdge, kBrickPlane, fx, fy, fz);
+    return trilinear_at<T, GLOBAL>(p, kBrickEdge, kBrickPlane, fx, fy, fz);
 }
 
 }  // namespace

@@ -29,7 +29,7 @@ EXPORTED = ("drr_render", "drr_render_adjoint", "drr_render_adjoint_ws",
             "drr_render_siddon", "drr_render_siddon_adjoint", "drr_render_batched",
             "drr_render_adjoint_batched", "drr_adjoint_batched_workspace_bytes",
             "drr_render_pose_grad_batched", "drr_render_alpha_adjoint_batched",
-            "drr_render_adjoint_batched_ws",
+            "drr_render_adjoint_batched_ws", "drr_render_staged",
             "drr_prepared_bytes", "drr_prepare_volume", "drr_get_last_error", "drr_abi_version")
 DRR_NOALLOC_SCRATCH_BYTES = 32 << 20
 
@@ -71,6 +71,9 @@ def lib():
     L.drr_render.argtypes = [_vp, _c.c_int, _c.c_int, _i3, _f3, _f3, _f9, _vp, _c.c_int,
                              _c.c_int, _c.c_int, _c.c_int, _c.c_float, _c.c_int, _vp, _vp]
     L.drr_render.restype = _c.c_int
+    L.drr_render_staged.argtypes = [_vp, _c.c_int, _i3, _f3, _f3, _f9, _vp, _c.c_int, _c.c_int,
+                                    _c.c_int, _c.c_int, _c.c_float, _c.c_int, _vp, _vp]
+    L.drr_render_staged.restype = _c.c_int
     L.drr_render_adjoint.argtypes = [_i3, _f3, _f3, _f9, _vp, _c.c_int, _c.c_int, _c.c_int,
                                      _c.c_int, _c.c_float, _c.c_int, _vp, _vp, _vp, _vp]
     L.drr_render_adjoint.restype = _c.c_int
@@ -219,6 +222,14 @@ def drr_render(vol, dtype, layout, dims, spacing, origin, K, Rt, B, H, W, n_samp
                             _f3v(spacing), _f3v(origin), _f9v(K), _dev(Rt, "Rt", True), int(B),
                             int(H), int(W), int(n_samples), float(density_factor), int(mode),
                             _dev(out, "out", True), _stream(stream)))
+
+
+def drr_render_staged(vol, dtype, dims, spacing, origin, K, Rt, B, H, W, n_samples,
+                      density_factor, mode, out, stream=None):
+    _check(lib().drr_render_staged(_dev(vol, "vol", True), int(dtype), _i3v(dims), _f3v(spacing),
+                                   _f3v(origin), _f9v(K), _dev(Rt, "Rt", True), int(B), int(H),
+                                   int(W), int(n_samples), float(density_factor), int(mode),
+                                   _dev(out, "out", True), _stream(stream)))
 
 
 def drr_render_adjoint(dims, spacing, origin, K, Rt, B, H, W, n_samples, density_factor, mode,

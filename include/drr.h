@@ -154,6 +154,31 @@ DRR_API drr_status drr_render(const void *vol, drr_dtype dtype, drr_layout layou
                               int n_samples, float density_factor, drr_mode mode, float *out,
                               void *stream);
 
+/* drr_render of a DRR_LAYOUT_BRICKS volume with each layer of a tile's
+ * frustum staged in shared memory: the volume layout's optional staging of
+ * bricks for narrow frusta.  A CTA renders a 16 x 16 pixel tile; where its
+ * rays are sparse (the tile spans 8 voxels or more at the volume centre) it
+ * walks the tile's pyramid one layer of 8^3-cell bricks at a time along the
+ * major axis of its central ray, copying the layer's bricks (at most 16;
+ * the window comes from the tile's corner rays) from global into shared
+ * memory with bulk copies of the Tensor Memory Accelerator while the rays
+ * sample the previous layer; denser tiles read global memory.  The result
+ * is bit for bit drr_render's with DRR_LAYOUT_BRICKS (and DRR_LAYOUT_LINEAR).
+ * Measured on B200 it is slower than drr_render's bricked forward on every
+ * workload of this library's benchmark (one barrier per layer hides too
+ * little copy latency at 2 CTAs per SM), so drr_render does not use it; it
+ * is kept as the measured comparison.
+ *   vol         DEVICE, DRR_LAYOUT_BRICKS as written by drr_prepare_volume,
+ *               16-byte aligned.
+ *   mode        DRR_MODE_RAW or DRR_MODE_BEER_LAMBERT (alpha:
+ *               DRR_ERR_UNSUPPORTED).
+ * Other arguments, limits and errors as drr_render. */
+DRR_API drr_status drr_render_staged(const void *vol, drr_dtype dtype, const int dims[3],
+                                     const float spacing[3], const float origin[3],
+                                     const float K[9], const float *Rt, int B, int H, int W,
+                                     int n_samples, float density_factor, drr_mode mode,
+                                     float *out, void *stream);
+
 /* Adjoint (transpose) of drr_render with respect to the volume, i.e. the
  * volume gradient of sum(grad_out * out).
  *   grad_out    DEVICE float[B*H*W], upstream gradient dL/d(out).

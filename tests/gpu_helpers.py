@@ -45,6 +45,21 @@ def gpu_forward(w, layout=PADDED, dtype=None, mode=None, vol=None, Rt=None):
     return out.cpu().numpy()
 
 
+def gpu_forward_staged(w, dtype=None, mode=None):
+    """drr_render_staged: the bricked forward with each frustum layer staged in
+    shared memory."""
+    import torch
+    dtype = w.dtype if dtype is None else dtype
+    mode = w.mode if mode is None else mode
+    v32, Rt_d = device_inputs(w)
+    src = prepared(v32, w.dims, dtype, BRICKS)
+    out = torch.full((w.B, w.H, w.W), float("nan"), dtype=torch.float32, device="cuda")
+    drr.drr_render_staged(src, dtype, w.dims, w.spacing, w.origin, w.K, Rt_d, w.B, w.H, w.W,
+                          w.n_samples, w.density_factor, mode, out)
+    torch.cuda.synchronize()
+    return out.cpu().numpy()
+
+
 def gpu_adjoint(w, grad_out, mode=None, fwd_out=None, workspace=False):
     """Volume gradient through drr_render_adjoint, or drr_render_adjoint_ws
     with a fresh workspace (filled with garbage first: its content on entry

@@ -151,6 +151,38 @@ ADJOINT_BAD = [
 ]
 
 
+def _staged(**kw):
+    args = dict(vol=FAKE, dtype=drr.DRR_F32, dims=DIMS, spacing=SP, origin=ORG, K=K_OK,
+                Rt=FAKE + (1 << 26), B=2, H=8, W=8, n_samples=16, density_factor=1.0,
+                mode=drr.DRR_MODE_RAW, out=FAKE + (1 << 27), stream=0)
+    args.update(kw)
+    return drr.drr_render_staged(**args)
+
+
+STAGED_BAD = [
+    (dict(vol=0), drr.DRR_ERR_INVALID_ARG, "vol"),
+    (dict(vol=FAKE + 8), drr.DRR_ERR_INVALID_ARG, "16-byte"),
+    (dict(out=0), drr.DRR_ERR_INVALID_ARG, "out"),
+    (dict(mode=drr.DRR_MODE_ALPHA), drr.DRR_ERR_UNSUPPORTED, "alpha"),
+    (dict(dtype=7), drr.DRR_ERR_INVALID_ARG, "dtype"),
+    (dict(n_samples=0), drr.DRR_ERR_INVALID_ARG, "n_samples"),
+    (dict(dims=(1, 16, 16)), drr.DRR_ERR_INVALID_ARG, "dims"),
+]
+
+
+@pytest.mark.parametrize("kw,status,word", STAGED_BAD)
+def test_staged_render_rejects_bad_arguments(kw, status, word):
+    with pytest.raises(drr.DrrError) as e:
+        _staged(**kw)
+    assert e.value.status == status
+    assert word in drr.drr_get_last_error()
+
+
+def test_staged_render_empty_batch_is_a_no_op():
+    _staged(B=0, vol=None, out=None, Rt=None)
+    assert drr.drr_get_last_error() == ""
+
+
 @pytest.mark.parametrize("kw,status", ADJOINT_BAD)
 def test_adjoint_rejects_bad_arguments(kw, status):
     with pytest.raises(drr.DrrError) as e:

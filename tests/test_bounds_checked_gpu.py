@@ -46,6 +46,10 @@ def test_forward_every_layout_dtype_and_mode_stays_in_bounds(checked, case):
             for mode in (wl.MODE_RAW, wl.MODE_BEER_LAMBERT, wl.MODE_ALPHA):
                 H.gpu_forward(w, layout=layout, dtype=dtype, mode=mode)
                 _clean(checked, f"forward layout {layout} dtype {dtype} mode {mode}")
+    for dtype in (H.F32, H.BF16):
+        for mode in (wl.MODE_RAW, wl.MODE_BEER_LAMBERT):
+            H.gpu_forward_staged(w, dtype=dtype, mode=mode)
+            _clean(checked, f"staged bricked forward dtype {dtype} mode {mode}")
 
 
 @pytest.mark.parametrize("case", range(len(CASES)))

@@ -17,7 +17,7 @@ import pytest
 import oracle
 from cone_beam_ct_b200 import workloads as wl
 from tests.gpu_helpers import (BF16, BRICKS, CORNERS, F32, LAYOUTS, LINEAR, PADDED, QUADS, assert_parity,
-                               bf16_values, gpu_forward)
+                               bf16_values, gpu_forward, gpu_forward_staged)
 
 pytestmark = pytest.mark.gpu
 TOL_F32, TOL_BF16 = 1e-4, 1e-2
@@ -110,7 +110,7 @@ def _sampled_oracle(w, ids, vol=None, mode=None):
 
 
 @pytest.mark.slow
-@pytest.mark.parametrize("layout", [PADDED, CORNERS])
+@pytest.mark.parametrize("layout", [PADDED, CORNERS, BRICKS])
 def test_config3_bf16_sampled(cuda, layout):
     w = wl.make_config(3)
     got = gpu_forward(w, layout=layout, dtype=BF16).reshape(-1)
@@ -139,7 +139,58 @@ def test_layouts_agree(cuda):
         # same positions, fractions and lerps: corner records and quads are bit-identical
         assert np.array_equal(a, gpu_forward(w, layout=CORNERS, dtype=dtype))
         assert np.array_equal(a, gpu_forward(w, layout=QUADS, dtype=dtype))
+        assert np.array_equal(a, gpu_forward(w, layout=BRICKS, dtype=dtype))
         assert_parity(a, gpu_forward(w, layout=PADDED, dtype=dtype), 1e-5, what="linear vs padded")
+
+
+def _inside_camera(w):
+    """The same case with the camera moved inside the volume (near its centre)."""
+    Rt = w.Rt.astype(np.float64).reshape(-1, 3, 4).copy()
+    centre = np.asarray(w.origin, np.float64) + 0.5 * (np.asarray(w.dims) - 1) * np.asarray(
+        w.spacing, np.float64) + np.array([0.31, -0.17, 0.23])
+    for b in range(Rt.shape[0]):
+        Rt[b, :, 3] = -Rt[b, :, :3] @ centre
+    w.Rt = Rt.astype(np.float32)
+    return w
+
+
+# geometries for the bricked forward, whose integral modes stage each layer
+# of a tile's bricks in shared memory: ragged small volumes, rays a voxel
+# apart and rays much closer (staged layers), a wide-angle camera (layers
+# wider than the staging window: global reads), a camera inside the volume
+STAGED_CASES = {
+    "small ragged": lambda: wl.small_random_case(131),
+    "sparse rays, 40 views": lambda: wl.small_random_case(132, dims=(70, 66, 75), B=40, H=48,
+                                                          W=40, n_samples=90),
+    "dense rays": lambda: wl.small_random_case(133, dims=(23, 17, 29), H=150, W=170,
+                                               n_samples=40),
+    "wide angle": lambda: _wide_angle(wl.small_random_case(134, dims=(90, 80, 70), H=64, W=64)),
+    "camera inside": lambda: _inside_camera(wl.small_random_case(135, dims=(40, 44, 36))),
+}
+
+
+def _wide_angle(w):
+    K = np.asarray(w.K, np.float32).reshape(3, 3).copy()
+    K[0, 0] /= 8.0
+    K[1, 1] /= 8.0
+    w.K = K.reshape(-1)
+    return w
+
+
+@pytest.mark.parametrize("name", sorted(STAGED_CASES))
+@pytest.mark.parametrize("mode", [wl.MODE_RAW, wl.MODE_BEER_LAMBERT])
+def test_staged_bricks_match_the_linear_layout_bit_for_bit(cuda, name, mode):
+    # staged and global samples read the same 8 voxels and take the same lerps
+    w = STAGED_CASES[name]()
+    for dtype in (F32, BF16):
+        a = gpu_forward(w, layout=LINEAR, dtype=dtype, mode=mode)
+        got = gpu_forward(w, layout=BRICKS, dtype=dtype, mode=mode)
+        assert np.array_equal(a, got), f"{name}: {np.count_nonzero(a != got)} pixels differ"
+        staged = gpu_forward_staged(w, dtype=dtype, mode=mode)
+        assert np.array_equal(a, staged), f"{name}: {np.count_nonzero(a != staged)} pixels differ"
+    ref = oracle.render(w.vol, w.dims, w.spacing, w.origin, w.K, w.Rt, w.H, w.W, w.n_samples,
+                        w.density_factor, mode)
+    assert_parity(gpu_forward(w, layout=BRICKS, dtype=F32, mode=mode), ref, TOL_F32, what=name)
 
 
 def test_forward_is_deterministic(cuda):
