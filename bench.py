@@ -73,6 +73,9 @@ def parse_args():
                         "workload's views split one per volume over as many volumes "
                         "(drr_render_batched, drr_render_adjoint_batched_ws, "
                         "drr_render_pose_grad_batched)")
+    p.add_argument("--views", type=int, default=0,
+                   help="render only the first VIEWS views of the workload (a smaller case of "
+                        "the same kernels, for profilers; 0: all)")
     p.add_argument("--no-extras", action="store_true",
                    help="skip the widened rows the default run also times (pose gradient, alpha "
                         "compositing, Siddon pair, batches)")
@@ -126,9 +129,13 @@ def job_throughput(world, units_per_rank_step, steps, max_ms):
 AUTO_LAYOUT = {1: "corners", 2: "quads", 3: "corners", 4: "quads"}
 
 
-def workload(cfg):
+def workload(cfg, views=0):
     from cone_beam_ct_b200 import workloads as wl
     w = wl.make_config(cfg)
+    if views and views < w.B:
+        w.Rt = w.Rt[:views]
+        if w.grad_out is not None:
+            w.grad_out = w.grad_out[:views]
     if w.grad_out is None:
         w.grad_out = np.random.default_rng(2000 + cfg).standard_normal(
             (w.B, w.H, w.W)).astype(np.float32)
@@ -360,7 +367,7 @@ def run_reference(args):
         return 0
     import oracle
     oracle.build()
-    w = workload(args.config)
+    w = workload(args.config, args.views)
     cores = len(os.sched_getaffinity(0))
     rows_per_step = max(1, min(w.H, REF_SAMPLES_PER_STEP // (w.W * w.n_samples)))
 
@@ -823,7 +830,7 @@ def run_ours(args):
     dev = torch.device("cuda", torch.cuda.current_device())
     drr.lib()
 
-    w = workload(args.config)
+    w = workload(args.config, args.views)
     if args.layout == "auto":
         args.layout = AUTO_LAYOUT[args.config]
     layout = {"padded": drr.DRR_LAYOUT_PADDED, "corners": drr.DRR_LAYOUT_CORNERS,
@@ -1083,7 +1090,7 @@ def run_partitioned(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     dev = torch.device("cuda", torch.cuda.current_device())
     drr.lib()
-    w = workload(args.config)
+    w = workload(args.config, args.views)
     if args.layout == "auto":
         args.layout = AUTO_LAYOUT[args.config]
     layout = {"padded": drr.DRR_LAYOUT_PADDED, "corners": drr.DRR_LAYOUT_CORNERS,

@@ -157,8 +157,15 @@ __device__ __forceinline__ float march_quads(const T* __restrict__ vol, const Ge
     return acc;
 }
 
+// CTAs per SM the compiler must fit: 5 for bf16 corner records (at most 51
+// registers; B200, 1024^2 x 512 C-arm views: 2.80 against 2.86 ms), no
+// minimum (0) for the rest (the fp32 quad forward ran 2-7 % slower when held
+// to 5 or 6)
+template <typename T, int LAYOUT>
+constexpr int kForwardMinBlocks = (sizeof(T) == 2 && LAYOUT == 2) ? 5 : 0;
+
 template <typename T, int LAYOUT, int MODE>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, (kForwardMinBlocks<T, LAYOUT>))
 forward_kernel(const T* __restrict__ vol_base, const float* __restrict__ Rt,
                float* __restrict__ out, const Geom g) {
     __shared__ View sv;
