@@ -108,23 +108,57 @@ MUTANTS = {
 }
 
 
-@pytest.mark.slow
-@pytest.mark.parametrize("name", sorted(MUTANTS))
-def test_pins_catch_mutant(name, tmp_path):
+PIN_FILES = {"core": "test_oracle_pins.py", "pose": "test_oracle_pose_pins.py",
+             "alpha_noise": "test_oracle_alpha_noise_pins.py",
+             "siddon": "test_oracle_siddon_pins.py"}
+
+
+def pin_files_for(name):
+    """Every pin file, the mutated part's own first: the run stops at the
+    first failing pin (-x), so a mutant fails fast and the suite is the same
+    whatever the order."""
+    area = ("siddon" if "siddon" in name else "pose" if "pose" in name else
+            "alpha_noise" if ("alpha" in name or "noise" in name) else "core")
+    order = [area] + [k for k in PIN_FILES if k != area]
+    return [os.path.join(ROOT, "tests", PIN_FILES[k]) for k in order]
+
+
+def run_mutant(name, workdir):
+    """Build the oracle with mutant `name` planted and run the pin suite
+    against it; returns (returncode, end of its output)."""
     before, after = MUTANTS[name]
     src = open(SRC).read()
-    assert src.count(before) == 1, "mutation site not found: " + name
-    c_file = tmp_path / "mutant.c"
-    lib = tmp_path / "mutant.so"
-    c_file.write_text(src.replace(before, after))
-    subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-o", str(lib),
-                           str(c_file), "-lm", "-lpthread"])
-    env = dict(os.environ, DRR_ORACLE_LIB=str(lib))
-    r = subprocess.run([sys.executable, "-m", "pytest",
-                        os.path.join(ROOT, "tests", "test_oracle_pins.py"),
-                        os.path.join(ROOT, "tests", "test_oracle_pose_pins.py"),
-                        os.path.join(ROOT, "tests", "test_oracle_alpha_noise_pins.py"),
-                        os.path.join(ROOT, "tests", "test_oracle_siddon_pins.py"),
-                        "-q", "-x", "-p", "no:cacheprovider"],
-                       env=env, cwd=ROOT, capture_output=True, text=True, timeout=600)
-    assert r.returncode != 0, f"mutant '{name}' passed every pin:\n{r.stdout[-2000:]}"
+    if src.count(before) != 1:
+        return None, "mutation site not found: " + name
+    tag = "".join(c if c.isalnum() else "_" for c in name)
+    c_file = os.path.join(workdir, tag + ".c")
+    lib = os.path.join(workdir, tag + ".so")
+    with open(c_file, "w") as f:
+        f.write(src.replace(before, after))
+    subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-o", lib, c_file, "-lm",
+                           "-lpthread"])
+    env = dict(os.environ, DRR_ORACLE_LIB=lib)
+    r = subprocess.run([sys.executable, "-m", "pytest"] + pin_files_for(name) +
+                       ["-q", "-x", "-p", "no:cacheprovider"],
+                       env=env, cwd=ROOT, capture_output=True, text=True, timeout=900)
+    return r.returncode, r.stdout[-2000:]
+
+
+@pytest.fixture(scope="module")
+def mutant_results(tmp_path_factory):
+    """Every mutant's pin run, several at once (each is a separate build and
+    interpreter, so they share nothing)."""
+    from concurrent.futures import ThreadPoolExecutor
+    workdir = str(tmp_path_factory.mktemp("mutants"))
+    workers = max(1, min(8, len(os.sched_getaffinity(0))))
+    with ThreadPoolExecutor(max_workers=workers) as pool:
+        futures = {name: pool.submit(run_mutant, name, workdir) for name in MUTANTS}
+        return {name: f.result() for name, f in futures.items()}
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_mutant(name, mutant_results):
+    code, out = mutant_results[name]
+    assert code is not None, out
+    assert code != 0, f"mutant '{name}' passed every pin:\n{out}"
