@@ -339,8 +339,9 @@ def traffic_for(kernel, workload_name, layout_name):
 
 # the volume adjoint's launches, timed as one group; the record kernel (dense
 # views) dominates it
-ADJOINT_GROUP = ("volume adjoint: plan_views + zero_records + adjoint_kernel + records_kernel "
-                 "+ gather_records (records_kernel dominant)")
+ADJOINT_GROUP = ("volume adjoint: plan_views + zero_records + records_kernel + scatter_records "
+                 "+ slab_adjoint_kernel (records_kernel dominant where the views are dense, "
+                 "slab_adjoint_kernel where they are sparse)")
 
 REF_SAMPLES_PER_STEP = 4_000_000      # ray-samples per reference-arm step (~0.6 s of fp64 CPU)
 BASELINE_SAMPLES = 100_000_000        # ray-samples of the cpu_baseline sample (~15 s)
@@ -1060,7 +1061,8 @@ def run_ours(args):
         "batched": batched,
         "configs": configs,
         "bricks": bricks,
-        "gpu_launches": 7 * args.steps,   # prepare, forward, plan, zero, 2 adjoint paths, gather
+        # prepare, forward; adjoint: plan, zero, records, scatter, slab pass
+        "gpu_launches": 7 * args.steps,
         "clocks": clocks,
         "bracket_ms": bracket[0].elapsed_time(bracket[1]),
     }
@@ -1145,7 +1147,8 @@ def run_partitioned(args):
     if world > 1:
         dist.barrier()
     total_ms = max_over_ranks([total], dev)[0]
-    launches = 1 + 6 * len(part.segments)      # prepare; per call: forward, plan, zero, 3 adjoint
+    # prepare; per call: forward, then plan, zero, records, scatter, slab pass
+    launches = 1 + 6 * len(part.segments)
     line = {
         "metric": METRIC, "value": w.samples * args.steps / (total_ms * 1e-3) / 1e9,
         "unit": "Gsamples/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,

@@ -40,4 +40,5 @@ from .drr import (  # noqa: F401
     drr_render_siddon,
     drr_render_siddon_adjoint,
     drr_render_staged,
+    drr_wait_timeouts,
 )

@@ -43,12 +43,18 @@
 // record sums the moments of its samples (records_kernel); a scatter pass
 // then turns each record into corner weights and adds them to the gradient
 // volume.  The alpha gradient (records of weights, added by a gather pass)
-// and batched calls (records per volume-channel) take the same path.  Sparse views gain nothing from records (measured: the records
-// path ran 12-20 ms against the direct path's 9.3 on the 256^3 / 200^2
-// workload) and keep the direct path above.
+// and batched calls (records per volume-channel) take the same path.
+//
+// The sparse views of a call with a workspace accumulate into records too,
+// but one slab of cell layers at a time, each slab's records small enough to
+// stay in the L2 (slab_adjoint_kernel): the whole record array gained
+// nothing there (12-20 ms against the direct path's 9.3 on the 256^3 volume
+// seen by 64 views of 200^2, the records going to DRAM between views), the
+// slabs take 6.7 ms.  Without a workspace every view takes the direct path.
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "drr_internal.cuh"
@@ -131,58 +137,102 @@ __device__ __forceinline__ bool dense_tile(const View& v, const Geom& g, double 
     return (sqrt(c2) * ang / min_sp) < 8.0;
 }
 
-// Flush a pending corner record: two 16-byte vector atomics into one sector.
-// (n: floats of the record array at rec, for the bounds-checked build)
+// Fire-and-forget fp32 reductions into global memory, spelled out so that
+// they are L2 reductions whatever the compiler can prove about the pointer
+// (an add it cannot place in global memory becomes a generic atomic that
+// waits for its old value: the slab pass took 9.6 instead of 6.8 ms).  No memory
+// clobber: nothing in a kernel reads what these add before a barrier or a
+// fence, which order them for the compiler.
+__device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, float d) {
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(__cvta_generic_to_global(p)),
+                 "f"(a), "f"(b), "f"(c), "f"(d));
+}
+__device__ __forceinline__ void red_add(float* p, float a) {
+    asm volatile("red.global.add.f32 [%0], %1;" ::"l"(__cvta_generic_to_global(p)), "f"(a));
+}
+
+// Flush a pending corner record: two 16-byte vector reductions into one
+// sector.  (n: floats of the record array at rec, for the bounds-checked
+// build)
 __device__ __forceinline__ void flush_record(float* __restrict__ rec, int cell, const float a[8],
                                              long long n) {
     if (!in_bounds((long long)cell * 8, 8, n)) return;
-    float4* p = reinterpret_cast<float4*>(rec + (size_t)cell * 8);
-    atomicAdd(p, make_float4(a[0], a[1], a[2], a[3]));
-    atomicAdd(p + 1, make_float4(a[4], a[5], a[6], a[7]));
+    float* p = rec + (size_t)cell * 8;
+    red_add_v4(p, a[0], a[1], a[2], a[3]);
+    red_add_v4(p + 4, a[4], a[5], a[6], a[7]);
 }
 __device__ __forceinline__ void flush_record(float* __restrict__ rec, int cell, const float2 a[4],
                                              long long n) {
     if (!in_bounds((long long)cell * 8, 8, n)) return;
-    float4* p = reinterpret_cast<float4*>(rec + (size_t)cell * 8);
-    atomicAdd(p, make_float4(a[0].x, a[0].y, a[1].x, a[1].y));
-    atomicAdd(p + 1, make_float4(a[2].x, a[2].y, a[3].x, a[3].y));
+    float* p = rec + (size_t)cell * 8;
+    red_add_v4(p, a[0].x, a[0].y, a[1].x, a[1].y);
+    red_add_v4(p + 4, a[2].x, a[2].y, a[3].x, a[3].y);
 }
 
-// Workspace layout (drr_render_adjoint_ws): a 256-byte aligned header of
-// ints -- [0] "some view is dense", [1 + b] "view b is dense" (b: output
-// image) -- then the corner records of each volume-channel slot, 8 floats per
-// cell, cell = (k * (ny-1) + j) * (nx-1) + i.
+// Workspace layout (drr_render_adjoint_ws, header_layout below): a header
+// of ints -- [0] bit 0 "some view is dense", bit 1 "some view is sparse";
+// [1 + b] "view b is dense" (b: output image) -- then, 16-byte aligned, the
+// slab pass's grid-barrier words, then, 256-byte aligned, every view's View
+// (K^-1 R^T and camera centre, written by plan_views); then, 256-byte
+// aligned, the corner records of each volume-channel slot, 8 floats per
+// cell, cell = (k * (ny-1) + j) * (nx-1) + i.  The sparse views' slabs
+// (slab_adjoint_kernel) reuse the start of the record area once the dense
+// views' records are scattered.
+constexpr int kSomeDense = 1, kSomeSparse = 2;
+struct HeaderLayout {
+    size_t bar, views, rec;                      // byte offsets
+};
+__host__ __device__ inline HeaderLayout header_layout(int B) {
+    const size_t bar = ((size_t)(1 + B) * sizeof(int) + 15) / 16 * 16;
+    const size_t views = (bar + 4 * sizeof(unsigned) + 255) / 256 * 256;
+    const size_t rec = (views + (size_t)B * sizeof(View) + 255) / 256 * 256;
+    return {bar, views, rec};
+}
+
 struct Workspace {
     int* flags;        // NULL: no workspace, every view takes the direct path
     float* rec;        // records of volume-channel slot 0; slot s at rec + s * rec_stride
     long long rec_stride;
+    // the record kernel's 16 warp phases are spread over 2^-phase_shift of
+    // the ray's length (see launch_adjoint)
+    int phase_shift;
+    unsigned* bar;     // grid barrier: [0] arrivals, [1] released epoch, [2] abort
+    const View* views;
 };
 
 // Which views accumulate into records: one CTA loops over the views, so
-// that flags[0] ("some view is dense") is written once, after all of them.
+// that flags[0] is written once, after all of them.  It also stores each
+// view's View and clears the barrier words for the slab pass.
 __global__ void __launch_bounds__(256) plan_views(const float* __restrict__ Rt, const Geom g,
-                                                  int* __restrict__ flags) {
+                                                  int* __restrict__ flags,
+                                                  View* __restrict__ views,
+                                                  unsigned* __restrict__ bar) {
     __shared__ int any;
-    if (threadIdx.x == 0) any = 0;
+    if (threadIdx.x == 0) {
+        any = 0;
+        for (int k = 0; k < 4; ++k) bar[k] = 0u;
+    }
     __syncthreads();
     int mine = 0;
     for (int b = threadIdx.x; b < g.B; b += blockDim.x) {
         View v;
         view_setup(Rt + 12 * (size_t)batch_item(g, b).pose, g, v);
+        views[b] = v;
         // a view is judged by its first tile: every tile subtends nearly the
         // same angle (the pixel pitch is constant across the detector)
         const int dense = dense_tile(v, g, 0.0, 0.0) ? 1 : 0;
         flags[1 + b] = dense;
-        mine |= dense;
+        mine |= dense ? kSomeDense : kSomeSparse;
     }
-    if (mine) atomicOr(&any, 1);
+    if (mine) atomicOr(&any, mine);
     __syncthreads();
     if (threadIdx.x == 0) flags[0] = any;
 }
 
-// Zero the records when some view will use them.
-__global__ void zero_records(const int* __restrict__ flags, float4* __restrict__ rec, int64_t n4) {
-    if (flags[0] == 0) return;
+// Zero n4 float4 of records when some view will use them (flags[0] & use).
+__global__ void zero_records(const int* __restrict__ flags, int use, float4* __restrict__ rec,
+                             int64_t n4) {
+    if ((flags[0] & use) == 0) return;
     const float4 z = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
     for (int64_t m = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; m < n4;
          m += (int64_t)gridDim.x * blockDim.x)
@@ -210,7 +260,7 @@ __device__ __forceinline__ void moments_to_corner_weights(float v[8]) {
 __global__ void scatter_records(const int* __restrict__ flags, const float* __restrict__ rec,
                                 long long rec_stride, float* __restrict__ grad, int nx, int ny,
                                 int nz, int slots) {
-    if (flags[0] == 0) return;
+    if ((flags[0] & kSomeDense) == 0) return;
     const int crow = nx - 1, rows = (ny - 1) * (nz - 1);    // cells per row, rows per slot
     const long long total = (long long)rows * slots;
     const long long nxy = (long long)nx * ny, nvox = nxy * nz;
@@ -244,7 +294,7 @@ __global__ void scatter_records(const int* __restrict__ flags, const float* __re
 __global__ void gather_records(const int* __restrict__ flags, const float* __restrict__ rec,
                                long long rec_stride, float* __restrict__ grad, int nx, int ny,
                                int nz, int slots) {
-    if (flags[0] == 0) return;
+    if ((flags[0] & kSomeDense) == 0) return;
     const int rows = ny * nz;                    // x rows per slot (nx*ny*nz < 2^31)
     const long long total = (long long)rows * slots;
     const int cr = nx - 1, cs = (nx - 1) * (ny - 1);
@@ -414,7 +464,7 @@ records_kernel(const float* __restrict__ Rt, const float* __restrict__ grad_out,
     const int px = (warp & 3) * 4 + (lane & 3), py = (warp >> 2) * 8 + (lane >> 2);
     const int c0 = blockIdx.x * kRecTileW + px * kBundleX, r0 = blockIdx.y * kRecTileH + py * kBundleY;
     const int ph = (warp + blockIdx.x * 3 + blockIdx.y * 5 + blockIdx.z) & 15;   // 16 phases
-    const int start = (int)(((long long)g.N * ph) >> 4);
+    const int start = (int)(((long long)g.N * ph) >> ws.phase_shift);
 
     // per ray: its position at the current sample (32.32) and step; the start
     // of the second pass is recovered from the position after the first
@@ -502,6 +552,244 @@ records_kernel(const float* __restrict__ Rt, const float* __restrict__ grad_out,
 #pragma unroll
         for (int h = 0; h < kSlots; ++h)
             if (pc[h] >= 0) flush_record(rec, pc[h], p[h], ws.rec_stride);
+    }
+}
+
+// Slab records for the sparse views (rays about a voxel apart or more).
+// With a workspace those views leave the direct path for per-cell records,
+// built one slab of cell layers at a time: a slab's records (at most
+// kSlabRecordBytes) stay in the L2, which the whole record array (8 floats
+// per cell, 4x the gradient volume) does not, so every update is an L2
+// reduction and no record goes to DRAM between two views.  A warp walks 8 x
+// 4 neighbouring rays, each over the samples whose cell lies in the slab,
+// keeps the moments of its current cell pending and flushes them (two
+// 16-byte vector reductions into one sector) when the cell changes.  A ray
+// about a voxel per sample changes cell nearly every sample, and the record
+// then costs 2 sector operations per sample where the direct path's faces
+// cost 3.5 (measured on the 256^3 volume seen by 64 views of 200^2 with 256
+// samples: 1.6 reduction sectors per sample).  Then the slab's records go
+// into the gradient (moments to corner weights, as scatter_records) and are
+// cleared for the next slab.
+//
+// One cooperative launch does every slab, its phases separated by a grid
+// barrier, so that a call whose views are all dense pays one launch that
+// returns at once (separate launches per slab and phase cost 0.13 ms on the
+// 4-view 1024^2 workload, 2.7 us each).  Measured slab sizes on that 64-view
+// workload (B200): 24 / 32 / 48 MiB, 7.08 / 6.82 / 6.74 ms (separate
+// launches per slab: 16 / 24 / 32 / 48 / 64 / 96 MiB, 7.63 / 7.07 / 6.85 /
+// 6.95 / 7.06 / 7.60 ms).
+constexpr long long kSlabRecordBytes = 48ll << 20;
+
+// A barrier wait gives up after this long (the slowest legitimate phase of a
+// huge call is far shorter); it then raises the abort word, so that every
+// other CTA leaves at its next wait, and is counted in g_wait_timeouts.
+constexpr unsigned long long kBarrierTimeoutNs = 20ull * 1000 * 1000 * 1000;
+__device__ unsigned long long g_wait_timeouts;
+
+__device__ __forceinline__ unsigned long long global_ns() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Grid-wide barrier over a cooperative launch (every CTA resident).  bar[0]
+// counts arrivals over the launch (epoch e is complete at e * gridDim.x),
+// bar[1] holds the last released epoch, bar[2] the abort word.  Returns
+// false if this or another CTA gave up (the caller returns).
+__device__ bool grid_barrier(unsigned* bar, unsigned& epoch) {
+    __shared__ int s_ok;
+    __syncthreads();
+    ++epoch;
+    if (threadIdx.x == 0) {
+        volatile unsigned* vb = bar;
+        int ok = vb[2] == 0u;
+        if (ok) {
+            __threadfence();                     // this CTA's writes before its arrival
+            const unsigned arrived = atomicAdd(&bar[0], 1u) + 1u;
+            if (arrived == epoch * gridDim.x) {
+                __threadfence();
+                atomicExch(&bar[1], epoch);
+            } else {
+                const unsigned long long t0 = global_ns();
+                while (vb[1] < epoch) {
+                    if (vb[2] != 0u) {
+                        ok = 0;
+                        break;
+                    }
+                    if (global_ns() - t0 > kBarrierTimeoutNs) {
+                        atomicExch(&bar[2], 1u);
+                        atomicAdd(&g_wait_timeouts, 1ull);
+                        ok = 0;
+                        break;
+                    }
+                    __nanosleep(256);
+                }
+            }
+            __threadfence();                     // the other CTAs' writes before ours
+        }
+        s_ok = ok;
+    }
+    __syncthreads();
+    return s_ok != 0;
+}
+
+// Sample indices i in [0, N) whose 32.32 coordinate q0 + i s lies in [z0, z1):
+// an interval, since the coordinate is monotone in i.  Exact integer bounds,
+// so consecutive slabs share no sample and miss none.
+__device__ __forceinline__ void slab_range(long long q0, long long s, int N, long long z0,
+                                           long long z1, int& i0, int& i1) {
+    if (s == 0) {
+        i0 = 0;
+        i1 = (q0 >= z0 && q0 < z1) ? N : 0;
+        return;
+    }
+    // first index at which the coordinate is >= z (s > 0) or < z (s < 0)
+    auto first = [&](long long z) -> int {
+        long long k;
+        if (s > 0) k = q0 >= z ? 0 : (z - q0 + s - 1) / s;
+        else k = q0 < z ? 0 : (q0 - z) / (-s) + 1;
+        return (int)min(k, (long long)N);
+    };
+    if (s > 0) {
+        i0 = first(z0);
+        i1 = first(z1);
+    } else {
+        i0 = first(z1);
+        i1 = first(z0);
+    }
+}
+
+// Records of one slab [cz0, cz1): slot s at rec + s * slab_stride, cell (i, j,
+// k) at ((k - cz0) * (ny-1) + j) * (nx-1) + i.  Work items are 8 x 4 ray
+// blocks of the sparse views, taken by the grid's warps in turn.
+template <int MODE>
+__device__ __forceinline__ void slab_records(const float* __restrict__ grad_out,
+                                             const float* __restrict__ fwd_out, const Geom g,
+                                             const Workspace ws, int cz0, int cz1,
+                                             long long slab_stride) {
+    const int lane = threadIdx.x & 31;
+    const long long nwarps = ((long long)gridDim.x * blockDim.x) >> 5;
+    const long long gwarp = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int bx = (g.W + kWarpW - 1) / kWarpW, by = (g.H + kWarpH - 1) / kWarpH;
+    const long long per_view = (long long)bx * by, items = per_view * g.B;
+    const int cr = g.nx - 1, cs = (g.nx - 1) * (g.ny - 1);
+    const long long z0 = (long long)cz0 << 32, z1 = (long long)cz1 << 32;
+    const long long slots = batch_slots(g);
+    for (long long item = gwarp; item < items; item += nwarps) {
+        // Every lane takes the same items; lanes without work in an item
+        // wait here for the others, so that the warp's lanes do not drift
+        // onto different items (without this wait: 16.0 against 9.6 ms).
+        __syncwarp();
+        const int b = (int)(item / per_view);
+        const int t = (int)(item - (long long)b * per_view);
+        const int wy = t / bx, wx = t - wy * bx;
+        if (ws.flags[1 + b] != 0) continue;      // dense view: records_kernel's
+        const BatchItem it = batch_item(g, b);
+        if (!in_bounds(it.slot * slab_stride, slab_stride, slots * slab_stride)) continue;
+        float* const rec = ws.rec + it.slot * slab_stride;
+        const int c = wx * kWarpW + (lane % kWarpW), r = wy * kWarpH + (lane / kWarpW);
+        if (r >= g.H || c >= g.W) continue;
+        const size_t pix = ((size_t)b * g.H + r) * g.W + c;
+        if (!in_bounds(pix, 1, (long long)g.B * g.H * g.W)) continue;
+        float go = grad_out[pix];
+        if (MODE == 1) go *= 1.0f - fwd_out[pix];
+        Ray ray;
+        if (go == 0.0f || !ray_setup(ws.views[b], g, (double)c, (double)r, 0.0, ray)) continue;
+        int i0, i1;
+        slab_range(ray.q0[2], ray.s[2], g.N, z0, z1, i0, i1);
+        if (i0 >= i1) continue;
+        const float scale = go * (g.density_factor * ray.dt);
+        long long qx = ray.q0[0] + (long long)i0 * ray.s[0];
+        long long qy = ray.q0[1] + (long long)i0 * ray.s[1];
+        long long qz = ray.q0[2] + (long long)i0 * ray.s[2];
+        int pc = -1;
+        float2 p[4];
+        for (int i = i0; i < i1; ++i) {
+            const int cell = (fix_cell(qz) - cz0) * cs + fix_cell(qy) * cr + fix_cell(qx);
+            const float fx = fix_frac(qx), fy = fix_frac(qy), fz = fix_frac(qz);
+            qx += ray.s[0];
+            qy += ray.s[1];
+            qz += ray.s[2];
+            const float2 mx = make_float2(scale, scale * fx);
+            const float2 mxy = __fmul2_rn(mx, make_float2(fy, fy));
+            const float2 w[4] = {mx, mxy, __fmul2_rn(mx, make_float2(fz, fz)),
+                                 __fmul2_rn(mxy, make_float2(fz, fz))};
+            if (cell != pc) {
+                if (pc >= 0) flush_record(rec, pc, p, slab_stride);
+                pc = cell;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) p[e] = w[e];
+            } else {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) p[e] = __fadd2_rn(p[e], w[e]);
+            }
+        }
+        flush_record(rec, pc, p, slab_stride);
+    }
+}
+
+// A slab's records into the gradient (as scatter_records: moments to corner
+// weights, 8 coalesced atomic adds per cell), each record cleared after it is
+// read so that the next slab starts from zeros.  A CTA takes whole x rows.
+// Records are read and cleared in the L2 (.cg): the reductions wrote them
+// there, and the next slab's reductions reuse the lines.
+__device__ __forceinline__ void slab_scatter(float* __restrict__ rec, long long slab_stride,
+                                             float* __restrict__ grad, const Geom g, int slots,
+                                             int cz0, int cz1) {
+    const int nx = g.nx, ny = g.ny;
+    const int crow = nx - 1, rows = (ny - 1) * (cz1 - cz0);   // cells per row, rows per slot
+    const long long total = (long long)rows * slots;
+    const long long nxy = (long long)nx * ny, nvox = nxy * g.nz;
+    const float4 zero = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    for (long long row = blockIdx.x; row < total; row += gridDim.x) {
+        const int slot = (int)(row / rows);
+        const int rr = (int)(row - (long long)slot * rows);
+        const int kk = rr / (ny - 1), j = rr - kk * (ny - 1);
+        const int k = cz0 + kk;
+        float4* __restrict__ r =
+            reinterpret_cast<float4*>(rec + slot * slab_stride + (long long)rr * crow * 8);
+        float* __restrict__ gr = grad + slot * nvox + k * nxy + (long long)j * nx;
+        for (int i = threadIdx.x; i < crow; i += blockDim.x) {
+            if (!in_bounds(((long long)rr * crow + i) * 8, 8, slab_stride)) continue;
+            const float4 lo = __ldcg(r + 2 * i), hi = __ldcg(r + 2 * i + 1);
+            __stcg(r + 2 * i, zero);
+            __stcg(r + 2 * i + 1, zero);
+            float v[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+            moments_to_corner_weights(v);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const long long off = i + (e & 1) + ((e >> 1) & 1) * nx + (e >> 2) * nxy;
+                if (v[e] != 0.0f && in_bounds(k * nxy + (long long)j * nx + off, 1, nvox))
+                    red_add(gr + off, v[e]);
+            }
+        }
+    }
+}
+
+// Every slab of the sparse views: clear the slab records, then per slab the
+// records and the scatter, with a grid barrier after each phase.  Launched
+// cooperatively (all CTAs resident); returns at once when no view is sparse.
+template <int MODE>
+__global__ void __launch_bounds__(kThreads, 4)
+slab_adjoint_kernel(const float* __restrict__ grad_out, const float* __restrict__ fwd_out,
+                    float* __restrict__ grad, const Geom g, const Workspace ws, int layers,
+                    long long slab_stride) {
+    if ((ws.flags[0] & kSomeSparse) == 0) return;   // the same in every CTA
+    const int slots = batch_slots(g);
+    const long long n4 = slab_stride / 4 * slots;
+    float4* const r4 = reinterpret_cast<float4*>(ws.rec);
+    const float4 zero = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    for (long long m = (long long)blockIdx.x * blockDim.x + threadIdx.x; m < n4;
+         m += (long long)gridDim.x * blockDim.x)
+        __stcg(r4 + m, zero);
+    unsigned epoch = 0;
+    if (!grid_barrier(ws.bar, epoch)) return;
+    for (int cz0 = 0; cz0 < g.nz - 1; cz0 += layers) {
+        const int cz1 = min(cz0 + layers, g.nz - 1);
+        slab_records<MODE>(grad_out, fwd_out, g, ws, cz0, cz1, slab_stride);
+        if (!grid_barrier(ws.bar, epoch)) return;
+        slab_scatter(ws.rec, slab_stride, grad, g, slots, cz0, cz1);
+        if (!grid_barrier(ws.bar, epoch)) return;
     }
 }
 
@@ -734,9 +1022,7 @@ alpha_records_kernel(const T* __restrict__ vol_base, const float* __restrict__ R
 
 }  // namespace
 
-size_t adjoint_workspace_header(int B) {
-    return ((size_t)(1 + B) * sizeof(int) + 255) / 256 * 256;
-}
+size_t adjoint_workspace_header(int B) { return header_layout(B).rec; }
 
 namespace {
 constexpr int kMaxDevices = 64;
@@ -766,43 +1052,107 @@ cudaError_t noalloc_scratch(void** out) {
 
 DRR_BOUNDS_READER(bounds_word_adjoint)
 
+cudaError_t wait_timeouts(unsigned long long* out) {
+    cudaError_t e = cudaMemcpyFromSymbol(out, g_wait_timeouts, sizeof(*out));
+    if (e != cudaSuccess) return e;
+    const unsigned long long zero = 0ull;
+    return cudaMemcpyToSymbol(g_wait_timeouts, &zero, sizeof(zero));
+}
+
 size_t adjoint_workspace_bytes(int nx, int ny, int nz, int B, int slots) {
     return adjoint_workspace_header(B) +
            (size_t)(nx - 1) * (ny - 1) * (nz - 1) * 8 * sizeof(float) * (size_t)slots;
 }
 
+namespace {
+
+// The workspace's parts (header_layout) for B output images, and the plan
+// launch that fills its header.
+Workspace workspace_parts(void* workspace, const Geom& g) {
+    Workspace ws{};
+    ws.phase_shift = 4;
+    if (!workspace) return ws;
+    char* const base = static_cast<char*>(workspace);
+    const HeaderLayout h = header_layout(g.B);
+    ws.flags = static_cast<int*>(workspace);
+    ws.bar = reinterpret_cast<unsigned*>(base + h.bar);
+    ws.views = reinterpret_cast<const View*>(base + h.views);
+    ws.rec = reinterpret_cast<float*>(base + h.rec);
+    ws.rec_stride = (long long)(g.nx - 1) * (g.ny - 1) * (g.nz - 1) * 8;
+    return ws;
+}
+
+void launch_plan(const Workspace& ws, const float* Rt, const Geom& g, cudaStream_t stream) {
+    plan_views<<<1, 256, 0, stream>>>(Rt, g, ws.flags, const_cast<View*>(ws.views), ws.bar);
+}
+
+// The sparse views' slab pass: one cooperative launch, as many CTAs as fit
+// on the device at once.
+cudaError_t launch_slabs(const Workspace& ws, const Geom& g, int mode, const float* grad_out,
+                         const float* fwd_out, float* grad_vol, cudaStream_t stream) {
+    const int slots = batch_slots(g);
+    const long long layer = (long long)(g.nx - 1) * (g.ny - 1) * 8;   // floats per cell layer
+    int layers = (int)std::max(1LL, std::min((long long)(g.nz - 1),
+                                             kSlabRecordBytes / (layer * 4 * slots)));
+    long long slab_stride = layer * layers;
+    const void* fn = mode == 1 ? (const void*)slab_adjoint_kernel<1>
+                               : (const void*)slab_adjoint_kernel<0>;
+    int dev = 0, sms = 0, per_sm = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kThreads, 0);
+    if (e != cudaSuccess) return e;
+    if (per_sm < 1) return cudaErrorLaunchOutOfResources;
+    Workspace w = ws;
+    Geom gg = g;
+    void* args[] = {(void*)&grad_out, (void*)&fwd_out, (void*)&grad_vol, (void*)&gg, (void*)&w,
+                    (void*)&layers, (void*)&slab_stride};
+    return cudaLaunchCooperativeKernel(fn, dim3(sms * per_sm), dim3(kThreads), args, 0, stream);
+}
+
+}  // namespace
+
 cudaError_t launch_adjoint(const Geom& g, const float* Rt, int mode, const float* grad_out,
                            const float* fwd_out, float* grad_vol, void* workspace,
                            cudaStream_t stream) {
-    const dim3 grid((g.W + kTileW - 1) / kTileW, (g.H + kTileH - 1) / kTileH, g.B);
-    Workspace ws{nullptr, nullptr, 0};
-    const int slots = batch_slots(g);
-    const long long cells = (long long)(g.nx - 1) * (g.ny - 1) * (g.nz - 1);
-    const int64_t n_rec4 = cells * 2 * slots;    // float4 per record: 2
-    const int fill_grid = 148 * 8;
-    if (workspace) {
-        ws.flags = static_cast<int*>(workspace);
-        ws.rec = reinterpret_cast<float*>(static_cast<char*>(workspace) +
-                                          adjoint_workspace_header(g.B));
-        ws.rec_stride = cells * 8;
-        plan_views<<<1, 256, 0, stream>>>(Rt, g, ws.flags);
-        zero_records<<<fill_grid, 256, 0, stream>>>(ws.flags, reinterpret_cast<float4*>(ws.rec),
-                                                    n_rec4);
-    }
-    if (mode == 1)
-        adjoint_kernel<1><<<grid, kThreads, 0, stream>>>(Rt, grad_out, fwd_out, grad_vol, g, ws);
-    else
-        adjoint_kernel<0><<<grid, kThreads, 0, stream>>>(Rt, grad_out, fwd_out, grad_vol, g, ws);
-    if (workspace) {
-        const dim3 rgrid((g.W + kRecTileW - 1) / kRecTileW, (g.H + kRecTileH - 1) / kRecTileH, g.B);
+    if (!workspace) {
+        const dim3 grid((g.W + kTileW - 1) / kTileW, (g.H + kTileH - 1) / kTileH, g.B);
+        const Workspace none = workspace_parts(nullptr, g);
         if (mode == 1)
-            records_kernel<1><<<rgrid, kThreads, 0, stream>>>(Rt, grad_out, fwd_out, g, ws);
+            adjoint_kernel<1><<<grid, kThreads, 0, stream>>>(Rt, grad_out, fwd_out, grad_vol, g,
+                                                             none);
         else
-            records_kernel<0><<<rgrid, kThreads, 0, stream>>>(Rt, grad_out, fwd_out, g, ws);
-        scatter_records<<<fill_grid, 256, 0, stream>>>(ws.flags, ws.rec, ws.rec_stride, grad_vol,
-                                                       g.nx, g.ny, g.nz, slots);
+            adjoint_kernel<0><<<grid, kThreads, 0, stream>>>(Rt, grad_out, fwd_out, grad_vol, g,
+                                                             none);
+        return cudaGetLastError();
     }
-    return cudaGetLastError();
+    Workspace ws = workspace_parts(workspace, g);
+    const int slots = batch_slots(g);
+    const int fill_grid = 148 * 8;
+    // Phases over the whole ray keep warps that cover neighbouring rays off
+    // the same records at the same time; over a record array many times the
+    // L2 they also keep every record of the CTAs' beams live at once.
+    // Beyond 1 GiB of records they span the first quarter of the ray instead
+    // (B200: 4.3 GB of records for 2 views of 2048^2, 10.79 -> 10.48 ms; 530
+    // MB for 4 views of 1024^2, the whole ray stays best: 6.00 against 6.03
+    // ms).
+    const double rec_bytes = (double)ws.rec_stride * 4.0 * slots;
+    ws.phase_shift = rec_bytes > 1073741824.0 ? 6 : 4;
+    launch_plan(ws, Rt, g, stream);
+    zero_records<<<fill_grid, 256, 0, stream>>>(ws.flags, kSomeDense,
+                                                reinterpret_cast<float4*>(ws.rec),
+                                                ws.rec_stride / 4 * slots);
+    const dim3 rgrid((g.W + kRecTileW - 1) / kRecTileW, (g.H + kRecTileH - 1) / kRecTileH, g.B);
+    if (mode == 1)
+        records_kernel<1><<<rgrid, kThreads, 0, stream>>>(Rt, grad_out, fwd_out, g, ws);
+    else
+        records_kernel<0><<<rgrid, kThreads, 0, stream>>>(Rt, grad_out, fwd_out, g, ws);
+    scatter_records<<<fill_grid, 256, 0, stream>>>(ws.flags, ws.rec, ws.rec_stride, grad_vol, g.nx,
+                                                   g.ny, g.nz, slots);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    // the sparse views, slab by slab, in the (now scattered) record area
+    return launch_slabs(ws, g, mode, grad_out, fwd_out, grad_vol, stream);
 }
 
 template <typename T, int LAYOUT>
@@ -828,18 +1178,14 @@ void alpha_kernels(const void* vol, const Geom& g, const float* Rt, const float*
 cudaError_t launch_alpha_adjoint(const void* vol, int dtype, int layout, const Geom& g,
                                  const float* Rt, const float* grad_out, const float* fwd_out,
                                  float* grad_vol, void* workspace, cudaStream_t stream) {
-    Workspace ws{nullptr, nullptr, 0};
+    const Workspace ws = workspace_parts(workspace, g);
     const int fill_grid = 148 * 8;
     const int slots = batch_slots(g);
     if (workspace) {
-        ws.flags = static_cast<int*>(workspace);
-        ws.rec = reinterpret_cast<float*>(static_cast<char*>(workspace) +
-                                          adjoint_workspace_header(g.B));
-        ws.rec_stride = (long long)(g.nx - 1) * (g.ny - 1) * (g.nz - 1) * 8;
-        const int64_t n_rec4 = (int64_t)(g.nx - 1) * (g.ny - 1) * (g.nz - 1) * 2 * slots;
-        plan_views<<<1, 256, 0, stream>>>(Rt, g, ws.flags);
-        zero_records<<<fill_grid, 256, 0, stream>>>(ws.flags, reinterpret_cast<float4*>(ws.rec),
-                                                    n_rec4);
+        launch_plan(ws, Rt, g, stream);
+        zero_records<<<fill_grid, 256, 0, stream>>>(ws.flags, kSomeDense,
+                                                    reinterpret_cast<float4*>(ws.rec),
+                                                    ws.rec_stride / 4 * slots);
     }
     if (dtype == 0) {
         if (layout == 4) alpha_kernels<float, 4>(vol, g, Rt, grad_out, fwd_out, grad_vol, ws, stream);

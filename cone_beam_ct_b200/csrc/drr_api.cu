@@ -382,6 +382,13 @@ DRR_API drr_status drr_debug_bounds_errors(unsigned long long* count, long long*
 }
 #endif
 
+DRR_API drr_status drr_wait_timeouts(unsigned long long* count) {
+    if (!count) return fail(DRR_ERR_INVALID_ARG, "count must be non-NULL");
+    const cudaError_t e = drr::wait_timeouts(count);
+    if (e != cudaSuccess) return cuda_status(e, "drr_wait_timeouts");
+    return ok();
+}
+
 DRR_API int drr_abi_version(void) { return 1; }
 
 DRR_API const char* drr_get_last_error(void) { return g_last_error; }

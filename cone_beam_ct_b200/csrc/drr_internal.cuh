@@ -362,6 +362,9 @@ constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;
 // Device address of that scratch on the current device (drr_adjoint.cu),
 // looked up once per device and cached for the life of the process.
 cudaError_t noalloc_scratch(void** out);
+// Grid-barrier waits of the adjoint's slab pass that gave up, on the current
+// device, since the last read (drr_adjoint.cu); the count is cleared.
+cudaError_t wait_timeouts(unsigned long long* out);
 cudaError_t launch_prepare(const float* src, int nx, int ny, int nz, int dtype, int layout,
                            void* dst, cudaStream_t stream);
 // workspace: NULL (every view on the direct path) or the layout of

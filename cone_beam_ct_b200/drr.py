@@ -30,7 +30,8 @@ EXPORTED = ("drr_render", "drr_render_adjoint", "drr_render_adjoint_ws",
             "drr_render_adjoint_batched", "drr_adjoint_batched_workspace_bytes",
             "drr_render_pose_grad_batched", "drr_render_alpha_adjoint_batched",
             "drr_render_adjoint_batched_ws", "drr_render_staged",
-            "drr_prepared_bytes", "drr_prepare_volume", "drr_get_last_error", "drr_abi_version")
+            "drr_prepared_bytes", "drr_prepare_volume", "drr_get_last_error", "drr_abi_version",
+            "drr_wait_timeouts")
 DRR_NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
@@ -140,6 +141,8 @@ def lib():
     L.drr_get_last_error.restype = _c.c_char_p
     L.drr_abi_version.argtypes = []
     L.drr_abi_version.restype = _c.c_int
+    L.drr_wait_timeouts.argtypes = [_c.POINTER(_c.c_ulonglong)]
+    L.drr_wait_timeouts.restype = _c.c_int
     if hasattr(L, "drr_debug_bounds_errors"):
         L.drr_debug_bounds_errors.argtypes = [_c.POINTER(_c.c_ulonglong), _c.POINTER(_c.c_longlong)]
         L.drr_debug_bounds_errors.restype = _c.c_int
@@ -415,6 +418,15 @@ def drr_render_adjoint_noalloc(dims, spacing, origin, K, Rt, B, H, W, n_samples,
                                             _dev(grad_out, "grad_out", True),
                                             _dev(fwd_out, "fwd_out", True),
                                             _dev(grad_vol, "grad_vol", True), _stream(stream)))
+
+
+def drr_wait_timeouts():
+    """Grid-barrier waits of the adjoint's slab pass that gave up on the
+    current device since the last call (0 in normal operation); the count is
+    cleared.  Call after the work has completed."""
+    count = _c.c_ulonglong(0)
+    _check(lib().drr_wait_timeouts(_c.byref(count)))
+    return int(count.value)
 
 
 def drr_debug_bounds_errors():

@@ -200,17 +200,23 @@ DRR_API drr_status drr_render_adjoint(const int dims[3], const float spacing[3],
                                       float *grad_vol, void *stream);
 
 /* Bytes of the workspace drr_render_adjoint_ws needs for a volume of dims
- * and B views (0 if the arguments are invalid): a 256-byte header of view
- * flags plus one 32-byte corner record per cell, (nx-1)(ny-1)(nz-1) of them
- * (about 8x the fp32 volume). */
+ * and B views (0 if the arguments are invalid): a header (view flags, the
+ * views' camera matrices, 96 bytes per view, and a few words of
+ * synchronisation, in 256-byte units) plus one 32-byte corner record per
+ * cell, (nx-1)(ny-1)(nz-1) of them (about 8x the fp32 volume). */
 DRR_API size_t drr_adjoint_workspace_bytes(const int dims[3], int B);
 
 /* drr_render_adjoint with a caller-provided workspace, for speed: views
  * whose rays are much closer than a voxel (a 16-pixel tile spanning fewer
  * than 8 voxels at the volume centre) accumulate into per-cell corner
- * records with 16-byte vector atomics, which a final pass adds into
- * grad_vol; other views scatter into grad_vol directly, as in
- * drr_render_adjoint.  Same result up to fp32 summation order.
+ * records with 16-byte vector atomics, which a pass then adds into
+ * grad_vol.  The other views accumulate into the records of one slab of
+ * cell layers at a time (a slab small enough to stay in the L2), added into
+ * grad_vol after each slab; that pass is one cooperative launch, its phases
+ * separated by grid-wide barriers.  A barrier wait that has not ended after
+ * 20 s gives up, the pass is abandoned (grad_vol then lacks part of those
+ * views' contributions) and the event is counted: drr_wait_timeouts.  Same
+ * result as drr_render_adjoint up to fp32 summation order.
  *   workspace        DEVICE, 256-byte aligned, at least
  *                    drr_adjoint_workspace_bytes(dims, B) bytes; its content
  *                    on entry is ignored and on return is unspecified; must
@@ -225,6 +231,14 @@ DRR_API drr_status drr_render_adjoint_ws(const int dims[3], const float spacing[
                                          const float *grad_out, const float *fwd_out,
                                          float *grad_vol, void *workspace,
                                          size_t workspace_bytes, void *stream);
+
+/* Grid-barrier waits of the slab pass (drr_render_adjoint_ws and the calls
+ * built on it) that gave up on the current device since the last call; the
+ * count is cleared.  0 in normal operation: every CTA of the cooperative
+ * launch is resident, so a wait ends when the slowest CTA arrives.  Reads
+ * device memory synchronously (call it once the work has completed).
+ * Returns DRR_OK, DRR_ERR_INVALID_ARG for a NULL count, or DRR_ERR_CUDA. */
+DRR_API drr_status drr_wait_timeouts(unsigned long long *count);
 
 /* Size of the scratch built into the library for drr_render_adjoint_noalloc. */
 #define DRR_NOALLOC_SCRATCH_BYTES (32u << 20)

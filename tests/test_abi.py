@@ -220,10 +220,20 @@ def test_workspace_adjoint_rejects_bad_arguments(kw, word):
     assert word in drr.drr_get_last_error()
 
 
+def ws_header(B):
+    """Adjoint workspace header for B output images: 1 + B int flags; 16
+    bytes of barrier words (16-byte aligned); B views of 96 bytes (256-byte
+    aligned); the records then start 256-byte aligned."""
+    up = lambda n, a: (n + a - 1) // a * a
+    bar = up((1 + B) * 4, 16)
+    views = up(bar + 16, 256)
+    return up(views + 96 * B, 256)
+
+
 def test_workspace_bytes():
-    # 256-byte header of view flags, then 32 bytes per cell
-    assert drr.drr_adjoint_workspace_bytes((16, 16, 16), 2) == 256 + 15 ** 3 * 32
-    assert drr.drr_adjoint_workspace_bytes((256, 256, 256), 64) == 512 + 255 ** 3 * 32
+    assert ws_header(2) == 512 and ws_header(64) == 6656
+    assert drr.drr_adjoint_workspace_bytes((16, 16, 16), 2) == ws_header(2) + 15 ** 3 * 32
+    assert drr.drr_adjoint_workspace_bytes((256, 256, 256), 64) == ws_header(64) + 255 ** 3 * 32
     assert drr.drr_adjoint_workspace_bytes((1, 16, 16), 2) == 0
     assert drr.drr_adjoint_workspace_bytes((16, 16, 16), -1) == 0
     _adjoint_ws(B=0, workspace=None, grad_out=None, grad_vol=None, Rt=None)   # empty: no-op
@@ -479,10 +489,13 @@ def test_batched_rejects_bad_arguments():
 
 
 def test_batched_workspace_bytes():
-    # header: one int per output image plus one, rounded to 256 bytes; then 32 bytes per
+    # the header of one output image per (view, channel) -- 4 x 3 images; 2
+    # x 3 when one view is broadcast to both volumes -- then 32 bytes per
     # cell for each of the n_vols * channels volume-channels
-    assert drr.drr_adjoint_batched_workspace_bytes((16, 16, 16), 2, 3, 4) == 256 + 6 * 15 ** 3 * 32
-    assert drr.drr_adjoint_batched_workspace_bytes((16, 16, 16), 2, 3, 1) == 256 + 6 * 15 ** 3 * 32
+    assert drr.drr_adjoint_batched_workspace_bytes((16, 16, 16), 2, 3, 4) == \
+        ws_header(12) + 6 * 15 ** 3 * 32
+    assert drr.drr_adjoint_batched_workspace_bytes((16, 16, 16), 2, 3, 1) == \
+        ws_header(6) + 6 * 15 ** 3 * 32
     assert drr.drr_adjoint_batched_workspace_bytes((16, 16, 16), 1, 1, 64) == \
         drr.drr_adjoint_workspace_bytes((16, 16, 16), 64)
     assert drr.drr_adjoint_batched_workspace_bytes((16, 16, 16), 2, 3, 3) == 0   # 3 % 2 != 0

@@ -97,10 +97,44 @@ def test_mixed_dense_and_sparse_views_in_one_call(cuda):
                               w.density_factor, wl.MODE_RAW, torch.from_numpy(go).cuda(), None,
                               grad, ws)
     torch.cuda.synchronize()
-    # white-box: the plan's view flags at the head of the workspace
+    # white-box: the plan's flags at the head of the workspace (bit 0: some
+    # view dense, bit 1: some view sparse; then one per view)
     flags = ws[:4 * (1 + w.B)].cpu().numpy().view(np.int32)
-    assert flags.tolist() == [1, 1, 1, 0]
+    assert flags.tolist() == [3, 1, 1, 0]
     assert_adjoint_parity(grad.cpu().numpy(), ref, what="mixed dense and sparse views")
+
+
+# A wide, flat volume seen by small detectors: every view is sparse (rays
+# ~20 voxels apart), and a cell layer's records (699^2 cells x 32 bytes) are
+# so large that the workspace adjoint takes its slab path in several slabs of
+# 4 layers (the last one ragged: 11 cell layers), with rays crossing slab
+# boundaries at every angle.
+WIDE_FLAT = dict(dims=(700, 700, 12), spacing=(1.0, 1.1, 0.9), H=40, W=44, n_samples=37)
+
+
+@pytest.mark.parametrize("mode", [wl.MODE_RAW, wl.MODE_BEER_LAMBERT])
+def test_sparse_views_take_the_slab_records(cuda, mode):
+    import torch
+    from cone_beam_ct_b200 import drr
+    w = wl.small_random_case(216, **WIDE_FLAT)
+    go = np.random.default_rng(216).standard_normal((w.B, w.H, w.W)).astype(np.float32)
+    fwd = gpu_forward(w, layout=PADDED, dtype=F32, mode=mode) if mode else None
+    ref = _oracle_adjoint(w, go, mode)
+    got = gpu_adjoint(w, go, mode=mode, fwd_out=fwd, workspace=True)
+    assert_adjoint_parity(got, ref, what=f"slab records, mode {mode}")
+    # the plan sent every view to the sparse side
+    Rt = torch.from_numpy(np.ascontiguousarray(w.Rt.reshape(-1, 12))).cuda()
+    nx, ny, nz = w.dims
+    grad = torch.zeros((nz, ny, nx), dtype=torch.float32, device="cuda")
+    ws = torch.full((drr.drr_adjoint_workspace_bytes(w.dims, w.B),), 0x7F, dtype=torch.uint8,
+                    device="cuda")
+    drr.drr_render_adjoint_ws(w.dims, w.spacing, w.origin, w.K, Rt, w.B, w.H, w.W, w.n_samples,
+                              w.density_factor, wl.MODE_RAW, torch.from_numpy(go).cuda(), None,
+                              grad, ws)
+    torch.cuda.synchronize()
+    assert ws[:4 * (1 + w.B)].cpu().numpy().view(np.int32).tolist() == [2] + [0] * w.B
+    # no grid-barrier wait of the slab pass gave up
+    assert drr.drr_wait_timeouts() == 0
 
 
 def test_record_path_dot_product_identity(cuda):
