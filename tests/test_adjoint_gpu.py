@@ -104,12 +104,13 @@ def test_mixed_dense_and_sparse_views_in_one_call(cuda):
     assert_adjoint_parity(grad.cpu().numpy(), ref, what="mixed dense and sparse views")
 
 
-# A wide, flat volume seen by small detectors: every view is sparse (rays
-# ~20 voxels apart), and a cell layer's records (699^2 cells x 32 bytes) are
-# so large that the workspace adjoint takes its slab path in several slabs of
-# 4 layers (the last one ragged: 11 cell layers), with rays crossing slab
-# boundaries at every angle.
-WIDE_FLAT = dict(dims=(700, 700, 12), spacing=(1.0, 1.1, 0.9), H=40, W=44, n_samples=37)
+# A wide, flat volume: every view is sparse (rays ~4 voxels apart), and a
+# cell layer's records (699^2 cells x 32 bytes) are so large that the
+# workspace adjoint's slab pass takes several slabs of 3 layers (the last one
+# ragged: 11 cell layers), with rays crossing slab boundaries at every
+# angle.  3 x 200 x 210 rays x 211 samples (26.6e6) is above the size below
+# which a call sends its sparse views to the direct path instead.
+WIDE_FLAT = dict(dims=(700, 700, 12), spacing=(1.0, 1.1, 0.9), H=200, W=210, n_samples=211)
 
 
 @pytest.mark.parametrize("mode", [wl.MODE_RAW, wl.MODE_BEER_LAMBERT])

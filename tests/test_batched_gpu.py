@@ -149,6 +149,22 @@ def test_batched_adjoint_with_workspace_sparse_views(cuda):
     _assert_batched_adjoint(got, ref, "sparse, workspace")
 
 
+def test_batched_adjoint_slab_pass(cuda):
+    # sparse images of 2 volumes x 3 channels, a call large enough (31e6
+    # ray-samples) for the slab pass: 13 slabs of 3 cell layers, records per
+    # volume-channel slot
+    w = wl.small_random_case(642, B=4, dims=(300, 280, 40), H=160, W=170, n_samples=96)
+    nx, ny, nz = w.dims
+    vols = np.random.default_rng(642).uniform(0.0, 0.05, (2, 3, nz, ny, nx)).astype(np.float32)
+    go = np.random.default_rng(8).standard_normal((4, 3, w.H, w.W)).astype(np.float32)
+    ref = oracle.adjoint_batched(w.dims, w.spacing, w.origin, w.K, w.Rt, 2, 4, w.H, w.W,
+                                 w.n_samples, w.density_factor, wl.MODE_RAW, go, vols=vols,
+                                 nthreads=8)
+    got = _gpu_adjoint_batched(w, 2, 3, 4, go, wl.MODE_RAW, workspace=True)
+    _assert_batched_adjoint(got, ref, "sparse, slab pass")
+    assert drr.drr_wait_timeouts() == 0
+
+
 def test_batched_dot_product_identity(cuda):
     w, x = _batch(2, 2, 6, 621)
     y = np.random.default_rng(9).standard_normal((6, 2, w.H, w.W)).astype(np.float32)

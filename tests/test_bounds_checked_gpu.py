@@ -2,7 +2,8 @@
 every gather and scatter of every kernel range-checked against the extent
 of its buffer.  Small ragged cases run through every entry point and layout
 on it -- forward (4 layouts x fp32/bf16 x raw/Beer-Lambert/alpha), volume
-adjoint (direct and with a workspace, sparse and dense views), pose gradient,
+adjoint (direct and with a workspace, sparse and dense views, the slab pass
+of large sparse calls), pose gradient,
 alpha gradient, Siddon pair, batches, prepare -- and the device error word
 must stay 0: no index of any kernel leaves its buffer.  The results must also
 match the ordinary build's (same arithmetic; the checks only guard)."""
@@ -122,6 +123,19 @@ def test_batches_stay_in_bounds(checked):
                                              n_views, w.H, w.W, w.n_samples, w.density_factor,
                                              wl.MODE_BEER_LAMBERT, go, out, g_rt)
             _clean(drr, f"batches, layout {layout}, {n_views} views")
+
+
+def test_slab_pass_stays_in_bounds(checked):
+    # sparse views in a call large enough for the adjoint's slab pass (26.6e6
+    # ray-samples, 4 slabs of 3 cell layers over a wide, flat volume)
+    w = wl.small_random_case(506, dims=(700, 700, 12), spacing=(1.0, 1.1, 0.9), H=200, W=210,
+                             n_samples=211)
+    go = np.random.default_rng(9).standard_normal((w.B, w.H, w.W)).astype(np.float32)
+    for mode in (wl.MODE_RAW, wl.MODE_BEER_LAMBERT):
+        fwd = H.gpu_forward(w, layout=H.PADDED, dtype=H.F32, mode=mode) if mode else None
+        H.gpu_adjoint(w, go, mode=mode, fwd_out=fwd, workspace=True)
+        _clean(checked, f"slab pass mode {mode}")
+    assert checked.drr_wait_timeouts() == 0
 
 
 def test_checked_results_match_the_ordinary_build(checked):
