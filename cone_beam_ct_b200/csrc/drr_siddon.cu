@@ -34,12 +34,17 @@ __device__ __forceinline__ float voxel_value<uint16_t>(const uint16_t* p) {
     return __uint_as_float((uint32_t)__ldg(reinterpret_cast<const unsigned short*>(p)) << 16);
 }
 
-// The walk's state for one ray.
+// The walk's state for one ray.  Indexed only by constants (walk_step picks
+// the axis with selects), so it lives in registers: indexing it by the axis
+// number put it in local memory (a 96-byte stack frame; B200, 256^3 fp32
+// volume, 4 views of 1024^2: forward 7.18 -> 4.61 ms, backprojection 15.26
+// -> 7.09 ms).
 struct Walk {
     double t, t1;          // current parameter (mm) and the exit
     double next[3];        // parameter of the next plane on each axis (inf: parallel)
     double delta[3];       // 1 / |d_a|: parameter between planes
     int cell[3], step[3];  // current cell, +-1 per axis
+    int didx[3];           // change of the linear index for a step along each axis
     int idx;               // linear index of the cell
 };
 
@@ -95,31 +100,41 @@ __device__ __forceinline__ bool walk_setup(const View& v, const Geom& g, double 
         }
     }
     k.idx = (k.cell[2] * g.ny + k.cell[1]) * g.nx + k.cell[0];
+    k.didx[0] = k.step[0];
+    k.didx[1] = k.step[1] * g.nx;
+    k.didx[2] = k.step[2] * g.nx * g.ny;
     return true;
 }
 
 // One step: the length of the current piece; advances to the next cell.
 // Returns false when the walk has left the box (the piece is still valid).
 __device__ __forceinline__ bool walk_step(const Geom& g, Walk& k, double& len) {
-    int ax = 0;
-    double tn = k.next[0];
-    if (k.next[1] < tn) {
-        tn = k.next[1];
-        ax = 1;
-    }
-    if (k.next[2] < tn) {
-        tn = k.next[2];
-        ax = 2;
-    }
+    // the axis whose plane comes first (ties: the lower axis)
+    const bool y_first = k.next[1] < k.next[0];
+    const double t01 = y_first ? k.next[1] : k.next[0];
+    const bool a2 = k.next[2] < t01;
+    const double tn = a2 ? k.next[2] : t01;
+    const bool a1 = y_first && !a2, a0 = !y_first && !a2;
     const double te = fmin(tn, k.t1);
     len = fmax(te - k.t, 0.0);
     k.t = fmax(k.t, te);
     if (tn >= k.t1) return false;
-    k.cell[ax] += k.step[ax];
-    k.next[ax] += k.delta[ax];
-    const int n = ax == 0 ? g.nx : (ax == 1 ? g.ny : g.nz);
-    if (k.cell[ax] < 0 || k.cell[ax] >= n) return false;
-    k.idx += k.step[ax] * (ax == 0 ? 1 : (ax == 1 ? g.nx : g.nx * g.ny));
+    if (a0) {
+        k.cell[0] += k.step[0];
+        k.next[0] += k.delta[0];
+    }
+    if (a1) {
+        k.cell[1] += k.step[1];
+        k.next[1] += k.delta[1];
+    }
+    if (a2) {
+        k.cell[2] += k.step[2];
+        k.next[2] += k.delta[2];
+    }
+    const int c = a0 ? k.cell[0] : (a1 ? k.cell[1] : k.cell[2]);
+    const int n = a0 ? g.nx : (a1 ? g.ny : g.nz);
+    if (c < 0 || c >= n) return false;
+    k.idx += a0 ? k.didx[0] : (a1 ? k.didx[1] : k.didx[2]);
     return true;
 }
 
