@@ -42,8 +42,8 @@
 // bundle flushes once where its rays would have flushed up to six times.  A
 // record sums the moments of its samples (records_kernel); a scatter pass
 // then turns each record into corner weights and adds them to the gradient
-// volume.  The alpha gradient (records of weights, added by a gather pass)
-// and batched calls (records per volume-channel) take the same path.
+// volume.  The alpha gradient (its per-sample factor in place of the ray's
+// scale) and batched calls (records per volume-channel) take the same path.
 //
 // The sparse views of a call with a workspace accumulate into records too,
 // but one slab of cell layers at a time, each slab's records small enough to
@@ -282,39 +282,6 @@ __global__ void scatter_records(const int* __restrict__ flags, const float* __re
                 if (v[e] != 0.0f && in_bounds(k * nxy + (long long)j * nx + off, 1, nvox))
                     atomicAdd(gr + off, v[e]);
             }
-        }
-    }
-}
-
-// grad[k][j][i] += the 8 record entries of voxel (i, j, k): entry a + 2b + 4c of
-// cell (i - a, j - b, k - c), for the cells that exist; for every
-// volume-channel slot (slot s: gradient s * nx*ny*nz elements on, records
-// s * rec_stride floats on).  A CTA takes whole x rows, so the row's (j, k)
-// and slot come from one division per row, not three 64-bit ones per voxel.
-__global__ void gather_records(const int* __restrict__ flags, const float* __restrict__ rec,
-                               long long rec_stride, float* __restrict__ grad, int nx, int ny,
-                               int nz, int slots) {
-    if ((flags[0] & kSomeDense) == 0) return;
-    const int rows = ny * nz;                    // x rows per slot (nx*ny*nz < 2^31)
-    const long long total = (long long)rows * slots;
-    const int cr = nx - 1, cs = (nx - 1) * (ny - 1);
-    for (long long row = blockIdx.x; row < total; row += gridDim.x) {
-        const int slot = (int)(row / rows);
-        const int rr = (int)(row - (long long)slot * rows);
-        const int k = rr / ny, j = rr - k * ny;
-        const float* __restrict__ r = rec + slot * rec_stride;
-        float* __restrict__ gr = grad + row * nx;
-        for (int i = threadIdx.x; i < nx; i += blockDim.x) {
-            float s = 0.0f;
-#pragma unroll
-            for (int corner = 0; corner < 8; ++corner) {
-                const int ci = i - (corner & 1), cj = j - ((corner >> 1) & 1), ck = k - (corner >> 2);
-                const long long off = (long long)(ck * cs + cj * cr + ci) * 8 + corner;
-                if (ci >= 0 && cj >= 0 && ck >= 0 && ci < nx - 1 && cj < ny - 1 && ck < nz - 1 &&
-                    in_bounds(off, 1, rec_stride))
-                    s += __ldg(r + off);
-            }
-            if (in_bounds((long long)rr * nx + i, 1, (long long)rows * nx)) gr[i] += s;
         }
     }
 }
@@ -908,7 +875,9 @@ alpha_adjoint_kernel(const T* __restrict__ vol_base, const float* __restrict__ R
 // Measured on the 256^3 bf16 volume seen by 4 views of 1024^2, 512 samples:
 // 12.0 ms against 31.4 for the direct path; 3 x 2 bundles 13.4 ms (spills
 // at 128 registers) or 19.6 ms (148 registers, 1 CTA per SM); packed fp32x2
-// weights 12.1 ms.
+// weights 12.1 ms.  The records hold moments, as records_kernel's, turned
+// into weights by scatter_records (11.13 against 11.53 ms with weight
+// records and a voxel-centric gather pass).
 constexpr int kAlphaBundle = 2;                          // rays per bundle, across and down
 constexpr int kAlphaTile = 16 * kAlphaBundle;            // 32 x 32 pixels per CTA
 
@@ -963,7 +932,7 @@ alpha_records_kernel(const T* __restrict__ vol_base, const float* __restrict__ R
     }
     // cells stay in [0, n-2] per axis (lim as for the linear layout), inside the records
     const int cr = g.nx - 1, cs = (g.nx - 1) * (g.ny - 1);
-    float p[kSlots][8];
+    float2 p[kSlots][4];
     int pc[kSlots];
 #pragma unroll
     for (int h = 0; h < kSlots; ++h) pc[h] = -1;
@@ -989,19 +958,18 @@ alpha_records_kernel(const T* __restrict__ vol_base, const float* __restrict__ R
             Tr[k] *= 1.0f - a;
             const float scale = go[k] * dmu;
             const int cell = cz * cs + cy * cr + cx;
-            const float wz1 = scale * fz, wz0 = scale * (1.0f - fz);
-            const float w00 = wz0 * (1.0f - fy), w01 = wz0 * fy;
-            const float w10 = wz1 * (1.0f - fy), w11 = wz1 * fy;
-            const float gx = 1.0f - fx;
-            const float w[8] = {w00 * gx, w00 * fx, w01 * gx, w01 * fx,
-                                w10 * gx, w10 * fx, w11 * gx, w11 * fx};
+            // the sample's 8 moments scale fx^a fy^b fz^c, as records_kernel
+            const float2 mx = make_float2(scale, scale * fx);
+            const float2 mxy = __fmul2_rn(mx, make_float2(fy, fy));
+            const float2 w[4] = {mx, mxy, __fmul2_rn(mx, make_float2(fz, fz)),
+                                 __fmul2_rn(mxy, make_float2(fz, fz))};
             const int home = k / kAlphaBundle, other = 1 - home;
             if (pc[other] == cell && pc[home] != cell) {
 #pragma unroll
                 for (int h = 0; h < kSlots; ++h)
                     if (h == other)
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) p[h][e] += w[e];
+                        for (int e = 0; e < 4; ++e) p[h][e] = __fadd2_rn(p[h][e], w[e]);
             } else {
 #pragma unroll
                 for (int h = 0; h < kSlots; ++h) {
@@ -1010,10 +978,10 @@ alpha_records_kernel(const T* __restrict__ vol_base, const float* __restrict__ R
                         if (pc[h] >= 0) flush_record(rec, pc[h], p[h], ws.rec_stride);
                         pc[h] = cell;
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) p[h][e] = 0.0f;
+                        for (int e = 0; e < 4; ++e) p[h][e] = make_float2(0.0f, 0.0f);
                     }
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) p[h][e] += w[e];
+                    for (int e = 0; e < 4; ++e) p[h][e] = __fadd2_rn(p[h][e], w[e]);
                 }
             }
         }
@@ -1214,8 +1182,8 @@ cudaError_t launch_alpha_adjoint(const void* vol, int dtype, int layout, const G
         else alpha_kernels<uint16_t, 0>(vol, g, Rt, grad_out, fwd_out, grad_vol, ws, stream);
     }
     if (workspace)
-        gather_records<<<fill_grid, 256, 0, stream>>>(ws.flags, ws.rec, ws.rec_stride, grad_vol,
-                                                      g.nx, g.ny, g.nz, slots);
+        scatter_records<<<fill_grid, 256, 0, stream>>>(ws.flags, ws.rec, ws.rec_stride, grad_vol,
+                                                       g.nx, g.ny, g.nz, slots);
     return cudaGetLastError();
 }
 

@@ -206,15 +206,19 @@ __device__ __forceinline__ void pose_terms(const Clip& k, const Geom& g, const f
     }
 }
 
-// 3 CTAs per SM: caps the kernel at 80 registers (the fp64 per-ray epilogue
-// spills a little) instead of 96 and 2 CTAs; measured on B200 at 1024^2 x
-// 512: 4.78 against 5.80 ms (before the packed bf16 sample and the unroll,
-// which brought it to 4.18 ms).
+// 4 CTAs per SM: caps the kernel at 64 registers.  The fp64 per-ray
+// epilogue then spills (up to ~200 bytes, once per ray), the sample loop
+// gains the occupancy; measured on B200 against 3 CTAs (80 registers): 3.95
+// against 4.24 ms (256^3 bf16 corner records, 4 views of 1024^2 x 512),
+// 2.29 against 2.49 ms (fp32 quads, 64 views of 200^2 x 256), 5.08 against
+// 6.10 ms (512^3 fp32 corner records, 2 views of 2048^2 x 256).  (3 CTAs
+// had beaten 2, 96 registers, 4.78 against 5.80 ms, before the packed bf16
+// sample and the unroll.)
 // BATCH: images map to poses and volume-channels by the batch rule (a
 // separate instantiation, so that the single-volume kernel carries none of
 // its registers).
 template <typename T, int LAYOUT, int MODE, bool BATCH>
-__global__ void __launch_bounds__(kThreads, 3)
+__global__ void __launch_bounds__(kThreads, 4)
 pose_kernel(const T* __restrict__ vol_base, const float* __restrict__ Rt,
             const float* __restrict__ grad_out, const float* __restrict__ fwd_out,
             float* __restrict__ grad_Rt, const Geom g) {
