@@ -154,13 +154,6 @@ __device__ __forceinline__ void red_add(float* p, float a) {
 // Flush a pending corner record: two 16-byte vector reductions into one
 // sector.  (n: floats of the record array at rec, for the bounds-checked
 // build)
-__device__ __forceinline__ void flush_record(float* __restrict__ rec, int cell, const float a[8],
-                                             long long n) {
-    if (!in_bounds((long long)cell * 8, 8, n)) return;
-    float* p = rec + (size_t)cell * 8;
-    red_add_v4(p, a[0], a[1], a[2], a[3]);
-    red_add_v4(p + 4, a[4], a[5], a[6], a[7]);
-}
 __device__ __forceinline__ void flush_record(float* __restrict__ rec, int cell, const float2 a[4],
                                              long long n) {
     if (!in_bounds((long long)cell * 8, 8, n)) return;
