@@ -57,6 +57,7 @@
 #include <algorithm>
 #include <mutex>
 
+#include "drr_barrier.cuh"
 #include "drr_internal.cuh"
 #include "drr_sample.cuh"
 
@@ -549,53 +550,6 @@ constexpr double kSlabMinSamples = 8.0 * (1 << 20);
 constexpr unsigned long long kBarrierTimeoutNs = 20ull * 1000 * 1000 * 1000;
 __device__ unsigned long long g_wait_timeouts;
 
-__device__ __forceinline__ unsigned long long global_ns() {
-    unsigned long long t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
-}
-
-// Grid-wide barrier over a cooperative launch (every CTA resident).  bar[0]
-// counts arrivals over the launch (epoch e is complete at e * gridDim.x),
-// bar[1] holds the last released epoch, bar[2] the abort word.  Returns
-// false if this or another CTA gave up (the caller returns).
-__device__ bool grid_barrier(unsigned* bar, unsigned& epoch) {
-    __shared__ int s_ok;
-    __syncthreads();
-    ++epoch;
-    if (threadIdx.x == 0) {
-        volatile unsigned* vb = bar;
-        int ok = vb[2] == 0u;
-        if (ok) {
-            __threadfence();                     // this CTA's writes before its arrival
-            const unsigned arrived = atomicAdd(&bar[0], 1u) + 1u;
-            if (arrived == epoch * gridDim.x) {
-                __threadfence();
-                atomicExch(&bar[1], epoch);
-            } else {
-                const unsigned long long t0 = global_ns();
-                while (vb[1] < epoch) {
-                    if (vb[2] != 0u) {
-                        ok = 0;
-                        break;
-                    }
-                    if (global_ns() - t0 > kBarrierTimeoutNs) {
-                        atomicExch(&bar[2], 1u);
-                        atomicAdd(&g_wait_timeouts, 1ull);
-                        ok = 0;
-                        break;
-                    }
-                    __nanosleep(256);
-                }
-            }
-            __threadfence();                     // the other CTAs' writes before ours
-        }
-        s_ok = ok;
-    }
-    __syncthreads();
-    return s_ok != 0;
-}
-
 // Sample indices i in [0, N) whose 32.32 coordinate q0 + i s lies in [z0, z1):
 // an interval, since the coordinate is monotone in i.  Exact integer bounds,
 // so consecutive slabs share no sample and miss none.
@@ -746,13 +700,13 @@ slab_adjoint_kernel(const float* __restrict__ grad_out, const float* __restrict_
          m += (long long)gridDim.x * blockDim.x)
         __stcg(r4 + m, zero);
     unsigned epoch = 0;
-    if (!grid_barrier(ws.bar, epoch)) return;
+    if (!grid_barrier(ws.bar, epoch, gridDim.x, kBarrierTimeoutNs, &g_wait_timeouts)) return;
     for (int cz0 = 0; cz0 < g.nz - 1; cz0 += layers) {
         const int cz1 = min(cz0 + layers, g.nz - 1);
         slab_records<MODE>(grad_out, fwd_out, g, ws, cz0, cz1, slab_stride);
-        if (!grid_barrier(ws.bar, epoch)) return;
+        if (!grid_barrier(ws.bar, epoch, gridDim.x, kBarrierTimeoutNs, &g_wait_timeouts)) return;
         slab_scatter(ws.rec, slab_stride, grad, g, slots, cz0, cz1);
-        if (!grid_barrier(ws.bar, epoch)) return;
+        if (!grid_barrier(ws.bar, epoch, gridDim.x, kBarrierTimeoutNs, &g_wait_timeouts)) return;
     }
 }
 

@@ -7,8 +7,25 @@
 #include <stdint.h>
 
 #include "../../include/drr_probe.h"
+#include "drr_barrier.cuh"
 
 namespace {
+
+// Self-test of the grid barrier: every CTA passes `rounds` barriers that
+// expect `expected` arrivals each and counts the ones it got through.  With
+// expected above the grid's CTA count no epoch completes: the first wait
+// that runs out raises the abort word and the others leave.
+__global__ void __launch_bounds__(256) barrier_probe(unsigned* bar, unsigned expected,
+                                                     unsigned long long timeout_ns, int rounds,
+                                                     unsigned long long* timeouts, int* passes) {
+    unsigned epoch = 0;
+    int n = 0;
+    for (int r = 0; r < rounds; ++r) {
+        if (!drr::grid_barrier(bar, epoch, expected, timeout_ns, timeouts)) break;
+        ++n;
+    }
+    if (threadIdx.x == 0) atomicAdd(passes, n);
+}
 
 __global__ void __launch_bounds__(512) l2_read(const float4* __restrict__ buf, size_t n, int reps,
                                                float* __restrict__ sink) {
@@ -88,4 +105,46 @@ extern "C" DRR_PROBE_API int drr_probe_l2_read(const void* buf, size_t n_vec16, 
     l2_read<<<sms * 4, 512, 0, static_cast<cudaStream_t>(stream)>>>(
         static_cast<const float4*>(buf), n_vec16, reps, sink);
     return (int)cudaGetLastError();
+}
+
+extern "C" DRR_PROBE_API int drr_probe_grid_barrier(int extra_arrivals, int rounds,
+                                                    double timeout_ms,
+                                                    unsigned long long* timeouts_out,
+                                                    int* passes_out, int* ctas_out) {
+    if (extra_arrivals < 0 || rounds < 1 || rounds > 4096 || !(timeout_ms > 0.0) ||
+        timeout_ms > 60000.0 || !timeouts_out || !passes_out || !ctas_out)
+        return -1;
+    int dev = 0, sms = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return (int)e;
+    struct Words {
+        unsigned bar[4];
+        unsigned long long timeouts;
+        int passes;
+    };
+    Words* w = nullptr;
+    e = cudaMalloc(&w, sizeof(Words));
+    if (e != cudaSuccess) return (int)e;
+    e = cudaMemset(w, 0, sizeof(Words));
+    unsigned* bar = w->bar;
+    unsigned expected = (unsigned)(sms + extra_arrivals);
+    unsigned long long timeout_ns = (unsigned long long)(timeout_ms * 1e6);
+    unsigned long long* timeouts = &w->timeouts;
+    int* passes = &w->passes;
+    void* args[] = {(void*)&bar, (void*)&expected, (void*)&timeout_ns, (void*)&rounds,
+                    (void*)&timeouts, (void*)&passes};
+    // one CTA per SM, launched cooperatively: all resident
+    if (e == cudaSuccess)
+        e = cudaLaunchCooperativeKernel((const void*)barrier_probe, dim3(sms), dim3(256), args, 0,
+                                        0);
+    if (e == cudaSuccess) e = cudaDeviceSynchronize();
+    Words h{};
+    if (e == cudaSuccess) e = cudaMemcpy(&h, w, sizeof(Words), cudaMemcpyDeviceToHost);
+    cudaFree(w);
+    if (e != cudaSuccess) return (int)e;
+    *timeouts_out = h.timeouts;
+    *passes_out = h.passes;
+    *ctas_out = sms;
+    return 0;
 }

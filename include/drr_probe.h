@@ -1,9 +1,10 @@
 /*
- * drr_probe.h -- measurement helpers of the benchmark (libdrr_probe.so), not
+ * drr_probe.h -- measurement and self-test helpers (libdrr_probe.so), not
  * part of the ray-march.  They measure the L2 read bandwidth that is the
  * denominator of the gather roofline while a volume fits in L2 (the
- * measured-peaks file of the GPU pool has HBM and GEMM peaks only), and the
- * L2's fp32 reduction throughput, the ceiling of the adjoint's scatter.
+ * measured peak figures at hand cover HBM and GEMMs only), and the
+ * L2's fp32 reduction throughput, the ceiling of the adjoint's scatter; and
+ * they drive the adjoint's grid barrier, including a wait that runs out.
  */
 #ifndef DRR_PROBE_H
 #define DRR_PROBE_H
@@ -44,6 +45,21 @@ DRR_PROBE_API int drr_probe_l2_read(const void *buf, size_t n_vec16, int reps, f
  * launched), or the CUDA error code of a failed launch. */
 DRR_PROBE_API int drr_probe_l2_red(float *buf, size_t n_floats, int reps, int kind,
                                    void *stream);
+
+/* Self-test of the bounded grid barrier that separates the phases of the
+ * volume adjoint's slab pass (drr_render_adjoint_ws): one CTA per SM,
+ * launched cooperatively, passes `rounds` barriers, each expecting the
+ * grid's CTA count plus `extra_arrivals`.  With extra_arrivals = 0 every
+ * barrier completes; with more, no epoch completes, the first wait that
+ * lasts timeout_ms raises the abort word and every CTA returns.  Reports the
+ * waits that gave up (*timeouts_out), the barriers passed summed over CTAs
+ * (*passes_out) and the CTA count (*ctas_out).  Synchronous (allocates and
+ * frees a few words, synchronises the device).  Returns 0, -1 for bad
+ * arguments (rounds in [1, 4096], timeout_ms in (0, 60000]), or a CUDA
+ * error code. */
+DRR_PROBE_API int drr_probe_grid_barrier(int extra_arrivals, int rounds, double timeout_ms,
+                                         unsigned long long *timeouts_out, int *passes_out,
+                                         int *ctas_out);
 
 #ifdef __cplusplus
 }

@@ -62,11 +62,11 @@ def test_checked_library_debug_call_rejects_null_pointers():
     assert b"non-NULL" in L.drr_get_last_error()
 
 
-def test_probe_library_exports_its_declared_symbol():
+def test_probe_library_exports_its_declared_symbols():
     import ctypes
     ctypes.CDLL(PROBE_LIB)
     names = declared_names(PROBE_HEADER, "DRR_PROBE_API")
-    assert names == ["drr_probe_l2_read", "drr_probe_l2_red"]
+    assert names == ["drr_probe_grid_barrier", "drr_probe_l2_read", "drr_probe_l2_red"]
     assert exported_names(PROBE_LIB) == set(names)
 
 
@@ -651,3 +651,21 @@ def test_binding_fails_loudly_without_the_library(monkeypatch, tmp_path):
     monkeypatch.setattr(drr, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError, match="no CPU fallback"):
         drr.lib()
+
+
+def test_grid_barrier_probe_rejects_bad_arguments():
+    # no GPU needed: argument checks come before any CUDA call
+    import ctypes
+    lib = ctypes.CDLL(PROBE_LIB)
+    f = lib.drr_probe_grid_barrier
+    f.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_void_p, ctypes.c_void_p,
+                  ctypes.c_void_p]
+    f.restype = ctypes.c_int
+    t, p, c = ctypes.c_ulonglong(), ctypes.c_int(), ctypes.c_int()
+    ok = (ctypes.byref(t), ctypes.byref(p), ctypes.byref(c))
+    assert f(-1, 1, 10.0, *ok) == -1
+    assert f(0, 0, 10.0, *ok) == -1
+    assert f(0, 5000, 10.0, *ok) == -1
+    assert f(0, 1, 0.0, *ok) == -1
+    assert f(0, 1, 1e9, *ok) == -1
+    assert f(0, 1, 10.0, None, ok[1], ok[2]) == -1
