@@ -142,7 +142,9 @@ def workload(cfg, views=0):
     return w
 
 
-def config_block(w, cfg, layout_name):
+def config_block(w, cfg):
+    """The workload, the same for both arms (how each arm stores the volume
+    is reported beside it, not in it)."""
     from cone_beam_ct_b200 import workloads as wl
     nx, ny, nz = w.dims
     vol_dtype = "bf16" if w.dtype == wl.DTYPE_BF16 else "fp32"
@@ -151,11 +153,11 @@ def config_block(w, cfg, layout_name):
         "workload": f"{nx}^3 {vol_dtype} volume, {w.B} views x {w.H}x{w.W}, "
                     f"{w.n_samples} samples/ray: prepare + forward ({mode}) + adjoint",
         "config_index": cfg,
-        "volume": f"{nx}x{ny}x{nz} {vol_dtype}, {layout_name} layout, "
-                  f"{float(w.spacing[0])} mm voxels",
+        "volume": f"{nx}x{ny}x{nz} {vol_dtype}, {float(w.spacing[0])} mm voxels",
         "views": w.B, "detector": [w.H, w.W], "samples_per_ray": w.n_samples,
         "samples_per_step": w.samples,
-        "l2": "flushed before every step (256 MiB write, outside the step timing)",
+        "l2": "GPU arm: flushed before every step (256 MiB write, outside the step timing); "
+              "CPU arm: not applicable",
         "inputs": "seeded synthetic phantom and poses (cone_beam_ct_b200.workloads)",
     }
 
@@ -395,7 +397,8 @@ def run_reference(args):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": config_block(w, args.config, "linear"),
+        "config": config_block(w, args.config),
+        "layout": "linear fp32 (the oracle's own arrays)",
         "cpu_baseline": {"value": value, "unit": "Gsamples/s", "cores": cores, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": "Gsamples/s", "h2d_bytes_per_step": 0,
@@ -794,7 +797,7 @@ def config_timing(torch, cfg, hbm_peak, l2_cache):
                              "unit": "GB/s", "frac": a / peak,
                              "algorithmic_bytes_per_launch": int(nbytes)}}
 
-    res = {"workload": config_block(w, cfg, lname)["workload"], "layout": lname,
+    res = {"workload": config_block(w, cfg)["workload"], "layout": lname,
            "samples": w.samples}
     fwd()
     if cfg != 5:
@@ -1016,7 +1019,7 @@ def run_ours(args):
                 "algorithmic_bytes_per_launch": int(nbytes), "ms_per_launch": ms,
                 "traffic": traffic_for(kernel_key, wname, args.layout)}
 
-    wname = config_block(w, args.config, "")["workload"]
+    wname = config_block(w, args.config)["workload"]
     fwd_roof = roof("forward_kernel", fwd_ms, fwd_bytes, "forward_kernel", wname)
     adj_roof = roof(ADJOINT_GROUP, adj_ms, adj_bytes, "adjoint_kernel", wname)
     # the ceiling of a scatter: the L2's fp32 reduction rate, measured beside
@@ -1074,7 +1077,8 @@ def run_ours(args):
         "ms_per_step": ms_per_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f32", "data": "synthetic",
-        "config": config_block(w, args.config, args.layout),
+        "config": config_block(w, args.config),
+        "layout": args.layout,
         "fps": fps,
         "kernels_ms": {"prepare": float(kern_ms[0]), "forward": fwd_ms,
                        "zero_grad (torch)": float(kern_ms[2]), "adjoint": adj_ms},
@@ -1184,7 +1188,8 @@ def run_partitioned(args):
         "unit": "Gsamples/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "strong",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": dict(config_block(w, args.config, args.layout),
+        "layout": args.layout,
+        "config": dict(config_block(w, args.config),
                        parallelism=f"detector rows split over {world} ranks, volume replicated, "
                                    "gradient all-reduced (NCCL) every step"),
         "fps": w.B * args.steps / (total_ms * 1e-3),

@@ -53,7 +53,7 @@ def test_a_comment_edit_keeps_the_traffic(tmp_path, monkeypatch):
 def test_committed_traffic_names_the_bench_workloads():
     with open(bench.os.path.join(bench.ROOT, "profiles", "traffic.json")) as f:
         table = json.load(f)
-    names = {bench.config_block(bench.workload(c), c, "")["workload"] for c in (2, 3)}
+    names = {bench.config_block(bench.workload(c), c)["workload"] for c in (2, 3)}
     for kernel in ("forward_kernel", "adjoint_kernel"):
         assert set(table[kernel]) <= names
         for entry in table[kernel].values():
