@@ -65,12 +65,14 @@ def _close(got, ref, what):
 
 
 # dense views (rays much closer than a voxel) use the scratch's corner records;
-# sparse views use it only for the view flags
+# the sparse views of a small call use it only for the view flags, those of a
+# call of at least 8 * 2^20 ray-samples for the slab pass's records
 CASES = {
     "dense": dict(seed=301, dims=(23, 17, 29), H=150, W=170, n_samples=40),
     "dense, near the size limit": dict(seed=302, dims=(96, 96, 90), B=2, H=400, W=400,
                                         n_samples=64),
     "sparse": dict(seed=303),
+    "sparse, slab pass": dict(seed=305, dims=(90, 84, 88), B=3, H=150, W=150, n_samples=160),
 }
 
 
@@ -89,6 +91,21 @@ def test_noalloc_matches_the_oracle_and_the_workspace_adjoint_twice_in_a_row(cud
         got = _adjoint(cuda, w, Rt, go, fwd, mode, noalloc=True)
         _close(got, ref, f"{name}, mode {mode}, call {call} against the oracle")
         _close(got, with_ws, f"{name}, mode {mode}, call {call} against the workspace adjoint")
+
+
+def test_the_slab_case_is_all_sparse(cuda):
+    # white-box: the plan sends every view of that case to the sparse side
+    from cone_beam_ct_b200 import drr
+    w = wl.small_random_case(**CASES["sparse, slab pass"])
+    Rt, go, _, _ = _inputs(cuda, w, 7, wl.MODE_RAW)
+    nx, ny, nz = w.dims
+    grad = cuda.zeros((nz, ny, nx), dtype=cuda.float32, device="cuda")
+    ws = cuda.full((drr.drr_adjoint_workspace_bytes(w.dims, w.B),), 0x7F, dtype=cuda.uint8,
+                   device="cuda")
+    drr.drr_render_adjoint_ws(w.dims, w.spacing, w.origin, w.K, Rt, w.B, w.H, w.W, w.n_samples,
+                              w.density_factor, wl.MODE_RAW, go, None, grad, ws)
+    cuda.cuda.synchronize()
+    assert ws[:4 * (1 + w.B)].cpu().numpy().view(np.int32).tolist() == [2] + [0] * w.B
 
 
 def test_noalloc_rejects_volumes_beyond_its_scratch(cuda):
