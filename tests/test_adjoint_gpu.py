@@ -138,6 +138,29 @@ def test_sparse_views_take_the_slab_records(cuda, mode):
     assert drr.drr_wait_timeouts() == 0
 
 
+@pytest.mark.parametrize("nz", [2, 3])
+def test_slab_pass_on_one_or_two_cell_layers(cuda, nz):
+    # the degenerate depths: one cell layer (nz = 2) and two (nz = 3), one
+    # slab either way, every ray crossing the whole depth in a few samples
+    w = wl.small_random_case(217 + nz, dims=(400, 380, nz), B=2, H=256, W=256, n_samples=80)
+    assert w.B * w.H * w.W * w.n_samples >= 8 * 2 ** 20       # the slab pass's size
+    go = np.random.default_rng(nz).standard_normal((w.B, w.H, w.W)).astype(np.float32)
+    ref = _oracle_adjoint(w, go, wl.MODE_RAW)
+    import torch
+    from cone_beam_ct_b200 import drr
+    Rt = torch.from_numpy(np.ascontiguousarray(w.Rt.reshape(-1, 12))).cuda()
+    nx, ny, _ = w.dims
+    grad = torch.zeros((nz, ny, nx), dtype=torch.float32, device="cuda")
+    ws = torch.full((drr.drr_adjoint_workspace_bytes(w.dims, w.B),), 0x7F, dtype=torch.uint8,
+                    device="cuda")
+    drr.drr_render_adjoint_ws(w.dims, w.spacing, w.origin, w.K, Rt, w.B, w.H, w.W, w.n_samples,
+                              w.density_factor, wl.MODE_RAW, torch.from_numpy(go).cuda(), None,
+                              grad, ws)
+    torch.cuda.synchronize()
+    assert ws[:4 * (1 + w.B)].cpu().numpy().view(np.int32).tolist() == [2] + [0] * w.B
+    assert_adjoint_parity(grad.cpu().numpy(), ref, what=f"slab pass, nz = {nz}")
+
+
 def test_record_path_dot_product_identity(cuda):
     w = wl.small_random_case(213, **DENSE)
     rng = np.random.default_rng(7)
