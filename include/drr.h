@@ -215,8 +215,13 @@ DRR_API size_t drr_adjoint_workspace_bytes(const int dims[3], int B);
  * grad_vol after each slab; that pass is one cooperative launch, its phases
  * separated by grid-wide barriers.  A barrier wait that has not ended after
  * 20 s gives up, the pass is abandoned (grad_vol then lacks part of those
- * views' contributions) and the event is counted: drr_wait_timeouts.  Same
- * result as drr_render_adjoint up to fp32 summation order.
+ * views' contributions) and the event is counted: drr_wait_timeouts.  The
+ * pass's grid is sized to what the device reports it can hold at once; if
+ * the launch is refused (fewer SMs available to the process than the
+ * device has, say), the call returns DRR_ERR_CUDA.  Calls of fewer than
+ * 8 * 2^20 ray-samples (B * H * W * n_samples) send their sparse views to
+ * the direct path instead.  Same result as drr_render_adjoint up to fp32
+ * summation order.
  *   workspace        DEVICE, 256-byte aligned, at least
  *                    drr_adjoint_workspace_bytes(dims, B) bytes; its content
  *                    on entry is ignored and on return is unspecified; must
