@@ -528,7 +528,7 @@ records_kernel(const float* __restrict__ Rt, const float* __restrict__ grad_out,
 // about a voxel per sample changes cell nearly every sample, and the record
 // then costs 2 sector operations per sample where the direct path's faces
 // cost 3.5 (measured on the 256^3 volume seen by 64 views of 200^2 with 256
-// samples: 1.6 reduction sectors per sample).  Then the slab's records go
+// samples: 1.93 reduction sectors per sample).  Then the slab's records go
 // into the gradient (moments to corner weights, as scatter_records) and are
 // cleared for the next slab.
 //
