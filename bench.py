@@ -819,7 +819,7 @@ def config_timing(torch, cfg, hbm_peak, l2_cache):
 
 
 def run_e2e(torch, drr, w, args, world, dev, stream, flush, dtype, layout, prep, pbytes, ws,
-            ws_bytes, fwd_needed):
+            ws_bytes, fwd_needed, ref_out, ref_grad):
     """The step through the public API from and to pinned host memory: every
     step uploads its volume, poses and upstream gradient and downloads its
     image and gradient volume, inside the timed region.  Steps are pipelined
@@ -894,9 +894,16 @@ def run_e2e(torch, drr, w, args, world, dev, stream, flush, dtype, layout, prep,
     e2e_ms = max_over_ranks([e0.elapsed_time(e1)], dev)[0]
     h2d = h_vol.numel() * 4 + h_Rt.numel() * 4 + h_go.numel() * 4
     d2h = h_out[0].numel() * 4 + h_grad[0].numel() * 4
+    # the last step's downloads against the device-timed step's results (same
+    # inputs): the image bit for bit, the gradient up to the atomics' order
+    last = (args.steps - 1) & 1
+    img_same = bool(torch.equal(h_out[last], ref_out.cpu()))
+    g_ref = ref_grad.cpu()
+    g_err = float((h_grad[last] - g_ref).abs().max() / g_ref.abs().max().clamp_min(1e-30))
     return {"value": job_throughput(world, w.samples, args.steps, e2e_ms) / 1e9,
             "unit": "Gsamples/s", "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
             "ms_per_step": e2e_ms / args.steps,
+            "check": {"image_equal": img_same, "gradient_max_rel_diff": g_err},
             "note": "pipelined over two buffer sets: uploads of step k+1 and downloads of step k "
                     "overlap the kernels; includes the 256 MiB L2 flush write before each step"}
 
@@ -993,7 +1000,7 @@ def run_ours(args):
     e2e = None
     if not args.no_e2e:
         e2e = run_e2e(torch, drr, w, args, world, dev, stream, flush, dtype, layout, prep, pbytes,
-                      ws, ws_bytes, fwd_needed)
+                      ws, ws_bytes, fwd_needed, out, grad)
 
     # roofline of the dominant kernel
     peaks, peak_src = measured_peaks()
