@@ -72,20 +72,24 @@ def test_dense_views_take_the_record_path(cuda, seed, mode):
         assert_adjoint_parity(got, ref, what=f"dense seed {seed} workspace {workspace}")
 
 
-def _mixed_case(seed):
+def _mixed_case(seed, n_samples=DENSE["n_samples"]):
     """DENSE geometry with its last view moved 4x farther: one call whose plan
-    sends two views to the record path and one to the direct path."""
-    w = wl.small_random_case(seed, **DENSE)
+    sends two views to the record path and one to the sparse side (the
+    direct path; the slab pass once the call has 8 * 2^20 ray-samples)."""
+    w = wl.small_random_case(seed, **dict(DENSE, n_samples=n_samples))
     Rt = w.Rt.copy()
     Rt[2, :, 3] *= 4.0
     w.Rt = Rt
     return w
 
 
-def test_mixed_dense_and_sparse_views_in_one_call(cuda):
+@pytest.mark.parametrize("n_samples", [40, 120])
+def test_mixed_dense_and_sparse_views_in_one_call(cuda, n_samples):
+    # 40 samples: the sparse view on the direct path; 120 (9.2e6 ray-samples):
+    # the slab pass, in the record area the dense views' scatter just read
     import torch
     from cone_beam_ct_b200 import drr
-    w = _mixed_case(214)
+    w = _mixed_case(214, n_samples)
     go = np.random.default_rng(214).standard_normal((w.B, w.H, w.W)).astype(np.float32)
     ref = _oracle_adjoint(w, go, wl.MODE_RAW)
     Rt = torch.from_numpy(np.ascontiguousarray(w.Rt.reshape(-1, 12))).cuda()
