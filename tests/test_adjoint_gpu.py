@@ -15,8 +15,8 @@ import pytest
 
 import oracle
 from cone_beam_ct_b200 import workloads as wl
-from tests.gpu_helpers import (BF16, CORNERS, F32, LINEAR, PADDED, bf16_values, gpu_adjoint,
-                               gpu_forward)
+from tests.gpu_helpers import (BF16, CORNERS, F32, LINEAR, PADDED, QUADS, bf16_values,
+                               gpu_adjoint, gpu_forward)
 
 pytestmark = pytest.mark.gpu
 TOL_ADJ, TOL_DOT = 1e-4, 1e-5
@@ -224,6 +224,21 @@ def test_config5_full_adjoint_and_dot_product(cuda):
     x = rng.uniform(0, 1, (nz, ny, nx)).astype(np.float32)
     y = rng.standard_normal((w.B, w.H, w.W)).astype(np.float32)
     assert _dot_residual(w, x, y, PADDED) <= TOL_DOT
+
+
+@pytest.mark.slow
+def test_config2_full_adjoint_as_timed(cuda):
+    # the 64-view workload's adjoint as the throughput run's configs block
+    # times it: Beer-Lambert, a dense N(0, 1) upstream gradient, fwd_out from
+    # the GPU forward in the xy-quad layout, a workspace (every view sparse:
+    # the slab pass, 11 slabs), against the oracle on the whole volume
+    w = wl.make_config(2)
+    go = np.random.default_rng(2002).standard_normal((w.B, w.H, w.W)).astype(np.float32)
+    fwd = gpu_forward(w, layout=QUADS, dtype=F32, mode=wl.MODE_BEER_LAMBERT)
+    ref = oracle.adjoint(w.dims, w.spacing, w.origin, w.K, w.Rt, w.H, w.W, w.n_samples,
+                         w.density_factor, wl.MODE_BEER_LAMBERT, go, vol=w.vol, nthreads=16)
+    got = gpu_adjoint(w, go, mode=wl.MODE_BEER_LAMBERT, fwd_out=fwd, workspace=True)
+    assert_adjoint_parity(got, ref, what="config 2, Beer-Lambert, workspace")
 
 
 @pytest.mark.slow
