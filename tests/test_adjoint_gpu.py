@@ -242,6 +242,22 @@ def test_config2_full_adjoint_as_timed(cuda):
 
 
 @pytest.mark.slow
+def test_config4_dense_band_adjoint(cuda):
+    # the 512^3 volume seen by 2 C-arm views of 2048^2 with 256 samples, raw:
+    # its record array (4.3 GB) is past 1 GiB, where the record kernel spreads
+    # its warp phases over the first quarter of each ray; a band of 40 full
+    # detector rows per view carries a dense N(0, 1) upstream gradient
+    w = wl.make_config(4)
+    go = np.zeros((w.B, w.H, w.W), np.float32)
+    go[:, 1004:1044, :] = np.random.default_rng(44).standard_normal(
+        (w.B, 40, w.W)).astype(np.float32)
+    ref = oracle.adjoint(w.dims, w.spacing, w.origin, w.K, w.Rt, w.H, w.W, w.n_samples,
+                         w.density_factor, wl.MODE_RAW, go, nthreads=16)
+    got = gpu_adjoint(w, go, mode=wl.MODE_RAW, workspace=True)
+    assert_adjoint_parity(got, ref, what="config 4 dense band")
+
+
+@pytest.mark.slow
 def test_config3_geometry_adjoint(cuda):
     # the 1024^2 x 512 C-arm geometry with an fp32 gradient volume: the dot-product
     # identity at full size, and the oracle on a sparse upstream gradient (2000 rays)
