@@ -153,6 +153,23 @@ def test_alpha_adjoint_config3_sparse_upstream(cuda):
         _assert_adjoint(got, ref, f"config 3, 3000 rays, workspace {workspace}")
 
 
+@pytest.mark.slow
+def test_alpha_adjoint_config3_dense_band(cuda):
+    # the alpha gradient with a workspace as the throughput run's widened row
+    # times it (bf16 corner records, 4 views of 1024^2 x 512, every view dense:
+    # the moment records of alpha_records_kernel), on a band of 96 full
+    # detector rows per view with a dense N(0, 1) upstream gradient
+    w = wl.make_config(3)
+    go = np.zeros((w.B, w.H, w.W), np.float32)
+    go[:, 472:568, :] = np.random.default_rng(38).standard_normal((w.B, 96, w.W)).astype(
+        np.float32)
+    fwd = gpu_forward(w, layout=CORNERS, dtype=BF16, mode=ALPHA)
+    ref = oracle.adjoint(w.dims, w.spacing, w.origin, w.K, w.Rt, w.H, w.W, w.n_samples,
+                         w.density_factor, ALPHA, go, vol=bf16_values(w.vol), nthreads=16)
+    got = gpu_alpha_adjoint(w, go, fwd, layout=CORNERS, dtype=BF16, workspace=True)
+    _assert_adjoint(got, ref, "config 3 dense band, workspace")
+
+
 def _noise_inputs(n, seed):
     rng = np.random.default_rng(seed)
     image = rng.uniform(0.0, 1.0, n).astype(np.float32)
