@@ -776,7 +776,7 @@ alpha_adjoint_kernel(const T* __restrict__ vol_base, const float* __restrict__ R
             : LAYOUT == 2 ? sample_corners(vol + (size_t)at * 8, fx, fy, fz)
             : LAYOUT == 3 ? sample_quads(vol + (size_t)at * 4, g.slice, fx, fy, fz)
                           : trilinear_at(vol + at, g.row, g.slice, fx, fy, fz);
-        const float a = -expm1f(-s * mu);
+        const float a = opacity<T>(s * mu);
         Ci = fmaf(Tr * a, mu, Ci);
         const float dmu = Tr * fmaf(s * (1.0f - a), mu, a) - s * (Cray - Ci);
         Tr *= 1.0f - a;
@@ -899,7 +899,7 @@ alpha_records_kernel(const T* __restrict__ vol_base, const float* __restrict__ R
                 : LAYOUT == 2 ? sample_corners(vol + (size_t)at * 8, fx, fy, fz)
                 : LAYOUT == 3 ? sample_quads(vol + (size_t)at * 4, g.slice, fx, fy, fz)
                               : trilinear_at(vol + at, g.row, g.slice, fx, fy, fz);
-            const float a = -expm1f(-sa[k] * mu);
+            const float a = opacity<T>(sa[k] * mu);
             Ci[k] = fmaf(Tr[k] * a, mu, Ci[k]);
             const float dmu = Tr[k] * fmaf(sa[k] * (1.0f - a), mu, a) - sa[k] * (Cray[k] - Ci[k]);
             Tr[k] *= 1.0f - a;

@@ -101,8 +101,9 @@ __device__ __forceinline__ float march_bricks(const T* __restrict__ vol, const G
 // read as the emission-absorption sum: sample i has opacity
 // a_i = 1 - exp(-s mu_i), s = density_factor * dt, and colour mu_i;
 // C = sum_i T_i a_i mu_i with T_0 = 1, T_{i+1} = T_i (1 - a_i).  The same
-// samples and interpolation as the integral; a_i by expm1f, which keeps its
-// relative accuracy for the small opacities of thin samples.
+// samples and interpolation as the integral; a_i by opacity<T>
+// (drr_sample.cuh), which keeps its relative accuracy for the small
+// opacities of thin samples.
 template <typename T, int LAYOUT>
 __device__ __forceinline__ float march_alpha(const T* __restrict__ vol, const Geom& g,
                                              const Ray& ray, float s) {
@@ -119,7 +120,7 @@ __device__ __forceinline__ float march_alpha(const T* __restrict__ vol, const Ge
             : LAYOUT == 2 ? sample_corners(vol + (size_t)cell * 8, fx, fy, fz)
             : LAYOUT == 3 ? sample_quads(vol + (size_t)cell * 4, slice, fx, fy, fz)
                           : trilinear_at(vol + cell, row, slice, fx, fy, fz);
-        const float a = -expm1f(-s * mu);
+        const float a = opacity<T>(s * mu);
         C = fmaf(Tr * a, mu, C);
         Tr *= 1.0f - a;
         qx += sx;

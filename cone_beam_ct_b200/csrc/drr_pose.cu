@@ -291,7 +291,7 @@ pose_kernel(const T* __restrict__ vol_base, const float* __restrict__ Rt,
                     // dC/dmu_i = T_i (s (1 - a_i) mu_i + a_i) - s (C - C_i) weights the
                     // sample's gradient; S collects dC/ds = sum T_i mu_i^2 (1 - a_i)
                     // - mu_i (C - C_i) (a_i = 1 - exp(-s mu_i), as the forward)
-                    const float a = -expm1f(-sa * val);
+                    const float a = opacity<T>(sa * val);
                     const float keep = 1.0f - a;
                     Ci = fmaf(Tr * a, val, Ci);
                     const float rest = Cray - Ci;

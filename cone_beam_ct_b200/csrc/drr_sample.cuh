@@ -39,6 +39,34 @@ __device__ __forceinline__ float load_voxel_any(const uint16_t* p) {
 
 // GLOBAL: the volume is in global memory (read through the read-only path);
 // else anywhere, shared memory included.  The same lerps either way.
+// Opacity of a sample, a = 1 - exp(-x), x = s mu (front-to-back alpha
+// compositing).  fp32 volumes: -expm1f(-x), which keeps its relative
+// accuracy for the thin samples of fine sampling.  bf16 volumes: the
+// Maclaurin series of 1 - e^-x, x (1 - x/2 (1 - x/3 (1 - x/4 (1 - x/5)))),
+// for |x| < 1/8, where the first omitted term, x^6 / 6!, is below 5e-8 of
+// the result, and 1 - __expf(-x) above, where the result is at least 0.1175
+// and __expf's error stays near fp32 rounding.  Measured on B200 (256^3
+// bf16 corner records, 4 views of 1024^2 x 512) against expm1f: alpha
+// forward 4.76 -> 4.02 ms, its pose gradient 6.96 -> 6.36 ms, its volume
+// gradient 11.12 -> 10.94 ms.  On fp32 volumes of the 64-view 200^2
+// workload the same split was slower than expm1f (forward 2.17 against 2.08
+// ms), so they keep it.
+template <typename T>
+__device__ __forceinline__ float opacity(float x) {
+    if constexpr (sizeof(T) == 2) {
+        if (fabsf(x) < 0.125f) {
+            const float p = fmaf(-0.2f * x, 1.0f, 1.0f);              // 1 - x/5
+            const float q = fmaf(-0.25f * x, p, 1.0f);                // 1 - x/4 (...)
+            const float r = fmaf(-(1.0f / 3.0f) * x, q, 1.0f);        // 1 - x/3 (...)
+            const float t = fmaf(-0.5f * x, r, 1.0f);                 // 1 - x/2 (...)
+            return x * t;
+        }
+        return 1.0f - __expf(-x);
+    } else {
+        return -expm1f(-x);
+    }
+}
+
 template <typename T, bool GLOBAL = true>
 __device__ __forceinline__ float trilinear_at(const T* __restrict__ base, int row, int slice,
                                               float fx, float fy, float fz) {

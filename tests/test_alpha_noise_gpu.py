@@ -56,12 +56,16 @@ def test_alpha_forward_small_ragged(cuda, layout, df):
     assert_parity(got, _oracle_image(w), 1e-4, what=f"alpha layout {layout} df {df}")
 
 
+# bf16 volumes take the series / __expf opacity: with df 0.7 every sample's
+# s mu is below 1/8 (the series), with df 20 they spread to about 1 (both)
+@pytest.mark.parametrize("df", [0.7, 20.0])
 @pytest.mark.parametrize("layout", LAYOUTS)
-def test_alpha_forward_bf16(cuda, layout):
+def test_alpha_forward_bf16(cuda, layout, df):
     w = wl.small_random_case(402)
-    w.density_factor = 20.0
+    w.density_factor = df
     got = gpu_forward(w, layout=layout, dtype=BF16, mode=ALPHA)
-    assert_parity(got, _oracle_image(w, vol=bf16_values(w.vol)), 1e-4, what=f"bf16 layout {layout}")
+    assert_parity(got, _oracle_image(w, vol=bf16_values(w.vol)), 1e-4,
+                  what=f"bf16 layout {layout} df {df}")
 
 
 @pytest.mark.slow
